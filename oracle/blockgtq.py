@@ -1,0 +1,390 @@
+"""Block-GTQ on a TQ-MSE-style scalar quantizer: the oracle. TEST INFRASTRUCTURE ONLY.
+
+Source: "RoPE-aware bit allocation for KV cache quantization" (Liang, Zhang,
+Jia; arXiv 2606.24033), abstract: for each layer and KV head, a label-free
+energy score per RoPE block, then a greedy integer bit allocation by marginal
+gain, on top of TurboQuant-MSE; matched K/V bit budgets (K2V2, K3V3, ...);
+"uniform TQ-MSE" as the baseline allocation; a packed-cache serving path that
+runs attention on the packed cache.
+
+The page names these steps without defining them. The readings taken here
+(each restated in the function that uses it):
+
+  energy     E_b = mean over calibration tokens of ||k_b||^2, block b = dims
+             (b, b + d/2); fp64, summed in a fixed order (64-token chunks).
+  greedy     d/2 * bits_k steps; each adds one bit to the block with the
+             largest E_b * (delta(w_b) - delta(w_b + 1)) among blocks below
+             w_max; ties go to the lowest block index.
+  gain       g_b = sqrt(2 sum(E) / (d E_b)) (unit variance per coordinate of
+             block b after the global sqrt(d)/||k|| scaling), 1 if E_b = 0;
+             f_b = 1 / (sqrt(d) g_b) is the matching dequant factor.
+  quantizer  per token row: fp16 norm of the row, a = sqrt(d)/norm in fp32,
+             y = (x * a) * g_b in fp32, code = #{thresholds strictly below y}
+             of the width-w_b Lloyd-Max codebook. Values use width bits_v, g = 1.
+  layout     32-token tiles; bit planes transposed so that each 32-bit word
+             holds one bit plane of 32 codes (see pack_cache).
+  attention  softmax over cached positions 0..T-1 of q . k_hat / sqrt(d),
+             k_hat = norm * c[code] * f_b, v_hat = norm * c[code] / sqrt(d).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from . import codebooks
+
+TILE = 32            # tokens per packed tile
+CALIB_CHUNK = 64     # tokens per fixed-order partial sum of the energy score
+
+MODE_BLOCKGTQ = 0
+MODE_UNIFORM = 1
+
+
+# --------------------------------------------------------------------------- calibration
+
+def calibration_energies(K: np.ndarray, n_calib: int = 0) -> tuple[np.ndarray, int]:
+    """Label-free energy score per (KV head, RoPE block).
+
+    K: [B][H][T][d] array whose values are exactly the stored keys (any float type).
+    n_calib: number of leading tokens of every sequence to use (0 = all T).
+    The calibration tokens of all sequences are pooled in the order
+    u = s * n_calib + t. Each term is fl(fl(x_b^2) + fl(x_{b+h}^2)) in fp64;
+    terms are summed left to right within consecutive chunks of 64 pooled
+    tokens (the last chunk may be shorter), chunk sums are added left to right,
+    and the total is divided by N = B * n_calib.
+    Returns (E [H][d/2] float64, N).
+    """
+    B, H, T, d = K.shape
+    h = d // 2
+    n = T if n_calib <= 0 else n_calib
+    if n > T:
+        raise ValueError("n_calib exceeds the sequence length")
+    X = np.asarray(K[:, :, :n, :], dtype=np.float64)
+    X = np.transpose(X, (1, 0, 2, 3)).reshape(H, B * n, d)            # pooled token order
+    terms = X[:, :, :h] * X[:, :, :h] + X[:, :, h:] * X[:, :, h:]     # [H][N][h]
+    N = B * n
+    total = np.zeros((H, h), dtype=np.float64)
+    for c0 in range(0, N, CALIB_CHUNK):
+        acc = np.zeros((H, h), dtype=np.float64)
+        for u in range(c0, min(N, c0 + CALIB_CHUNK)):
+            acc = acc + terms[:, u, :]
+        total = total + acc
+    return total / float(N), N
+
+
+def greedy_widths(E: np.ndarray, bits: int, w_max: int, delta: np.ndarray | None = None) -> np.ndarray:
+    """Greedy integer bit allocation by marginal gain for one KV head.
+
+    E: [h] energies. Runs bits * h steps; at each step the block b with
+    w_b < w_max maximising E_b * (delta[w_b] - delta[w_b + 1]) (fp64, delta
+    taken from the fp32 table) gets one more bit; ties go to the lowest b.
+    """
+    if delta is None:
+        delta = codebooks.delta_table()
+    D = np.asarray(delta, dtype=np.float64)
+    h = len(E)
+    if not (1 <= bits <= w_max <= 8):
+        raise ValueError("need 1 <= bits <= w_max <= 8")
+    w = np.zeros(h, dtype=np.int64)
+    for _ in range(bits * h):
+        best_b, best_gain = -1, -math.inf
+        for b in range(h):
+            if w[b] < w_max:
+                gain = float(E[b]) * (D[w[b]] - D[w[b] + 1])
+                if gain > best_gain:
+                    best_b, best_gain = b, gain
+        w[best_b] += 1
+    return w
+
+
+def block_gains(E: np.ndarray, d: int) -> tuple[np.ndarray, np.ndarray]:
+    """Per-block gain g_b (fp32) and dequant factor f_b (fp32) for one KV head.
+
+    S = sum_b E_b left to right (fp64); g_b = fp32(sqrt((2 S) / (d E_b))) if E_b > 0
+    else 1; f_b = fp32(1 / (sqrt(d) * g_b)) with g_b taken as its fp32 value.
+    """
+    E = np.asarray(E, dtype=np.float64)
+    S = 0.0
+    for e in E:
+        S = S + float(e)
+    g = np.ones(len(E), dtype=np.float32)
+    for b, e in enumerate(E):
+        if e > 0.0 and S > 0.0:
+            g[b] = np.float32(math.sqrt((2.0 * S) / (float(d) * float(e))))
+    f = np.array([np.float32(1.0 / (math.sqrt(float(d)) * float(gb))) for gb in g], dtype=np.float32)
+    return g, f
+
+
+def allocate(E: np.ndarray, d: int, bits_k: int, w_max: int = 8, mode: int = MODE_BLOCKGTQ) -> dict:
+    """Allocation for every KV head: widths w [H][h], gains g, dequant factors f, energies E."""
+    H, h = E.shape
+    assert h == d // 2
+    w = np.zeros((H, h), dtype=np.int64)
+    g = np.ones((H, h), dtype=np.float32)
+    f = np.zeros((H, h), dtype=np.float32)
+    for hh in range(H):
+        if mode == MODE_BLOCKGTQ:
+            w[hh] = greedy_widths(E[hh], bits_k, w_max)
+            g[hh], f[hh] = block_gains(E[hh], d)
+        elif mode == MODE_UNIFORM:
+            w[hh] = bits_k
+            g[hh] = 1.0
+            f[hh] = np.float32(1.0 / math.sqrt(float(d)))
+        else:
+            raise ValueError("mode")
+    return {"E": E.copy(), "w": w, "g": g, "f": f, "d": d, "bits_k": bits_k, "w_max": w_max, "mode": mode}
+
+
+def calibrate(K: np.ndarray, bits_k: int, n_calib: int = 0, w_max: int = 8, mode: int = MODE_BLOCKGTQ) -> dict:
+    E, _ = calibration_energies(K, n_calib)
+    return allocate(E, K.shape[-1], bits_k, w_max, mode)
+
+
+# --------------------------------------------------------------------------- quantizer
+
+def row_norms_f16(X: np.ndarray) -> np.ndarray:
+    """fp16 norm of every row: fp16(sqrt(s2)), s2 = sum of x_j^2 left to right in fp64."""
+    X = np.asarray(X, dtype=np.float64)
+    s2 = np.add.accumulate(X * X, axis=-1)[..., -1]
+    return np.sqrt(s2).astype(np.float16)
+
+
+def quantize_rows(X: np.ndarray, widths_dim: np.ndarray, gains_dim: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """TQ-MSE-style scalar quantizer for rows X[..., d].
+
+    X holds exactly the stored values (converted to fp32 exactly).
+    norm = fp16 norm; a = fp32(sqrt(d)) / fp32(norm) (a = 0 when norm = 0);
+    y_j = fp32(fp32(x_j * a) * g_j); code_j = #{thresholds of width w_j strictly
+    below y_j} (0 where w_j = 0). Returns (codes uint8 [..., d], norms fp16 [...]).
+    """
+    X32 = np.asarray(X, dtype=np.float32)
+    d = X32.shape[-1]
+    n16 = row_norms_f16(X32)
+    sqd = np.float32(math.sqrt(float(d)))
+    n32 = n16.astype(np.float32)
+    with np.errstate(divide="ignore"):
+        a = np.where(n32 == 0, np.float32(0.0), sqd / np.where(n32 == 0, np.float32(1.0), n32)).astype(np.float32)
+    y = (X32 * a[..., None]).astype(np.float32)
+    y = (y * np.asarray(gains_dim, dtype=np.float32)).astype(np.float32)
+    codes = np.zeros(X32.shape, dtype=np.uint8)
+    for w in range(1, 9):
+        sel = np.asarray(widths_dim) == w
+        if not np.any(sel):
+            continue
+        _, t32 = codebooks.stored_codebook(w)
+        # side="left": the count of thresholds t with t < y, i.e. y > t strictly.
+        codes[..., sel] = np.searchsorted(t32, y[..., sel], side="left").astype(np.uint8)
+    return codes, n16
+
+
+def widths_per_dim(w_blocks: np.ndarray) -> np.ndarray:
+    return np.concatenate([w_blocks, w_blocks])
+
+
+def quantize(K: np.ndarray, V: np.ndarray, alloc: dict, bits_v: int) -> dict:
+    """Codes and fp16 norms for K (Block-GTQ widths and gains) and V (uniform bits_v, g = 1)."""
+    B, H, T, d = K.shape
+    Kc = np.zeros((B, H, T, d), dtype=np.uint8)
+    Kn = np.zeros((B, H, T), dtype=np.float16)
+    for hh in range(H):
+        wd = widths_per_dim(alloc["w"][hh])
+        gd = np.concatenate([alloc["g"][hh], alloc["g"][hh]])
+        Kc[:, hh], Kn[:, hh] = quantize_rows(K[:, hh], wd, gd)
+    Vc, Vn = quantize_rows(V, np.full(d, bits_v), np.ones(d, dtype=np.float32))
+    return {"Kc": Kc, "Kn": Kn, "Vc": Vc, "Vn": Vn}
+
+
+# --------------------------------------------------------------------------- packed layout
+
+def tile_k_words(bits_k: int, d: int) -> int:
+    return bits_k * d
+
+
+def tile_v_words(bits_v: int, d: int) -> int:
+    return bits_v * d
+
+
+def tile_record_bytes(d: int, bits_k: int, bits_v: int) -> int:
+    """Bytes of one 32-token tile record: K words, V words, 32 K norms, 32 V norms (fp16)."""
+    return 4 * tile_k_words(bits_k, d) + 4 * tile_v_words(bits_v, d) + 2 * TILE * 2
+
+
+def packed_bytes(batch: int, n_kv_heads: int, capacity: int, d: int, bits_k: int, bits_v: int) -> int:
+    n_tiles = -(-capacity // TILE)
+    return batch * n_kv_heads * n_tiles * tile_record_bytes(d, bits_k, bits_v)
+
+
+def _k_bit_source(H: int, q: int, b: int, h: int) -> tuple[int, int]:
+    """(token in tile, dim) whose code bit sits at bit q of K word half H of block b.
+
+    q = s + 4 m with s = q mod 4, m = q div 4: token = 4H + s + 8 (m div 2),
+    dim = b if m is even else b + h.
+    """
+    s, m = q % 4, q // 4
+    return 4 * H + s + 8 * (m // 2), b + h * (m % 2)
+
+
+def _v_bit_source(q: int) -> int:
+    """Token in tile whose code bit sits at bit q of a V word: q = c + 4 m ->
+    token = 8 (m div 2) + 2 c + (m mod 2)."""
+    c, m = q % 4, q // 4
+    return 8 * (m // 2) + 2 * c + (m % 2)
+
+
+def k_word_offsets(w_blocks: np.ndarray) -> np.ndarray:
+    """Word offset of block b's segment inside the K part of a tile (blocks ascending,
+    2 * w_b words each: planes p ascending, halves H = 0, 1)."""
+    off = np.zeros(len(w_blocks), dtype=np.int64)
+    acc = 0
+    for b, w in enumerate(w_blocks):
+        off[b] = acc
+        acc += 2 * int(w)
+    return off
+
+
+def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarray:
+    """Packed cache bytes [B][Hkv][n_tiles][record] for capacity tokens per sequence.
+
+    Tile record (little-endian):
+      K part, bits_k * d words: for each block b ascending with w_b > 0, for each
+        plane p < w_b, two words (H = 0, 1); bit q of word H holds bit p of the
+        code at (token, dim) = _k_bit_source(H, q, b, h).
+      V part, bits_v * d words: for each plane p < bits_v, for each dim j, one
+        word; bit q holds bit p of the code of token _v_bit_source(q), dim j.
+      32 fp16 K norms, 32 fp16 V norms, in token order.
+    Tokens at or beyond the sequence length T are stored with code 0 and norm 0.
+    """
+    Kc, Kn, Vc, Vn = codes["Kc"], codes["Kn"], codes["Vc"], codes["Vn"]
+    B, H, T, d = Kc.shape
+    h = d // 2
+    bits_k = int(alloc["bits_k"])
+    n_tiles = -(-capacity // TILE)
+    if T > capacity:
+        raise ValueError("more tokens than capacity")
+    cap = n_tiles * TILE
+
+    def padded(a, fill=0):
+        out = np.full(a.shape[:2] + (cap,) + a.shape[3:], fill, dtype=a.dtype)
+        out[:, :, :T] = a
+        return out
+
+    Kc, Vc, Kn, Vn = padded(Kc), padded(Vc), padded(Kn), padded(Vn)
+    Kc = Kc.reshape(B, H, n_tiles, TILE, d)
+    Vc = Vc.reshape(B, H, n_tiles, TILE, d)
+    rec = tile_record_bytes(d, bits_k, bits_v)
+    out = np.zeros((B, H, n_tiles, rec), dtype=np.uint8)
+    qs = np.arange(32, dtype=np.uint64)
+    for hh in range(H):
+        w_blocks = alloc["w"][hh]
+        kwords = np.zeros((B, n_tiles, tile_k_words(bits_k, d)), dtype=np.uint64)
+        off = k_word_offsets(w_blocks)
+        for b in range(h):
+            for p in range(int(w_blocks[b])):
+                for Hh in (0, 1):
+                    src = [_k_bit_source(Hh, q, b, h) for q in range(32)]
+                    tok = np.array([s[0] for s in src])
+                    dim = np.array([s[1] for s in src])
+                    bits = ((Kc[:, hh][:, :, tok, dim] >> p) & 1).astype(np.uint64)   # [B][n_tiles][32]
+                    kwords[:, :, off[b] + 2 * p + Hh] = np.sum(bits << qs, axis=-1)
+        vwords = np.zeros((B, n_tiles, tile_v_words(bits_v, d)), dtype=np.uint64)
+        vtok = np.array([_v_bit_source(q) for q in range(32)])
+        for p in range(bits_v):
+            bits = ((Vc[:, hh][:, :, vtok, :] >> p) & 1).astype(np.uint64)                # [B][n_tiles][32][d]
+            vwords[:, :, p * d:(p + 1) * d] = np.sum(bits << qs[:, None], axis=2)
+        parts = [kwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1),
+                 vwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1),
+                 Kn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1),
+                 Vn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1)]
+        out[:, hh] = np.concatenate(parts, axis=-1)
+    return out
+
+
+def unpack_cache(packed: np.ndarray, alloc: dict, bits_v: int, seq_len: int) -> dict:
+    """Inverse of pack_cache for the first seq_len tokens: codes and norms per token."""
+    B, H, n_tiles, rec = packed.shape
+    d = int(alloc["d"])
+    h = d // 2
+    bits_k = int(alloc["bits_k"])
+    nk, nv = tile_k_words(bits_k, d), tile_v_words(bits_v, d)
+    cap = n_tiles * TILE
+    Kc = np.zeros((B, H, n_tiles, TILE, d), dtype=np.uint8)
+    Vc = np.zeros((B, H, n_tiles, TILE, d), dtype=np.uint8)
+    words = packed[..., :4 * (nk + nv)].copy().view("<u4")
+    kw, vw = words[..., :nk], words[..., nk:]
+    norms = packed[..., 4 * (nk + nv):].copy().view("<f2")
+    Kn = norms[..., :TILE].reshape(B, H, cap)
+    Vn = norms[..., TILE:].reshape(B, H, cap)
+    for hh in range(H):
+        w_blocks = alloc["w"][hh]
+        off = k_word_offsets(w_blocks)
+        for b in range(h):
+            for p in range(int(w_blocks[b])):
+                for Hh in (0, 1):
+                    word = kw[:, hh, :, off[b] + 2 * p + Hh].astype(np.uint64)
+                    for q in range(32):
+                        tok, dim = _k_bit_source(Hh, q, b, h)
+                        bit = ((word >> np.uint64(q)) & np.uint64(1)).astype(np.uint8)
+                        Kc[:, hh, :, tok, dim] |= bit << p
+        for p in range(bits_v):
+            for q in range(32):
+                tok = _v_bit_source(q)
+                word = vw[:, hh, :, p * d:(p + 1) * d].astype(np.uint64)
+                bit = ((word >> np.uint64(q)) & np.uint64(1)).astype(np.uint8)
+                Vc[:, hh, :, tok, :] |= bit << p
+    Kc = Kc.reshape(B, H, cap, d)[:, :, :seq_len]
+    Vc = Vc.reshape(B, H, cap, d)[:, :, :seq_len]
+    return {"Kc": Kc, "Kn": Kn[:, :, :seq_len].astype(np.float16),
+            "Vc": Vc, "Vn": Vn[:, :, :seq_len].astype(np.float16)}
+
+
+# --------------------------------------------------------------------------- dequant + attention
+
+def dequantize_keys(Kc: np.ndarray, Kn: np.ndarray, alloc: dict) -> np.ndarray:
+    """k_hat[b,h,t,j] = norm * c_{w}[code] * f_b in fp64 (0 where w_b = 0)."""
+    B, H, T, d = Kc.shape
+    out = np.zeros((B, H, T, d), dtype=np.float64)
+    for hh in range(H):
+        wd = widths_per_dim(alloc["w"][hh])
+        fd = np.concatenate([alloc["f"][hh], alloc["f"][hh]]).astype(np.float64)
+        for j in range(d):
+            if wd[j] == 0:
+                continue
+            c16, _ = codebooks.stored_codebook(int(wd[j]))
+            cval = c16.astype(np.float64)[Kc[:, hh, :, j]]
+            out[:, hh, :, j] = Kn[:, hh].astype(np.float64) * cval * fd[j]
+    return out
+
+
+def dequantize_values(Vc: np.ndarray, Vn: np.ndarray, bits_v: int) -> np.ndarray:
+    """v_hat = norm * c_{bits_v}[code] / sqrt(d) in fp64."""
+    d = Vc.shape[-1]
+    c16, _ = codebooks.stored_codebook(bits_v)
+    return Vn.astype(np.float64)[..., None] * c16.astype(np.float64)[Vc] / math.sqrt(float(d))
+
+
+def decode_attention(q: np.ndarray, Khat: np.ndarray, Vhat: np.ndarray) -> np.ndarray:
+    """out[b, hq] = sum_t softmax_t(q . k_hat_t / sqrt(d)) v_hat_t over all given tokens (fp64).
+
+    q: [B][Hq][d]; Khat, Vhat: [B][Hkv][T][d]; q-head hq reads KV head hq // (Hq / Hkv).
+    """
+    B, Hq, d = q.shape
+    Hkv = Khat.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    for b in range(B):
+        for hq in range(Hq):
+            kv = hq // G
+            logits = Khat[b, kv] @ np.asarray(q[b, hq], dtype=np.float64) / math.sqrt(float(d))
+            m = np.max(logits)
+            p = np.exp(logits - m)
+            out[b, hq] = (p @ Vhat[b, kv]) / np.sum(p)
+    return out
+
+
+def decode(q: np.ndarray, packed: np.ndarray, alloc: dict, bits_v: int, seq_len: int) -> np.ndarray:
+    """Fused-path reference: unpack the stored bits, dequantize, attend (fp64)."""
+    u = unpack_cache(packed, alloc, bits_v, seq_len)
+    Khat = dequantize_keys(u["Kc"], u["Kn"], alloc)
+    Vhat = dequantize_values(u["Vc"], u["Vn"], bits_v)
+    return decode_attention(q, Khat, Vhat)

@@ -1,0 +1,565 @@
+"""Pins for the CPU oracle: closed forms, textbook constants, brute force, invariants.
+
+None of these compares the oracle with itself: each value on the right-hand
+side comes from mathematics, an independent routine (quadrature, exhaustive
+search, dynamic programming, Monte Carlo) or a published constant.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy import integrate
+from scipy.stats import norm
+
+from oracle import blockgtq as bg
+from oracle import codebooks as cb
+from oracle import nqkv
+from oracle import rope
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([float(x) for x in line.split()])
+    return rows
+
+
+# ----------------------------------------------------------------- pin 1: RoPE blocks
+
+def test_rope_logit_is_sum_of_block_terms():
+    """Block-GTQ abstract: under RoPE a key's logit contribution is a position-dependent
+    sum over 2-D frequency blocks. Checked at every key position of the tiny workload."""
+    rng = np.random.default_rng(0)
+    d, base = 128, 1e4
+    q = rng.standard_normal(d)
+    for n in range(512):
+        k = rng.standard_normal(d) * 10.0 ** rng.uniform(-1, 1, d)
+        direct = float(np.dot(rope.rotate(q, 512.0, base), rope.rotate(k, float(n), base)))
+        terms = rope.block_logit_terms(q, k, 512.0, float(n), base)
+        assert abs(math.fsum(terms) - direct) <= 1e-12 * max(1.0, float(np.sum(np.abs(q) * np.abs(k))))
+
+
+def test_rope_preserves_block_energy():
+    rng = np.random.default_rng(1)
+    k = rng.standard_normal(128) * 3.0
+    e0 = rope.block_energy(k)
+    for pos in (1.0, 17.0, 511.0, 131071.0):
+        e1 = rope.block_energy(rope.rotate(k, pos, 1e6))
+        np.testing.assert_allclose(e1, e0, rtol=1e-13, atol=0)
+
+
+def test_rope_pairing_is_rotate_half():
+    """A planted change of pairing (adjacent dims instead of (i, i + d/2)) breaks the identity."""
+    rng = np.random.default_rng(2)
+    q, k = rng.standard_normal(8), rng.standard_normal(8)
+    perm = np.array([0, 2, 4, 6, 1, 3, 5, 7])           # interleaved pairing
+    direct = np.dot(rope.rotate(q, 5.0, 1e4), rope.rotate(k, 2.0, 1e4))
+    wrong = np.sum(rope.block_logit_terms(q[perm], k[perm], 5.0, 2.0, 1e4))
+    assert abs(direct - wrong) > 1e-6
+
+
+# ----------------------------------------------------------------- pin 2: Lloyd-Max
+
+def test_lloyd_max_closed_form_one_bit():
+    c, t = cb.lloyd_max_f64(1)
+    assert abs(c[1] - math.sqrt(2.0 / math.pi)) < 1e-14
+    assert abs(c[0] + math.sqrt(2.0 / math.pi)) < 1e-14
+    assert t[0] == 0.0
+    assert abs(cb.quantizer_mse(c, t) - (1.0 - 2.0 / math.pi)) < 1e-14
+
+
+def test_lloyd_max_textbook_distortions():
+    """Agreement within one unit of the last quoted digit (the table quotes 4 significant
+    digits; 0.0345478 is quoted as 0.03454 there)."""
+    for bits, mse in _golden_rows("lloyd_max_textbook.txt"):
+        c, t = cb.lloyd_max_f64(int(bits))
+        got = cb.quantizer_mse(c, t)
+        unit = 10.0 ** (math.floor(math.log10(mse)) - 3)
+        assert abs(got - mse) <= unit, (bits, got, mse)
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 4, 5, 6])
+def test_lloyd_max_centroids_are_conditional_means(w):
+    """Independent check by adaptive quadrature of x phi(x) and phi(x) over each cell."""
+    c, t = cb.lloyd_max_f64(w)
+    a = np.concatenate([[-np.inf], t])
+    b = np.concatenate([t, [np.inf]])
+    for ci, ai, bi in zip(c, a, b):
+        num = integrate.quad(lambda x: x * norm.pdf(x), ai, bi, epsabs=1e-14, epsrel=1e-13)[0]
+        den = integrate.quad(norm.pdf, ai, bi, epsabs=1e-14, epsrel=1e-13)[0]
+        assert abs(num / den - ci) < 1e-11
+    np.testing.assert_allclose(t, 0.5 * (c[:-1] + c[1:]), rtol=0, atol=0)
+
+
+def test_lloyd_max_mse_by_quadrature():
+    for w in (2, 3, 4, 8):
+        c, t = cb.lloyd_max_f64(w)
+        a = np.concatenate([[-np.inf], t])
+        b = np.concatenate([t, [np.inf]])
+        mse = math.fsum(integrate.quad(lambda x: (x - ci) ** 2 * norm.pdf(x), ai, bi,
+                                       epsabs=1e-15, epsrel=1e-13)[0] for ai, bi, ci in zip(a, b, c))
+        assert abs(mse - cb.quantizer_mse(c, t)) < 1e-12
+
+
+def test_stored_codebooks_symmetric_and_sorted():
+    for w in range(1, 9):
+        c16, t32 = cb.stored_codebook(w)
+        assert len(c16) == 2 ** w and len(t32) == 2 ** w - 1
+        assert np.all(np.diff(c16.astype(np.float64)) > 0)
+        assert np.all(np.diff(t32.astype(np.float64)) > 0)
+        np.testing.assert_array_equal(c16, -c16[::-1])
+        assert t32[(len(t32) - 1) // 2] == 0.0          # middle threshold is exactly 0
+        # each stored centroid is the fp16 value nearest the exact one
+        exact, _ = cb.lloyd_max_f64(w)
+        assert np.all(np.abs(c16.astype(np.float64) - exact) <= np.spacing(np.abs(c16)).astype(np.float64) / 2)
+
+
+def test_delta_table_convex_and_close_to_exact():
+    delta = cb.delta_table().astype(np.float64)
+    assert delta[0] == 1.0
+    gains = delta[:-1] - delta[1:]
+    assert np.all(gains > 0)
+    assert np.all(np.diff(gains) < 0)                   # strictly convex
+    for w in range(1, 9):
+        # The exact Lloyd-Max quantizer is MSE-optimal, so rounding its centroids to fp16 can
+        # only raise the MSE, and by at most the largest squared centroid shift.
+        c, t = cb.lloyd_max_f64(w)
+        exact = cb.quantizer_mse(c, t)
+        shift = np.max(np.abs(cb.stored_codebook(w)[0].astype(np.float64) - c))
+        assert exact * (1 - 1e-7) <= delta[w] <= exact * (1 + 1e-7) + shift ** 2
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 4])
+def test_stored_quantizer_monte_carlo(w):
+    """10^7 N(0,1) draws through the fp32 threshold quantizer: MSE within 3 sigma of delta(w)."""
+    rng = np.random.default_rng(100 + w)
+    x = rng.standard_normal(10_000_000).astype(np.float32)
+    c16, t32 = cb.stored_codebook(w)
+    codes = np.searchsorted(t32, x, side="left")
+    err = (x.astype(np.float64) - c16.astype(np.float64)[codes]) ** 2
+    mean, sd = err.mean(), err.std() / math.sqrt(len(err))
+    assert abs(mean - float(cb.delta_table()[w])) < 3 * sd
+
+
+def test_threshold_count_is_nearest_centroid():
+    """code = #{t < y} equals the brute-force nearest fp16 centroid (away from exact ties)."""
+    rng = np.random.default_rng(3)
+    for w in range(1, 9):
+        c16, t32 = cb.stored_codebook(w)
+        y = (rng.standard_normal(20000) * 1.5).astype(np.float32)
+        codes = np.sum(y[:, None] > t32[None, :], axis=1)
+        dist = np.abs(y[:, None].astype(np.float64) - c16[None, :].astype(np.float64))
+        near = np.argmin(dist, axis=1)
+        srt = np.sort(dist, axis=1)
+        clear = srt[:, 1] - srt[:, 0] > 1e-6
+        np.testing.assert_array_equal(codes[clear], near[clear])
+
+
+# ----------------------------------------------------------------- pin 3: NF4
+
+def test_nf4_matches_published_table():
+    vals = np.array([r[0] for r in _golden_rows("nf4_qlora.txt")])
+    got = cb.nf4_values().astype(np.float64)
+    assert got.shape == (16,)
+    np.testing.assert_allclose(got, vals, rtol=0, atol=5e-7)
+
+
+def test_nf4_structure_and_quantile_spacing():
+    v = cb.nf4_values().astype(np.float64)
+    assert np.all(np.diff(v) > 0) and v[0] == -1.0 and v[-1] == 1.0
+    assert np.sum(v == 0.0) == 1 and np.sum(v < 0) == 7 and np.sum(v > 0) == 8
+    # Undo the normalisation with the quantile of the outermost level; the levels are then
+    # standard-normal quantiles at evenly spaced probabilities on each side (scipy's norm.cdf).
+    off = 0.5 * ((1 - 1 / 30) + (1 - 1 / 32))
+    z = norm.ppf(off)
+    ppos = norm.cdf(v[v > 0] * z)
+    pneg = norm.cdf(-v[v < 0] * z)
+    np.testing.assert_allclose(np.diff(ppos), (off - 0.5) / 8, rtol=1e-5)
+    np.testing.assert_allclose(np.diff(np.sort(pneg)), (off - 0.5) / 7, rtol=1e-5)
+
+
+def test_nf4_midpoints_between_levels():
+    v = cb.nf4_values()
+    m = cb.nf4_midpoints()
+    assert np.all(m > v[:-1]) and np.all(m < v[1:])
+
+
+# ----------------------------------------------------------------- pin 4/5/6: greedy allocation
+
+def _objective(E, w):
+    delta = cb.delta_table().astype(np.float64)
+    return math.fsum(float(e) * delta[int(x)] for e, x in zip(E, w))
+
+
+def _brute_min(E, bits, w_max):
+    h = len(E)
+    delta = cb.delta_table().astype(np.float64)
+    grid = np.array(list(itertools.product(range(w_max + 1), repeat=h)), dtype=np.int64)
+    grid = grid[grid.sum(axis=1) == bits * h]
+    obj = (delta[grid] * np.asarray(E)[None, :]).sum(axis=1)
+    best = obj.min()
+    return best, grid[np.isclose(obj, best, rtol=1e-13, atol=0)]
+
+
+def _dp_min(E, bits, w_max):
+    delta = cb.delta_table().astype(np.float64)
+    budget = bits * len(E)
+    dp = np.full(budget + 1, np.inf)
+    dp[0] = 0.0
+    for e in E:
+        nxt = np.full(budget + 1, np.inf)
+        for s in range(budget + 1):
+            for w in range(min(w_max, s) + 1):
+                nxt[s] = min(nxt[s], dp[s - w] + e * delta[w])
+        dp = nxt
+    return dp[budget]
+
+
+@pytest.mark.parametrize("d", [4, 8, 12])
+def test_greedy_matches_exhaustive_search(d):
+    rng = np.random.default_rng(d)
+    h = d // 2
+    for trial in range(3):
+        E = np.exp(rng.standard_normal(h) * 1.5)
+        for bits in range(1, 9):
+            w = bg.greedy_widths(E, bits, 8)
+            assert int(w.sum()) == bits * h
+            best, argmins = _brute_min(E, bits, 8)
+            assert abs(_objective(E, w) - best) <= 1e-12 * best
+            if len(argmins) == 1:
+                np.testing.assert_array_equal(w, argmins[0])
+
+
+def test_greedy_matches_dynamic_programming_d16():
+    rng = np.random.default_rng(16)
+    for trial in range(3):
+        E = np.exp(rng.standard_normal(8) * 2.0)
+        for bits in range(1, 9):
+            w = bg.greedy_widths(E, bits, 8)
+            best = _dp_min(E, bits, 8)
+            assert abs(_objective(E, w) - best) <= 1e-12 * best
+
+
+def test_greedy_budget_and_wmax():
+    rng = np.random.default_rng(5)
+    E = np.exp(rng.standard_normal(64) * 2.0)
+    E[[3, 40]] *= 400.0
+    for bits in (2, 3, 4):
+        for w_max in (bits, 6, 8):
+            w = bg.greedy_widths(E, bits, w_max)
+            assert int(2 * w.sum()) == bits * 128            # allocated bits equal the budget
+            assert w.max() <= w_max and w.min() >= 0
+    assert np.all(bg.greedy_widths(E, 4, 4) == 4)            # budget at w_max forces uniform
+    with pytest.raises(ValueError):
+        bg.greedy_widths(E, 5, 4)
+
+
+def test_greedy_tie_breaks_to_lowest_block():
+    w = bg.greedy_widths(np.array([1.0, 1.0, 1.0]), 1, 8)
+    np.testing.assert_array_equal(w, [1, 1, 1])
+    # one step only: three equal candidates, the first wins
+    E = np.array([2.0, 2.0])
+    delta = cb.delta_table().astype(np.float64)
+    w = np.zeros(2, dtype=int)
+    gains = [E[b] * (delta[w[b]] - delta[w[b] + 1]) for b in range(2)]
+    assert gains[0] == gains[1]
+    np.testing.assert_array_equal(bg.greedy_widths(E, 1, 8), [1, 1])
+
+
+def test_equal_energies_give_uniform_tqmse():
+    d = 128
+    E = np.ones((1, 64))
+    for bits in (2, 3, 4):
+        a = bg.allocate(E, d, bits)
+        assert np.all(a["w"] == bits)
+        assert np.all(a["g"] == np.float32(1.0))
+        assert np.all(a["f"] == np.float32(1.0 / math.sqrt(d)))
+        rng = np.random.default_rng(bits)
+        X = rng.standard_normal((2, 1, 40, d)).astype(np.float32)
+        u = bg.allocate(E, d, bits, mode=bg.MODE_UNIFORM)
+        c1 = bg.quantize(X, X, a, bits)
+        c2 = bg.quantize(X, X, u, bits)
+        np.testing.assert_array_equal(c1["Kc"], c2["Kc"])
+        np.testing.assert_array_equal(c1["Kn"], c2["Kn"])
+
+
+def test_block_gains_restore_unit_variance():
+    """After the global sqrt(d)/||k|| scaling, block b's coordinates have variance
+    (E_b/2) d / sum E; g_b^2 times that is 1 for every block (closed form)."""
+    rng = np.random.default_rng(9)
+    E = np.exp(rng.standard_normal(64))
+    g, f = bg.block_gains(E, 128)
+    var = (E / 2.0) * 128 / E.sum()
+    np.testing.assert_allclose(g.astype(np.float64) ** 2 * var, 1.0, rtol=2e-7)
+    np.testing.assert_allclose(f.astype(np.float64) * math.sqrt(128) * g.astype(np.float64), 1.0, rtol=2e-7)
+
+
+# ----------------------------------------------------------------- calibration energy
+
+def test_energy_matches_exact_mean():
+    rng = np.random.default_rng(11)
+    K = (rng.standard_normal((3, 2, 200, 16)) * 10.0 ** rng.uniform(-1, 1, 16)).astype(np.float32)
+    E, N = bg.calibration_energies(K, n_calib=150)
+    assert N == 450
+    for hh in range(2):
+        X = K[:, hh, :150].reshape(-1, 16).astype(np.float64)
+        for b in range(8):
+            exact = math.fsum((X[:, b] ** 2 + X[:, b + 8] ** 2).tolist()) / N
+            assert abs(E[hh, b] - exact) <= 1e-13 * exact
+
+
+def test_energy_is_rope_invariant():
+    rng = np.random.default_rng(12)
+    d, T = 32, 300
+    k0 = rng.standard_normal((T, d)) * 10.0 ** rng.uniform(-1, 1, d // 2).repeat(2).reshape(2, -1).T.reshape(-1)
+    k1 = np.stack([rope.rotate(k0[t], float(t), 1e4) for t in range(T)])
+    E0, _ = bg.calibration_energies(k0[None, None], 0)
+    E1, _ = bg.calibration_energies(k1[None, None], 0)
+    np.testing.assert_allclose(E1, E0, rtol=1e-12)
+
+
+# ----------------------------------------------------------------- pin 8: quantizer
+
+def test_quantizer_zero_row_and_known_norm():
+    X = np.zeros((2, 128), dtype=np.float32)
+    X[1] = 1.0
+    for w in (1, 3, 8):
+        codes, n16 = bg.quantize_rows(X, np.full(128, w), np.ones(128, np.float32))
+        assert n16[0] == 0 and np.all(codes[0] == 2 ** (w - 1) - 1)   # y = 0 sits on the middle threshold
+        assert float(n16[1]) == 11.3125                                  # fp16(sqrt(128))
+    # y = 1 * fp32(sqrt 128) / 11.3125 = 1.000107..., width 1: above 0 -> code 1
+    codes, _ = bg.quantize_rows(X[1:], np.full(128, 1), np.ones(128, np.float32))
+    assert np.all(codes == 1)
+
+
+def test_quantizer_tie_goes_to_lower_code():
+    """A coordinate landing exactly on a threshold takes the lower code.
+
+    d = 4, row (t, r, 0, 0) with r chosen so the fp16 norm is exactly 2; then
+    a = fp32(sqrt 4) / 2 = 1 and y_0 = t, the sixth width-3 threshold.
+    """
+    c16, t32 = cb.stored_codebook(3)
+    x = np.zeros(4, dtype=np.float32)
+    x[0] = t32[5]
+    x[1] = np.float32(math.sqrt(4.0 - float(x[0]) ** 2))
+    codes, n16 = bg.quantize_rows(x[None], np.full(4, 3), np.ones(4, np.float32))
+    assert float(n16[0]) == 2.0
+    assert codes[0, 0] == 5                      # thresholds 0..4 lie strictly below y_0
+    x[0] = np.nextafter(t32[5], np.float32(10))
+    codes, _ = bg.quantize_rows(x[None], np.full(4, 3), np.ones(4, np.float32))
+    assert codes[0, 0] == 6
+
+
+def test_append_one_token_at_a_time_equals_batch():
+    """Append-only cache (NQKV assumptions): a per-row quantizer gives identical codes."""
+    rng = np.random.default_rng(13)
+    X = (rng.standard_normal((1, 1, 70, 128)) * 3).astype(np.float32)
+    E, _ = bg.calibration_energies(X, 0)
+    a = bg.allocate(E, 128, 3)
+    full = bg.quantize(X, X, a, 3)
+    for t in range(70):
+        one = bg.quantize(X[:, :, t:t + 1], X[:, :, t:t + 1], a, 3)
+        np.testing.assert_array_equal(one["Kc"][0, 0, 0], full["Kc"][0, 0, t])
+        assert one["Kn"][0, 0, 0] == full["Kn"][0, 0, t]
+
+
+# ----------------------------------------------------------------- pin 7: packed byte count
+
+def test_packed_bytes_per_token():
+    assert bg.tile_record_bytes(128, 3, 3) == 32 * 100                 # 48 + 48 + 4 bytes per token
+    fp16_bytes = 2 * 2 * 128
+    assert fp16_bytes / (bg.tile_record_bytes(128, 3, 3) / 32) == 5.12
+    assert bg.tile_record_bytes(128, 2, 2) == 32 * 68
+    assert bg.tile_record_bytes(128, 4, 4) == 32 * 132
+    assert bg.packed_bytes(1, 2, 131072, 128, 3, 3) == 26_214_400
+    assert bg.packed_bytes(1, 2, 100, 128, 3, 3) == 2 * 4 * 3200         # ragged tail rounds up to tiles
+    # NF4: 128 bytes of codes + one fp16 scale per 256 values
+    assert (128 + 2) * 8 / 256 == 4.0625
+    assert round(16 / 4.0625, 2) == 3.94
+
+
+# ----------------------------------------------------------------- layout
+
+def _alloc_with(w_blocks, d=128):
+    h = d // 2
+    return {"w": np.array([w_blocks]), "g": np.ones((1, h), np.float32),
+            "f": np.full((1, h), 1 / math.sqrt(d), np.float32), "E": np.ones((1, h)),
+            "d": d, "bits_k": int(sum(w_blocks)) * 2 // d, "w_max": 8, "mode": 0}
+
+
+def test_pack_single_code_position_by_hand():
+    """Hand-placed code: token 9, dim 3 + 64 (block 3), width 3, code 0b101.
+
+    Block widths: blocks 0..2 have 3 bits, block 3 has 3 bits, the rest are set so the
+    K budget is 3 bits/dim. Token 9 = 4*0 + 1 + 8*1 -> half H = 0, s = 1, m div 2 = 1;
+    dim b + h -> m odd -> m = 3; bit q = s + 4 m = 13. Block 3's segment starts at
+    word 2 * (3 + 3 + 3) = 18; planes 0 and 2 are words 18 + 0 and 18 + 4.
+    """
+    w = [3] * 64
+    a = _alloc_with(w)
+    Kc = np.zeros((1, 1, 32, 128), np.uint8)
+    Kc[0, 0, 9, 3 + 64] = 0b101
+    Vc = np.zeros((1, 1, 32, 128), np.uint8)
+    Vc[0, 0, 13, 70] = 0b011          # token 13 = 8*1 + 2*2 + 1 -> c = 2, m = 3 -> q = 2 + 12 = 14
+    codes = {"Kc": Kc, "Kn": np.zeros((1, 1, 32), np.float16), "Vc": Vc, "Vn": np.zeros((1, 1, 32), np.float16)}
+    packed = bg.pack_cache(codes, a, 3, 32)
+    words = packed[0, 0, 0, :4 * (384 + 384)].copy().view("<u4")
+    kw, vw = words[:384], words[384:]
+    nz = {i: int(x) for i, x in enumerate(kw) if x}
+    assert nz == {18: 1 << 13, 22: 1 << 13}
+    vnz = {i: int(x) for i, x in enumerate(vw) if x}
+    assert vnz == {0 * 128 + 70: 1 << 14, 1 * 128 + 70: 1 << 14}
+
+
+def test_pack_unpack_roundtrip_mixed_widths():
+    rng = np.random.default_rng(14)
+    d, h = 128, 64
+    w = np.full(h, 3)
+    w[:8] = [8, 0, 6, 0, 1, 5, 2, 2]
+    w[8] = 3 * h - int(w.sum() - w[8])
+    assert 0 <= w[8] <= 8
+    a = _alloc_with(list(w))
+    T = 77
+    wd = np.concatenate([w, w])
+    Kc = np.zeros((2, 1, T, d), np.uint8)
+    for j in range(d):
+        Kc[..., j] = rng.integers(0, 2 ** wd[j], size=(2, 1, T)) if wd[j] else 0
+    Vc = rng.integers(0, 8, size=(2, 1, T, d)).astype(np.uint8)
+    Kn = rng.standard_normal((2, 1, T)).astype(np.float16)
+    Vn = rng.standard_normal((2, 1, T)).astype(np.float16)
+    packed = bg.pack_cache({"Kc": Kc, "Kn": Kn, "Vc": Vc, "Vn": Vn}, a, 3, 100)
+    assert packed.shape == (2, 1, 4, 3200)
+    u = bg.unpack_cache(packed, a, 3, T)
+    np.testing.assert_array_equal(u["Kc"], Kc)
+    np.testing.assert_array_equal(u["Vc"], Vc)
+    np.testing.assert_array_equal(u["Kn"], Kn)
+    np.testing.assert_array_equal(u["Vn"], Vn)
+    tail = bg.unpack_cache(packed, a, 3, 128)
+    assert np.all(tail["Kc"][:, :, T:] == 0) and np.all(tail["Kn"][:, :, T:] == 0)
+
+
+# ----------------------------------------------------------------- pin 9: attention
+
+def test_attention_single_token_returns_its_value():
+    rng = np.random.default_rng(15)
+    q = rng.standard_normal((1, 4, 16))
+    K = rng.standard_normal((1, 2, 1, 16))
+    V = rng.standard_normal((1, 2, 1, 16))
+    out = bg.decode_attention(q, K, V)
+    np.testing.assert_allclose(out[0, :2], np.repeat(V[0, 0], 2, axis=0), rtol=1e-15)
+    np.testing.assert_allclose(out[0, 2:], np.repeat(V[0, 1], 2, axis=0), rtol=1e-15)
+
+
+def test_attention_zero_query_is_mean_of_values():
+    rng = np.random.default_rng(16)
+    K = rng.standard_normal((1, 1, 50, 8))
+    V = rng.standard_normal((1, 1, 50, 8))
+    out = bg.decode_attention(np.zeros((1, 1, 8)), K, V)
+    np.testing.assert_allclose(out[0, 0], V[0, 0].mean(axis=0), rtol=1e-13)
+
+
+def test_attention_matches_online_softmax_restatement():
+    """Two-pass softmax vs the running-max (online) form over 7 chunks, both fp64."""
+    rng = np.random.default_rng(17)
+    d = 32
+    q = rng.standard_normal((1, 1, d)) * 3
+    K = rng.standard_normal((1, 1, 300, d)) * 2
+    V = rng.standard_normal((1, 1, 300, d))
+    ref = bg.decode_attention(q, K, V)[0, 0]
+    m, l, o = -np.inf, 0.0, np.zeros(d)
+    for chunk in np.array_split(np.arange(300), 7):
+        s = K[0, 0, chunk] @ q[0, 0] / math.sqrt(d)
+        mn = max(m, s.max())
+        scale = math.exp(m - mn) if np.isfinite(m) else 0.0
+        p = np.exp(s - mn)
+        l = l * scale + p.sum()
+        o = o * scale + p @ V[0, 0, chunk]
+        m = mn
+    np.testing.assert_allclose(o / l, ref, rtol=1e-14, atol=1e-15)
+
+
+def test_decode_from_packed_equals_direct_dequant():
+    rng = np.random.default_rng(18)
+    K = (rng.standard_normal((1, 2, 45, 128)) * np.exp(rng.standard_normal(128))).astype(np.float32)
+    V = rng.standard_normal((1, 2, 45, 128)).astype(np.float32)
+    q = rng.standard_normal((1, 4, 128)).astype(np.float32)
+    a = bg.calibrate(K, 3)
+    c = bg.quantize(K, V, a, 2)
+    packed = bg.pack_cache(c, a, 2, 64)
+    out = bg.decode(q, packed, a, 2, 45)
+    Khat = bg.dequantize_keys(c["Kc"], c["Kn"], a)
+    Vhat = bg.dequantize_values(c["Vc"], c["Vn"], 2)
+    np.testing.assert_array_equal(out, bg.decode_attention(q, Khat, Vhat))
+    # the dequantised keys approximate the originals (quantizer sanity, not exactness)
+    rel = np.linalg.norm(Khat - K) / np.linalg.norm(K)
+    assert rel < 0.25
+
+
+# ----------------------------------------------------------------- NF4
+
+def test_nf4_quantize_special_cases():
+    X = np.zeros((1, 2, 3, 128), np.float16)
+    X[0, 0, 1, 5] = 3.0
+    X[0, 1, 1, 0] = -1.5
+    X[0, :, 2, :] = np.float16(-0.25)
+    idx, s = nqkv.quantize(X)
+    assert idx.shape == (1, 1, 3, 256) and s.shape == (1, 1, 3)
+    assert s[0, 0, 0] == 0 and np.all(idx[0, 0, 0] == 7)            # zero block -> the exact-zero level
+    assert s[0, 0, 1] == 3.0 and idx[0, 0, 1, 5] == 15               # +absmax -> +1
+    assert idx[0, 0, 1, 128] == int(np.searchsorted(cb.nf4_midpoints(), np.float32(-0.5), "left"))
+    assert s[0, 0, 2] == 0.25 and np.all(idx[0, 0, 2] == 0)           # every value equals -absmax -> -1
+
+
+def test_nf4_pack_roundtrip_and_padding():
+    rng = np.random.default_rng(19)
+    idx = rng.integers(0, 16, size=(2, 3, 21, 256)).astype(np.uint8)
+    sc = rng.standard_normal((2, 3, 21)).astype(np.float16)
+    codes, scales = nqkv.pack(idx, sc, 21)
+    assert codes.shape == (2, 3, 32, 128) and scales.shape == (2, 3, 32)
+    assert codes[0, 0, 0, 0] == (idx[0, 0, 0, 0] | (idx[0, 0, 0, 1] << 4))
+    assert np.all(codes[:, :, 21:] == 0) and np.all(scales[:, :, 21:] == 0)
+    i2, s2 = nqkv.unpack(codes, scales, 21)
+    np.testing.assert_array_equal(i2, idx)
+    np.testing.assert_array_equal(s2, sc)
+
+
+def test_nf4_fig5_worked_shape():
+    """NQKV Fig. 5 shape: hidden 24, 1024 tokens, block 6 -> 4 blocks per token."""
+    rng = np.random.default_rng(20)
+    X = rng.standard_normal((1, 4, 1024, 6)).astype(np.float16)
+    idx, s = nqkv.quantize(X, block=6)
+    assert idx.shape == (1, 4, 1024, 6)
+    xh = nqkv.dequantize(idx, s, 4, 6)
+    v = cb.nf4_values().astype(np.float64)
+    gap = np.max(np.diff(v)) / 2
+    # with block == head_dim, block k of a token is head k, so scales align with X's heads
+    err = np.abs(xh - X.astype(np.float64))
+    bound = s.astype(np.float64)[..., None] * gap * (1 + 1e-6)
+    assert np.all(err <= bound)
+    # each block's absmax element is reconstructed exactly (+-1 times the fp16 scale)
+    amax = np.argmax(np.abs(X.astype(np.float64)), axis=-1)
+    got = np.take_along_axis(xh, amax[..., None], -1)[..., 0]
+    want = np.take_along_axis(X.astype(np.float64), amax[..., None], -1)[..., 0]
+    np.testing.assert_array_equal(got, want)
+
+
+def test_nf4_decode_masks_padding():
+    rng = np.random.default_rng(21)
+    X = rng.standard_normal((1, 2, 19, 128)).astype(np.float16)
+    q = rng.standard_normal((1, 2, 128)).astype(np.float16)
+    idx, s = nqkv.quantize(X)
+    kc, ks = nqkv.pack(idx, s, 19)
+    out = nqkv.decode(q, kc, ks, kc, ks, 2, 128, 19)
+    kc2 = kc.copy()
+    kc2[:, :, 19:] = 0x77                                             # garbage in the padded rows
+    out2 = nqkv.decode(q, kc2, ks, kc2, ks, 2, 128, 19)
+    np.testing.assert_array_equal(out, out2)
+    xh = nqkv.dequantize(*nqkv.unpack(kc, ks, 19), 2, 128)
+    np.testing.assert_allclose(out, bg.decode_attention(q.astype(np.float64), xh, xh), rtol=1e-14)
