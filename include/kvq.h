@@ -1,0 +1,217 @@
+/*
+ * libkvq — packed KV-cache quantization and fused decode attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Every data pointer is a DEVICE pointer unless the comment says "host". The caller
+ * owns all memory; the library never allocates. Buffer sizes come from the kvq_*_bytes
+ * queries. Every launch is asynchronous on the stream passed as `stream` (a cudaStream_t,
+ * NULL = legacy default stream). Argument errors are detected on the host and returned
+ * before anything is launched. A launch failure returns KVQ_ERR_CUDA. Device-side failures
+ * (a bounded wait that ran out) are recorded in the workspace's status word and read back
+ * with kvq_workspace_status(). No C++ exception crosses this boundary.
+ *
+ * The first call that launches work on a device uploads the constant tables (codebooks, NF4
+ * levels) to that device with a synchronous copy, so it must not be made while a stream is
+ * being captured; kvq_init() does the upload explicitly.
+ *
+ * Sources (restated in each declaration):
+ *   [BGTQ] "RoPE-aware bit allocation for KV cache quantization" (Liang, Zhang, Jia;
+ *          arXiv 2606.24033), abstract.
+ *   [NQKV] review of "NQKV: A KV Cache Quantization Scheme Based on Normal Distribution
+ *          Characteristics" (arXiv 2505.16210): mechanism paragraph, referee major
+ *          comment 1, assumptions, Figs. 5-7.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_ABI_VERSION 1
+#define KVQ_TILE_TOKENS 32     /* tokens per packed Block-GTQ tile */
+#define KVQ_HEAD_DIM 128       /* head dimension the kernels are built for */
+#define KVQ_MAX_WIDTH 8        /* widest Lloyd-Max codebook */
+#define KVQ_NF4_BLOCK 256      /* values per NF4 block */
+#define KVQ_NF4_PAD 16         /* NF4 token padding multiple */
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_ARG = 1,          /* null pointer, bad stride or alignment, inconsistent sizes */
+  KVQ_ERR_SHAPE = 2,        /* shape the kernels do not support (e.g. head_dim != 128) */
+  KVQ_ERR_DTYPE = 3,        /* unknown element type */
+  KVQ_ERR_BUDGET = 4,       /* bit budget outside 1..w_max or w_max outside 1..8 */
+  KVQ_ERR_RANGE = 5,        /* seq_len beyond the buffer's capacity */
+  KVQ_ERR_WORKSPACE = 6,    /* workspace missing or smaller than the size query says */
+  KVQ_ERR_CUDA = 7,         /* a CUDA runtime call or launch failed */
+  KVQ_ERR_TIMEOUT = 8,      /* a device-side bounded wait gave up (read via kvq_workspace_status) */
+  KVQ_ERR_UNSUPPORTED = 9   /* a combination the library does not implement */
+} kvq_status;
+
+typedef enum { KVQ_F32 = 0, KVQ_F16 = 1, KVQ_BF16 = 2 } kvq_dtype;
+
+typedef enum { KVQ_MODE_BLOCKGTQ = 0, KVQ_MODE_UNIFORM = 1 } kvq_mode;
+
+/* A [batch][n_heads][seq_len][head_dim] tensor view. Strides are in elements; the last
+ * dimension is contiguous. Every row start must be 16-byte aligned. */
+typedef struct {
+  int32_t batch;
+  int32_t n_heads;
+  int32_t seq_len;
+  int32_t head_dim;
+  int64_t stride_b;
+  int64_t stride_h;
+  int64_t stride_t;
+  int32_t dtype;            /* kvq_dtype */
+  int32_t reserved;
+} kvq_tensor4;
+
+/* Calibration settings. bits_k: K budget in bits per dimension (1..w_max). w_max: widest
+ * width a block may receive (1..8; 8 recommended). n_calib: leading tokens of every
+ * sequence used for the energy score (0 = all). mode: kvq_mode. */
+typedef struct {
+  int32_t bits_k;
+  int32_t w_max;
+  int32_t n_calib;
+  int32_t mode;
+} kvq_calib_params;
+
+/* Shape of one packed Block-GTQ cache buffer (one layer). capacity = tokens per sequence
+ * the buffer holds; storage is rounded up to whole 32-token tiles. */
+typedef struct {
+  int32_t batch;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t capacity;
+  int32_t bits_k;
+  int32_t bits_v;
+} kvq_cache_desc;
+
+/* Allocation record of one KV head, as written by kvq_calibrate (device memory, array of
+ * n_kv_heads records). Block b covers dims b and b + head_dim/2. */
+typedef struct {
+  double energy[64];        /* E_b, mean ||k_b||^2 over the calibration tokens */
+  float gain[64];           /* g_b, per-block scale applied before the codebook */
+  float dequant[64];        /* f_b = 1 / (sqrt(d) g_b) */
+  uint16_t word_off[64];    /* word offset of block b's segment in a tile's K part */
+  uint8_t width[64];        /* w_b, bits per dim of block b */
+  uint8_t step_width[32];   /* decode k-steps: width of the blocks in step s */
+  int8_t step_block[32][4]; /* decode k-steps: up to 4 blocks per step (-1 = none) */
+  int32_t head_dim;
+  int32_t bits_k;
+  int32_t w_max;
+  int32_t mode;
+  int32_t n_steps;          /* number of valid decode k-steps */
+  int32_t k_words;          /* 32-bit words in a tile's K part (= bits_k * head_dim) */
+  int32_t reserved[2];
+} kvq_head_alloc;
+
+/* ---------------------------------------------------------------- queries (host only) */
+
+int kvq_abi_version(void);
+const char* kvq_status_string(int status);
+
+/* Host copy of the width-w Lloyd-Max codebook (w = 1..8) for N(0,1), as used by the
+ * kernels: 2^w centroids as fp16 bit patterns, 2^w - 1 fp32 thresholds (midpoints of
+ * adjacent fp16 centroids) and delta = fp32 MSE of that quantizer on N(0,1).
+ * Any output pointer (host) may be NULL. [BGTQ]: TQ-MSE is the base quantizer. */
+kvq_status kvq_codebook(int width, uint16_t* centroids_f16, float* thresholds, float* delta);
+
+/* Host copy of the 16 NF4 levels (fp32, ascending) and 15 fp32 midpoints.
+ * [NQKV] mechanism paragraph: 16 standard-normal quantiles imported from QLoRA. */
+kvq_status kvq_nf4_table(float* levels, float* midpoints);
+
+/* Bytes of the allocation buffer for n_kv_heads heads (n_kv_heads * sizeof(kvq_head_alloc)). */
+size_t kvq_alloc_bytes(int n_kv_heads);
+
+/* Workspace bytes kvq_calibrate needs for this many sequences, KV heads and calibration
+ * tokens per sequence. */
+size_t kvq_calibrate_workspace_bytes(int batch, int n_kv_heads, int n_calib_tokens);
+
+/* Bytes of one packed cache: batch * n_kv_heads * ceil(capacity/32) tile records, each
+ * 4 * head_dim * (bits_k + bits_v) + 128 bytes. Returns 0 for an invalid descriptor. */
+size_t kvq_packed_bytes(const kvq_cache_desc* cache);
+
+/* Workspace bytes kvq_decode_attn needs for this cache and n_q_heads query heads. */
+size_t kvq_decode_workspace_bytes(const kvq_cache_desc* cache, int n_q_heads);
+
+/* ---------------------------------------------------------------- setup and status */
+
+/* Uploads the constant tables to the current device (synchronous). Optional: the first
+ * launching call does it too. */
+kvq_status kvq_init(void);
+
+/* Zero a decode or calibrate workspace (async memset on `stream`). A decode workspace must
+ * be zeroed once before its first use; the kernels leave it reusable. */
+kvq_status kvq_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronizes `stream`, copies the workspace status word to *device_code (host) and
+ * returns KVQ_OK if it is 0, else the recorded kvq_status (e.g. KVQ_ERR_TIMEOUT). */
+kvq_status kvq_workspace_status(const void* ws, void* stream, int* device_code);
+
+/* ---------------------------------------------------------------- Block-GTQ hot path */
+
+/* Calibration ([BGTQ]: "for each layer and KV head, a label-free energy score for each
+ * RoPE block, then greedily allocates integer bit widths by marginal gain").
+ * K: keys [batch][n_kv_heads][seq_len][128] in kd->dtype (post-RoPE, as cached).
+ * Two launches: a fixed-order fp64 reduction of E_b = mean_t (k_b^2 + k_{b+64}^2) over the
+ * first n_calib tokens of every sequence (pooled), then the greedy allocation:
+ * bits_k * 64 steps, each adding one bit to the block with the largest
+ * E_b (delta(w_b) - delta(w_b + 1)) below w_max, ties to the lowest block.
+ * Writes n_kv_heads kvq_head_alloc records to alloc_out.
+ * ws: workspace of kvq_calibrate_workspace_bytes(batch, n_kv_heads, n_calib) bytes. */
+kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_params* params,
+                         void* alloc_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Quantize and pack the first kd->seq_len tokens of K and V into `packed` ([BGTQ]: Block-GTQ
+ * on TQ-MSE, matched K/V budgets, packed cache). Per token row: fp16 norm, a = sqrt(d)/norm,
+ * y = (x a) g_b in fp32, code = number of thresholds below y; K uses the allocation's
+ * widths and gains, V uses width cache->bits_v and g = 1. Tiles past seq_len are not
+ * written; tokens of the last tile beyond seq_len are stored as code 0, norm 0.
+ * K, V: [batch][n_kv_heads][seq_len][128] (kd, vd may differ in strides, not in shape).
+ * alloc: records from kvq_calibrate with bits_k == cache->bits_k.
+ * packed: kvq_packed_bytes(cache) bytes, 16-byte aligned. */
+kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd,
+                        const void* alloc, const kvq_cache_desc* cache, void* packed, void* stream);
+
+/* Fused decode attention straight from the packed cache ([BGTQ]: packed-cache serving path).
+ * q: [batch][n_q_heads][1][128] (qd->seq_len must be 1), query head hq reads KV head
+ * hq / (n_q_heads / n_kv_heads); n_q_heads / n_kv_heads must be 1..8.
+ * out: fp32 [batch][n_q_heads][128], contiguous. Attends over cached positions
+ * 0..seq_len-1: out = sum_t softmax_t(q . k_hat_t / sqrt(d)) v_hat_t with
+ * k_hat = norm * c[code] * f_b and v_hat = norm * c[code] / sqrt(d).
+ * ws: kvq_decode_workspace_bytes bytes, zeroed once by kvq_workspace_init. */
+kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
+                           const kvq_cache_desc* cache, int seq_len, float* out, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- NQKV-style NF4 variant */
+
+/* Bytes of an NF4 cache for K and V: per (sequence, 256-value block): T_pad rows of 128
+ * code bytes, for K then V, followed by fp16 scales for K then V; T_pad = ceil(capacity/16)*16. */
+size_t kvq_nf4_packed_bytes(int batch, int n_heads, int capacity, int head_dim);
+
+/* Workspace bytes kvq_nf4_decode_attn needs. */
+size_t kvq_nf4_decode_workspace_bytes(int batch, int n_heads, int capacity, int head_dim);
+
+/* NF4 quantize ([NQKV]: blocks of 256 values along each token's head-major hidden vector,
+ * scale = fp16(absmax) with no mean subtraction, index = nearest NF4 level, 2 nibbles per
+ * byte with value 2k in the low nibble of byte k; token rows padded to a multiple of 16).
+ * K, V: [batch][n_heads][seq_len][128], n_heads even. Rows seq_len..T_pad-1 are written as
+ * code 0, scale 0. */
+kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd,
+                            int capacity, void* packed, void* stream);
+
+/* NF4 MHA decode attention ([NQKV]: dequantization is a table lookup; padding zeros are
+ * masked): out[b][h] = sum_t softmax_t(q . x_hat / sqrt(d)) v_hat over t < seq_len with
+ * x_hat = scale * NF4[idx]. q: [batch][n_heads][1][128]; out fp32 [batch][n_heads][128]. */
+kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, int capacity,
+                               int seq_len, float* out, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

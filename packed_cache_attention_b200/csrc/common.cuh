@@ -1,0 +1,106 @@
+// Device-side helpers shared by the libkvq kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "../../include/kvq.h"
+#include "tables.h"
+
+namespace kvq {
+
+constexpr int kTile = KVQ_TILE_TOKENS;   // tokens per packed tile
+constexpr int kD = KVQ_HEAD_DIM;         // head dim of the kernels
+constexpr int kH = kD / 2;               // RoPE blocks per head
+constexpr int kCalibChunk = 64;          // tokens per fixed-order energy partial sum
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Constant tables on the device (uploaded once per device from tables()).
+struct DevTables {
+  uint16_t centroid_f16[kCentroidCount];
+  float threshold[kThresholdCount];
+  float delta[9];
+  float nf4[16];
+  float nf4_mid[15];
+};
+
+// Device copy of the tables. This header is compiled into a single translation unit
+// (kvq.cu), which owns the symbol and uploads it once per device.
+__constant__ DevTables c_tab;
+
+// Workspace status word: first 4 bytes of every workspace.
+struct WsHeader {
+  unsigned int status;
+  unsigned int pad[31];   // keep the payload 128-byte aligned
+};
+
+// ---------------------------------------------------------------- element loads
+
+template <int DT> struct Elem;
+template <> struct Elem<KVQ_F32> {
+  using T = float;
+  __device__ __forceinline__ static float to_f32(float x) { return x; }
+};
+template <> struct Elem<KVQ_F16> {
+  using T = __half;
+  __device__ __forceinline__ static float to_f32(__half x) { return __half2float(x); }
+};
+template <> struct Elem<KVQ_BF16> {
+  using T = __nv_bfloat16;
+  __device__ __forceinline__ static float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+};
+
+// ---------------------------------------------------------------- bit helpers
+
+__device__ __forceinline__ uint32_t rotr(uint32_t x, uint32_t n) { return __funnelshift_r(x, x, n); }
+
+__device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
+  return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_u16x2(uint32_t lo, uint32_t hi) { return (lo & 0xffffu) | (hi << 16); }
+
+// ---------------------------------------------------------------- tensor-core fragments
+// mma.sync m16n8k8 / m16n8k16, fp16 operands, fp32 accumulate (row.col).
+
+__device__ __forceinline__ void mma_m16n8k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+__device__ __forceinline__ void mma_m16n8k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Split an fp32 value into fp16 hi + lo with hi + lo == x to ~2^-22 relative.
+__device__ __forceinline__ void split_hilo(float x, __half& hi, __half& lo) {
+  hi = __float2half_rn(x);
+  lo = __float2half_rn(x - __half2float(hi));
+}
+
+// ---------------------------------------------------------------- async copies (cp.async, 16 B)
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+}  // namespace kvq

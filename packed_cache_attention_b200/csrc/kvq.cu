@@ -1,0 +1,393 @@
+// libkvq C ABI: argument validation, buffer-size queries, table upload and kernel launches.
+// The declarations, with the passages each operation follows, are in include/kvq.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "calibrate.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+#include "nf4.cuh"
+#include "quantize.cuh"
+
+using namespace kvq;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_upload_mu;
+bool g_uploaded[kMaxDevices] = {};
+
+kvq_status ensure_tables() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_upload_mu);
+  if (g_uploaded[dev]) return KVQ_OK;
+  const Tables& t = tables();
+  DevTables d;
+  std::memcpy(d.centroid_f16, t.centroid_f16, sizeof(d.centroid_f16));
+  std::memcpy(d.threshold, t.threshold, sizeof(d.threshold));
+  std::memcpy(d.delta, t.delta, sizeof(d.delta));
+  std::memcpy(d.nf4, t.nf4, sizeof(d.nf4));
+  std::memcpy(d.nf4_mid, t.nf4_mid, sizeof(d.nf4_mid));
+  if (cudaMemcpyToSymbol(c_tab, &d, sizeof(d)) != cudaSuccess) return KVQ_ERR_CUDA;
+  g_uploaded[dev] = true;
+  return KVQ_OK;
+}
+
+size_t elem_size(int dtype) {
+  switch (dtype) {
+    case KVQ_F32: return 4;
+    case KVQ_F16: return 2;
+    case KVQ_BF16: return 2;
+    default: return 0;
+  }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks a [B][H][T][128] view: supported dtype, positive sizes, 16-byte aligned rows.
+kvq_status check_tensor(const void* ptr, const kvq_tensor4* t) {
+  if (!ptr || !t) return KVQ_ERR_ARG;
+  const size_t es = elem_size(t->dtype);
+  if (es == 0) return KVQ_ERR_DTYPE;
+  if (t->head_dim != kD) return KVQ_ERR_SHAPE;
+  if (t->batch < 1 || t->n_heads < 1 || t->seq_len < 1) return KVQ_ERR_SHAPE;
+  if (t->stride_b < 0 || t->stride_h < 0 || t->stride_t < 0) return KVQ_ERR_ARG;
+  if (!aligned16(ptr)) return KVQ_ERR_ARG;
+  if (((t->stride_b * es) % 16) || ((t->stride_h * es) % 16) || ((t->stride_t * es) % 16)) return KVQ_ERR_ARG;
+  if (t->seq_len > 1 && t->stride_t < kD) return KVQ_ERR_ARG;
+  return KVQ_OK;
+}
+
+bool cache_ok(const kvq_cache_desc* c) {
+  return c && c->batch >= 1 && c->n_kv_heads >= 1 && c->head_dim == kD && c->capacity >= 1 && c->bits_k >= 1 &&
+         c->bits_k <= 8 && c->bits_v >= 1 && c->bits_v <= 8;
+}
+
+size_t tile_record_bytes(int bits_k, int bits_v) { return 4ull * kD * (bits_k + bits_v) + 4ull * kTile; }
+
+int n_tiles_of(int tokens) { return (tokens + kTile - 1) / kTile; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int decode_splits(int bh, int n_tiles) {
+  const int want = (kTargetCtas + bh - 1) / bh;
+  return std::max(1, std::min(want, n_tiles));
+}
+
+struct DecodeWs {
+  size_t tickets, part_m, part_l, part_o, total;
+};
+
+DecodeWs decode_ws_layout(int bh, int splits, int rows) {
+  DecodeWs w;
+  w.tickets = sizeof(WsHeader);
+  w.part_m = align_up(w.tickets + 4ull * bh, 128);
+  w.part_l = align_up(w.part_m + 4ull * bh * splits * rows, 128);
+  w.part_o = align_up(w.part_l + 4ull * bh * splits * rows, 128);
+  w.total = align_up(w.part_o + 4ull * bh * splits * rows * kD, 128);
+  return w;
+}
+
+kvq_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+Nf4Layout nf4_layout(int batch, int n_heads, int capacity) {
+  Nf4Layout L;
+  L.nblk = n_heads * kD / KVQ_NF4_BLOCK;
+  L.t_pad = (capacity + KVQ_NF4_PAD - 1) / KVQ_NF4_PAD * KVQ_NF4_PAD;
+  L.codes_bytes = static_cast<size_t>(batch) * L.nblk * L.t_pad * 128;
+  return L;
+}
+
+size_t decode_smem_bytes(int rec_bytes) {
+  const size_t head = align_up(sizeof(DecodeSmem), 128);
+  const size_t stage = align_up(rec_bytes, 128) * kDecStages * kDecWarps;
+  const size_t combine = sizeof(float) * (kDecWarps * 8 * 2 + kDecWarps * 8 * kD);
+  return head + std::max(stage, combine);
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvq_abi_version(void) { return KVQ_ABI_VERSION; }
+
+const char* kvq_status_string(int s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_ARG: return "invalid argument";
+    case KVQ_ERR_SHAPE: return "unsupported shape";
+    case KVQ_ERR_DTYPE: return "unsupported dtype";
+    case KVQ_ERR_BUDGET: return "bit budget out of range";
+    case KVQ_ERR_RANGE: return "sequence length out of range";
+    case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case KVQ_ERR_CUDA: return "CUDA error";
+    case KVQ_ERR_TIMEOUT: return "device wait timed out";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    default: return "unknown status";
+  }
+}
+
+kvq_status kvq_codebook(int width, uint16_t* centroids_f16, float* thresholds, float* delta) {
+  if (width < 1 || width > 8) return KVQ_ERR_ARG;
+  const Tables& t = tables();
+  const int n = 1 << width;
+  if (centroids_f16) std::memcpy(centroids_f16, t.centroid_f16 + centroid_offset(width), n * sizeof(uint16_t));
+  if (thresholds) std::memcpy(thresholds, t.threshold + threshold_offset(width), (n - 1) * sizeof(float));
+  if (delta) *delta = t.delta[width];
+  return KVQ_OK;
+}
+
+kvq_status kvq_nf4_table(float* levels, float* midpoints) {
+  const Tables& t = tables();
+  if (levels) std::memcpy(levels, t.nf4, sizeof(t.nf4));
+  if (midpoints) std::memcpy(midpoints, t.nf4_mid, sizeof(t.nf4_mid));
+  return KVQ_OK;
+}
+
+size_t kvq_alloc_bytes(int n_kv_heads) {
+  return n_kv_heads > 0 ? static_cast<size_t>(n_kv_heads) * sizeof(kvq_head_alloc) : 0;
+}
+
+size_t kvq_calibrate_workspace_bytes(int batch, int n_kv_heads, int n_calib_tokens) {
+  if (batch < 1 || n_kv_heads < 1 || n_calib_tokens < 1) return 0;
+  const long long N = static_cast<long long>(batch) * n_calib_tokens;
+  const long long chunks = (N + kCalibChunk - 1) / kCalibChunk;
+  return sizeof(WsHeader) + static_cast<size_t>(n_kv_heads) * chunks * kH * sizeof(double);
+}
+
+size_t kvq_packed_bytes(const kvq_cache_desc* c) {
+  if (!cache_ok(c)) return 0;
+  return static_cast<size_t>(c->batch) * c->n_kv_heads * n_tiles_of(c->capacity) * tile_record_bytes(c->bits_k, c->bits_v);
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_cache_desc* c, int n_q_heads) {
+  if (!cache_ok(c) || n_q_heads < 1) return 0;
+  const int bh = c->batch * c->n_kv_heads;
+  return decode_ws_layout(bh, decode_splits(bh, n_tiles_of(c->capacity)), 8).total;
+}
+
+kvq_status kvq_init(void) { return ensure_tables(); }
+
+kvq_status kvq_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < sizeof(WsHeader)) return KVQ_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_workspace_status(const void* ws, void* stream, int* device_code) {
+  if (!ws) return KVQ_ERR_WORKSPACE;
+  unsigned int code = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&code, ws, sizeof(code), cudaMemcpyDeviceToHost, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (device_code) *device_code = static_cast<int>(code);
+  return code == 0 ? KVQ_OK : static_cast<kvq_status>(code);
+}
+
+kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_params* p, void* alloc_out,
+                         void* ws, size_t ws_bytes, void* stream) {
+  kvq_status st = check_tensor(K, kd);
+  if (st != KVQ_OK) return st;
+  if (!p || !alloc_out) return KVQ_ERR_ARG;
+  if (p->w_max < 1 || p->w_max > 8 || p->bits_k < 1 || p->bits_k > p->w_max) return KVQ_ERR_BUDGET;
+  if (p->mode != KVQ_MODE_BLOCKGTQ && p->mode != KVQ_MODE_UNIFORM) return KVQ_ERR_ARG;
+  if (p->n_calib < 0 || p->n_calib > kd->seq_len) return KVQ_ERR_RANGE;
+  const int n_calib = p->n_calib == 0 ? kd->seq_len : p->n_calib;
+  const size_t need = kvq_calibrate_workspace_bytes(kd->batch, kd->n_heads, n_calib);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return KVQ_ERR_WORKSPACE;
+  if ((st = ensure_tables()) != KVQ_OK) return st;
+  const long long N = static_cast<long long>(kd->batch) * n_calib;
+  if (N > 0x7fffffffLL) return KVQ_ERR_RANGE;
+  const int n_chunks = static_cast<int>((N + kCalibChunk - 1) / kCalibChunk);
+  double* partial = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + sizeof(WsHeader));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid(n_chunks, kd->n_heads);
+  switch (kd->dtype) {
+    case KVQ_F32:
+      kvq_calib_reduce<KVQ_F32><<<grid, 32, 0, s>>>(static_cast<const float*>(K), n_calib, kd->stride_b, kd->stride_h,
+                                                    kd->stride_t, static_cast<int>(N), n_chunks, partial);
+      break;
+    case KVQ_F16:
+      kvq_calib_reduce<KVQ_F16><<<grid, 32, 0, s>>>(static_cast<const __half*>(K), n_calib, kd->stride_b, kd->stride_h,
+                                                    kd->stride_t, static_cast<int>(N), n_chunks, partial);
+      break;
+    default:
+      kvq_calib_reduce<KVQ_BF16><<<grid, 32, 0, s>>>(static_cast<const __nv_bfloat16*>(K), n_calib, kd->stride_b,
+                                                     kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, partial);
+  }
+  if ((st = launch_status()) != KVQ_OK) return st;
+  kvq_greedy_alloc<<<kd->n_heads, 512, 0, s>>>(partial, n_chunks, static_cast<int>(N), p->bits_k, p->w_max, p->mode,
+                                               static_cast<kvq_head_alloc*>(alloc_out));
+  return launch_status();
+}
+
+kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, const void* alloc,
+                        const kvq_cache_desc* c, void* packed, void* stream) {
+  kvq_status st;
+  if ((st = check_tensor(K, kd)) != KVQ_OK) return st;
+  if ((st = check_tensor(V, vd)) != KVQ_OK) return st;
+  if (!alloc || !packed || !aligned16(packed)) return KVQ_ERR_ARG;
+  if (!cache_ok(c)) return KVQ_ERR_ARG;
+  if (vd->dtype != kd->dtype || vd->batch != kd->batch || vd->n_heads != kd->n_heads || vd->seq_len != kd->seq_len)
+    return KVQ_ERR_SHAPE;
+  if (kd->batch != c->batch || kd->n_heads != c->n_kv_heads) return KVQ_ERR_SHAPE;
+  if (kd->seq_len > c->capacity) return KVQ_ERR_RANGE;
+  if ((st = ensure_tables()) != KVQ_OK) return st;
+  const int tiles_written = n_tiles_of(kd->seq_len);
+  const int tiles_cap = n_tiles_of(c->capacity);
+  const long long n_tasks = static_cast<long long>(c->batch) * c->n_kv_heads * tiles_written;
+  const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
+  const size_t smem = 512 * 4 + static_cast<size_t>(kQuantWarps) * (c->bits_k + c->bits_v) * kD * 4;
+  const unsigned grid = static_cast<unsigned>((n_tasks + kQuantWarps - 1) / kQuantWarps);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+#define KVQ_LAUNCH_QUANT(DT, TY)                                                                                  \
+  do {                                                                                                            \
+    auto kern = kvq_quant_pack<DT>;                                                                               \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=        \
+        cudaSuccess)                                                                                              \
+      return KVQ_ERR_CUDA;                                                                                        \
+    kern<<<grid, kQuantWarps * 32, smem, s>>>(static_cast<const TY*>(K), kd->stride_b, kd->stride_h, kd->stride_t, \
+                                               static_cast<const TY*>(V), vd->stride_b, vd->stride_h, vd->stride_t, \
+                                               kd->seq_len, c->n_kv_heads, tiles_written, tiles_cap,              \
+                                               static_cast<const kvq_head_alloc*>(alloc), c->bits_k, c->bits_v,   \
+                                               static_cast<uint8_t*>(packed), rec, n_tasks);                      \
+  } while (0)
+  switch (kd->dtype) {
+    case KVQ_F32: KVQ_LAUNCH_QUANT(KVQ_F32, float); break;
+    case KVQ_F16: KVQ_LAUNCH_QUANT(KVQ_F16, __half); break;
+    default: KVQ_LAUNCH_QUANT(KVQ_BF16, __nv_bfloat16); break;
+  }
+#undef KVQ_LAUNCH_QUANT
+  return launch_status();
+}
+
+kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
+                           const kvq_cache_desc* c, int seq_len, float* out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  kvq_status st;
+  if ((st = check_tensor(q, qd)) != KVQ_OK) return st;
+  if (!packed || !alloc || !out || !aligned16(packed)) return KVQ_ERR_ARG;
+  if (!cache_ok(c)) return KVQ_ERR_ARG;
+  if (qd->seq_len != 1 || qd->batch != c->batch) return KVQ_ERR_SHAPE;
+  if (qd->n_heads % c->n_kv_heads != 0 || qd->n_heads / c->n_kv_heads > 8) return KVQ_ERR_UNSUPPORTED;
+  if (seq_len < 1 || seq_len > c->capacity) return KVQ_ERR_RANGE;
+  const int bh = c->batch * c->n_kv_heads;
+  const int n_tiles = n_tiles_of(seq_len);
+  const int splits = decode_splits(bh, n_tiles);
+  const DecodeWs L = decode_ws_layout(bh, splits, 8);
+  if (!ws || ws_bytes < L.total || !aligned16(ws) || ws_bytes < kvq_decode_workspace_bytes(c, qd->n_heads))
+    return KVQ_ERR_WORKSPACE;
+  if ((st = ensure_tables()) != KVQ_OK) return st;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
+  const size_t smem = decode_smem_bytes(rec);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid(splits, bh);
+#define KVQ_LAUNCH_DEC(DT, TY)                                                                                        \
+  do {                                                                                                                \
+    auto kern = kvq_decode_gtq<DT>;                                                                                   \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=            \
+        cudaSuccess)                                                                                                  \
+      return KVQ_ERR_CUDA;                                                                                            \
+    kern<<<grid, kDecWarps * 32, smem, s>>>(                                                                          \
+        static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, c->n_kv_heads,                             \
+        static_cast<const uint8_t*>(packed), static_cast<const kvq_head_alloc*>(alloc), n_tiles_of(c->capacity), rec, \
+        c->bits_v, seq_len, splits, out, reinterpret_cast<float*>(w8 + L.part_m),                                    \
+        reinterpret_cast<float*>(w8 + L.part_l), reinterpret_cast<float*>(w8 + L.part_o),                             \
+        reinterpret_cast<unsigned*>(w8 + L.tickets));                                                                 \
+  } while (0)
+  switch (qd->dtype) {
+    case KVQ_F32: KVQ_LAUNCH_DEC(KVQ_F32, float); break;
+    case KVQ_F16: KVQ_LAUNCH_DEC(KVQ_F16, __half); break;
+    default: KVQ_LAUNCH_DEC(KVQ_BF16, __nv_bfloat16); break;
+  }
+#undef KVQ_LAUNCH_DEC
+  return launch_status();
+}
+
+size_t kvq_nf4_packed_bytes(int batch, int n_heads, int capacity, int head_dim) {
+  if (batch < 1 || n_heads < 2 || (n_heads & 1) || capacity < 1 || head_dim != kD) return 0;
+  const Nf4Layout L = nf4_layout(batch, n_heads, capacity);
+  return 2 * L.codes_bytes + 2 * (L.codes_bytes / 128) * sizeof(__half);
+}
+
+size_t kvq_nf4_decode_workspace_bytes(int batch, int n_heads, int capacity, int head_dim) {
+  if (batch < 1 || n_heads < 1 || capacity < 1 || head_dim != kD) return 0;
+  const int bh = batch * n_heads;
+  return decode_ws_layout(bh, decode_splits(bh, (capacity + 31) / 32), 1).total;
+}
+
+kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, int capacity,
+                            void* packed, void* stream) {
+  kvq_status st;
+  if ((st = check_tensor(K, kd)) != KVQ_OK) return st;
+  if ((st = check_tensor(V, vd)) != KVQ_OK) return st;
+  if (!packed || !aligned16(packed)) return KVQ_ERR_ARG;
+  if (vd->dtype != kd->dtype || vd->batch != kd->batch || vd->n_heads != kd->n_heads || vd->seq_len != kd->seq_len)
+    return KVQ_ERR_SHAPE;
+  if (kd->n_heads & 1) return KVQ_ERR_SHAPE;
+  if (kd->seq_len > capacity) return KVQ_ERR_RANGE;
+  if ((st = ensure_tables()) != KVQ_OK) return st;
+  const Nf4Layout L = nf4_layout(kd->batch, kd->n_heads, capacity);
+  const long long tasks = 2LL * kd->batch * L.t_pad * L.nblk;
+  const unsigned grid = static_cast<unsigned>((tasks + kNf4Warps - 1) / kNf4Warps);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (kd->dtype) {
+    case KVQ_F32:
+      kvq_nf4_quant_pack<KVQ_F32><<<grid, kNf4Warps * 32, 0, s>>>(
+          static_cast<const float*>(K), kd->stride_b, kd->stride_h, kd->stride_t, static_cast<const float*>(V),
+          vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, kd->seq_len, L, static_cast<uint8_t*>(packed));
+      break;
+    case KVQ_F16:
+      kvq_nf4_quant_pack<KVQ_F16><<<grid, kNf4Warps * 32, 0, s>>>(
+          static_cast<const __half*>(K), kd->stride_b, kd->stride_h, kd->stride_t, static_cast<const __half*>(V),
+          vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, kd->seq_len, L, static_cast<uint8_t*>(packed));
+      break;
+    default:
+      kvq_nf4_quant_pack<KVQ_BF16><<<grid, kNf4Warps * 32, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(K), kd->stride_b, kd->stride_h, kd->stride_t,
+          static_cast<const __nv_bfloat16*>(V), vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, kd->seq_len, L,
+          static_cast<uint8_t*>(packed));
+  }
+  return launch_status();
+}
+
+kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, int capacity, int seq_len,
+                               float* out, void* ws, size_t ws_bytes, void* stream) {
+  kvq_status st;
+  if ((st = check_tensor(q, qd)) != KVQ_OK) return st;
+  if (!packed || !out) return KVQ_ERR_ARG;
+  if (qd->seq_len != 1 || (qd->n_heads & 1)) return KVQ_ERR_SHAPE;
+  if (seq_len < 1 || seq_len > capacity) return KVQ_ERR_RANGE;
+  const int bh = qd->batch * qd->n_heads;
+  const int splits = decode_splits(bh, (seq_len + 31) / 32);
+  const DecodeWs Lw = decode_ws_layout(bh, splits, 1);
+  if (!ws || ws_bytes < Lw.total || !aligned16(ws) ||
+      ws_bytes < kvq_nf4_decode_workspace_bytes(qd->batch, qd->n_heads, capacity, kD))
+    return KVQ_ERR_WORKSPACE;
+  if ((st = ensure_tables()) != KVQ_OK) return st;
+  const Nf4Layout L = nf4_layout(qd->batch, qd->n_heads, capacity);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid(splits, bh);
+#define KVQ_LAUNCH_NF4DEC(DT, TY)                                                                              \
+  kvq_nf4_decode<DT><<<grid, kDecWarps * 32, 0, s>>>(                                                          \
+      static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, static_cast<const uint8_t*>(packed), L, \
+      seq_len, splits, out, reinterpret_cast<float*>(w8 + Lw.part_m), reinterpret_cast<float*>(w8 + Lw.part_l),  \
+      reinterpret_cast<float*>(w8 + Lw.part_o), reinterpret_cast<unsigned*>(w8 + Lw.tickets))
+  switch (qd->dtype) {
+    case KVQ_F32: KVQ_LAUNCH_NF4DEC(KVQ_F32, float); break;
+    case KVQ_F16: KVQ_LAUNCH_NF4DEC(KVQ_F16, __half); break;
+    default: KVQ_LAUNCH_NF4DEC(KVQ_BF16, __nv_bfloat16); break;
+  }
+#undef KVQ_LAUNCH_NF4DEC
+  return launch_status();
+}
+
+}  // extern "C"

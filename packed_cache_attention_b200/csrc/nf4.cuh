@@ -1,0 +1,204 @@
+// NQKV-style NF4 variant (review of "NQKV: A KV Cache Quantization Scheme Based on Normal
+// Distribution Characteristics": 256-value blocks along each token's hidden vector, a
+// block scale from the maximum absolute value with no mean subtraction, 4-bit NF4
+// indices, dequantization by table lookup, token rows padded to a multiple of 16).
+//
+// Buffer layout (nblk = n_heads * 128 / 256 blocks per token, T_pad = ceil(capacity/16)*16):
+//   K codes [batch][nblk][T_pad][128 B] | V codes (same) | K scales [batch][nblk][T_pad] fp16
+//   | V scales (same). Byte k of a row holds value 2k (low nibble) and 2k+1 (high nibble);
+//   block blk of a token covers heads 2*blk (values 0..127) and 2*blk+1 (values 128..255).
+#pragma once
+
+#include "common.cuh"
+
+namespace kvq {
+
+constexpr int kNf4Warps = 8;
+
+struct Nf4Layout {
+  int nblk, t_pad;
+  size_t codes_bytes;   // one of K/V
+  __host__ __device__ size_t row(int b, int blk, int t) const {
+    return (static_cast<size_t>(b) * nblk + blk) * t_pad + t;
+  }
+};
+
+// One warp per (sequence, token row < T_pad, block, K-or-V). Lane l holds values
+// 8l..8l+7 of the block: head 2*blk + l/16, dims 8(l%16)..8(l%16)+7.
+template <int DT>
+__global__ void __launch_bounds__(kNf4Warps * 32) kvq_nf4_quant_pack(
+    const typename Elem<DT>::T* __restrict__ K, int64_t ksb, int64_t ksh, int64_t kst,
+    const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst, int batch,
+    int seq_len, Nf4Layout L, uint8_t* __restrict__ packed) {
+  using T = typename Elem<DT>::T;
+  __shared__ float sMid[16];
+  if (threadIdx.x < 15) sMid[threadIdx.x] = c_tab.nf4_mid[threadIdx.x];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long task = static_cast<long long>(blockIdx.x) * kNf4Warps + warp;
+  const long long per_kv = static_cast<long long>(batch) * L.t_pad * L.nblk;
+  if (task >= 2 * per_kv) return;
+  const int which = static_cast<int>(task / per_kv);          // 0 = K, 1 = V
+  long long r = task % per_kv;
+  const int blk = static_cast<int>(r % L.nblk);
+  r /= L.nblk;
+  const int t = static_cast<int>(r % L.t_pad);
+  const int b = static_cast<int>(r / L.t_pad);
+  const size_t row = L.row(b, blk, t);
+  uint32_t* codes = reinterpret_cast<uint32_t*>(packed + which * L.codes_bytes + row * 128);
+  __half* scales = reinterpret_cast<__half*>(packed + 2 * L.codes_bytes) + which * (L.codes_bytes / 128) + row;
+  if (t >= seq_len) {
+    codes[lane] = 0u;
+    if (lane == 0) *scales = __ushort_as_half(0);
+    return;
+  }
+  const T* X = which ? V : K;
+  const int64_t sb = which ? vsb : ksb, sh = which ? vsh : ksh, st = which ? vst : kst;
+  const int head = 2 * blk + (lane >> 4), d0 = 8 * (lane & 15);
+  const T* src = X + b * sb + head * sh + static_cast<int64_t>(t) * st + d0;
+  float x[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = Elem<DT>::to_f32(src[i]);
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const __half s16 = __float2half_rn(amax);
+  const float s = __half2float(s16);
+  uint32_t word = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float u = (s == 0.0f) ? 0.0f : __fdiv_rn(x[i], s);
+    int idx = 0;
+#pragma unroll
+    for (int k = 3; k >= 0; --k) idx += (u > sMid[idx + (1 << k) - 1]) ? (1 << k) : 0;
+    word |= static_cast<uint32_t>(idx) << (4 * i);
+  }
+  codes[lane] = word;
+  if (lane == 0) *scales = s16;
+}
+
+// MHA decode (G = 1), CUDA cores. Grid (splits, batch * n_heads), 4 warps per CTA, each
+// warp every 4th 32-token group of the CTA's range. Q.K: lane t scores token t of the
+// group from its 64 code bytes; P.V: lane l accumulates dims 4l..4l+3 over the group.
+template <int DT>
+__global__ void __launch_bounds__(kDecWarps * 32) kvq_nf4_decode(
+    const typename Elem<DT>::T* __restrict__ q, int64_t qsb, int64_t qsh, int n_heads, const uint8_t* __restrict__ packed,
+    Nf4Layout L, int seq_len, int splits, float* __restrict__ out, float* __restrict__ part_m,
+    float* __restrict__ part_l, float* __restrict__ part_o, unsigned* __restrict__ tickets) {
+  __shared__ float sQ[kD];
+  __shared__ float sLut[16];
+  __shared__ float cm[kDecWarps], cl[kDecWarps];
+  __shared__ float co[kDecWarps][kD];
+  __shared__ int sLast;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / n_heads, hh = bh % n_heads;
+  const int blk = hh >> 1, half_off = 64 * (hh & 1);
+  const float scl = 0.08838834764831845f * kLog2e;
+  if (tid < kD) sQ[tid] = Elem<DT>::to_f32(q[b * qsb + hh * qsh + tid]) * scl;
+  if (tid < 16) sLut[tid] = c_tab.nf4[tid];
+  __syncthreads();
+
+  const int n_groups = (seq_len + 31) / 32;
+  const int g0 = static_cast<int>((static_cast<long long>(split) * n_groups) / splits);
+  const int g1 = static_cast<int>((static_cast<long long>(split + 1) * n_groups) / splits);
+  const uint8_t* kc = packed;
+  const uint8_t* vc = packed + L.codes_bytes;
+  const __half* ks = reinterpret_cast<const __half*>(packed + 2 * L.codes_bytes);
+  const __half* vs = ks + L.codes_bytes / 128;
+
+  float m_run = -INFINITY, l_run = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int grp = g0 + warp; grp < g1; grp += kDecWarps) {
+    const int t = grp * 32 + lane;
+    float logit = -INFINITY;
+    if (t < seq_len) {
+      const size_t row = L.row(b, blk, t);
+      const uint4* kr = reinterpret_cast<const uint4*>(kc + row * 128 + half_off);
+      float accd = 0.0f;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 w4 = __ldg(kr + v);
+        const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int n = 0; n < 8; ++n) accd = fmaf(sQ[32 * v + 8 * k + n], sLut[(ws[k] >> (4 * n)) & 15u], accd);
+      }
+      logit = accd * __half2float(ks[row]);
+    }
+    float gmax = logit;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, off));
+    const float m_new = fmaxf(m_run, gmax);
+    const float alpha = (m_run == -INFINITY) ? 0.0f : fast_exp2(m_run - m_new);
+    const float p = (logit == -INFINITY) ? 0.0f : fast_exp2(logit - m_new);
+    float psum = p;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+    l_run = l_run * alpha + psum;
+    m_run = m_new;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[k] *= alpha;
+    const float pv = (t < seq_len) ? p * __half2float(vs[L.row(b, blk, min(t, seq_len - 1))]) : 0.0f;
+    for (int i = 0; i < 32; ++i) {
+      const float pi = __shfl_sync(0xffffffffu, pv, i);
+      const int ti = grp * 32 + i;
+      if (ti >= seq_len) break;
+      const uint16_t two = *reinterpret_cast<const uint16_t*>(vc + L.row(b, blk, ti) * 128 + half_off + 2 * lane);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] = fmaf(pi, sLut[(two >> (4 * k)) & 15u], o[k]);
+    }
+  }
+  if (lane == 0) {
+    cm[warp] = m_run;
+    cl[warp] = l_run;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) co[warp][4 * lane + k] = o[k];
+  __syncthreads();
+  if (tid < kD) {
+    float M = -INFINITY;
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, cm[w]);
+    float Ls = 0.0f, O = 0.0f;
+    for (int w = 0; w < kDecWarps; ++w) {
+      const float wt = (cm[w] == -INFINITY) ? 0.0f : fast_exp2(cm[w] - M);
+      Ls += cl[w] * wt;
+      O += co[w][tid] * wt;
+    }
+    if (splits == 1) {
+      out[static_cast<size_t>(bh) * kD + tid] = O / Ls;
+    } else {
+      const size_t pb = static_cast<size_t>(bh) * splits + split;
+      part_o[pb * kD + tid] = O;
+      if (tid == 0) {
+        part_m[pb] = M;
+        part_l[pb] = Ls;
+      }
+    }
+  }
+  if (splits == 1) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sLast = (atomicAdd(&tickets[bh], 1u) == static_cast<unsigned>(splits - 1));
+  __syncthreads();
+  if (!sLast) return;
+  __threadfence();
+  if (tid < kD) {
+    const size_t p0 = static_cast<size_t>(bh) * splits;
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(part_m + p0 + s));
+    float Ls = 0.0f, O = 0.0f;
+    for (int s = 0; s < splits; ++s) {
+      const float ms = __ldcg(part_m + p0 + s);
+      const float wt = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
+      Ls += __ldcg(part_l + p0 + s) * wt;
+      O += __ldcg(part_o + (p0 + s) * kD + tid) * wt;
+    }
+    out[static_cast<size_t>(bh) * kD + tid] = O / Ls;
+  }
+  if (tid == 0) tickets[bh] = 0u;
+}
+
+}  // namespace kvq

@@ -1,0 +1,70 @@
+"""Shared helpers for the GPU parity tests: run the oracle on the same inputs and compare."""
+import math
+
+import numpy as np
+
+from oracle import blockgtq as bg
+
+TOL = 2e-3   # max_j |o_j - o*_j| / max_j |o*_j| per (sequence, q-head)
+
+
+def host_f32(t):
+    """Exact fp32 host copy of a device tensor in any float dtype."""
+    return t.detach().float().cpu().numpy()
+
+
+def rel_err(out, ref):
+    """Max over (b, h) of max_j |o - ref| / max_j |ref|."""
+    out = np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    num = np.max(np.abs(out - ref), axis=-1)
+    den = np.max(np.abs(ref), axis=-1)
+    return float(np.max(num / den))
+
+
+def compare_alloc(gpu_heads, ref):
+    """Bit-exact comparison of the library allocation with the oracle's."""
+    H = ref["w"].shape[0]
+    assert len(gpu_heads) == H
+    for h in range(H):
+        g = gpu_heads[h]
+        np.testing.assert_array_equal(g["E"].view(np.uint64), ref["E"][h].astype(np.float64).view(np.uint64))
+        np.testing.assert_array_equal(g["w"], ref["w"][h])
+        np.testing.assert_array_equal(g["g"].view(np.uint32), ref["g"][h].view(np.uint32))
+        np.testing.assert_array_equal(g["f"].view(np.uint32), ref["f"][h].view(np.uint32))
+        np.testing.assert_array_equal(g["word_off"], bg.k_word_offsets(ref["w"][h]))
+        assert g["k_words"] == int(2 * ref["w"][h].sum())
+        check_steps(g, ref["w"][h])
+
+
+def check_steps(g, w):
+    """The decode k-step table lists every block with w > 0 once, widths descending, 4 per step."""
+    seen = []
+    prev_w = 99
+    for s in range(g["n_steps"]):
+        sw = g["step_width"][s]
+        assert 1 <= sw <= prev_w
+        prev_w = sw
+        blks = [b for b in g["step_block"][s] if b >= 0]
+        assert blks and all(w[b] == sw for b in blks)
+        seen += blks
+    assert sorted(seen) == [b for b in range(len(w)) if w[b] > 0]
+    assert len(seen) == len(set(seen))
+
+
+def oracle_pipeline(K, V, q, bits_k, bits_v, n_calib=0, w_max=8, mode=0, capacity=None):
+    """Oracle calibrate -> quantize -> pack -> decode on host fp32 copies."""
+    Kh, Vh = host_f32(K), host_f32(V)
+    alloc = bg.calibrate(Kh, bits_k, n_calib=n_calib, w_max=w_max, mode=mode)
+    T = Kh.shape[2]
+    cap = T if capacity is None else capacity
+    codes = bg.quantize(Kh, Vh, alloc, bits_v)
+    packed = bg.pack_cache(codes, alloc, bits_v, cap)
+    out = None
+    if q is not None:
+        out = bg.decode(host_f32(q), packed, alloc, bits_v, T)
+    return alloc, packed, out
+
+
+def tiles_written(T):
+    return -(-T // bg.TILE)
