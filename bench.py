@@ -1,0 +1,370 @@
+"""Benchmark of the packed-cache hot path (libkvq) on B200.
+
+One step = one pass of the whole path over a stack of L = 36 layers shaped like the
+Qwen2.5-3B 128K decode workload (16 q-heads, 2 KV heads, head_dim 128, batch 1,
+131072 tokens, bf16, K3V3): for every layer calibrate (energy reduction + greedy
+allocation) and quantize/pack its K and V (the prefill write of the cache), then one
+decode step of attention through all layers reading the packed caches. Qwen2.5-3B has
+36 layers; with 36 x 160 MB touched per step, every layer's inputs and cache have left
+L2 by the time they are read again.
+
+Prints one JSON line (rank 0). `--impl reference` times the CPU oracle instead, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "packed-KV decode attn: KV-tokens/s & % HBM peak; quantize/pack tokens/s"
+UNIT = "layer-tokens/s"
+LAYERS = 36
+WORKLOAD = "qwen3b"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="libkvq", choices=["libkvq", "reference"])
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=0, help="override the context length (profiling only)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "packed_cache_attention_b200", "csrc", name), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, src: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash(src)
+    with open(path) as fh:
+        for line in fh:
+            f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+            if f.get("kernel") == kernel and f.get("src_sha") == want and f.get("workload") == WORKLOAD:
+                return int(f["bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from packed_cache_attention_b200 import kvq
+    from packed_cache_attention_b200 import workloads as wl
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    W = wl.WORKLOADS[WORKLOAD]
+    T = args.seq_len or W.seq_len
+    B, Hq, Hkv, d = W.batch, W.n_q_heads, W.n_kv_heads, W.head_dim
+    bk, bv = W.bits_k, W.bits_v
+    L = args.layers
+    kvq.lib()
+    kvq._check("kvq_init", kvq.lib().kvq_init())
+
+    # Inputs for all layers, resident in HBM; one seed per (rank, layer).
+    Ks, Vs, qs = [], [], []
+    for layer in range(L):
+        x = wl.make_blockgtq_inputs(B, Hq, Hkv, d, T, W.dtype, W.rope_base, W.key_profile,
+                                    seed=1000 * rank + layer, device=dev)
+        Ks.append(x["K"]); Vs.append(x["V"]); qs.append(x["q"])
+    cache = kvq.cache_desc(B, Hkv, T, bk, bv)
+    allocs = [torch.empty(kvq.kvq_alloc_bytes(Hkv), dtype=torch.uint8, device=dev) for _ in range(L)]
+    packs = [torch.empty(kvq.kvq_packed_bytes(cache), dtype=torch.uint8, device=dev) for _ in range(L)]
+    outs = [torch.empty((B, Hq, d), dtype=torch.float32, device=dev) for _ in range(L)]
+    cws = torch.empty(kvq.kvq_calibrate_workspace_bytes(B, Hkv, T), dtype=torch.uint8, device=dev)
+    dws = [torch.zeros(kvq.kvq_decode_workspace_bytes(cache, Hq), dtype=torch.uint8, device=dev) for _ in range(L)]
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        for layer in range(L):
+            kvq.kvq_calibrate(Ks[layer], bk, n_calib=W.n_calib, alloc=allocs[layer], ws=cws, stream=stream)
+        if ev: ev[1].record(stream)
+        for layer in range(L):
+            kvq.kvq_quantize(Ks[layer], Vs[layer], allocs[layer], cache, packed=packs[layer], stream=stream)
+        if ev: ev[2].record(stream)
+        for layer in range(L):
+            kvq.kvq_decode_attn(qs[layer], packs[layer], allocs[layer], cache, T, out=outs[layer], ws=dws[layer],
+                                stream=stream)
+        if ev: ev[3].record(stream)
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    barrier()
+    for w in dws:
+        assert kvq.kvq_workspace_status(w) == 0
+
+    sampler = ClockSampler(local_rank)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    cal_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    qnt_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    if dist:
+        t = torch.tensor([total_ms, cal_ms, qnt_ms, dec_ms], dtype=torch.float64, device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms, cal_ms, qnt_ms, dec_ms = t.tolist()
+
+    # ---------------------------------------------------------------- end to end through the C ABI
+    e2e = None
+    if args.e2e_steps > 0:
+        hK = [k.cpu().pin_memory() for k in Ks]
+        hV = [v.cpu().pin_memory() for v in Vs]
+        hq = [q.cpu().pin_memory() for q in qs]
+        hout = [torch.empty((B, Hq, d), dtype=torch.float32).pin_memory() for _ in range(L)]
+        h2d = sum(x.numel() * x.element_size() for x in hK + hV + hq)
+        d2h = sum(x.numel() * x.element_size() for x in hout)
+
+        def e2e_step():
+            for layer in range(L):
+                Ks[layer].copy_(hK[layer], non_blocking=True)
+                Vs[layer].copy_(hV[layer], non_blocking=True)
+                qs[layer].copy_(hq[layer], non_blocking=True)
+            step()
+            for layer in range(L):
+                hout[layer].copy_(outs[layer], non_blocking=True)
+
+        e2e_step()
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        z.record(stream)
+        barrier()
+        e2e_ms = a.elapsed_time(z) / args.e2e_steps
+        if dist:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        e2e = {"value": world * L * B * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    steps = args.steps
+    ms_step = total_ms / steps
+    tokens = world * L * B * T
+    hbm, peak_kind = peaks()
+    q_bytes = B * Hkv * T * d * 2 * 2 + kvq.kvq_packed_bytes(cache)
+    d_bytes = kvq.kvq_packed_bytes(cache)
+    c_bytes = B * Hkv * T * d * 2
+    q_launch_ms = qnt_ms / (steps * L)
+    d_launch_ms = dec_ms / (steps * L)
+    c_launch_ms = cal_ms / (steps * L)
+    q_gbs = q_bytes / (q_launch_ms * 1e-3) / 1e9
+    d_gbs = d_bytes / (d_launch_ms * 1e-3) / 1e9
+    c_gbs = c_bytes / (c_launch_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": tokens / (ms_step * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 in; f64 norms/energies, f32 scaling, u32 bit planes; f16 mma + f32 accumulate",
+        "data": "synthetic (seeded Qwen2.5-3B-shaped K/V/q, lognormal block scales + 2 outlier blocks, RoPE 1e6)",
+        "config": {"workload": f"{WORKLOAD}: {L} layers x (Hq {Hq}, Hkv {Hkv}, d {d}, B {B}, T {T}, bf16), K{bk}V{bv}",
+                   "layers": L, "global_batch": B * world, "seq_len": T, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: each step touches 36 x 160 MB; no explicit flush"},
+        "roofline": {"bound": "hbm", "achieved": q_gbs, "peak": hbm, "unit": "GB/s", "frac": q_gbs / hbm,
+                     "traffic": recorded_traffic("kvq_quant_pack", "quantize.cuh"),
+                     "kernel": "kvq_quant_pack", "bytes_per_launch": q_bytes, "launch_ms": q_launch_ms,
+                     "peak_kind": peak_kind},
+        "breakdown": {
+            "decode": {"kv_tokens_per_s": tokens / (dec_ms / steps * 1e-3), "launch_ms": d_launch_ms,
+                       "bytes_per_launch": d_bytes, "gb_s": d_gbs, "hbm_frac": d_gbs / hbm,
+                       "traffic": recorded_traffic("kvq_decode_gtq", "decode.cuh")},
+            "quantize": {"tokens_per_s": tokens / (qnt_ms / steps * 1e-3), "launch_ms": q_launch_ms,
+                         "bytes_per_launch": q_bytes, "gb_s": q_gbs, "hbm_frac": q_gbs / hbm},
+            "calibrate": {"tokens_per_s": tokens / (cal_ms / steps * 1e-3), "launch_ms": c_launch_ms,
+                          "bytes_per_launch": c_bytes, "gb_s": c_gbs, "hbm_frac": c_gbs / hbm},
+            "bytes_per_token_per_kv_head": d_bytes // (B * Hkv * T),
+            "compression_vs_bf16": (2 * 2 * d) / (d_bytes / (B * Hkv * T)),
+        },
+        "e2e": e2e,
+        "gpu_launches": steps * L * 4,
+        "clocks": clocks,
+    }
+    return result
+
+
+# ------------------------------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(n_tokens: int, seed: int = 0):
+    """Time the oracle's calibrate + quantize/pack + decode on the first n_tokens of one layer
+    of the workload (both KV heads, all 16 q-heads). Returns (seconds, layer-tokens)."""
+    import numpy as np
+    import torch
+    from oracle import blockgtq as bg
+    from packed_cache_attention_b200 import workloads as wl
+    W = wl.WORKLOADS[WORKLOAD]
+    x = wl.make_blockgtq_inputs(W.batch, W.n_q_heads, W.n_kv_heads, W.head_dim, n_tokens, W.dtype, W.rope_base,
+                                W.key_profile, seed=seed, device="cpu")
+    K = x["K"].float().numpy()
+    V = x["V"].float().numpy()
+    q = x["q"].float().numpy()
+    t0 = time.perf_counter()
+    alloc = bg.calibrate(K, W.bits_k)
+    codes = bg.quantize(K, V, alloc, W.bits_v)
+    packed = bg.pack_cache(codes, alloc, W.bits_v, n_tokens)
+    bg.decode(q, packed, alloc, W.bits_v, n_tokens)
+    return time.perf_counter() - t0, W.batch * n_tokens
+
+
+def cpu_baseline(n_tokens: int = 131072):
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        secs, toks = oracle_sample(n_tokens)
+    return {"value": toks / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"one layer of {WORKLOAD}, first {n_tokens} tokens of both KV heads: calibrate + quantize/pack "
+                      f"+ decode for 16 q-heads ({secs:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from threadpoolctl import threadpool_limits
+    n_tokens = 2048
+    with threadpool_limits(limits=1):
+        for i in range(args.warmup):
+            oracle_sample(n_tokens, seed=i)
+        t0 = time.perf_counter()
+        toks = 0
+        for i in range(args.steps):
+            s, t = oracle_sample(n_tokens, seed=100 + i)
+            toks += t
+        total = time.perf_counter() - t0
+    value = toks / total
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (numpy oracle)", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"{WORKLOAD}: one layer, first {n_tokens} tokens per step (bounded sample)",
+                       "layers": 1, "global_batch": 1, "seq_len": n_tokens, "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{n_tokens} tokens of one layer per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline()       # before any CUDA work in this process
+    res = run_gpu(args, rank, world, local_rank)
+    if rank == 0:
+        res["cpu_baseline"] = base
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+        tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
