@@ -11,7 +11,8 @@ The page names these steps without defining them. The readings taken here
 (each restated in the function that uses it):
 
   energy     E_b = mean over calibration tokens of ||k_b||^2, block b = dims
-             (b, b + d/2); fp64, summed in a fixed order (64-token chunks).
+             (b, b + d/2); fp64, summed in a fixed order (64-token chunks,
+             64-chunk segments, then segments).
   greedy     d/2 * bits_k steps; each adds one bit to the block with the
              largest E_b * (delta(w_b) - delta(w_b + 1)) among blocks below
              w_max; ties go to the lowest block index.
@@ -36,6 +37,7 @@ from . import codebooks
 
 TILE = 32            # tokens per packed tile
 CALIB_CHUNK = 64     # tokens per fixed-order partial sum of the energy score
+CALIB_SEGMENT = 64   # chunk sums per fixed-order segment sum
 
 MODE_BLOCKGTQ = 0
 MODE_UNIFORM = 1
@@ -49,10 +51,11 @@ def calibration_energies(K: np.ndarray, n_calib: int = 0) -> tuple[np.ndarray, i
     K: [B][H][T][d] array whose values are exactly the stored keys (any float type).
     n_calib: number of leading tokens of every sequence to use (0 = all T).
     The calibration tokens of all sequences are pooled in the order
-    u = s * n_calib + t. Each term is fl(fl(x_b^2) + fl(x_{b+h}^2)) in fp64;
-    terms are summed left to right within consecutive chunks of 64 pooled
-    tokens (the last chunk may be shorter), chunk sums are added left to right,
-    and the total is divided by N = B * n_calib.
+    u = s * n_calib + t. Each term is fl(fl(x_b^2) + fl(x_{b+h}^2)) in fp64. The
+    sum has a fixed three-level order, every level left to right: terms within
+    chunks of 64 consecutive pooled tokens, chunk sums within segments of 64
+    consecutive chunks, then the segment sums; the last chunk and segment may be
+    shorter. The total is divided by N = B * n_calib.
     Returns (E [H][d/2] float64, N).
     """
     B, H, T, d = K.shape
@@ -64,12 +67,18 @@ def calibration_energies(K: np.ndarray, n_calib: int = 0) -> tuple[np.ndarray, i
     X = np.transpose(X, (1, 0, 2, 3)).reshape(H, B * n, d)            # pooled token order
     terms = X[:, :, :h] * X[:, :, :h] + X[:, :, h:] * X[:, :, h:]     # [H][N][h]
     N = B * n
-    total = np.zeros((H, h), dtype=np.float64)
+    chunk_sums = []
     for c0 in range(0, N, CALIB_CHUNK):
         acc = np.zeros((H, h), dtype=np.float64)
         for u in range(c0, min(N, c0 + CALIB_CHUNK)):
             acc = acc + terms[:, u, :]
-        total = total + acc
+        chunk_sums.append(acc)
+    total = np.zeros((H, h), dtype=np.float64)
+    for s0 in range(0, len(chunk_sums), CALIB_SEGMENT):
+        seg = np.zeros((H, h), dtype=np.float64)
+        for c in chunk_sums[s0:s0 + CALIB_SEGMENT]:
+            seg = seg + c
+        total = total + seg
     return total / float(N), N
 
 

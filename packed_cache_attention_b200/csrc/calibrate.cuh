@@ -8,70 +8,103 @@
 
 namespace kvq {
 
-// One warp per (64-token chunk, KV head). Lane l owns blocks 2l and 2l+1, i.e. dims
-// (2l, 2l+1) and (64+2l, 65+2l), read as one 2-element vector each (coalesced 128 B per
-// warp-load for 16-bit inputs). Within the chunk the pooled tokens u = s*n_calib + t are
-// summed left to right in fp64, each term being fl(fl(x^2) + fl(y^2)).
+constexpr int kCalibSegment = 64;      // chunk sums per fixed-order segment sum
+constexpr int kCalibChunksPerCta = 8;  // 16 lanes per chunk, 128 threads
+
+// Grid (ceil(n_chunks / 8), n_kv_heads), 128 threads: 16 lanes per 64-token chunk. Lane k
+// (0..15) of a chunk owns blocks 4k..4k+3, i.e. dims 4k..4k+3 and 64+4k..67+4k, read as two
+// 4-element vectors per token (128 contiguous bytes per half-warp for 16-bit inputs). Within
+// the chunk the pooled tokens u = s*n_calib + t are summed left to right in fp64, each term
+// being fl(fl(x^2) + fl(y^2)).
 template <int DT>
-__global__ void __launch_bounds__(32) kvq_calib_reduce(const typename Elem<DT>::T* __restrict__ K,
-                                                       int n_calib, int64_t sb, int64_t sh, int64_t st,
-                                                       int N, int n_chunks, double* __restrict__ partial) {
+__global__ void __launch_bounds__(16 * kCalibChunksPerCta) kvq_calib_reduce(
+    const typename Elem<DT>::T* __restrict__ K, int n_calib, int64_t sb, int64_t sh, int64_t st, int N,
+    int n_chunks, double* __restrict__ partial) {
   using T = typename Elem<DT>::T;
-  const int c = blockIdx.x, h = blockIdx.y, l = threadIdx.x;
-  const int u0 = c * kCalibChunk;
-  const int u1 = min(N, u0 + kCalibChunk);
-  double acc0 = 0.0, acc1 = 0.0;
-#pragma unroll 8
-  for (int u = u0; u < u1; ++u) {
-    const int s = u / n_calib;
-    const int t = u - s * n_calib;
+  const int h = blockIdx.y;
+  const int chunk = blockIdx.x * kCalibChunksPerCta + (threadIdx.x >> 4);
+  const int k = threadIdx.x & 15;
+  if (chunk >= n_chunks) return;
+  const int u0 = chunk * kCalibChunk;
+  const int n = min(N - u0, kCalibChunk);
+  int s = u0 / n_calib;
+  int t = u0 - s * n_calib;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 16
+  for (int i = 0; i < n; ++i) {
     const T* row = K + s * sb + h * sh + static_cast<int64_t>(t) * st;
-    float x0, x1, y0, y1;
+    float x[4], y[4];
     if constexpr (DT == KVQ_F32) {
-      const float2 a = *reinterpret_cast<const float2*>(row + 2 * l);
-      const float2 b = *reinterpret_cast<const float2*>(row + kH + 2 * l);
-      x0 = a.x; x1 = a.y; y0 = b.x; y1 = b.y;
+      const float4 a = __ldg(reinterpret_cast<const float4*>(row + 4 * k));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(row + kH + 4 * k));
+      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+      y[0] = b.x; y[1] = b.y; y[2] = b.z; y[3] = b.w;
     } else {
-      const T* pa = row + 2 * l;
-      const T* pb = row + kH + 2 * l;
-      x0 = Elem<DT>::to_f32(pa[0]); x1 = Elem<DT>::to_f32(pa[1]);
-      y0 = Elem<DT>::to_f32(pb[0]); y1 = Elem<DT>::to_f32(pb[1]);
+      const uint2 a = __ldg(reinterpret_cast<const uint2*>(row + 4 * k));
+      const uint2 b = __ldg(reinterpret_cast<const uint2*>(row + kH + 4 * k));
+      const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        x[2 * j] = Elem<DT>::to_f32(bits_to<T>(av[j] & 0xffffu));
+        x[2 * j + 1] = Elem<DT>::to_f32(bits_to<T>(av[j] >> 16));
+        y[2 * j] = Elem<DT>::to_f32(bits_to<T>(bv[j] & 0xffffu));
+        y[2 * j + 1] = Elem<DT>::to_f32(bits_to<T>(bv[j] >> 16));
+      }
     }
-    const double dx0 = x0, dx1 = x1, dy0 = y0, dy1 = y1;
-    acc0 = __dadd_rn(acc0, __dadd_rn(__dmul_rn(dx0, dx0), __dmul_rn(dy0, dy0)));
-    acc1 = __dadd_rn(acc1, __dadd_rn(__dmul_rn(dx1, dx1), __dmul_rn(dy1, dy1)));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const double dx = x[j], dy = y[j];
+      acc[j] = __dadd_rn(acc[j], __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)));
+    }
+    if (++t == n_calib) {
+      t = 0;
+      ++s;
+    }
   }
-  double* dst = partial + (static_cast<size_t>(h) * n_chunks + c) * kH;
-  dst[2 * l] = acc0;
-  dst[2 * l + 1] = acc1;
+  double* dst = partial + (static_cast<size_t>(h) * n_chunks + chunk) * kH + 4 * k;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) dst[j] = acc[j];
 }
 
 // One CTA of 512 threads per KV head.
-//  1. E_b = (sum of chunk partials, left to right) / N, fp64.
+//  1. E_b: chunk partials summed left to right within segments of 64 chunks (8 segments in
+//     flight per block), segment sums left to right, divided by N; fp64.
 //  2. Greedy allocation in rank form: entry e = 8b + w (w < w_max) has marginal gain
 //     E_b (delta(w) - delta(w+1)); the greedy takes the bits_k * 64 first entries in the
 //     order (gain descending, e ascending). Because delta is strictly convex each block's
 //     gains are non-increasing in w, so this is the step-by-step greedy with ties to the
-//     lowest block, and the picked entries of a block are a prefix: w_b = their count.
+//     lowest block, the entries of a block that precede a given entry form a prefix (found
+//     by binary search), and the picked entries of a block are a prefix: w_b = their count.
 //  3. g_b, f_b, the K word offsets and the decode k-step table (blocks grouped by width,
 //     widest first, 4 per step, ascending block index within a width).
-__global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict__ partial, int n_chunks,
+__global__ void __launch_bounds__(512) kvq_greedy_alloc(double* __restrict__ partial, int n_chunks,
                                                         int N, int bits_k, int w_max, int mode,
                                                         kvq_head_alloc* __restrict__ alloc) {
   __shared__ double sE[kH];
   __shared__ double sGain[kH * 8];
   __shared__ int sWidth[kH];
-  __shared__ float sG[kH];
   __shared__ int sStepStart[9];
   __shared__ int sCount[9];
   __shared__ double sSum;
   const int h = blockIdx.x, tid = threadIdx.x;
   kvq_head_alloc* al = alloc + h;
+  double* ph = partial + static_cast<size_t>(h) * n_chunks * kH;
+  const int n_seg = (n_chunks + kCalibSegment - 1) / kCalibSegment;
 
+  {
+    const int b = tid & (kH - 1), r = tid >> 6;
+    for (int sg = r; sg < n_seg; sg += 8) {
+      const int c0 = sg * kCalibSegment, c1 = min(n_chunks, c0 + kCalibSegment);
+      double acc = 0.0;
+#pragma unroll 8
+      for (int c = c0; c < c1; ++c) acc = __dadd_rn(acc, ph[static_cast<size_t>(c) * kH + b]);
+      ph[static_cast<size_t>(c0) * kH + b] = acc;     // the segment's first slot holds its sum
+    }
+  }
+  __syncthreads();
   if (tid < kH) {
     double S = 0.0;
-    const double* p = partial + static_cast<size_t>(h) * n_chunks * kH + tid;
-    for (int c = 0; c < n_chunks; ++c) S = __dadd_rn(S, p[static_cast<size_t>(c) * kH]);
+    for (int sg = 0; sg < n_seg; ++sg) S = __dadd_rn(S, __ldcg(ph + static_cast<size_t>(sg) * kCalibSegment * kH + tid));
     sE[tid] = __ddiv_rn(S, static_cast<double>(N));
   }
   __syncthreads();
@@ -94,9 +127,19 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     const double gain = sGain[tid];
     const bool valid = (tid & 7) < w_max;
     int rank = 0;
-    for (int e = 0; e < kH * 8; ++e) {
-      const double ge = sGain[e];
-      rank += (ge > gain) || (ge == gain && e < tid);
+    if (valid) {
+      for (int bb = 0; bb < kH; ++bb) {
+        // entries of block bb preceding entry tid form a prefix of w = 0..w_max-1
+        int lo = 0, hi = w_max;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          const int e = 8 * bb + mid;
+          const double ge = sGain[e];
+          if (ge > gain || (ge == gain && e < tid)) lo = mid + 1;
+          else hi = mid;
+        }
+        rank += lo;
+      }
     }
     const bool picked = valid && rank < bits_k * kH;
     const unsigned mask = __ballot_sync(0xffffffffu, picked);
@@ -110,7 +153,6 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     float g = 1.0f;
     if (mode != KVQ_MODE_UNIFORM && sE[b] > 0.0 && sSum > 0.0)
       g = __double2float_rn(__dsqrt_rn(__ddiv_rn(__dmul_rn(2.0, sSum), __dmul_rn(static_cast<double>(kD), sE[b]))));
-    sG[b] = g;
     al->energy[b] = sE[b];
     al->gain[b] = g;
     al->dequant[b] = __double2float_rn(__ddiv_rn(1.0, __dmul_rn(__dsqrt_rn(static_cast<double>(kD)),

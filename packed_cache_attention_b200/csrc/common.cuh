@@ -51,6 +51,15 @@ template <> struct Elem<KVQ_BF16> {
   __device__ __forceinline__ static float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 };
 
+template <typename T>
+__device__ __forceinline__ T bits_to(uint32_t b);
+template <>
+__device__ __forceinline__ __half bits_to<__half>(uint32_t b) { return __ushort_as_half(static_cast<unsigned short>(b)); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 bits_to<__nv_bfloat16>(uint32_t b) {
+  return __ushort_as_bfloat16(static_cast<unsigned short>(b));
+}
+
 // ---------------------------------------------------------------- bit helpers
 
 __device__ __forceinline__ uint32_t rotr(uint32_t x, uint32_t n) { return __funnelshift_r(x, x, n); }

@@ -24,7 +24,7 @@
 
 namespace kvq {
 
-constexpr int kDecWarps = 4;
+constexpr int kDecWarps = 8;
 constexpr int kDecStages = 3;
 constexpr int kMaxSteps = 32;
 constexpr int kTargetCtas = 296;   // 2 CTAs per SM on a 148-SM B200
@@ -34,12 +34,88 @@ struct DecodeSmem {
   float qp[8][kD];                  // Q' in fp32 before scaling
   float qmul[8];                    // 2^e that undoes the per-head scaling of Q'
   uint16_t cent[kCentroidCount];    // fp16 centroid bit patterns
+  uint4 lut8[4];                    // widths 1..3: {lo bytes 0-3, lo 4-7, hi 0-3, hi 4-7}
+  uint4 lut16[2];                   // width 4: {loA0, loA1, loB0, loB1}, {hiA0, hiA1, hiB0, hiB1}
   uint16_t woff[kH];
   int8_t step_blk[kMaxSteps][4];
   uint8_t step_w[kMaxSteps];
   int n_steps;
   int last;
 };
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Gather bit p of 8 codes from `w` plane words (word p at words[p * stride]; code m at bit
+// shift + 4m) into 4-bit nibbles: nibble m of the result is code m.
+__device__ __forceinline__ uint32_t gather_nibbles(const uint32_t* words, int stride, int w, int shift) {
+  uint32_t x = 0;
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+    if (p < w) x |= rotr(words[p * stride], static_cast<uint32_t>(shift - p) & 31u) & (0x11111111u << p);
+  return x;
+}
+
+// Register lookup of 8 codes (nibbles of x, each < 8) in an 8-entry fp16 table split into
+// low and high bytes; r[k] = fp16x2(entry[code 2k], entry[code 2k+1]).
+__device__ __forceinline__ void lut8(uint32_t x, const uint4& L, uint32_t (&r)[4]) {
+  const uint32_t la = prmt(L.x, L.y, x), ha = prmt(L.z, L.w, x);
+  const uint32_t xh = x >> 16;
+  const uint32_t lb = prmt(L.x, L.y, xh), hb = prmt(L.z, L.w, xh);
+  r[0] = prmt(la, ha, 0x5140u);
+  r[1] = prmt(la, ha, 0x7362u);
+  r[2] = prmt(lb, hb, 0x5140u);
+  r[3] = prmt(lb, hb, 0x7362u);
+}
+
+// 16-entry version: the low 3 bits of a nibble index two 8-entry halves, bit 3 picks the
+// half through a byte mask made with prmt's sign-replicate mode.
+__device__ __forceinline__ void lut16(uint32_t x, const uint4& LO, const uint4& HI, uint32_t (&r)[4]) {
+  const uint32_t x7 = x & 0x77777777u;
+  const uint32_t xh = x >> 16, x7h = x7 >> 16;
+  const uint32_t ma = prmt(x << 4, x, 0xD9C8u), mb = prmt(xh << 4, xh, 0xD9C8u);
+  const uint32_t la = (prmt(LO.x, LO.y, x7) & ~ma) | (prmt(LO.z, LO.w, x7) & ma);
+  const uint32_t ha = (prmt(HI.x, HI.y, x7) & ~ma) | (prmt(HI.z, HI.w, x7) & ma);
+  const uint32_t lb = (prmt(LO.x, LO.y, x7h) & ~mb) | (prmt(LO.z, LO.w, x7h) & mb);
+  const uint32_t hb = (prmt(HI.x, HI.y, x7h) & ~mb) | (prmt(HI.z, HI.w, x7h) & mb);
+  r[0] = prmt(la, ha, 0x5140u);
+  r[1] = prmt(la, ha, 0x7362u);
+  r[2] = prmt(lb, hb, 0x5140u);
+  r[3] = prmt(lb, hb, 0x7362u);
+}
+
+// Any width: assemble each code from its planes and look it up in the shared table.
+__device__ __forceinline__ void lut_generic(const uint32_t* words, int stride, int w, int shift,
+                                            const uint16_t* table, uint32_t (&r)[4]) {
+  uint32_t W[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) W[p] = (p < w) ? words[p * stride] : 0u;
+  uint32_t val[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    uint32_t code = 0;
+#pragma unroll
+    for (int p = 0; p < 8; ++p) code |= ((W[p] >> (shift + 4 * m)) & 1u) << p;
+    val[m] = table[code];
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) r[k] = pack_u16x2(val[2 * k], val[2 * k + 1]);
+}
+
+// The 8 codes at bits shift + 4m of `w` plane words, as 4 fp16x2 fragments.
+__device__ __forceinline__ void decode8(const uint32_t* words, int stride, int w, int shift, const DecodeSmem& S,
+                                        uint32_t (&r)[4]) {
+  if (w <= 3) {
+    lut8(gather_nibbles(words, stride, w, shift), S.lut8[w], r);
+  } else if (w == 4) {
+    lut16(gather_nibbles(words, stride, 4, shift), S.lut16[0], S.lut16[1], r);
+  } else {
+    lut_generic(words, stride, w, shift, S.cent + ((1 << w) - 2), r);
+  }
+}
 
 __device__ __forceinline__ void decode_load_tile(uint8_t* dst, const uint8_t* src, int rec_bytes, int lane) {
   for (int k = lane; k < rec_bytes / 16; k += 32) cp_async16(dst + 16 * k, src + 16 * k);
@@ -70,8 +146,42 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
   const int t_end = static_cast<int>((static_cast<long long>(split + 1) * n_tiles) / splits);
   const float inv_sqrt_d = 0.08838834764831845f;
 
+  const int stage_bytes = ((rec_bytes + 127) / 128) * 128;
+  uint8_t* my_stages = stages + warp * kDecStages * stage_bytes;
+  const uint8_t* src_base = packed + static_cast<size_t>(bh) * tiles_cap * rec_bytes;
+  const int first = t_begin + warp;
+  const int my_n = (first < t_end) ? (t_end - first + kDecWarps - 1) / kDecWarps : 0;
+  // Start streaming the first tiles before the prologue.
+#pragma unroll
+  for (int i = 0; i < kDecStages - 1; ++i) {
+    if (i < my_n)
+      decode_load_tile(my_stages + i * stage_bytes, src_base + static_cast<size_t>(first + i * kDecWarps) * rec_bytes,
+                       rec_bytes, lane);
+    cp_async_commit();
+  }
+
   // ------------------------------------------------------------------ prologue
   for (int i = tid; i < kCentroidCount; i += blockDim.x) S.cent[i] = c_tab.centroid_f16[i];
+  if (tid < 4) {
+    uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
+    if (tid >= 1) {
+      for (int e = 0; e < (1 << tid); ++e) {
+        const uint32_t c16 = c_tab.centroid_f16[(1 << tid) - 2 + e];
+        lo[e >> 2] |= (c16 & 0xffu) << (8 * (e & 3));
+        hi[e >> 2] |= (c16 >> 8) << (8 * (e & 3));
+      }
+    }
+    S.lut8[tid] = make_uint4(lo[0], lo[1], hi[0], hi[1]);
+  } else if (tid == 4) {
+    uint32_t lo[4] = {0u, 0u, 0u, 0u}, hi[4] = {0u, 0u, 0u, 0u};
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t c16 = c_tab.centroid_f16[14 + e];
+      lo[e >> 2] |= (c16 & 0xffu) << (8 * (e & 3));
+      hi[e >> 2] |= (c16 >> 8) << (8 * (e & 3));
+    }
+    S.lut16[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    S.lut16[1] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  }
   for (int i = tid; i < kH; i += blockDim.x) S.woff[i] = al->word_off[i];
   for (int i = tid; i < kMaxSteps * 4; i += blockDim.x) S.step_blk[i >> 2][i & 3] = al->step_block[i >> 2][i & 3];
   for (int i = tid; i < kMaxSteps; i += blockDim.x) S.step_w[i] = al->step_width[i];
@@ -122,20 +232,6 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt) o_acc[nt][0] = o_acc[nt][1] = o_acc[nt][2] = o_acc[nt][3] = 0.0f;
 
-  const int stage_bytes = ((rec_bytes + 127) / 128) * 128;
-  uint8_t* my_stages = stages + warp * kDecStages * stage_bytes;
-  const uint8_t* src_base = packed + static_cast<size_t>(bh) * tiles_cap * rec_bytes;
-  const int first = t_begin + warp;
-  const int my_n = (first < t_end) ? (t_end - first + kDecWarps - 1) / kDecWarps : 0;
-
-#pragma unroll
-  for (int i = 0; i < kDecStages - 1; ++i) {
-    if (i < my_n)
-      decode_load_tile(my_stages + i * stage_bytes, src_base + static_cast<size_t>(first + i * kDecWarps) * rec_bytes,
-                       rec_bytes, lane);
-    cp_async_commit();
-  }
-
   const int H = g >> 2, sh = g & 3;
   for (int i = 0; i < my_n; ++i) {
     {
@@ -162,22 +258,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
       const int w = min(max(static_cast<int>(S.step_w[s]), 1), 8);
       int blk = S.step_blk[s][c];
       if (blk < 0) blk = max(static_cast<int>(S.step_blk[s][0]), 0);   // empty slot: Q' is 0 there
-      const uint32_t* bw = kw + S.woff[blk] + H;
-      uint32_t W[8];
-#pragma unroll
-      for (int p = 0; p < 8; ++p) W[p] = (p < w) ? bw[2 * p] : 0u;
-      const uint16_t* cb = S.cent + ((1 << w) - 2);
-      uint32_t val[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        int code = 0;
-#pragma unroll
-        for (int p = 0; p < 8; ++p) code |= ((W[p] >> (sh + 4 * m)) & 1u) << p;
-        val[m] = cb[code];
-      }
+      uint32_t bf[4];
+      decode8(kw + S.woff[blk] + H, 2, w, sh, S, bf);
       const uint2 a = S.qfrag[s][g][c];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) mma_m16n8k8(acc[j], a.x, a.y, pack_u16x2(val[2 * j], val[2 * j + 1]));
+      for (int j = 0; j < 4; ++j) mma_m16n8k8(acc[j], a.x, a.y, bf[j]);
     }
 
     // ---- online softmax over the 8 tokens this lane holds: 8j + 2c + {0,1}
@@ -201,9 +286,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
     const float alpha = (m_run == -INFINITY) ? 0.0f : fast_exp2(m_run - m_new);
     m_run = m_new;
     l_run *= alpha;
+    if (!__all_sync(0xffffffffu, alpha == 1.0f)) {
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      o_acc[nt][0] *= alpha; o_acc[nt][1] *= alpha; o_acc[nt][2] *= alpha; o_acc[nt][3] *= alpha;
+      for (int nt = 0; nt < 16; ++nt) {
+        o_acc[nt][0] *= alpha; o_acc[nt][1] *= alpha; o_acc[nt][2] *= alpha; o_acc[nt][3] *= alpha;
+      }
     }
     uint32_t pa_hi[4], pa_lo[4];   // per n-tile j: packed (token 8j+2c, 8j+2c+1)
 #pragma unroll
@@ -222,25 +309,33 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
     }
 
     // ---- O += P' Vhat over 16 dim n-tiles, two 16-token k-steps
-    const uint16_t* vcb = S.cent + ((1 << bits_v) - 2);
+    if (bits_v <= 3) {
+      const uint4 L = S.lut8[bits_v];
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int jd = 8 * nt + g;
-      uint32_t W[8];
-#pragma unroll
-      for (int p = 0; p < 8; ++p) W[p] = (p < bits_v) ? vw[p * kD + jd] : 0u;
-      uint32_t val[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        int code = 0;
-#pragma unroll
-        for (int p = 0; p < 8; ++p) code |= ((W[p] >> (c + 4 * m)) & 1u) << p;
-        val[m] = vcb[code];
+      for (int nt = 0; nt < 16; ++nt) {
+        uint32_t vf[4];
+        lut8(gather_nibbles(vw + 8 * nt + g, kD, bits_v, c), L, vf);
+        mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], vf[0], vf[1]);
+        mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], vf[2], vf[3]);
       }
-      mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], pack_u16x2(val[0], val[1]),
-                   pack_u16x2(val[2], val[3]));
-      mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], pack_u16x2(val[4], val[5]),
-                   pack_u16x2(val[6], val[7]));
+    } else if (bits_v == 4) {
+      const uint4 LO = S.lut16[0], HI = S.lut16[1];
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        uint32_t vf[4];
+        lut16(gather_nibbles(vw + 8 * nt + g, kD, 4, c), LO, HI, vf);
+        mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], vf[0], vf[1]);
+        mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], vf[2], vf[3]);
+      }
+    } else {
+      const uint16_t* table = S.cent + ((1 << bits_v) - 2);
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        uint32_t vf[4];
+        lut_generic(vw + 8 * nt + g, kD, bits_v, c, table, vf);
+        mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], vf[0], vf[1]);
+        mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], vf[2], vf[3]);
+      }
     }
     __syncwarp();
   }

@@ -92,6 +92,18 @@ DecodeWs decode_ws_layout(int bh, int splits, int rows) {
   return w;
 }
 
+int sm_count() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
 kvq_status launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
@@ -207,18 +219,19 @@ kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_p
   const int n_chunks = static_cast<int>((N + kCalibChunk - 1) / kCalibChunk);
   double* partial = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + sizeof(WsHeader));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dim3 grid(n_chunks, kd->n_heads);
+  dim3 grid((n_chunks + kCalibChunksPerCta - 1) / kCalibChunksPerCta, kd->n_heads);
+  const int threads = 16 * kCalibChunksPerCta;
   switch (kd->dtype) {
     case KVQ_F32:
-      kvq_calib_reduce<KVQ_F32><<<grid, 32, 0, s>>>(static_cast<const float*>(K), n_calib, kd->stride_b, kd->stride_h,
+      kvq_calib_reduce<KVQ_F32><<<grid, threads, 0, s>>>(static_cast<const float*>(K), n_calib, kd->stride_b, kd->stride_h,
                                                     kd->stride_t, static_cast<int>(N), n_chunks, partial);
       break;
     case KVQ_F16:
-      kvq_calib_reduce<KVQ_F16><<<grid, 32, 0, s>>>(static_cast<const __half*>(K), n_calib, kd->stride_b, kd->stride_h,
+      kvq_calib_reduce<KVQ_F16><<<grid, threads, 0, s>>>(static_cast<const __half*>(K), n_calib, kd->stride_b, kd->stride_h,
                                                     kd->stride_t, static_cast<int>(N), n_chunks, partial);
       break;
     default:
-      kvq_calib_reduce<KVQ_BF16><<<grid, 32, 0, s>>>(static_cast<const __nv_bfloat16*>(K), n_calib, kd->stride_b,
+      kvq_calib_reduce<KVQ_BF16><<<grid, threads, 0, s>>>(static_cast<const __nv_bfloat16*>(K), n_calib, kd->stride_b,
                                                      kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, partial);
   }
   if ((st = launch_status()) != KVQ_OK) return st;
@@ -243,8 +256,10 @@ kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, con
   const int tiles_cap = n_tiles_of(c->capacity);
   const long long n_tasks = static_cast<long long>(c->batch) * c->n_kv_heads * tiles_written;
   const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
-  const size_t smem = 512 * 4 + static_cast<size_t>(kQuantWarps) * (c->bits_k + c->bits_v) * kD * 4;
-  const unsigned grid = static_cast<unsigned>((n_tasks + kQuantWarps - 1) / kQuantWarps);
+  const size_t smem = quant_smem_bytes(kd->dtype, c->bits_k, c->bits_v);
+  const int ctas_per_sm = static_cast<int>(std::max<size_t>(1, (227u * 1024u) / smem));
+  const long long want = (n_tasks + kQuantWarps - 1) / kQuantWarps;
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sm_count()) * ctas_per_sm));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 #define KVQ_LAUNCH_QUANT(DT, TY)                                                                                  \
   do {                                                                                                            \

@@ -2,15 +2,20 @@
 // width for V ("RoPE-aware bit allocation for KV cache quantization", abstract: Block-GTQ
 // is "built on TurboQuant-MSE", "matched K/V bit budgets", "packed K3V3").
 //
-// One warp per 32-token tile of one (sequence, KV head); lane t quantizes token t of the
-// tile. For a token row x (128 values):
+// One warp per 32-token tile of one (sequence, KV head) at a time (persistent warps);
+// lane t quantizes token t of the tile. For a token row x (128 values):
 //   s2   = sum_j x_j^2 in fp64, j ascending (exact products, rounded sums)
 //   norm = fp16(sqrt(s2)) (round to nearest even)
 //   a    = fp32(sqrt(128)) / fp32(norm), 0 if norm == 0
 //   y_j  = fp32(fp32(x_j a) g_b)            (V: g = 1, the multiply is skipped as exact)
-//   code = #{thresholds of width w_b strictly below y_j}  (branch-free binary search)
-// Bit planes are gathered with warp ballots (bit t = token t) and staged in shared memory;
-// a last pass permutes them into the tile layout and writes whole 128-byte lines:
+//   code = #{thresholds of width w_b strictly below y_j}
+// The code is found by binary search over the 2^w - 1 sorted thresholds, most significant
+// bit first; the comparison at level p is bit p of the code, so its warp ballot (bit t =
+// token t) is directly the tile's bit-plane word for that dim and plane.
+// The tile is first copied into shared memory with a padded row pitch (65 words for 16-bit
+// inputs), so that the 32 lanes reading the same dim of their own rows hit 32 banks.
+// Ballot words are staged in shared memory; a last pass permutes them into the tile layout
+// and writes whole lines:
 //   K, per block b (ascending, w_b > 0), per plane p: two words built from the ballots
 //      A (dim b) and B (dim b+64): word0 = lo nibbles of A's bytes | lo nibbles of B's bytes
 //      << 4, word1 = hi nibbles of A | hi nibbles of B. Bit s+4m of word H then holds token
@@ -26,68 +31,66 @@ namespace kvq {
 
 constexpr int kQuantWarps = 8;
 
-// Row of 128 stored values of one token, held in registers.
-template <int DT> struct RowRegs;
-template <> struct RowRegs<KVQ_F32> {
-  float r[kD];
-  __device__ __forceinline__ void load(const float* p) {
-#pragma unroll
-    for (int i = 0; i < kD / 4; ++i) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(p) + i);
-      r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
+template <int DT> struct QuantRow;
+// 16-bit inputs: a row is 64 words (2 values each), pitch 65 words.
+template <int DT> struct QuantRow16 {
+  static constexpr int kPitch = kD / 2 + 1;
+  static constexpr int kWords = kTile * kPitch;
+  // Copy 32 rows (32 * 256 B, rows `row_stride` elements apart) into shared memory.
+  __device__ __forceinline__ static void load(uint32_t* dst, const void* src, int64_t row_stride, int valid_rows,
+                                              int lane) {
+    const uint8_t* s8 = static_cast<const uint8_t*>(src);
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const int idx = i * 32 + lane;           // 16-byte chunk of the tile
+      const int r = idx >> 4, c = idx & 15;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < valid_rows) v = __ldg(reinterpret_cast<const uint4*>(s8 + (static_cast<int64_t>(r) * row_stride * 2)) + c);
+      uint32_t* d = dst + r * kPitch + 4 * c;
+      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
     }
   }
-  __device__ __forceinline__ void zero() {
-#pragma unroll
-    for (int i = 0; i < kD; ++i) r[i] = 0.0f;
-  }
-  __device__ __forceinline__ float get(int j) const { return r[j]; }
-};
-template <int DT> struct RowRegs16 {
-  uint32_t r[kD / 2];
-  __device__ __forceinline__ void load(const void* p) {
-#pragma unroll
-    for (int i = 0; i < kD / 8; ++i) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + i);
-      r[4 * i] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
-    }
-  }
-  __device__ __forceinline__ void zero() {
-#pragma unroll
-    for (int i = 0; i < kD / 2; ++i) r[i] = 0u;
-  }
-  __device__ __forceinline__ float get(int j) const {
-    const uint32_t bits = (j & 1) ? (r[j >> 1] >> 16) : (r[j >> 1] & 0xffffu);
-    if constexpr (DT == KVQ_BF16) return __uint_as_float(bits << 16);
-    else return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
+  // Values 2i and 2i+1 of a row.
+  __device__ __forceinline__ static float2 pair(const uint32_t* row, int i) {
+    const uint32_t w = row[i];
+    if constexpr (DT == KVQ_BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    else return __half22float2(*reinterpret_cast<const __half2*>(&w));
   }
 };
-template <> struct RowRegs<KVQ_F16> : RowRegs16<KVQ_F16> {};
-template <> struct RowRegs<KVQ_BF16> : RowRegs16<KVQ_BF16> {};
-
-// code = #{t in thresholds(w) : t < y} by branch-free binary search over the 2^w - 1
-// sorted thresholds (shared-memory copy of the constant table).
-__device__ __forceinline__ int lm_code(float y, int w, const float* __restrict__ sThr) {
-  const float* t = sThr + ((1 << w) - w - 1);
-  int idx = 0;
-#pragma unroll
-  for (int k = 7; k >= 0; --k) {
-    if (k < w) {
-      const int s = 1 << k;
-      idx += (y > t[idx + s - 1]) ? s : 0;
+template <> struct QuantRow<KVQ_BF16> : QuantRow16<KVQ_BF16> {};
+template <> struct QuantRow<KVQ_F16> : QuantRow16<KVQ_F16> {};
+// fp32 inputs: a row is 128 words, pitch 129 words.
+template <> struct QuantRow<KVQ_F32> {
+  static constexpr int kPitch = kD + 1;
+  static constexpr int kWords = kTile * kPitch;
+  __device__ __forceinline__ static void load(uint32_t* dst, const void* src, int64_t row_stride, int valid_rows,
+                                              int lane) {
+    const uint8_t* s8 = static_cast<const uint8_t*>(src);
+#pragma unroll 4
+    for (int i = 0; i < 32; ++i) {
+      const int idx = i * 32 + lane;
+      const int r = idx >> 5, c = idx & 31;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < valid_rows) v = __ldg(reinterpret_cast<const uint4*>(s8 + (static_cast<int64_t>(r) * row_stride * 4)) + c);
+      uint32_t* d = dst + r * kPitch + 4 * c;
+      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
     }
   }
-  return idx;
-}
+  __device__ __forceinline__ static float2 pair(const uint32_t* row, int i) {
+    return make_float2(__uint_as_float(row[2 * i]), __uint_as_float(row[2 * i + 1]));
+  }
+};
 
-// fp16 norm and scale of a row, as in the header comment.
+// fp16 norm of one row and the scale a = sqrt(128)/norm (0 for a zero norm).
 template <int DT>
-__device__ __forceinline__ void row_norm_scale(const RowRegs<DT>& row, __half& n16, float& a) {
+__device__ __forceinline__ void row_norm_scale(const uint32_t* row, __half& n16, float& a) {
   double s2 = 0.0;
-#pragma unroll
-  for (int j = 0; j < kD; ++j) {
-    const double x = static_cast<double>(row.get(j));
-    s2 = __fma_rn(x, x, s2);        // x*x is exact in fp64, so this is fl(s2 + x^2)
+#pragma unroll 8
+  for (int i = 0; i < kD / 2; ++i) {
+    const float2 v = QuantRow<DT>::pair(row, i);
+    const double x0 = v.x, x1 = v.y;
+    s2 = __fma_rn(x0, x0, s2);      // x*x is exact in fp64, so this is fl(s2 + x^2)
+    s2 = __fma_rn(x1, x1, s2);
   }
   n16 = __double2half(__dsqrt_rn(s2));
   const float nf = __half2float(n16);
@@ -103,90 +106,133 @@ __device__ __forceinline__ uint32_t unzip_bytes(uint32_t x) {
   return x;
 }
 
+// Binary search for two values of the same width; the ballot of the comparison at level p
+// (bit p of the code) is written to out[p * pstride] (first value) and out[p * pstride + 1]
+// (second value, when `two`), by lane 0.
+__device__ __forceinline__ void search_ballot2(float y1, float y2, int w, const float* __restrict__ thr, bool valid,
+                                               uint32_t* out, int pstride, int second_off, int lane) {
+  int i1 = 0, i2 = 0;
+  for (int p = w - 1; p >= 0; --p) {
+    const int s = 1 << p;
+    const bool b1 = y1 > thr[i1 + s - 1];
+    const bool b2 = y2 > thr[i2 + s - 1];
+    const unsigned A = __ballot_sync(0xffffffffu, valid && b1);
+    const unsigned B = __ballot_sync(0xffffffffu, valid && b2);
+    if (lane == 0) {
+      out[p * pstride] = A;
+      out[p * pstride + second_off] = B;
+    }
+    i1 += b1 ? s : 0;
+    i2 += b2 ? s : 0;
+  }
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
     const typename Elem<DT>::T* __restrict__ K, int64_t ksb, int64_t ksh, int64_t kst,
     const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst,
     int seq_len, int n_kv_heads, int tiles_written, int tiles_cap, const kvq_head_alloc* __restrict__ alloc,
     int bits_k, int bits_v, uint8_t* __restrict__ packed, int rec_bytes, long long n_tasks) {
+  using Row = QuantRow<DT>;
   extern __shared__ __align__(16) uint32_t smem[];
   float* sThr = reinterpret_cast<float*>(smem);
   for (int i = threadIdx.x; i < kThresholdCount; i += blockDim.x) sThr[i] = c_tab.threshold[i];
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long task = static_cast<long long>(blockIdx.x) * kQuantWarps + warp;
-  if (task >= n_tasks) return;
   const int k_words = bits_k * kD, v_words = bits_v * kD;
-  uint32_t* stage = smem + 512 + warp * (k_words + v_words);
+  const int warp_words = Row::kWords + k_words + v_words + 3 * kH;
+  uint32_t* rows = smem + 512 + warp * warp_words;
+  uint32_t* stage = rows + Row::kWords;
   uint32_t* vstage = stage + k_words;
+  int* tw = reinterpret_cast<int*>(vstage + v_words);   // per block: width
+  float* tg = reinterpret_cast<float*>(tw + kH);        // per block: gain
+  int* to = tw + 2 * kH;                                 // per block: K word offset
+  const float* vthr = sThr + ((1 << bits_v) - bits_v - 1);
+  const uint32_t* myrow = rows + lane * Row::kPitch;
+  int cur_h = -1;
 
-  const int tile = static_cast<int>(task % tiles_written);
-  const int bh = static_cast<int>(task / tiles_written);
-  const int h = bh % n_kv_heads, b = bh / n_kv_heads;
-  const kvq_head_alloc* al = alloc + h;
-  if (al->k_words != k_words) return;        // allocation made for another budget: write nothing
-  const int token = tile * kTile + lane;
-  const bool valid = token < seq_len;
+  for (long long task = static_cast<long long>(blockIdx.x) * kQuantWarps + warp; task < n_tasks;
+       task += static_cast<long long>(gridDim.x) * kQuantWarps) {
+    const int tile = static_cast<int>(task % tiles_written);
+    const int bh = static_cast<int>(task / tiles_written);
+    const int h = bh % n_kv_heads, b = bh / n_kv_heads;
+    const kvq_head_alloc* al = alloc + h;
+    if (al->k_words != k_words) continue;      // allocation made for another budget: write nothing
+    if (h != cur_h) {
+      __syncwarp();
+      for (int i = lane; i < kH; i += 32) {
+        tw[i] = al->width[i];
+        tg[i] = al->gain[i];
+        to[i] = al->word_off[i];
+      }
+      cur_h = h;
+    }
+    const int t0 = tile * kTile;
+    const int valid_rows = min(kTile, seq_len - t0);
+    const bool valid = lane < valid_rows;
 
-  RowRegs<DT> row;
-  __half kn16, vn16;
-  float a;
-
-  // ---------------------------------------------------------------- K (Block-GTQ widths)
-  if (valid) row.load(K + b * ksb + h * ksh + static_cast<int64_t>(token) * kst);
-  else row.zero();
-  row_norm_scale<DT>(row, kn16, a);
+    // ---------------------------------------------------------------- K (Block-GTQ widths)
+    __syncwarp();
+    Row::load(rows, K + b * ksb + h * ksh + static_cast<int64_t>(t0) * kst, kst, valid_rows, lane);
+    __syncwarp();
+    __half kn16, vn16;
+    float a;
+    row_norm_scale<DT>(myrow, kn16, a);
+#pragma unroll 1
+    for (int bp = 0; bp < kH / 2; ++bp) {
+      const float2 lo = Row::pair(myrow, bp);             // dims 2bp, 2bp+1
+      const float2 hi = Row::pair(myrow, kH / 2 + bp);    // dims 64+2bp, 65+2bp
 #pragma unroll
-  for (int blk = 0; blk < kH; ++blk) {
-    const int w = al->width[blk];
-    if (w == 0) continue;
-    const float g = al->gain[blk];
-    const float y1 = __fmul_rn(__fmul_rn(row.get(blk), a), g);
-    const float y2 = __fmul_rn(__fmul_rn(row.get(blk + kH), a), g);
-    const int c1 = lm_code(y1, w, sThr);
-    const int c2 = lm_code(y2, w, sThr);
-    uint32_t* dst = stage + al->word_off[blk];
-    for (int p = 0; p < w; ++p) {
-      const unsigned A = __ballot_sync(0xffffffffu, valid && ((c1 >> p) & 1));
-      const unsigned B = __ballot_sync(0xffffffffu, valid && ((c2 >> p) & 1));
-      if (lane == 0) {
-        dst[2 * p] = A;
-        dst[2 * p + 1] = B;
+      for (int u = 0; u < 2; ++u) {
+        const int blk = 2 * bp + u;
+        const int w = tw[blk];
+        if (w == 0) continue;
+        const float g = tg[blk];
+        const float y1 = __fmul_rn(__fmul_rn(u ? lo.y : lo.x, a), g);
+        const float y2 = __fmul_rn(__fmul_rn(u ? hi.y : hi.x, a), g);
+        search_ballot2(y1, y2, w, sThr + ((1 << w) - w - 1), valid, stage + to[blk], 2, 1, lane);
       }
     }
-  }
 
-  // ---------------------------------------------------------------- V (uniform width)
-  if (valid) row.load(V + b * vsb + h * vsh + static_cast<int64_t>(token) * vst);
-  else row.zero();
-  row_norm_scale<DT>(row, vn16, a);
-#pragma unroll
-  for (int j = 0; j < kD; ++j) {
-    const float y = __fmul_rn(row.get(j), a);
-    const int c = lm_code(y, bits_v, sThr);
-    for (int p = 0; p < bits_v; ++p) {
-      const unsigned W = __ballot_sync(0xffffffffu, valid && ((c >> p) & 1));
-      if (lane == 0) vstage[p * kD + j] = W;
+    // ---------------------------------------------------------------- V (uniform width)
+    __syncwarp();
+    Row::load(rows, V + b * vsb + h * vsh + static_cast<int64_t>(t0) * vst, vst, valid_rows, lane);
+    __syncwarp();
+    row_norm_scale<DT>(myrow, vn16, a);
+#pragma unroll 2
+    for (int i = 0; i < kD / 2; ++i) {
+      const float2 x = Row::pair(myrow, i);
+      search_ballot2(__fmul_rn(x.x, a), __fmul_rn(x.y, a), bits_v, vthr, valid, vstage + 2 * i, kD, 1, lane);
     }
-  }
-  __syncwarp();
+    __syncwarp();
 
-  // ---------------------------------------------------------------- permute + store
-  uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
-  uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
-  for (int k = lane; k < k_words / 2; k += 32) {
-    const uint32_t A = stage[2 * k], B = stage[2 * k + 1];
-    uint2 o;
-    o.x = (A & 0x0f0f0f0fu) | ((B & 0x0f0f0f0fu) << 4);
-    o.y = ((A >> 4) & 0x0f0f0f0fu) | (B & 0xf0f0f0f0u);
-    reinterpret_cast<uint2*>(kout)[k] = o;
+    // ---------------------------------------------------------------- permute + store
+    uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
+    uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
+    for (int k = lane; k < k_words / 2; k += 32) {
+      const uint32_t A = stage[2 * k], B = stage[2 * k + 1];
+      uint2 o;
+      o.x = (A & 0x0f0f0f0fu) | ((B & 0x0f0f0f0fu) << 4);
+      o.y = ((A >> 4) & 0x0f0f0f0fu) | (B & 0xf0f0f0f0u);
+      reinterpret_cast<uint2*>(kout)[k] = o;
+    }
+    uint32_t* vout = kout + k_words;
+    for (int k = lane; k < v_words / 4; k += 32) {
+      const uint4 v = reinterpret_cast<const uint4*>(vstage)[k];
+      reinterpret_cast<uint4*>(vout)[k] = make_uint4(unzip_bytes(v.x), unzip_bytes(v.y), unzip_bytes(v.z),
+                                                     unzip_bytes(v.w));
+    }
+    uint16_t* norms = reinterpret_cast<uint16_t*>(vout + v_words);
+    norms[lane] = valid ? __half_as_ushort(kn16) : 0;
+    norms[kTile + lane] = valid ? __half_as_ushort(vn16) : 0;
   }
-  uint32_t* vout = kout + k_words;
-  for (int k = lane; k < v_words; k += 32) vout[k] = unzip_bytes(vstage[k]);
-  uint16_t* norms = reinterpret_cast<uint16_t*>(vout + v_words);
-  norms[lane] = valid ? __half_as_ushort(kn16) : 0;
-  norms[kTile + lane] = valid ? __half_as_ushort(vn16) : 0;
+}
+
+// Dynamic shared memory of kvq_quant_pack for the input type's row pitch.
+inline size_t quant_smem_bytes(int dtype, int bits_k, int bits_v) {
+  const int row_words = (dtype == KVQ_F32) ? QuantRow<KVQ_F32>::kWords : QuantRow<KVQ_BF16>::kWords;
+  return 4 * (512 + static_cast<size_t>(kQuantWarps) * (row_words + (bits_k + bits_v) * kD + 3 * kH));
 }
 
 }  // namespace kvq
