@@ -146,7 +146,7 @@ def run_gpu(args, rank, world, local_rank):
     allocs = [torch.empty(kvq.kvq_alloc_bytes(Hkv), dtype=torch.uint8, device=dev) for _ in range(L)]
     packs = [torch.empty(kvq.kvq_packed_bytes(cache), dtype=torch.uint8, device=dev) for _ in range(L)]
     outs = [torch.empty((B, Hq, d), dtype=torch.float32, device=dev) for _ in range(L)]
-    cws = torch.empty(kvq.kvq_calibrate_workspace_bytes(B, Hkv, T), dtype=torch.uint8, device=dev)
+    cws = torch.zeros(kvq.kvq_calibrate_workspace_bytes(B, Hkv, T), dtype=torch.uint8, device=dev)
     dws = [torch.zeros(kvq.kvq_decode_workspace_bytes(cache, Hq), dtype=torch.uint8, device=dev) for _ in range(L)]
     stream = torch.cuda.current_stream()
 

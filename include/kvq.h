@@ -143,8 +143,9 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* cache, int n_q_heads);
  * launching call does it too. */
 kvq_status kvq_init(void);
 
-/* Zero a decode or calibrate workspace (async memset on `stream`). A decode workspace must
- * be zeroed once before its first use; the kernels leave it reusable. */
+/* Zero a decode or calibrate workspace (async memset on `stream`). Both hold counters that
+ * must start at zero: zero a workspace once before its first use; the kernels return the
+ * counters to zero, so it stays reusable. Calls sharing one workspace must not overlap. */
 kvq_status kvq_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronizes `stream`, copies the workspace status word to *device_code (host) and
@@ -160,8 +161,11 @@ kvq_status kvq_workspace_status(const void* ws, void* stream, int* device_code);
  * first n_calib tokens of every sequence (pooled), then the greedy allocation:
  * bits_k * 64 steps, each adding one bit to the block with the largest
  * E_b (delta(w_b) - delta(w_b + 1)) below w_max, ties to the lowest block.
+ * The sum runs in a fixed order (64-token chunks, 64-chunk segments, segments), so the
+ * energies are reproducible bit for bit.
  * Writes n_kv_heads kvq_head_alloc records to alloc_out.
- * ws: workspace of kvq_calibrate_workspace_bytes(batch, n_kv_heads, n_calib) bytes. */
+ * ws: workspace of kvq_calibrate_workspace_bytes(batch, n_kv_heads, n_calib) bytes, zeroed
+ * once by kvq_workspace_init. */
 kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_params* params,
                          void* alloc_out, void* ws, size_t ws_bytes, void* stream);
 

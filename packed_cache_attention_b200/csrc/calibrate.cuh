@@ -11,75 +11,138 @@ namespace kvq {
 constexpr int kCalibSegment = 64;      // chunk sums per fixed-order segment sum
 constexpr int kCalibChunksPerCta = 8;  // 16 lanes per chunk, 128 threads
 
+// Calibration workspace after the status header: per KV head a head counter and one counter
+// per segment (unsigned, zero between calls), then energies E[h][64], segment sums
+// [h][n_seg][64] and chunk sums [h][n_chunks][64] (fp64).
+struct CalibWs {
+  unsigned* head_count;   // [H]
+  unsigned* seg_count;    // [H][n_seg]
+  double* energy;         // [H][64]
+  double* seg_sum;        // [H][n_seg][64]
+  double* chunk_sum;      // [H][n_chunks][64]
+};
+
 // Grid (ceil(n_chunks / 8), n_kv_heads), 128 threads: 16 lanes per 64-token chunk. Lane k
 // (0..15) of a chunk owns blocks 4k..4k+3, i.e. dims 4k..4k+3 and 64+4k..67+4k, read as two
 // 4-element vectors per token (128 contiguous bytes per half-warp for 16-bit inputs). Within
 // the chunk the pooled tokens u = s*n_calib + t are summed left to right in fp64, each term
 // being fl(fl(x^2) + fl(y^2)).
+// The CTA that completes a segment (atomic ticket per segment) sums that segment's 64 chunk
+// sums left to right; the CTA that completes the last segment of a head sums the segment
+// sums left to right and writes E_b = total / N. Counters are reset to zero for the next call.
 template <int DT>
 __global__ void __launch_bounds__(16 * kCalibChunksPerCta) kvq_calib_reduce(
     const typename Elem<DT>::T* __restrict__ K, int n_calib, int64_t sb, int64_t sh, int64_t st, int N,
-    int n_chunks, double* __restrict__ partial) {
+    int n_chunks, CalibWs ws) {
   using T = typename Elem<DT>::T;
+  __shared__ int sTicket;
   const int h = blockIdx.y;
   const int chunk = blockIdx.x * kCalibChunksPerCta + (threadIdx.x >> 4);
   const int k = threadIdx.x & 15;
-  if (chunk >= n_chunks) return;
-  const int u0 = chunk * kCalibChunk;
-  const int n = min(N - u0, kCalibChunk);
-  int s = u0 / n_calib;
-  int t = u0 - s * n_calib;
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 16
-  for (int i = 0; i < n; ++i) {
-    const T* row = K + s * sb + h * sh + static_cast<int64_t>(t) * st;
-    float x[4], y[4];
-    if constexpr (DT == KVQ_F32) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(row + 4 * k));
-      const float4 b = __ldg(reinterpret_cast<const float4*>(row + kH + 4 * k));
-      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-      y[0] = b.x; y[1] = b.y; y[2] = b.z; y[3] = b.w;
-    } else {
-      const uint2 a = __ldg(reinterpret_cast<const uint2*>(row + 4 * k));
-      const uint2 b = __ldg(reinterpret_cast<const uint2*>(row + kH + 4 * k));
-      const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
+  const int n_seg = (n_chunks + kCalibSegment - 1) / kCalibSegment;
+  if (chunk < n_chunks) {
+    const int u0 = chunk * kCalibChunk;
+    const int n = min(N - u0, kCalibChunk);
+    int s = u0 / n_calib;
+    int t = u0 - s * n_calib;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    auto add_row = [&](const T* row) {
+      float x[4], y[4];
+      if constexpr (DT == KVQ_F32) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(row + 4 * k));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(row + kH + 4 * k));
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        y[0] = b.x; y[1] = b.y; y[2] = b.z; y[3] = b.w;
+      } else {
+        const uint2 a = __ldg(reinterpret_cast<const uint2*>(row + 4 * k));
+        const uint2 b = __ldg(reinterpret_cast<const uint2*>(row + kH + 4 * k));
+        const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        x[2 * j] = Elem<DT>::to_f32(bits_to<T>(av[j] & 0xffffu));
-        x[2 * j + 1] = Elem<DT>::to_f32(bits_to<T>(av[j] >> 16));
-        y[2 * j] = Elem<DT>::to_f32(bits_to<T>(bv[j] & 0xffffu));
-        y[2 * j + 1] = Elem<DT>::to_f32(bits_to<T>(bv[j] >> 16));
+        for (int j = 0; j < 2; ++j) {
+          x[2 * j] = Elem<DT>::to_f32(bits_to<T>(av[j] & 0xffffu));
+          x[2 * j + 1] = Elem<DT>::to_f32(bits_to<T>(av[j] >> 16));
+          y[2 * j] = Elem<DT>::to_f32(bits_to<T>(bv[j] & 0xffffu));
+          y[2 * j + 1] = Elem<DT>::to_f32(bits_to<T>(bv[j] >> 16));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const double dx = x[j], dy = y[j];
+        acc[j] = __dadd_rn(acc[j], __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)));
+      }
+    };
+    if (n == kCalibChunk && t + kCalibChunk <= n_calib) {
+      // whole chunk inside one sequence: independent row addresses, loads pipeline freely
+      const T* base = K + s * sb + h * sh + static_cast<int64_t>(t) * st;
+#pragma unroll 16
+      for (int i = 0; i < kCalibChunk; ++i) add_row(base + static_cast<int64_t>(i) * st);
+    } else {
+      for (int i = 0; i < n; ++i) {
+        add_row(K + s * sb + h * sh + static_cast<int64_t>(t) * st);
+        if (++t == n_calib) {
+          t = 0;
+          ++s;
+        }
       }
     }
+    double* dst = ws.chunk_sum + (static_cast<size_t>(h) * n_chunks + chunk) * kH + 4 * k;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const double dx = x[j], dy = y[j];
-      acc[j] = __dadd_rn(acc[j], __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)));
-    }
-    if (++t == n_calib) {
-      t = 0;
-      ++s;
-    }
+    for (int j = 0; j < 4; ++j) dst[j] = acc[j];
   }
-  double* dst = partial + (static_cast<size_t>(h) * n_chunks + chunk) * kH + 4 * k;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) dst[j] = acc[j];
+
+  // ---- segment completion (chunks of one CTA always lie in one segment: 8 divides 64)
+  const int seg = (blockIdx.x * kCalibChunksPerCta) / kCalibSegment;
+  const int c0 = seg * kCalibSegment, c1 = min(n_chunks, c0 + kCalibSegment);
+  const int mine = min(n_chunks, (blockIdx.x + 1) * kCalibChunksPerCta) - blockIdx.x * kCalibChunksPerCta;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned* cnt = ws.seg_count + static_cast<size_t>(h) * n_seg + seg;
+    const unsigned done = atomicAdd(cnt, static_cast<unsigned>(mine)) + mine;
+    sTicket = (done == static_cast<unsigned>(c1 - c0));
+    if (sTicket) *cnt = 0u;
+  }
+  __syncthreads();
+  if (!sTicket) return;
+  __threadfence();
+  if (threadIdx.x < kH) {
+    const double* src = ws.chunk_sum + (static_cast<size_t>(h) * n_chunks) * kH + threadIdx.x;
+    double acc = 0.0;
+#pragma unroll 16
+    for (int c = c0; c < c1; ++c) acc = __dadd_rn(acc, __ldcg(src + static_cast<size_t>(c) * kH));
+    ws.seg_sum[(static_cast<size_t>(h) * n_seg + seg) * kH + threadIdx.x] = acc;
+  }
+  // ---- head completion
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned done = atomicAdd(ws.head_count + h, 1u) + 1u;
+    sTicket = (done == static_cast<unsigned>(n_seg));
+    if (sTicket) ws.head_count[h] = 0u;
+  }
+  __syncthreads();
+  if (!sTicket) return;
+  __threadfence();
+  if (threadIdx.x < kH) {
+    const double* src = ws.seg_sum + static_cast<size_t>(h) * n_seg * kH + threadIdx.x;
+    double S = 0.0;
+#pragma unroll 8
+    for (int g = 0; g < n_seg; ++g) S = __dadd_rn(S, __ldcg(src + static_cast<size_t>(g) * kH));
+    ws.energy[static_cast<size_t>(h) * kH + threadIdx.x] = __ddiv_rn(S, static_cast<double>(N));
+  }
 }
 
-// One CTA of 512 threads per KV head.
-//  1. E_b: chunk partials summed left to right within segments of 64 chunks (8 segments in
-//     flight per block), segment sums left to right, divided by N; fp64.
-//  2. Greedy allocation in rank form: entry e = 8b + w (w < w_max) has marginal gain
+// One CTA of 512 threads per KV head, after kvq_calib_reduce has written E[h][64].
+//  1. Greedy allocation in rank form: entry e = 8b + w (w < w_max) has marginal gain
 //     E_b (delta(w) - delta(w+1)); the greedy takes the bits_k * 64 first entries in the
 //     order (gain descending, e ascending). Because delta is strictly convex each block's
 //     gains are non-increasing in w, so this is the step-by-step greedy with ties to the
 //     lowest block, the entries of a block that precede a given entry form a prefix (found
 //     by binary search), and the picked entries of a block are a prefix: w_b = their count.
-//  3. g_b, f_b, the K word offsets and the decode k-step table (blocks grouped by width,
+//  2. g_b, f_b, the K word offsets and the decode k-step table (blocks grouped by width,
 //     widest first, 4 per step, ascending block index within a width).
-__global__ void __launch_bounds__(512) kvq_greedy_alloc(double* __restrict__ partial, int n_chunks,
-                                                        int N, int bits_k, int w_max, int mode,
-                                                        kvq_head_alloc* __restrict__ alloc) {
+__global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict__ energy, int bits_k, int w_max,
+                                                        int mode, kvq_head_alloc* __restrict__ alloc) {
   __shared__ double sE[kH];
   __shared__ double sGain[kH * 8];
   __shared__ int sWidth[kH];
@@ -88,25 +151,7 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(double* __restrict__ par
   __shared__ double sSum;
   const int h = blockIdx.x, tid = threadIdx.x;
   kvq_head_alloc* al = alloc + h;
-  double* ph = partial + static_cast<size_t>(h) * n_chunks * kH;
-  const int n_seg = (n_chunks + kCalibSegment - 1) / kCalibSegment;
-
-  {
-    const int b = tid & (kH - 1), r = tid >> 6;
-    for (int sg = r; sg < n_seg; sg += 8) {
-      const int c0 = sg * kCalibSegment, c1 = min(n_chunks, c0 + kCalibSegment);
-      double acc = 0.0;
-#pragma unroll 8
-      for (int c = c0; c < c1; ++c) acc = __dadd_rn(acc, ph[static_cast<size_t>(c) * kH + b]);
-      ph[static_cast<size_t>(c0) * kH + b] = acc;     // the segment's first slot holds its sum
-    }
-  }
-  __syncthreads();
-  if (tid < kH) {
-    double S = 0.0;
-    for (int sg = 0; sg < n_seg; ++sg) S = __dadd_rn(S, __ldcg(ph + static_cast<size_t>(sg) * kCalibSegment * kH + tid));
-    sE[tid] = __ddiv_rn(S, static_cast<double>(N));
-  }
+  if (tid < kH) sE[tid] = __ldcg(energy + static_cast<size_t>(h) * kH + tid);
   __syncthreads();
   if (tid == 0) {
     double S = 0.0;

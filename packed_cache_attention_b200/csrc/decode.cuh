@@ -24,10 +24,11 @@
 
 namespace kvq {
 
-constexpr int kDecWarps = 8;
-constexpr int kDecStages = 3;
+constexpr int kDecWarps = 16;
+constexpr int kDecStages = 3;        // deepest cp.async pipeline per warp (fewer when records are large)
 constexpr int kMaxSteps = 32;
-constexpr int kTargetCtas = 296;   // 2 CTAs per SM on a 148-SM B200
+constexpr int kMaxMergeSplits = 160;
+constexpr int kTargetCtas = 148;   // 1 CTA of 16 warps per SM on a 148-SM B200
 
 struct DecodeSmem {
   uint2 qfrag[kMaxSteps][8][4];     // A fragments of Q' per k-step, head row g, lane c
@@ -39,8 +40,11 @@ struct DecodeSmem {
   uint16_t woff[kH];
   int8_t step_blk[kMaxSteps][4];
   uint8_t step_w[kMaxSteps];
+  uint32_t step_info[kMaxSteps][4];  // per step and lane c: width | K word offset of its block << 8
   int n_steps;
   int last;
+  float mw[8][kMaxMergeSplits];     // cross-split merge: weight 2^(m_s - M) per head and split
+  float Lsum[8];
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -49,13 +53,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// Gather bit p of 8 codes from `w` plane words (word p at words[p * stride]; code m at bit
+// Gather bit p of 8 codes from W plane words (word p at words[p * stride]; code m at bit
 // shift + 4m) into 4-bit nibbles: nibble m of the result is code m.
-__device__ __forceinline__ uint32_t gather_nibbles(const uint32_t* words, int stride, int w, int shift) {
+template <int W>
+__device__ __forceinline__ uint32_t gather_nibbles(const uint32_t* words, int stride, int shift) {
   uint32_t x = 0;
 #pragma unroll
-  for (int p = 0; p < 4; ++p)
-    if (p < w) x |= rotr(words[p * stride], static_cast<uint32_t>(shift - p) & 31u) & (0x11111111u << p);
+  for (int p = 0; p < W; ++p) x |= rotr(words[p * stride], static_cast<uint32_t>(shift - p) & 31u) & (0x11111111u << p);
   return x;
 }
 
@@ -87,33 +91,58 @@ __device__ __forceinline__ void lut16(uint32_t x, const uint4& LO, const uint4& 
   r[3] = prmt(lb, hb, 0x7362u);
 }
 
-// Any width: assemble each code from its planes and look it up in the shared table.
-__device__ __forceinline__ void lut_generic(const uint32_t* words, int stride, int w, int shift,
-                                            const uint16_t* table, uint32_t (&r)[4]) {
-  uint32_t W[8];
+// Widths 5..8: gather the 8 codes as bytes (even codes in `ev`, odd codes in `od`, byte k =
+// code 2k / 2k+1), one rotate + mask per plane and parity, then look each byte up in the
+// shared fp16 table.
+template <int W>
+__device__ __forceinline__ void lut_wide(const uint32_t* words, int stride, int shift, const uint16_t* table,
+                                         uint32_t (&r)[4]) {
+  uint32_t ev = 0u, od = 0u;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) W[p] = (p < w) ? words[p * stride] : 0u;
-  uint32_t val[8];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    uint32_t code = 0;
-#pragma unroll
-    for (int p = 0; p < 8; ++p) code |= ((W[p] >> (shift + 4 * m)) & 1u) << p;
-    val[m] = table[code];
+  for (int p = 0; p < W; ++p) {
+    const uint32_t w = words[p * stride];
+    ev |= rotr(w, static_cast<uint32_t>(shift - p) & 31u) & (0x01010101u << p);
+    od |= rotr(w, static_cast<uint32_t>(shift + 4 - p) & 31u) & (0x01010101u << p);
   }
 #pragma unroll
-  for (int k = 0; k < 4; ++k) r[k] = pack_u16x2(val[2 * k], val[2 * k + 1]);
+  for (int k = 0; k < 4; ++k)
+    r[k] = pack_u16x2(table[(ev >> (8 * k)) & 0xffu], table[(od >> (8 * k)) & 0xffu]);
 }
 
-// The 8 codes at bits shift + 4m of `w` plane words, as 4 fp16x2 fragments.
-__device__ __forceinline__ void decode8(const uint32_t* words, int stride, int w, int shift, const DecodeSmem& S,
+// The 8 codes of width W at bits shift + 4m of W plane words, as 4 fp16x2 fragments
+// (r[k] = (code 2k, code 2k+1)).
+template <int W>
+__device__ __forceinline__ void decode8(const uint32_t* words, int stride, int shift, const DecodeSmem& S,
                                         uint32_t (&r)[4]) {
-  if (w <= 3) {
-    lut8(gather_nibbles(words, stride, w, shift), S.lut8[w], r);
-  } else if (w == 4) {
-    lut16(gather_nibbles(words, stride, 4, shift), S.lut16[0], S.lut16[1], r);
+  if constexpr (W <= 3) {
+    lut8(gather_nibbles<W>(words, stride, shift), S.lut8[W], r);
+  } else if constexpr (W == 4) {
+    lut16(gather_nibbles<4>(words, stride, shift), S.lut16[0], S.lut16[1], r);
   } else {
-    lut_generic(words, stride, w, shift, S.cent + ((1 << w) - 2), r);
+    lut_wide<W>(words, stride, shift, S.cent + ((1 << W) - 2), r);
+  }
+}
+
+// One QK k-step: 4 RoPE blocks (one per lane c) x 32 tokens (4 n-tiles).
+template <int W>
+__device__ __forceinline__ void qk_step(const uint32_t* kw, uint32_t info, int H, int sh, uint2 a, const DecodeSmem& S,
+                                        float (&acc)[4][4]) {
+  uint32_t bf[4];
+  decode8<W>(kw + (info >> 8) + H, 2, sh, S, bf);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) mma_m16n8k8(acc[j], a.x, a.y, bf[j]);
+}
+
+// O += P' V over the 16 dim n-tiles for value width W.
+template <int W>
+__device__ __forceinline__ void pv_all(const uint32_t* vw, int g, int c, const uint32_t (&pa_hi)[4],
+                                       const uint32_t (&pa_lo)[4], const DecodeSmem& S, float (&o_acc)[16][4]) {
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) {
+    uint32_t vf[4];
+    decode8<W>(vw + 8 * nt + g, kD, c, S, vf);
+    mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], vf[0], vf[1]);
+    mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], vf[2], vf[3]);
   }
 }
 
@@ -125,7 +154,7 @@ template <int DT>
 __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
     const typename Elem<DT>::T* __restrict__ q, int64_t qsb, int64_t qsh, int n_q_heads, int n_kv_heads,
     const uint8_t* __restrict__ packed, const kvq_head_alloc* __restrict__ alloc, int tiles_cap,
-    int rec_bytes, int bits_v, int seq_len, int splits, float* __restrict__ out,
+    int rec_bytes, int bits_v, int seq_len, int splits, int n_stages, float* __restrict__ out,
     float* __restrict__ part_m, float* __restrict__ part_l, float* __restrict__ part_o,
     unsigned* __restrict__ tickets) {
   extern __shared__ __align__(16) uint8_t dsmem[];
@@ -147,13 +176,12 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
   const float inv_sqrt_d = 0.08838834764831845f;
 
   const int stage_bytes = ((rec_bytes + 127) / 128) * 128;
-  uint8_t* my_stages = stages + warp * kDecStages * stage_bytes;
+  uint8_t* my_stages = stages + warp * n_stages * stage_bytes;
   const uint8_t* src_base = packed + static_cast<size_t>(bh) * tiles_cap * rec_bytes;
   const int first = t_begin + warp;
   const int my_n = (first < t_end) ? (t_end - first + kDecWarps - 1) / kDecWarps : 0;
   // Start streaming the first tiles before the prologue.
-#pragma unroll
-  for (int i = 0; i < kDecStages - 1; ++i) {
+  for (int i = 0; i < n_stages - 1; ++i) {
     if (i < my_n)
       decode_load_tile(my_stages + i * stage_bytes, src_base + static_cast<size_t>(first + i * kDecWarps) * rec_bytes,
                        rec_bytes, lane);
@@ -210,6 +238,13 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
   }
   __syncthreads();
   const int n_steps = S.n_steps;
+  for (int i = tid; i < n_steps * 4; i += blockDim.x) {
+    const int st = i >> 2, cc = i & 3;
+    int blk = S.step_blk[st][cc];
+    if (blk < 0) blk = max(static_cast<int>(S.step_blk[st][0]), 0);   // empty slot: Q' is 0 there
+    const int w = min(max(static_cast<int>(S.step_w[st]), 1), 8);
+    S.step_info[st][cc] = static_cast<uint32_t>(w) | (static_cast<uint32_t>(S.woff[min(blk, kH - 1)]) << 8);
+  }
   for (int i = tid; i < n_steps * 32; i += blockDim.x) {
     const int s = i >> 5, hg = (i >> 2) & 7, cc = i & 3;
     const int blk = S.step_blk[s][cc];
@@ -235,16 +270,16 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
   const int H = g >> 2, sh = g & 3;
   for (int i = 0; i < my_n; ++i) {
     {
-      const int nxt = i + kDecStages - 1;
+      const int nxt = i + n_stages - 1;
       if (nxt < my_n)
-        decode_load_tile(my_stages + (nxt % kDecStages) * stage_bytes,
+        decode_load_tile(my_stages + (nxt % n_stages) * stage_bytes,
                          src_base + static_cast<size_t>(first + nxt * kDecWarps) * rec_bytes, rec_bytes, lane);
       cp_async_commit();
     }
-    cp_async_wait<kDecStages - 1>();
+    cp_async_wait_pending(n_stages - 1);
     __syncwarp();
     const int tile = first + i * kDecWarps;
-    const uint8_t* st = my_stages + (i % kDecStages) * stage_bytes;
+    const uint8_t* st = my_stages + (i % n_stages) * stage_bytes;
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(st);
     const uint32_t* vw = kw + k_words;
     const uint16_t* kn = reinterpret_cast<const uint16_t*>(vw + bits_v * kD);
@@ -255,14 +290,18 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
     for (int s = 0; s < n_steps; ++s) {
-      const int w = min(max(static_cast<int>(S.step_w[s]), 1), 8);
-      int blk = S.step_blk[s][c];
-      if (blk < 0) blk = max(static_cast<int>(S.step_blk[s][0]), 0);   // empty slot: Q' is 0 there
-      uint32_t bf[4];
-      decode8(kw + S.woff[blk] + H, 2, w, sh, S, bf);
+      const uint32_t info = S.step_info[s][c];
       const uint2 a = S.qfrag[s][g][c];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) mma_m16n8k8(acc[j], a.x, a.y, bf[j]);
+      switch (info & 0xffu) {
+        case 1: qk_step<1>(kw, info, H, sh, a, S, acc); break;
+        case 2: qk_step<2>(kw, info, H, sh, a, S, acc); break;
+        case 3: qk_step<3>(kw, info, H, sh, a, S, acc); break;
+        case 4: qk_step<4>(kw, info, H, sh, a, S, acc); break;
+        case 5: qk_step<5>(kw, info, H, sh, a, S, acc); break;
+        case 6: qk_step<6>(kw, info, H, sh, a, S, acc); break;
+        case 7: qk_step<7>(kw, info, H, sh, a, S, acc); break;
+        default: qk_step<8>(kw, info, H, sh, a, S, acc); break;
+      }
     }
 
     // ---- online softmax over the 8 tokens this lane holds: 8j + 2c + {0,1}
@@ -309,37 +348,19 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
     }
 
     // ---- O += P' Vhat over 16 dim n-tiles, two 16-token k-steps
-    if (bits_v <= 3) {
-      const uint4 L = S.lut8[bits_v];
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        uint32_t vf[4];
-        lut8(gather_nibbles(vw + 8 * nt + g, kD, bits_v, c), L, vf);
-        mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], vf[0], vf[1]);
-        mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], vf[2], vf[3]);
-      }
-    } else if (bits_v == 4) {
-      const uint4 LO = S.lut16[0], HI = S.lut16[1];
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        uint32_t vf[4];
-        lut16(gather_nibbles(vw + 8 * nt + g, kD, 4, c), LO, HI, vf);
-        mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], vf[0], vf[1]);
-        mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], vf[2], vf[3]);
-      }
-    } else {
-      const uint16_t* table = S.cent + ((1 << bits_v) - 2);
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        uint32_t vf[4];
-        lut_generic(vw + 8 * nt + g, kD, bits_v, c, table, vf);
-        mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], vf[0], vf[1]);
-        mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], vf[2], vf[3]);
-      }
+    switch (bits_v) {
+      case 1: pv_all<1>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
+      case 2: pv_all<2>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
+      case 3: pv_all<3>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
+      case 4: pv_all<4>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
+      case 5: pv_all<5>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
+      case 6: pv_all<6>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
+      case 7: pv_all<7>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
+      default: pv_all<8>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
     }
     __syncwarp();
   }
-  cp_async_wait<0>();
+  cp_async_wait_pending(0);
 
   // ------------------------------------------------------------------ combine warps
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
@@ -392,21 +413,50 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
   __syncthreads();
   if (!S.last) return;
   __threadfence();
-  for (int i = tid; i < 8 * kD; i += blockDim.x) {
-    const int hg = i / kD, j = i % kD;
-    if (hg >= G) continue;
+  // weights 2^(m_s - M) per (head, split) and the merged denominators, one warp per head
+  for (int hg = warp; hg < 8; hg += kDecWarps) {
     const size_t p0 = static_cast<size_t>(bh) * splits * 8 + hg;
     float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(part_m + p0 + static_cast<size_t>(s) * 8));
-    float L = 0.0f, O = 0.0f;
-    for (int s = 0; s < splits; ++s) {
+    for (int s = lane; s < splits; s += 32) M = fmaxf(M, __ldcg(part_m + p0 + static_cast<size_t>(s) * 8));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.0f;
+    for (int s = lane; s < splits; s += 32) {
       const size_t pi = p0 + static_cast<size_t>(s) * 8;
       const float ms = __ldcg(part_m + pi);
       const float wt = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
+      S.mw[hg][s] = wt;
       L += __ldcg(part_l + pi) * wt;
-      O += __ldcg(part_o + pi * kD + j) * wt;
     }
-    out[(static_cast<size_t>(b) * n_q_heads + hkv * G + hg) * kD + j] = O / L;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) S.Lsum[hg] = L;
+  }
+  __syncthreads();
+  // O: 256 (head, 4-dim) quads, two threads each over the two halves of the splits
+  {
+    const int quad = tid & 255, half = tid >> 8;
+    const int hg = quad >> 5, j4 = (quad & 31) * 4;
+    const int s_mid = splits / 2;
+    const int s0 = half ? s_mid : 0, s1 = half ? splits : s_mid;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* po = reinterpret_cast<const float4*>(part_o);
+#pragma unroll 8
+    for (int s = s0; s < s1; ++s) {
+      const float wt = S.mw[hg][s];
+      const float4 v = __ldcg(po + ((static_cast<size_t>(bh) * splits + s) * 8 + hg) * (kD / 4) + j4 / 4);
+      o.x += v.x * wt; o.y += v.y * wt; o.z += v.z * wt; o.w += v.w * wt;
+    }
+    float4* red = reinterpret_cast<float4*>(stages);
+    if (half) red[quad] = o;
+    __syncthreads();
+    if (!half && hg < G) {
+      const float4 v = red[quad];
+      const float inv = 1.0f / S.Lsum[hg];
+      float4 r;
+      r.x = (o.x + v.x) * inv; r.y = (o.y + v.y) * inv; r.z = (o.z + v.z) * inv; r.w = (o.w + v.w) * inv;
+      reinterpret_cast<float4*>(out + (static_cast<size_t>(b) * n_q_heads + hkv * G + hg) * kD)[j4 / 4] = r;
+    }
   }
   if (tid == 0) tickets[bh] = 0u;
 }

@@ -75,7 +75,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int decode_splits(int bh, int n_tiles) {
   const int want = (kTargetCtas + bh - 1) / bh;
-  return std::max(1, std::min(want, n_tiles));
+  return std::max(1, std::min(std::min(want, n_tiles), kMaxMergeSplits));
 }
 
 struct DecodeWs {
@@ -117,11 +117,21 @@ Nf4Layout nf4_layout(int batch, int n_heads, int capacity) {
   return L;
 }
 
+constexpr size_t kMaxSmem = 227 * 1024;
+
+size_t decode_head_bytes() { return align_up(sizeof(DecodeSmem), 128); }
+size_t decode_combine_bytes() { return sizeof(float) * (kDecWarps * 8 * 2 + kDecWarps * 8 * kD); }
+
+// Deepest cp.async pipeline (1..3 tile records per warp) that fits in shared memory.
+int decode_stages(int rec_bytes) {
+  const size_t per = align_up(rec_bytes, 128) * kDecWarps;
+  const size_t room = kMaxSmem - decode_head_bytes();
+  return static_cast<int>(std::max<size_t>(1, std::min<size_t>(kDecStages, room / per)));
+}
+
 size_t decode_smem_bytes(int rec_bytes) {
-  const size_t head = align_up(sizeof(DecodeSmem), 128);
-  const size_t stage = align_up(rec_bytes, 128) * kDecStages * kDecWarps;
-  const size_t combine = sizeof(float) * (kDecWarps * 8 * 2 + kDecWarps * 8 * kD);
-  return head + std::max(stage, combine);
+  const size_t stage = align_up(rec_bytes, 128) * decode_stages(rec_bytes) * kDecWarps;
+  return decode_head_bytes() + std::max(stage, decode_combine_bytes());
 }
 
 }  // namespace
@@ -167,11 +177,33 @@ size_t kvq_alloc_bytes(int n_kv_heads) {
   return n_kv_heads > 0 ? static_cast<size_t>(n_kv_heads) * sizeof(kvq_head_alloc) : 0;
 }
 
+}  // extern "C"
+namespace {
+struct CalibWsLayout {
+  size_t head_count, seg_count, energy, seg_sum, chunk_sum, total;
+  int n_chunks, n_seg;
+};
+
+CalibWsLayout calib_ws_layout(int batch, int n_kv_heads, int n_calib_tokens) {
+  CalibWsLayout L;
+  const long long N = static_cast<long long>(batch) * n_calib_tokens;
+  L.n_chunks = static_cast<int>((N + kCalibChunk - 1) / kCalibChunk);
+  L.n_seg = (L.n_chunks + kCalibSegment - 1) / kCalibSegment;
+  L.head_count = sizeof(WsHeader);
+  L.seg_count = align_up(L.head_count + 4ull * n_kv_heads, 128);
+  L.energy = align_up(L.seg_count + 4ull * n_kv_heads * L.n_seg, 128);
+  L.seg_sum = align_up(L.energy + 8ull * n_kv_heads * kH, 128);
+  L.chunk_sum = align_up(L.seg_sum + 8ull * n_kv_heads * L.n_seg * kH, 128);
+  L.total = align_up(L.chunk_sum + 8ull * n_kv_heads * L.n_chunks * kH, 128);
+  return L;
+}
+}  // namespace
+extern "C" {
+
 size_t kvq_calibrate_workspace_bytes(int batch, int n_kv_heads, int n_calib_tokens) {
   if (batch < 1 || n_kv_heads < 1 || n_calib_tokens < 1) return 0;
-  const long long N = static_cast<long long>(batch) * n_calib_tokens;
-  const long long chunks = (N + kCalibChunk - 1) / kCalibChunk;
-  return sizeof(WsHeader) + static_cast<size_t>(n_kv_heads) * chunks * kH * sizeof(double);
+  if (static_cast<long long>(batch) * n_calib_tokens > 0x7fffffffLL) return 0;
+  return calib_ws_layout(batch, n_kv_heads, n_calib_tokens).total;
 }
 
 size_t kvq_packed_bytes(const kvq_cache_desc* c) {
@@ -216,26 +248,33 @@ kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_p
   if ((st = ensure_tables()) != KVQ_OK) return st;
   const long long N = static_cast<long long>(kd->batch) * n_calib;
   if (N > 0x7fffffffLL) return KVQ_ERR_RANGE;
-  const int n_chunks = static_cast<int>((N + kCalibChunk - 1) / kCalibChunk);
-  double* partial = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + sizeof(WsHeader));
+  const CalibWsLayout L = calib_ws_layout(kd->batch, kd->n_heads, n_calib);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  CalibWs cws;
+  cws.head_count = reinterpret_cast<unsigned*>(w8 + L.head_count);
+  cws.seg_count = reinterpret_cast<unsigned*>(w8 + L.seg_count);
+  cws.energy = reinterpret_cast<double*>(w8 + L.energy);
+  cws.seg_sum = reinterpret_cast<double*>(w8 + L.seg_sum);
+  cws.chunk_sum = reinterpret_cast<double*>(w8 + L.chunk_sum);
+  const int n_chunks = L.n_chunks;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid((n_chunks + kCalibChunksPerCta - 1) / kCalibChunksPerCta, kd->n_heads);
   const int threads = 16 * kCalibChunksPerCta;
   switch (kd->dtype) {
     case KVQ_F32:
-      kvq_calib_reduce<KVQ_F32><<<grid, threads, 0, s>>>(static_cast<const float*>(K), n_calib, kd->stride_b, kd->stride_h,
-                                                    kd->stride_t, static_cast<int>(N), n_chunks, partial);
+      kvq_calib_reduce<KVQ_F32><<<grid, threads, 0, s>>>(static_cast<const float*>(K), n_calib, kd->stride_b,
+                                                         kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
       break;
     case KVQ_F16:
-      kvq_calib_reduce<KVQ_F16><<<grid, threads, 0, s>>>(static_cast<const __half*>(K), n_calib, kd->stride_b, kd->stride_h,
-                                                    kd->stride_t, static_cast<int>(N), n_chunks, partial);
+      kvq_calib_reduce<KVQ_F16><<<grid, threads, 0, s>>>(static_cast<const __half*>(K), n_calib, kd->stride_b,
+                                                         kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
       break;
     default:
       kvq_calib_reduce<KVQ_BF16><<<grid, threads, 0, s>>>(static_cast<const __nv_bfloat16*>(K), n_calib, kd->stride_b,
-                                                     kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, partial);
+                                                          kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
   }
   if ((st = launch_status()) != KVQ_OK) return st;
-  kvq_greedy_alloc<<<kd->n_heads, 512, 0, s>>>(partial, n_chunks, static_cast<int>(N), p->bits_k, p->w_max, p->mode,
+  kvq_greedy_alloc<<<kd->n_heads, 512, 0, s>>>(cws.energy, p->bits_k, p->w_max, p->mode,
                                                static_cast<kvq_head_alloc*>(alloc_out));
   return launch_status();
 }
@@ -313,7 +352,7 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
     kern<<<grid, kDecWarps * 32, smem, s>>>(                                                                          \
         static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, c->n_kv_heads,                             \
         static_cast<const uint8_t*>(packed), static_cast<const kvq_head_alloc*>(alloc), n_tiles_of(c->capacity), rec, \
-        c->bits_v, seq_len, splits, out, reinterpret_cast<float*>(w8 + L.part_m),                                    \
+        c->bits_v, seq_len, splits, decode_stages(rec), out, reinterpret_cast<float*>(w8 + L.part_m),                                    \
         reinterpret_cast<float*>(w8 + L.part_l), reinterpret_cast<float*>(w8 + L.part_o),                             \
         reinterpret_cast<unsigned*>(w8 + L.tickets));                                                                 \
   } while (0)

@@ -106,24 +106,77 @@ __device__ __forceinline__ uint32_t unzip_bytes(uint32_t x) {
   return x;
 }
 
-// Binary search for two values of the same width; the ballot of the comparison at level p
-// (bit p of the code) is written to out[p * pstride] (first value) and out[p * pstride + 1]
-// (second value, when `two`), by lane 0.
-__device__ __forceinline__ void search_ballot2(float y1, float y2, int w, const float* __restrict__ thr, bool valid,
-                                               uint32_t* out, int pstride, int second_off, int lane) {
-  int i1 = 0, i2 = 0;
-  for (int p = w - 1; p >= 0; --p) {
-    const int s = 1 << p;
-    const bool b1 = y1 > thr[i1 + s - 1];
-    const bool b2 = y2 > thr[i2 + s - 1];
-    const unsigned A = __ballot_sync(0xffffffffu, valid && b1);
-    const unsigned B = __ballot_sync(0xffffffffu, valid && b2);
-    if (lane == 0) {
-      out[p * pstride] = A;
-      out[p * pstride + second_off] = B;
+// Binary search for two values of the same width W; the ballot of the comparison at level p
+// (bit p of the code) is written by lane 0 to out[p * pstride] (first value) and
+// out[p * pstride + 1] (second value). The top level compares with the middle threshold,
+// which is exactly 0 for these symmetric codebooks. Widths up to 3 select the next
+// threshold from registers (t[] holds the 2^W - 1 thresholds); wider ones index the
+// shared-memory table.
+template <int W>
+__device__ __forceinline__ void search_ballot2(float y1, float y2, const float* __restrict__ thr, const float* t,
+                                               uint32_t* out, int pstride, bool writer) {
+  // out[p * pstride] and out[p * pstride + 1] are adjacent, 8-byte aligned words.
+  auto put = [&](int p, bool c1, bool c2) {
+    const unsigned A = __ballot_sync(0xffffffffu, c1);
+    const unsigned B = __ballot_sync(0xffffffffu, c2);
+    if (writer) *reinterpret_cast<uint2*>(out + p * pstride) = make_uint2(A, B);
+  };
+  const bool h1 = y1 > 0.0f, h2 = y2 > 0.0f;
+  put(W - 1, h1, h2);
+  if constexpr (W == 2) {
+    put(0, y1 > (h1 ? t[2] : t[0]), y2 > (h2 ? t[2] : t[0]));
+  } else if constexpr (W == 3) {
+    const bool m1 = y1 > (h1 ? t[5] : t[1]), m2 = y2 > (h2 ? t[5] : t[1]);
+    put(1, m1, m2);
+    const float u1 = h1 ? (m1 ? t[6] : t[4]) : (m1 ? t[2] : t[0]);
+    const float u2 = h2 ? (m2 ? t[6] : t[4]) : (m2 ? t[2] : t[0]);
+    put(0, y1 > u1, y2 > u2);
+  } else if constexpr (W >= 4) {
+    int i1 = h1 ? (1 << (W - 1)) : 0, i2 = h2 ? (1 << (W - 1)) : 0;
+#pragma unroll
+    for (int p = W - 2; p >= 0; --p) {
+      const int s = 1 << p;
+      const bool c1 = y1 > thr[i1 + s - 1];
+      const bool c2 = y2 > thr[i2 + s - 1];
+      put(p, c1, c2);
+      i1 += c1 ? s : 0;
+      i2 += c2 ? s : 0;
     }
-    i1 += b1 ? s : 0;
-    i2 += b2 ? s : 0;
+  }
+}
+
+// Dispatch on a runtime width (uniform across the warp).
+__device__ __forceinline__ void search_ballot2_any(int w, float y1, float y2, const float* __restrict__ sThr,
+                                                   const float* t3, uint32_t* out, int pstride, bool writer) {
+  const float* thr = sThr + ((1 << w) - w - 1);
+  switch (w) {
+    case 1: search_ballot2<1>(y1, y2, thr, nullptr, out, pstride, writer); break;
+    case 2: {
+      const float t2[3] = {thr[0], thr[1], thr[2]};
+      search_ballot2<2>(y1, y2, thr, t2, out, pstride, writer);
+      break;
+    }
+    case 3: search_ballot2<3>(y1, y2, thr, t3, out, pstride, writer); break;
+    case 4: search_ballot2<4>(y1, y2, thr, nullptr, out, pstride, writer); break;
+    case 5: search_ballot2<5>(y1, y2, thr, nullptr, out, pstride, writer); break;
+    case 6: search_ballot2<6>(y1, y2, thr, nullptr, out, pstride, writer); break;
+    case 7: search_ballot2<7>(y1, y2, thr, nullptr, out, pstride, writer); break;
+    default: search_ballot2<8>(y1, y2, thr, nullptr, out, pstride, writer); break;
+  }
+}
+
+// Values: uniform width W for the whole row, dims processed in pairs.
+template <int DT, int W>
+__device__ __forceinline__ void quant_values(const uint32_t* myrow, float a, const float* __restrict__ sThr,
+                                             uint32_t* vstage, bool writer) {
+  const float* thr = sThr + ((1 << W) - W - 1);
+  float t[7];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) t[i] = (i < (1 << W) - 1) ? thr[i] : 0.0f;
+#pragma unroll 4
+  for (int i = 0; i < kD / 2; ++i) {
+    const float2 x = QuantRow<DT>::pair(myrow, i);
+    search_ballot2<W>(__fmul_rn(x.x, a), __fmul_rn(x.y, a), thr, t, vstage + 2 * i, kD, writer);
   }
 }
 
@@ -145,11 +198,12 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
   uint32_t* rows = smem + 512 + warp * warp_words;
   uint32_t* stage = rows + Row::kWords;
   uint32_t* vstage = stage + k_words;
-  int* tw = reinterpret_cast<int*>(vstage + v_words);   // per block: width
-  float* tg = reinterpret_cast<float*>(tw + kH);        // per block: gain
-  int* to = tw + 2 * kH;                                 // per block: K word offset
-  const float* vthr = sThr + ((1 << bits_v) - bits_v - 1);
+  uint2* tb = reinterpret_cast<uint2*>(vstage + v_words);   // per block: {gain bits, width | offset << 8}
   const uint32_t* myrow = rows + lane * Row::kPitch;
+  const bool writer = lane == 0;
+  float t3[7];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) t3[i] = sThr[(1 << 3) - 3 - 1 + i];   // width-3 thresholds
   int cur_h = -1;
 
   for (long long task = static_cast<long long>(blockIdx.x) * kQuantWarps + warp; task < n_tasks;
@@ -161,11 +215,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
     if (al->k_words != k_words) continue;      // allocation made for another budget: write nothing
     if (h != cur_h) {
       __syncwarp();
-      for (int i = lane; i < kH; i += 32) {
-        tw[i] = al->width[i];
-        tg[i] = al->gain[i];
-        to[i] = al->word_off[i];
-      }
+      for (int i = lane; i < kH; i += 32)
+        tb[i] = make_uint2(__float_as_uint(al->gain[i]), static_cast<uint32_t>(al->width[i]) |
+                                                             (static_cast<uint32_t>(al->word_off[i]) << 8));
       cur_h = h;
     }
     const int t0 = tile * kTile;
@@ -179,19 +231,20 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
     __half kn16, vn16;
     float a;
     row_norm_scale<DT>(myrow, kn16, a);
-#pragma unroll 1
+    if (!valid) a = __int_as_float(0x7fc00000);   // NaN: every comparison false, so all code bits are 0
+#pragma unroll 2
     for (int bp = 0; bp < kH / 2; ++bp) {
       const float2 lo = Row::pair(myrow, bp);             // dims 2bp, 2bp+1
       const float2 hi = Row::pair(myrow, kH / 2 + bp);    // dims 64+2bp, 65+2bp
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int blk = 2 * bp + u;
-        const int w = tw[blk];
+        const uint2 e = tb[2 * bp + u];
+        const int w = e.y & 0xffu;
         if (w == 0) continue;
-        const float g = tg[blk];
+        const float g = __uint_as_float(e.x);
         const float y1 = __fmul_rn(__fmul_rn(u ? lo.y : lo.x, a), g);
         const float y2 = __fmul_rn(__fmul_rn(u ? hi.y : hi.x, a), g);
-        search_ballot2(y1, y2, w, sThr + ((1 << w) - w - 1), valid, stage + to[blk], 2, 1, lane);
+        search_ballot2_any(w, y1, y2, sThr, t3, stage + (e.y >> 8), 2, writer);
       }
     }
 
@@ -200,10 +253,16 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
     Row::load(rows, V + b * vsb + h * vsh + static_cast<int64_t>(t0) * vst, vst, valid_rows, lane);
     __syncwarp();
     row_norm_scale<DT>(myrow, vn16, a);
-#pragma unroll 2
-    for (int i = 0; i < kD / 2; ++i) {
-      const float2 x = Row::pair(myrow, i);
-      search_ballot2(__fmul_rn(x.x, a), __fmul_rn(x.y, a), bits_v, vthr, valid, vstage + 2 * i, kD, 1, lane);
+    if (!valid) a = __int_as_float(0x7fc00000);
+    switch (bits_v) {
+      case 1: quant_values<DT, 1>(myrow, a, sThr, vstage, writer); break;
+      case 2: quant_values<DT, 2>(myrow, a, sThr, vstage, writer); break;
+      case 3: quant_values<DT, 3>(myrow, a, sThr, vstage, writer); break;
+      case 4: quant_values<DT, 4>(myrow, a, sThr, vstage, writer); break;
+      case 5: quant_values<DT, 5>(myrow, a, sThr, vstage, writer); break;
+      case 6: quant_values<DT, 6>(myrow, a, sThr, vstage, writer); break;
+      case 7: quant_values<DT, 7>(myrow, a, sThr, vstage, writer); break;
+      default: quant_values<DT, 8>(myrow, a, sThr, vstage, writer); break;
     }
     __syncwarp();
 

@@ -234,7 +234,7 @@ def kvq_calibrate(K, bits_k: int, w_max: int = 8, n_calib: int = 0, mode: int = 
     if alloc is None:
         alloc = _empty_bytes(kvq_alloc_bytes(H), K.device)
     if ws is None:
-        ws = _empty_bytes(kvq_calibrate_workspace_bytes(B, H, n), K.device)
+        ws = _torch().zeros(kvq_calibrate_workspace_bytes(B, H, n), dtype=_torch().uint8, device=K.device)
     kd = tensor4(K)
     p = CalibParams(bits_k, w_max, n_calib, mode)
     _check("kvq_calibrate", lib().kvq_calibrate(K.data_ptr(), ctypes.byref(kd), ctypes.byref(p), alloc.data_ptr(),
