@@ -214,6 +214,30 @@ kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V,
 kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, int capacity,
                                int seq_len, float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- allocation-free decode */
+
+/* Decode attention for callers that cannot allocate device memory. No counterpart on the
+ * pages: it is a convenience of this library. Some hosts give the library only their
+ * input and output buffers and have no device allocator of their own (a plain-C host that
+ * links no CUDA memory manager, an engine plugin whose interface forbids allocating on the
+ * hot path), so they cannot supply the workspace kvq_decode_attn takes. This call computes
+ * exactly what kvq_decode_attn computes (same arguments, without ws / ws_bytes) and uses as
+ * its workspace a fixed scratch array of kvq_decode_noalloc_scratch_bytes() bytes (2 MiB)
+ * that the library holds in device memory on every GPU that loads it, until the process
+ * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
+ * - The first call on a device looks up the array's address and zeroes it (synchronous);
+ *   make that first call before any stream capture.
+ * - Shapes whose decode workspace (kvq_decode_workspace_bytes) exceeds the array return
+ *   KVQ_ERR_WORKSPACE before anything is launched.
+ * - Every call on a device shares the one array, which keeps the last call's contents; the
+ *   split counters in it that must start at zero are returned to zero by every call. Calls
+ *   that overlap on the GPU (other streams, other host threads) race on it: serialize them. */
+kvq_status kvq_decode_attn_noalloc(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
+                                   const kvq_cache_desc* cache, int seq_len, float* out, void* stream);
+
+/* Size in bytes of the scratch array kvq_decode_attn_noalloc uses (2 MiB). */
+size_t kvq_decode_noalloc_scratch_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -445,3 +445,60 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Decode attention for callers that cannot allocate device memory.
+//
+// Some hosts of this library hand it only their input and output buffers and own no device
+// allocator of their own: a plain-C host that never links a CUDA memory manager, or an
+// inference-engine plugin whose interface forbids allocating on the hot path. They cannot
+// provide the split-merge workspace kvq_decode_attn needs. This entry point uses a fixed
+// scratch array instead: a file-scope __device__ array that every GPU loading the library
+// holds until the process exits. Its device address is looked up once per device (with that
+// device current) and handed to the ordinary decode kernel as its workspace.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 2u << 20;   // 2 MiB per device
+__device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. The first call on a device
+// resolves it with cudaGetSymbolAddress and zeroes the array (the split tickets in it must
+// start at zero; the kernel returns them to zero after every call).
+kvq_status decode_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return KVQ_ERR_CUDA;
+    if (cudaMemset(p, 0, kNoAllocScratchBytes) != cudaSuccess) return KVQ_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_decode_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+kvq_status kvq_decode_attn_noalloc(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
+                                   const kvq_cache_desc* cache, int seq_len, float* out, void* stream) {
+  if (!qd || !cache_ok(cache)) return KVQ_ERR_ARG;
+  const size_t need = kvq_decode_workspace_bytes(cache, qd->n_heads);
+  if (need == 0) return KVQ_ERR_ARG;
+  if (need > kNoAllocScratchBytes) return KVQ_ERR_WORKSPACE;
+  kvq_status st = ensure_tables();
+  if (st != KVQ_OK) return st;
+  void* scratch = nullptr;
+  if ((st = decode_scratch(&scratch)) != KVQ_OK) return st;
+  return kvq_decode_attn(q, qd, packed, alloc, cache, seq_len, out, scratch, kNoAllocScratchBytes, stream);
+}
+
+}  // extern "C"
+

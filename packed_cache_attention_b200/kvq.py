@@ -80,6 +80,8 @@ _SIGNATURES = {
     "kvq_nf4_decode_workspace_bytes": ([_I, _I, _I, _I], _SZ),
     "kvq_nf4_quantize": ([_VP, _P4, _VP, _P4, _I, _VP, _VP], _I),
     "kvq_nf4_decode_attn": ([_VP, _P4, _VP, _I, _I, _VP, _VP, _SZ, _VP], _I),
+    "kvq_decode_attn_noalloc": ([_VP, _P4, _VP, _VP, _PC, _I, _VP, _VP], _I),
+    "kvq_decode_noalloc_scratch_bytes": ([], _SZ),
 }
 
 _lib = None
@@ -266,6 +268,24 @@ def kvq_decode_attn(q, packed, alloc, cache: CacheDesc, seq_len: int, out=None, 
                                                     alloc.data_ptr(), ctypes.byref(cache), seq_len, out.data_ptr(),
                                                     ws.data_ptr(), ws.numel(), _stream(stream)))
     return out
+
+
+def kvq_decode_attn_noalloc(q, packed, alloc, cache: CacheDesc, seq_len: int, out=None, stream=None):
+    """Decode attention without a caller workspace: the library's fixed device scratch array
+    serves as the split-merge workspace (calls on one device must not overlap)."""
+    torch = _torch()
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    qd = tensor4(q)
+    _check("kvq_decode_attn_noalloc", lib().kvq_decode_attn_noalloc(q.data_ptr(), ctypes.byref(qd), packed.data_ptr(),
+                                                                    alloc.data_ptr(), ctypes.byref(cache), seq_len,
+                                                                    out.data_ptr(), _stream(stream)))
+    return out
+
+
+def kvq_decode_noalloc_scratch_bytes() -> int:
+    return lib().kvq_decode_noalloc_scratch_bytes()
 
 
 def kvq_nf4_quantize(K, V, capacity: int | None = None, packed=None, stream=None):
