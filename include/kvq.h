@@ -154,8 +154,8 @@ kvq_status kvq_workspace_status(const void* ws, void* stream, int* device_code);
 
 /* ---------------------------------------------------------------- Block-GTQ hot path */
 
-/* Calibration ([BGTQ]: "for each layer and KV head, a label-free energy score for each
- * RoPE block, then greedily allocates integer bit widths by marginal gain").
+/* Calibration ([BGTQ] abstract: per layer and KV head, a label-free energy score for every
+ * RoPE block, then a greedy integer bit allocation by marginal gain).
  * K: keys [batch][n_kv_heads][seq_len][128] in kd->dtype (post-RoPE, as cached).
  * Two launches: a fixed-order fp64 reduction of E_b = mean_t (k_b^2 + k_{b+64}^2) over the
  * first n_calib tokens of every sequence (pooled), then the greedy allocation:

@@ -1,11 +1,12 @@
 """Block-GTQ on a TQ-MSE-style scalar quantizer: the oracle. TEST INFRASTRUCTURE ONLY.
 
-Source: "RoPE-aware bit allocation for KV cache quantization" (Liang, Zhang,
-Jia; arXiv 2606.24033), abstract: for each layer and KV head, a label-free
-energy score per RoPE block, then a greedy integer bit allocation by marginal
-gain, on top of TurboQuant-MSE; matched K/V bit budgets (K2V2, K3V3, ...);
-"uniform TQ-MSE" as the baseline allocation; a packed-cache serving path that
-runs attention on the packed cache.
+Source: page "RoPE-aware bit allocation for KV cache quantization" (Liang,
+Zhang, Jia; arXiv 2606.24033), abstract. As summarised there: per layer and KV
+head an energy score is computed for each RoPE block without labels, and
+integer bit widths are then handed out greedily by marginal gain; the
+allocator sits on TurboQuant-MSE; K and V get matched budgets (K2V2, K3V3, ...);
+the baseline gives every coordinate the same width (uniform TQ-MSE); attention
+is served straight from a packed cache.
 
 The page names these steps without defining them. The readings taken here
 (each restated in the function that uses it):

@@ -12,9 +12,9 @@ Normal Distribution Characteristics" (arXiv 2505.16210):
   * Figs. 6-7: padding with zeros is done during computation.
 
 Readings: blocks run along each token's head-major hidden vector (the
-review's "Core claim" sentence says "along the token dimension"; the figure
-captions and the mechanism paragraph put them along the hidden dimension,
-which is what is followed). Scale s = fp16(absmax of the block); u = fp32(x) /
+review's core-claim paragraph puts the blocks on the token axis; the figure
+captions and the mechanism paragraph put them on the hidden axis, which is
+what is followed). Scale s = fp16(absmax of the block); u = fp32(x) /
 fp32(s) (u = 0 when s = 0); index = #{NF4 midpoints strictly below u}.
 Padded tokens hold index 0 and scale 0 and are masked out of the softmax.
 Storage per (sequence, block): codes[T_pad][128 bytes] with value 2k in the

@@ -1,8 +1,8 @@
 """RoPE block decomposition — the premise of Block-GTQ. TEST INFRASTRUCTURE ONLY.
 
-"RoPE-aware bit allocation for KV cache quantization", abstract: under RoPE a
-key's contribution to a future attention logit is a position-dependent sum
-over two-dimensional frequency blocks. Reading (rotate-half pairing): block i
+Page "RoPE-aware bit allocation for KV cache quantization", abstract: with
+RoPE, the logit a cached key later produces splits into one term per 2-D
+frequency block, each depending on the position gap. Reading (rotate-half pairing): block i
 holds dims (i, i + h), h = d/2, and rotates by angle p * theta_i with
 theta_i = base^(-2i/d).
 """

@@ -1,7 +1,6 @@
 // Calibration kernels: the label-free energy score per RoPE block and the greedy integer
-// bit allocation by marginal gain ("RoPE-aware bit allocation for KV cache quantization",
-// abstract: "for each layer and KV head, Block-GTQ computes a label-free energy score for
-// each RoPE block and greedily allocates integer bit widths by marginal gain").
+// bit allocation by marginal gain, computed per layer and KV head (page "RoPE-aware bit
+// allocation for KV cache quantization", abstract).
 #pragma once
 
 #include "common.cuh"

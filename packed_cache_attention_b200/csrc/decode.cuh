@@ -1,6 +1,6 @@
-// Fused decode attention read straight from the packed Block-GTQ cache ("RoPE-aware bit
-// allocation for KV cache quantization", abstract: "packed-cache serving path"; the NQKV
-// review's editorial extension: fuse the table lookup into the attention kernel).
+// Fused decode attention read straight from the packed Block-GTQ cache (page "RoPE-aware bit
+// allocation for KV cache quantization", abstract: attention served from the packed cache;
+// the NQKV review's editorial extensions propose folding the table lookup into attention).
 //
 // Grid: (splits, batch * n_kv_heads); 4 warps per CTA; each CTA owns a contiguous range of
 // 32-token tiles of one (sequence, KV head) and each warp every 4th tile of that range.

@@ -1,6 +1,6 @@
 // Quantize + pack: TQ-MSE-style scalar quantizer with Block-GTQ widths for K and a uniform
-// width for V ("RoPE-aware bit allocation for KV cache quantization", abstract: Block-GTQ
-// is "built on TurboQuant-MSE", "matched K/V bit budgets", "packed K3V3").
+// width for V (page "RoPE-aware bit allocation for KV cache quantization", abstract: the
+// allocator sits on TurboQuant-MSE, K and V get matched bit budgets, the cache is packed).
 //
 // One warp per 32-token tile of one (sequence, KV head) at a time (persistent warps);
 // lane t quantizes token t of the tile. For a token row x (128 values):

@@ -6,10 +6,10 @@ arithmetic (no energy, allocation, quantizer, packing or attention). Both the
 CUDA path and the CPU oracle consume exactly the tensors built here.
 
 RoPE is applied here because the cache stores post-RoPE keys: the decode
-query and the cached keys come out of the model already rotated
-("RoPE-aware bit allocation for KV cache quantization", abstract: a key's
-contribution to a future logit is a sum over 2-D frequency blocks). The
-pairing is rotate-half: block i = dims (i, i + d/2), angle p * base^(-2i/d).
+query and the cached keys come out of the model already rotated (page
+"RoPE-aware bit allocation for KV cache quantization", abstract: under RoPE a
+key's share of a later logit splits over 2-D frequency blocks). The pairing is
+rotate-half: block i = dims (i, i + d/2), angle p * base^(-2i/d).
 
 Workloads (all seeded; synthetic stand-ins for the pages' models):
   tiny        1 KV head, 1 q head, d 128, T 512, fp32. sigma_b = 10^U(-1,1)
