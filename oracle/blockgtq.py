@@ -20,7 +20,7 @@ The page names these steps without defining them. The readings taken here
   gain       g_b = sqrt(2 sum(E) / (d E_b)) (unit variance per coordinate of
              block b after the global sqrt(d)/||k|| scaling), 1 if E_b = 0;
              f_b = 1 / (sqrt(d) g_b) is the matching dequant factor.
-  quantizer  per token row: fp16 norm of the row, a = sqrt(d)/norm in fp32,
+  quantizer  per token row: fp16 norm of the row (fp32 sum of squares), a = sqrt(d)/norm in fp32,
              y = (x * a) * g_b in fp32, code = #{thresholds strictly below y}
              of the width-w_b Lloyd-Max codebook. Values use width bits_v, g = 1.
   layout     32-token tiles; bit planes transposed so that each 32-bit word
@@ -154,17 +154,18 @@ def calibrate(K: np.ndarray, bits_k: int, n_calib: int = 0, w_max: int = 8, mode
 # --------------------------------------------------------------------------- quantizer
 
 def row_norms_f16(X: np.ndarray) -> np.ndarray:
-    """fp16 norm of every row: fp16(sqrt(s2)), s2 = sum of x_j^2 left to right in fp64."""
-    X = np.asarray(X, dtype=np.float64)
-    s2 = np.add.accumulate(X * X, axis=-1)[..., -1]
-    return np.sqrt(s2).astype(np.float16)
+    """fp16 norm of every row: fp16(fp32 sqrt(s2)), s2 = sum of x_j^2 left to right in fp32,
+    each step fl32(s2 + fl32(x_j * x_j)) (the square is exact for 16-bit inputs)."""
+    X32 = np.asarray(X, dtype=np.float32)
+    s2 = np.add.accumulate((X32 * X32).astype(np.float32), axis=-1, dtype=np.float32)[..., -1]
+    return np.sqrt(s2).astype(np.float32).astype(np.float16)
 
 
 def quantize_rows(X: np.ndarray, widths_dim: np.ndarray, gains_dim: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     """TQ-MSE-style scalar quantizer for rows X[..., d].
 
     X holds exactly the stored values (converted to fp32 exactly).
-    norm = fp16 norm; a = fp32(sqrt(d)) / fp32(norm) (a = 0 when norm = 0);
+    norm = row_norms_f16; a = fp32(sqrt(d)) / fp32(norm) (a = 0 when norm = 0);
     y_j = fp32(fp32(x_j * a) * g_j); code_j = #{thresholds of width w_j strictly
     below y_j} (0 where w_j = 0). Returns (codes uint8 [..., d], norms fp16 [...]).
     """

@@ -5,7 +5,7 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
-#include "../../include/kvq.h"
+#include "kvq.h"
 #include "tables.h"
 
 namespace kvq {

@@ -28,6 +28,7 @@ constexpr int kDecWarps = 16;
 constexpr int kDecStages = 3;        // deepest cp.async pipeline per warp (fewer when records are large)
 constexpr int kMaxSteps = 32;
 constexpr int kMaxMergeSplits = 160;
+constexpr int kMergeGroup = 8;      // splits merged by the last CTA of each group (first level)
 constexpr int kTargetCtas = 148;   // 1 CTA of 16 warps per SM on a 148-SM B200
 
 struct DecodeSmem {
@@ -43,8 +44,9 @@ struct DecodeSmem {
   uint32_t step_info[kMaxSteps][4];  // per step and lane c: width | K word offset of its block << 8
   int n_steps;
   int last;
-  float mw[8][kMaxMergeSplits];     // cross-split merge: weight 2^(m_s - M) per head and split
+  float mw[8][kMaxMergeSplits];     // cross-split merge: weight 2^(m_s - M) per head and member
   float Lsum[8];
+  float Mmax[8];
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -150,11 +152,77 @@ __device__ __forceinline__ void decode_load_tile(uint8_t* dst, const uint8_t* sr
   for (int k = lane; k < rec_bytes / 16; k += 32) cp_async16(dst + 16 * k, src + 16 * k);
 }
 
+// Merge n (m, l, O) partials, entries first..first+n-1 of row `bh` (row pitch `pitch` entries,
+// 8 head rows per entry), in entry order: M = max m, L = sum l 2^(m - M),
+// O = sum O 2^(m - M). Writes either the merged partial to entry `dst` or, when `out` is
+// non-null, out = O / L for the G real heads. Needs all 512 threads of the CTA.
+__device__ __forceinline__ void merge_partials(DecodeSmem& S, uint8_t* scratch, int bh, int pitch, int first, int n,
+                                               float* part_m, float* part_l, float* part_o, int dst, float* out,
+                                               int G) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int hg = warp; hg < 8; hg += kDecWarps) {
+    const size_t p0 = (static_cast<size_t>(bh) * pitch + first) * 8 + hg;
+    float M = -INFINITY;
+    for (int s = lane; s < n; s += 32) M = fmaxf(M, __ldcg(part_m + p0 + static_cast<size_t>(s) * 8));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.0f;
+    for (int s = lane; s < n; s += 32) {
+      const size_t pi = p0 + static_cast<size_t>(s) * 8;
+      const float ms = __ldcg(part_m + pi);
+      const float wt = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
+      S.mw[hg][s] = wt;
+      L += __ldcg(part_l + pi) * wt;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) {
+      S.Lsum[hg] = L;
+      S.Mmax[hg] = M;
+    }
+  }
+  __syncthreads();
+  // O: 256 (head, 4-dim) quads, two threads each over the two halves of the members
+  const int quad = tid & 255, half = tid >> 8;
+  const int hg = quad >> 5, j4 = quad & 31;
+  const int s_mid = n / 2;
+  const int s0 = half ? s_mid : 0, s1 = half ? n : s_mid;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* po = reinterpret_cast<const float4*>(part_o);
+#pragma unroll 4
+  for (int s = s0; s < s1; ++s) {
+    const float wt = S.mw[hg][s];
+    const float4 v = __ldcg(po + ((static_cast<size_t>(bh) * pitch + first + s) * 8 + hg) * (kD / 4) + j4);
+    o.x += v.x * wt; o.y += v.y * wt; o.z += v.z * wt; o.w += v.w * wt;
+  }
+  float4* red = reinterpret_cast<float4*>(scratch);
+  if (half) red[quad] = o;
+  __syncthreads();
+  if (!half) {
+    const float4 v = red[quad];
+    o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+    if (out != nullptr) {
+      if (hg < G) {
+        const float inv = 1.0f / S.Lsum[hg];
+        reinterpret_cast<float4*>(out + static_cast<size_t>(hg) * kD)[j4] =
+            make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      }
+    } else {
+      const size_t pd = (static_cast<size_t>(bh) * pitch + dst) * 8 + hg;
+      reinterpret_cast<float4*>(part_o + pd * kD)[j4] = o;
+      if (j4 == 0) {
+        part_m[pd] = S.Mmax[hg];
+        part_l[pd] = S.Lsum[hg];
+      }
+    }
+  }
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
     const typename Elem<DT>::T* __restrict__ q, int64_t qsb, int64_t qsh, int n_q_heads, int n_kv_heads,
     const uint8_t* __restrict__ packed, const kvq_head_alloc* __restrict__ alloc, int tiles_cap,
-    int rec_bytes, int bits_v, int seq_len, int splits, int n_stages, float* __restrict__ out,
+    int rec_bytes, int bits_v, int seq_len, int splits, int n_groups, int n_stages, float* __restrict__ out,
     float* __restrict__ part_m, float* __restrict__ part_l, float* __restrict__ part_o,
     unsigned* __restrict__ tickets) {
   extern __shared__ __align__(16) uint8_t dsmem[];
@@ -393,7 +461,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
     if (splits == 1) {
       if (hg < G) out[(static_cast<size_t>(b) * n_q_heads + hkv * G + hg) * kD + j] = O / L;
     } else {
-      const size_t pb = (static_cast<size_t>(bh) * splits + split) * 8 + hg;
+      const size_t pb = (static_cast<size_t>(bh) * (splits + n_groups) + split) * 8 + hg;
       part_o[pb * kD + j] = O;
       if (j == 0) {
         part_m[pb] = M;
@@ -404,61 +472,39 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
   if (splits == 1) return;
 
   // ------------------------------------------------------------------ cross-split merge
+  // Two levels: the last CTA of each group of kMergeGroup splits merges its group into a
+  // group partial (entry splits + group); the last group merges the group partials.
+  const int pitch = splits + n_groups;
+  const int grp = split / kMergeGroup;
+  const int g0 = grp * kMergeGroup, gn = min(splits, g0 + kMergeGroup) - g0;
+  float* out_bh = out + (static_cast<size_t>(b) * n_q_heads + hkv * G) * kD;
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const unsigned ticket = atomicAdd(&tickets[bh], 1u);
-    S.last = (ticket == static_cast<unsigned>(splits - 1));
+    unsigned* gt = tickets + gridDim.y + static_cast<size_t>(bh) * n_groups + grp;
+    const unsigned t = atomicAdd(gt, 1u);
+    S.last = (t == static_cast<unsigned>(gn - 1));
+    if (S.last) *gt = 0u;
   }
   __syncthreads();
   if (!S.last) return;
   __threadfence();
-  // weights 2^(m_s - M) per (head, split) and the merged denominators, one warp per head
-  for (int hg = warp; hg < 8; hg += kDecWarps) {
-    const size_t p0 = static_cast<size_t>(bh) * splits * 8 + hg;
-    float M = -INFINITY;
-    for (int s = lane; s < splits; s += 32) M = fmaxf(M, __ldcg(part_m + p0 + static_cast<size_t>(s) * 8));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.0f;
-    for (int s = lane; s < splits; s += 32) {
-      const size_t pi = p0 + static_cast<size_t>(s) * 8;
-      const float ms = __ldcg(part_m + pi);
-      const float wt = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-      S.mw[hg][s] = wt;
-      L += __ldcg(part_l + pi) * wt;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) S.Lsum[hg] = L;
+  if (n_groups == 1) {
+    merge_partials(S, stages, bh, pitch, 0, splits, part_m, part_l, part_o, 0, out_bh, G);
+    return;
+  }
+  merge_partials(S, stages, bh, pitch, g0, gn, part_m, part_l, part_o, splits + grp, nullptr, G);
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned t = atomicAdd(&tickets[bh], 1u);
+    S.last = (t == static_cast<unsigned>(n_groups - 1));
+    if (S.last) tickets[bh] = 0u;
   }
   __syncthreads();
-  // O: 256 (head, 4-dim) quads, two threads each over the two halves of the splits
-  {
-    const int quad = tid & 255, half = tid >> 8;
-    const int hg = quad >> 5, j4 = (quad & 31) * 4;
-    const int s_mid = splits / 2;
-    const int s0 = half ? s_mid : 0, s1 = half ? splits : s_mid;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4* po = reinterpret_cast<const float4*>(part_o);
-#pragma unroll 8
-    for (int s = s0; s < s1; ++s) {
-      const float wt = S.mw[hg][s];
-      const float4 v = __ldcg(po + ((static_cast<size_t>(bh) * splits + s) * 8 + hg) * (kD / 4) + j4 / 4);
-      o.x += v.x * wt; o.y += v.y * wt; o.z += v.z * wt; o.w += v.w * wt;
-    }
-    float4* red = reinterpret_cast<float4*>(stages);
-    if (half) red[quad] = o;
-    __syncthreads();
-    if (!half && hg < G) {
-      const float4 v = red[quad];
-      const float inv = 1.0f / S.Lsum[hg];
-      float4 r;
-      r.x = (o.x + v.x) * inv; r.y = (o.y + v.y) * inv; r.z = (o.z + v.z) * inv; r.w = (o.w + v.w) * inv;
-      reinterpret_cast<float4*>(out + (static_cast<size_t>(b) * n_q_heads + hkv * G + hg) * kD)[j4 / 4] = r;
-    }
-  }
-  if (tid == 0) tickets[bh] = 0u;
+  if (!S.last) return;
+  __threadfence();
+  merge_partials(S, stages, bh, pitch, splits, n_groups, part_m, part_l, part_o, 0, out_bh, G);
 }
 
 }  // namespace kvq

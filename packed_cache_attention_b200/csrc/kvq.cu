@@ -82,14 +82,23 @@ struct DecodeWs {
   size_t tickets, part_m, part_l, part_o, total;
 };
 
-DecodeWs decode_ws_layout(int bh, int splits, int rows) {
+// Workspace of the decode kernels: tickets (per row: one final counter, then one counter per
+// merge group), then (m, l, O) partials for `entries` entries per row.
+DecodeWs decode_ws_layout(int bh, int entries, int rows, int groups) {
   DecodeWs w;
   w.tickets = sizeof(WsHeader);
-  w.part_m = align_up(w.tickets + 4ull * bh, 128);
-  w.part_l = align_up(w.part_m + 4ull * bh * splits * rows, 128);
-  w.part_o = align_up(w.part_l + 4ull * bh * splits * rows, 128);
-  w.total = align_up(w.part_o + 4ull * bh * splits * rows * kD, 128);
+  w.part_m = align_up(w.tickets + 4ull * bh * (1 + groups), 128);
+  w.part_l = align_up(w.part_m + 4ull * bh * entries * rows, 128);
+  w.part_o = align_up(w.part_l + 4ull * bh * entries * rows, 128);
+  w.total = align_up(w.part_o + 4ull * bh * entries * rows * kD, 128);
   return w;
+}
+
+int merge_groups(int splits) { return (splits + kMergeGroup - 1) / kMergeGroup; }
+
+DecodeWs gtq_ws_layout(int bh, int splits) {
+  const int groups = merge_groups(splits);
+  return decode_ws_layout(bh, splits + groups, 8, groups);
 }
 
 int sm_count() {
@@ -214,7 +223,7 @@ size_t kvq_packed_bytes(const kvq_cache_desc* c) {
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* c, int n_q_heads) {
   if (!cache_ok(c) || n_q_heads < 1) return 0;
   const int bh = c->batch * c->n_kv_heads;
-  return decode_ws_layout(bh, decode_splits(bh, n_tiles_of(c->capacity)), 8).total;
+  return gtq_ws_layout(bh, decode_splits(bh, n_tiles_of(c->capacity))).total;
 }
 
 kvq_status kvq_init(void) { return ensure_tables(); }
@@ -334,7 +343,7 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
   const int bh = c->batch * c->n_kv_heads;
   const int n_tiles = n_tiles_of(seq_len);
   const int splits = decode_splits(bh, n_tiles);
-  const DecodeWs L = decode_ws_layout(bh, splits, 8);
+  const DecodeWs L = gtq_ws_layout(bh, splits);
   if (!ws || ws_bytes < L.total || !aligned16(ws) || ws_bytes < kvq_decode_workspace_bytes(c, qd->n_heads))
     return KVQ_ERR_WORKSPACE;
   if ((st = ensure_tables()) != KVQ_OK) return st;
@@ -352,7 +361,8 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
     kern<<<grid, kDecWarps * 32, smem, s>>>(                                                                          \
         static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, c->n_kv_heads,                             \
         static_cast<const uint8_t*>(packed), static_cast<const kvq_head_alloc*>(alloc), n_tiles_of(c->capacity), rec, \
-        c->bits_v, seq_len, splits, decode_stages(rec), out, reinterpret_cast<float*>(w8 + L.part_m),                                    \
+        c->bits_v, seq_len, splits, merge_groups(splits), decode_stages(rec), out,                                    \
+        reinterpret_cast<float*>(w8 + L.part_m),                                    \
         reinterpret_cast<float*>(w8 + L.part_l), reinterpret_cast<float*>(w8 + L.part_o),                             \
         reinterpret_cast<unsigned*>(w8 + L.tickets));                                                                 \
   } while (0)
@@ -374,7 +384,7 @@ size_t kvq_nf4_packed_bytes(int batch, int n_heads, int capacity, int head_dim) 
 size_t kvq_nf4_decode_workspace_bytes(int batch, int n_heads, int capacity, int head_dim) {
   if (batch < 1 || n_heads < 1 || capacity < 1 || head_dim != kD) return 0;
   const int bh = batch * n_heads;
-  return decode_ws_layout(bh, decode_splits(bh, (capacity + 31) / 32), 1).total;
+  return decode_ws_layout(bh, decode_splits(bh, (capacity + 31) / 32), 1, 0).total;
 }
 
 kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, int capacity,
@@ -421,7 +431,7 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
   if (seq_len < 1 || seq_len > capacity) return KVQ_ERR_RANGE;
   const int bh = qd->batch * qd->n_heads;
   const int splits = decode_splits(bh, (seq_len + 31) / 32);
-  const DecodeWs Lw = decode_ws_layout(bh, splits, 1);
+  const DecodeWs Lw = decode_ws_layout(bh, splits, 1, 0);
   if (!ws || ws_bytes < Lw.total || !aligned16(ws) ||
       ws_bytes < kvq_nf4_decode_workspace_bytes(qd->batch, qd->n_heads, capacity, kD))
     return KVQ_ERR_WORKSPACE;

@@ -4,8 +4,8 @@
 //
 // One warp per 32-token tile of one (sequence, KV head) at a time (persistent warps);
 // lane t quantizes token t of the tile. For a token row x (128 values):
-//   s2   = sum_j x_j^2 in fp64, j ascending (exact products, rounded sums)
-//   norm = fp16(sqrt(s2)) (round to nearest even)
+//   s2   = sum_j x_j^2 in fp32, j ascending: fl32(s2 + fl32(x_j x_j))
+//   norm = fp16(fp32 sqrt(s2)) (round to nearest even)
 //   a    = fp32(sqrt(128)) / fp32(norm), 0 if norm == 0
 //   y_j  = fp32(fp32(x_j a) g_b)            (V: g = 1, the multiply is skipped as exact)
 //   code = #{thresholds of width w_b strictly below y_j}
@@ -14,15 +14,13 @@
 // token t) is directly the tile's bit-plane word for that dim and plane.
 // The tile is first copied into shared memory with a padded row pitch (65 words for 16-bit
 // inputs), so that the 32 lanes reading the same dim of their own rows hit 32 banks.
-// Ballot words are staged in shared memory; a last pass permutes them into the tile layout
-// and writes whole lines:
-//   K, per block b (ascending, w_b > 0), per plane p: two words built from the ballots
-//      A (dim b) and B (dim b+64): word0 = lo nibbles of A's bytes | lo nibbles of B's bytes
-//      << 4, word1 = hi nibbles of A | hi nibbles of B. Bit s+4m of word H then holds token
-//      4H + s + 8(m/2) at dim b (m even) or b+64 (m odd).
-//   V, per plane p, per dim j: the ballot word with each byte's bits unzipped (even bits
-//      to the low nibble, odd bits to the high nibble): bit c+4m holds token
-//      8(m/2) + 2c + (m%2).
+// K: lane t works on token t. The ballot words are staged in shared memory and a last pass
+//   turns each pair into the tile layout and writes whole lines. Per block b (ascending,
+//   w_b > 0) and plane p, the ballots A (dim b) and B (dim b+64) give word0 = lo nibbles of
+//   A's bytes | lo nibbles of B's bytes << 4 and word1 = hi nibbles of A | hi nibbles of B.
+//   Bit s+4m of word H then holds token 4H + s + 8(m/2) at dim b (m even) or b+64 (m odd).
+// V: lane l = c + 4m works on token 8(m/2) + 2c + (m%2), so a ballot is already the layout's
+//   word (bit c+4m holds that token) and lane 0 stores each pair of words directly.
 #pragma once
 
 #include "common.cuh"
@@ -40,14 +38,20 @@ template <int DT> struct QuantRow16 {
   __device__ __forceinline__ static void load(uint32_t* dst, const void* src, int64_t row_stride, int valid_rows,
                                               int lane) {
     const uint8_t* s8 = static_cast<const uint8_t*>(src);
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
+    uint4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {             // all 16 loads in flight before any store
       const int idx = i * 32 + lane;           // 16-byte chunk of the tile
       const int r = idx >> 4, c = idx & 15;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (r < valid_rows) v = __ldg(reinterpret_cast<const uint4*>(s8 + (static_cast<int64_t>(r) * row_stride * 2)) + c);
+      v[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (r < valid_rows) v[i] = __ldg(reinterpret_cast<const uint4*>(s8 + (static_cast<int64_t>(r) * row_stride * 2)) + c);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int idx = i * 32 + lane;
+      const int r = idx >> 4, c = idx & 15;
       uint32_t* d = dst + r * kPitch + 4 * c;
-      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+      d[0] = v[i].x; d[1] = v[i].y; d[2] = v[i].z; d[3] = v[i].w;
     }
   }
   // Values 2i and 2i+1 of a row.
@@ -66,14 +70,23 @@ template <> struct QuantRow<KVQ_F32> {
   __device__ __forceinline__ static void load(uint32_t* dst, const void* src, int64_t row_stride, int valid_rows,
                                               int lane) {
     const uint8_t* s8 = static_cast<const uint8_t*>(src);
-#pragma unroll 4
-    for (int i = 0; i < 32; ++i) {
-      const int idx = i * 32 + lane;
-      const int r = idx >> 5, c = idx & 31;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (r < valid_rows) v = __ldg(reinterpret_cast<const uint4*>(s8 + (static_cast<int64_t>(r) * row_stride * 4)) + c);
-      uint32_t* d = dst + r * kPitch + 4 * c;
-      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {              // two batches of 16 loads in flight
+      uint4 v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int idx = (16 * h + i) * 32 + lane;
+        const int r = idx >> 5, c = idx & 31;
+        v[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < valid_rows) v[i] = __ldg(reinterpret_cast<const uint4*>(s8 + (static_cast<int64_t>(r) * row_stride * 4)) + c);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int idx = (16 * h + i) * 32 + lane;
+        const int r = idx >> 5, c = idx & 31;
+        uint32_t* d = dst + r * kPitch + 4 * c;
+        d[0] = v[i].x; d[1] = v[i].y; d[2] = v[i].z; d[3] = v[i].w;
+      }
     }
   }
   __device__ __forceinline__ static float2 pair(const uint32_t* row, int i) {
@@ -84,27 +97,21 @@ template <> struct QuantRow<KVQ_F32> {
 // fp16 norm of one row and the scale a = sqrt(128)/norm (0 for a zero norm).
 template <int DT>
 __device__ __forceinline__ void row_norm_scale(const uint32_t* row, __half& n16, float& a) {
-  double s2 = 0.0;
-#pragma unroll 8
+  float s2 = 0.0f;
+#pragma unroll 16
   for (int i = 0; i < kD / 2; ++i) {
     const float2 v = QuantRow<DT>::pair(row, i);
-    const double x0 = v.x, x1 = v.y;
-    s2 = __fma_rn(x0, x0, s2);      // x*x is exact in fp64, so this is fl(s2 + x^2)
-    s2 = __fma_rn(x1, x1, s2);
+    s2 = __fadd_rn(s2, __fmul_rn(v.x, v.x));
+    s2 = __fadd_rn(s2, __fmul_rn(v.y, v.y));
   }
-  n16 = __double2half(__dsqrt_rn(s2));
+  n16 = __float2half_rn(__fsqrt_rn(s2));
   const float nf = __half2float(n16);
   const float sqd = 11.313708305358887f;       // fp32(sqrt(128))
   a = (nf == 0.0f) ? 0.0f : __fdiv_rn(sqd, nf);
 }
 
-__device__ __forceinline__ uint32_t unzip_bytes(uint32_t x) {
-  uint32_t t = (x ^ (x >> 1)) & 0x22222222u;
-  x ^= t ^ (t << 1);
-  t = (x ^ (x >> 2)) & 0x0c0c0c0cu;
-  x ^= t ^ (t << 2);
-  return x;
-}
+// Token handled by lane l in the values pass: l = c + 4m  ->  8(m/2) + 2c + (m%2).
+__device__ __forceinline__ int value_token(int lane) { return 8 * (lane >> 3) + 2 * (lane & 3) + ((lane >> 2) & 1); }
 
 // Binary search for two values of the same width W; the ballot of the comparison at level p
 // (bit p of the code) is written by lane 0 to out[p * pstride] (first value) and
@@ -194,12 +201,13 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k_words = bits_k * kD, v_words = bits_v * kD;
-  const int warp_words = Row::kWords + k_words + v_words + 3 * kH;
+  const int warp_words = Row::kWords + k_words + 2 * kH;
   uint32_t* rows = smem + 512 + warp * warp_words;
   uint32_t* stage = rows + Row::kWords;
-  uint32_t* vstage = stage + k_words;
-  uint2* tb = reinterpret_cast<uint2*>(vstage + v_words);   // per block: {gain bits, width | offset << 8}
+  uint2* tb = reinterpret_cast<uint2*>(stage + k_words);   // per block: {gain bits, width | offset << 8}
   const uint32_t* myrow = rows + lane * Row::kPitch;
+  const int vtok = value_token(lane);
+  const uint32_t* myvrow = rows + vtok * Row::kPitch;
   const bool writer = lane == 0;
   float t3[7];
 #pragma unroll
@@ -249,26 +257,28 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
     }
 
     // ---------------------------------------------------------------- V (uniform width)
+    uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
+    uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
+    uint32_t* vout = kout + k_words;
+    const bool vvalid = vtok < valid_rows;
     __syncwarp();
     Row::load(rows, V + b * vsb + h * vsh + static_cast<int64_t>(t0) * vst, vst, valid_rows, lane);
     __syncwarp();
-    row_norm_scale<DT>(myrow, vn16, a);
-    if (!valid) a = __int_as_float(0x7fc00000);
+    row_norm_scale<DT>(myvrow, vn16, a);
+    if (!vvalid) a = __int_as_float(0x7fc00000);
     switch (bits_v) {
-      case 1: quant_values<DT, 1>(myrow, a, sThr, vstage, writer); break;
-      case 2: quant_values<DT, 2>(myrow, a, sThr, vstage, writer); break;
-      case 3: quant_values<DT, 3>(myrow, a, sThr, vstage, writer); break;
-      case 4: quant_values<DT, 4>(myrow, a, sThr, vstage, writer); break;
-      case 5: quant_values<DT, 5>(myrow, a, sThr, vstage, writer); break;
-      case 6: quant_values<DT, 6>(myrow, a, sThr, vstage, writer); break;
-      case 7: quant_values<DT, 7>(myrow, a, sThr, vstage, writer); break;
-      default: quant_values<DT, 8>(myrow, a, sThr, vstage, writer); break;
+      case 1: quant_values<DT, 1>(myvrow, a, sThr, vout, writer); break;
+      case 2: quant_values<DT, 2>(myvrow, a, sThr, vout, writer); break;
+      case 3: quant_values<DT, 3>(myvrow, a, sThr, vout, writer); break;
+      case 4: quant_values<DT, 4>(myvrow, a, sThr, vout, writer); break;
+      case 5: quant_values<DT, 5>(myvrow, a, sThr, vout, writer); break;
+      case 6: quant_values<DT, 6>(myvrow, a, sThr, vout, writer); break;
+      case 7: quant_values<DT, 7>(myvrow, a, sThr, vout, writer); break;
+      default: quant_values<DT, 8>(myvrow, a, sThr, vout, writer); break;
     }
     __syncwarp();
 
-    // ---------------------------------------------------------------- permute + store
-    uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
-    uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
+    // ---------------------------------------------------------------- K words: permute + store
     for (int k = lane; k < k_words / 2; k += 32) {
       const uint32_t A = stage[2 * k], B = stage[2 * k + 1];
       uint2 o;
@@ -276,22 +286,16 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
       o.y = ((A >> 4) & 0x0f0f0f0fu) | (B & 0xf0f0f0f0u);
       reinterpret_cast<uint2*>(kout)[k] = o;
     }
-    uint32_t* vout = kout + k_words;
-    for (int k = lane; k < v_words / 4; k += 32) {
-      const uint4 v = reinterpret_cast<const uint4*>(vstage)[k];
-      reinterpret_cast<uint4*>(vout)[k] = make_uint4(unzip_bytes(v.x), unzip_bytes(v.y), unzip_bytes(v.z),
-                                                     unzip_bytes(v.w));
-    }
     uint16_t* norms = reinterpret_cast<uint16_t*>(vout + v_words);
     norms[lane] = valid ? __half_as_ushort(kn16) : 0;
-    norms[kTile + lane] = valid ? __half_as_ushort(vn16) : 0;
+    norms[kTile + vtok] = vvalid ? __half_as_ushort(vn16) : 0;
   }
 }
 
 // Dynamic shared memory of kvq_quant_pack for the input type's row pitch.
 inline size_t quant_smem_bytes(int dtype, int bits_k, int bits_v) {
   const int row_words = (dtype == KVQ_F32) ? QuantRow<KVQ_F32>::kWords : QuantRow<KVQ_BF16>::kWords;
-  return 4 * (512 + static_cast<size_t>(kQuantWarps) * (row_words + (bits_k + bits_v) * kD + 3 * kH));
+  return 4 * (512 + static_cast<size_t>(kQuantWarps) * (row_words + bits_k * kD + 2 * kH));
 }
 
 }  // namespace kvq
