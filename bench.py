@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0, help="override the context length (profiling only)")
+    ap.add_argument("--no-nf4", action="store_true", help="skip the NF4-variant measurement")
     return ap.parse_args()
 
 
@@ -230,6 +231,8 @@ def run_gpu(args, rank, world, local_rank):
         e2e = {"value": world * L * B * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
+    nf4 = measure_nf4(kvq, wl, dev, stream, hbm_peak=peaks()[0]) if (rank == 0 and not args.no_nf4) else None
+
     steps = args.steps
     ms_step = total_ms / steps
     tokens = world * L * B * T
@@ -274,11 +277,52 @@ def run_gpu(args, rank, world, local_rank):
             "bytes_per_token_per_kv_head": d_bytes // (B * Hkv * T),
             "compression_vs_bf16": (2 * 2 * d) / (d_bytes / (B * Hkv * T)),
         },
+        "nf4": nf4,
         "e2e": e2e,
         "gpu_launches": steps * L * 4,
         "clocks": clocks,
     }
     return result
+
+
+def measure_nf4(kvq, wl, dev, stream, hbm_peak, iters=10):
+    """NQKV-style NF4 variant at the OPT-30B shape (one layer: B8 x 56 heads x 8192 tokens,
+    fp16), timed outside the step: quantize/pack and MHA decode, CUDA events per launch."""
+    import torch
+    W = wl.WORKLOADS["nqkv_opt30b"]
+    x = wl.make_nf4_inputs(W.batch, W.n_q_heads, W.head_dim, W.seq_len, W.dtype, seed=7, device=dev)
+    B, H, T, d = W.batch, W.n_q_heads, W.seq_len, W.head_dim
+    packed = torch.empty(kvq.kvq_nf4_packed_bytes(B, H, T, d), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    ws = torch.zeros(kvq.kvq_nf4_decode_workspace_bytes(B, H, T, d), dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(iters):
+            fn()
+        z.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(z) / iters
+
+    q_ms = timed(lambda: kvq.kvq_nf4_quantize(x["K"], x["V"], capacity=T, packed=packed, stream=stream))
+    d_ms = timed(lambda: kvq.kvq_nf4_decode_attn(x["q"], packed, T, T, out=out, ws=ws, stream=stream))
+    in_bytes = 2 * B * H * T * d * 2
+    pk_bytes = packed.numel()
+    res = {"workload": f"nqkv_opt30b: B{B} x H{H} x T{T} x d{d}, fp16, NF4 block 256",
+           "quantize": {"tokens_per_s": B * T / (q_ms * 1e-3), "launch_ms": q_ms, "bytes_per_launch": in_bytes + pk_bytes,
+                        "gb_s": (in_bytes + pk_bytes) / (q_ms * 1e-3) / 1e9},
+           "decode": {"kv_tokens_per_s": B * T / (d_ms * 1e-3), "launch_ms": d_ms, "bytes_per_launch": pk_bytes,
+                      "gb_s": pk_bytes / (d_ms * 1e-3) / 1e9},
+           "bytes_per_token_per_256_values": 130}
+    for k in ("quantize", "decode"):
+        res[k]["hbm_frac"] = res[k]["gb_s"] / hbm_peak
+    del x, packed
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------------------------------ CPU oracle

@@ -3,9 +3,27 @@
 // allocation for KV cache quantization", abstract).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace kvq {
+
+// Non-coherent global loads issued as volatile asm, so all loads of a batch are issued
+// before the arithmetic that consumes them (keeps many rows in flight per lane).
+template <typename V> __device__ __forceinline__ V ldg_stream(const void* p);
+template <> __device__ __forceinline__ uint2 ldg_stream<uint2>(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+template <> __device__ __forceinline__ float4 ldg_stream<float4>(const void* p) {
+  float4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
 
 constexpr int kCalibSegment = 64;      // chunk sums per fixed-order segment sum
 constexpr int kCalibChunksPerCta = 8;  // 16 lanes per chunk, 128 threads
@@ -30,7 +48,7 @@ struct CalibWs {
 // sums left to right; the CTA that completes the last segment of a head sums the segment
 // sums left to right and writes E_b = total / N. Counters are reset to zero for the next call.
 template <int DT>
-__global__ void __launch_bounds__(16 * kCalibChunksPerCta) kvq_calib_reduce(
+__global__ void __launch_bounds__(16 * kCalibChunksPerCta, 4) kvq_calib_reduce(
     const typename Elem<DT>::T* __restrict__ K, int n_calib, int64_t sb, int64_t sh, int64_t st, int N,
     int n_chunks, CalibWs ws) {
   using T = typename Elem<DT>::T;
@@ -45,16 +63,13 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta) kvq_calib_reduce(
     int s = u0 / n_calib;
     int t = u0 - s * n_calib;
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    auto add_row = [&](const T* row) {
+    // acc_j += fl(fl(x_j^2) + fl(y_j^2)) for the 4 dims x (blocks 4k..4k+3) and their partners y
+    auto add_vals = [&](const auto& a, const auto& b) {
       float x[4], y[4];
       if constexpr (DT == KVQ_F32) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(row + 4 * k));
-        const float4 b = __ldg(reinterpret_cast<const float4*>(row + kH + 4 * k));
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
         y[0] = b.x; y[1] = b.y; y[2] = b.z; y[3] = b.w;
       } else {
-        const uint2 a = __ldg(reinterpret_cast<const uint2*>(row + 4 * k));
-        const uint2 b = __ldg(reinterpret_cast<const uint2*>(row + kH + 4 * k));
         const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -70,11 +85,26 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta) kvq_calib_reduce(
         acc[j] = __dadd_rn(acc[j], __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)));
       }
     };
+    auto add_row = [&](const T* row) {
+      using V2 = typename std::conditional<DT == KVQ_F32, float4, uint2>::type;
+      add_vals(__ldg(reinterpret_cast<const V2*>(row + 4 * k)), __ldg(reinterpret_cast<const V2*>(row + kH + 4 * k)));
+    };
     if (n == kCalibChunk && t + kCalibChunk <= n_calib) {
-      // whole chunk inside one sequence: independent row addresses, loads pipeline freely
+      // whole chunk inside one sequence: 16 rows of loads in flight before any arithmetic
       const T* base = K + s * sb + h * sh + static_cast<int64_t>(t) * st;
-#pragma unroll 16
-      for (int i = 0; i < kCalibChunk; ++i) add_row(base + static_cast<int64_t>(i) * st);
+#pragma unroll 1
+      for (int i0 = 0; i0 < kCalibChunk; i0 += 16) {
+        using V2 = typename std::conditional<DT == KVQ_F32, float4, uint2>::type;
+        V2 va[16], vb[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const T* row = base + static_cast<int64_t>(i0 + i) * st;
+          va[i] = ldg_stream<V2>(row + 4 * k);
+          vb[i] = ldg_stream<V2>(row + kH + 4 * k);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) add_vals(va[i], vb[i]);
+      }
     } else {
       for (int i = 0; i < n; ++i) {
         add_row(K + s * sb + h * sh + static_cast<int64_t>(t) * st);
@@ -107,7 +137,7 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta) kvq_calib_reduce(
   if (threadIdx.x < kH) {
     const double* src = ws.chunk_sum + (static_cast<size_t>(h) * n_chunks) * kH + threadIdx.x;
     double acc = 0.0;
-#pragma unroll 16
+#pragma unroll 32
     for (int c = c0; c < c1; ++c) acc = __dadd_rn(acc, __ldcg(src + static_cast<size_t>(c) * kH));
     ws.seg_sum[(static_cast<size_t>(h) * n_seg + seg) * kH + threadIdx.x] = acc;
   }
@@ -144,6 +174,7 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
                                                         int mode, kvq_head_alloc* __restrict__ alloc) {
   __shared__ double sE[kH];
   __shared__ double sGain[kH * 8];
+  __shared__ long long sKey[kH * 8];
   __shared__ int sWidth[kH];
   __shared__ int sStepStart[9];
   __shared__ int sCount[9];
@@ -160,27 +191,37 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
   {
     const int b = tid >> 3, w = tid & 7;
     const bool valid = w < w_max;
-    sGain[tid] = valid ? __dmul_rn(sE[b], __dsub_rn(static_cast<double>(c_tab.delta[w]),
-                                                    static_cast<double>(c_tab.delta[w + 1])))
-                       : -1.0;
+    const double gv = valid ? __dmul_rn(sE[b], __dsub_rn(static_cast<double>(c_tab.delta[w]),
+                                                          static_cast<double>(c_tab.delta[w + 1])))
+                            : -1.0;
+    sGain[tid] = gv;
+    // valid gains are >= 0 (+0 for a zero energy); invalid entries never precede a valid one
+    sKey[tid] = valid ? __double_as_longlong(gv) : -1LL;
   }
   __syncthreads();
   if (mode == KVQ_MODE_UNIFORM) {
     if (tid < kH) sWidth[tid] = bits_k;
   } else {
-    const double gain = sGain[tid];
+    // Non-negative doubles order like their bit patterns, so the comparisons run on 64-bit
+    // integers (invalid entries hold -1.0, whose pattern is above every valid one, and are
+    // excluded separately).
+    const long long key = __double_as_longlong(sGain[tid]);
     const bool valid = (tid & 7) < w_max;
     int rank = 0;
     if (valid) {
+#pragma unroll 4
       for (int bb = 0; bb < kH; ++bb) {
         // entries of block bb preceding entry tid form a prefix of w = 0..w_max-1
         int lo = 0, hi = w_max;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          const int e = 8 * bb + mid;
-          const double ge = sGain[e];
-          if (ge > gain || (ge == gain && e < tid)) lo = mid + 1;
-          else hi = mid;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          if (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            const int e = 8 * bb + mid;
+            const long long ke = sKey[e];
+            if (ke > key || (ke == key && e < tid)) lo = mid + 1;
+            else hi = mid;
+          }
         }
         rank += lo;
       }

@@ -32,7 +32,7 @@ constexpr int kMergeGroup = 8;      // splits merged by the last CTA of each gro
 constexpr int kTargetCtas = 148;   // 1 CTA of 16 warps per SM on a 148-SM B200
 
 struct DecodeSmem {
-  uint2 qfrag[kMaxSteps][8][4];     // A fragments of Q' per k-step, head row g, lane c
+  uint4 kstep[kMaxSteps][8][4];     // per k-step, head row g, lane c: {Q' hi, Q' lo, K word offset + H, 0}
   float qp[8][kD];                  // Q' in fp32 before scaling
   float qmul[8];                    // 2^e that undoes the per-head scaling of Q'
   uint16_t cent[kCentroidCount];    // fp16 centroid bit patterns
@@ -41,7 +41,9 @@ struct DecodeSmem {
   uint16_t woff[kH];
   int8_t step_blk[kMaxSteps][4];
   uint8_t step_w[kMaxSteps];
-  uint32_t step_info[kMaxSteps][4];  // per step and lane c: width | K word offset of its block << 8
+  int cls_w[9];                      // k-steps grouped by width: width of class i,
+  int cls_begin[10];                 // first step of class i (cls_begin[n_cls] = n_steps)
+  int n_cls;
   int n_steps;
   int last;
   float mw[8][kMaxMergeSplits];     // cross-split merge: weight 2^(m_s - M) per head and member
@@ -125,14 +127,22 @@ __device__ __forceinline__ void decode8(const uint32_t* words, int stride, int s
   }
 }
 
-// One QK k-step: 4 RoPE blocks (one per lane c) x 32 tokens (4 n-tiles).
+// One QK k-step: 4 RoPE blocks (one per lane c) x 32 tokens (4 n-tiles). e = {Q' hi pair,
+// Q' lo pair, word offset of this lane's plane-0 word (block offset + half H), unused}.
 template <int W>
-__device__ __forceinline__ void qk_step(const uint32_t* kw, uint32_t info, int H, int sh, uint2 a, const DecodeSmem& S,
+__device__ __forceinline__ void qk_step(const uint32_t* kw, const uint4& e, int sh, const DecodeSmem& S,
                                         float (&acc)[4][4]) {
   uint32_t bf[4];
-  decode8<W>(kw + (info >> 8) + H, 2, sh, S, bf);
+  decode8<W>(kw + e.z, 2, sh, S, bf);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) mma_m16n8k8(acc[j], a.x, a.y, bf[j]);
+  for (int j = 0; j < 4; ++j) mma_m16n8k8(acc[j], e.x, e.y, bf[j]);
+}
+
+// All k-steps of one width class.
+template <int W>
+__device__ __forceinline__ void qk_class(const uint32_t* kw, int s0, int s1, int g, int c, int sh,
+                                         const DecodeSmem& S, float (&acc)[4][4]) {
+  for (int s = s0; s < s1; ++s) qk_step<W>(kw, S.kstep[s][g][c], sh, S, acc);
 }
 
 // O += P' V over the 16 dim n-tiles for value width W.
@@ -155,7 +165,7 @@ __device__ __forceinline__ void decode_load_tile(uint8_t* dst, const uint8_t* sr
 // Merge n (m, l, O) partials, entries first..first+n-1 of row `bh` (row pitch `pitch` entries,
 // 8 head rows per entry), in entry order: M = max m, L = sum l 2^(m - M),
 // O = sum O 2^(m - M). Writes either the merged partial to entry `dst` or, when `out` is
-// non-null, out = O / L for the G real heads. Needs all 512 threads of the CTA.
+// non-null, out = O / L for the G real heads. Needs all threads of the CTA (256 or 512).
 __device__ __forceinline__ void merge_partials(DecodeSmem& S, uint8_t* scratch, int bh, int pitch, int first, int n,
                                                float* part_m, float* part_l, float* part_o, int dst, float* out,
                                                int G) {
@@ -182,10 +192,12 @@ __device__ __forceinline__ void merge_partials(DecodeSmem& S, uint8_t* scratch, 
     }
   }
   __syncthreads();
-  // O: 256 (head, 4-dim) quads, two threads each over the two halves of the members
+  // O: 256 (head, 4-dim) quads; with 512 threads two threads share a quad (halves of the
+  // member list), with 256 threads one thread does all members.
+  const int halves = blockDim.x >> 8;
   const int quad = tid & 255, half = tid >> 8;
   const int hg = quad >> 5, j4 = quad & 31;
-  const int s_mid = n / 2;
+  const int s_mid = (halves == 2) ? n / 2 : n;
   const int s0 = half ? s_mid : 0, s1 = half ? n : s_mid;
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
   const float4* po = reinterpret_cast<const float4*>(part_o);
@@ -199,8 +211,10 @@ __device__ __forceinline__ void merge_partials(DecodeSmem& S, uint8_t* scratch, 
   if (half) red[quad] = o;
   __syncthreads();
   if (!half) {
-    const float4 v = red[quad];
-    o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+    if (halves == 2) {
+      const float4 v = red[quad];
+      o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+    }
     if (out != nullptr) {
       if (hg < G) {
         const float inv = 1.0f / S.Lsum[hg];
@@ -306,25 +320,35 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
   }
   __syncthreads();
   const int n_steps = S.n_steps;
-  for (int i = tid; i < n_steps * 4; i += blockDim.x) {
-    const int st = i >> 2, cc = i & 3;
-    int blk = S.step_blk[st][cc];
-    if (blk < 0) blk = max(static_cast<int>(S.step_blk[st][0]), 0);   // empty slot: Q' is 0 there
-    const int w = min(max(static_cast<int>(S.step_w[st]), 1), 8);
-    S.step_info[st][cc] = static_cast<uint32_t>(w) | (static_cast<uint32_t>(S.woff[min(blk, kH - 1)]) << 8);
-  }
   for (int i = tid; i < n_steps * 32; i += blockDim.x) {
-    const int s = i >> 5, hg = (i >> 2) & 7, cc = i & 3;
-    const int blk = S.step_blk[s][cc];
-    uint2 fr = make_uint2(0u, 0u);
+    const int st = i >> 5, hg = (i >> 2) & 7, cc = i & 3;
+    const int blk = S.step_blk[st][cc];
+    uint4 e = make_uint4(0u, 0u, 0u, 0u);
+    int wblk = blk;
     if (blk >= 0 && blk < kH) {
       __half h1, l1, h2, l2;
       split_hilo(S.qp[hg][blk], h1, l1);
       split_hilo(S.qp[hg][blk + kH], h2, l2);
-      fr.x = pack_half2(h1, h2);
-      fr.y = pack_half2(l1, l2);
+      e.x = pack_half2(h1, h2);
+      e.y = pack_half2(l1, l2);
+    } else {
+      wblk = max(static_cast<int>(S.step_blk[st][0]), 0);   // empty slot: Q' is 0, read any valid block
     }
-    S.qfrag[s][hg][cc] = fr;
+    e.z = static_cast<uint32_t>(S.woff[min(wblk, kH - 1)]) + (hg >> 2);   // lane (hg, cc) uses half H = hg / 4
+    S.kstep[st][hg][cc] = e;
+  }
+  if (tid == 0) {
+    int n = 0;
+    for (int st = 0; st < n_steps; ++st) {
+      const int w = min(max(static_cast<int>(S.step_w[st]), 1), 8);
+      if (n == 0 || S.cls_w[n - 1] != w) {
+        S.cls_w[n] = w;
+        S.cls_begin[n] = st;
+        ++n;
+      }
+    }
+    S.cls_begin[n] = n_steps;
+    S.n_cls = n;
   }
   __syncthreads();
 
@@ -335,7 +359,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt) o_acc[nt][0] = o_acc[nt][1] = o_acc[nt][2] = o_acc[nt][3] = 0.0f;
 
-  const int H = g >> 2, sh = g & 3;
+  const int sh = g & 3;
   for (int i = 0; i < my_n; ++i) {
     {
       const int nxt = i + n_stages - 1;
@@ -357,18 +381,17 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
     float acc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-    for (int s = 0; s < n_steps; ++s) {
-      const uint32_t info = S.step_info[s][c];
-      const uint2 a = S.qfrag[s][g][c];
-      switch (info & 0xffu) {
-        case 1: qk_step<1>(kw, info, H, sh, a, S, acc); break;
-        case 2: qk_step<2>(kw, info, H, sh, a, S, acc); break;
-        case 3: qk_step<3>(kw, info, H, sh, a, S, acc); break;
-        case 4: qk_step<4>(kw, info, H, sh, a, S, acc); break;
-        case 5: qk_step<5>(kw, info, H, sh, a, S, acc); break;
-        case 6: qk_step<6>(kw, info, H, sh, a, S, acc); break;
-        case 7: qk_step<7>(kw, info, H, sh, a, S, acc); break;
-        default: qk_step<8>(kw, info, H, sh, a, S, acc); break;
+    for (int ci = 0; ci < S.n_cls; ++ci) {
+      const int s0 = S.cls_begin[ci], s1 = S.cls_begin[ci + 1];
+      switch (S.cls_w[ci]) {
+        case 1: qk_class<1>(kw, s0, s1, g, c, sh, S, acc); break;
+        case 2: qk_class<2>(kw, s0, s1, g, c, sh, S, acc); break;
+        case 3: qk_class<3>(kw, s0, s1, g, c, sh, S, acc); break;
+        case 4: qk_class<4>(kw, s0, s1, g, c, sh, S, acc); break;
+        case 5: qk_class<5>(kw, s0, s1, g, c, sh, S, acc); break;
+        case 6: qk_class<6>(kw, s0, s1, g, c, sh, S, acc); break;
+        case 7: qk_class<7>(kw, s0, s1, g, c, sh, S, acc); break;
+        default: qk_class<8>(kw, s0, s1, g, c, sh, S, acc); break;
       }
     }
 

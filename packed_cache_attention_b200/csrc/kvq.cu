@@ -399,7 +399,7 @@ kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V,
   if (kd->seq_len > capacity) return KVQ_ERR_RANGE;
   if ((st = ensure_tables()) != KVQ_OK) return st;
   const Nf4Layout L = nf4_layout(kd->batch, kd->n_heads, capacity);
-  const long long tasks = 2LL * kd->batch * L.t_pad * L.nblk;
+  const long long tasks = 2LL * kd->batch * L.nblk * (L.t_pad / kNf4Rows);
   const unsigned grid = static_cast<unsigned>((tasks + kNf4Warps - 1) / kNf4Warps);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (kd->dtype) {

@@ -23,10 +23,13 @@ struct Nf4Layout {
   }
 };
 
-// One warp per (sequence, token row < T_pad, block, K-or-V). Lane l holds values
-// 8l..8l+7 of the block: head 2*blk + l/16, dims 8(l%16)..8(l%16)+7.
+constexpr int kNf4Rows = 4;   // token rows per warp task
+
+// One warp per (K-or-V, sequence, block, group of 4 token rows < T_pad). Lane l holds values
+// 8l..8l+7 of the block: head 2*blk + l/16, dims 8(l%16)..8(l%16)+7. All rows of the group
+// are loaded before any is quantized.
 template <int DT>
-__global__ void __launch_bounds__(kNf4Warps * 32) kvq_nf4_quant_pack(
+__global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
     const typename Elem<DT>::T* __restrict__ K, int64_t ksb, int64_t ksh, int64_t kst,
     const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst, int batch,
     int seq_len, Nf4Layout L, uint8_t* __restrict__ packed) {
@@ -35,48 +38,70 @@ __global__ void __launch_bounds__(kNf4Warps * 32) kvq_nf4_quant_pack(
   if (threadIdx.x < 15) sMid[threadIdx.x] = c_tab.nf4_mid[threadIdx.x];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int groups = L.t_pad / kNf4Rows;
   const long long task = static_cast<long long>(blockIdx.x) * kNf4Warps + warp;
-  const long long per_kv = static_cast<long long>(batch) * L.t_pad * L.nblk;
+  const long long per_kv = static_cast<long long>(batch) * L.nblk * groups;
   if (task >= 2 * per_kv) return;
   const int which = static_cast<int>(task / per_kv);          // 0 = K, 1 = V
   long long r = task % per_kv;
+  const int grp = static_cast<int>(r % groups);
+  r /= groups;
   const int blk = static_cast<int>(r % L.nblk);
-  r /= L.nblk;
-  const int t = static_cast<int>(r % L.t_pad);
-  const int b = static_cast<int>(r / L.t_pad);
-  const size_t row = L.row(b, blk, t);
-  uint32_t* codes = reinterpret_cast<uint32_t*>(packed + which * L.codes_bytes + row * 128);
-  __half* scales = reinterpret_cast<__half*>(packed + 2 * L.codes_bytes) + which * (L.codes_bytes / 128) + row;
-  if (t >= seq_len) {
-    codes[lane] = 0u;
-    if (lane == 0) *scales = __ushort_as_half(0);
-    return;
-  }
+  const int b = static_cast<int>(r / L.nblk);
   const T* X = which ? V : K;
   const int64_t sb = which ? vsb : ksb, sh = which ? vsh : ksh, st = which ? vst : kst;
   const int head = 2 * blk + (lane >> 4), d0 = 8 * (lane & 15);
-  const T* src = X + b * sb + head * sh + static_cast<int64_t>(t) * st + d0;
-  float x[8];
+  const int t0 = grp * kNf4Rows;
+  float x[kNf4Rows][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] = Elem<DT>::to_f32(src[i]);
-  float amax = 0.0f;
+  for (int rr = 0; rr < kNf4Rows; ++rr) {
+    const int t = t0 + rr;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    for (int i = 0; i < 8; ++i) x[rr][i] = 0.0f;
+    if (t < seq_len) {
+      const T* src = X + b * sb + head * sh + static_cast<int64_t>(t) * st + d0;
+      if constexpr (DT == KVQ_F32) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+        const float4 c = __ldg(reinterpret_cast<const float4*>(src) + 1);
+        x[rr][0] = a.x; x[rr][1] = a.y; x[rr][2] = a.z; x[rr][3] = a.w;
+        x[rr][4] = c.x; x[rr][5] = c.y; x[rr][6] = c.z; x[rr][7] = c.w;
+      } else {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+        const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const __half s16 = __float2half_rn(amax);
-  const float s = __half2float(s16);
-  uint32_t word = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float u = (s == 0.0f) ? 0.0f : __fdiv_rn(x[i], s);
-    int idx = 0;
-#pragma unroll
-    for (int k = 3; k >= 0; --k) idx += (u > sMid[idx + (1 << k) - 1]) ? (1 << k) : 0;
-    word |= static_cast<uint32_t>(idx) << (4 * i);
+        for (int i = 0; i < 4; ++i) {
+          x[rr][2 * i] = Elem<DT>::to_f32(bits_to<T>(wv[i] & 0xffffu));
+          x[rr][2 * i + 1] = Elem<DT>::to_f32(bits_to<T>(wv[i] >> 16));
+        }
+      }
+    }
   }
-  codes[lane] = word;
-  if (lane == 0) *scales = s16;
+#pragma unroll
+  for (int rr = 0; rr < kNf4Rows; ++rr) {
+    const int t = t0 + rr;
+    const size_t row = L.row(b, blk, t);
+    uint32_t* codes = reinterpret_cast<uint32_t*>(packed + which * L.codes_bytes + row * 128);
+    __half* scales = reinterpret_cast<__half*>(packed + 2 * L.codes_bytes) + which * (L.codes_bytes / 128) + row;
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[rr][i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const __half s16 = __float2half_rn(amax);        // rows past seq_len are all zero: scale 0, codes 0
+    const float s = __half2float(s16);
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float u = (s == 0.0f) ? 0.0f : __fdiv_rn(x[rr][i], s);
+      int idx = 0;
+#pragma unroll
+      for (int k = 3; k >= 0; --k) idx += (u > sMid[idx + (1 << k) - 1]) ? (1 << k) : 0;
+      word |= static_cast<uint32_t>(idx) << (4 * i);
+    }
+    if (t >= seq_len) word = 0u;
+    codes[lane] = word;
+    if (lane == 0) *scales = (t < seq_len) ? s16 : __ushort_as_half(0);
+  }
 }
 
 // MHA decode (G = 1), CUDA cores. Grid (splits, batch * n_heads), 4 warps per CTA, each
