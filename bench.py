@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0, help="override the context length (profiling only)")
     ap.add_argument("--no-nf4", action="store_true", help="skip the NF4-variant measurement")
+    ap.add_argument("--nf4-batch", type=int, default=0, help="override the NF4 batch (profiling only)")
     return ap.parse_args()
 
 
@@ -231,7 +232,8 @@ def run_gpu(args, rank, world, local_rank):
         e2e = {"value": world * L * B * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    nf4 = measure_nf4(kvq, wl, dev, stream, hbm_peak=peaks()[0]) if (rank == 0 and not args.no_nf4) else None
+    nf4 = (measure_nf4(kvq, wl, dev, stream, hbm_peak=peaks()[0], batch=args.nf4_batch)
+           if (rank == 0 and not args.no_nf4) else None)
 
     steps = args.steps
     ms_step = total_ms / steps
@@ -285,13 +287,13 @@ def run_gpu(args, rank, world, local_rank):
     return result
 
 
-def measure_nf4(kvq, wl, dev, stream, hbm_peak, iters=10):
+def measure_nf4(kvq, wl, dev, stream, hbm_peak, iters=10, batch=0):
     """NQKV-style NF4 variant at the OPT-30B shape (one layer: B8 x 56 heads x 8192 tokens,
     fp16), timed outside the step: quantize/pack and MHA decode, CUDA events per launch."""
     import torch
     W = wl.WORKLOADS["nqkv_opt30b"]
-    x = wl.make_nf4_inputs(W.batch, W.n_q_heads, W.head_dim, W.seq_len, W.dtype, seed=7, device=dev)
-    B, H, T, d = W.batch, W.n_q_heads, W.seq_len, W.head_dim
+    B, H, T, d = (batch or W.batch), W.n_q_heads, W.seq_len, W.head_dim
+    x = wl.make_nf4_inputs(B, H, d, T, W.dtype, seed=7, device=dev)
     packed = torch.empty(kvq.kvq_nf4_packed_bytes(B, H, T, d), dtype=torch.uint8, device=dev)
     out = torch.empty((B, H, d), dtype=torch.float32, device=dev)
     ws = torch.zeros(kvq.kvq_nf4_decode_workspace_bytes(B, H, T, d), dtype=torch.uint8, device=dev)

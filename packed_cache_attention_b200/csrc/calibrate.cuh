@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
   __shared__ double sE[kH];
   __shared__ double sGain[kH * 8];
   __shared__ long long sKey[kH * 8];
+  __shared__ short sIdx[kH * 8];
   __shared__ int sWidth[kH];
   __shared__ int sStepStart[9];
   __shared__ int sCount[9];
@@ -197,38 +198,35 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     sGain[tid] = gv;
     // valid gains are >= 0 (+0 for a zero energy); invalid entries never precede a valid one
     sKey[tid] = valid ? __double_as_longlong(gv) : -1LL;
+    sIdx[tid] = static_cast<short>(tid);
+    if (tid < kH) sWidth[tid] = 0;
   }
   __syncthreads();
   if (mode == KVQ_MODE_UNIFORM) {
     if (tid < kH) sWidth[tid] = bits_k;
   } else {
-    // Non-negative doubles order like their bit patterns, so the comparisons run on 64-bit
-    // integers (invalid entries hold -1.0, whose pattern is above every valid one, and are
-    // excluded separately).
-    const long long key = __double_as_longlong(sGain[tid]);
-    const bool valid = (tid & 7) < w_max;
-    int rank = 0;
-    if (valid) {
-#pragma unroll 4
-      for (int bb = 0; bb < kH; ++bb) {
-        // entries of block bb preceding entry tid form a prefix of w = 0..w_max-1
-        int lo = 0, hi = w_max;
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          if (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            const int e = 8 * bb + mid;
-            const long long ke = sKey[e];
-            if (ke > key || (ke == key && e < tid)) lo = mid + 1;
-            else hi = mid;
+    // Sort the 512 entries by (gain descending, entry ascending) with a bitonic network;
+    // the first bits_k * 64 are the greedy's picks. Non-negative doubles order like their
+    // bit patterns, so keys are 64-bit integers; entries at or above w_max get key -1 and
+    // sort after every valid one.
+    __syncthreads();
+    for (int k = 2; k <= kH * 8; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const int i = tid, ixj = tid ^ j;
+        if (ixj > i) {
+          const long long ka = sKey[i], kb = sKey[ixj];
+          const int ia = sIdx[i], ib = sIdx[ixj];
+          const bool a_first = (ka > kb) || (ka == kb && ia < ib);
+          const bool want_a_first = (i & k) == 0;
+          if (a_first != want_a_first) {
+            sKey[i] = kb; sKey[ixj] = ka;
+            sIdx[i] = static_cast<short>(ib); sIdx[ixj] = static_cast<short>(ia);
           }
         }
-        rank += lo;
+        __syncthreads();
       }
     }
-    const bool picked = valid && rank < bits_k * kH;
-    const unsigned mask = __ballot_sync(0xffffffffu, picked);
-    if ((tid & 7) == 0) sWidth[tid >> 3] = __popc((mask >> (tid & 24)) & 0xffu);
+    if (tid < bits_k * kH) atomicAdd(&sWidth[sIdx[tid] >> 3], 1);
   }
   if (tid < 9) sCount[tid] = 0;
   __syncthreads();
