@@ -30,7 +30,7 @@
 extern "C" {
 #endif
 
-#define KVQ_ABI_VERSION 1
+#define KVQ_ABI_VERSION 2
 #define KVQ_TILE_TOKENS 32     /* tokens per packed Block-GTQ tile */
 #define KVQ_HEAD_DIM 128       /* head dimension the kernels are built for */
 #define KVQ_MAX_WIDTH 8        /* widest Lloyd-Max codebook */
@@ -90,22 +90,30 @@ typedef struct {
 } kvq_cache_desc;
 
 /* Allocation record of one KV head, as written by kvq_calibrate (device memory, array of
- * n_kv_heads records). Block b covers dims b and b + head_dim/2. */
+ * n_kv_heads records). Block b covers dims b and b + head_dim/2.
+ * A token's K codes form one bit stream in "stream order": width classes from 8 bits down
+ * to 1 bit, blocks ascending within a class, each block contributing the code of dim b and
+ * then the code of dim b + head_dim/2; blocks of width 0 contribute nothing. */
 typedef struct {
   double energy[64];        /* E_b, mean ||k_b||^2 over the calibration tokens */
   float gain[64];           /* g_b, per-block scale applied before the codebook */
   float dequant[64];        /* f_b = 1 / (sqrt(d) g_b) */
-  uint16_t word_off[64];    /* word offset of block b's segment in a tile's K part */
+  int16_t bit_off[64];      /* bit offset of block b's code pair in the K stream (-1: width 0) */
   uint8_t width[64];        /* w_b, bits per dim of block b */
-  uint8_t step_width[32];   /* decode k-steps: width of the blocks in step s */
-  int8_t step_block[32][4]; /* decode k-steps: up to 4 blocks per step (-1 = none) */
+  uint8_t stream_block[64]; /* blocks in stream order; 255 after the last one */
+  uint16_t class_bit[8];    /* class c (stream order): bit offset of its first code */
+  uint8_t class_width[8];   /* class c: width (0 = no such class) */
+  uint8_t class_first[8];   /* class c: index of its first block in stream_block */
+  uint8_t class_blocks[8];  /* class c: number of blocks */
+  uint8_t reserved_b[56];
   int32_t head_dim;
   int32_t bits_k;
   int32_t w_max;
   int32_t mode;
-  int32_t n_steps;          /* number of valid decode k-steps */
+  int32_t n_classes;        /* number of classes with at least one block */
   int32_t k_words;          /* 32-bit words in a tile's K part (= bits_k * head_dim) */
-  int32_t reserved[2];
+  int32_t n_blocks;         /* blocks with w_b > 0 */
+  int32_t reserved;
 } kvq_head_alloc;
 
 /* ---------------------------------------------------------------- queries (host only) */
@@ -174,6 +182,13 @@ kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_p
  * y = (x a) g_b in fp32, code = number of thresholds below y; K uses the allocation's
  * widths and gains, V uses width cache->bits_v and g = 1. Tiles past seq_len are not
  * written; tokens of the last tile beyond seq_len are stored as code 0, norm 0.
+ * Layout: per (sequence, KV head) consecutive 32-token tile records of
+ * 4 * head_dim * (bits_k + bits_v) + 128 bytes, little-endian:
+ *   K part: 32-bit word 32 i + t is word i (i < 4 bits_k) of token t's K stream (see
+ *           kvq_head_alloc; codes least significant bit first, bits_k * head_dim bits).
+ *   V part: word 128 i + j is word i (i < bits_v) of dim j's V stream: the codes of the
+ *           tile's tokens 0..31 at dim j, bits_v bits each, least significant bit first.
+ *   32 fp16 K norms, then 32 fp16 V norms, in token order.
  * K, V: [batch][n_kv_heads][seq_len][128] (kd, vd may differ in strides, not in shape).
  * alloc: records from kvq_calibrate with bits_k == cache->bits_k.
  * packed: kvq_packed_bytes(cache) bytes, 16-byte aligned. */

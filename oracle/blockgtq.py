@@ -23,8 +23,9 @@ The page names these steps without defining them. The readings taken here
   quantizer  per token row: fp16 norm of the row (fp32 sum of squares), a = sqrt(d)/norm in fp32,
              y = (x * a) * g_b in fp32, code = #{thresholds strictly below y}
              of the width-w_b Lloyd-Max codebook. Values use width bits_v, g = 1.
-  layout     32-token tiles; bit planes transposed so that each 32-bit word
-             holds one bit plane of 32 codes (see pack_cache).
+  layout     32-token tiles; per token one K bit stream (codes in width-class
+             order), per dim one V bit stream over the tile's tokens, both stored
+             word-planar (see pack_cache).
   attention  softmax over cached positions 0..T-1 of q . k_hat / sqrt(d),
              k_hat = norm * c[code] * f_b, v_hat = norm * c[code] / sqrt(d).
 """
@@ -226,43 +227,67 @@ def packed_bytes(batch: int, n_kv_heads: int, capacity: int, d: int, bits_k: int
     return batch * n_kv_heads * n_tiles * tile_record_bytes(d, bits_k, bits_v)
 
 
-def _k_bit_source(H: int, q: int, b: int, h: int) -> tuple[int, int]:
-    """(token in tile, dim) whose code bit sits at bit q of K word half H of block b.
-
-    q = s + 4 m with s = q mod 4, m = q div 4: token = 4H + s + 8 (m div 2),
-    dim = b if m is even else b + h.
-    """
-    s, m = q % 4, q // 4
-    return 4 * H + s + 8 * (m // 2), b + h * (m % 2)
+def k_stream_blocks(w_blocks: np.ndarray) -> list[int]:
+    """Blocks in the order their codes appear in a token's K bit stream: widths descending
+    (8 down to 1), blocks ascending within one width; blocks of width 0 are left out."""
+    w_blocks = [int(x) for x in w_blocks]
+    return [b for w in range(8, 0, -1) for b in range(len(w_blocks)) if w_blocks[b] == w]
 
 
-def _v_bit_source(q: int) -> int:
-    """Token in tile whose code bit sits at bit q of a V word: q = c + 4 m ->
-    token = 8 (m div 2) + 2 c + (m mod 2)."""
-    c, m = q % 4, q // 4
-    return 8 * (m // 2) + 2 * c + (m % 2)
-
-
-def k_word_offsets(w_blocks: np.ndarray) -> np.ndarray:
-    """Word offset of block b's segment inside the K part of a tile (blocks ascending,
-    2 * w_b words each: planes p ascending, halves H = 0, 1)."""
-    off = np.zeros(len(w_blocks), dtype=np.int64)
+def k_bit_offsets(w_blocks: np.ndarray) -> np.ndarray:
+    """Bit offset of block b's code pair in a token's K stream (-1 for width 0): the code of
+    dim b sits at that offset and the code of dim b + d/2 right after it."""
+    off = np.full(len(w_blocks), -1, dtype=np.int64)
     acc = 0
-    for b, w in enumerate(w_blocks):
+    for b in k_stream_blocks(w_blocks):
         off[b] = acc
-        acc += 2 * int(w)
+        acc += 2 * int(w_blocks[b])
     return off
+
+
+def pack_bits(values: np.ndarray, widths: list[int]) -> np.ndarray:
+    """Concatenate values[..., i] (widths[i] bits each, least significant bit first) into one
+    bit stream and return it as little-endian 32-bit words [..., ceil(sum/32)]."""
+    values = np.asarray(values, dtype=np.uint64)
+    total = int(sum(widths))
+    n_words = -(-total // 32)
+    bits = np.zeros(values.shape[:-1] + (32 * n_words,), dtype=np.uint8)
+    pos = 0
+    for i, w in enumerate(widths):
+        for p in range(w):
+            bits[..., pos] = ((values[..., i] >> np.uint64(p)) & np.uint64(1)).astype(np.uint8)
+            pos += 1
+    weights = (np.uint64(1) << np.arange(32, dtype=np.uint64))
+    return np.sum(bits.reshape(values.shape[:-1] + (n_words, 32)).astype(np.uint64) * weights, axis=-1)
+
+
+def unpack_bits(words: np.ndarray, widths: list[int]) -> np.ndarray:
+    """Inverse of pack_bits: values [..., len(widths)] from words [..., n_words]."""
+    words = np.asarray(words, dtype=np.uint64)
+    n_words = words.shape[-1]
+    bits = ((words[..., :, None] >> np.arange(32, dtype=np.uint64)) & np.uint64(1)).reshape(
+        words.shape[:-1] + (32 * n_words,))
+    out = np.zeros(words.shape[:-1] + (len(widths),), dtype=np.uint64)
+    pos = 0
+    for i, w in enumerate(widths):
+        for p in range(w):
+            out[..., i] |= bits[..., pos] << np.uint64(p)
+            pos += 1
+    return out
 
 
 def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarray:
     """Packed cache bytes [B][Hkv][n_tiles][record] for capacity tokens per sequence.
 
-    Tile record (little-endian):
-      K part, bits_k * d words: for each block b ascending with w_b > 0, for each
-        plane p < w_b, two words (H = 0, 1); bit q of word H holds bit p of the
-        code at (token, dim) = _k_bit_source(H, q, b, h).
-      V part, bits_v * d words: for each plane p < bits_v, for each dim j, one
-        word; bit q holds bit p of the code of token _v_bit_source(q), dim j.
+    Tile record (little-endian 32-bit words, then fp16 norms):
+      K part, bits_k * d words, stored word-planar: word 32 i + t is word i of token t's
+        K stream (i < 4 bits_k). A token's K stream is its K codes concatenated, least
+        significant bit first, in the order of k_stream_blocks; each block gives the code
+        of dim b (w_b bits) and then the code of dim b + d/2 (w_b bits). The stream is
+        exactly bits_k * d bits long.
+      V part, bits_v * d words, stored word-planar: word d i + j is word i of dim j's V
+        stream (i < bits_v), which is the codes of tokens 0..31 of the tile at dim j,
+        concatenated, bits_v bits each, least significant bit first.
       32 fp16 K norms, 32 fp16 V norms, in token order.
     Tokens at or beyond the sequence length T are stored with code 0 and norm 0.
     """
@@ -285,24 +310,17 @@ def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarr
     Vc = Vc.reshape(B, H, n_tiles, TILE, d)
     rec = tile_record_bytes(d, bits_k, bits_v)
     out = np.zeros((B, H, n_tiles, rec), dtype=np.uint8)
-    qs = np.arange(32, dtype=np.uint64)
     for hh in range(H):
         w_blocks = alloc["w"][hh]
-        kwords = np.zeros((B, n_tiles, tile_k_words(bits_k, d)), dtype=np.uint64)
-        off = k_word_offsets(w_blocks)
-        for b in range(h):
-            for p in range(int(w_blocks[b])):
-                for Hh in (0, 1):
-                    src = [_k_bit_source(Hh, q, b, h) for q in range(32)]
-                    tok = np.array([s[0] for s in src])
-                    dim = np.array([s[1] for s in src])
-                    bits = ((Kc[:, hh][:, :, tok, dim] >> p) & 1).astype(np.uint64)   # [B][n_tiles][32]
-                    kwords[:, :, off[b] + 2 * p + Hh] = np.sum(bits << qs, axis=-1)
-        vwords = np.zeros((B, n_tiles, tile_v_words(bits_v, d)), dtype=np.uint64)
-        vtok = np.array([_v_bit_source(q) for q in range(32)])
-        for p in range(bits_v):
-            bits = ((Vc[:, hh][:, :, vtok, :] >> p) & 1).astype(np.uint64)                # [B][n_tiles][32][d]
-            vwords[:, :, p * d:(p + 1) * d] = np.sum(bits << qs[:, None], axis=2)
+        order = k_stream_blocks(w_blocks)
+        dims = [j for b in order for j in (b, b + h)]
+        widths = [int(w_blocks[b]) for b in order for _ in (0, 1)]
+        kstream = pack_bits(Kc[:, hh][..., dims], widths)                     # [B][n_tiles][32][kw]
+        if kstream.shape[-1] != tile_k_words(bits_k, d) // TILE:
+            raise ValueError("widths do not fill the K budget")
+        kwords = np.transpose(kstream, (0, 1, 3, 2)).reshape(B, n_tiles, -1)   # word-planar
+        vstream = pack_bits(np.transpose(Vc[:, hh], (0, 1, 3, 2)), [bits_v] * TILE)   # [B][n_tiles][d][bv]
+        vwords = np.transpose(vstream, (0, 1, 3, 2)).reshape(B, n_tiles, -1)
         parts = [kwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1),
                  vwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1),
                  Kn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1),
@@ -328,21 +346,13 @@ def unpack_cache(packed: np.ndarray, alloc: dict, bits_v: int, seq_len: int) -> 
     Vn = norms[..., TILE:].reshape(B, H, cap)
     for hh in range(H):
         w_blocks = alloc["w"][hh]
-        off = k_word_offsets(w_blocks)
-        for b in range(h):
-            for p in range(int(w_blocks[b])):
-                for Hh in (0, 1):
-                    word = kw[:, hh, :, off[b] + 2 * p + Hh].astype(np.uint64)
-                    for q in range(32):
-                        tok, dim = _k_bit_source(Hh, q, b, h)
-                        bit = ((word >> np.uint64(q)) & np.uint64(1)).astype(np.uint8)
-                        Kc[:, hh, :, tok, dim] |= bit << p
-        for p in range(bits_v):
-            for q in range(32):
-                tok = _v_bit_source(q)
-                word = vw[:, hh, :, p * d:(p + 1) * d].astype(np.uint64)
-                bit = ((word >> np.uint64(q)) & np.uint64(1)).astype(np.uint8)
-                Vc[:, hh, :, tok, :] |= bit << p
+        order = k_stream_blocks(w_blocks)
+        dims = [j for b in order for j in (b, b + h)]
+        widths = [int(w_blocks[b]) for b in order for _ in (0, 1)]
+        kstream = np.transpose(kw[:, hh].reshape(B, n_tiles, nk // TILE, TILE), (0, 1, 3, 2))
+        Kc[:, hh][..., dims] = unpack_bits(kstream, widths).astype(np.uint8)
+        vstream = np.transpose(vw[:, hh].reshape(B, n_tiles, bits_v, d), (0, 1, 3, 2))   # [B][n][d][bv]
+        Vc[:, hh] = np.transpose(unpack_bits(vstream, [bits_v] * TILE), (0, 1, 3, 2)).astype(np.uint8)
     Kc = Kc.reshape(B, H, cap, d)[:, :, :seq_len]
     Vc = Vc.reshape(B, H, cap, d)[:, :, :seq_len]
     return {"Kc": Kc, "Kn": Kn[:, :, :seq_len].astype(np.float16),

@@ -173,11 +173,9 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta, 4) kvq_calib_reduce(
 __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict__ energy, int bits_k, int w_max,
                                                         int mode, kvq_head_alloc* __restrict__ alloc) {
   __shared__ double sE[kH];
-  __shared__ double sGain[kH * 8];
   __shared__ long long sKey[kH * 8];
   __shared__ short sIdx[kH * 8];
   __shared__ int sWidth[kH];
-  __shared__ int sStepStart[9];
   __shared__ int sCount[9];
   __shared__ double sSum;
   const int h = blockIdx.x, tid = threadIdx.x;
@@ -195,7 +193,6 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     const double gv = valid ? __dmul_rn(sE[b], __dsub_rn(static_cast<double>(c_tab.delta[w]),
                                                           static_cast<double>(c_tab.delta[w + 1])))
                             : -1.0;
-    sGain[tid] = gv;
     // valid gains are >= 0 (+0 for a zero energy); invalid entries never precede a valid one
     sKey[tid] = valid ? __double_as_longlong(gv) : -1LL;
     sIdx[tid] = static_cast<short>(tid);
@@ -243,43 +240,44 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     al->width[b] = static_cast<uint8_t>(sWidth[b]);
     atomicAdd(&sCount[sWidth[b]], 1);
   }
-  if (tid < 32 * 4) {
-    al->step_block[tid >> 2][tid & 3] = -1;
-  }
-  if (tid >= 128 && tid < 160) al->step_width[tid - 128] = 0;
   __syncthreads();
+  // Stream order: width classes 8..1, blocks ascending inside a class; each block is a pair
+  // of codes (dim b, dim b + 64) of w_b bits each.
   if (tid == 0) {
-    int off = 0;
-    for (int b = 0; b < kH; ++b) {
-      al->word_off[b] = static_cast<uint16_t>(off);
-      off += 2 * sWidth[b];
-    }
-    int steps = 0;
+    int pos = 0, bit = 0, n_cls = 0;
     for (int w = 8; w >= 1; --w) {
-      sStepStart[w] = steps;
-      steps += (sCount[w] + 3) / 4;
+      if (sCount[w] == 0) continue;
+      al->class_width[n_cls] = static_cast<uint8_t>(w);
+      al->class_first[n_cls] = static_cast<uint8_t>(pos);
+      al->class_blocks[n_cls] = static_cast<uint8_t>(sCount[w]);
+      al->class_bit[n_cls] = static_cast<uint16_t>(bit);
+      for (int b = 0; b < kH; ++b) {
+        if (sWidth[b] != w) continue;
+        al->stream_block[pos++] = static_cast<uint8_t>(b);
+        al->bit_off[b] = static_cast<int16_t>(bit);
+        bit += 2 * w;
+      }
+      ++n_cls;
     }
-    sStepStart[0] = steps;
-    al->n_steps = steps;
-    al->k_words = off;
+    for (int c = n_cls; c < 8; ++c) {
+      al->class_width[c] = 0;
+      al->class_first[c] = static_cast<uint8_t>(pos);
+      al->class_blocks[c] = 0;
+      al->class_bit[c] = static_cast<uint16_t>(bit);
+    }
+    for (int i = pos; i < kH; ++i) al->stream_block[i] = 0xffu;
+    for (int b = 0; b < kH; ++b)
+      if (sWidth[b] == 0) al->bit_off[b] = -1;
+    al->n_classes = n_cls;
+    al->n_blocks = pos;
+    al->k_words = bit / 32 * kTile;     // bits per token * 32 tokens / 32 bits per word
     al->head_dim = kD;
     al->bits_k = bits_k;
     al->w_max = w_max;
     al->mode = mode;
-    al->reserved[0] = 0;
-    al->reserved[1] = 0;
+    al->reserved = 0;
   }
-  __syncthreads();
-  if (tid < kH) {
-    const int b = tid, w = sWidth[b];
-    if (w > 0) {
-      int r = 0;
-      for (int j = 0; j < b; ++j) r += (sWidth[j] == w);
-      const int s = sStepStart[w] + r / 4;
-      al->step_block[s][r & 3] = static_cast<int8_t>(b);
-      al->step_width[s] = static_cast<uint8_t>(w);
-    }
-  }
+  if (tid < 56) al->reserved_b[tid] = 0;
 }
 
 }  // namespace kvq

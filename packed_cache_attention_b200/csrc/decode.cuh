@@ -2,175 +2,196 @@
 // allocation for KV cache quantization", abstract: attention served from the packed cache;
 // the NQKV review's editorial extensions propose folding the table lookup into attention).
 //
-// Grid: (splits, batch * n_kv_heads); 4 warps per CTA; each CTA owns a contiguous range of
-// 32-token tiles of one (sequence, KV head) and each warp every 4th tile of that range.
-// Tiles are staged into shared memory with 16-byte cp.async copies, kStages deep per warp.
-//
-// Per tile, on the tensor cores (mma.sync, fp16 operands, fp32 accumulate), for the G <= 8
-// query heads of the KV head held as 16 rows (8 heads' fp16 high parts, 8 low parts):
-//   S^T[16][32 tokens] = Q'[16][k-steps of 4 RoPE blocks] x Khat_codes^T
-//     Q'_{h,j} = q_{h,j} f_b log2(e) / sqrt(d) scaled per head by a power of two; the key
-//     norm is applied to S after the MMA, so the B operand is the raw fp16 centroid.
-//   online softmax in the log2 domain, P' = p * vnorm / sqrt(d) split into fp16 hi + lo,
-//   O[16][128] += P'[16][32 tokens] x Vhat_codes[32][128].
-// Fragment order follows the tile layout: lane (g = lane/4, c = lane%4) holds token g + 8j
-// (n-tile j) for K and tokens 8(m/2) + 2c + (m%2) for V, so its codes are the nibbles at
-// bits (g%4) + 4m of a K word and c + 4m of a V word.
-// Splits write (m, l, O) partials to the workspace; the last CTA of a (sequence, KV head),
-// found with an atomic ticket, merges them in split order and writes out = O / l.
+// Grid: (splits, batch * n_kv_heads). Each CTA owns a contiguous range of 128-token chunks
+// (4 tile records) of one (sequence, KV head) and runs a pipeline over them:
+//   load warp     bulk-copies each chunk's tile records into a shared-memory stage;
+//   16 warps      dequantize codes through shared-memory lookup tables straight into tensor
+//                 memory: K-hat rows (lane = token, one fp16 pair per column) and V-hat^T
+//                 rows (lane = dim, columns = token pairs); then run the softmax;
+//   MMA warp      one thread issues tcgen05.mma (M = 128, N = 16, fp16 -> fp32):
+//                   S^T[128 tokens][16]  = Khat[128][K cols]  x  Q'^T  (Q' hi rows 0-7, lo 8-15)
+//                   O^T[128 dims][16]   = Vhat^T[128][128]   x  P'^T  (P' hi rows 0-7, lo 8-15)
+// with K-hat and V-hat^T as the A operand in tensor memory and Q', P' as the small B operand
+// in shared memory. K columns follow the stream order of the tile layout (width classes,
+// each padded to whole groups of 4 block pairs); Q' carries f_b, log2(e)/sqrt(d) and a per
+// query power of two that keeps its fp16 split in range, and the key norm scales S after
+// the MMA. Softmax runs online in the log2 domain with P' = p * vnorm / sqrt(d) split into
+// fp16 hi + lo. Warp group g handles query rows 2g, 2g+1 of the softmax and of O.
+// Tensor memory and shared buffers are double-buffered by chunk parity; every hand-off is
+// an mbarrier with a bounded wait.
+// Splits write (m, l, O) partials to the workspace; the last CTA of each group of 8 splits
+// merges its group, and the last group merges the groups (atomic tickets), writing
+// out = O / l.
 #pragma once
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace kvq {
 
-constexpr int kDecWarps = 16;
-constexpr int kDecStages = 3;        // deepest cp.async pipeline per warp (fewer when records are large)
-constexpr int kMaxSteps = 32;
+constexpr int kDecComputeWarps = 16;
+constexpr int kDecMmaWarp = 16;
+constexpr int kDecLoadWarp = 17;
+constexpr int kDecThreads = 18 * 32;
+constexpr int kChunkTiles = 4;
+constexpr int kChunkTokens = kChunkTiles * kTile;   // = MMA M = tensor-memory lanes
+constexpr int kDecStagesMax = 4;
 constexpr int kMaxMergeSplits = 160;
-constexpr int kMergeGroup = 8;      // splits merged by the last CTA of each group (first level)
-constexpr int kTargetCtas = 148;   // 1 CTA of 16 warps per SM on a 148-SM B200
+constexpr int kMergeGroup = 8;       // splits merged by the last CTA of each group (first level)
+constexpr int kTargetCtas = 148;     // one CTA per SM on a 148-SM B200
+constexpr int kGroupPairs = 4;       // block pairs (tensor-memory columns) per K decode group
+constexpr int kMaxKGroups = 32;      // at most 64 / 4 + 8 groups per head
+constexpr uint32_t kWaitLimit = 1u << 20;
 
-struct DecodeSmem {
-  uint4 kstep[kMaxSteps][8][4];     // per k-step, head row g, lane c: {Q' hi, Q' lo, K word offset + H, 0}
-  float qp[8][kD];                  // Q' in fp32 before scaling
-  float qmul[8];                    // 2^e that undoes the per-head scaling of Q'
-  uint16_t cent[kCentroidCount];    // fp16 centroid bit patterns
-  uint4 lut8[4];                    // widths 1..3: {lo bytes 0-3, lo 4-7, hi 0-3, hi 4-7}
-  uint4 lut16[2];                   // width 4: {loA0, loA1, loB0, loB1}, {hiA0, hiA1, hiB0, hiB1}
-  uint16_t woff[kH];
-  int8_t step_blk[kMaxSteps][4];
-  uint8_t step_w[kMaxSteps];
-  int cls_w[9];                      // k-steps grouped by width: width of class i,
-  int cls_begin[10];                 // first step of class i (cls_begin[n_cls] = n_steps)
-  int n_cls;
-  int n_steps;
+// Tensor-memory columns (512 allocated): A_K[2] (128 each), A_V[2] (64 each), S[2], O[2] (16 each).
+constexpr uint32_t kTmemCols = 512;
+__device__ __forceinline__ uint32_t col_ak(int b) { return 128u * b; }
+__device__ __forceinline__ uint32_t col_av(int b) { return 256u + 64u * b; }
+__device__ __forceinline__ uint32_t col_s(int b) { return 384u + 16u * b; }
+__device__ __forceinline__ uint32_t col_o(int b) { return 416u + 16u * b; }
+
+// Shared-memory map (byte offsets from the start of dynamic shared memory).
+// Pair tables give the fp16 pair {c[i & m], c[i >> w]} for the 2w-bit index i of two
+// consecutive codes. Widths 1..3 keep one copy per lane (entry e of lane l at word 32 e + l)
+// so that 32 lanes never conflict; widths 4..6 keep one copy; widths 7, 8 use single-code
+// fp16 tables.
+__host__ __device__ constexpr int lut_off(int w) {
+  return w == 1 ? 0 : w == 2 ? 512 : w == 3 ? 2560 : w == 4 ? 10752 : w == 5 ? 11776 : w == 6 ? 15872 : w == 7 ? 32256
+                                                                                                             : 32512;
+}
+constexpr int kCentOff = 33024;                 // 510 fp16 centroids
+constexpr int kBQOff = 34048;                   // Q' (B operand of S), K-major, up to 256 K elements
+constexpr int kBQBytes = 32 * 256;
+constexpr int kBPOff = kBQOff + kBQBytes;       // P' (B operand of O), 2 buffers, N-major
+constexpr int kBPBytes = 4096;
+constexpr int kHdrOff = kBPOff + 2 * kBPBytes;
+
+struct DecHeader {
+  uint64_t full[kDecStagesMax];
+  uint64_t empty[kDecStagesMax];
+  uint64_t kready[2], vready[2], pready[2], sfull[2], ofull[2];
+  uint32_t tmem_base;
+  int k_cols;                        // K columns used by the S MMA (multiple of 8)
+  int n_kgroups[4];
+  uint32_t kgroup[4][kMaxKGroups];   // width | bit offset << 4 | column << 16
+  int8_t col_block[128];             // block of K column c (-1 = padding)
+  float qscale[8];                   // 2^e that undoes the range scaling of Q' row h
+  float xmax[2][4][4][2];            // chunk max: [parity][warp group][quarter][query]
+  float lpart[4][4][2];              // row sums: [warp group][quarter][query]
   int last;
-  float mw[8][kMaxMergeSplits];     // cross-split merge: weight 2^(m_s - M) per head and member
+  float mw[8][kMaxMergeSplits];      // cross-split merge: weight 2^(m_s - M) per head and member
   float Lsum[8];
   float Mmax[8];
 };
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
+__host__ __device__ constexpr int decode_stage_off() { return kHdrOff + ((static_cast<int>(sizeof(DecHeader)) + 127) / 128) * 128; }
+
+// ---------------------------------------------------------------- code extraction + lookup
+
+// Bits [p, p + n) of the 64-bit value hi:lo (p, n constant after unrolling, n <= 16).
+__device__ __forceinline__ uint32_t field(uint32_t lo, uint32_t hi, int p, int n) {
+  uint32_t v;
+  if (p >= 32) v = hi >> (p - 32);
+  else if (p + n <= 32) v = lo >> p;
+  else v = __funnelshift_r(lo, hi, p);
+  return v & ((1u << n) - 1u);
 }
 
-// Gather bit p of 8 codes from W plane words (word p at words[p * stride]; code m at bit
-// shift + 4m) into 4-bit nibbles: nibble m of the result is code m.
+// fp16 pair for the pair index idx = code_a | code_b << W (code_a in the low half).
 template <int W>
-__device__ __forceinline__ uint32_t gather_nibbles(const uint32_t* words, int stride, int shift) {
-  uint32_t x = 0;
-#pragma unroll
-  for (int p = 0; p < W; ++p) x |= rotr(words[p * stride], static_cast<uint32_t>(shift - p) & 31u) & (0x11111111u << p);
-  return x;
-}
-
-// Register lookup of 8 codes (nibbles of x, each < 8) in an 8-entry fp16 table split into
-// low and high bytes; r[k] = fp16x2(entry[code 2k], entry[code 2k+1]).
-__device__ __forceinline__ void lut8(uint32_t x, const uint4& L, uint32_t (&r)[4]) {
-  const uint32_t la = prmt(L.x, L.y, x), ha = prmt(L.z, L.w, x);
-  const uint32_t xh = x >> 16;
-  const uint32_t lb = prmt(L.x, L.y, xh), hb = prmt(L.z, L.w, xh);
-  r[0] = prmt(la, ha, 0x5140u);
-  r[1] = prmt(la, ha, 0x7362u);
-  r[2] = prmt(lb, hb, 0x5140u);
-  r[3] = prmt(lb, hb, 0x7362u);
-}
-
-// 16-entry version: the low 3 bits of a nibble index two 8-entry halves, bit 3 picks the
-// half through a byte mask made with prmt's sign-replicate mode.
-__device__ __forceinline__ void lut16(uint32_t x, const uint4& LO, const uint4& HI, uint32_t (&r)[4]) {
-  const uint32_t x7 = x & 0x77777777u;
-  const uint32_t xh = x >> 16, x7h = x7 >> 16;
-  const uint32_t ma = prmt(x << 4, x, 0xD9C8u), mb = prmt(xh << 4, xh, 0xD9C8u);
-  const uint32_t la = (prmt(LO.x, LO.y, x7) & ~ma) | (prmt(LO.z, LO.w, x7) & ma);
-  const uint32_t ha = (prmt(HI.x, HI.y, x7) & ~ma) | (prmt(HI.z, HI.w, x7) & ma);
-  const uint32_t lb = (prmt(LO.x, LO.y, x7h) & ~mb) | (prmt(LO.z, LO.w, x7h) & mb);
-  const uint32_t hb = (prmt(HI.x, HI.y, x7h) & ~mb) | (prmt(HI.z, HI.w, x7h) & mb);
-  r[0] = prmt(la, ha, 0x5140u);
-  r[1] = prmt(la, ha, 0x7362u);
-  r[2] = prmt(lb, hb, 0x5140u);
-  r[3] = prmt(lb, hb, 0x7362u);
-}
-
-// Widths 5..8: gather the 8 codes as bytes (even codes in `ev`, odd codes in `od`, byte k =
-// code 2k / 2k+1), one rotate + mask per plane and parity, then look each byte up in the
-// shared fp16 table.
-template <int W>
-__device__ __forceinline__ void lut_wide(const uint32_t* words, int stride, int shift, const uint16_t* table,
-                                         uint32_t (&r)[4]) {
-  uint32_t ev = 0u, od = 0u;
-#pragma unroll
-  for (int p = 0; p < W; ++p) {
-    const uint32_t w = words[p * stride];
-    ev |= rotr(w, static_cast<uint32_t>(shift - p) & 31u) & (0x01010101u << p);
-    od |= rotr(w, static_cast<uint32_t>(shift + 4 - p) & 31u) & (0x01010101u << p);
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    r[k] = pack_u16x2(table[(ev >> (8 * k)) & 0xffu], table[(od >> (8 * k)) & 0xffu]);
-}
-
-// The 8 codes of width W at bits shift + 4m of W plane words, as 4 fp16x2 fragments
-// (r[k] = (code 2k, code 2k+1)).
-template <int W>
-__device__ __forceinline__ void decode8(const uint32_t* words, int stride, int shift, const DecodeSmem& S,
-                                        uint32_t (&r)[4]) {
+__device__ __forceinline__ uint32_t pair_value(uint32_t idx, const uint8_t* sm, uint32_t lane4) {
   if constexpr (W <= 3) {
-    lut8(gather_nibbles<W>(words, stride, shift), S.lut8[W], r);
-  } else if constexpr (W == 4) {
-    lut16(gather_nibbles<4>(words, stride, shift), S.lut16[0], S.lut16[1], r);
+    return *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + ((idx << 7) | lane4));
+  } else if constexpr (W <= 6) {
+    return *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + (idx << 2));
   } else {
-    lut_wide<W>(words, stride, shift, S.cent + ((1 << W) - 2), r);
+    const uint16_t* t = reinterpret_cast<const uint16_t*>(sm + lut_off(W));
+    return static_cast<uint32_t>(t[idx & ((1u << W) - 1u)]) | (static_cast<uint32_t>(t[idx >> W]) << 16);
   }
 }
 
-// One QK k-step: 4 RoPE blocks (one per lane c) x 32 tokens (4 n-tiles). e = {Q' hi pair,
-// Q' lo pair, word offset of this lane's plane-0 word (block offset + half H), unused}.
+// One K decode group: 4 consecutive block pairs of width W whose first code starts at bit
+// `off` of this lane's token stream; kw points at word 0 of the token (word i at kw[32 i]).
 template <int W>
-__device__ __forceinline__ void qk_step(const uint32_t* kw, const uint4& e, int sh, const DecodeSmem& S,
-                                        float (&acc)[4][4]) {
-  uint32_t bf[4];
-  decode8<W>(kw + e.z, 2, sh, S, bf);
+__device__ __forceinline__ void k_group(const uint32_t* kw, uint32_t off, uint32_t taddr, const uint8_t* sm,
+                                        uint32_t lane4) {
+  const uint32_t j0 = off >> 5, s = off & 31u;
+  const uint32_t x0 = kw[j0 * 32], x1 = kw[(j0 + 1) * 32];
+  const uint32_t x2 = (W >= 5) ? kw[(j0 + 2) * 32] : 0u;
+  const uint32_t r0 = __funnelshift_r(x0, x1, s);
+  const uint32_t r1 = __funnelshift_r(x1, x2, s);
+  uint32_t v[kGroupPairs];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) mma_m16n8k8(acc[j], e.x, e.y, bf[j]);
+  for (int k = 0; k < kGroupPairs; ++k) v[k] = pair_value<W>(field(r0, r1, 2 * W * k, 2 * W), sm, lane4);
+  tc::tmem_st<kGroupPairs>(taddr, v);
 }
 
-// All k-steps of one width class.
-template <int W>
-__device__ __forceinline__ void qk_class(const uint32_t* kw, int s0, int s1, int g, int c, int sh,
-                                         const DecodeSmem& S, float (&acc)[4][4]) {
-  for (int s = s0; s < s1; ++s) qk_step<W>(kw, S.kstep[s][g][c], sh, S, acc);
+// V-hat^T row of one dim for one tile: 16 token pairs (2u, 2u+1) -> 16 columns.
+template <int BV>
+__device__ __forceinline__ void v_tile(const uint32_t* vw, uint32_t taddr, const uint8_t* sm, uint32_t lane4) {
+  uint32_t x[BV + 1];
+#pragma unroll
+  for (int i = 0; i < BV; ++i) x[i] = vw[i * kD];
+  x[BV] = 0u;
+  uint32_t v[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int p = 2 * BV * u;
+    v[u] = pair_value<BV>(field(x[p >> 5], x[(p >> 5) + 1], p & 31, 2 * BV), sm, lane4);
+  }
+  tc::tmem_st<16>(taddr, v);
 }
 
-// O += P' V over the 16 dim n-tiles for value width W.
-template <int W>
-__device__ __forceinline__ void pv_all(const uint32_t* vw, int g, int c, const uint32_t (&pa_hi)[4],
-                                       const uint32_t (&pa_lo)[4], const DecodeSmem& S, float (&o_acc)[16][4]) {
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt) {
-    uint32_t vf[4];
-    decode8<W>(vw + 8 * nt + g, kD, c, S, vf);
-    mma_m16n8k16(o_acc[nt], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], vf[0], vf[1]);
-    mma_m16n8k16(o_acc[nt], pa_hi[2], pa_lo[2], pa_hi[3], pa_lo[3], vf[2], vf[3]);
+__device__ __forceinline__ void k_group_any(int w, const uint32_t* kw, uint32_t off, uint32_t taddr,
+                                            const uint8_t* sm, uint32_t lane4) {
+  switch (w) {
+    case 1: k_group<1>(kw, off, taddr, sm, lane4); break;
+    case 2: k_group<2>(kw, off, taddr, sm, lane4); break;
+    case 3: k_group<3>(kw, off, taddr, sm, lane4); break;
+    case 4: k_group<4>(kw, off, taddr, sm, lane4); break;
+    case 5: k_group<5>(kw, off, taddr, sm, lane4); break;
+    case 6: k_group<6>(kw, off, taddr, sm, lane4); break;
+    case 7: k_group<7>(kw, off, taddr, sm, lane4); break;
+    default: k_group<8>(kw, off, taddr, sm, lane4); break;
   }
 }
 
-__device__ __forceinline__ void decode_load_tile(uint8_t* dst, const uint8_t* src, int rec_bytes, int lane) {
-  for (int k = lane; k < rec_bytes / 16; k += 32) cp_async16(dst + 16 * k, src + 16 * k);
+__device__ __forceinline__ void v_tile_any(int bv, const uint32_t* vw, uint32_t taddr, const uint8_t* sm,
+                                           uint32_t lane4) {
+  switch (bv) {
+    case 1: v_tile<1>(vw, taddr, sm, lane4); break;
+    case 2: v_tile<2>(vw, taddr, sm, lane4); break;
+    case 3: v_tile<3>(vw, taddr, sm, lane4); break;
+    case 4: v_tile<4>(vw, taddr, sm, lane4); break;
+    case 5: v_tile<5>(vw, taddr, sm, lane4); break;
+    case 6: v_tile<6>(vw, taddr, sm, lane4); break;
+    case 7: v_tile<7>(vw, taddr, sm, lane4); break;
+    default: v_tile<8>(vw, taddr, sm, lane4); break;
+  }
 }
 
-// Merge n (m, l, O) partials, entries first..first+n-1 of row `bh` (row pitch `pitch` entries,
-// 8 head rows per entry), in entry order: M = max m, L = sum l 2^(m - M),
-// O = sum O 2^(m - M). Writes either the merged partial to entry `dst` or, when `out` is
-// non-null, out = O / L for the G real heads. Needs all threads of the CTA (256 or 512).
-__device__ __forceinline__ void merge_partials(DecodeSmem& S, uint8_t* scratch, int bh, int pitch, int first, int n,
+// Order-preserving map of fp32 to int32 (and back: the map is its own inverse).
+__device__ __forceinline__ int ordered(float x) {
+  const int i = __float_as_int(x);
+  return i ^ ((i >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float from_ordered(int i) { return __int_as_float(i ^ ((i >> 31) & 0x7fffffff)); }
+
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+__device__ __forceinline__ void record_timeout(unsigned* status) { atomicCAS(status, 0u, static_cast<unsigned>(KVQ_ERR_TIMEOUT)); }
+
+// ---------------------------------------------------------------- cross-split merge
+
+// Merge the (m, l, O) partials first .. first+n-1 of (sequence, KV head) bh: into entry dst
+// of the workspace (out == nullptr) or into out = O / l for the G real query heads. Called
+// by every thread of the CTA; the 16 compute warps do the work.
+__device__ __forceinline__ void merge_partials(DecHeader& S, uint8_t* scratch, int bh, int pitch, int first, int n,
                                                float* part_m, float* part_l, float* part_o, int dst, float* out,
                                                int G) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int hg = warp; hg < 8; hg += kDecWarps) {
+  if (warp < 8) {
+    const int hg = warp;
     const size_t p0 = (static_cast<size_t>(bh) * pitch + first) * 8 + hg;
     float M = -INFINITY;
     for (int s = lane; s < n; s += 32) M = fmaxf(M, __ldcg(part_m + p0 + static_cast<size_t>(s) * 8));
@@ -192,29 +213,27 @@ __device__ __forceinline__ void merge_partials(DecodeSmem& S, uint8_t* scratch, 
     }
   }
   __syncthreads();
-  // O: 256 (head, 4-dim) quads; with 512 threads two threads share a quad (halves of the
-  // member list), with 256 threads one thread does all members.
-  const int halves = blockDim.x >> 8;
+  // O: 256 (head, 4-dim) quads; threads 0..255 and 256..511 take halves of the member list.
   const int quad = tid & 255, half = tid >> 8;
   const int hg = quad >> 5, j4 = quad & 31;
-  const int s_mid = (halves == 2) ? n / 2 : n;
-  const int s0 = half ? s_mid : 0, s1 = half ? n : s_mid;
+  const int s_mid = n / 2;
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4* po = reinterpret_cast<const float4*>(part_o);
+  if (half < 2) {
+    const int s0 = half ? s_mid : 0, s1 = half ? n : s_mid;
+    const float4* po = reinterpret_cast<const float4*>(part_o);
 #pragma unroll 4
-  for (int s = s0; s < s1; ++s) {
-    const float wt = S.mw[hg][s];
-    const float4 v = __ldcg(po + ((static_cast<size_t>(bh) * pitch + first + s) * 8 + hg) * (kD / 4) + j4);
-    o.x += v.x * wt; o.y += v.y * wt; o.z += v.z * wt; o.w += v.w * wt;
+    for (int s = s0; s < s1; ++s) {
+      const float wt = S.mw[hg][s];
+      const float4 v = __ldcg(po + ((static_cast<size_t>(bh) * pitch + first + s) * 8 + hg) * (kD / 4) + j4);
+      o.x += v.x * wt; o.y += v.y * wt; o.z += v.z * wt; o.w += v.w * wt;
+    }
   }
   float4* red = reinterpret_cast<float4*>(scratch);
-  if (half) red[quad] = o;
+  if (half == 1) red[quad] = o;
   __syncthreads();
-  if (!half) {
-    if (halves == 2) {
-      const float4 v = red[quad];
-      o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
-    }
+  if (half == 0) {
+    const float4 v = red[quad];
+    o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
     if (out != nullptr) {
       if (hg < G) {
         const float inv = 1.0f / S.Lsum[hg];
@@ -230,268 +249,365 @@ __device__ __forceinline__ void merge_partials(DecodeSmem& S, uint8_t* scratch, 
       }
     }
   }
+  __syncthreads();
 }
 
+// ---------------------------------------------------------------- the kernel
+
 template <int DT>
-__global__ void __launch_bounds__(kDecWarps * 32) kvq_decode_gtq(
+__global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
     const typename Elem<DT>::T* __restrict__ q, int64_t qsb, int64_t qsh, int n_q_heads, int n_kv_heads,
-    const uint8_t* __restrict__ packed, const kvq_head_alloc* __restrict__ alloc, int tiles_cap,
-    int rec_bytes, int bits_v, int seq_len, int splits, int n_groups, int n_stages, float* __restrict__ out,
+    const uint8_t* __restrict__ packed, const kvq_head_alloc* __restrict__ alloc, int tiles_cap, int rec_bytes,
+    int bits_k, int bits_v, int seq_len, int splits, int n_groups, int n_stages, float* __restrict__ out,
     float* __restrict__ part_m, float* __restrict__ part_l, float* __restrict__ part_o,
-    unsigned* __restrict__ tickets) {
-  extern __shared__ __align__(16) uint8_t dsmem[];
-  DecodeSmem& S = *reinterpret_cast<DecodeSmem*>(dsmem);
-  uint8_t* stages = dsmem + ((sizeof(DecodeSmem) + 127) / 128) * 128;
+    unsigned* __restrict__ tickets, unsigned* __restrict__ status) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  DecHeader& S = *reinterpret_cast<DecHeader*>(sm + kHdrOff);
+  uint8_t* stages = sm + decode_stage_off();
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, c = lane & 3;
   const int split = blockIdx.x, bh = blockIdx.y;
   const int b = bh / n_kv_heads, hkv = bh % n_kv_heads;
   const int G = n_q_heads / n_kv_heads;
   const kvq_head_alloc* al = alloc + hkv;
-  const int k_words = al->k_words;
   // An allocation made for another budget does not match the record size: write nothing.
-  if (4 * (k_words + bits_v * kD) + 4 * kTile != rec_bytes) return;
+  if (al->k_words != bits_k * kD || al->bits_k != bits_k) return;
   const int n_tiles = (seq_len + kTile - 1) / kTile;
-  const int t_begin = static_cast<int>((static_cast<long long>(split) * n_tiles) / splits);
-  const int t_end = static_cast<int>((static_cast<long long>(split + 1) * n_tiles) / splits);
+  const int n_chunks_all = (n_tiles + kChunkTiles - 1) / kChunkTiles;
+  const int c_begin = static_cast<int>((static_cast<long long>(split) * n_chunks_all) / splits);
+  const int c_end = static_cast<int>((static_cast<long long>(split + 1) * n_chunks_all) / splits);
+  const int n_chunks = c_end - c_begin;
+  const int tile_end = min(n_tiles, c_end * kChunkTiles);
+  const uint8_t* src = packed + static_cast<size_t>(bh) * tiles_cap * rec_bytes;
+  const int stage_bytes = kChunkTiles * rec_bytes;
   const float inv_sqrt_d = 0.08838834764831845f;
 
-  const int stage_bytes = ((rec_bytes + 127) / 128) * 128;
-  uint8_t* my_stages = stages + warp * n_stages * stage_bytes;
-  const uint8_t* src_base = packed + static_cast<size_t>(bh) * tiles_cap * rec_bytes;
-  const int first = t_begin + warp;
-  const int my_n = (first < t_end) ? (t_end - first + kDecWarps - 1) / kDecWarps : 0;
-  // Start streaming the first tiles before the prologue.
-  for (int i = 0; i < n_stages - 1; ++i) {
-    if (i < my_n)
-      decode_load_tile(my_stages + i * stage_bytes, src_base + static_cast<size_t>(first + i * kDecWarps) * rec_bytes,
-                       rec_bytes, lane);
-    cp_async_commit();
+  // ------------------------------------------------------------------ setup
+  if (tid == 0) {
+    for (int i = 0; i < kDecStagesMax; ++i) {
+      tc::mbar_init(&S.full[i], 1);
+      tc::mbar_init(&S.empty[i], kDecComputeWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&S.kready[i], kDecComputeWarps);
+      tc::mbar_init(&S.vready[i], kDecComputeWarps);
+      tc::mbar_init(&S.pready[i], kDecComputeWarps);
+      tc::mbar_init(&S.sfull[i], 1);
+      tc::mbar_init(&S.ofull[i], 1);
+    }
+    tc::mbar_fence_init();
   }
-
-  // ------------------------------------------------------------------ prologue
-  for (int i = tid; i < kCentroidCount; i += blockDim.x) S.cent[i] = c_tab.centroid_f16[i];
-  if (tid < 4) {
-    uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
-    if (tid >= 1) {
-      for (int e = 0; e < (1 << tid); ++e) {
-        const uint32_t c16 = c_tab.centroid_f16[(1 << tid) - 2 + e];
-        lo[e >> 2] |= (c16 & 0xffu) << (8 * (e & 3));
-        hi[e >> 2] |= (c16 >> 8) << (8 * (e & 3));
+  if (warp == kDecMmaWarp) tc::tmem_alloc(&S.tmem_base, kTmemCols);
+  uint16_t* cent = reinterpret_cast<uint16_t*>(sm + kCentOff);
+  for (int i = tid; i < kCentroidCount; i += blockDim.x) cent[i] = c_tab.centroid_f16[i];
+  // K columns: classes in stream order, each padded to whole groups of 4 block pairs.
+  if (tid == 0) {
+    int col = 0, ng = 0;
+    uint32_t groups[kMaxKGroups];
+    for (int i = 0; i < 128; ++i) S.col_block[i] = -1;
+    const int n_cls = min(max(al->n_classes, 0), 8);
+    for (int c = 0; c < n_cls; ++c) {
+      const int w = al->class_width[c], first = al->class_first[c], nb = al->class_blocks[c];
+      const int bit = al->class_bit[c];
+      for (int k0 = 0; k0 < nb && ng < kMaxKGroups; k0 += kGroupPairs) {
+        groups[ng++] = static_cast<uint32_t>(w) | (static_cast<uint32_t>(bit + 2 * w * k0) << 4) |
+                       (static_cast<uint32_t>(col) << 16);
+        for (int k = 0; k < kGroupPairs && k0 + k < nb; ++k) S.col_block[col + k] = static_cast<int8_t>(al->stream_block[first + k0 + k]);
+        col += kGroupPairs;
       }
     }
-    S.lut8[tid] = make_uint4(lo[0], lo[1], hi[0], hi[1]);
-  } else if (tid == 4) {
-    uint32_t lo[4] = {0u, 0u, 0u, 0u}, hi[4] = {0u, 0u, 0u, 0u};
-    for (int e = 0; e < 16; ++e) {
-      const uint32_t c16 = c_tab.centroid_f16[14 + e];
-      lo[e >> 2] |= (c16 & 0xffu) << (8 * (e & 3));
-      hi[e >> 2] |= (c16 >> 8) << (8 * (e & 3));
+    S.k_cols = (col + 7) & ~7;
+    // Balance the groups over the 4 warp groups (cost: 1 per pair lookup, 2 for the
+    // single-code widths 7 and 8, plus the word loads).
+    int load[4] = {0, 0, 0, 0};
+    for (int g = 0; g < 4; ++g) S.n_kgroups[g] = 0;
+    for (int i = 0; i < ng; ++i) {
+      const int w = groups[i] & 15;
+      const int cost = kGroupPairs * (w >= 7 ? 2 : 1) + 2 + (w >= 5 ? 1 : 0);
+      int best = 0;
+      for (int g = 1; g < 4; ++g)
+        if (load[g] < load[best]) best = g;
+      load[best] += cost;
+      S.kgroup[best][S.n_kgroups[best]++] = groups[i];
     }
-    S.lut16[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    S.lut16[1] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
   }
-  for (int i = tid; i < kH; i += blockDim.x) S.woff[i] = al->word_off[i];
-  for (int i = tid; i < kMaxSteps * 4; i += blockDim.x) S.step_blk[i >> 2][i & 3] = al->step_block[i >> 2][i & 3];
-  for (int i = tid; i < kMaxSteps; i += blockDim.x) S.step_w[i] = al->step_width[i];
-  if (tid == 0) S.n_steps = min(max(al->n_steps, 0), kMaxSteps);
+  __syncthreads();
+  // Lookup tables.
+  for (int w = 1; w <= 3; ++w) {
+    const int n = 1 << (2 * w);
+    uint32_t* t = reinterpret_cast<uint32_t*>(sm + lut_off(w));
+    for (int i = tid; i < n * 32; i += blockDim.x) {
+      const int e = i >> 5;
+      const uint16_t* c = cent + ((1 << w) - 2);
+      t[i] = static_cast<uint32_t>(c[e & ((1 << w) - 1)]) | (static_cast<uint32_t>(c[e >> w]) << 16);
+    }
+  }
+  for (int w = 4; w <= 6; ++w) {
+    const int n = 1 << (2 * w);
+    uint32_t* t = reinterpret_cast<uint32_t*>(sm + lut_off(w));
+    const uint16_t* c = cent + ((1 << w) - 2);
+    for (int e = tid; e < n; e += blockDim.x)
+      t[e] = static_cast<uint32_t>(c[e & ((1 << w) - 1)]) | (static_cast<uint32_t>(c[e >> w]) << 16);
+  }
+  for (int w = 7; w <= 8; ++w) {
+    uint16_t* t = reinterpret_cast<uint16_t*>(sm + lut_off(w));
+    for (int e = tid; e < (1 << w); e += blockDim.x) t[e] = cent[(1 << w) - 2 + e];
+  }
+  // Q' rows: q_h * f_b * log2(e) / sqrt(d), scaled per row by 2^-e so the largest |Q'| is in
+  // [0.5, 1); the MMA result is multiplied back by qscale[h] = 2^e.
+  float* qtmp = reinterpret_cast<float*>(stages);   // [8][128] fp32, before the stages are used
   for (int i = tid; i < 8 * kD; i += blockDim.x) {
     const int hg = i / kD, j = i % kD;
     float v = 0.0f;
-    if (hg < G) {
-      const float qv = Elem<DT>::to_f32(q[b * qsb + (hkv * G + hg) * qsh + j]);
-      v = qv * al->dequant[j % kH] * (inv_sqrt_d * kLog2e);
-    }
-    S.qp[hg][j] = v;
+    if (hg < G) v = Elem<DT>::to_f32(q[b * qsb + (hkv * G + hg) * qsh + j]) * al->dequant[j % kH] * (inv_sqrt_d * kLog2e);
+    qtmp[i] = v;
   }
   __syncthreads();
-  // per-head power-of-two scaling so the largest |Q'| lies in [0.5, 1)
-  for (int hg = warp; hg < 8; hg += kDecWarps) {
+  if (warp < 8) {
+    const int hg = warp;
     float mx = 0.0f;
-    for (int j = lane; j < kD; j += 32) mx = fmaxf(mx, fabsf(S.qp[hg][j]));
+    for (int j = lane; j < kD; j += 32) mx = fmaxf(mx, fabsf(qtmp[hg * kD + j]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     int e = 0;
     if (mx > 0.0f) frexpf(mx, &e);
-    if (lane == 0) S.qmul[hg] = ldexpf(1.0f, e);
+    if (lane == 0) S.qscale[hg] = ldexpf(1.0f, e);
     const float sc = ldexpf(1.0f, -e);
-    for (int j = lane; j < kD; j += 32) S.qp[hg][j] *= sc;
+    for (int j = lane; j < kD; j += 32) qtmp[hg * kD + j] *= sc;
   }
   __syncthreads();
-  const int n_steps = S.n_steps;
-  for (int i = tid; i < n_steps * 32; i += blockDim.x) {
-    const int st = i >> 5, hg = (i >> 2) & 7, cc = i & 3;
-    const int blk = S.step_blk[st][cc];
-    uint4 e = make_uint4(0u, 0u, 0u, 0u);
-    int wblk = blk;
-    if (blk >= 0 && blk < kH) {
-      __half h1, l1, h2, l2;
-      split_hilo(S.qp[hg][blk], h1, l1);
-      split_hilo(S.qp[hg][blk + kH], h2, l2);
-      e.x = pack_half2(h1, h2);
-      e.y = pack_half2(l1, l2);
-    } else {
-      wblk = max(static_cast<int>(S.step_blk[st][0]), 0);   // empty slot: Q' is 0, read any valid block
+  // B operand of S, K-major, no swizzle: element (n, k) at (k/8)*256 + (n/8)*128 + (n%8)*16 + (k%8)*2;
+  // K element k = 2c + r is dim b + 64 r of the block in column c; n < 8: hi part of row n,
+  // n >= 8: lo part of row n - 8.
+  {
+    const int k_elems = 2 * S.k_cols;
+    for (int i = tid; i < 8 * k_elems; i += blockDim.x) {
+      const int n = i / k_elems, k = i % k_elems;
+      const int blk = S.col_block[k >> 1];
+      __half hi = __float2half_rn(0.0f), lo = hi;
+      if (blk >= 0) split_hilo(qtmp[n * kD + blk + kH * (k & 1)], hi, lo);
+      const int base = (k >> 3) * 256 + (k & 7) * 2;
+      *reinterpret_cast<__half*>(sm + kBQOff + base + n * 16) = hi;
+      *reinterpret_cast<__half*>(sm + kBQOff + base + 128 + n * 16) = lo;
     }
-    e.z = static_cast<uint32_t>(S.woff[min(wblk, kH - 1)]) + (hg >> 2);   // lane (hg, cc) uses half H = hg / 4
-    S.kstep[st][hg][cc] = e;
   }
-  if (tid == 0) {
-    int n = 0;
-    for (int st = 0; st < n_steps; ++st) {
-      const int w = min(max(static_cast<int>(S.step_w[st]), 1), 8);
-      if (n == 0 || S.cls_w[n - 1] != w) {
-        S.cls_w[n] = w;
-        S.cls_begin[n] = st;
-        ++n;
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = S.tmem_base;
+
+  if (warp == kDecLoadWarp) {
+    // ---------------------------------------------------------------- bulk loads
+    if (lane == 0) {
+      for (int i = 0; i < n_chunks; ++i) {
+        const int s = i % n_stages;
+        if (i >= n_stages && !tc::mbar_wait(&S.empty[s], ((i / n_stages) - 1) & 1, kWaitLimit)) {
+          record_timeout(status);
+          break;
+        }
+        const int tile0 = (c_begin + i) * kChunkTiles;
+        const int nt = min(kChunkTiles, tile_end - tile0);
+        const uint32_t bytes = static_cast<uint32_t>(nt * rec_bytes);
+        tc::mbar_arrive_expect_tx(&S.full[s], bytes);
+        tc::bulk_g2s(stages + s * stage_bytes, src + static_cast<size_t>(tile0) * rec_bytes, bytes, &S.full[s]);
       }
     }
-    S.cls_begin[n] = n_steps;
-    S.n_cls = n;
-  }
-  __syncthreads();
-
-  // ------------------------------------------------------------------ main loop
-  const float qmul = S.qmul[g];
-  float m_run = -INFINITY, l_run = 0.0f;
-  float o_acc[16][4];
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt) o_acc[nt][0] = o_acc[nt][1] = o_acc[nt][2] = o_acc[nt][3] = 0.0f;
-
-  const int sh = g & 3;
-  for (int i = 0; i < my_n; ++i) {
+  } else if (warp == kDecMmaWarp) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      const uint32_t id_s = tc::idesc_f16(128, 16, false), id_o = tc::idesc_f16(128, 16, true);
+      const uint32_t bq = tc::smem_u32(sm + kBQOff), bp = tc::smem_u32(sm + kBPOff);
+      const int ksteps = S.k_cols / 8;
+      bool ok = true;
+      for (int i = 0; i <= n_chunks && ok; ++i) {
+        if (i < n_chunks) {
+          const int bb = i & 1;
+          if (!tc::mbar_wait(&S.kready[bb], (i >> 1) & 1, kWaitLimit)) { ok = false; break; }
+          tc::fence_after_sync();
+          for (int ks = 0; ks < ksteps; ++ks)
+            tc::mma_ts(tbase + col_s(bb), tbase + col_ak(bb) + 8 * ks, tc::sdesc(bq + 512 * ks, 256, 128), id_s,
+                       ks > 0);
+          tc::mma_commit(&S.sfull[bb]);
+        }
+        if (i >= 1) {
+          const int j = i - 1, bj = j & 1;
+          if (!tc::mbar_wait(&S.pready[bj], (j >> 1) & 1, kWaitLimit) ||
+              !tc::mbar_wait(&S.vready[bj], (j >> 1) & 1, kWaitLimit)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          for (int ks = 0; ks < kChunkTokens / 16; ++ks)
+            tc::mma_ts(tbase + col_o(bj), tbase + col_av(bj) + 8 * ks,
+                       tc::sdesc(bp + kBPBytes * bj + 512 * ks, 256, 128), id_o, ks > 0);
+          tc::mma_commit(&S.ofull[bj]);
+        }
+      }
+      if (!ok) record_timeout(status);
+    }
+  } else {
+    // ---------------------------------------------------------------- compute warps
+    const int wg = warp >> 2, qt = warp & 3;                // warp group, tensor-memory quarter
+    const uint32_t lane_base = static_cast<uint32_t>(32 * qt) << 16;
+    const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
+    const int ngk = S.n_kgroups[wg];
+    const uint32_t* kg = S.kgroup[wg];
+    const int norm_off = 4 * kD * (bits_k + bits_v);
+    const float qs0 = S.qscale[2 * wg], qs1 = S.qscale[2 * wg + 1];
+    // Zero both K buffers once: columns past the last group stay zero (their Q' is 0 too).
     {
-      const int nxt = i + n_stages - 1;
-      if (nxt < my_n)
-        decode_load_tile(my_stages + (nxt % n_stages) * stage_bytes,
-                         src_base + static_cast<size_t>(first + nxt * kDecWarps) * rec_bytes, rec_bytes, lane);
-      cp_async_commit();
+      uint32_t z[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) z[i] = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tc::tmem_st<16>(tbase + lane_base + 64 * wg + 16 * i, z);
     }
-    cp_async_wait_pending(n_stages - 1);
-    __syncwarp();
-    const int tile = first + i * kDecWarps;
-    const uint8_t* st = my_stages + (i % n_stages) * stage_bytes;
-    const uint32_t* kw = reinterpret_cast<const uint32_t*>(st);
-    const uint32_t* vw = kw + k_words;
-    const uint16_t* kn = reinterpret_cast<const uint16_t*>(vw + bits_v * kD);
-    const uint16_t* vn = kn + kTile;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f, o0 = 0.0f, o1 = 0.0f;
+    float al00 = 0.0f, al01 = 0.0f, al10 = 0.0f, al11 = 0.0f;   // alpha[parity][query]
+    float kn_prev = 0.0f, vn_prev = 0.0f;
+    bool ok = true;
 
-    // ---- S^T = Q' K^T over the k-steps
-    float acc[4][4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-    for (int ci = 0; ci < S.n_cls; ++ci) {
-      const int s0 = S.cls_begin[ci], s1 = S.cls_begin[ci + 1];
-      switch (S.cls_w[ci]) {
-        case 1: qk_class<1>(kw, s0, s1, g, c, sh, S, acc); break;
-        case 2: qk_class<2>(kw, s0, s1, g, c, sh, S, acc); break;
-        case 3: qk_class<3>(kw, s0, s1, g, c, sh, S, acc); break;
-        case 4: qk_class<4>(kw, s0, s1, g, c, sh, S, acc); break;
-        case 5: qk_class<5>(kw, s0, s1, g, c, sh, S, acc); break;
-        case 6: qk_class<6>(kw, s0, s1, g, c, sh, S, acc); break;
-        case 7: qk_class<7>(kw, s0, s1, g, c, sh, S, acc); break;
-        default: qk_class<8>(kw, s0, s1, g, c, sh, S, acc); break;
+    auto softmax = [&](int j, float kn, float vn) {
+      const int bj = j & 1;
+      if (ok && !tc::mbar_wait(&S.sfull[bj], (j >> 1) & 1, kWaitLimit)) ok = false;
+      tc::fence_after_sync();
+      uint32_t sh[2], sl[2];
+      tc::tmem_ld<2>(tbase + lane_base + col_s(bj) + 2 * wg, sh);
+      tc::tmem_ld<2>(tbase + lane_base + col_s(bj) + 8 + 2 * wg, sl);
+      tc::wait_ld();
+      const int tile = (c_begin + j) * kChunkTiles + qt;
+      const int tok = tile * kTile + lane;
+      const bool valid = tile < tile_end && tok < seq_len;
+      float s0 = (__uint_as_float(sh[0]) + __uint_as_float(sl[0])) * (kn * qs0);
+      float s1 = (__uint_as_float(sh[1]) + __uint_as_float(sl[1])) * (kn * qs1);
+      if (!valid) { s0 = -INFINITY; s1 = -INFINITY; }
+      const int k0 = __reduce_max_sync(0xffffffffu, ordered(s0));
+      const int k1 = __reduce_max_sync(0xffffffffu, ordered(s1));
+      if (lane == 0) {
+        S.xmax[bj][wg][qt][0] = from_ordered(k0);
+        S.xmax[bj][wg][qt][1] = from_ordered(k1);
       }
-    }
+      named_sync(1 + wg, 128);
+      float c0 = S.xmax[bj][wg][0][0], c1 = S.xmax[bj][wg][0][1];
+#pragma unroll
+      for (int u = 1; u < 4; ++u) {
+        c0 = fmaxf(c0, S.xmax[bj][wg][u][0]);
+        c1 = fmaxf(c1, S.xmax[bj][wg][u][1]);
+      }
+      const float n0 = fmaxf(m0, c0), n1 = fmaxf(m1, c1);
+      const float a0 = (m0 == -INFINITY) ? 0.0f : fast_exp2(m0 - n0);
+      const float a1 = (m1 == -INFINITY) ? 0.0f : fast_exp2(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      const float p0 = valid ? fast_exp2(s0 - n0) : 0.0f;
+      const float p1 = valid ? fast_exp2(s1 - n1) : 0.0f;
+      l0 = l0 * a0 + p0;
+      l1 = l1 * a1 + p1;
+      const float vs = valid ? vn * inv_sqrt_d : 0.0f;
+      __half h0, lo0, h1, lo1;
+      split_hilo(p0 * vs, h0, lo0);
+      split_hilo(p1 * vs, h1, lo1);
+      const int t = 32 * qt + lane;
+      uint8_t* pb = sm + kBPOff + kBPBytes * bj + (t >> 3) * 256 + (t & 7) * 16 + 4 * wg;
+      *reinterpret_cast<uint32_t*>(pb) = pack_half2(h0, h1);
+      *reinterpret_cast<uint32_t*>(pb + 128) = pack_half2(lo0, lo1);
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&S.pready[bj]);
+      if (bj) { al10 = a0; al11 = a1; } else { al00 = a0; al01 = a1; }
+    };
 
-    // ---- online softmax over the 8 tokens this lane holds: 8j + 2c + {0,1}
-    float sv[4][2];
-    float tmax = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int tt = 8 * j + 2 * c + u;
-        const float nk = __half2float(__ushort_as_half(kn[tt]));
-        float sval = (acc[j][u] + acc[j][u + 2]) * nk * qmul;
-        if (tile * kTile + tt >= seq_len) sval = -INFINITY;
-        sv[j][u] = sval;
-        tmax = fmaxf(tmax, sval);
-      }
-    }
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-    const float m_new = fmaxf(m_run, tmax);
-    const float alpha = (m_run == -INFINITY) ? 0.0f : fast_exp2(m_run - m_new);
-    m_run = m_new;
-    l_run *= alpha;
-    if (!__all_sync(0xffffffffu, alpha == 1.0f)) {
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        o_acc[nt][0] *= alpha; o_acc[nt][1] *= alpha; o_acc[nt][2] *= alpha; o_acc[nt][3] *= alpha;
-      }
-    }
-    uint32_t pa_hi[4], pa_lo[4];   // per n-tile j: packed (token 8j+2c, 8j+2c+1)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      __half hh[2], ll[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int tt = 8 * j + 2 * c + u;
-        const float p = (sv[j][u] == -INFINITY) ? 0.0f : fast_exp2(sv[j][u] - m_new);
-        l_run += p;
-        const float pv = p * __half2float(__ushort_as_half(vn[tt])) * inv_sqrt_d;
-        split_hilo(pv, hh[u], ll[u]);
-      }
-      pa_hi[j] = pack_half2(hh[0], hh[1]);
-      pa_lo[j] = pack_half2(ll[0], ll[1]);
-    }
+    auto o_acc = [&](int j) {
+      const int bj = j & 1;
+      if (ok && !tc::mbar_wait(&S.ofull[bj], (j >> 1) & 1, kWaitLimit)) ok = false;
+      tc::fence_after_sync();
+      uint32_t oh[2], ol[2];
+      tc::tmem_ld<2>(tbase + lane_base + col_o(bj) + 2 * wg, oh);
+      tc::tmem_ld<2>(tbase + lane_base + col_o(bj) + 8 + 2 * wg, ol);
+      tc::wait_ld();
+      const float a0 = bj ? al10 : al00, a1 = bj ? al11 : al01;
+      o0 = o0 * a0 + (__uint_as_float(oh[0]) + __uint_as_float(ol[0]));
+      o1 = o1 * a1 + (__uint_as_float(oh[1]) + __uint_as_float(ol[1]));
+    };
 
-    // ---- O += P' Vhat over 16 dim n-tiles, two 16-token k-steps
-    switch (bits_v) {
-      case 1: pv_all<1>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
-      case 2: pv_all<2>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
-      case 3: pv_all<3>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
-      case 4: pv_all<4>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
-      case 5: pv_all<5>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
-      case 6: pv_all<6>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
-      case 7: pv_all<7>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
-      default: pv_all<8>(vw, g, c, pa_hi, pa_lo, S, o_acc); break;
+    for (int i = 0; i < n_chunks; ++i) {
+      const int bb = i & 1, s = i % n_stages;
+      if (ok && !tc::mbar_wait(&S.full[s], (i / n_stages) & 1, kWaitLimit)) ok = false;
+      const uint8_t* st = stages + s * stage_bytes;
+      // K-hat rows: token 32 qt + lane = token `lane` of tile qt.
+      {
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(st + qt * rec_bytes) + lane;
+        const uint32_t ta = tbase + lane_base + col_ak(bb);
+        for (int gi = 0; gi < ngk; ++gi) {
+          const uint32_t g = kg[gi];
+          k_group_any(static_cast<int>(g & 15u), kw, (g >> 4) & 0xfffu, ta + (g >> 16), sm, lane4);
+        }
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&S.kready[bb]);
+      if (i >= 2) o_acc(i - 2);          // also frees A_V, P' and O of this parity
+      // V-hat^T rows: dim 32 qt + lane, tokens of tile wg -> columns 16 wg .. 16 wg + 15.
+      {
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(st + wg * rec_bytes + 4 * kD * bits_k) + 32 * qt + lane;
+        v_tile_any(bits_v, vw, tbase + lane_base + col_av(bb) + 16 * wg, sm, lane4);
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      const uint16_t* nrm = reinterpret_cast<const uint16_t*>(st + qt * rec_bytes + norm_off);
+      const float kn = __half2float(__ushort_as_half(nrm[lane]));
+      const float vn = __half2float(__ushort_as_half(nrm[kTile + lane]));
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(&S.vready[bb]);
+        tc::mbar_arrive(&S.empty[s]);
+      }
+      if (i >= 1) softmax(i - 1, kn_prev, vn_prev);
+      kn_prev = kn;
+      vn_prev = vn;
     }
-    __syncwarp();
-  }
-  cp_async_wait_pending(0);
+    if (n_chunks >= 1) softmax(n_chunks - 1, kn_prev, vn_prev);
+    if (n_chunks >= 2) o_acc(n_chunks - 2);
+    if (n_chunks >= 1) o_acc(n_chunks - 1);
+    if (!ok) record_timeout(status);
 
-  // ------------------------------------------------------------------ combine warps
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  __syncthreads();
-  float* cm = reinterpret_cast<float*>(stages);                  // [4][8]
-  float* cl = cm + kDecWarps * 8;                                 // [4][8]
-  float* co = cl + kDecWarps * 8;                                 // [4][8][128]
-  if (c == 0) {
-    cm[warp * 8 + g] = m_run;
-    cl[warp * 8 + g] = l_run;
-  }
+    // ---------------------------------------------------------------- CTA result
 #pragma unroll
-  for (int nt = 0; nt < 16; ++nt) {
-    co[(warp * 8 + g) * kD + 8 * nt + 2 * c] = o_acc[nt][0] + o_acc[nt][2];
-    co[(warp * 8 + g) * kD + 8 * nt + 2 * c + 1] = o_acc[nt][1] + o_acc[nt][3];
-  }
-  __syncthreads();
-  for (int i = tid; i < 8 * kD; i += blockDim.x) {
-    const int hg = i / kD, j = i % kD;
-    float M = -INFINITY;
-    for (int wv = 0; wv < kDecWarps; ++wv) M = fmaxf(M, cm[wv * 8 + hg]);
-    float L = 0.0f, O = 0.0f;
-    for (int wv = 0; wv < kDecWarps; ++wv) {
-      const float mw = cm[wv * 8 + hg];
-      const float wt = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - M);
-      L += cl[wv * 8 + hg] * wt;
-      O += co[(wv * 8 + hg) * kD + j] * wt;
+    for (int o = 16; o > 0; o >>= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
+    if (lane == 0) {
+      S.lpart[wg][qt][0] = l0;
+      S.lpart[wg][qt][1] = l1;
+    }
+    named_sync(1 + wg, 128);
+    const float L0 = S.lpart[wg][0][0] + S.lpart[wg][1][0] + S.lpart[wg][2][0] + S.lpart[wg][3][0];
+    const float L1 = S.lpart[wg][0][1] + S.lpart[wg][1][1] + S.lpart[wg][2][1] + S.lpart[wg][3][1];
+    const int d = 32 * qt + lane;
+    const int h0 = 2 * wg, h1 = 2 * wg + 1;
     if (splits == 1) {
-      if (hg < G) out[(static_cast<size_t>(b) * n_q_heads + hkv * G + hg) * kD + j] = O / L;
+      float* ob = out + (static_cast<size_t>(b) * n_q_heads + hkv * G) * kD;
+      if (h0 < G) ob[h0 * kD + d] = o0 / L0;
+      if (h1 < G) ob[h1 * kD + d] = o1 / L1;
     } else {
-      const size_t pb = (static_cast<size_t>(bh) * (splits + n_groups) + split) * 8 + hg;
-      part_o[pb * kD + j] = O;
-      if (j == 0) {
-        part_m[pb] = M;
-        part_l[pb] = L;
+      const size_t pb0 = (static_cast<size_t>(bh) * (splits + n_groups) + split) * 8;
+      part_o[(pb0 + h0) * kD + d] = o0;
+      part_o[(pb0 + h1) * kD + d] = o1;
+      if (d == 0) {
+        part_m[pb0 + h0] = m0;
+        part_l[pb0 + h0] = L0;
+        part_m[pb0 + h1] = m1;
+        part_l[pb0 + h1] = L1;
       }
     }
   }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == kDecMmaWarp) tc::tmem_dealloc(tbase, kTmemCols);
   if (splits == 1) return;
 
   // ------------------------------------------------------------------ cross-split merge

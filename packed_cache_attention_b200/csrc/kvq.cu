@@ -78,6 +78,13 @@ int decode_splits(int bh, int n_tiles) {
   return std::max(1, std::min(std::min(want, n_tiles), kMaxMergeSplits));
 }
 
+// Block-GTQ decode: splits of whole 128-token chunks, about one CTA per SM in total.
+int gtq_splits(int bh, int n_tiles) {
+  const int n_chunks = (n_tiles + kChunkTiles - 1) / kChunkTiles;
+  const int want = (kTargetCtas + bh - 1) / bh;
+  return std::max(1, std::min(std::min(want, n_chunks), kMaxMergeSplits));
+}
+
 struct DecodeWs {
   size_t tickets, part_m, part_l, part_o, total;
 };
@@ -128,19 +135,17 @@ Nf4Layout nf4_layout(int batch, int n_heads, int capacity) {
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
-size_t decode_head_bytes() { return align_up(sizeof(DecodeSmem), 128); }
-size_t decode_combine_bytes() { return sizeof(float) * (kDecWarps * 8 * 2 + kDecWarps * 8 * kD); }
-
-// Deepest cp.async pipeline (1..3 tile records per warp) that fits in shared memory.
+// Deepest bulk-copy pipeline (1..4 chunks of 4 tile records) that fits in shared memory.
 int decode_stages(int rec_bytes) {
-  const size_t per = align_up(rec_bytes, 128) * kDecWarps;
-  const size_t room = kMaxSmem - decode_head_bytes();
-  return static_cast<int>(std::max<size_t>(1, std::min<size_t>(kDecStages, room / per)));
+  const size_t per = static_cast<size_t>(kChunkTiles) * rec_bytes;
+  const size_t room = kMaxSmem - decode_stage_off();
+  return static_cast<int>(std::max<size_t>(1, std::min<size_t>(kDecStagesMax, room / per)));
 }
 
 size_t decode_smem_bytes(int rec_bytes) {
-  const size_t stage = align_up(rec_bytes, 128) * decode_stages(rec_bytes) * kDecWarps;
-  return decode_head_bytes() + std::max(stage, decode_combine_bytes());
+  const size_t stage = static_cast<size_t>(kChunkTiles) * rec_bytes * decode_stages(rec_bytes);
+  // the stage area also holds the Q' staging (4 KB) and the merge scratch (4 KB)
+  return decode_stage_off() + std::max<size_t>(stage, 8 * kD * sizeof(float));
 }
 
 }  // namespace
@@ -223,7 +228,7 @@ size_t kvq_packed_bytes(const kvq_cache_desc* c) {
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* c, int n_q_heads) {
   if (!cache_ok(c) || n_q_heads < 1) return 0;
   const int bh = c->batch * c->n_kv_heads;
-  return gtq_ws_layout(bh, decode_splits(bh, n_tiles_of(c->capacity))).total;
+  return gtq_ws_layout(bh, gtq_splits(bh, n_tiles_of(c->capacity))).total;
 }
 
 kvq_status kvq_init(void) { return ensure_tables(); }
@@ -304,7 +309,7 @@ kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, con
   const int tiles_cap = n_tiles_of(c->capacity);
   const long long n_tasks = static_cast<long long>(c->batch) * c->n_kv_heads * tiles_written;
   const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
-  const size_t smem = quant_smem_bytes(kd->dtype, c->bits_k, c->bits_v);
+  const size_t smem = quant_smem_bytes(kd->dtype);
   const int ctas_per_sm = static_cast<int>(std::max<size_t>(1, (227u * 1024u) / smem));
   const long long want = (n_tasks + kQuantWarps - 1) / kQuantWarps;
   const unsigned grid = static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sm_count()) * ctas_per_sm));
@@ -342,7 +347,7 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
   if (seq_len < 1 || seq_len > c->capacity) return KVQ_ERR_RANGE;
   const int bh = c->batch * c->n_kv_heads;
   const int n_tiles = n_tiles_of(seq_len);
-  const int splits = decode_splits(bh, n_tiles);
+  const int splits = gtq_splits(bh, n_tiles);
   const DecodeWs L = gtq_ws_layout(bh, splits);
   if (!ws || ws_bytes < L.total || !aligned16(ws) || ws_bytes < kvq_decode_workspace_bytes(c, qd->n_heads))
     return KVQ_ERR_WORKSPACE;
@@ -358,13 +363,13 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=            \
         cudaSuccess)                                                                                                  \
       return KVQ_ERR_CUDA;                                                                                            \
-    kern<<<grid, kDecWarps * 32, smem, s>>>(                                                                          \
+    kern<<<grid, kDecThreads, smem, s>>>(                                                                             \
         static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, c->n_kv_heads,                             \
         static_cast<const uint8_t*>(packed), static_cast<const kvq_head_alloc*>(alloc), n_tiles_of(c->capacity), rec, \
-        c->bits_v, seq_len, splits, merge_groups(splits), decode_stages(rec), out,                                    \
-        reinterpret_cast<float*>(w8 + L.part_m),                                    \
-        reinterpret_cast<float*>(w8 + L.part_l), reinterpret_cast<float*>(w8 + L.part_o),                             \
-        reinterpret_cast<unsigned*>(w8 + L.tickets));                                                                 \
+        c->bits_k, c->bits_v, seq_len, splits, merge_groups(splits), decode_stages(rec), out,                         \
+        reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_l),                            \
+        reinterpret_cast<float*>(w8 + L.part_o), reinterpret_cast<unsigned*>(w8 + L.tickets),                        \
+        reinterpret_cast<unsigned*>(w8));                                                                             \
   } while (0)
   switch (qd->dtype) {
     case KVQ_F32: KVQ_LAUNCH_DEC(KVQ_F32, float); break;
@@ -441,7 +446,7 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(splits, bh);
 #define KVQ_LAUNCH_NF4DEC(DT, TY)                                                                              \
-  kvq_nf4_decode<DT><<<grid, kDecWarps * 32, 0, s>>>(                                                          \
+  kvq_nf4_decode<DT><<<grid, kNf4DecWarps * 32, 0, s>>>(                                                          \
       static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, static_cast<const uint8_t*>(packed), L, \
       seq_len, splits, out, reinterpret_cast<float*>(w8 + Lw.part_m), reinterpret_cast<float*>(w8 + Lw.part_l),  \
       reinterpret_cast<float*>(w8 + Lw.part_o), reinterpret_cast<unsigned*>(w8 + Lw.tickets))

@@ -24,6 +24,7 @@ struct Nf4Layout {
 };
 
 constexpr int kNf4Rows = 4;   // token rows per warp task
+constexpr int kNf4DecWarps = 16;   // warps per CTA of the NF4 decode
 
 // One warp per (K-or-V, sequence, block, group of 4 token rows < T_pad). Lane l holds values
 // 8l..8l+7 of the block: head 2*blk + l/16, dims 8(l%16)..8(l%16)+7. All rows of the group
@@ -108,14 +109,14 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
 // warp every 4th 32-token group of the CTA's range. Q.K: lane t scores token t of the
 // group from its 64 code bytes; P.V: lane l accumulates dims 4l..4l+3 over the group.
 template <int DT>
-__global__ void __launch_bounds__(kDecWarps * 32) kvq_nf4_decode(
+__global__ void __launch_bounds__(kNf4DecWarps * 32) kvq_nf4_decode(
     const typename Elem<DT>::T* __restrict__ q, int64_t qsb, int64_t qsh, int n_heads, const uint8_t* __restrict__ packed,
     Nf4Layout L, int seq_len, int splits, float* __restrict__ out, float* __restrict__ part_m,
     float* __restrict__ part_l, float* __restrict__ part_o, unsigned* __restrict__ tickets) {
   __shared__ float sQ[kD];
   __shared__ float sLut[16];
-  __shared__ float cm[kDecWarps], cl[kDecWarps];
-  __shared__ float co[kDecWarps][kD];
+  __shared__ float cm[kNf4DecWarps], cl[kNf4DecWarps];
+  __shared__ float co[kNf4DecWarps][kD];
   __shared__ int sLast;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, bh = blockIdx.y;
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_nf4_decode(
   const __half* vs = ks + L.codes_bytes / 128;
 
   float m_run = -INFINITY, l_run = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int grp = g0 + warp; grp < g1; grp += kDecWarps) {
+  for (int grp = g0 + warp; grp < g1; grp += kNf4DecWarps) {
     const int t = grp * 32 + lane;
     float logit = -INFINITY;
     if (t < seq_len) {
@@ -185,9 +186,9 @@ __global__ void __launch_bounds__(kDecWarps * 32) kvq_nf4_decode(
   __syncthreads();
   if (tid < kD) {
     float M = -INFINITY;
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, cm[w]);
+    for (int w = 0; w < kNf4DecWarps; ++w) M = fmaxf(M, cm[w]);
     float Ls = 0.0f, O = 0.0f;
-    for (int w = 0; w < kDecWarps; ++w) {
+    for (int w = 0; w < kNf4DecWarps; ++w) {
       const float wt = (cm[w] == -INFINITY) ? 0.0f : fast_exp2(cm[w] - M);
       Ls += cl[w] * wt;
       O += co[w][tid] * wt;

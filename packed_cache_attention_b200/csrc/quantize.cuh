@@ -2,25 +2,23 @@
 // width for V (page "RoPE-aware bit allocation for KV cache quantization", abstract: the
 // allocator sits on TurboQuant-MSE, K and V get matched bit budgets, the cache is packed).
 //
-// One warp per 32-token tile of one (sequence, KV head) at a time (persistent warps);
-// lane t quantizes token t of the tile. For a token row x (128 values):
+// One warp per 32-token tile of one (sequence, KV head) at a time (persistent warps). For a
+// token row x (128 values):
 //   s2   = sum_j x_j^2 in fp32, j ascending: fl32(s2 + fl32(x_j x_j))
 //   norm = fp16(fp32 sqrt(s2)) (round to nearest even)
 //   a    = fp32(sqrt(128)) / fp32(norm), 0 if norm == 0
 //   y_j  = fp32(fp32(x_j a) g_b)            (V: g = 1, the multiply is skipped as exact)
 //   code = #{thresholds of width w_b strictly below y_j}
 // The code is found by binary search over the 2^w - 1 sorted thresholds, most significant
-// bit first; the comparison at level p is bit p of the code, so its warp ballot (bit t =
-// token t) is directly the tile's bit-plane word for that dim and plane.
+// bit first. Tokens past the sequence length get a NaN scale, so every comparison is false
+// and their codes are 0.
 // The tile is first copied into shared memory with a padded row pitch (65 words for 16-bit
-// inputs), so that the 32 lanes reading the same dim of their own rows hit 32 banks.
-// K: lane t works on token t. The ballot words are staged in shared memory and a last pass
-//   turns each pair into the tile layout and writes whole lines. Per block b (ascending,
-//   w_b > 0) and plane p, the ballots A (dim b) and B (dim b+64) give word0 = lo nibbles of
-//   A's bytes | lo nibbles of B's bytes << 4 and word1 = hi nibbles of A | hi nibbles of B.
-//   Bit s+4m of word H then holds token 4H + s + 8(m/2) at dim b (m even) or b+64 (m odd).
-// V: lane l = c + 4m works on token 8(m/2) + 2c + (m%2), so a ballot is already the layout's
-//   word (bit c+4m holds that token) and lane 0 stores each pair of words directly.
+// inputs), so that 32 lanes reading one dim of their own rows hit 32 banks.
+// K: lane t quantizes token t and appends its codes, in the allocation's stream order, to a
+//   32-bit accumulator; the accumulator fills at the same code for every lane, so each full
+//   word is one coalesced 128-byte warp store (word-planar tile layout).
+// V: lane l quantizes dims 2l, 2l+1, 64+2l, 65+2l for the 32 tokens of the tile, placing
+//   token t's code at bit bits_v * t of the dim's stream (positions known at compile time).
 #pragma once
 
 #include "common.cuh"
@@ -28,6 +26,7 @@
 namespace kvq {
 
 constexpr int kQuantWarps = 8;
+constexpr int kQuantExtraWords = kTile + kH + kH / 4 + 8;   // per warp: 32 scales, 64 gains, 64 block indices, 8 classes
 
 template <int DT> struct QuantRow;
 // 16-bit inputs: a row is 64 words (2 values each), pitch 65 words.
@@ -59,6 +58,13 @@ template <int DT> struct QuantRow16 {
     const uint32_t w = row[i];
     if constexpr (DT == KVQ_BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
     else return __half22float2(*reinterpret_cast<const __half2*>(&w));
+  }
+  // Value j of a row.
+  __device__ __forceinline__ static float value(const uint32_t* row, int j) {
+    const uint32_t w = row[j >> 1];
+    const uint32_t u = (j & 1) ? (w >> 16) : (w & 0xffffu);
+    if constexpr (DT == KVQ_BF16) return __uint_as_float(u << 16);
+    else return __half2float(__ushort_as_half(static_cast<unsigned short>(u)));
   }
 };
 template <> struct QuantRow<KVQ_BF16> : QuantRow16<KVQ_BF16> {};
@@ -92,6 +98,7 @@ template <> struct QuantRow<KVQ_F32> {
   __device__ __forceinline__ static float2 pair(const uint32_t* row, int i) {
     return make_float2(__uint_as_float(row[2 * i]), __uint_as_float(row[2 * i + 1]));
   }
+  __device__ __forceinline__ static float value(const uint32_t* row, int j) { return __uint_as_float(row[j]); }
 };
 
 // fp16 norm of one row and the scale a = sqrt(128)/norm (0 for a zero norm).
@@ -110,80 +117,107 @@ __device__ __forceinline__ void row_norm_scale(const uint32_t* row, __half& n16,
   a = (nf == 0.0f) ? 0.0f : __fdiv_rn(sqd, nf);
 }
 
-// Token handled by lane l in the values pass: l = c + 4m  ->  8(m/2) + 2c + (m%2).
-__device__ __forceinline__ int value_token(int lane) { return 8 * (lane >> 3) + 2 * (lane & 3) + ((lane >> 2) & 1); }
-
-// Binary search for two values of the same width W; the ballot of the comparison at level p
-// (bit p of the code) is written by lane 0 to out[p * pstride] (first value) and
-// out[p * pstride + 1] (second value). The top level compares with the middle threshold,
-// which is exactly 0 for these symmetric codebooks. Widths up to 3 select the next
-// threshold from registers (t[] holds the 2^W - 1 thresholds); wider ones index the
-// shared-memory table.
+// Code of y for a width-W codebook: binary search, most significant bit first. The top
+// level compares with the middle threshold, which is exactly 0 for these symmetric
+// codebooks. Widths up to 3 select the next threshold from registers (t[] holds the
+// 2^W - 1 thresholds); wider ones index the shared-memory table `thr`.
 template <int W>
-__device__ __forceinline__ void search_ballot2(float y1, float y2, const float* __restrict__ thr, const float* t,
-                                               uint32_t* out, int pstride, bool writer) {
-  // out[p * pstride] and out[p * pstride + 1] are adjacent, 8-byte aligned words.
-  auto put = [&](int p, bool c1, bool c2) {
-    const unsigned A = __ballot_sync(0xffffffffu, c1);
-    const unsigned B = __ballot_sync(0xffffffffu, c2);
-    if (writer) *reinterpret_cast<uint2*>(out + p * pstride) = make_uint2(A, B);
-  };
-  const bool h1 = y1 > 0.0f, h2 = y2 > 0.0f;
-  put(W - 1, h1, h2);
-  if constexpr (W == 2) {
-    put(0, y1 > (h1 ? t[2] : t[0]), y2 > (h2 ? t[2] : t[0]));
+__device__ __forceinline__ uint32_t search_code(float y, const float* __restrict__ thr, const float* t) {
+  const bool hi = y > 0.0f;
+  if constexpr (W == 1) {
+    return hi ? 1u : 0u;
+  } else if constexpr (W == 2) {
+    const bool lo = y > (hi ? t[2] : t[0]);
+    return (hi ? 2u : 0u) | (lo ? 1u : 0u);
   } else if constexpr (W == 3) {
-    const bool m1 = y1 > (h1 ? t[5] : t[1]), m2 = y2 > (h2 ? t[5] : t[1]);
-    put(1, m1, m2);
-    const float u1 = h1 ? (m1 ? t[6] : t[4]) : (m1 ? t[2] : t[0]);
-    const float u2 = h2 ? (m2 ? t[6] : t[4]) : (m2 ? t[2] : t[0]);
-    put(0, y1 > u1, y2 > u2);
-  } else if constexpr (W >= 4) {
-    int i1 = h1 ? (1 << (W - 1)) : 0, i2 = h2 ? (1 << (W - 1)) : 0;
+    const bool m = y > (hi ? t[5] : t[1]);
+    const float u = hi ? (m ? t[6] : t[4]) : (m ? t[2] : t[0]);
+    return (hi ? 4u : 0u) | (m ? 2u : 0u) | (y > u ? 1u : 0u);
+  } else {
+    int idx = hi ? (1 << (W - 1)) : 0;
 #pragma unroll
     for (int p = W - 2; p >= 0; --p) {
       const int s = 1 << p;
-      const bool c1 = y1 > thr[i1 + s - 1];
-      const bool c2 = y2 > thr[i2 + s - 1];
-      put(p, c1, c2);
-      i1 += c1 ? s : 0;
-      i2 += c2 ? s : 0;
+      idx += (y > thr[idx + s - 1]) ? s : 0;
     }
+    return static_cast<uint32_t>(idx);
   }
 }
 
-// Dispatch on a runtime width (uniform across the warp).
-__device__ __forceinline__ void search_ballot2_any(int w, float y1, float y2, const float* __restrict__ sThr,
-                                                   const float* t3, uint32_t* out, int pstride, bool writer) {
-  const float* thr = sThr + ((1 << w) - w - 1);
-  switch (w) {
-    case 1: search_ballot2<1>(y1, y2, thr, nullptr, out, pstride, writer); break;
-    case 2: {
-      const float t2[3] = {thr[0], thr[1], thr[2]};
-      search_ballot2<2>(y1, y2, thr, t2, out, pstride, writer);
-      break;
-    }
-    case 3: search_ballot2<3>(y1, y2, thr, t3, out, pstride, writer); break;
-    case 4: search_ballot2<4>(y1, y2, thr, nullptr, out, pstride, writer); break;
-    case 5: search_ballot2<5>(y1, y2, thr, nullptr, out, pstride, writer); break;
-    case 6: search_ballot2<6>(y1, y2, thr, nullptr, out, pstride, writer); break;
-    case 7: search_ballot2<7>(y1, y2, thr, nullptr, out, pstride, writer); break;
-    default: search_ballot2<8>(y1, y2, thr, nullptr, out, pstride, writer); break;
-  }
-}
+// Thresholds of width W from the shared table (all widths concatenated, width w at 2^w - w - 1).
+__device__ __forceinline__ const float* width_thresholds(const float* sThr, int w) { return sThr + ((1 << w) - w - 1); }
 
-// Values: uniform width W for the whole row, dims processed in pairs.
+// Bit stream writer for one lane's K codes; `fill` and `word` advance identically in every
+// lane, so every flush is a full-warp store of one word-planar row (word i of 32 tokens).
+struct KStream {
+  uint32_t cur = 0;
+  int fill = 0;
+  int word = 0;
+  template <int W>
+  __device__ __forceinline__ void put(uint32_t code, uint32_t* __restrict__ kout, int lane) {
+    cur |= code << fill;
+    fill += W;
+    if (fill >= 32) {
+      kout[word * kTile + lane] = cur;
+      ++word;
+      fill -= 32;
+      cur = fill ? (code >> (W - fill)) : 0u;
+    }
+  }
+};
+
+// All blocks of one width class: for each block b (stream order), the codes of dims b and
+// b + 64. tb[b] = {gain bits of block b}; sb = the class's blocks.
 template <int DT, int W>
-__device__ __forceinline__ void quant_values(const uint32_t* myrow, float a, const float* __restrict__ sThr,
-                                             uint32_t* vstage, bool writer) {
-  const float* thr = sThr + ((1 << W) - W - 1);
+__device__ __forceinline__ void quant_k_class(const uint32_t* myrow, float a, const float* __restrict__ gains,
+                                              const uint8_t* __restrict__ sb, int nb, const float* __restrict__ sThr,
+                                              KStream& ks, uint32_t* __restrict__ kout, int lane) {
+  const float* thr = width_thresholds(sThr, W);
   float t[7];
 #pragma unroll
-  for (int i = 0; i < 7; ++i) t[i] = (i < (1 << W) - 1) ? thr[i] : 0.0f;
-#pragma unroll 4
-  for (int i = 0; i < kD / 2; ++i) {
-    const float2 x = QuantRow<DT>::pair(myrow, i);
-    search_ballot2<W>(__fmul_rn(x.x, a), __fmul_rn(x.y, a), thr, t, vstage + 2 * i, kD, writer);
+  for (int i = 0; i < 7; ++i) t[i] = (W <= 3 && i < (1 << W) - 1) ? thr[i] : 0.0f;
+  for (int k = 0; k < nb; ++k) {
+    const int b = sb[k];
+    const float g = gains[b];
+    const float y1 = __fmul_rn(__fmul_rn(QuantRow<DT>::value(myrow, b), a), g);
+    const float y2 = __fmul_rn(__fmul_rn(QuantRow<DT>::value(myrow, b + kH), a), g);
+    ks.template put<W>(search_code<W>(y1, thr, t), kout, lane);
+    ks.template put<W>(search_code<W>(y2, thr, t), kout, lane);
+  }
+}
+
+// Values: width BV for every dim. Lane l handles dims {2l, 2l+1} and {64+2l, 65+2l}; sA[t]
+// is token t's scale (NaN past the sequence length). Word i of dim j goes to vout[128 i + j].
+template <int DT, int BV>
+__device__ __forceinline__ void quant_v_tile(const uint32_t* rows, const float* sA, const float* __restrict__ sThr,
+                                             uint32_t* __restrict__ vout, int lane) {
+  const float* thr = width_thresholds(sThr, BV);
+  float t[7];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) t[i] = (BV <= 3 && i < (1 << BV) - 1) ? thr[i] : 0.0f;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int j0 = 2 * lane + kH * half;
+    uint32_t w0[BV], w1[BV];
+#pragma unroll
+    for (int i = 0; i < BV; ++i) { w0[i] = 0u; w1[i] = 0u; }
+#pragma unroll
+    for (int tok = 0; tok < kTile; ++tok) {
+      const float2 x = QuantRow<DT>::pair(rows + tok * QuantRow<DT>::kPitch, j0 >> 1);
+      const float at = sA[tok];
+      const uint32_t c0 = search_code<BV>(__fmul_rn(x.x, at), thr, t);
+      const uint32_t c1 = search_code<BV>(__fmul_rn(x.y, at), thr, t);
+      const int bit = BV * tok, wi = bit >> 5, sh = bit & 31;
+      w0[wi] |= c0 << sh;
+      w1[wi] |= c1 << sh;
+      if (sh + BV > 32) {
+        w0[wi + 1] |= c0 >> (32 - sh);
+        w1[wi + 1] |= c1 >> (32 - sh);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < BV; ++i)
+      *reinterpret_cast<uint2*>(vout + i * kD + j0) = make_uint2(w0[i], w1[i]);
   }
 }
 
@@ -201,18 +235,14 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k_words = bits_k * kD, v_words = bits_v * kD;
-  const int warp_words = Row::kWords + k_words + 2 * kH;
-  uint32_t* rows = smem + 512 + warp * warp_words;
-  uint32_t* stage = rows + Row::kWords;
-  uint2* tb = reinterpret_cast<uint2*>(stage + k_words);   // per block: {gain bits, width | offset << 8}
+  uint32_t* wbase = smem + 512 + warp * (Row::kWords + kQuantExtraWords);
+  uint32_t* rows = wbase;
+  float* sA = reinterpret_cast<float*>(wbase + Row::kWords);             // 32 value scales
+  float* sGain = sA + kTile;                                              // 64 block gains
+  uint8_t* sBlk = reinterpret_cast<uint8_t*>(sGain + kH);                 // 64 blocks, stream order
   const uint32_t* myrow = rows + lane * Row::kPitch;
-  const int vtok = value_token(lane);
-  const uint32_t* myvrow = rows + vtok * Row::kPitch;
-  const bool writer = lane == 0;
-  float t3[7];
-#pragma unroll
-  for (int i = 0; i < 7; ++i) t3[i] = sThr[(1 << 3) - 3 - 1 + i];   // width-3 thresholds
-  int cur_h = -1;
+  uint32_t* sCls = reinterpret_cast<uint32_t*>(sBlk + kH);              // 8 classes: width | first << 8 | blocks << 16
+  int cur_h = -1, n_cls = 0;
 
   for (long long task = static_cast<long long>(blockIdx.x) * kQuantWarps + warp; task < n_tasks;
        task += static_cast<long long>(gridDim.x) * kQuantWarps) {
@@ -223,79 +253,77 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
     if (al->k_words != k_words) continue;      // allocation made for another budget: write nothing
     if (h != cur_h) {
       __syncwarp();
-      for (int i = lane; i < kH; i += 32)
-        tb[i] = make_uint2(__float_as_uint(al->gain[i]), static_cast<uint32_t>(al->width[i]) |
-                                                             (static_cast<uint32_t>(al->word_off[i]) << 8));
+      for (int i = lane; i < kH; i += 32) {
+        sGain[i] = al->gain[i];
+        sBlk[i] = al->stream_block[i];
+      }
+      n_cls = min(max(al->n_classes, 0), 8);
+      if (lane < 8)
+        sCls[lane] = static_cast<uint32_t>(al->class_width[lane]) | (static_cast<uint32_t>(al->class_first[lane]) << 8) |
+                     (static_cast<uint32_t>(al->class_blocks[lane]) << 16);
+      __syncwarp();
       cur_h = h;
     }
     const int t0 = tile * kTile;
     const int valid_rows = min(kTile, seq_len - t0);
     const bool valid = lane < valid_rows;
+    uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
+    uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
+    uint32_t* vout = kout + k_words;
+    uint16_t* norms = reinterpret_cast<uint16_t*>(vout + v_words);
 
     // ---------------------------------------------------------------- K (Block-GTQ widths)
     __syncwarp();
     Row::load(rows, K + b * ksb + h * ksh + static_cast<int64_t>(t0) * kst, kst, valid_rows, lane);
     __syncwarp();
-    __half kn16, vn16;
+    __half n16;
     float a;
-    row_norm_scale<DT>(myrow, kn16, a);
-    if (!valid) a = __int_as_float(0x7fc00000);   // NaN: every comparison false, so all code bits are 0
-#pragma unroll 2
-    for (int bp = 0; bp < kH / 2; ++bp) {
-      const float2 lo = Row::pair(myrow, bp);             // dims 2bp, 2bp+1
-      const float2 hi = Row::pair(myrow, kH / 2 + bp);    // dims 64+2bp, 65+2bp
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const uint2 e = tb[2 * bp + u];
-        const int w = e.y & 0xffu;
-        if (w == 0) continue;
-        const float g = __uint_as_float(e.x);
-        const float y1 = __fmul_rn(__fmul_rn(u ? lo.y : lo.x, a), g);
-        const float y2 = __fmul_rn(__fmul_rn(u ? hi.y : hi.x, a), g);
-        search_ballot2_any(w, y1, y2, sThr, t3, stage + (e.y >> 8), 2, writer);
+    row_norm_scale<DT>(myrow, n16, a);
+    norms[lane] = valid ? __half_as_ushort(n16) : 0;
+    if (!valid) a = __int_as_float(0x7fc00000);   // NaN: every comparison false, so all codes are 0
+    KStream ks;
+    for (int c = 0; c < n_cls; ++c) {
+      const uint32_t e = sCls[c];
+      const int w = e & 0xffu, first = (e >> 8) & 0xffu, nb = e >> 16;
+      const uint8_t* sb = sBlk + first;
+      switch (w) {
+        case 1: quant_k_class<DT, 1>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
+        case 2: quant_k_class<DT, 2>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
+        case 3: quant_k_class<DT, 3>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
+        case 4: quant_k_class<DT, 4>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
+        case 5: quant_k_class<DT, 5>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
+        case 6: quant_k_class<DT, 6>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
+        case 7: quant_k_class<DT, 7>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
+        default: quant_k_class<DT, 8>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
       }
     }
 
     // ---------------------------------------------------------------- V (uniform width)
-    uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
-    uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
-    uint32_t* vout = kout + k_words;
-    const bool vvalid = vtok < valid_rows;
     __syncwarp();
     Row::load(rows, V + b * vsb + h * vsh + static_cast<int64_t>(t0) * vst, vst, valid_rows, lane);
     __syncwarp();
-    row_norm_scale<DT>(myvrow, vn16, a);
-    if (!vvalid) a = __int_as_float(0x7fc00000);
-    switch (bits_v) {
-      case 1: quant_values<DT, 1>(myvrow, a, sThr, vout, writer); break;
-      case 2: quant_values<DT, 2>(myvrow, a, sThr, vout, writer); break;
-      case 3: quant_values<DT, 3>(myvrow, a, sThr, vout, writer); break;
-      case 4: quant_values<DT, 4>(myvrow, a, sThr, vout, writer); break;
-      case 5: quant_values<DT, 5>(myvrow, a, sThr, vout, writer); break;
-      case 6: quant_values<DT, 6>(myvrow, a, sThr, vout, writer); break;
-      case 7: quant_values<DT, 7>(myvrow, a, sThr, vout, writer); break;
-      default: quant_values<DT, 8>(myvrow, a, sThr, vout, writer); break;
-    }
+    row_norm_scale<DT>(myrow, n16, a);
+    norms[kTile + lane] = valid ? __half_as_ushort(n16) : 0;
+    sA[lane] = valid ? a : __int_as_float(0x7fc00000);
     __syncwarp();
-
-    // ---------------------------------------------------------------- K words: permute + store
-    for (int k = lane; k < k_words / 2; k += 32) {
-      const uint32_t A = stage[2 * k], B = stage[2 * k + 1];
-      uint2 o;
-      o.x = (A & 0x0f0f0f0fu) | ((B & 0x0f0f0f0fu) << 4);
-      o.y = ((A >> 4) & 0x0f0f0f0fu) | (B & 0xf0f0f0f0u);
-      reinterpret_cast<uint2*>(kout)[k] = o;
+    switch (bits_v) {
+      case 1: quant_v_tile<DT, 1>(rows, sA, sThr, vout, lane); break;
+      case 2: quant_v_tile<DT, 2>(rows, sA, sThr, vout, lane); break;
+      case 3: quant_v_tile<DT, 3>(rows, sA, sThr, vout, lane); break;
+      case 4: quant_v_tile<DT, 4>(rows, sA, sThr, vout, lane); break;
+      case 5: quant_v_tile<DT, 5>(rows, sA, sThr, vout, lane); break;
+      case 6: quant_v_tile<DT, 6>(rows, sA, sThr, vout, lane); break;
+      case 7: quant_v_tile<DT, 7>(rows, sA, sThr, vout, lane); break;
+      default: quant_v_tile<DT, 8>(rows, sA, sThr, vout, lane); break;
     }
-    uint16_t* norms = reinterpret_cast<uint16_t*>(vout + v_words);
-    norms[lane] = valid ? __half_as_ushort(kn16) : 0;
-    norms[kTile + vtok] = vvalid ? __half_as_ushort(vn16) : 0;
   }
 }
 
-// Dynamic shared memory of kvq_quant_pack for the input type's row pitch.
-inline size_t quant_smem_bytes(int dtype, int bits_k, int bits_v) {
+// Dynamic shared memory of kvq_quant_pack: thresholds + per warp the row tile, 32 value
+// scales, 64 gains, 64 stream-order block indices and the 8-entry class table.
+inline size_t quant_smem_bytes(int dtype) {
   const int row_words = (dtype == KVQ_F32) ? QuantRow<KVQ_F32>::kWords : QuantRow<KVQ_BF16>::kWords;
-  return 4 * (512 + static_cast<size_t>(kQuantWarps) * (row_words + bits_k * kD + 2 * kH));
+  return 4 * (512 + static_cast<size_t>(kQuantWarps) * (row_words + kQuantExtraWords));
 }
 
 }  // namespace kvq

@@ -48,11 +48,13 @@ class CacheDesc(ctypes.Structure):
 
 class HeadAlloc(ctypes.Structure):
     _fields_ = [("energy", ctypes.c_double * 64), ("gain", ctypes.c_float * 64), ("dequant", ctypes.c_float * 64),
-                ("word_off", ctypes.c_uint16 * 64), ("width", ctypes.c_uint8 * 64),
-                ("step_width", ctypes.c_uint8 * 32), ("step_block", (ctypes.c_int8 * 4) * 32),
+                ("bit_off", ctypes.c_int16 * 64), ("width", ctypes.c_uint8 * 64),
+                ("stream_block", ctypes.c_uint8 * 64), ("class_bit", ctypes.c_uint16 * 8),
+                ("class_width", ctypes.c_uint8 * 8), ("class_first", ctypes.c_uint8 * 8),
+                ("class_blocks", ctypes.c_uint8 * 8), ("reserved_b", ctypes.c_uint8 * 56),
                 ("head_dim", ctypes.c_int32), ("bits_k", ctypes.c_int32), ("w_max", ctypes.c_int32),
-                ("mode", ctypes.c_int32), ("n_steps", ctypes.c_int32), ("k_words", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 2)]
+                ("mode", ctypes.c_int32), ("n_classes", ctypes.c_int32), ("k_words", ctypes.c_int32),
+                ("n_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _VP = ctypes.c_void_p
@@ -174,10 +176,14 @@ def parse_alloc(raw: np.ndarray) -> list[dict]:
             "g": np.array(rec.gain[:], dtype=np.float32),
             "f": np.array(rec.dequant[:], dtype=np.float32),
             "w": np.array(rec.width[:], dtype=np.int64),
-            "word_off": np.array(rec.word_off[:], dtype=np.int64),
-            "step_width": np.array(rec.step_width[:], dtype=np.int64),
-            "step_block": np.array([list(r) for r in rec.step_block], dtype=np.int64),
-            "n_steps": rec.n_steps, "k_words": rec.k_words, "bits_k": rec.bits_k, "w_max": rec.w_max,
+            "bit_off": np.array(rec.bit_off[:], dtype=np.int64),
+            "stream_block": np.array(rec.stream_block[:], dtype=np.int64),
+            "class_bit": np.array(rec.class_bit[:], dtype=np.int64),
+            "class_width": np.array(rec.class_width[:], dtype=np.int64),
+            "class_first": np.array(rec.class_first[:], dtype=np.int64),
+            "class_blocks": np.array(rec.class_blocks[:], dtype=np.int64),
+            "n_classes": rec.n_classes, "n_blocks": rec.n_blocks, "k_words": rec.k_words,
+            "bits_k": rec.bits_k, "w_max": rec.w_max,
             "mode": rec.mode,
         })
     return heads

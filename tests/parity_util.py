@@ -32,24 +32,28 @@ def compare_alloc(gpu_heads, ref):
         np.testing.assert_array_equal(g["w"], ref["w"][h])
         np.testing.assert_array_equal(g["g"].view(np.uint32), ref["g"][h].view(np.uint32))
         np.testing.assert_array_equal(g["f"].view(np.uint32), ref["f"][h].view(np.uint32))
-        np.testing.assert_array_equal(g["word_off"], bg.k_word_offsets(ref["w"][h]))
+        np.testing.assert_array_equal(g["bit_off"], bg.k_bit_offsets(ref["w"][h]))
         assert g["k_words"] == int(2 * ref["w"][h].sum())
-        check_steps(g, ref["w"][h])
+        check_classes(g, ref["w"][h])
 
 
-def check_steps(g, w):
-    """The decode k-step table lists every block with w > 0 once, widths descending, 4 per step."""
-    seen = []
-    prev_w = 99
-    for s in range(g["n_steps"]):
-        sw = g["step_width"][s]
-        assert 1 <= sw <= prev_w
-        prev_w = sw
-        blks = [b for b in g["step_block"][s] if b >= 0]
-        assert blks and all(w[b] == sw for b in blks)
-        seen += blks
-    assert sorted(seen) == [b for b in range(len(w)) if w[b] > 0]
-    assert len(seen) == len(set(seen))
+def check_classes(g, w):
+    """The class table lists the stream order: widths descending, blocks ascending inside a
+    class, bit offsets consistent with 2 * w bits per block."""
+    order = bg.k_stream_blocks(w)
+    n = len(order)
+    assert g["n_blocks"] == n
+    assert list(g["stream_block"][:n]) == order and all(x == 255 for x in g["stream_block"][n:])
+    widths = sorted({int(x) for x in w if x > 0}, reverse=True)
+    assert g["n_classes"] == len(widths)
+    bit = 0
+    for c, cw in enumerate(widths):
+        blocks = [b for b in range(len(w)) if w[b] == cw]
+        assert g["class_width"][c] == cw and g["class_blocks"][c] == len(blocks)
+        assert order[g["class_first"][c]:g["class_first"][c] + len(blocks)] == blocks
+        assert g["class_bit"][c] == bit
+        bit += 2 * cw * len(blocks)
+    assert all(x == 0 for x in g["class_width"][len(widths):])
 
 
 def oracle_pipeline(K, V, q, bits_k, bits_v, n_calib=0, w_max=8, mode=0, capacity=None):

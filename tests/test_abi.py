@@ -43,7 +43,7 @@ def test_struct_sizes_match_header(L):
     assert ctypes.sizeof(kvq.HeadAlloc) == 1408
     assert ctypes.sizeof(kvq.Tensor4) == 48
     assert kvq.kvq_alloc_bytes(3) == 3 * 1408
-    assert kvq.kvq_abi_version() == 1
+    assert kvq.kvq_abi_version() == 2
 
 
 @pytest.mark.parametrize("w", range(1, 9))

@@ -394,28 +394,47 @@ def _alloc_with(w_blocks, d=128):
             "d": d, "bits_k": int(sum(w_blocks)) * 2 // d, "w_max": 8, "mode": 0}
 
 
-def test_pack_single_code_position_by_hand():
-    """Hand-placed code: token 9, dim 3 + 64 (block 3), width 3, code 0b101.
+def test_k_stream_order_by_hand():
+    """d = 8 (4 blocks), widths [2, 5, 0, 1]: the stream holds block 1 (width 5), block 0
+    (width 2), block 3 (width 1); block 2 has no bits. Each block is a pair of codes."""
+    w = np.array([2, 5, 0, 1])
+    assert bg.k_stream_blocks(w) == [1, 0, 3]
+    np.testing.assert_array_equal(bg.k_bit_offsets(w), [10, 0, -1, 14])
 
-    Block widths: blocks 0..2 have 3 bits, block 3 has 3 bits, the rest are set so the
-    K budget is 3 bits/dim. Token 9 = 4*0 + 1 + 8*1 -> half H = 0, s = 1, m div 2 = 1;
-    dim b + h -> m odd -> m = 3; bit q = s + 4 m = 13. Block 3's segment starts at
-    word 2 * (3 + 3 + 3) = 18; planes 0 and 2 are words 18 + 0 and 18 + 4.
+
+def test_pack_bits_by_hand():
+    words = bg.pack_bits(np.array([[0b101, 0b11, 0b1]]), [3, 30, 1])
+    assert words.shape == (1, 2)
+    assert int(words[0, 0]) == 0b101 | (0b11 << 3)
+    assert int(words[0, 1]) == 1 << 1
+    np.testing.assert_array_equal(bg.unpack_bits(words, [3, 30, 1]), [[0b101, 0b11, 0b1]])
+
+
+def test_pack_single_code_position_by_hand():
+    """Every block 3 bits wide, so the K stream is blocks 0..63 in order, 6 bits per block.
+
+    K: token 9, dim 3 + 64 (second code of block 3) with code 0b101 sits at stream bits
+    18 + 3 = 21..23, i.e. word 0 of token 9 -> word-planar index 0 * 32 + 9. Token 5, dim 5
+    (first code of block 5) with code 0b111 sits at bits 30..32 and straddles words 0 and 1
+    -> indices 5 and 32 + 5.
+    V: token 13, dim 70, code 0b011 sits at bits 39..41 of dim 70's stream, i.e. bits 7..9
+    of its word 1 -> index 1 * 128 + 70.
     """
     w = [3] * 64
     a = _alloc_with(w)
     Kc = np.zeros((1, 1, 32, 128), np.uint8)
     Kc[0, 0, 9, 3 + 64] = 0b101
+    Kc[0, 0, 5, 5] = 0b111
     Vc = np.zeros((1, 1, 32, 128), np.uint8)
-    Vc[0, 0, 13, 70] = 0b011          # token 13 = 8*1 + 2*2 + 1 -> c = 2, m = 3 -> q = 2 + 12 = 14
+    Vc[0, 0, 13, 70] = 0b011
     codes = {"Kc": Kc, "Kn": np.zeros((1, 1, 32), np.float16), "Vc": Vc, "Vn": np.zeros((1, 1, 32), np.float16)}
     packed = bg.pack_cache(codes, a, 3, 32)
     words = packed[0, 0, 0, :4 * (384 + 384)].copy().view("<u4")
     kw, vw = words[:384], words[384:]
     nz = {i: int(x) for i, x in enumerate(kw) if x}
-    assert nz == {18: 1 << 13, 22: 1 << 13}
+    assert nz == {9: 0b101 << 21, 5: 0b11 << 30, 37: 1}
     vnz = {i: int(x) for i, x in enumerate(vw) if x}
-    assert vnz == {0 * 128 + 70: 1 << 14, 1 * 128 + 70: 1 << 14}
+    assert vnz == {1 * 128 + 70: 0b011 << 7}
 
 
 def test_pack_unpack_roundtrip_mixed_widths():

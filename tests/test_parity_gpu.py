@@ -12,7 +12,7 @@ from oracle import blockgtq as bg
 from oracle import nqkv
 from packed_cache_attention_b200 import kvq
 from packed_cache_attention_b200 import workloads as wl
-from tests.parity_util import TOL, check_steps, compare_alloc, host_f32, oracle_pipeline, rel_err, tiles_written
+from tests.parity_util import TOL, compare_alloc, host_f32, oracle_pipeline, rel_err, tiles_written
 
 pytestmark = pytest.mark.gpu
 
