@@ -30,7 +30,7 @@
 extern "C" {
 #endif
 
-#define KVQ_ABI_VERSION 2
+#define KVQ_ABI_VERSION 3
 #define KVQ_TILE_TOKENS 32     /* tokens per packed Block-GTQ tile */
 #define KVQ_HEAD_DIM 128       /* head dimension the kernels are built for */
 #define KVQ_MAX_WIDTH 8        /* widest Lloyd-Max codebook */
@@ -114,6 +114,18 @@ typedef struct {
   int32_t k_words;          /* 32-bit words in a tile's K part (= bits_k * head_dim) */
   int32_t n_blocks;         /* blocks with w_b > 0 */
   int32_t reserved;
+  /* Decode plan, derived from the classes (written by kvq_calibrate, read by the decode).
+   * The K operand of the tensor-core product has one column per block pair, in stream order;
+   * each class is cut into groups of 4 pairs, its last group holding 2 pairs when at most 2
+   * remain (4 when 3 remain). Group x (counted over all classes) belongs to warp group
+   * g = x % 4 as its entry i = x / 4 and fills columns 24 g + 4 i .. 24 g + 4 i + 3; a run is a
+   * warp group's consecutive groups of one class. */
+  uint32_t plan_run[4][8];      /* width | first entry << 8 | groups << 16 | last group half << 24 */
+  uint32_t plan_group[4][16];   /* bit offset of the group in the K stream | first column << 16 */
+  int8_t plan_col_block[128];   /* block of column c, -1 for a padding column */
+  int32_t plan_n_runs[4];
+  int32_t plan_k_cols;          /* columns of the product (96) */
+  uint8_t reserved_c[108];
 } kvq_head_alloc;
 
 /* ---------------------------------------------------------------- queries (host only) */
@@ -131,7 +143,7 @@ kvq_status kvq_codebook(int width, uint16_t* centroids_f16, float* thresholds, f
  * [NQKV] mechanism paragraph: 16 standard-normal quantiles imported from QLoRA. */
 kvq_status kvq_nf4_table(float* levels, float* midpoints);
 
-/* Bytes of the allocation buffer for n_kv_heads heads (n_kv_heads * sizeof(kvq_head_alloc)). */
+/* Bytes of the allocation buffer for n_kv_heads heads (n_kv_heads * sizeof(kvq_head_alloc) = 2048 each). */
 size_t kvq_alloc_bytes(int n_kv_heads);
 
 /* Workspace bytes kvq_calibrate needs for this many sequences, KV heads and calibration
@@ -186,9 +198,9 @@ kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_p
  * 4 * head_dim * (bits_k + bits_v) + 128 bytes, little-endian:
  *   K part: 32-bit word 32 i + t is word i (i < 4 bits_k) of token t's K stream (see
  *           kvq_head_alloc; codes least significant bit first, bits_k * head_dim bits).
+ *   32 fp16 K norms, then 32 fp16 V norms, in token order.
  *   V part: word 128 i + j is word i (i < bits_v) of dim j's V stream: the codes of the
  *           tile's tokens 0..31 at dim j, bits_v bits each, least significant bit first.
- *   32 fp16 K norms, then 32 fp16 V norms, in token order.
  * K, V: [batch][n_kv_heads][seq_len][128] (kd, vd may differ in strides, not in shape).
  * alloc: records from kvq_calibrate with bits_k == cache->bits_k.
  * packed: kvq_packed_bytes(cache) bytes, 16-byte aligned. */
@@ -201,6 +213,7 @@ kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, con
  * out: fp32 [batch][n_q_heads][128], contiguous. Attends over cached positions
  * 0..seq_len-1: out = sum_t softmax_t(q . k_hat_t / sqrt(d)) v_hat_t with
  * k_hat = norm * c[code] * f_b and v_hat = norm * c[code] / sqrt(d).
+ * packed, alloc: 16-byte aligned (as allocated by any CUDA allocator).
  * ws: kvq_decode_workspace_bytes bytes, zeroed once by kvq_workspace_init. */
 kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
                            const kvq_cache_desc* cache, int seq_len, float* out, void* ws,

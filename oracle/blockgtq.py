@@ -218,7 +218,7 @@ def tile_v_words(bits_v: int, d: int) -> int:
 
 
 def tile_record_bytes(d: int, bits_k: int, bits_v: int) -> int:
-    """Bytes of one 32-token tile record: K words, V words, 32 K norms, 32 V norms (fp16)."""
+    """Bytes of one 32-token tile record: K words, 32 K norms, 32 V norms (fp16), V words."""
     return 4 * tile_k_words(bits_k, d) + 4 * tile_v_words(bits_v, d) + 2 * TILE * 2
 
 
@@ -285,10 +285,12 @@ def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarr
         significant bit first, in the order of k_stream_blocks; each block gives the code
         of dim b (w_b bits) and then the code of dim b + d/2 (w_b bits). The stream is
         exactly bits_k * d bits long.
+      32 fp16 K norms, then 32 fp16 V norms, in token order.
       V part, bits_v * d words, stored word-planar: word d i + j is word i of dim j's V
         stream (i < bits_v), which is the codes of tokens 0..31 of the tile at dim j,
         concatenated, bits_v bits each, least significant bit first.
-      32 fp16 K norms, 32 fp16 V norms, in token order.
+    Keys and their norms come first and values with theirs last, so that a reader can fetch
+    either half of a record in one contiguous piece.
     Tokens at or beyond the sequence length T are stored with code 0 and norm 0.
     """
     Kc, Kn, Vc, Vn = codes["Kc"], codes["Kn"], codes["Vc"], codes["Vn"]
@@ -322,9 +324,9 @@ def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarr
         vstream = pack_bits(np.transpose(Vc[:, hh], (0, 1, 3, 2)), [bits_v] * TILE)   # [B][n_tiles][d][bv]
         vwords = np.transpose(vstream, (0, 1, 3, 2)).reshape(B, n_tiles, -1)
         parts = [kwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1),
-                 vwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1),
                  Kn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1),
-                 Vn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1)]
+                 Vn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1),
+                 vwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1)]
         out[:, hh] = np.concatenate(parts, axis=-1)
     return out
 
@@ -339,9 +341,9 @@ def unpack_cache(packed: np.ndarray, alloc: dict, bits_v: int, seq_len: int) -> 
     cap = n_tiles * TILE
     Kc = np.zeros((B, H, n_tiles, TILE, d), dtype=np.uint8)
     Vc = np.zeros((B, H, n_tiles, TILE, d), dtype=np.uint8)
-    words = packed[..., :4 * (nk + nv)].copy().view("<u4")
-    kw, vw = words[..., :nk], words[..., nk:]
-    norms = packed[..., 4 * (nk + nv):].copy().view("<f2")
+    kw = packed[..., :4 * nk].copy().view("<u4")
+    norms = packed[..., 4 * nk:4 * nk + 4 * TILE].copy().view("<f2")
+    vw = packed[..., 4 * nk + 4 * TILE:].copy().view("<u4")
     Kn = norms[..., :TILE].reshape(B, H, cap)
     Vn = norms[..., TILE:].reshape(B, H, cap)
     for hh in range(H):

@@ -270,6 +270,37 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
       if (sWidth[b] == 0) al->bit_off[b] = -1;
     al->n_classes = n_cls;
     al->n_blocks = pos;
+    // Decode plan: classes in stream order cut into groups of 4 block pairs (the last group
+    // 2 pairs when at most 2 remain); group x goes to warp group g = x % 4 as entry i = x / 4
+    // and fills columns 24 g + 4 i .. + 3 of the tensor-core operand.
+    {
+      int x0 = 0, nr[4] = {0, 0, 0, 0};
+      for (int i = 0; i < 128; ++i) al->plan_col_block[i] = -1;
+      int first = 0, bit0 = 0;
+      for (int w = 8; w >= 1; --w) {
+        const int nb = sCount[w];
+        if (nb == 0) continue;
+        const int r = nb & 3, ng = (nb >> 2) + (r ? 1 : 0);
+        for (int k = 0; k < ng; ++k) {
+          const int x = x0 + k, g = x & 3, col = 24 * g + 4 * (x >> 2);
+          al->plan_group[g][x >> 2] = static_cast<uint32_t>(bit0 + 8 * w * k) | (static_cast<uint32_t>(col) << 16);
+          if (nr[g] == 0 || (al->plan_run[g][nr[g] - 1] & 15u) != static_cast<uint32_t>(w))
+            al->plan_run[g][nr[g]++] = static_cast<uint32_t>(w) | (static_cast<uint32_t>(x >> 2) << 8);
+          al->plan_run[g][nr[g] - 1] += 1u << 16;
+          if (k == ng - 1 && r != 0 && r <= 2) al->plan_run[g][nr[g] - 1] |= 1u << 24;
+          for (int i = 0; i < 4 && 4 * k + i < nb; ++i)
+            al->plan_col_block[col + i] = static_cast<int8_t>(al->stream_block[first + 4 * k + i]);
+        }
+        x0 += ng;
+        first += nb;
+        bit0 += 2 * w * nb;
+      }
+      for (int g = 0; g < 4; ++g) {
+        al->plan_n_runs[g] = nr[g];
+        for (int i = nr[g]; i < 8; ++i) al->plan_run[g][i] = 0u;
+      }
+      al->plan_k_cols = 96;
+    }
     al->k_words = bit / 32 * kTile;     // bits per token * 32 tokens / 32 bits per word
     al->head_dim = kD;
     al->bits_k = bits_k;
@@ -278,6 +309,7 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     al->reserved = 0;
   }
   if (tid < 56) al->reserved_b[tid] = 0;
+  if (tid < 108) al->reserved_c[tid] = 0;
 }
 
 }  // namespace kvq

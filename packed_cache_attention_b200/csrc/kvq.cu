@@ -33,6 +33,9 @@ kvq_status ensure_tables() {
   std::memcpy(d.nf4, t.nf4, sizeof(d.nf4));
   std::memcpy(d.nf4_mid, t.nf4_mid, sizeof(d.nf4_mid));
   if (cudaMemcpyToSymbol(c_tab, &d, sizeof(d)) != cudaSuccess) return KVQ_ERR_CUDA;
+  static uint8_t lut[kLutBytes];
+  decode_lut_image(t.centroid_f16, lut);
+  if (cudaMemcpyToSymbol(g_dec_lut, lut, sizeof(lut)) != cudaSuccess) return KVQ_ERR_CUDA;
   g_uploaded[dev] = true;
   return KVQ_OK;
 }
@@ -135,17 +138,18 @@ Nf4Layout nf4_layout(int batch, int n_heads, int capacity) {
 
 constexpr size_t kMaxSmem = 227 * 1024;
 
-// Deepest bulk-copy pipeline (1..4 chunks of 4 tile records) that fits in shared memory.
-int decode_stages(int rec_bytes) {
-  const size_t per = static_cast<size_t>(kChunkTiles) * rec_bytes;
+// Deepest bulk-copy pipeline (1..4 stages of 4 tile halves) that fits in shared memory.
+int decode_stages(int bits_k, int bits_v) {
+  const size_t per = static_cast<size_t>(kChunkTiles) * stage_tile_stride(bits_k, bits_v);
   const size_t room = kMaxSmem - decode_stage_off();
   return static_cast<int>(std::max<size_t>(1, std::min<size_t>(kDecStagesMax, room / per)));
 }
 
-size_t decode_smem_bytes(int rec_bytes) {
-  const size_t stage = static_cast<size_t>(kChunkTiles) * rec_bytes * decode_stages(rec_bytes);
-  // the stage area also holds the Q' staging (4 KB) and the merge scratch (4 KB)
-  return decode_stage_off() + std::max<size_t>(stage, 8 * kD * sizeof(float));
+size_t decode_smem_bytes(int bits_k, int bits_v) {
+  const size_t stage =
+      static_cast<size_t>(kChunkTiles) * stage_tile_stride(bits_k, bits_v) * decode_stages(bits_k, bits_v);
+  // the stage area also holds the merge scratch (4 KB)
+  return decode_stage_off() + std::max<size_t>(stage, 256 * sizeof(float4));
 }
 
 }  // namespace
@@ -340,7 +344,7 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
                            void* stream) {
   kvq_status st;
   if ((st = check_tensor(q, qd)) != KVQ_OK) return st;
-  if (!packed || !alloc || !out || !aligned16(packed)) return KVQ_ERR_ARG;
+  if (!packed || !alloc || !out || !aligned16(packed) || !aligned16(alloc)) return KVQ_ERR_ARG;
   if (!cache_ok(c)) return KVQ_ERR_ARG;
   if (qd->seq_len != 1 || qd->batch != c->batch) return KVQ_ERR_SHAPE;
   if (qd->n_heads % c->n_kv_heads != 0 || qd->n_heads / c->n_kv_heads > 8) return KVQ_ERR_UNSUPPORTED;
@@ -354,7 +358,7 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
   if ((st = ensure_tables()) != KVQ_OK) return st;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
-  const size_t smem = decode_smem_bytes(rec);
+  const size_t smem = decode_smem_bytes(c->bits_k, c->bits_v);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(splits, bh);
 #define KVQ_LAUNCH_DEC(DT, TY)                                                                                        \
@@ -366,7 +370,7 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
     kern<<<grid, kDecThreads, smem, s>>>(                                                                             \
         static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, c->n_kv_heads,                             \
         static_cast<const uint8_t*>(packed), static_cast<const kvq_head_alloc*>(alloc), n_tiles_of(c->capacity), rec, \
-        c->bits_k, c->bits_v, seq_len, splits, merge_groups(splits), decode_stages(rec), out,                         \
+        c->bits_k, c->bits_v, seq_len, splits, merge_groups(splits), decode_stages(c->bits_k, c->bits_v), out,                         \
         reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_l),                            \
         reinterpret_cast<float*>(w8 + L.part_o), reinterpret_cast<unsigned*>(w8 + L.tickets),                        \
         reinterpret_cast<unsigned*>(w8));                                                                             \

@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k_words = bits_k * kD, v_words = bits_v * kD;
+  const int k_words = bits_k * kD;
   uint32_t* wbase = smem + 512 + warp * (Row::kWords + kQuantExtraWords);
   uint32_t* rows = wbase;
   float* sA = reinterpret_cast<float*>(wbase + Row::kWords);             // 32 value scales
@@ -269,8 +269,8 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
     const bool valid = lane < valid_rows;
     uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
     uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
-    uint32_t* vout = kout + k_words;
-    uint16_t* norms = reinterpret_cast<uint16_t*>(vout + v_words);
+    uint16_t* norms = reinterpret_cast<uint16_t*>(kout + k_words);   // 32 K norms, then 32 V norms
+    uint32_t* vout = kout + k_words + kTile;
 
     // ---------------------------------------------------------------- K (Block-GTQ widths)
     __syncwarp();

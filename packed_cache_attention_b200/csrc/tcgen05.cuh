@@ -46,20 +46,24 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
       : "memory");
 }
 
+// One try: the thread is suspended until the phase completes or about `kSuspendNs`
+// nanoseconds pass (a hint; it then returns false), so waiting warps do not take issue slots.
+constexpr uint32_t kSuspendNs = 1u << 20;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
 
-// Bounded wait: spins at most `limit` times (each try_wait itself suspends for a
-// hardware-defined interval); returns false when the phase never completed.
+// Bounded wait: at most `limit` suspended tries (about limit * 1 ms); returns false when the
+// phase never completed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
   for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
@@ -108,6 +112,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------- TMEM loads / stores (32x32b)
+// Stores name no memory clobber: they write tensor memory only, and their order against the
+// code that follows is kept by tcgen05.wait::st and the fences (volatile statements, which the
+// compiler does not reorder); a clobber would make every shared-memory value after a store be
+// reloaded.
 
 template <int N>
 __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]);
@@ -119,20 +127,20 @@ __device__ __forceinline__ void tmem_st<1>(uint32_t taddr, const uint32_t (&r)[1
 template <>
 __device__ __forceinline__ void tmem_st<2>(uint32_t taddr, const uint32_t (&r)[2]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(r[0]), "r"(r[1])
-               : "memory");
+               );
 }
 template <>
 __device__ __forceinline__ void tmem_st<4>(uint32_t taddr, const uint32_t (&r)[4]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]),
                "r"(r[1]), "r"(r[2]), "r"(r[3])
-               : "memory");
+               );
 }
 template <>
 __device__ __forceinline__ void tmem_st<8>(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]),
       "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-      : "memory");
+      );
 }
 template <>
 __device__ __forceinline__ void tmem_st<16>(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -141,7 +149,7 @@ __device__ __forceinline__ void tmem_st<16>(uint32_t taddr, const uint32_t (&r)[
       "%13, %14, %15, %16};" ::"r"(taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
+      );
 }
 
 template <int N>
@@ -177,6 +185,18 @@ __device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t (&r)[16]) {
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
+      : "memory");
+}
+
+// Two 2-column loads and the wait for them in one statement, so that no use of the results
+// can be scheduled before the wait.
+__device__ __forceinline__ void tmem_ld2x2_wait(uint32_t ta, uint32_t tb, uint32_t (&a)[2], uint32_t (&b)[2]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%4];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%2, %3}, [%5];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(b[0]), "=r"(b[1])
+      : "r"(ta), "r"(tb)
       : "memory");
 }
 

@@ -54,7 +54,10 @@ class HeadAlloc(ctypes.Structure):
                 ("class_blocks", ctypes.c_uint8 * 8), ("reserved_b", ctypes.c_uint8 * 56),
                 ("head_dim", ctypes.c_int32), ("bits_k", ctypes.c_int32), ("w_max", ctypes.c_int32),
                 ("mode", ctypes.c_int32), ("n_classes", ctypes.c_int32), ("k_words", ctypes.c_int32),
-                ("n_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("n_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("plan_run", (ctypes.c_uint32 * 8) * 4), ("plan_group", (ctypes.c_uint32 * 16) * 4),
+                ("plan_col_block", ctypes.c_int8 * 128), ("plan_n_runs", ctypes.c_int32 * 4),
+                ("plan_k_cols", ctypes.c_int32), ("reserved_c", ctypes.c_uint8 * 108)]
 
 
 _VP = ctypes.c_void_p
@@ -183,6 +186,10 @@ def parse_alloc(raw: np.ndarray) -> list[dict]:
             "class_first": np.array(rec.class_first[:], dtype=np.int64),
             "class_blocks": np.array(rec.class_blocks[:], dtype=np.int64),
             "n_classes": rec.n_classes, "n_blocks": rec.n_blocks, "k_words": rec.k_words,
+            "plan_col_block": np.array(rec.plan_col_block[:], dtype=np.int64), "plan_k_cols": rec.plan_k_cols,
+            "plan_n_runs": np.array(rec.plan_n_runs[:], dtype=np.int64),
+            "plan_run": np.array([list(r) for r in rec.plan_run], dtype=np.int64),
+            "plan_group": np.array([list(r) for r in rec.plan_group], dtype=np.int64),
             "bits_k": rec.bits_k, "w_max": rec.w_max,
             "mode": rec.mode,
         })

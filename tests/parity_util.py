@@ -35,6 +35,7 @@ def compare_alloc(gpu_heads, ref):
         np.testing.assert_array_equal(g["bit_off"], bg.k_bit_offsets(ref["w"][h]))
         assert g["k_words"] == int(2 * ref["w"][h].sum())
         check_classes(g, ref["w"][h])
+        check_plan(g, ref["w"][h])
 
 
 def check_classes(g, w):
@@ -54,6 +55,35 @@ def check_classes(g, w):
         assert g["class_bit"][c] == bit
         bit += 2 * cw * len(blocks)
     assert all(x == 0 for x in g["class_width"][len(widths):])
+
+
+def check_plan(g, w):
+    """Decode plan: every block with w > 0 owns exactly one column; each group starts at the
+    bit offset of its first block and covers consecutive columns of one width."""
+    cb = g["plan_col_block"]
+    kc = g["plan_k_cols"]
+    assert kc == 96
+    blocks = [int(x) for x in cb if x >= 0]
+    assert sorted(blocks) == [b for b in range(len(w)) if w[b] > 0]
+    assert all(x == -1 for x in cb[kc:])
+    off = bg.k_bit_offsets(w)
+    seen = 0
+    for wg in range(4):
+        for r in range(int(g["plan_n_runs"][wg])):
+            e = int(g["plan_run"][wg][r])
+            width, first, n, half = e & 15, (e >> 8) & 0xff, (e >> 16) & 0xff, e >> 24
+            for i in range(n):
+                ge = int(g["plan_group"][wg][first + i])
+                bit, col = ge & 0xffff, ge >> 16
+                npairs = 2 if (half and i == n - 1) else 4
+                b0 = int(cb[col])
+                assert b0 >= 0 and w[b0] == width and off[b0] == bit
+                for k in range(npairs):
+                    bk = int(cb[col + k])
+                    if bk >= 0:
+                        assert w[bk] == width and off[bk] == bit + 2 * width * k
+                seen += 1
+    assert seen == sum(-(-sum(1 for x in w if x == cw) // 4) for cw in set(int(x) for x in w if x > 0))
 
 
 def oracle_pipeline(K, V, q, bits_k, bits_v, n_calib=0, w_max=8, mode=0, capacity=None):

@@ -40,10 +40,10 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_struct_sizes_match_header(L):
-    assert ctypes.sizeof(kvq.HeadAlloc) == 1408
+    assert ctypes.sizeof(kvq.HeadAlloc) == 2048
     assert ctypes.sizeof(kvq.Tensor4) == 48
-    assert kvq.kvq_alloc_bytes(3) == 3 * 1408
-    assert kvq.kvq_abi_version() == 2
+    assert kvq.kvq_alloc_bytes(3) == 3 * 2048
+    assert kvq.kvq_abi_version() == 3
 
 
 @pytest.mark.parametrize("w", range(1, 9))

@@ -427,10 +427,17 @@ def test_pack_single_code_position_by_hand():
     Kc[0, 0, 5, 5] = 0b111
     Vc = np.zeros((1, 1, 32, 128), np.uint8)
     Vc[0, 0, 13, 70] = 0b011
-    codes = {"Kc": Kc, "Kn": np.zeros((1, 1, 32), np.float16), "Vc": Vc, "Vn": np.zeros((1, 1, 32), np.float16)}
+    Kn = np.zeros((1, 1, 32), np.float16)
+    Vn = np.zeros((1, 1, 32), np.float16)
+    Kn[0, 0, 3] = 1.5
+    Vn[0, 0, 7] = -2.0
+    codes = {"Kc": Kc, "Kn": Kn, "Vc": Vc, "Vn": Vn}
     packed = bg.pack_cache(codes, a, 3, 32)
-    words = packed[0, 0, 0, :4 * (384 + 384)].copy().view("<u4")
-    kw, vw = words[:384], words[384:]
+    norms = packed[0, 0, 0, 4 * 384:4 * 384 + 128].copy().view("<f2")       # K norms, then V norms
+    assert norms[3] == 1.5 and norms[32 + 7] == -2.0 and np.count_nonzero(norms) == 2
+    kw = packed[0, 0, 0, :4 * 384].copy().view("<u4")
+    vw = packed[0, 0, 0, 4 * 384 + 128:].copy().view("<u4")
+    assert vw.shape == (384,)
     nz = {i: int(x) for i, x in enumerate(kw) if x}
     assert nz == {9: 0b101 << 21, 5: 0b11 << 30, 37: 1}
     vnz = {i: int(x) for i, x in enumerate(vw) if x}
