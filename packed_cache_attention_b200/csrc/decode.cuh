@@ -35,9 +35,10 @@
 namespace kvq {
 
 constexpr int kDecComputeWarps = 16;
-constexpr int kDecMmaWarp = 16;
+constexpr int kDecMmaWarp = 16;      // builds Q', issues the MMAs of even chunks
 constexpr int kDecLoadWarp = 17;
-constexpr int kDecThreads = 18 * 32;
+constexpr int kDecMma2Warp = 18;     // issues the MMAs of odd chunks
+constexpr int kDecThreads = 19 * 32;
 constexpr int kChunkTiles = 4;
 constexpr int kChunkTokens = kChunkTiles * kTile;   // = MMA M = tensor-memory lanes
 constexpr int kSegChunks = 16;                       // chunks per two-pass segment
@@ -54,10 +55,12 @@ constexpr uint32_t kWaitLimit = 2000;   // suspended tries (about 2 s) before a 
 
 // Tensor-memory columns (512 allocated).
 constexpr uint32_t kTmemCols = 512;
-__device__ __forceinline__ uint32_t col_ak(int b) { return 128u * b; }        // K-hat, 2 x 128
-__device__ __forceinline__ uint32_t col_s(int b) { return 256u + 16u * b; }   // S, 2 x 16
-__device__ __forceinline__ uint32_t col_av(int b) { return 288u + 64u * b; }  // V-hat^T, 2 x 64
-constexpr uint32_t kColO = 416;                                                // O, 16
+// The key pass keeps 3 chunks in flight (its logits trail the dequantization by 2 chunks),
+// the value pass 2.
+__device__ __forceinline__ uint32_t col_ak(int b) { return 96u * b; }         // K-hat, 3 x 96
+__device__ __forceinline__ uint32_t col_s(int b) { return 288u + 16u * b; }   // S, 3 x 16
+__device__ __forceinline__ uint32_t col_av(int b) { return 336u + 64u * b; }  // V-hat^T, 2 x 64
+__device__ __forceinline__ uint32_t col_o(int p) { return 464u + 16u * p; }  // O, 2 x 16 (chunk parity)
 
 // Lookup-table image, built once per device (decode_lut_image) and bulk-copied into every
 // CTA's shared memory at byte 0. Pair tables give the fp16 pair {c[i & m], c[i >> w]} for the
@@ -87,7 +90,7 @@ static_assert(kBQOff >= kAllocOff + static_cast<int>(sizeof(kvq_head_alloc)) && 
 struct DecHeader {
   uint64_t full[kDecStagesMax];
   uint64_t empty[kDecStagesMax];
-  uint64_t kready[2], vpready[2], sfull[2], ofull[2];
+  uint64_t kready[3], sfull[3], vpready[2], ofull[2];
   uint64_t setup;                    // lookup tables + allocation record copied in
   uint64_t qready;                   // Q' and qscale written (MMA warp)
   uint32_t tmem_base;
@@ -343,7 +346,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
   const int tstride = stage_tile_stride(bits_k, bits_v);
   const int stage_bytes = kChunkTiles * tstride;
   const float inv_sqrt_d = 0.08838834764831845f;
-  constexpr int kSetupThreads = (kDecComputeWarps + 1) * 32;
+  constexpr int kSetupThreads = (kDecComputeWarps + 2) * 32;   // compute warps and both MMA warps
 
   // ------------------------------------------------------------------ barriers
   if (tid == 0) {
@@ -351,10 +354,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
       tc::mbar_init(&S.full[i], 1);
       tc::mbar_init(&S.empty[i], kDecComputeWarps);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       tc::mbar_init(&S.kready[i], kDecComputeWarps);
-      tc::mbar_init(&S.vpready[i], kDecComputeWarps);
       tc::mbar_init(&S.sfull[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&S.vpready[i], kDecComputeWarps);
       tc::mbar_init(&S.ofull[i], 1);
     }
     tc::mbar_init(&S.setup, 1);
@@ -407,7 +412,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
     if (!tc::mbar_wait(&S.setup, 0, kWaitLimit)) record_timeout(status);
     const kvq_head_alloc& A = *reinterpret_cast<const kvq_head_alloc*>(sm + kAllocOff);
 
-    if (warp == kDecMmaWarp) {
+    if (warp == kDecMmaWarp || warp == kDecMma2Warp) {
+      const int par = (warp == kDecMmaWarp) ? 0 : 1;   // chunk parity this warp issues for
+      const int k_cols = 4 * kSlotCols;
+      if (par == 0) {
       // -------------------------------------------------------------- Q' (whole warp)
       // Row h: q_h * f_b * log2(e) / sqrt(d), scaled by 2^-e so that its largest |value| is in
       // [0.5, 1); qscale[h] = 2^e multiplies the product back. B operand of S, K-major, no
@@ -440,7 +448,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
         for (int u = 0; u < 4; ++u) qtmp[hg * kD + lane + 32 * u] = qv[hg][u] * sc;
       }
       __syncwarp();
-      const int k_cols = 4 * kSlotCols;
       const int k_elems = 2 * k_cols;
       for (int i = lane; i < 8 * k_elems; i += 32) {
         const int n = i / k_elems, k = i - n * k_elems;
@@ -453,32 +460,54 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
       }
       tc::fence_proxy_async_smem();
       __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&S.qready);
+      }
       // -------------------------------------------------------------- MMA issue
+      // Two issuing threads, one per chunk parity: independent MMA chains overlap in the
+      // tensor pipe, whose cost per instruction is mostly latency at these small tiles.
       if (lane == 0) {
-        tc::mbar_arrive(&S.qready);
+        if (par == 1 && !tc::mbar_wait(&S.qready, 0, kWaitLimit)) record_timeout(status);
         const uint32_t id_s = tc::idesc_f16(128, 16, false), id_o = tc::idesc_f16(128, 16, true);
         const uint32_t bq = tc::smem_u32(sm + kBQOff), bp = tc::smem_u32(sm + kBPOff);
-        const int ksteps = k_cols / 8;
+        // k-steps (8 columns each) that hold at least one real block pair
+        uint32_t kmask = 0u;
+        for (int c = 0; c < k_cols; ++c)
+          if (A.plan_col_block[c] >= 0) kmask |= 1u << (c >> 3);
+        const int first_ks = __ffs(kmask) - 1;
+        // Every k-step's B descriptor, built once (the 14-bit start field wraps, so offsets are
+        // not added to a built descriptor).
+        uint64_t dq[12], dpv[2][kChunkTokens / 16];
+#pragma unroll
+        for (int ks = 0; ks < 12; ++ks) dq[ks] = tc::sdesc(bq + 512 * ks, 256, 128);
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+          for (int ks = 0; ks < kChunkTokens / 16; ++ks)
+            dpv[bb][ks] = (bb == par) ? tc::sdesc(bp + kBPBytes * bb + 512 * ks, 256, 128) : 0ull;
         int kc = 0, vc = 0;
         bool ok = true;
         for (int sg = 0; sg < n_segs && ok; ++sg) {
           const int nu = min(kSegChunks, n_chunks - sg * kSegChunks);
           for (int u = 0; u < nu; ++u, ++kc) {
-            const int bb = kc & 1;
-            if (!tc::mbar_wait(&S.kready[bb], (kc >> 1) & 1, kWaitLimit)) { ok = false; break; }
+            if ((kc & 1) != par) continue;
+            const int bb = kc % 3;
+            if (!tc::mbar_wait(&S.kready[bb], (kc / 3) & 1, kWaitLimit)) { ok = false; break; }
             tc::fence_after_sync();
-            for (int ks = 0; ks < ksteps; ++ks)
-              tc::mma_ts(tbase + col_s(bb), tbase + col_ak(bb) + 8 * ks, tc::sdesc(bq + 512 * ks, 256, 128), id_s,
-                         ks > 0);
+            const uint32_t d = tbase + col_s(bb), a = tbase + col_ak(bb);
+#pragma unroll
+            for (int ks = 0; ks < 12; ++ks)
+              if (kmask & (1u << ks)) tc::mma_ts(d, a + 8 * ks, dq[ks], id_s, ks != first_ks);
             tc::mma_commit(&S.sfull[bb]);
           }
           for (int u = 0; u < nu && ok; ++u, ++vc) {
+            if ((vc & 1) != par) continue;
             const int bb = vc & 1;
             if (!tc::mbar_wait(&S.vpready[bb], (vc >> 1) & 1, kWaitLimit)) { ok = false; break; }
             tc::fence_after_sync();
-            for (int ks = 0; ks < kChunkTokens / 16; ++ks)
-              tc::mma_ts(tbase + kColO, tbase + col_av(bb) + 8 * ks, tc::sdesc(bp + kBPBytes * bb + 512 * ks, 256, 128),
-                         id_o, (u > 0 || ks > 0) ? 1u : 0u);
+            const uint32_t a = tbase + col_av(bb), d = tbase + col_o(bb);
+            tc::mma_ts(d, a, dpv[par][0], id_o, u >= 2);   // first chunk of this parity starts O
+#pragma unroll
+            for (int ks = 1; ks < kChunkTokens / 16; ++ks) tc::mma_ts(d, a + 8 * ks, dpv[par][ks], id_o, 1u);
             tc::mma_commit(&S.ofull[bb]);
           }
         }
@@ -521,14 +550,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
 
       // Logits of chunk u of the segment (K count j): s = S * knorm * qscale, -inf past the end.
       auto logits = [&](int u0, int u, int j, float kn, float& sm0, float& sm1) {
-        const int bj = j & 1;
+        const int bj = j % 3;
         if (!have_q) {   // Q' scaling of this warp group's rows (written by the MMA warp)
           if (ok && !tc::mbar_wait(&S.qready, 0, kWaitLimit)) ok = false;
           qs0 = S.qscale[2 * wg];
           qs1 = S.qscale[2 * wg + 1];
           have_q = true;
         }
-        if (ok && !tc::mbar_wait(&S.sfull[bj], (j >> 1) & 1, kWaitLimit)) ok = false;
+        if (ok && !tc::mbar_wait(&S.sfull[bj], (j / 3) & 1, kWaitLimit)) ok = false;
         tc::fence_after_sync();
         uint32_t sh[2], sl[2];
         tc::tmem_ld2x2_wait(tbase + lane_base + col_s(bj) + 2 * wg, tbase + lane_base + col_s(bj) + 8 + 2 * wg, sh, sl);
@@ -546,13 +575,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
       for (int sg = 0; sg < n_segs; ++sg) {
         const int u0 = sg * kSegChunks, nu = min(kSegChunks, n_chunks - u0);
         // ------------------------------------------------------------ pass 1: keys
-        float sm0 = -INFINITY, sm1 = -INFINITY, kn_prev = 0.0f;
+        float sm0 = -INFINITY, sm1 = -INFINITY, kn1 = 0.0f, kn2 = 0.0f;   // norms of chunks u-1, u-2
         for (int u = 0; u < nu; ++u, ++k) {
           const int s = k % n_stages, j = kc0 + u;
           if (ok && !tc::mbar_wait(&S.full[s], (k / n_stages) & 1, kWaitLimit)) ok = false;
           const uint8_t* st = stages + s * stage_bytes + qt * tstride;   // tile qt: token `lane`
           const uint32_t* kw = reinterpret_cast<const uint32_t*>(st) + lane;
-          const uint32_t ta = tbase + lane_base + col_ak(j & 1) + kSlotCols * wg;
+          const uint32_t ta = tbase + lane_base + col_ak(j % 3) + kSlotCols * wg;
           {
             uint32_t t[kSlots][kGroupPairs];
 #pragma unroll
@@ -570,13 +599,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
           tc::fence_before_sync();
           __syncwarp();
           if (lane == 0) {
-            tc::mbar_arrive(&S.kready[j & 1]);
+            tc::mbar_arrive(&S.kready[j % 3]);
             tc::mbar_arrive(&S.empty[s]);
           }
-          if (u >= 1) logits(u0, u - 1, j - 1, kn_prev, sm0, sm1);
-          kn_prev = kn;
+          if (u >= 2) logits(u0, u - 2, j - 2, kn2, sm0, sm1);
+          kn2 = kn1;
+          kn1 = kn;
         }
-        logits(u0, nu - 1, kc0 + nu - 1, kn_prev, sm0, sm1);
+        if (nu >= 2) logits(u0, nu - 2, kc0 + nu - 2, kn2, sm0, sm1);
+        logits(u0, nu - 1, kc0 + nu - 1, kn1, sm0, sm1);
         kc0 += nu;
         // ------------------------------------------------------------ segment maximum
         {
@@ -637,14 +668,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
         }
         vc0 += nu;
         // ------------------------------------------------------------ segment O
+        // One accumulator per chunk parity: wait for the last chunk of each, add both.
         {
           const int jl = vc0 - 1;
-          if (ok && !tc::mbar_wait(&S.ofull[jl & 1], (jl >> 1) & 1, kWaitLimit)) ok = false;
-          tc::fence_after_sync();
-          uint32_t oh[2], ol[2];
-          tc::tmem_ld2x2_wait(tbase + lane_base + kColO + 2 * wg, tbase + lane_base + kColO + 8 + 2 * wg, oh, ol);
-          o0 += __uint_as_float(oh[0]) + __uint_as_float(ol[0]);
-          o1 += __uint_as_float(oh[1]) + __uint_as_float(ol[1]);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int jq = jl - q;
+            if (q == 1 && nu < 2) break;
+            if (ok && !tc::mbar_wait(&S.ofull[jq & 1], (jq >> 1) & 1, kWaitLimit)) ok = false;
+            tc::fence_after_sync();
+            uint32_t oh[2], ol[2];
+            tc::tmem_ld2x2_wait(tbase + lane_base + col_o(jq & 1) + 2 * wg, tbase + lane_base + col_o(jq & 1) + 8 + 2 * wg,
+                                oh, ol);
+            o0 += __uint_as_float(oh[0]) + __uint_as_float(ol[0]);
+            o1 += __uint_as_float(oh[1]) + __uint_as_float(ol[1]);
+          }
           tc::fence_before_sync();
         }
       }
