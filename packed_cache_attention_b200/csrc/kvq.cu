@@ -314,16 +314,21 @@ kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, con
   const long long n_tasks = static_cast<long long>(c->batch) * c->n_kv_heads * tiles_written;
   const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
   const size_t smem = quant_smem_bytes(kd->dtype);
-  const int ctas_per_sm = static_cast<int>(std::max<size_t>(1, (227u * 1024u) / smem));
-  const long long want = (n_tasks + kQuantWarps - 1) / kQuantWarps;
-  const unsigned grid = static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sm_count()) * ctas_per_sm));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Persistent grid: exactly the CTAs that are resident at once (registers and shared memory
+  // both limit it), so every warp starts at launch and the tiles are spread evenly.
 #define KVQ_LAUNCH_QUANT(DT, TY)                                                                                  \
   do {                                                                                                            \
     auto kern = kvq_quant_pack<DT>;                                                                               \
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=        \
         cudaSuccess)                                                                                              \
       return KVQ_ERR_CUDA;                                                                                        \
+    int per_sm = 0;                                                                                               \
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQuantWarps * 32, smem) != cudaSuccess)     \
+      return KVQ_ERR_CUDA;                                                                                        \
+    const long long want = (n_tasks + kQuantWarps - 1) / kQuantWarps;                                           \
+    const unsigned grid =                                                                                         \
+        static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sm_count()) * std::max(1, per_sm))); \
     kern<<<grid, kQuantWarps * 32, smem, s>>>(static_cast<const TY*>(K), kd->stride_b, kd->stride_h, kd->stride_t, \
                                                static_cast<const TY*>(V), vd->stride_b, vd->stride_h, vd->stride_t, \
                                                kd->seq_len, c->n_kv_heads, tiles_written, tiles_cap,              \
