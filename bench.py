@@ -234,6 +234,7 @@ def run_gpu(args, rank, world, local_rank):
 
     nf4 = (measure_nf4(kvq, wl, dev, stream, hbm_peak=peaks()[0], batch=args.nf4_batch)
            if (rank == 0 and not args.no_nf4) else None)
+    append = measure_append(kvq, Ks[0], Vs[0], allocs[0], cache, packs[0], stream, T) if rank == 0 else None
 
     steps = args.steps
     ms_step = total_ms / steps
@@ -280,11 +281,41 @@ def run_gpu(args, rank, world, local_rank):
             "compression_vs_bf16": (2 * 2 * d) / (d_bytes / (B * Hkv * T)),
         },
         "nf4": nf4,
+        "append": append,
         "e2e": e2e,
         "gpu_launches": steps * L * 4,
         "clocks": clocks,
     }
     return result
+
+
+def measure_append(kvq, K, V, alloc, cache, packed, stream, T, iters=50, chunk=4096):
+    """Decode-step growth of the packed cache: one token appended at position T - 1 (a partly
+    filled tile, so the value words are merged), and a 4096-token chunk (chunked prefill).
+    The same tokens are re-appended, so the cache content is unchanged."""
+    import torch
+
+    def timed(fn, n):
+        fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        z.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(z) / n
+
+    k1, v1 = K[:, :, T - 1:T], V[:, :, T - 1:T]
+    one_ms = timed(lambda: kvq.kvq_append(k1, v1, alloc, cache, T - 1, packed, stream=stream), iters)
+    kc, vc = K[:, :, T - chunk:T], V[:, :, T - chunk:T]
+    chunk_ms = timed(lambda: kvq.kvq_append(kc, vc, alloc, cache, T - chunk, packed, stream=stream), iters)
+    B, H = K.shape[0], K.shape[1]
+    per_tok = 2 * 2 * K.shape[3] + kvq.kvq_packed_bytes(cache) // (B * H * T)
+    return {"one_token_launch_ms": one_ms, "chunk_tokens": chunk, "chunk_launch_ms": chunk_ms,
+            "chunk_tokens_per_s": B * H * chunk / (chunk_ms * 1e-3),
+            "chunk_gb_s": B * H * chunk * per_tok / (chunk_ms * 1e-3) / 1e9}
 
 
 def measure_nf4(kvq, wl, dev, stream, hbm_peak, iters=10, batch=0):

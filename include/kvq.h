@@ -207,6 +207,22 @@ kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_p
 kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd,
                         const void* alloc, const kvq_cache_desc* cache, void* packed, void* stream);
 
+/* Append tokens to a packed cache ([NQKV] assumptions: the cache only grows, so new tokens are
+ * encoded without re-quantizing the stored ones; Fig. 6, decoding phase: each new token's
+ * keys and values are quantized and appended). Quantizes tokens t_begin .. t_begin + n - 1,
+ * n = kd->seq_len, exactly as kvq_quantize quantizes them (the per-row quantizer depends on
+ * nothing but the row and the allocation), so appending a sequence in any number of calls
+ * stores the same bytes as one kvq_quantize call.
+ * K, V: [batch][n_kv_heads][n][128]; input row i is token t_begin + i. Codes and norms of
+ * tokens below t_begin in the first touched tile are kept (read back and merged); tokens from
+ * t_begin + n to the end of the last touched tile are stored as code 0, norm 0. Tiles before
+ * t_begin / 32 and after the last touched tile are not accessed.
+ * Requires 0 <= t_begin and t_begin + n <= cache->capacity (else KVQ_ERR_RANGE); the stored
+ * tokens below t_begin must have been written by an earlier call on the same stream (or one
+ * that has completed). Attend over the grown cache with kvq_decode_attn(seq_len = t_begin + n). */
+kvq_status kvq_append(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd,
+                      const void* alloc, const kvq_cache_desc* cache, int t_begin, void* packed, void* stream);
+
 /* Fused decode attention straight from the packed cache ([BGTQ]: packed-cache serving path).
  * q: [batch][n_q_heads][1][128] (qd->seq_len must be 1), query head hq reads KV head
  * hq / (n_q_heads / n_kv_heads); n_q_heads / n_kv_heads must be 1..8.

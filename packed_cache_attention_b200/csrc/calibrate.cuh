@@ -170,16 +170,23 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta, 4) kvq_calib_reduce(
 //     by binary search), and the picked entries of a block are a prefix: w_b = their count.
 //  2. g_b, f_b, the K word offsets and the decode k-step table (blocks grouped by width,
 //     widest first, 4 per step, ascending block index within a width).
+// The record is built in shared memory and copied out whole at the end.
 __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict__ energy, int bits_k, int w_max,
                                                         int mode, kvq_head_alloc* __restrict__ alloc) {
+  static_assert(sizeof(kvq_head_alloc) % 16 == 0 && sizeof(kvq_head_alloc) <= 512 * 16, "record copy");
   __shared__ double sE[kH];
   __shared__ long long sKey[kH * 8];
   __shared__ short sIdx[kH * 8];
   __shared__ int sWidth[kH];
   __shared__ int sCount[9];
+  __shared__ int sClsX0[9];
   __shared__ double sSum;
+  __shared__ __align__(16) kvq_head_alloc sRec;
   const int h = blockIdx.x, tid = threadIdx.x;
-  kvq_head_alloc* al = alloc + h;
+  kvq_head_alloc* al = &sRec;
+  uint32_t* rec_words = reinterpret_cast<uint32_t*>(&sRec);
+  constexpr int kRecWords = static_cast<int>(sizeof(kvq_head_alloc) / 4);
+  for (int i = tid; i < kRecWords; i += blockDim.x) rec_words[i] = 0u;
   if (tid < kH) sE[tid] = __ldcg(energy + static_cast<size_t>(h) * kH + tid);
   __syncthreads();
   if (tid == 0) {
@@ -206,24 +213,34 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     // the first bits_k * 64 are the greedy's picks. Non-negative doubles order like their
     // bit patterns, so keys are 64-bit integers; entries at or above w_max get key -1 and
     // sort after every valid one.
-    __syncthreads();
+    // Compare-exchange distances of 32 and more go through shared memory, shorter ones
+    // between the lanes of a warp (thread tid holds entry tid in registers there).
+    long long key = sKey[tid];
+    int idx = sIdx[tid];
     for (int k = 2; k <= kH * 8; k <<= 1) {
       for (int j = k >> 1; j > 0; j >>= 1) {
-        const int i = tid, ixj = tid ^ j;
-        if (ixj > i) {
-          const long long ka = sKey[i], kb = sKey[ixj];
-          const int ia = sIdx[i], ib = sIdx[ixj];
-          const bool a_first = (ka > kb) || (ka == kb && ia < ib);
-          const bool want_a_first = (i & k) == 0;
-          if (a_first != want_a_first) {
-            sKey[i] = kb; sKey[ixj] = ka;
-            sIdx[i] = static_cast<short>(ib); sIdx[ixj] = static_cast<short>(ia);
-          }
+        if (j >= 32) {
+          sKey[tid] = key;
+          sIdx[tid] = static_cast<short>(idx);
+          __syncthreads();
+          const long long ko = sKey[tid ^ j];
+          const int io = sIdx[tid ^ j];
+          __syncthreads();
+          const bool lower = (tid & j) == 0;                     // this thread holds the pair's first slot
+          const bool up = (tid & k) == 0;                        // the pair's block sorts descending-first
+          const bool mine_first = (key > ko) || (key == ko && idx < io);
+          if (mine_first != (lower == up)) { key = ko; idx = io; }
+        } else {
+          const long long ko = __shfl_xor_sync(0xffffffffu, key, j);
+          const int io = __shfl_xor_sync(0xffffffffu, idx, j);
+          const bool lower = (tid & j) == 0;
+          const bool up = (tid & k) == 0;
+          const bool mine_first = (key > ko) || (key == ko && idx < io);
+          if (mine_first != (lower == up)) { key = ko; idx = io; }
         }
-        __syncthreads();
       }
     }
-    if (tid < bits_k * kH) atomicAdd(&sWidth[sIdx[tid] >> 3], 1);
+    if (tid < bits_k * kH) atomicAdd(&sWidth[idx >> 3], 1);
   }
   if (tid < 9) sCount[tid] = 0;
   __syncthreads();
@@ -237,26 +254,42 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     al->gain[b] = g;
     al->dequant[b] = __double2float_rn(__ddiv_rn(1.0, __dmul_rn(__dsqrt_rn(static_cast<double>(kD)),
                                                                 static_cast<double>(g))));
-    al->width[b] = static_cast<uint8_t>(sWidth[b]);
-    atomicAdd(&sCount[sWidth[b]], 1);
+    const int w = sWidth[b];
+    al->width[b] = static_cast<uint8_t>(w);
+    atomicAdd(&sCount[w], 1);
+    // Stream order: width classes 8..1, blocks ascending inside a class; each block is a
+    // pair of codes (dim b, dim b + 64) of w_b bits each. Block b's position and bit offset
+    // count the wider blocks and the lower blocks of its own width.
+    int pos = 0, bit = 0;
+    for (int c = 0; c < kH; ++c) {
+      const int wc = sWidth[c];
+      if (wc > w || (wc == w && c < b)) {
+        ++pos;
+        bit += 2 * wc;
+      }
+    }
+    if (w > 0) {
+      al->stream_block[pos] = static_cast<uint8_t>(b);
+      al->bit_off[b] = static_cast<int16_t>(bit);
+    } else {
+      al->bit_off[b] = -1;
+    }
   }
   __syncthreads();
-  // Stream order: width classes 8..1, blocks ascending inside a class; each block is a pair
-  // of codes (dim b, dim b + 64) of w_b bits each.
+  // Class table (stream order: widths 8..1) and, per class, its first group of the decode plan.
   if (tid == 0) {
-    int pos = 0, bit = 0, n_cls = 0;
+    int pos = 0, bit = 0, n_cls = 0, x0 = 0;
     for (int w = 8; w >= 1; --w) {
-      if (sCount[w] == 0) continue;
+      const int nb = sCount[w];
+      if (nb == 0) continue;
       al->class_width[n_cls] = static_cast<uint8_t>(w);
       al->class_first[n_cls] = static_cast<uint8_t>(pos);
-      al->class_blocks[n_cls] = static_cast<uint8_t>(sCount[w]);
+      al->class_blocks[n_cls] = static_cast<uint8_t>(nb);
       al->class_bit[n_cls] = static_cast<uint16_t>(bit);
-      for (int b = 0; b < kH; ++b) {
-        if (sWidth[b] != w) continue;
-        al->stream_block[pos++] = static_cast<uint8_t>(b);
-        al->bit_off[b] = static_cast<int16_t>(bit);
-        bit += 2 * w;
-      }
+      sClsX0[n_cls] = x0;
+      x0 += (nb + 3) >> 2;
+      pos += nb;
+      bit += 2 * w * nb;
       ++n_cls;
     }
     for (int c = n_cls; c < 8; ++c) {
@@ -264,52 +297,59 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
       al->class_first[c] = static_cast<uint8_t>(pos);
       al->class_blocks[c] = 0;
       al->class_bit[c] = static_cast<uint16_t>(bit);
+      sClsX0[c] = x0;
     }
-    for (int i = pos; i < kH; ++i) al->stream_block[i] = 0xffu;
-    for (int b = 0; b < kH; ++b)
-      if (sWidth[b] == 0) al->bit_off[b] = -1;
+    sClsX0[8] = x0;
     al->n_classes = n_cls;
     al->n_blocks = pos;
-    // Decode plan: classes in stream order cut into groups of 4 block pairs (the last group
-    // 2 pairs when at most 2 remain); group x goes to warp group g = x % 4 as entry i = x / 4
-    // and fills columns 24 g + 4 i .. + 3 of the tensor-core operand.
-    {
-      int x0 = 0, nr[4] = {0, 0, 0, 0};
-      for (int i = 0; i < 128; ++i) al->plan_col_block[i] = -1;
-      int first = 0, bit0 = 0;
-      for (int w = 8; w >= 1; --w) {
-        const int nb = sCount[w];
-        if (nb == 0) continue;
-        const int r = nb & 3, ng = (nb >> 2) + (r ? 1 : 0);
-        for (int k = 0; k < ng; ++k) {
-          const int x = x0 + k, g = x & 3, col = 24 * g + 4 * (x >> 2);
-          al->plan_group[g][x >> 2] = static_cast<uint32_t>(bit0 + 8 * w * k) | (static_cast<uint32_t>(col) << 16);
-          if (nr[g] == 0 || (al->plan_run[g][nr[g] - 1] & 15u) != static_cast<uint32_t>(w))
-            al->plan_run[g][nr[g]++] = static_cast<uint32_t>(w) | (static_cast<uint32_t>(x >> 2) << 8);
-          al->plan_run[g][nr[g] - 1] += 1u << 16;
-          if (k == ng - 1 && r != 0 && r <= 2) al->plan_run[g][nr[g] - 1] |= 1u << 24;
-          for (int i = 0; i < 4 && 4 * k + i < nb; ++i)
-            al->plan_col_block[col + i] = static_cast<int8_t>(al->stream_block[first + 4 * k + i]);
-        }
-        x0 += ng;
-        first += nb;
-        bit0 += 2 * w * nb;
-      }
-      for (int g = 0; g < 4; ++g) {
-        al->plan_n_runs[g] = nr[g];
-        for (int i = nr[g]; i < 8; ++i) al->plan_run[g][i] = 0u;
-      }
-      al->plan_k_cols = 96;
-    }
     al->k_words = bit / 32 * kTile;     // bits per token * 32 tokens / 32 bits per word
     al->head_dim = kD;
     al->bits_k = bits_k;
     al->w_max = w_max;
     al->mode = mode;
     al->reserved = 0;
+    al->plan_k_cols = 96;
   }
-  if (tid < 56) al->reserved_b[tid] = 0;
-  if (tid < 108) al->reserved_c[tid] = 0;
+  if (tid < kH && tid >= kH - sCount[0]) al->stream_block[tid] = 0xffu;   // positions past the last block
+  if (tid < 128) al->plan_col_block[tid] = -1;
+  __syncthreads();
+  // Decode plan: classes in stream order cut into groups of 4 block pairs (the last group
+  // 2 pairs when at most 2 remain); group x goes to warp group g = x % 4 as entry i = x / 4
+  // and fills columns 24 g + 4 i .. + 3 of the tensor-core operand. One thread per group.
+  const int n_groups = sClsX0[8];
+  if (tid < n_groups) {
+    const int x = tid;
+    int c = 0;
+    while (sClsX0[c + 1] <= x) ++c;
+    const int w = al->class_width[c], nb = al->class_blocks[c], first = al->class_first[c];
+    const int k = x - sClsX0[c], g = x & 3, col = 24 * g + 4 * (x >> 2);
+    al->plan_group[g][x >> 2] = static_cast<uint32_t>(al->class_bit[c] + 8 * w * k) | (static_cast<uint32_t>(col) << 16);
+    for (int i = 0; i < 4 && 4 * k + i < nb; ++i)
+      al->plan_col_block[col + i] = static_cast<int8_t>(al->stream_block[first + 4 * k + i]);
+  }
+  // Runs: a warp group's consecutive entries of one class; flagged when the run holds its
+  // class's last group and that group has 1 or 2 pairs. One thread per warp group.
+  if (tid >= 128 && tid < 132) {
+    const int g = tid - 128;
+    int nr = 0, prev = -1;
+    for (int x = g; x < n_groups; x += 4) {
+      int c = 0;
+      while (sClsX0[c + 1] <= x) ++c;
+      const int w = al->class_width[c], nb = al->class_blocks[c];
+      if (c != prev) {
+        al->plan_run[g][nr++] = static_cast<uint32_t>(w) | (static_cast<uint32_t>(x >> 2) << 8);
+        prev = c;
+      }
+      al->plan_run[g][nr - 1] += 1u << 16;
+      const int r = nb & 3;
+      if (x == sClsX0[c + 1] - 1 && r != 0 && r <= 2) al->plan_run[g][nr - 1] |= 1u << 24;
+    }
+    al->plan_n_runs[g] = nr;
+  }
+  __syncthreads();
+  uint4* dst = reinterpret_cast<uint4*>(alloc + h);
+  const uint4* src = reinterpret_cast<const uint4*>(&sRec);
+  for (int i = tid; i < kRecWords / 4; i += blockDim.x) dst[i] = src[i];
 }
 
 }  // namespace kvq

@@ -36,6 +36,9 @@ kvq_status ensure_tables() {
   static uint8_t lut[kLutBytes];
   decode_lut_image(t.centroid_f16, lut);
   if (cudaMemcpyToSymbol(g_dec_lut, lut, sizeof(lut)) != cudaSuccess) return KVQ_ERR_CUDA;
+  static uint32_t qlut[2 * kLutEntries];
+  if (!quant_lut_image(t.threshold, qlut)) return KVQ_ERR_UNSUPPORTED;
+  if (cudaMemcpyToSymbol(g_quant_lut, qlut, sizeof(qlut)) != cudaSuccess) return KVQ_ERR_CUDA;
   g_uploaded[dev] = true;
   return KVQ_OK;
 }
@@ -297,8 +300,12 @@ kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_p
   return launch_status();
 }
 
-kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, const void* alloc,
-                        const kvq_cache_desc* c, void* packed, void* stream) {
+namespace {
+
+// Quantizes tokens t_begin .. t_begin + kd->seq_len - 1 (input row i = token t_begin + i) into
+// their tiles of `packed`; the rest of a partly covered first tile keeps its stored codes.
+kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, const void* alloc,
+                        const kvq_cache_desc* c, int t_begin, void* packed, void* stream) {
   kvq_status st;
   if ((st = check_tensor(K, kd)) != KVQ_OK) return st;
   if ((st = check_tensor(V, vd)) != KVQ_OK) return st;
@@ -307,13 +314,17 @@ kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, con
   if (vd->dtype != kd->dtype || vd->batch != kd->batch || vd->n_heads != kd->n_heads || vd->seq_len != kd->seq_len)
     return KVQ_ERR_SHAPE;
   if (kd->batch != c->batch || kd->n_heads != c->n_kv_heads) return KVQ_ERR_SHAPE;
-  if (kd->seq_len > c->capacity) return KVQ_ERR_RANGE;
+  if (t_begin < 0 || static_cast<long long>(t_begin) + kd->seq_len > c->capacity) return KVQ_ERR_RANGE;
   if ((st = ensure_tables()) != KVQ_OK) return st;
-  const int tiles_written = n_tiles_of(kd->seq_len);
+  const int t_end = t_begin + kd->seq_len;
+  const int tile_lo = t_begin / kTile;
+  const int n_tiles = n_tiles_of(t_end) - tile_lo;
   const int tiles_cap = n_tiles_of(c->capacity);
-  const long long n_tasks = static_cast<long long>(c->batch) * c->n_kv_heads * tiles_written;
+  const long long n_tasks = static_cast<long long>(c->batch) * c->n_kv_heads * n_tiles;
+  if (n_tasks > 0x7fffffffLL - 4096LL * 64) return KVQ_ERR_RANGE;   // task indices are 32-bit
   const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
   const size_t smem = quant_smem_bytes(kd->dtype);
+  const int qw = quant_warps(kd->dtype);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Persistent grid: exactly the CTAs that are resident at once (registers and shared memory
   // both limit it), so every warp starts at launch and the tiles are spread evenly.
@@ -324,16 +335,16 @@ kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, con
         cudaSuccess)                                                                                              \
       return KVQ_ERR_CUDA;                                                                                        \
     int per_sm = 0;                                                                                               \
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kQuantWarps * 32, smem) != cudaSuccess)     \
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, qw * 32, smem) != cudaSuccess)              \
       return KVQ_ERR_CUDA;                                                                                        \
-    const long long want = (n_tasks + kQuantWarps - 1) / kQuantWarps;                                           \
+    const long long want = (n_tasks + qw - 1) / qw;                                                             \
     const unsigned grid =                                                                                         \
         static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sm_count()) * std::max(1, per_sm))); \
-    kern<<<grid, kQuantWarps * 32, smem, s>>>(static_cast<const TY*>(K), kd->stride_b, kd->stride_h, kd->stride_t, \
-                                               static_cast<const TY*>(V), vd->stride_b, vd->stride_h, vd->stride_t, \
-                                               kd->seq_len, c->n_kv_heads, tiles_written, tiles_cap,              \
-                                               static_cast<const kvq_head_alloc*>(alloc), c->bits_k, c->bits_v,   \
-                                               static_cast<uint8_t*>(packed), rec, n_tasks);                      \
+    kern<<<grid, qw * 32, smem, s>>>(static_cast<const TY*>(K), kd->stride_b, kd->stride_h, kd->stride_t,         \
+                                     static_cast<const TY*>(V), vd->stride_b, vd->stride_h, vd->stride_t, t_begin, \
+                                     t_end, tile_lo, n_tiles, c->n_kv_heads, tiles_cap,                           \
+                                     static_cast<const kvq_head_alloc*>(alloc), c->bits_k, c->bits_v,             \
+                                     static_cast<uint8_t*>(packed), rec, static_cast<int>(n_tasks));              \
   } while (0)
   switch (kd->dtype) {
     case KVQ_F32: KVQ_LAUNCH_QUANT(KVQ_F32, float); break;
@@ -342,6 +353,18 @@ kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, con
   }
 #undef KVQ_LAUNCH_QUANT
   return launch_status();
+}
+
+}  // namespace
+
+kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, const void* alloc,
+                        const kvq_cache_desc* c, void* packed, void* stream) {
+  return launch_quant(K, kd, V, vd, alloc, c, 0, packed, stream);
+}
+
+kvq_status kvq_append(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, const void* alloc,
+                      const kvq_cache_desc* c, int t_begin, void* packed, void* stream) {
+  return launch_quant(K, kd, V, vd, alloc, c, t_begin, packed, stream);
 }
 
 kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,

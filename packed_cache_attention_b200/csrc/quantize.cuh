@@ -2,114 +2,179 @@
 // width for V (page "RoPE-aware bit allocation for KV cache quantization", abstract: the
 // allocator sits on TurboQuant-MSE, K and V get matched bit budgets, the cache is packed).
 //
-// One warp per 32-token tile of one (sequence, KV head) at a time (persistent warps). For a
-// token row x (128 values):
+// For a token row x (128 values):
 //   s2   = sum_j x_j^2 in fp32, j ascending: fl32(s2 + fl32(x_j x_j))
 //   norm = fp16(fp32 sqrt(s2)) (round to nearest even)
 //   a    = fp32(sqrt(128)) / fp32(norm), 0 if norm == 0
 //   y_j  = fp32(fp32(x_j a) g_b)            (V: g = 1, the multiply is skipped as exact)
 //   code = #{thresholds of width w_b strictly below y_j}
-// The code is found by binary search over the 2^w - 1 sorted thresholds, most significant
-// bit first. Tokens past the sequence length get a NaN scale, so every comparison is false
-// and their codes are 0.
-// The tile is first copied into shared memory with a padded row pitch (65 words for 16-bit
-// inputs), so that 32 lanes reading one dim of their own rows hit 32 banks.
+//
+// Work split. Persistent warps; one warp owns a 32-token tile of one (sequence, KV head) at
+// a time. Each warp keeps two shared-memory tile buffers, one for K rows and one for V rows,
+// filled by cp.async (16-byte pieces, zero fill past the sequence end) one half-task ahead:
+// the next tile's K rows load while this tile's V codes are computed, and the next V rows
+// while the next K codes are computed. Rows sit at a pitch of 16-byte pieces plus one
+// (68 words for 16-bit inputs), so a lane reading 16 bytes of its own row and a warp
+// reading one word of one row are both free of bank conflicts.
+//
+// Code search. Width 1 is the sign. Wider codebooks use a lookup table on a uniform grid
+// of cells of 2^-max(w-2, 1) over [-R_w, R_w): no cell holds two thresholds, so for y in cell k
+//   code = (thresholds below the cell) + (y > the threshold inside the cell, if any),
+// with y clamped into the grid (NaN clamps to the lowest cell and compares false, so a NaN
+// scale yields code 0: tokens past the sequence end are written as code 0). The cell is
+// floor(y / cell) read off an fp32 fma rounded toward minus infinity into [2^23, 2^24).
+// This is the same count as a search over the sorted thresholds, ties going to the lower
+// code, for every fp32 y.
+//
 // K: lane t quantizes token t and appends its codes, in the allocation's stream order, to a
 //   32-bit accumulator; the accumulator fills at the same code for every lane, so each full
-//   word is one coalesced 128-byte warp store (word-planar tile layout).
+//   word is one coalesced 128-byte warp store (word-planar tile layout). Codes are built in
+//   groups of blocks at compile-time bit positions (4 blocks for widths up to 4, else 2) and
+//   each group is merged into the stream with one funnel shift.
 // V: lane l quantizes dims 2l, 2l+1, 64+2l, 65+2l for the 32 tokens of the tile, placing
 //   token t's code at bit bits_v * t of the dim's stream (positions known at compile time).
 #pragma once
+
+#include <cstring>
 
 #include "common.cuh"
 
 namespace kvq {
 
-constexpr int kQuantWarps = 8;
-constexpr int kQuantExtraWords = kTile + kH + kH / 4 + 8;   // per warp: 32 scales, 64 gains, 64 block indices, 8 classes
+// ---------------------------------------------------------------- code lookup table
 
-template <int DT> struct QuantRow;
-// 16-bit inputs: a row is 64 words (2 values each), pitch 65 words.
-template <int DT> struct QuantRow16 {
-  static constexpr int kPitch = kD / 2 + 1;
-  static constexpr int kWords = kTile * kPitch;
-  // Copy 32 rows (32 * 256 B, rows `row_stride` elements apart) into shared memory.
-  __device__ __forceinline__ static void load(uint32_t* dst, const void* src, int64_t row_stride, int valid_rows,
-                                              int lane) {
-    const uint8_t* s8 = static_cast<const uint8_t*>(src);
-    uint4 v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {             // all 16 loads in flight before any store
-      const int idx = i * 32 + lane;           // 16-byte chunk of the tile
-      const int r = idx >> 4, c = idx & 15;
-      v[i] = make_uint4(0u, 0u, 0u, 0u);
-      if (r < valid_rows) v[i] = __ldg(reinterpret_cast<const uint4*>(s8 + (static_cast<int64_t>(r) * row_stride * 2)) + c);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int idx = i * 32 + lane;
-      const int r = idx >> 4, c = idx & 15;
-      uint32_t* d = dst + r * kPitch + 4 * c;
-      d[0] = v[i].x; d[1] = v[i].y; d[2] = v[i].z; d[3] = v[i].w;
-    }
-  }
-  // Values 2i and 2i+1 of a row.
-  __device__ __forceinline__ static float2 pair(const uint32_t* row, int i) {
-    const uint32_t w = row[i];
-    if constexpr (DT == KVQ_BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-    else return __half22float2(*reinterpret_cast<const __half2*>(&w));
-  }
-  // Value j of a row.
-  __device__ __forceinline__ static float value(const uint32_t* row, int j) {
-    const uint32_t w = row[j >> 1];
-    const uint32_t u = (j & 1) ? (w >> 16) : (w & 0xffffu);
-    if constexpr (DT == KVQ_BF16) return __uint_as_float(u << 16);
-    else return __half2float(__ushort_as_half(static_cast<unsigned short>(u)));
-  }
-};
-template <> struct QuantRow<KVQ_BF16> : QuantRow16<KVQ_BF16> {};
-template <> struct QuantRow<KVQ_F16> : QuantRow16<KVQ_F16> {};
-// fp32 inputs: a row is 128 words, pitch 129 words.
-template <> struct QuantRow<KVQ_F32> {
-  static constexpr int kPitch = kD + 1;
-  static constexpr int kWords = kTile * kPitch;
-  __device__ __forceinline__ static void load(uint32_t* dst, const void* src, int64_t row_stride, int valid_rows,
-                                              int lane) {
-    const uint8_t* s8 = static_cast<const uint8_t*>(src);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {              // two batches of 16 loads in flight
-      uint4 v[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int idx = (16 * h + i) * 32 + lane;
-        const int r = idx >> 5, c = idx & 31;
-        v[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (r < valid_rows) v[i] = __ldg(reinterpret_cast<const uint4*>(s8 + (static_cast<int64_t>(r) * row_stride * 4)) + c);
+// Grid of width w (2..8): cells of 1/s_w, s_w = 2^max(w-2, 1), half-range kLutHalf[w] cells.
+constexpr int kLutHalf[9] = {0, 0, 2, 4, 10, 24, 56, 128, 288};
+constexpr int kLutOffset[9] = {0, 0, 0, 4, 12, 32, 80, 192, 448};
+constexpr int kLutEntries = 1024;
+
+__host__ __device__ constexpr int lut_scale(int w) { return 1 << (w > 3 ? w - 2 : 1); }
+
+// Host: builds the table from the fp32 thresholds (all widths concatenated, width w at
+// 2^w - w - 1). Entry k of width w is {number of thresholds below the cell's left edge,
+// bits of the threshold inside the cell or +inf}. Returns false if a cell would hold two
+// thresholds or a threshold falls outside the grid.
+inline bool quant_lut_image(const float* thresholds, uint32_t* out /* 2 * kLutEntries */) {
+  for (int w = 2; w <= 8; ++w) {
+    const float* t = thresholds + ((1 << w) - w - 1);
+    const int n = (1 << w) - 1, K = kLutHalf[w];
+    const double s = lut_scale(w);
+    for (int k = 0; k < 2 * K; ++k) {
+      const double lo = (k - K) / s, hi = (k - K + 1) / s;
+      uint32_t below = 0, inside = 0, tau = 0x7f800000u;
+      for (int i = 0; i < n; ++i) {
+        const double ti = t[i];
+        if (ti < lo) ++below;
+        else if (ti < hi) {
+          ++inside;
+          uint32_t b;
+          std::memcpy(&b, &t[i], 4);
+          tau = b;
+        }
       }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int idx = (16 * h + i) * 32 + lane;
-        const int r = idx >> 5, c = idx & 31;
-        uint32_t* d = dst + r * kPitch + 4 * c;
-        d[0] = v[i].x; d[1] = v[i].y; d[2] = v[i].z; d[3] = v[i].w;
-      }
+      if (inside > 1) return false;
+      out[2 * (kLutOffset[w] + k)] = below;
+      out[2 * (kLutOffset[w] + k) + 1] = tau;
     }
+    if (static_cast<double>(t[0]) < -K / s || static_cast<double>(t[n - 1]) >= K / s) return false;
   }
-  __device__ __forceinline__ static float2 pair(const uint32_t* row, int i) {
-    return make_float2(__uint_as_float(row[2 * i]), __uint_as_float(row[2 * i + 1]));
+  return true;
+}
+
+__device__ __align__(16) uint32_t g_quant_lut[2 * kLutEntries];
+
+// Code of y for width W (1..8) from the table in shared memory.
+template <int W>
+__device__ __forceinline__ uint32_t lut_code(float y, const uint2* __restrict__ lut) {
+  if constexpr (W == 1) {
+    return y > 0.0f ? 1u : 0u;
+  } else {
+    constexpr int K = kLutHalf[W];
+    constexpr float s = static_cast<float>(lut_scale(W));
+    constexpr float lo = -static_cast<float>(K) / s;
+    constexpr float hi = (static_cast<float>(K) - 0.5f) / s;   // inside the last cell
+    const float yc = fminf(fmaxf(y, lo), hi);                  // NaN -> lo
+    const float f = __fmaf_rd(yc, s, 12582912.0f + static_cast<float>(K));   // 1.5 * 2^23 + K + floor(yc s)
+    const int idx = __float_as_int(f) - 0x4B400000;
+    const uint2 e = lut[kLutOffset[W] + idx];
+    return e.x + (y > __uint_as_float(e.y) ? 1u : 0u);
   }
-  __device__ __forceinline__ static float value(const uint32_t* row, int j) { return __uint_as_float(row[j]); }
+}
+
+// Two fp32 products in one instruction, each rounded to nearest even.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t ua, ub, ud;
+  memcpy(&ua, &a, 8);
+  memcpy(&ub, &b, 8);
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(ud) : "l"(ua), "l"(ub));
+  float2 d;
+  memcpy(&d, &ud, 8);
+  return d;
+}
+
+// ---------------------------------------------------------------- tile staging
+
+template <int DT> struct QTile {
+  static constexpr int kRowWords = (DT == KVQ_F32) ? kD : kD / 2;
+  static constexpr int kPitch = kRowWords + 4;                 // words; 16-byte aligned rows
+  static constexpr int kWords = kTile * kPitch;
+  static constexpr int kPieces = kRowWords / 4;                // 16-byte pieces per row
+  static constexpr int kPerLane = kTile * kPieces / 32;        // pieces a lane copies
+  static constexpr int kWarps = (DT == KVQ_F32) ? 6 : 12;      // warps per CTA (one CTA per SM)
 };
 
-// fp16 norm of one row and the scale a = sqrt(128)/norm (0 for a zero norm).
+// Starts the copy of tile rows r_lo .. r_hi - 1 into `dst` (row r_lo at `src`, rows
+// `row_stride` elements apart); the other rows are zero-filled without reading global memory.
+template <int DT>
+__device__ __forceinline__ void tile_load_async(uint32_t* dst, const void* src, int64_t row_stride, int r_lo, int r_hi,
+                                                int lane) {
+  using Q = QTile<DT>;
+  constexpr int esz = (DT == KVQ_F32) ? 4 : 2;
+  const uint8_t* s8 = static_cast<const uint8_t*>(src);
+  const uint32_t d0 = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+#pragma unroll
+  for (int i = 0; i < Q::kPerLane; ++i) {
+    const int idx = i * 32 + lane;
+    const int r = idx / Q::kPieces, c = idx % Q::kPieces;
+    const bool ok = r >= r_lo && r < r_hi;
+    const uint8_t* g = ok ? s8 + static_cast<int64_t>(r - r_lo) * row_stride * esz + 16 * c : s8;
+    const uint32_t d = d0 + 4u * static_cast<uint32_t>(r * Q::kPitch + 4 * c);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(g), "r"(ok ? 16 : 0) : "memory");
+  }
+}
+
+// Two consecutive values of a staged 16-bit or fp32 row as fp32.
+template <int DT>
+__device__ __forceinline__ float2 unpack_pair(uint32_t w) {
+  if constexpr (DT == KVQ_BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  else return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+// fp16 norm of the lane's own staged row and the scale a = sqrt(128)/norm (0 for a zero norm).
 template <int DT>
 __device__ __forceinline__ void row_norm_scale(const uint32_t* row, __half& n16, float& a) {
   float s2 = 0.0f;
-#pragma unroll 16
-  for (int i = 0; i < kD / 2; ++i) {
-    const float2 v = QuantRow<DT>::pair(row, i);
-    s2 = __fadd_rn(s2, __fmul_rn(v.x, v.x));
-    s2 = __fadd_rn(s2, __fmul_rn(v.y, v.y));
+#pragma unroll 4
+  for (int c = 0; c < QTile<DT>::kPieces; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(row + 4 * c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    if constexpr (DT == KVQ_F32) {
+#pragma unroll
+      for (int i = 0; i < 4; i += 2) {
+        const float2 x = make_float2(__uint_as_float(w[i]), __uint_as_float(w[i + 1]));
+        const float2 q = mul2(x, x);
+        s2 = __fadd_rn(s2, q.x);
+        s2 = __fadd_rn(s2, q.y);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = unpack_pair<DT>(w[i]);
+        const float2 q = mul2(x, x);
+        s2 = __fadd_rn(s2, q.x);
+        s2 = __fadd_rn(s2, q.y);
+      }
+    }
   }
   n16 = __float2half_rn(__fsqrt_rn(s2));
   const float nf = __half2float(n16);
@@ -117,85 +182,95 @@ __device__ __forceinline__ void row_norm_scale(const uint32_t* row, __half& n16,
   a = (nf == 0.0f) ? 0.0f : __fdiv_rn(sqd, nf);
 }
 
-// Code of y for a width-W codebook: binary search, most significant bit first. The top
-// level compares with the middle threshold, which is exactly 0 for these symmetric
-// codebooks. Widths up to 3 select the next threshold from registers (t[] holds the
-// 2^W - 1 thresholds); wider ones index the shared-memory table `thr`.
-template <int W>
-__device__ __forceinline__ uint32_t search_code(float y, const float* __restrict__ thr, const float* t) {
-  const bool hi = y > 0.0f;
-  if constexpr (W == 1) {
-    return hi ? 1u : 0u;
-  } else if constexpr (W == 2) {
-    const bool lo = y > (hi ? t[2] : t[0]);
-    return (hi ? 2u : 0u) | (lo ? 1u : 0u);
-  } else if constexpr (W == 3) {
-    const bool m = y > (hi ? t[5] : t[1]);
-    const float u = hi ? (m ? t[6] : t[4]) : (m ? t[2] : t[0]);
-    return (hi ? 4u : 0u) | (m ? 2u : 0u) | (y > u ? 1u : 0u);
-  } else {
-    int idx = hi ? (1 << (W - 1)) : 0;
-#pragma unroll
-    for (int p = W - 2; p >= 0; --p) {
-      const int s = 1 << p;
-      idx += (y > thr[idx + s - 1]) ? s : 0;
-    }
-    return static_cast<uint32_t>(idx);
-  }
-}
+// ---------------------------------------------------------------- K codes
 
-// Thresholds of width W from the shared table (all widths concatenated, width w at 2^w - w - 1).
-__device__ __forceinline__ const float* width_thresholds(const float* sThr, int w) { return sThr + ((1 << w) - w - 1); }
+// Per-warp table of the current head's blocks in stream order (plus 4 padding entries that
+// a partial group may read): {byte selector that moves the block's half of its word into
+// place | byte offset of that word in a staged row << 16, g}.
+struct KEntry {
+  uint32_t selofs;
+  float g;
+};
+constexpr int kKEntries = kH + 4;
 
 // Bit stream writer for one lane's K codes; `fill` and `word` advance identically in every
-// lane, so every flush is a full-warp store of one word-planar row (word i of 32 tokens).
+// lane, so every flushed word is a full-warp store of one word-planar row.
 struct KStream {
   uint32_t cur = 0;
   int fill = 0;
   int word = 0;
-  template <int W>
-  __device__ __forceinline__ void put(uint32_t code, uint32_t* __restrict__ kout, int lane) {
-    cur |= code << fill;
-    fill += W;
-    if (fill >= 32) {
-      kout[word * kTile + lane] = cur;
+  bool store = true;      // false: this lane's token is not written (it precedes an append)
+  // Appends the low `nbits` (1..32) bits of `buf` (higher bits zero).
+  __device__ __forceinline__ void append(uint32_t buf, int nbits, uint32_t* __restrict__ kout, int lane) {
+    const uint64_t sh = static_cast<uint64_t>(buf) << fill;
+    cur |= static_cast<uint32_t>(sh);
+    const int nf = fill + nbits;
+    if (nf >= 32) {
+      if (store) kout[word * kTile + lane] = cur;
       ++word;
-      fill -= 32;
-      cur = fill ? (code >> (W - fill)) : 0u;
+      cur = static_cast<uint32_t>(sh >> 32);
+      fill = nf - 32;
+    } else {
+      fill = nf;
     }
   }
 };
 
-// All blocks of one width class: for each block b (stream order), the codes of dims b and
-// b + 64. tb[b] = {gain bits of block b}; sb = the class's blocks.
-template <int DT, int W>
-__device__ __forceinline__ void quant_k_class(const uint32_t* myrow, float a, const float* __restrict__ gains,
-                                              const uint8_t* __restrict__ sb, int nb, const float* __restrict__ sThr,
-                                              KStream& ks, uint32_t* __restrict__ kout, int lane) {
-  const float* thr = width_thresholds(sThr, W);
-  float t[7];
-#pragma unroll
-  for (int i = 0; i < 7; ++i) t[i] = (W <= 3 && i < (1 << W) - 1) ? thr[i] : 0.0f;
-  for (int k = 0; k < nb; ++k) {
-    const int b = sb[k];
-    const float g = gains[b];
-    const float y1 = __fmul_rn(__fmul_rn(QuantRow<DT>::value(myrow, b), a), g);
-    const float y2 = __fmul_rn(__fmul_rn(QuantRow<DT>::value(myrow, b + kH), a), g);
-    ks.template put<W>(search_code<W>(y1, thr, t), kout, lane);
-    ks.template put<W>(search_code<W>(y2, thr, t), kout, lane);
+// Values of dims b and b + 64 of block `e` from the lane's staged row.
+// (The byte permute reads only the low 16 bits of its selector.)
+template <int DT>
+__device__ __forceinline__ float2 block_pair(const uint8_t* row, const KEntry& e) {
+  const uint8_t* p = row + (e.selofs >> 16);
+  if constexpr (DT == KVQ_F32) {
+    return make_float2(*reinterpret_cast<const float*>(p), *reinterpret_cast<const float*>(p + 256));
+  } else if constexpr (DT == KVQ_BF16) {
+    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(p);
+    const uint32_t w2 = *reinterpret_cast<const uint32_t*>(p + 128);
+    return make_float2(__uint_as_float(__byte_perm(w1, 0u, e.selofs)), __uint_as_float(__byte_perm(w2, 0u, e.selofs)));
+  } else {
+    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(p);
+    const uint32_t w2 = *reinterpret_cast<const uint32_t*>(p + 128);
+    const uint32_t h2 = __byte_perm(w1, w2, e.selofs);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h2));
   }
 }
 
-// Values: width BV for every dim. Lane l handles dims {2l, 2l+1} and {64+2l, 65+2l}; sA[t]
-// is token t's scale (NaN past the sequence length). Word i of dim j goes to vout[128 i + j].
+// All blocks of one width class (entries first .. first + nb - 1).
+template <int DT, int W>
+__device__ __forceinline__ void quant_k_class(const uint8_t* row, float2 aa, const KEntry* __restrict__ ent, int nb,
+                                              const uint2* __restrict__ lut, KStream& ks, uint32_t* __restrict__ kout,
+                                              int lane) {
+  constexpr int GB = (W <= 4) ? 4 : 2;                          // blocks per group: 2 W GB <= 32 bits
+  for (int k = 0; k < nb; k += GB) {
+    uint32_t buf = 0;
+#pragma unroll
+    for (int j = 0; j < GB; ++j) {
+      const KEntry e = ent[k + j];
+      const float2 x = block_pair<DT>(row, e);
+      const float2 y = mul2(mul2(x, aa), make_float2(e.g, e.g));
+      buf += lut_code<W>(y.x, lut) << (2 * W * j);          // disjoint bit fields: + is |
+      buf += lut_code<W>(y.y, lut) << (2 * W * j + W);
+    }
+    const int left = nb - k;
+    int nbits = 2 * W * GB;
+    if (left < GB) {
+      nbits = 2 * W * left;
+      buf &= (1u << nbits) - 1u;
+    }
+    ks.append(buf, nbits, kout, lane);
+  }
+}
+
+// ---------------------------------------------------------------- V codes
+
+// Width BV for every dim. Lane l handles dims {2l, 2l+1} and {64+2l, 65+2l}; sA2[t] = {a, a}
+// of token t (NaN for tokens not written). Word i of dim j goes to vout[128 i + j]. The first
+// `keep_bits` bits of every dim stream (tokens that precede an append) keep their stored value.
 template <int DT, int BV>
-__device__ __forceinline__ void quant_v_tile(const uint32_t* rows, const float* sA, const float* __restrict__ sThr,
-                                             uint32_t* __restrict__ vout, int lane) {
-  const float* thr = width_thresholds(sThr, BV);
-  float t[7];
-#pragma unroll
-  for (int i = 0; i < 7; ++i) t[i] = (BV <= 3 && i < (1 << BV) - 1) ? thr[i] : 0.0f;
-#pragma unroll
+__device__ __forceinline__ void quant_v_tile(const uint32_t* rows, const float2* sA2, const uint2* __restrict__ lut,
+                                             uint32_t* __restrict__ vout, int keep_bits, int lane) {
+  using Q = QTile<DT>;
+#pragma unroll 1
   for (int half = 0; half < 2; ++half) {
     const int j0 = 2 * lane + kH * half;
     uint32_t w0[BV], w1[BV];
@@ -203,16 +278,30 @@ __device__ __forceinline__ void quant_v_tile(const uint32_t* rows, const float* 
     for (int i = 0; i < BV; ++i) { w0[i] = 0u; w1[i] = 0u; }
 #pragma unroll
     for (int tok = 0; tok < kTile; ++tok) {
-      const float2 x = QuantRow<DT>::pair(rows + tok * QuantRow<DT>::kPitch, j0 >> 1);
-      const float at = sA[tok];
-      const uint32_t c0 = search_code<BV>(__fmul_rn(x.x, at), thr, t);
-      const uint32_t c1 = search_code<BV>(__fmul_rn(x.y, at), thr, t);
+      float2 x;
+      if constexpr (DT == KVQ_F32) x = *reinterpret_cast<const float2*>(rows + tok * Q::kPitch + j0);
+      else x = unpack_pair<DT>(rows[tok * Q::kPitch + (j0 >> 1)]);
+      const float2 y = mul2(x, sA2[tok]);
+      const uint32_t c0 = lut_code<BV>(y.x, lut);
+      const uint32_t c1 = lut_code<BV>(y.y, lut);
       const int bit = BV * tok, wi = bit >> 5, sh = bit & 31;
-      w0[wi] |= c0 << sh;
-      w1[wi] |= c1 << sh;
+      w0[wi] += c0 << sh;                                   // disjoint bit fields: + is |
+      w1[wi] += c1 << sh;
       if (sh + BV > 32) {
-        w0[wi + 1] |= c0 >> (32 - sh);
-        w1[wi + 1] |= c1 >> (32 - sh);
+        w0[wi + 1] += c0 >> (32 - sh);
+        w1[wi + 1] += c1 >> (32 - sh);
+      }
+    }
+    if (keep_bits > 0) {
+#pragma unroll
+      for (int i = 0; i < BV; ++i) {
+        const int kb = keep_bits - 32 * i;
+        if (kb > 0) {
+          const uint32_t m = kb >= 32 ? ~0u : (1u << kb) - 1u;
+          const uint2 old = *reinterpret_cast<const uint2*>(vout + i * kD + j0);
+          w0[i] |= old.x & m;
+          w1[i] |= old.y & m;
+        }
       }
     }
 #pragma unroll
@@ -221,41 +310,92 @@ __device__ __forceinline__ void quant_v_tile(const uint32_t* rows, const float* 
   }
 }
 
+// ---------------------------------------------------------------- kernel
+
+// Per-warp shared memory: K tile, V tile, 32 {a, a} pairs, the K entry table, 8 classes.
+template <int DT> struct QWarpSmem {
+  static constexpr int kBytes = 2 * 4 * QTile<DT>::kWords + kTile * 8 + kKEntries * 8 + 8 * 4;
+};
+
 template <int DT>
-__global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
+__global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
     const typename Elem<DT>::T* __restrict__ K, int64_t ksb, int64_t ksh, int64_t kst,
     const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst,
-    int seq_len, int n_kv_heads, int tiles_written, int tiles_cap, const kvq_head_alloc* __restrict__ alloc,
-    int bits_k, int bits_v, uint8_t* __restrict__ packed, int rec_bytes, long long n_tasks) {
-  using Row = QuantRow<DT>;
-  extern __shared__ __align__(16) uint32_t smem[];
-  float* sThr = reinterpret_cast<float*>(smem);
-  for (int i = threadIdx.x; i < kThresholdCount; i += blockDim.x) sThr[i] = c_tab.threshold[i];
+    int t_begin, int t_end, int tile_lo, int n_tiles, int n_kv_heads, int tiles_cap,
+    const kvq_head_alloc* __restrict__ alloc, int bits_k, int bits_v, uint8_t* __restrict__ packed, int rec_bytes,
+    int n_tasks) {
+  using Q = QTile<DT>;
+  constexpr int kWarps = Q::kWarps;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint2* sLut = reinterpret_cast<uint2*>(smem);
+  for (int i = threadIdx.x; i < kLutEntries; i += blockDim.x)
+    sLut[i] = make_uint2(g_quant_lut[2 * i], g_quant_lut[2 * i + 1]);
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k_words = bits_k * kD;
-  uint32_t* wbase = smem + 512 + warp * (Row::kWords + kQuantExtraWords);
-  uint32_t* rows = wbase;
-  float* sA = reinterpret_cast<float*>(wbase + Row::kWords);             // 32 value scales
-  float* sGain = sA + kTile;                                              // 64 block gains
-  uint8_t* sBlk = reinterpret_cast<uint8_t*>(sGain + kH);                 // 64 blocks, stream order
-  const uint32_t* myrow = rows + lane * Row::kPitch;
-  uint32_t* sCls = reinterpret_cast<uint32_t*>(sBlk + kH);              // 8 classes: width | first << 8 | blocks << 16
+  uint8_t* wbase = smem + kLutEntries * 8 + warp * QWarpSmem<DT>::kBytes;
+  uint32_t* kbuf = reinterpret_cast<uint32_t*>(wbase);
+  uint32_t* vbuf = kbuf + Q::kWords;
+  float2* sA2 = reinterpret_cast<float2*>(vbuf + Q::kWords);
+  KEntry* sEnt = reinterpret_cast<KEntry*>(sA2 + kTile);
+  uint32_t* sCls = reinterpret_cast<uint32_t*>(sEnt + kKEntries);     // width | first << 8 | blocks << 16
+  const uint32_t* myk = kbuf + lane * Q::kPitch;
+  const uint32_t* myv = vbuf + lane * Q::kPitch;
   int cur_h = -1, n_cls = 0;
 
-  for (long long task = static_cast<long long>(blockIdx.x) * kQuantWarps + warp; task < n_tasks;
-       task += static_cast<long long>(gridDim.x) * kQuantWarps) {
-    const int tile = static_cast<int>(task % tiles_written);
-    const int bh = static_cast<int>(task / tiles_written);
+  const int stride = gridDim.x * kWarps;
+  int task = blockIdx.x * kWarps + warp;
+
+  // A task's tile, the tile rows it writes [r_lo, r_hi) and the input rows of r_lo. Input row
+  // i holds token t_begin + i.
+  auto task_src = [&](int tk, int& bh, int& tile, int& r_lo, int& r_hi, const typename Elem<DT>::T*& kp,
+                      const typename Elem<DT>::T*& vp) {
+    bh = tk / n_tiles;
+    tile = tile_lo + (tk - bh * n_tiles);
     const int h = bh % n_kv_heads, b = bh / n_kv_heads;
-    const kvq_head_alloc* al = alloc + h;
-    if (al->k_words != k_words) continue;      // allocation made for another budget: write nothing
+    const int t0 = tile * kTile;
+    r_lo = max(0, t_begin - t0);
+    r_hi = min(kTile, t_end - t0);
+    const int64_t i0 = static_cast<int64_t>(t0 + r_lo - t_begin);
+    kp = K + b * ksb + h * ksh + i0 * kst;
+    vp = V + b * vsb + h * vsh + i0 * vst;
+  };
+
+  // The current task's coordinates; each iteration computes the next task's.
+  int bh = 0, tile = 0, r_lo = 0, r_hi = 0;
+  bool write = false;
+  if (task < n_tasks) {
+    const typename Elem<DT>::T *kp, *vp;
+    task_src(task, bh, tile, r_lo, r_hi, kp, vp);
+    tile_load_async<DT>(kbuf, kp, kst, r_lo, r_hi, lane);
+    cp_async_commit();
+    tile_load_async<DT>(vbuf, vp, vst, r_lo, r_hi, lane);
+    cp_async_commit();
+  }
+
+  for (; task < n_tasks; task += stride) {
+    const int h = bh % n_kv_heads;
+    const bool mine = lane >= r_lo;               // token written by this call (or past its end)
+    const bool valid = mine && lane < r_hi;       // token quantized by this call
+    const int next = task + stride;
+    int nbh = 0, ntile = 0, nlo = 0, nhi = 0;
+    const typename Elem<DT>::T *nkp = nullptr, *nvp = nullptr;
+    if (next < n_tasks) task_src(next, nbh, ntile, nlo, nhi, nkp, nvp);
+
     if (h != cur_h) {
-      __syncwarp();
-      for (int i = lane; i < kH; i += 32) {
-        sGain[i] = al->gain[i];
-        sBlk[i] = al->stream_block[i];
+      const kvq_head_alloc* al = alloc + h;
+      write = al->k_words == k_words;             // allocation made for another budget: write nothing
+      for (int i = lane; i < kKEntries; i += 32) {
+        const int blk = (i < kH) ? al->stream_block[i] : 0xff;
+        KEntry e{0x1044u, 0.0f};
+        if (blk < kH) {
+          const float g = al->gain[blk];
+          if constexpr (DT == KVQ_F32) e = KEntry{(4u * blk) << 16, g};
+          else if constexpr (DT == KVQ_BF16) e = KEntry{((4u * (blk >> 1)) << 16) | ((blk & 1) ? 0x3244u : 0x1044u), g};
+          else e = KEntry{((4u * (blk >> 1)) << 16) | ((blk & 1) ? 0x7632u : 0x5410u), g};
+        }
+        sEnt[i] = e;
       }
       n_cls = min(max(al->n_classes, 0), 8);
       if (lane < 8)
@@ -264,66 +404,81 @@ __global__ void __launch_bounds__(kQuantWarps * 32) kvq_quant_pack(
       __syncwarp();
       cur_h = h;
     }
-    const int t0 = tile * kTile;
-    const int valid_rows = min(kTile, seq_len - t0);
-    const bool valid = lane < valid_rows;
     uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
     uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
     uint16_t* norms = reinterpret_cast<uint16_t*>(kout + k_words);   // 32 K norms, then 32 V norms
     uint32_t* vout = kout + k_words + kTile;
 
     // ---------------------------------------------------------------- K (Block-GTQ widths)
+    cp_async_wait<1>();                          // this task's K rows (its V rows may be in flight)
     __syncwarp();
-    Row::load(rows, K + b * ksb + h * ksh + static_cast<int64_t>(t0) * kst, kst, valid_rows, lane);
-    __syncwarp();
-    __half n16;
-    float a;
-    row_norm_scale<DT>(myrow, n16, a);
-    norms[lane] = valid ? __half_as_ushort(n16) : 0;
-    if (!valid) a = __int_as_float(0x7fc00000);   // NaN: every comparison false, so all codes are 0
-    KStream ks;
-    for (int c = 0; c < n_cls; ++c) {
-      const uint32_t e = sCls[c];
-      const int w = e & 0xffu, first = (e >> 8) & 0xffu, nb = e >> 16;
-      const uint8_t* sb = sBlk + first;
-      switch (w) {
-        case 1: quant_k_class<DT, 1>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
-        case 2: quant_k_class<DT, 2>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
-        case 3: quant_k_class<DT, 3>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
-        case 4: quant_k_class<DT, 4>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
-        case 5: quant_k_class<DT, 5>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
-        case 6: quant_k_class<DT, 6>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
-        case 7: quant_k_class<DT, 7>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
-        default: quant_k_class<DT, 8>(myrow, a, sGain, sb, nb, sThr, ks, kout, lane); break;
+    if (write) {
+      __half n16;
+      float a;
+      row_norm_scale<DT>(myk, n16, a);
+      if (mine) norms[lane] = valid ? __half_as_ushort(n16) : 0;
+      if (!valid) a = __int_as_float(0x7fc00000);   // NaN: every code is 0
+      const float2 aa = make_float2(a, a);
+      const uint8_t* row = reinterpret_cast<const uint8_t*>(myk);
+      KStream ks;
+      ks.store = mine;
+      for (int c = 0; c < n_cls; ++c) {
+        const uint32_t e = sCls[c];
+        const int w = e & 0xffu, first = (e >> 8) & 0xffu, nb = e >> 16;
+        const KEntry* ent = sEnt + first;
+        switch (w) {
+          case 1: quant_k_class<DT, 1>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+          case 2: quant_k_class<DT, 2>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+          case 3: quant_k_class<DT, 3>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+          case 4: quant_k_class<DT, 4>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+          case 5: quant_k_class<DT, 5>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+          case 6: quant_k_class<DT, 6>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+          case 7: quant_k_class<DT, 7>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+          default: quant_k_class<DT, 8>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+        }
       }
     }
+    __syncwarp();                               // every lane is done with the K tile
+    if (nkp) tile_load_async<DT>(kbuf, nkp, kst, nlo, nhi, lane);
+    cp_async_commit();
 
     // ---------------------------------------------------------------- V (uniform width)
+    cp_async_wait<1>();                          // this task's V rows (next K rows may be in flight)
     __syncwarp();
-    Row::load(rows, V + b * vsb + h * vsh + static_cast<int64_t>(t0) * vst, vst, valid_rows, lane);
-    __syncwarp();
-    row_norm_scale<DT>(myrow, n16, a);
-    norms[kTile + lane] = valid ? __half_as_ushort(n16) : 0;
-    sA[lane] = valid ? a : __int_as_float(0x7fc00000);
-    __syncwarp();
-    switch (bits_v) {
-      case 1: quant_v_tile<DT, 1>(rows, sA, sThr, vout, lane); break;
-      case 2: quant_v_tile<DT, 2>(rows, sA, sThr, vout, lane); break;
-      case 3: quant_v_tile<DT, 3>(rows, sA, sThr, vout, lane); break;
-      case 4: quant_v_tile<DT, 4>(rows, sA, sThr, vout, lane); break;
-      case 5: quant_v_tile<DT, 5>(rows, sA, sThr, vout, lane); break;
-      case 6: quant_v_tile<DT, 6>(rows, sA, sThr, vout, lane); break;
-      case 7: quant_v_tile<DT, 7>(rows, sA, sThr, vout, lane); break;
-      default: quant_v_tile<DT, 8>(rows, sA, sThr, vout, lane); break;
+    if (write) {
+      __half n16;
+      float a;
+      row_norm_scale<DT>(myv, n16, a);
+      if (mine) norms[kTile + lane] = valid ? __half_as_ushort(n16) : 0;
+      if (!valid) a = __int_as_float(0x7fc00000);
+      sA2[lane] = make_float2(a, a);
+      const int keep = bits_v * r_lo;
+      __syncwarp();
+      switch (bits_v) {
+        case 1: quant_v_tile<DT, 1>(vbuf, sA2, sLut, vout, keep, lane); break;
+        case 2: quant_v_tile<DT, 2>(vbuf, sA2, sLut, vout, keep, lane); break;
+        case 3: quant_v_tile<DT, 3>(vbuf, sA2, sLut, vout, keep, lane); break;
+        case 4: quant_v_tile<DT, 4>(vbuf, sA2, sLut, vout, keep, lane); break;
+        case 5: quant_v_tile<DT, 5>(vbuf, sA2, sLut, vout, keep, lane); break;
+        case 6: quant_v_tile<DT, 6>(vbuf, sA2, sLut, vout, keep, lane); break;
+        case 7: quant_v_tile<DT, 7>(vbuf, sA2, sLut, vout, keep, lane); break;
+        default: quant_v_tile<DT, 8>(vbuf, sA2, sLut, vout, keep, lane); break;
+      }
     }
+    __syncwarp();                               // every lane is done with the V tile and sA2
+    if (nvp) tile_load_async<DT>(vbuf, nvp, vst, nlo, nhi, lane);
+    cp_async_commit();
+    bh = nbh; tile = ntile; r_lo = nlo; r_hi = nhi;
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// Dynamic shared memory of kvq_quant_pack: thresholds + per warp the row tile, 32 value
-// scales, 64 gains, 64 stream-order block indices and the 8-entry class table.
+// Dynamic shared memory of kvq_quant_pack: the code lookup table, then per warp the K and V
+// tiles, the value scales, the K entry table and the class table.
 inline size_t quant_smem_bytes(int dtype) {
-  const int row_words = (dtype == KVQ_F32) ? QuantRow<KVQ_F32>::kWords : QuantRow<KVQ_BF16>::kWords;
-  return 4 * (512 + static_cast<size_t>(kQuantWarps) * (row_words + kQuantExtraWords));
+  if (dtype == KVQ_F32) return kLutEntries * 8 + static_cast<size_t>(QTile<KVQ_F32>::kWarps) * QWarpSmem<KVQ_F32>::kBytes;
+  return kLutEntries * 8 + static_cast<size_t>(QTile<KVQ_BF16>::kWarps) * QWarpSmem<KVQ_BF16>::kBytes;
 }
+inline int quant_warps(int dtype) { return dtype == KVQ_F32 ? QTile<KVQ_F32>::kWarps : QTile<KVQ_BF16>::kWarps; }
 
 }  // namespace kvq

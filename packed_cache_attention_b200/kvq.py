@@ -80,6 +80,7 @@ _SIGNATURES = {
     "kvq_workspace_status": ([_VP, _VP, ctypes.POINTER(_I)], _I),
     "kvq_calibrate": ([_VP, _P4, ctypes.POINTER(CalibParams), _VP, _VP, _SZ, _VP], _I),
     "kvq_quantize": ([_VP, _P4, _VP, _P4, _VP, _PC, _VP, _VP], _I),
+    "kvq_append": ([_VP, _P4, _VP, _P4, _VP, _PC, _I, _VP, _VP], _I),
     "kvq_decode_attn": ([_VP, _P4, _VP, _VP, _PC, _I, _VP, _VP, _SZ, _VP], _I),
     "kvq_nf4_packed_bytes": ([_I, _I, _I, _I], _SZ),
     "kvq_nf4_decode_workspace_bytes": ([_I, _I, _I, _I], _SZ),
@@ -265,6 +266,15 @@ def kvq_quantize(K, V, alloc, cache: CacheDesc, packed=None, stream=None):
     _check("kvq_quantize", lib().kvq_quantize(K.data_ptr(), ctypes.byref(kd), V.data_ptr(), ctypes.byref(vd),
                                               alloc.data_ptr(), ctypes.byref(cache), packed.data_ptr(),
                                               _stream(stream)))
+    return packed
+
+
+def kvq_append(K, V, alloc, cache: CacheDesc, t_begin: int, packed, stream=None):
+    """Quantize K, V [B][Hkv][n][128] as tokens t_begin .. t_begin + n - 1 of `packed`."""
+    kd, vd = tensor4(K), tensor4(V)
+    _check("kvq_append", lib().kvq_append(K.data_ptr(), ctypes.byref(kd), V.data_ptr(), ctypes.byref(vd),
+                                          alloc.data_ptr(), ctypes.byref(cache), int(t_begin), packed.data_ptr(),
+                                          _stream(stream)))
     return packed
 
 

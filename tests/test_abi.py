@@ -132,6 +132,18 @@ def test_quantize_and_decode_reject_bad_arguments(L):
     assert L.kvq_workspace_init(None, 0, None) == 6
 
 
+def test_append_rejects_ranges_outside_the_cache(L):
+    """Append checks its token range against the capacity before anything is launched."""
+    app = lambda kd_, c_, t0: L.kvq_append(FAKE, ctypes.byref(kd_), FAKE, ctypes.byref(kd_), FAKE, ctypes.byref(c_),
+                                           t0, FAKE, None)
+    c = kvq.cache_desc(1, 2, 64, 3, 3)
+    assert app(_t4(T=1), c, -1) == 5                                      # negative first token
+    assert app(_t4(T=1), c, 64) == 5                                      # first token at capacity
+    assert app(_t4(T=10), c, 60) == 5                                     # range runs past capacity
+    assert app(_t4(T=1, H=3), c, 0) == 2                                  # head count mismatch
+    assert app(_t4(T=1), kvq.cache_desc(1, 2, 64, 0, 3), 0) == 1          # bad cache descriptor
+
+
 def test_binding_raises_on_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(kvq, "_lib", None)
     monkeypatch.setattr(kvq, "LIB_PATH", str(tmp_path / "libkvq.so"))

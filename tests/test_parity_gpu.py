@@ -117,6 +117,41 @@ def test_repeated_decode_reuses_workspace(dev):
     assert kvq.kvq_workspace_status(ws) == 0
 
 
+APPEND_CASES = [("bf16", 3, 3), ("f16", 5, 7), ("f32", 2, 4)]
+
+
+@pytest.mark.parametrize("case", APPEND_CASES, ids=lambda c: f"{c[0]}K{c[1]}V{c[2]}")
+def test_append_in_pieces_equals_one_quantize(dev, case):
+    """The cache only grows ([NQKV] assumptions), so appending a sequence piece by piece
+    (single tokens on both sides of tile boundaries, ragged chunks) must store the same bytes
+    as one quantize call, whatever the buffer held before; decode over the grown cache then
+    matches the oracle at every prefix length reached."""
+    import torch
+    dtype, bk, bv = case
+    T = 200
+    x = wl.make_blockgtq_inputs(2, 8, 2, 128, T, dtype, 1e6, "lognormal_outliers", seed=5 + bk, device=dev)
+    K, V, q = x["K"], x["V"], x["q"]
+    alloc = kvq.kvq_calibrate(K, bk)
+    cache = kvq.cache_desc(2, 2, 256, bk, bv)
+    one = kvq.kvq_quantize(K, V, alloc, cache)
+    grown = torch.full_like(one, 0xAB)
+    cuts = [0, 1, 2, 31, 32, 33, 64, 100, 101, 150, 199, 200]
+    ref_alloc = bg.calibrate(host_f32(K), bk)
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        kvq.kvq_append(K[:, :, a:b], V[:, :, a:b], alloc, cache, a, grown)
+        if b in (33, 101, 200):
+            out = kvq.kvq_decode_attn(q, grown, alloc, cache, b).cpu().numpy()
+            ref_packed = bg.pack_cache(bg.quantize(host_f32(K[:, :, :b]), host_f32(V[:, :, :b]), ref_alloc, bv),
+                                       ref_alloc, bv, b)
+            ref = bg.decode(host_f32(q), ref_packed, ref_alloc, bv, b)
+            assert rel_err(out, ref) <= TOL, b
+    torch.cuda.synchronize()
+    nt = tiles_written(T)
+    g = packed_view(grown.cpu().numpy(), 2, 2, 256, bk, bv)[:, :, :nt]
+    o = packed_view(one.cpu().numpy(), 2, 2, 256, bk, bv)[:, :, :nt]
+    np.testing.assert_array_equal(g, o)
+
+
 # ----------------------------------------------------------------------------- full-size workloads
 
 def _sample_tiles(n_tiles, k=6, seed=0):
