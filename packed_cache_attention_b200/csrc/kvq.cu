@@ -328,15 +328,29 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Persistent grid: exactly the CTAs that are resident at once (registers and shared memory
   // both limit it), so every warp starts at launch and the tiles are spread evenly.
+  // The shared-memory opt-in and the occupancy query are made once per device and dtype (they
+  // cost host time comparable to a small launch, e.g. a one-token append).
+  static std::mutex occ_mu;
+  static int occ[kMaxDevices][3] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
 #define KVQ_LAUNCH_QUANT(DT, TY)                                                                                  \
   do {                                                                                                            \
     auto kern = kvq_quant_pack<DT>;                                                                               \
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=        \
-        cudaSuccess)                                                                                              \
-      return KVQ_ERR_CUDA;                                                                                        \
     int per_sm = 0;                                                                                               \
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, qw * 32, smem) != cudaSuccess)              \
-      return KVQ_ERR_CUDA;                                                                                        \
+    {                                                                                                             \
+      std::lock_guard<std::mutex> lock(occ_mu);                                                                   \
+      if (occ[dev][DT] == 0) {                                                                                    \
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=    \
+            cudaSuccess)                                                                                          \
+          return KVQ_ERR_CUDA;                                                                                    \
+        int n = 0;                                                                                                \
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, qw * 32, smem) != cudaSuccess)                \
+          return KVQ_ERR_CUDA;                                                                                    \
+        occ[dev][DT] = std::max(1, n);                                                                            \
+      }                                                                                                           \
+      per_sm = occ[dev][DT];                                                                                      \
+    }                                                                                                             \
     const long long want = (n_tasks + qw - 1) / qw;                                                             \
     const unsigned grid =                                                                                         \
         static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sm_count()) * std::max(1, per_sm))); \
