@@ -26,7 +26,13 @@ template <> __device__ __forceinline__ float4 ldg_stream<float4>(const void* p) 
 }
 
 constexpr int kCalibSegment = 64;      // chunk sums per fixed-order segment sum
-constexpr int kCalibChunksPerCta = 8;  // 16 lanes per chunk, 128 threads
+#ifndef KVQ_CALIB_CHUNKS_PER_CTA
+#define KVQ_CALIB_CHUNKS_PER_CTA 4
+#endif
+// 16 lanes per chunk; 4 chunks (64 threads) per CTA give about 7 resident CTAs on every SM at
+// 128K tokens, so the single wave is evenly loaded. It must divide kCalibSegment.
+constexpr int kCalibChunksPerCta = KVQ_CALIB_CHUNKS_PER_CTA;
+static_assert(64 % kCalibChunksPerCta == 0, "a CTA's chunks lie in one segment");
 
 // Calibration workspace after the status header: per KV head a head counter and one counter
 // per segment (unsigned, zero between calls), then energies E[h][64], segment sums
@@ -39,7 +45,7 @@ struct CalibWs {
   double* chunk_sum;      // [H][n_chunks][64]
 };
 
-// Grid (ceil(n_chunks / 8), n_kv_heads), 128 threads: 16 lanes per 64-token chunk. Lane k
+// Grid (ceil(n_chunks / kCalibChunksPerCta), n_kv_heads), 16 lanes per 64-token chunk. Lane k
 // (0..15) of a chunk owns blocks 4k..4k+3, i.e. dims 4k..4k+3 and 64+4k..67+4k, read as two
 // 4-element vectors per token (128 contiguous bytes per half-warp for 16-bit inputs). Within
 // the chunk the pooled tokens u = s*n_calib + t are summed left to right in fp64, each term
@@ -48,7 +54,7 @@ struct CalibWs {
 // sums left to right; the CTA that completes the last segment of a head sums the segment
 // sums left to right and writes E_b = total / N. Counters are reset to zero for the next call.
 template <int DT>
-__global__ void __launch_bounds__(16 * kCalibChunksPerCta, 4) kvq_calib_reduce(
+__global__ void __launch_bounds__(16 * kCalibChunksPerCta, 32 / kCalibChunksPerCta) kvq_calib_reduce(
     const typename Elem<DT>::T* __restrict__ K, int n_calib, int64_t sb, int64_t sh, int64_t st, int N,
     int n_chunks, CalibWs ws) {
   using T = typename Elem<DT>::T;

@@ -142,17 +142,21 @@ __global__ void __launch_bounds__(kNf4DecWarps * 32) kvq_nf4_decode(
     if (t < seq_len) {
       const size_t row = L.row(b, blk, t);
       const uint4* kr = reinterpret_cast<const uint4*>(kc + row * 128 + half_off);
-      float accd = 0.0f;
+      // four partial sums (dims 8k'..8k'+7 of each 32-dim quarter go to sum k') keep the
+      // dependent chain short; they are added at the end.
+      uint4 w4[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) w4[v] = __ldg(kr + v);
+      float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const uint4 w4 = __ldg(kr + v);
-        const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+        const uint32_t ws[4] = {w4[v].x, w4[v].y, w4[v].z, w4[v].w};
 #pragma unroll
         for (int k = 0; k < 4; ++k)
 #pragma unroll
-          for (int n = 0; n < 8; ++n) accd = fmaf(sQ[32 * v + 8 * k + n], sLut[(ws[k] >> (4 * n)) & 15u], accd);
+          for (int n = 0; n < 8; ++n) acc4[k] = fmaf(sQ[32 * v + 8 * k + n], sLut[(ws[k] >> (4 * n)) & 15u], acc4[k]);
       }
-      logit = accd * __half2float(ks[row]);
+      logit = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) * __half2float(ks[row]);
     }
     float gmax = logit;
 #pragma unroll
@@ -168,13 +172,20 @@ __global__ void __launch_bounds__(kNf4DecWarps * 32) kvq_nf4_decode(
 #pragma unroll
     for (int k = 0; k < 4; ++k) o[k] *= alpha;
     const float pv = (t < seq_len) ? p * __half2float(vs[L.row(b, blk, min(t, seq_len - 1))]) : 0.0f;
+    // The group's 32 value-code pairs of this lane's dims are all loaded before any is used
+    // (one memory round trip per group); tokens past seq_len re-read the last token and get
+    // weight 0.
+    uint32_t two[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int ti = min(grp * 32 + i, seq_len - 1);
+      two[i] = __ldg(reinterpret_cast<const uint16_t*>(vc + L.row(b, blk, ti) * 128 + half_off + 2 * lane));
+    }
+#pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float pi = __shfl_sync(0xffffffffu, pv, i);
-      const int ti = grp * 32 + i;
-      if (ti >= seq_len) break;
-      const uint16_t two = *reinterpret_cast<const uint16_t*>(vc + L.row(b, blk, ti) * 128 + half_off + 2 * lane);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) o[k] = fmaf(pi, sLut[(two >> (4 * k)) & 15u], o[k]);
+      for (int k = 0; k < 4; ++k) o[k] = fmaf(pi, sLut[(two[i] >> (4 * k)) & 15u], o[k]);
     }
   }
   if (lane == 0) {

@@ -152,6 +152,27 @@ def test_append_in_pieces_equals_one_quantize(dev, case):
     np.testing.assert_array_equal(g, o)
 
 
+def test_append_full_size_matches_one_quantize(dev):
+    """At the 128K Qwen2.5-3B shape, in the calls the benchmark times (a 4096-token chunk and
+    a single token appended at the end of a cache that already holds the rest), the grown
+    cache is byte-identical to one quantize call over the whole sequence."""
+    import torch
+    W = wl.WORKLOADS["qwen3b"]
+    x = wl.make_blockgtq_inputs(W.batch, W.n_q_heads, W.n_kv_heads, W.head_dim, W.seq_len, W.dtype, W.rope_base,
+                                W.key_profile, seed=3, device=dev, with_q=False)
+    K, V, T = x["K"], x["V"], W.seq_len
+    alloc = kvq.kvq_calibrate(K, W.bits_k)
+    cache = kvq.cache_desc(W.batch, W.n_kv_heads, T, W.bits_k, W.bits_v)
+    one = kvq.kvq_quantize(K, V, alloc, cache)
+    grown = torch.full_like(one, 0x5A)
+    a = T - 4096 - 1
+    kvq.kvq_append(K[:, :, :a], V[:, :, :a], alloc, cache, 0, grown)
+    kvq.kvq_append(K[:, :, a:T - 1], V[:, :, a:T - 1], alloc, cache, a, grown)
+    kvq.kvq_append(K[:, :, T - 1:], V[:, :, T - 1:], alloc, cache, T - 1, grown)
+    torch.cuda.synchronize()
+    assert torch.equal(grown, one)
+
+
 # ----------------------------------------------------------------------------- full-size workloads
 
 def _sample_tiles(n_tiles, k=6, seed=0):
