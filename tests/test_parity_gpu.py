@@ -152,6 +152,32 @@ def test_append_in_pieces_equals_one_quantize(dev, case):
     np.testing.assert_array_equal(g, o)
 
 
+def test_append_edges_match_oracle(dev):
+    """Appends at the cache's edges: the first token into a buffer of garbage, a run that ends
+    exactly at the capacity, and a one-token append into a tile whose other 31 tokens are
+    stored; each stored tile equals the oracle's, and decode over 1 and over all tokens
+    matches the oracle."""
+    import torch
+    T = 96
+    x = wl.make_blockgtq_inputs(1, 8, 2, 128, T, "bf16", 1e6, "lognormal_outliers", seed=21, device=dev)
+    K, V, q = x["K"], x["V"], x["q"]
+    alloc = kvq.kvq_calibrate(K, 3)
+    cache = kvq.cache_desc(1, 2, T, 3, 3)
+    grown = torch.full((kvq.kvq_packed_bytes(cache),), 0xC3, dtype=torch.uint8, device=dev)
+    ref_alloc = bg.calibrate(host_f32(K), 3)
+    kvq.kvq_append(K[:, :, :1], V[:, :, :1], alloc, cache, 0, grown)
+    out1 = kvq.kvq_decode_attn(q, grown, alloc, cache, 1).cpu().numpy()
+    ref1 = bg.pack_cache(bg.quantize(host_f32(K[:, :, :1]), host_f32(V[:, :, :1]), ref_alloc, 3), ref_alloc, 3, 1)
+    assert rel_err(out1, bg.decode(host_f32(q), ref1, ref_alloc, 3, 1)) <= TOL
+    kvq.kvq_append(K[:, :, 1:63], V[:, :, 1:63], alloc, cache, 1, grown)
+    kvq.kvq_append(K[:, :, 64:], V[:, :, 64:], alloc, cache, 64, grown)     # ends at the capacity
+    kvq.kvq_append(K[:, :, 63:64], V[:, :, 63:64], alloc, cache, 63, grown)  # last hole of tile 1
+    ref = bg.pack_cache(bg.quantize(host_f32(K), host_f32(V), ref_alloc, 3), ref_alloc, 3, T)
+    np.testing.assert_array_equal(packed_view(grown.cpu().numpy(), 1, 2, T, 3, 3), ref)
+    out = kvq.kvq_decode_attn(q, grown, alloc, cache, T).cpu().numpy()
+    assert rel_err(out, bg.decode(host_f32(q), ref, ref_alloc, 3, T)) <= TOL
+
+
 def test_append_full_size_matches_one_quantize(dev):
     """At the 128K Qwen2.5-3B shape, in the calls the benchmark times (a 4096-token chunk and
     a single token appended at the end of a cache that already holds the rest), the grown
