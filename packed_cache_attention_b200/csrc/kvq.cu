@@ -79,6 +79,13 @@ int n_tiles_of(int tokens) { return (tokens + kTile - 1) / kTile; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// NF4 decode: about 8 waves of two 16-warp CTAs per SM, so the hardware's CTA scheduling
+// evens out the last wave, and at least one 32-token group per warp in every CTA.
+int nf4_splits(int bh, int n_groups) {
+  const int want = (16 * kTargetCtas + bh - 1) / bh;
+  return std::max(1, std::min(std::min(want, n_groups / kNf4DecWarps), kMaxMergeSplits));
+}
+
 int decode_splits(int bh, int n_tiles) {
   const int want = (kTargetCtas + bh - 1) / bh;
   return std::max(1, std::min(std::min(want, n_tiles), kMaxMergeSplits));
@@ -435,7 +442,7 @@ size_t kvq_nf4_packed_bytes(int batch, int n_heads, int capacity, int head_dim) 
 size_t kvq_nf4_decode_workspace_bytes(int batch, int n_heads, int capacity, int head_dim) {
   if (batch < 1 || n_heads < 1 || capacity < 1 || head_dim != kD) return 0;
   const int bh = batch * n_heads;
-  return decode_ws_layout(bh, decode_splits(bh, (capacity + 31) / 32), 1, 0).total;
+  return decode_ws_layout(bh, nf4_splits(bh, (capacity + 31) / 32), 1, 0).total;
 }
 
 kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, int capacity,
@@ -481,7 +488,7 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
   if (qd->seq_len != 1 || (qd->n_heads & 1)) return KVQ_ERR_SHAPE;
   if (seq_len < 1 || seq_len > capacity) return KVQ_ERR_RANGE;
   const int bh = qd->batch * qd->n_heads;
-  const int splits = decode_splits(bh, (seq_len + 31) / 32);
+  const int splits = nf4_splits(bh, (seq_len + 31) / 32);
   const DecodeWs Lw = decode_ws_layout(bh, splits, 1, 0);
   if (!ws || ws_bytes < Lw.total || !aligned16(ws) ||
       ws_bytes < kvq_nf4_decode_workspace_bytes(qd->batch, qd->n_heads, capacity, kD))
