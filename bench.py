@@ -32,6 +32,25 @@ LAYERS = 36
 WORKLOAD = "qwen3b"
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings (ms) over all ranks of the default process
+    group (the slowest rank sets the job's time); the values unchanged on a single rank."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world, layers, batch, seq_len, ms_per_step):
+    """Whole-job layer-tokens/s: every rank processes its own replica of the workload (the
+    (sequence, KV head) units are independent), so the units of all ranks count, over the
+    slowest rank's time."""
+    return world * layers * batch * seq_len / (ms_per_step * 1e-3)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -191,10 +210,7 @@ def run_gpu(args, rank, world, local_rank):
     cal_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     qnt_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
     dec_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
-    if dist:
-        t = torch.tensor([total_ms, cal_ms, qnt_ms, dec_ms], dtype=torch.float64, device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms, cal_ms, qnt_ms, dec_ms = t.tolist()
+    total_ms, cal_ms, qnt_ms, dec_ms = max_over_ranks([total_ms, cal_ms, qnt_ms, dec_ms], dev)
 
     # ---------------------------------------------------------------- end to end through the C ABI
     e2e = None
@@ -225,11 +241,8 @@ def run_gpu(args, rank, world, local_rank):
         z.record(stream)
         barrier()
         e2e_ms = a.elapsed_time(z) / args.e2e_steps
-        if dist:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-            e2e_ms = t.item()
-        e2e = {"value": world * L * B * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e_ms = max_over_ranks([e2e_ms], dev)[0]
+        e2e = {"value": job_throughput(world, L, B, T, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     nf4 = (measure_nf4(kvq, wl, dev, stream, hbm_peak=peaks()[0], batch=args.nf4_batch)
@@ -251,7 +264,7 @@ def run_gpu(args, rank, world, local_rank):
     c_gbs = c_bytes / (c_launch_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC,
-        "value": tokens / (ms_step * 1e-3),
+        "value": job_throughput(world, L, B, T, ms_step),
         "unit": UNIT,
         "n_gpus": world,
         "steps": steps,
