@@ -335,28 +335,28 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Persistent grid: exactly the CTAs that are resident at once (registers and shared memory
   // both limit it), so every warp starts at launch and the tiles are spread evenly.
-  // The shared-memory opt-in and the occupancy query are made once per device and dtype (they
-  // cost host time comparable to a small launch, e.g. a one-token append).
+  // The shared-memory opt-in and the occupancy query are made once per device, dtype and value
+  // width (they cost host time comparable to a small launch, e.g. a one-token append).
   static std::mutex occ_mu;
-  static int occ[kMaxDevices][3] = {};
+  static int occ[kMaxDevices][24] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
-#define KVQ_LAUNCH_QUANT(DT, TY)                                                                                  \
+#define KVQ_LAUNCH_QUANT(DT, TY, BV)                                                                              \
   do {                                                                                                            \
-    auto kern = kvq_quant_pack<DT>;                                                                               \
+    auto kern = kvq_quant_pack<DT, BV>;                                                                           \
     int per_sm = 0;                                                                                               \
     {                                                                                                             \
       std::lock_guard<std::mutex> lock(occ_mu);                                                                   \
-      if (occ[dev][DT] == 0) {                                                                                    \
+      if (occ[dev][DT * 8 + BV - 1] == 0) {                                                                       \
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=    \
             cudaSuccess)                                                                                          \
           return KVQ_ERR_CUDA;                                                                                    \
         int n = 0;                                                                                                \
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, qw * 32, smem) != cudaSuccess)                \
           return KVQ_ERR_CUDA;                                                                                    \
-        occ[dev][DT] = std::max(1, n);                                                                            \
+        occ[dev][DT * 8 + BV - 1] = std::max(1, n);                                                               \
       }                                                                                                           \
-      per_sm = occ[dev][DT];                                                                                      \
+      per_sm = occ[dev][DT * 8 + BV - 1];                                                                         \
     }                                                                                                             \
     const long long want = (n_tasks + qw - 1) / qw;                                                             \
     const unsigned grid =                                                                                         \
@@ -367,11 +367,23 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
                                      static_cast<const kvq_head_alloc*>(alloc), c->bits_k, c->bits_v,             \
                                      static_cast<uint8_t*>(packed), rec, static_cast<int>(n_tasks));              \
   } while (0)
-  switch (kd->dtype) {
-    case KVQ_F32: KVQ_LAUNCH_QUANT(KVQ_F32, float); break;
-    case KVQ_F16: KVQ_LAUNCH_QUANT(KVQ_F16, __half); break;
-    default: KVQ_LAUNCH_QUANT(KVQ_BF16, __nv_bfloat16); break;
+#define KVQ_QUANT_BV(DT, TY)                                                                                      \
+  switch (c->bits_v) {                                                                                            \
+    case 1: KVQ_LAUNCH_QUANT(DT, TY, 1); break;                                                                   \
+    case 2: KVQ_LAUNCH_QUANT(DT, TY, 2); break;                                                                   \
+    case 3: KVQ_LAUNCH_QUANT(DT, TY, 3); break;                                                                   \
+    case 4: KVQ_LAUNCH_QUANT(DT, TY, 4); break;                                                                   \
+    case 5: KVQ_LAUNCH_QUANT(DT, TY, 5); break;                                                                   \
+    case 6: KVQ_LAUNCH_QUANT(DT, TY, 6); break;                                                                   \
+    case 7: KVQ_LAUNCH_QUANT(DT, TY, 7); break;                                                                   \
+    default: KVQ_LAUNCH_QUANT(DT, TY, 8); break;                                                                  \
   }
+  switch (kd->dtype) {
+    case KVQ_F32: KVQ_QUANT_BV(KVQ_F32, float); break;
+    case KVQ_F16: KVQ_QUANT_BV(KVQ_F16, __half); break;
+    default: KVQ_QUANT_BV(KVQ_BF16, __nv_bfloat16); break;
+  }
+#undef KVQ_QUANT_BV
 #undef KVQ_LAUNCH_QUANT
   return launch_status();
 }

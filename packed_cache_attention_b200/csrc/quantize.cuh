@@ -317,7 +317,9 @@ template <int DT> struct QWarpSmem {
   static constexpr int kBytes = 2 * 4 * QTile<DT>::kWords + kTile * 8 + kKEntries * 8 + 8 * 4;
 };
 
-template <int DT>
+// One instantiation per value width BVT (= bits_v), so registers are allocated for one value
+// pass only.
+template <int DT, int BVT>
 __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
     const typename Elem<DT>::T* __restrict__ K, int64_t ksb, int64_t ksh, int64_t kst,
     const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst,
@@ -454,16 +456,7 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
       sA2[lane] = make_float2(a, a);
       const int keep = bits_v * r_lo;
       __syncwarp();
-      switch (bits_v) {
-        case 1: quant_v_tile<DT, 1>(vbuf, sA2, sLut, vout, keep, lane); break;
-        case 2: quant_v_tile<DT, 2>(vbuf, sA2, sLut, vout, keep, lane); break;
-        case 3: quant_v_tile<DT, 3>(vbuf, sA2, sLut, vout, keep, lane); break;
-        case 4: quant_v_tile<DT, 4>(vbuf, sA2, sLut, vout, keep, lane); break;
-        case 5: quant_v_tile<DT, 5>(vbuf, sA2, sLut, vout, keep, lane); break;
-        case 6: quant_v_tile<DT, 6>(vbuf, sA2, sLut, vout, keep, lane); break;
-        case 7: quant_v_tile<DT, 7>(vbuf, sA2, sLut, vout, keep, lane); break;
-        default: quant_v_tile<DT, 8>(vbuf, sA2, sLut, vout, keep, lane); break;
-      }
+      quant_v_tile<DT, BVT>(vbuf, sA2, sLut, vout, keep, lane);
     }
     __syncwarp();                               // every lane is done with the V tile and sA2
     if (nvp) tile_load_async<DT>(vbuf, nvp, vst, nlo, nhi, lane);
