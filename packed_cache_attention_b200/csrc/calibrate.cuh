@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
   __shared__ int sWidth[kH];
   __shared__ int sCount[9];
   __shared__ int sClsX0[9];
+  __shared__ int8_t sGrpCls[kH];   // class of each decode-plan group (at most 64 groups)
   __shared__ double sSum;
   __shared__ __align__(16) kvq_head_alloc sRec;
   const int h = blockIdx.x, tid = threadIdx.x;
@@ -221,9 +222,13 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     // sort after every valid one.
     // Compare-exchange distances of 32 and more go through shared memory, shorter ones
     // between the lanes of a warp (thread tid holds entry tid in registers there).
-    long long key = sKey[tid];
-    int idx = sIdx[tid];
-    for (int k = 2; k <= kH * 8; k <<= 1) {
+    // A block's 8 entries are already in order (its gains do not increase with w, and equal
+    // keys are ordered by entry), so the network starts at runs of 16: runs of 8 must be in
+    // order where (position & 8) == 0 and reversed elsewhere, so odd blocks are read reversed.
+    const int src = (tid & 8) ? (tid ^ 7) : tid;
+    long long key = sKey[src];
+    int idx = sIdx[src];
+    for (int k = 16; k <= kH * 8; k <<= 1) {
       for (int j = k >> 1; j > 0; j >>= 1) {
         if (j >= 32) {
           sKey[tid] = key;
@@ -329,27 +334,30 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     while (sClsX0[c + 1] <= x) ++c;
     const int w = al->class_width[c], nb = al->class_blocks[c], first = al->class_first[c];
     const int k = x - sClsX0[c], g = x & 3, col = 24 * g + 4 * (x >> 2);
+    sGrpCls[x] = static_cast<int8_t>(c);
     al->plan_group[g][x >> 2] = static_cast<uint32_t>(al->class_bit[c] + 8 * w * k) | (static_cast<uint32_t>(col) << 16);
     for (int i = 0; i < 4 && 4 * k + i < nb; ++i)
       al->plan_col_block[col + i] = static_cast<int8_t>(al->stream_block[first + 4 * k + i]);
   }
+  __syncthreads();
   // Runs: a warp group's consecutive entries of one class; flagged when the run holds its
   // class's last group and that group has 1 or 2 pairs. One thread per warp group.
   if (tid >= 128 && tid < 132) {
     const int g = tid - 128;
     int nr = 0, prev = -1;
+    uint32_t run = 0u;                          // the run being built
     for (int x = g; x < n_groups; x += 4) {
-      int c = 0;
-      while (sClsX0[c + 1] <= x) ++c;
-      const int w = al->class_width[c], nb = al->class_blocks[c];
+      const int c = sGrpCls[x];
       if (c != prev) {
-        al->plan_run[g][nr++] = static_cast<uint32_t>(w) | (static_cast<uint32_t>(x >> 2) << 8);
+        if (prev >= 0) al->plan_run[g][nr++] = run;
+        run = static_cast<uint32_t>(al->class_width[c]) | (static_cast<uint32_t>(x >> 2) << 8);
         prev = c;
       }
-      al->plan_run[g][nr - 1] += 1u << 16;
-      const int r = nb & 3;
-      if (x == sClsX0[c + 1] - 1 && r != 0 && r <= 2) al->plan_run[g][nr - 1] |= 1u << 24;
+      run += 1u << 16;
+      const int r = al->class_blocks[c] & 3;
+      if (x == sClsX0[c + 1] - 1 && r != 0 && r <= 2) run |= 1u << 24;
     }
+    if (prev >= 0) al->plan_run[g][nr++] = run;
     al->plan_n_runs[g] = nr;
   }
   __syncthreads();
