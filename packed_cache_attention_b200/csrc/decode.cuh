@@ -229,20 +229,6 @@ __device__ __forceinline__ void v_tile(const uint32_t* vw, uint32_t taddr, const
   tc::tmem_st<16>(taddr, v);
 }
 
-__device__ __forceinline__ void v_tile_any(int bv, const uint32_t* vw, uint32_t taddr, const uint8_t* sm,
-                                           uint32_t lane4) {
-  switch (bv) {
-    case 1: v_tile<1>(vw, taddr, sm, lane4); break;
-    case 2: v_tile<2>(vw, taddr, sm, lane4); break;
-    case 3: v_tile<3>(vw, taddr, sm, lane4); break;
-    case 4: v_tile<4>(vw, taddr, sm, lane4); break;
-    case 5: v_tile<5>(vw, taddr, sm, lane4); break;
-    case 6: v_tile<6>(vw, taddr, sm, lane4); break;
-    case 7: v_tile<7>(vw, taddr, sm, lane4); break;
-    default: v_tile<8>(vw, taddr, sm, lane4); break;
-  }
-}
-
 // Order-preserving map of fp32 to int32 (and back: the map is its own inverse).
 __device__ __forceinline__ int ordered(float x) {
   const int i = __float_as_int(x);
@@ -316,7 +302,8 @@ __device__ __forceinline__ void merge_partials(DecHeader& S, uint8_t* scratch, i
 
 // ---------------------------------------------------------------- the kernel
 
-template <int DT>
+// One instantiation per value width BVT (= bits_v).
+template <int DT, int BVT>
 __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
     const typename Elem<DT>::T* __restrict__ q, int64_t qsb, int64_t qsh, int n_q_heads, int n_kv_heads,
     const uint8_t* __restrict__ packed, const kvq_head_alloc* __restrict__ alloc, int tiles_cap, int rec_bytes,
@@ -640,7 +627,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
           const uint8_t* st = stages + s * stage_bytes;
           // V-hat^T row: dim t_lane, tokens of tile wg -> columns 16 wg .. 16 wg + 15.
           const uint32_t* vw = reinterpret_cast<const uint32_t*>(st + wg * tstride + 2 * kTile) + t_lane;
-          v_tile_any(bits_v, vw, tbase + lane_base + col_av(bj) + 16 * wg, sm, lane4);
+          v_tile<BVT>(vw, tbase + lane_base + col_av(bj) + 16 * wg, sm, lane4);
           // P' of token t_lane (tile qt, token lane), rows 2 wg, 2 wg + 1.
           const float vn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + qt * tstride)[lane]));
           const float s0 = stash[(u * 8 + 2 * wg) * kChunkTokens + t_lane];

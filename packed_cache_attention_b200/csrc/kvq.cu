@@ -422,25 +422,37 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
   const size_t smem = decode_smem_bytes(c->bits_k, c->bits_v);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(splits, bh);
-#define KVQ_LAUNCH_DEC(DT, TY)                                                                                        \
+#define KVQ_LAUNCH_DEC(DT, TY, BV)                                                                                    \
   do {                                                                                                                \
-    auto kern = kvq_decode_gtq<DT>;                                                                                   \
+    auto kern = kvq_decode_gtq<DT, BV>;                                                                               \
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=            \
         cudaSuccess)                                                                                                  \
       return KVQ_ERR_CUDA;                                                                                            \
     kern<<<grid, kDecThreads, smem, s>>>(                                                                             \
         static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, c->n_kv_heads,                             \
         static_cast<const uint8_t*>(packed), static_cast<const kvq_head_alloc*>(alloc), n_tiles_of(c->capacity), rec, \
-        c->bits_k, c->bits_v, seq_len, splits, merge_groups(splits), decode_stages(c->bits_k, c->bits_v), out,                         \
+        c->bits_k, c->bits_v, seq_len, splits, merge_groups(splits), decode_stages(c->bits_k, c->bits_v), out,       \
         reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_l),                            \
         reinterpret_cast<float*>(w8 + L.part_o), reinterpret_cast<unsigned*>(w8 + L.tickets),                        \
         reinterpret_cast<unsigned*>(w8));                                                                             \
   } while (0)
-  switch (qd->dtype) {
-    case KVQ_F32: KVQ_LAUNCH_DEC(KVQ_F32, float); break;
-    case KVQ_F16: KVQ_LAUNCH_DEC(KVQ_F16, __half); break;
-    default: KVQ_LAUNCH_DEC(KVQ_BF16, __nv_bfloat16); break;
+#define KVQ_DEC_BV(DT, TY)                                                                                            \
+  switch (c->bits_v) {                                                                                                \
+    case 1: KVQ_LAUNCH_DEC(DT, TY, 1); break;                                                                         \
+    case 2: KVQ_LAUNCH_DEC(DT, TY, 2); break;                                                                         \
+    case 3: KVQ_LAUNCH_DEC(DT, TY, 3); break;                                                                         \
+    case 4: KVQ_LAUNCH_DEC(DT, TY, 4); break;                                                                         \
+    case 5: KVQ_LAUNCH_DEC(DT, TY, 5); break;                                                                         \
+    case 6: KVQ_LAUNCH_DEC(DT, TY, 6); break;                                                                         \
+    case 7: KVQ_LAUNCH_DEC(DT, TY, 7); break;                                                                         \
+    default: KVQ_LAUNCH_DEC(DT, TY, 8); break;                                                                        \
   }
+  switch (qd->dtype) {
+    case KVQ_F32: KVQ_DEC_BV(KVQ_F32, float); break;
+    case KVQ_F16: KVQ_DEC_BV(KVQ_F16, __half); break;
+    default: KVQ_DEC_BV(KVQ_BF16, __nv_bfloat16); break;
+  }
+#undef KVQ_DEC_BV
 #undef KVQ_LAUNCH_DEC
   return launch_status();
 }
