@@ -252,6 +252,16 @@ size_t kvq_nf4_decode_workspace_bytes(int batch, int n_heads, int capacity, int 
 kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd,
                             int capacity, void* packed, void* stream);
 
+/* NF4 append ([NQKV] assumptions: the cache only grows, so a new token's blocks are encoded
+ * without re-quantizing stored ones; Fig. 6, decoding phase). Quantizes tokens t_begin ..
+ * t_begin + n - 1 (n = kd->seq_len; input row i is token t_begin + i) exactly as
+ * kvq_nf4_quantize does, writes padding rows (code 0, scale 0) from t_begin + n up to the next
+ * multiple of 16, and leaves every other row untouched. Requires 0 <= t_begin and
+ * t_begin + n <= capacity (else KVQ_ERR_RANGE). Rows below the next multiple of 16 after the
+ * last token then hold the same bytes as one kvq_nf4_quantize call over all tokens. */
+kvq_status kvq_nf4_append(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd,
+                          int capacity, int t_begin, void* packed, void* stream);
+
 /* NF4 MHA decode attention ([NQKV]: dequantization is a table lookup; padding zeros are
  * masked): out[b][h] = sum_t softmax_t(q . x_hat / sqrt(d)) v_hat over t < seq_len with
  * x_hat = scale * NF4[idx]. q: [batch][n_heads][1][128]; out fp32 [batch][n_heads][128]. */

@@ -469,8 +469,12 @@ size_t kvq_nf4_decode_workspace_bytes(int batch, int n_heads, int capacity, int 
   return decode_ws_layout(bh, nf4_splits(bh, (capacity + 31) / 32), 1, 0).total;
 }
 
-kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, int capacity,
-                            void* packed, void* stream) {
+namespace {
+
+// NF4 rows t_begin .. t_begin + kd->seq_len - 1 of a cache of `capacity` tokens; padding rows
+// after them are written up to t_stop.
+kvq_status launch_nf4_quant(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd,
+                            int capacity, int t_begin, bool pad_to_capacity, void* packed, void* stream) {
   kvq_status st;
   if ((st = check_tensor(K, kd)) != KVQ_OK) return st;
   if ((st = check_tensor(V, vd)) != KVQ_OK) return st;
@@ -478,30 +482,48 @@ kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V,
   if (vd->dtype != kd->dtype || vd->batch != kd->batch || vd->n_heads != kd->n_heads || vd->seq_len != kd->seq_len)
     return KVQ_ERR_SHAPE;
   if (kd->n_heads & 1) return KVQ_ERR_SHAPE;
-  if (kd->seq_len > capacity) return KVQ_ERR_RANGE;
+  if (t_begin < 0 || static_cast<long long>(t_begin) + kd->seq_len > capacity) return KVQ_ERR_RANGE;
   if ((st = ensure_tables()) != KVQ_OK) return st;
   const Nf4Layout L = nf4_layout(kd->batch, kd->n_heads, capacity);
-  const long long tasks = 2LL * kd->batch * L.nblk * (L.t_pad / kNf4Rows);
+  const int t_end = t_begin + kd->seq_len;
+  const int t_stop = pad_to_capacity ? L.t_pad
+                                     : std::min(L.t_pad, (t_end + KVQ_NF4_PAD - 1) / KVQ_NF4_PAD * KVQ_NF4_PAD);
+  const int groups = (t_stop + kNf4Rows - 1) / kNf4Rows - t_begin / kNf4Rows;
+  const long long tasks = 2LL * kd->batch * L.nblk * groups;
   const unsigned grid = static_cast<unsigned>((tasks + kNf4Warps - 1) / kNf4Warps);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (kd->dtype) {
     case KVQ_F32:
       kvq_nf4_quant_pack<KVQ_F32><<<grid, kNf4Warps * 32, 0, s>>>(
           static_cast<const float*>(K), kd->stride_b, kd->stride_h, kd->stride_t, static_cast<const float*>(V),
-          vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, kd->seq_len, L, static_cast<uint8_t*>(packed));
+          vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, t_begin, t_end, t_stop, L,
+          static_cast<uint8_t*>(packed));
       break;
     case KVQ_F16:
       kvq_nf4_quant_pack<KVQ_F16><<<grid, kNf4Warps * 32, 0, s>>>(
           static_cast<const __half*>(K), kd->stride_b, kd->stride_h, kd->stride_t, static_cast<const __half*>(V),
-          vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, kd->seq_len, L, static_cast<uint8_t*>(packed));
+          vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, t_begin, t_end, t_stop, L,
+          static_cast<uint8_t*>(packed));
       break;
     default:
       kvq_nf4_quant_pack<KVQ_BF16><<<grid, kNf4Warps * 32, 0, s>>>(
           static_cast<const __nv_bfloat16*>(K), kd->stride_b, kd->stride_h, kd->stride_t,
-          static_cast<const __nv_bfloat16*>(V), vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, kd->seq_len, L,
-          static_cast<uint8_t*>(packed));
+          static_cast<const __nv_bfloat16*>(V), vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, t_begin, t_end,
+          t_stop, L, static_cast<uint8_t*>(packed));
   }
   return launch_status();
+}
+
+}  // namespace
+
+kvq_status kvq_nf4_quantize(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, int capacity,
+                            void* packed, void* stream) {
+  return launch_nf4_quant(K, kd, V, vd, capacity, 0, true, packed, stream);
+}
+
+kvq_status kvq_nf4_append(const void* K, const kvq_tensor4* kd, const void* V, const kvq_tensor4* vd, int capacity,
+                          int t_begin, void* packed, void* stream) {
+  return launch_nf4_quant(K, kd, V, vd, capacity, t_begin, false, packed, stream);
 }
 
 kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, int capacity, int seq_len,

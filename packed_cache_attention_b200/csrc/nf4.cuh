@@ -26,26 +26,29 @@ struct Nf4Layout {
 constexpr int kNf4Rows = 4;   // token rows per warp task
 constexpr int kNf4DecWarps = 16;   // warps per CTA of the NF4 decode
 
-// One warp per (K-or-V, sequence, block, group of 4 token rows < T_pad). Lane l holds values
-// 8l..8l+7 of the block: head 2*blk + l/16, dims 8(l%16)..8(l%16)+7. All rows of the group
-// are loaded before any is quantized.
+// One warp per (K-or-V, sequence, block, group of 4 token rows). Lane l holds values 8l..8l+7
+// of the block: head 2*blk + l/16, dims 8(l%16)..8(l%16)+7. All rows of the group are loaded
+// before any is quantized. Rows t_begin .. t_end - 1 are quantized (input row i holds token
+// t_begin + i), rows t_end .. t_stop - 1 are written as padding (code 0, scale 0), and rows
+// outside [t_begin, t_stop) are not touched.
 template <int DT>
 __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
     const typename Elem<DT>::T* __restrict__ K, int64_t ksb, int64_t ksh, int64_t kst,
     const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst, int batch,
-    int seq_len, Nf4Layout L, uint8_t* __restrict__ packed) {
+    int t_begin, int t_end, int t_stop, Nf4Layout L, uint8_t* __restrict__ packed) {
   using T = typename Elem<DT>::T;
   __shared__ float sMid[16];
   if (threadIdx.x < 15) sMid[threadIdx.x] = c_tab.nf4_mid[threadIdx.x];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int groups = L.t_pad / kNf4Rows;
+  const int g_lo = t_begin / kNf4Rows;
+  const int groups = (t_stop + kNf4Rows - 1) / kNf4Rows - g_lo;
   const long long task = static_cast<long long>(blockIdx.x) * kNf4Warps + warp;
   const long long per_kv = static_cast<long long>(batch) * L.nblk * groups;
   if (task >= 2 * per_kv) return;
   const int which = static_cast<int>(task / per_kv);          // 0 = K, 1 = V
   long long r = task % per_kv;
-  const int grp = static_cast<int>(r % groups);
+  const int grp = g_lo + static_cast<int>(r % groups);
   r /= groups;
   const int blk = static_cast<int>(r % L.nblk);
   const int b = static_cast<int>(r / L.nblk);
@@ -59,8 +62,8 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
     const int t = t0 + rr;
 #pragma unroll
     for (int i = 0; i < 8; ++i) x[rr][i] = 0.0f;
-    if (t < seq_len) {
-      const T* src = X + b * sb + head * sh + static_cast<int64_t>(t) * st + d0;
+    if (t >= t_begin && t < t_end) {
+      const T* src = X + b * sb + head * sh + static_cast<int64_t>(t - t_begin) * st + d0;
       if constexpr (DT == KVQ_F32) {
         const float4 a = __ldg(reinterpret_cast<const float4*>(src));
         const float4 c = __ldg(reinterpret_cast<const float4*>(src) + 1);
@@ -80,6 +83,7 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
 #pragma unroll
   for (int rr = 0; rr < kNf4Rows; ++rr) {
     const int t = t0 + rr;
+    if (t < t_begin || t >= t_stop) continue;        // warp-uniform
     const size_t row = L.row(b, blk, t);
     uint32_t* codes = reinterpret_cast<uint32_t*>(packed + which * L.codes_bytes + row * 128);
     __half* scales = reinterpret_cast<__half*>(packed + 2 * L.codes_bytes) + which * (L.codes_bytes / 128) + row;
@@ -88,7 +92,7 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[rr][i]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const __half s16 = __float2half_rn(amax);        // rows past seq_len are all zero: scale 0, codes 0
+    const __half s16 = __float2half_rn(amax);        // padding rows are all zero: scale 0, codes 0
     const float s = __half2float(s16);
     uint32_t word = 0;
 #pragma unroll
@@ -99,9 +103,9 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
       for (int k = 3; k >= 0; --k) idx += (u > sMid[idx + (1 << k) - 1]) ? (1 << k) : 0;
       word |= static_cast<uint32_t>(idx) << (4 * i);
     }
-    if (t >= seq_len) word = 0u;
+    if (t >= t_end) word = 0u;
     codes[lane] = word;
-    if (lane == 0) *scales = (t < seq_len) ? s16 : __ushort_as_half(0);
+    if (lane == 0) *scales = (t < t_end) ? s16 : __ushort_as_half(0);
   }
 }
 

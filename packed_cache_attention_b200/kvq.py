@@ -85,6 +85,7 @@ _SIGNATURES = {
     "kvq_nf4_packed_bytes": ([_I, _I, _I, _I], _SZ),
     "kvq_nf4_decode_workspace_bytes": ([_I, _I, _I, _I], _SZ),
     "kvq_nf4_quantize": ([_VP, _P4, _VP, _P4, _I, _VP, _VP], _I),
+    "kvq_nf4_append": ([_VP, _P4, _VP, _P4, _I, _I, _VP, _VP], _I),
     "kvq_nf4_decode_attn": ([_VP, _P4, _VP, _I, _I, _VP, _VP, _SZ, _VP], _I),
     "kvq_decode_attn_noalloc": ([_VP, _P4, _VP, _VP, _PC, _I, _VP, _VP], _I),
     "kvq_decode_noalloc_scratch_bytes": ([], _SZ),
@@ -319,6 +320,14 @@ def kvq_nf4_quantize(K, V, capacity: int | None = None, packed=None, stream=None
     kd, vd = tensor4(K), tensor4(V)
     _check("kvq_nf4_quantize", lib().kvq_nf4_quantize(K.data_ptr(), ctypes.byref(kd), V.data_ptr(),
                                                       ctypes.byref(vd), cap, packed.data_ptr(), _stream(stream)))
+    return packed
+
+
+def kvq_nf4_append(K, V, capacity: int, t_begin: int, packed, stream=None):
+    """NF4-quantize K, V [B][H][n][128] as tokens t_begin .. t_begin + n - 1 of `packed`."""
+    kd, vd = tensor4(K), tensor4(V)
+    _check("kvq_nf4_append", lib().kvq_nf4_append(K.data_ptr(), ctypes.byref(kd), V.data_ptr(), ctypes.byref(vd),
+                                                  int(capacity), int(t_begin), packed.data_ptr(), _stream(stream)))
     return packed
 
 

@@ -132,6 +132,13 @@ def test_quantize_and_decode_reject_bad_arguments(L):
     assert L.kvq_workspace_init(None, 0, None) == 6
 
 
+def test_nf4_append_rejects_ranges_outside_the_cache(L):
+    app = lambda kd_, cap, t0: L.kvq_nf4_append(FAKE, ctypes.byref(kd_), FAKE, ctypes.byref(kd_), cap, t0, FAKE, None)
+    assert app(_t4(T=1), 64, -1) == 5                                     # negative first token
+    assert app(_t4(T=8), 64, 60) == 5                                     # range runs past capacity
+    assert app(_t4(T=1, H=3), 64, 0) == 2                                 # odd head count
+
+
 def test_append_rejects_ranges_outside_the_cache(L):
     """Append checks its token range against the capacity before anything is launched."""
     app = lambda kd_, c_, t0: L.kvq_append(FAKE, ctypes.byref(kd_), FAKE, ctypes.byref(kd_), FAKE, ctypes.byref(c_),

@@ -266,6 +266,36 @@ def test_nf4_small_cases_match_oracle(dev, case):
     assert rel_err(out, ref) <= TOL
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_nf4_append_in_pieces_equals_one_quantize(dev, dtype):
+    """NF4 append ([NQKV] assumptions: append-only cache; Fig. 6 decoding phase): pieces of one
+    token and ragged runs store the rows below the last padding boundary exactly as one
+    quantize call, whatever the buffer held; decode over the grown cache matches the oracle."""
+    import torch
+    B, H, T, cap = 2, 4, 45, 64
+    x = wl.make_nf4_inputs(B, H, 128, T, dtype, seed=9, device=dev)
+    K, V, q = x["K"], x["V"], x["q"]
+    one = kvq.kvq_nf4_quantize(K, V, capacity=cap)
+    grown = torch.full_like(one, 0x3C)
+    for a, b in zip([0, 1, 2, 15, 16, 17, 33, 44], [1, 2, 15, 16, 17, 33, 44, 45]):
+        kvq.kvq_nf4_append(K[:, :, a:b], V[:, :, a:b], cap, a, grown)
+    torch.cuda.synchronize()
+    kc, vc, ks, vs = kvq.nf4_sections(grown.cpu().numpy(), B, H, cap)
+    ok, ov, oks, ovs = kvq.nf4_sections(one.cpu().numpy(), B, H, cap)
+    rows = -(-T // 16) * 16
+    np.testing.assert_array_equal(kc[:, :, :rows], ok[:, :, :rows])
+    np.testing.assert_array_equal(vc[:, :, :rows], ov[:, :, :rows])
+    np.testing.assert_array_equal(ks[:, :, :rows].view(np.uint16), oks[:, :, :rows].view(np.uint16))
+    np.testing.assert_array_equal(vs[:, :, :rows].view(np.uint16), ovs[:, :, :rows].view(np.uint16))
+    out = kvq.kvq_nf4_decode_attn(q, grown, cap, T).cpu().numpy()
+    ki, ksc = nqkv.quantize(host_f32(K))
+    vi, vsc = nqkv.quantize(host_f32(V))
+    rkc, rks = nqkv.pack(ki, ksc, cap)
+    rvc, rvs = nqkv.pack(vi, vsc, cap)
+    ref = nqkv.decode(host_f32(q), rkc, rks, rvc, rvs, H, 128, T)
+    assert rel_err(out, ref) <= TOL
+
+
 def test_nf4_full_size(dev):
     """OPT-30B shape at full size: whole (sequence, block) rows bit-exact on sampled blocks,
     attention of their heads against the oracle's own quantized cache."""
