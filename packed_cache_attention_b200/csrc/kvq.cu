@@ -494,19 +494,22 @@ kvq_status launch_nf4_quant(const void* K, const kvq_tensor4* kd, const void* V,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (kd->dtype) {
     case KVQ_F32:
-      kvq_nf4_quant_pack<KVQ_F32><<<grid, kNf4Warps * 32, 0, s>>>(
+      (pad_to_capacity ? kvq_nf4_quant_pack<KVQ_F32, false>
+                       : kvq_nf4_quant_pack<KVQ_F32, true>)<<<grid, kNf4Warps * 32, 0, s>>>(
           static_cast<const float*>(K), kd->stride_b, kd->stride_h, kd->stride_t, static_cast<const float*>(V),
           vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, t_begin, t_end, t_stop, L,
           static_cast<uint8_t*>(packed));
       break;
     case KVQ_F16:
-      kvq_nf4_quant_pack<KVQ_F16><<<grid, kNf4Warps * 32, 0, s>>>(
+      (pad_to_capacity ? kvq_nf4_quant_pack<KVQ_F16, false>
+                       : kvq_nf4_quant_pack<KVQ_F16, true>)<<<grid, kNf4Warps * 32, 0, s>>>(
           static_cast<const __half*>(K), kd->stride_b, kd->stride_h, kd->stride_t, static_cast<const __half*>(V),
           vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, t_begin, t_end, t_stop, L,
           static_cast<uint8_t*>(packed));
       break;
     default:
-      kvq_nf4_quant_pack<KVQ_BF16><<<grid, kNf4Warps * 32, 0, s>>>(
+      (pad_to_capacity ? kvq_nf4_quant_pack<KVQ_BF16, false>
+                       : kvq_nf4_quant_pack<KVQ_BF16, true>)<<<grid, kNf4Warps * 32, 0, s>>>(
           static_cast<const __nv_bfloat16*>(K), kd->stride_b, kd->stride_h, kd->stride_t,
           static_cast<const __nv_bfloat16*>(V), vd->stride_b, vd->stride_h, vd->stride_t, kd->batch, t_begin, t_end,
           t_stop, L, static_cast<uint8_t*>(packed));

@@ -30,8 +30,9 @@ constexpr int kNf4DecWarps = 16;   // warps per CTA of the NF4 decode
 // of the block: head 2*blk + l/16, dims 8(l%16)..8(l%16)+7. All rows of the group are loaded
 // before any is quantized. Rows t_begin .. t_end - 1 are quantized (input row i holds token
 // t_begin + i), rows t_end .. t_stop - 1 are written as padding (code 0, scale 0), and rows
-// outside [t_begin, t_stop) are not touched.
-template <int DT>
+// outside [t_begin, t_stop) are not touched. kRange = false (a whole-cache quantize: t_begin
+// = 0, t_stop = T_pad) compiles without the range checks.
+template <int DT, bool kRange>
 __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
     const typename Elem<DT>::T* __restrict__ K, int64_t ksb, int64_t ksh, int64_t kst,
     const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst, int batch,
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
     const int t = t0 + rr;
 #pragma unroll
     for (int i = 0; i < 8; ++i) x[rr][i] = 0.0f;
-    if (t >= t_begin && t < t_end) {
+    if ((!kRange || t >= t_begin) && t < t_end) {
       const T* src = X + b * sb + head * sh + static_cast<int64_t>(t - t_begin) * st + d0;
       if constexpr (DT == KVQ_F32) {
         const float4 a = __ldg(reinterpret_cast<const float4*>(src));
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
 #pragma unroll
   for (int rr = 0; rr < kNf4Rows; ++rr) {
     const int t = t0 + rr;
-    if (t < t_begin || t >= t_stop) continue;        // warp-uniform
+    if (kRange && (t < t_begin || t >= t_stop)) continue;   // warp-uniform
     const size_t row = L.row(b, blk, t);
     uint32_t* codes = reinterpret_cast<uint32_t*>(packed + which * L.codes_bytes + row * 128);
     __half* scales = reinterpret_cast<__half*>(packed + 2 * L.codes_bytes) + which * (L.codes_bytes / 128) + row;
