@@ -20,7 +20,8 @@ The page names these steps without defining them. The readings taken here
   gain       g_b = sqrt(2 sum(E) / (d E_b)) (unit variance per coordinate of
              block b after the global sqrt(d)/||k|| scaling), 1 if E_b = 0;
              f_b = 1 / (sqrt(d) g_b) is the matching dequant factor.
-  quantizer  per token row: fp16 norm of the row (fp32 sum of squares), a = sqrt(d)/norm in fp32,
+  quantizer  per token row: fp16 norm of the row (fp32 sum of squares in a fixed order of
+             eight interleaved partial sums), a = sqrt(d)/norm in fp32,
              y = (x * a) * g_b in fp32, code = #{thresholds strictly below y}
              of the width-w_b Lloyd-Max codebook. Values use width bits_v, g = 1.
   layout     32-token tiles; per token one K bit stream (codes in width-class
@@ -155,11 +156,37 @@ def calibrate(K: np.ndarray, bits_k: int, n_calib: int = 0, w_max: int = 8, mode
 # --------------------------------------------------------------------------- quantizer
 
 def row_norms_f16(X: np.ndarray) -> np.ndarray:
-    """fp16 norm of every row: fp16(fp32 sqrt(s2)), s2 = sum of x_j^2 left to right in fp32,
-    each step fl32(s2 + fl32(x_j * x_j)) (the square is exact for 16-bit inputs)."""
+    """fp16 norm of every row: fp16(fp32 sqrt(s2)), round to nearest even.
+
+    s2 is an fp32 sum of the squares in a fixed order (reading R5; the page fixes neither the
+    precision nor the order of this sum). Eight partial sums s_r, r = 0..7, each run over the
+    coordinates j = r, r + 8, r + 16, ... in ascending j, one step being
+    s_r = fl32(s_r + fl32(x_j * x_j)); they are then combined as
+        s2 = fl32( fl32(fl32(s_0 + s_1) + fl32(s_2 + s_3))
+                 + fl32(fl32(s_4 + s_5) + fl32(s_6 + s_7)) ).
+    (The square is exact for 16-bit inputs.) The eight short chains keep the summation's
+    dependency depth at 16 instead of d.
+    """
     X32 = np.asarray(X, dtype=np.float32)
-    s2 = np.add.accumulate((X32 * X32).astype(np.float32), axis=-1, dtype=np.float32)[..., -1]
+    d = X32.shape[-1]
+    sq = (X32 * X32).astype(np.float32)
+    s = [np.zeros(X32.shape[:-1], dtype=np.float32) for _ in range(8)]
+    for j in range(d):
+        r = j % 8
+        s[r] = (s[r] + sq[..., j]).astype(np.float32)
+    f32 = np.float32
+    lo = ((s[0] + s[1]).astype(f32) + (s[2] + s[3]).astype(f32)).astype(f32)
+    hi = ((s[4] + s[5]).astype(f32) + (s[6] + s[7]).astype(f32)).astype(f32)
+    s2 = (lo + hi).astype(f32)
     return np.sqrt(s2).astype(np.float32).astype(np.float16)
+
+
+def threshold_count(t32: np.ndarray, y: np.ndarray) -> np.ndarray:
+    """code = #{thresholds t with t < y}, counted by comparison: a y on a threshold takes the
+    lower code, and a NaN y (no threshold compares below it) takes code 0."""
+    y = np.asarray(y, dtype=np.float32)
+    t = np.asarray(t32, dtype=np.float32)
+    return np.sum(t < y[..., None], axis=-1).astype(np.uint8)
 
 
 def quantize_rows(X: np.ndarray, widths_dim: np.ndarray, gains_dim: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
@@ -185,8 +212,7 @@ def quantize_rows(X: np.ndarray, widths_dim: np.ndarray, gains_dim: np.ndarray) 
         if not np.any(sel):
             continue
         _, t32 = codebooks.stored_codebook(w)
-        # side="left": the count of thresholds t with t < y, i.e. y > t strictly.
-        codes[..., sel] = np.searchsorted(t32, y[..., sel], side="left").astype(np.uint8)
+        codes[..., sel] = threshold_count(t32, y[..., sel])
     return codes, n16
 
 

@@ -52,7 +52,7 @@ def quantize(X: np.ndarray, block: int = BLOCK) -> tuple[np.ndarray, np.ndarray]
         u = np.where(s32[..., None] == 0, np.float32(0.0),
                      blocks / np.where(s32 == 0, np.float32(1.0), s32)[..., None]).astype(np.float32)
     mids = codebooks.nf4_midpoints()
-    idx = np.searchsorted(mids, u, side="left").astype(np.uint8)      # #{midpoints < u}
+    idx = np.sum(mids < u[..., None], axis=-1).astype(np.uint8)       # #{midpoints < u}
     return np.transpose(idx, (0, 2, 1, 3)), np.transpose(s16, (0, 2, 1))
 
 

@@ -315,6 +315,57 @@ def test_energy_matches_exact_mean():
             assert abs(E[hh, b] - exact) <= 1e-13 * exact
 
 
+def crafted_energy_keys():
+    """bf16-exact keys [1][1][8192][128] whose fp64 energies depend on the summation order.
+
+    8192 pooled tokens = 128 chunks of 64 = 2 segments of 64 chunks. Block b sums
+    x_b^2 + x_{b+64}^2; only blocks 0..3 are non-zero. The large terms are powers of two,
+    so a small term is lost exactly when it is below half an ulp of the running sum, or a tie
+    against an even mantissa.
+    """
+    K = np.zeros((1, 1, 8192, 128), dtype=np.float32)
+    # block 0: 2^53 (x = y = 2^26) at u = 0, then 1 at the first token of chunks 1..127
+    K[0, 0, 0, 0] = K[0, 0, 0, 64] = 2.0 ** 26
+    K[0, 0, 64::64, 0] = 1.0
+    # block 1: 2^54 (x = 2^27) at u = 0; 1 at u = 1..63 (chunk 0) and u = 64..127 (chunk 1)
+    K[0, 0, 0, 1] = 2.0 ** 27
+    K[0, 0, 1:128, 1] = 1.0
+    # block 2: 2^52 (x = 2^26) at u = 63, the last token of chunk 0; 0.25 (x = 0.5) at u = 0..62
+    K[0, 0, 63, 2] = 2.0 ** 26
+    K[0, 0, 0:63, 2] = 0.5
+    # block 3: 2^53 (x = y = 2^26) at u = 4096, the first token of segment 1; 1 at the
+    # first token of every other chunk
+    K[0, 0, 4096, 3] = K[0, 0, 4096, 67] = 2.0 ** 26
+    K[0, 0, 0::64, 3] = 1.0
+    K[0, 0, 4096, 3] = 2.0 ** 26
+    return K
+
+
+def test_energy_summation_order_by_hand():
+    """Reading R2 fixes the fp64 order of the energy sum: 64-token chunks, 64-chunk segments,
+    then the segments, each level left to right. Worked by hand (N = 8192):
+      block 0: chunk 0 = 2^53, chunks 1..127 = 1 each. Segment 0 = 2^53 + 63 ones, each a tie
+        that rounds back to 2^53 (ulp 2); segment 1 = 64 (exact). E = (2^53 + 64) / 8192
+        = 2^40 + 2^-7. (Summing the chunk sums straight, or the tokens, loses all 127 ones:
+        2^40; chunks of 32 or segments of 32 chunks keep 96: 2^40 + 96/8192.)
+      block 1: chunk 0 = 2^54 + 63 ones, each below half an ulp (2) -> 2^54; chunk 1 = 64,
+        added exactly. E = (2^54 + 64) / 8192 = 2^41 + 2^-7. (Chunks of 128 lose the 64.)
+      block 2: inside chunk 0, 63 quarters sum exactly to 15.75 before 2^52 arrives (ulp 1):
+        2^52 + 15.75 rounds to 2^52 + 16. E = (2^52 + 16) / 8192 = 2^39 + 2^-9. (Summing
+        the chunk right to left loses every quarter: 2^39.)
+      block 3: segment 0 = 64 ones = 64; segment 1 = 2^53 + 63 ones lost = 2^53. E =
+        (64 + 2^53) / 8192 = 2^40 + 2^-7. (A sum of the chunk sums left to right gives the
+        same; starting from the large term loses the first segment's 64: 2^40.)
+    """
+    K = crafted_energy_keys()
+    E, N = bg.calibration_energies(K.astype(np.float32), 0)
+    assert N == 8192
+    want = [2.0 ** 40 + 2.0 ** -7, 2.0 ** 41 + 2.0 ** -7, 2.0 ** 39 + 2.0 ** -9, 2.0 ** 40 + 2.0 ** -7]
+    for b, v in enumerate(want):
+        assert E[0, b] == v, (b, E[0, b], v)
+    assert np.all(E[0, 4:] == 0.0)
+
+
 def test_energy_is_rope_invariant():
     rng = np.random.default_rng(12)
     d, T = 32, 300
@@ -355,6 +406,98 @@ def test_quantizer_tie_goes_to_lower_code():
     x[0] = np.nextafter(t32[5], np.float32(10))
     codes, _ = bg.quantize_rows(x[None], np.full(4, 3), np.ones(4, np.float32))
     assert codes[0, 0] == 6
+
+
+def _norm_row(ones_at):
+    """fp32 row of 128: 4098 at coordinate 0, 1.0 at the given coordinates, 0 elsewhere."""
+    x = np.zeros(128, dtype=np.float32)
+    x[0] = 4098.0
+    x[list(ones_at)] = 1.0
+    return x
+
+
+def test_row_norm_summation_order_by_hand():
+    """Reading R5 fixes the fp32 order of the sum of squares: eight partial sums over
+    j = r (mod 8), j ascending, combined ((s0+s1)+(s2+s3))+((s4+s5)+(s6+s7)).
+
+    Worked by hand. 4098^2 = 16793604 is exact in fp32 (ulp 2 in [2^24, 2^25)), and its
+    square root 4098 is the midpoint of the fp16 neighbours 4096 and 4100, so it rounds to
+    4096 (even mantissa); any extra mass that survives gives a root above 4098 and the fp16
+    norm 4100. Adding 1 to an even value v in [2^24, 2^25) is a tie and rounds back to v:
+    a lone 1 added after the large square is lost, while 1s summed among themselves first
+    survive once they reach 2.
+      A: 1s at j = 1..127. s0 absorbs the 15 at j = 8, 16, ..; s1..s7 = 16 each; the tree
+         adds 112 -> 16793716 -> 4100. (A left-to-right sum loses every 1 -> 4096.)
+      B: 1s at j = 4 (mod 8). They all land in s4 = 16 -> 16793620 -> 4100. (Partial sums
+         mod 4 put them in s0 with the large square, where each is lost -> 4096.)
+      C: 1s at j = 0 (mod 8), j > 0. All fall into s0 after the large square: lost -> 4096.
+         (An exact fp64 sum keeps them -> 4100.)
+      D: 1s at j = 2, 3, 6, 7. s2 + s3 = 2 and s6 + s7 = 2; (s0 + s1) + (s2 + s3) = 16793606,
+         plus (s4 + s5) + (s6 + s7) = 2 gives 16793608, whose root 4098.000488 is above the
+         midpoint -> 4100. (Combining s0 .. s7 one after the other loses every 1 -> 4096.)
+    Codes at width 3 (g = 1): the 4098 coordinate lands far above every threshold (code
+    7), the 1s just above the middle threshold 0 (code 4), the zeros on it (code 3).
+    """
+    cases = {"A": (range(1, 128), 4100.0), "B": (range(4, 128, 8), 4100.0),
+             "C": (range(8, 128, 8), 4096.0), "D": ((2, 3, 6, 7), 4100.0)}
+    for name, (ones, want) in cases.items():
+        x = _norm_row(ones)
+        codes, n16 = bg.quantize_rows(x[None], np.full(128, 3), np.ones(128, np.float32))
+        assert float(n16[0]) == want, name
+        expect = np.full(128, 3, dtype=np.uint8)
+        expect[list(ones)] = 4
+        expect[0] = 7
+        np.testing.assert_array_equal(codes[0], expect, err_msg=name)
+
+
+def test_nan_coordinate_takes_code_zero():
+    """code = #{t < y}: no threshold compares below a NaN, so a NaN y takes code 0 (the rule
+    as stated, not a search that sorts NaN last)."""
+    _, t32 = cb.stored_codebook(3)
+    got = bg.threshold_count(t32, np.array([np.nan, -np.inf, np.inf, 0.0], dtype=np.float32))
+    np.testing.assert_array_equal(got, [0, 0, 7, 3])
+
+
+def _textbook_levels():
+    rows = _golden_rows("lloyd_max_centroids_textbook.txt")
+    return {int(r[0]): r[1:] for r in rows}
+
+
+def test_dequantizer_by_hand():
+    """k_hat = norm * c16_w[code] * f_b and v_hat = norm * c16[code] / sqrt(d), value by value.
+
+    d = 8 (blocks b = 0..3 cover dims b and b + 4), widths (2, 3, 0, 1), dequant factors
+    (0.5, 0.25, 1, 2), one token with key norm 2 and codes (3, 5, 1, 0 | 0, 7, 2, 1) on dims
+    0..7. The fp16 centroids used are c2 = (-1.5107421875, -0.452880859375, +.., +..),
+    c3[5] = 0.755859375, c3[7] = 2.15234375, c1 = (-0.7978515625, +0.7978515625): the fp16
+    roundings of the textbook Lloyd-Max levels (checked against them below). So
+      dim 0: 2 * c2[3] * 0.5  = 1.5107421875     dim 4: 2 * c2[0] * 0.5  = -1.5107421875
+      dim 1: 2 * c3[5] * 0.25 = 0.3779296875     dim 5: 2 * c3[7] * 0.25 = 1.076171875
+      dim 2, 6: width 0 -> 0                     dim 3: 2 * c1[0] * 2 = -3.19140625
+      dim 7: 2 * c1[1] * 2 = 3.19140625
+    Values at width 2, norm 4, codes (0, 1, 2, 3, 3, 2, 1, 0) on dims 0..7:
+      v_hat = 4 * c2[code] / sqrt(8).
+    """
+    c1 = [-0.7978515625, 0.7978515625]
+    c2 = [-1.5107421875, -0.452880859375, 0.452880859375, 1.5107421875]
+    c3_5, c3_7 = 0.755859375, 2.15234375
+    tb = _textbook_levels()
+    assert abs(c1[1] - tb[1][0]) < 1e-3
+    assert abs(c2[2] - tb[2][0]) < 1e-3 and abs(c2[3] - tb[2][1]) < 1e-3
+    assert abs(c3_5 - tb[3][1]) < 1e-3 and abs(c3_7 - tb[3][3]) < 1e-3
+    alloc = {"w": np.array([[2, 3, 0, 1]]), "f": np.array([[0.5, 0.25, 1.0, 2.0]], dtype=np.float32)}
+    Kc = np.array([3, 5, 1, 0, 0, 7, 2, 1], dtype=np.uint8).reshape(1, 1, 1, 8)
+    Kn = np.array([2.0], dtype=np.float16).reshape(1, 1, 1)
+    khat = bg.dequantize_keys(Kc, Kn, alloc)[0, 0, 0]
+    want = [1.5107421875, 0.3779296875, 0.0, -3.19140625, -1.5107421875, 1.076171875, 0.0, 3.19140625]
+    np.testing.assert_array_equal(khat, want)
+    Vc = np.array([0, 1, 2, 3, 3, 2, 1, 0], dtype=np.uint8).reshape(1, 1, 1, 8)
+    Vn = np.array([4.0], dtype=np.float16).reshape(1, 1, 1)
+    vhat = bg.dequantize_values(Vc, Vn, 2)[0, 0, 0]
+    s8 = math.sqrt(8.0)
+    want_v = [4 * c2[0] / s8, 4 * c2[1] / s8, 4 * c2[2] / s8, 4 * c2[3] / s8,
+              4 * c2[3] / s8, 4 * c2[2] / s8, 4 * c2[1] / s8, 4 * c2[0] / s8]
+    np.testing.assert_allclose(vhat, want_v, rtol=1e-15, atol=0)
 
 
 def test_append_one_token_at_a_time_equals_batch():
