@@ -221,7 +221,8 @@ def widths_per_dim(w_blocks: np.ndarray) -> np.ndarray:
 
 
 def quantize(K: np.ndarray, V: np.ndarray, alloc: dict, bits_v: int) -> dict:
-    """Codes and fp16 norms for K (Block-GTQ widths and gains) and V (uniform bits_v, g = 1)."""
+    """Codes and fp16 norms for K (Block-GTQ widths and gains) and V (uniform bits_v, g = 1;
+    bits_v = 0: keys only, V is not quantized)."""
     B, H, T, d = K.shape
     Kc = np.zeros((B, H, T, d), dtype=np.uint8)
     Kn = np.zeros((B, H, T), dtype=np.float16)
@@ -229,6 +230,8 @@ def quantize(K: np.ndarray, V: np.ndarray, alloc: dict, bits_v: int) -> dict:
         wd = widths_per_dim(alloc["w"][hh])
         gd = np.concatenate([alloc["g"][hh], alloc["g"][hh]])
         Kc[:, hh], Kn[:, hh] = quantize_rows(K[:, hh], wd, gd)
+    if bits_v == 0:                     # keys only: values stay unquantized outside the cache
+        return {"Kc": Kc, "Kn": Kn, "Vc": None, "Vn": None}
     Vc, Vn = quantize_rows(V, np.full(d, bits_v), np.ones(d, dtype=np.float32))
     return {"Kc": Kc, "Kn": Kn, "Vc": Vc, "Vn": Vn}
 
@@ -244,13 +247,17 @@ def tile_v_words(bits_v: int, d: int) -> int:
 
 
 def tile_record_bytes(d: int, bits_k: int, bits_v: int) -> int:
-    """Bytes of one 32-token tile record: K words, 32 K norms, 32 V norms (fp16), V words."""
+    """Bytes of one 32-token tile record: K words, 32 K norms, 32 V norms (fp16), V words;
+    a keys-only record (bits_v = 0) ends after the K norms."""
+    if bits_v == 0:
+        return 4 * tile_k_words(bits_k, d) + 2 * TILE
     return 4 * tile_k_words(bits_k, d) + 4 * tile_v_words(bits_v, d) + 2 * TILE * 2
 
 
 def packed_bytes(batch: int, n_kv_heads: int, capacity: int, d: int, bits_k: int, bits_v: int) -> int:
+    """Header plus tile records (bits_v = 0: keys only)."""
     n_tiles = -(-capacity // TILE)
-    return batch * n_kv_heads * n_tiles * tile_record_bytes(d, bits_k, bits_v)
+    return header_bytes(n_kv_heads) + batch * n_kv_heads * n_tiles * tile_record_bytes(d, bits_k, bits_v)
 
 
 def k_stream_blocks(w_blocks: np.ndarray) -> list[int]:
@@ -302,6 +309,75 @@ def unpack_bits(words: np.ndarray, widths: list[int]) -> np.ndarray:
     return out
 
 
+# --------------------------------------------------------------------------- packed header
+#
+# Reading (the pages define no interface): every packed cache starts with a header that
+# names its layout and the allocation its K codes were written with, so that a decode given
+# another layer's allocation, or a descriptor with other widths, can refuse instead of
+# returning wrong attention. Little-endian, header_bytes(n_kv_heads) long:
+#   0 u32 magic "KVQ1"     4 u16 layout version    6 u16 head_dim
+#   8 u8 bits_k            9 u8 bits_v (0: keys only)   10 u8 w_max   11 u8 mode
+#  12 u32 status (0; an append that found a mismatch records its kvq_status here)
+#  16 i32 batch           20 i32 n_kv_heads       24 i32 capacity    28 u32 record bytes
+#  32..63 zero            64 u64 digest of each KV head's allocation, head order
+# then zero padding to a multiple of 128 bytes; the tile records follow.
+
+HEADER_MAGIC = 0x3151564B        # bytes "KVQ1"
+LAYOUT_VERSION = 1
+_M64 = (1 << 64) - 1
+
+
+def splitmix64(z: int) -> int:
+    """The SplitMix64 output function (Steele, Lea and Flood, "Fast splittable pseudorandom
+    number generators", OOPSLA 2014; constants as published by Vigna): one 64-bit mix."""
+    z = (z + 0x9E3779B97F4A7C15) & _M64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def alloc_digest(w_blocks, g_blocks) -> int:
+    """64-bit digest of one KV head's allocation: the sum mod 2^64, over blocks b, of
+    splitmix64(b << 40 | w_b << 32 | fp32 bits of g_b). Any change of a width or a gain
+    changes it (up to 64-bit collisions); the sum does not depend on the order it is taken in."""
+    g32 = np.asarray(g_blocks, dtype=np.float32).view(np.uint32)
+    acc = 0
+    for b in range(len(w_blocks)):
+        acc = (acc + splitmix64((b << 40) | (int(w_blocks[b]) << 32) | int(g32[b]))) & _M64
+    return acc
+
+
+def header_bytes(n_kv_heads: int) -> int:
+    return -(-(64 + 8 * n_kv_heads) // 128) * 128
+
+
+def packed_header(batch: int, n_kv_heads: int, capacity: int, d: int, bits_k: int, bits_v: int,
+                  alloc: dict) -> np.ndarray:
+    """Header bytes of a packed cache written with allocation `alloc` (see the layout above)."""
+    out = np.zeros(header_bytes(n_kv_heads), dtype=np.uint8)
+    fields = np.zeros(8, dtype="<u4")
+    fields[0] = HEADER_MAGIC
+    fields[1] = LAYOUT_VERSION | (d << 16)
+    fields[2] = bits_k | (bits_v << 8) | (int(alloc["w_max"]) << 16) | (int(alloc["mode"]) << 24)
+    fields[3] = 0
+    fields[4] = batch
+    fields[5] = n_kv_heads
+    fields[6] = capacity
+    fields[7] = tile_record_bytes(d, bits_k, bits_v)
+    out[:32] = fields.view(np.uint8)
+    dig = np.array([alloc_digest(alloc["w"][h], alloc["g"][h]) for h in range(n_kv_heads)], dtype="<u8")
+    out[64:64 + 8 * n_kv_heads] = dig.view(np.uint8)
+    return out
+
+
+def pack_cache_bytes(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarray:
+    """The whole packed buffer: header, then the tile records of pack_cache, flat."""
+    rec = pack_cache(codes, alloc, bits_v, capacity)
+    B, H = rec.shape[:2]
+    hdr = packed_header(B, H, capacity, int(alloc["d"]), int(alloc["bits_k"]), bits_v, alloc)
+    return np.concatenate([hdr, rec.reshape(-1)])
+
+
 def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarray:
     """Packed cache bytes [B][Hkv][n_tiles][record] for capacity tokens per sequence.
 
@@ -316,7 +392,8 @@ def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarr
         stream (i < bits_v), which is the codes of tokens 0..31 of the tile at dim j,
         concatenated, bits_v bits each, least significant bit first.
     Keys and their norms come first and values with theirs last, so that a reader can fetch
-    either half of a record in one contiguous piece.
+    either half of a record in one contiguous piece. A keys-only record (bits_v = 0) holds the
+    K part and the K norms only.
     Tokens at or beyond the sequence length T are stored with code 0 and norm 0.
     """
     Kc, Kn, Vc, Vn = codes["Kc"], codes["Kn"], codes["Vc"], codes["Vn"]
@@ -333,9 +410,12 @@ def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarr
         out[:, :, :T] = a
         return out
 
-    Kc, Vc, Kn, Vn = padded(Kc), padded(Vc), padded(Kn), padded(Vn)
+    keys_only = bits_v == 0
+    Kc, Kn = padded(Kc), padded(Kn)
     Kc = Kc.reshape(B, H, n_tiles, TILE, d)
-    Vc = Vc.reshape(B, H, n_tiles, TILE, d)
+    if not keys_only:
+        Vc, Vn = padded(Vc), padded(Vn)
+        Vc = Vc.reshape(B, H, n_tiles, TILE, d)
     rec = tile_record_bytes(d, bits_k, bits_v)
     out = np.zeros((B, H, n_tiles, rec), dtype=np.uint8)
     for hh in range(H):
@@ -347,12 +427,13 @@ def pack_cache(codes: dict, alloc: dict, bits_v: int, capacity: int) -> np.ndarr
         if kstream.shape[-1] != tile_k_words(bits_k, d) // TILE:
             raise ValueError("widths do not fill the K budget")
         kwords = np.transpose(kstream, (0, 1, 3, 2)).reshape(B, n_tiles, -1)   # word-planar
-        vstream = pack_bits(np.transpose(Vc[:, hh], (0, 1, 3, 2)), [bits_v] * TILE)   # [B][n_tiles][d][bv]
-        vwords = np.transpose(vstream, (0, 1, 3, 2)).reshape(B, n_tiles, -1)
         parts = [kwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1),
-                 Kn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1),
-                 Vn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1),
-                 vwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1)]
+                 Kn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1)]
+        if not keys_only:
+            vstream = pack_bits(np.transpose(Vc[:, hh], (0, 1, 3, 2)), [bits_v] * TILE)   # [B][n_tiles][d][bv]
+            vwords = np.transpose(vstream, (0, 1, 3, 2)).reshape(B, n_tiles, -1)
+            parts += [Vn[:, hh].reshape(B, n_tiles, TILE).astype("<f2").view(np.uint8).reshape(B, n_tiles, -1),
+                      vwords.astype("<u4").view(np.uint8).reshape(B, n_tiles, -1)]
         out[:, hh] = np.concatenate(parts, axis=-1)
     return out
 
@@ -367,11 +448,12 @@ def unpack_cache(packed: np.ndarray, alloc: dict, bits_v: int, seq_len: int) -> 
     cap = n_tiles * TILE
     Kc = np.zeros((B, H, n_tiles, TILE, d), dtype=np.uint8)
     Vc = np.zeros((B, H, n_tiles, TILE, d), dtype=np.uint8)
+    keys_only = bits_v == 0
     kw = packed[..., :4 * nk].copy().view("<u4")
-    norms = packed[..., 4 * nk:4 * nk + 4 * TILE].copy().view("<f2")
-    vw = packed[..., 4 * nk + 4 * TILE:].copy().view("<u4")
+    norms = packed[..., 4 * nk:4 * nk + (2 if keys_only else 4) * TILE].copy().view("<f2")
+    vw = None if keys_only else packed[..., 4 * nk + 4 * TILE:].copy().view("<u4")
     Kn = norms[..., :TILE].reshape(B, H, cap)
-    Vn = norms[..., TILE:].reshape(B, H, cap)
+    Vn = None if keys_only else norms[..., TILE:].reshape(B, H, cap)
     for hh in range(H):
         w_blocks = alloc["w"][hh]
         order = k_stream_blocks(w_blocks)
@@ -379,9 +461,12 @@ def unpack_cache(packed: np.ndarray, alloc: dict, bits_v: int, seq_len: int) -> 
         widths = [int(w_blocks[b]) for b in order for _ in (0, 1)]
         kstream = np.transpose(kw[:, hh].reshape(B, n_tiles, nk // TILE, TILE), (0, 1, 3, 2))
         Kc[:, hh][..., dims] = unpack_bits(kstream, widths).astype(np.uint8)
-        vstream = np.transpose(vw[:, hh].reshape(B, n_tiles, bits_v, d), (0, 1, 3, 2))   # [B][n][d][bv]
-        Vc[:, hh] = np.transpose(unpack_bits(vstream, [bits_v] * TILE), (0, 1, 3, 2)).astype(np.uint8)
+        if not keys_only:
+            vstream = np.transpose(vw[:, hh].reshape(B, n_tiles, bits_v, d), (0, 1, 3, 2))   # [B][n][d][bv]
+            Vc[:, hh] = np.transpose(unpack_bits(vstream, [bits_v] * TILE), (0, 1, 3, 2)).astype(np.uint8)
     Kc = Kc.reshape(B, H, cap, d)[:, :, :seq_len]
+    if keys_only:
+        return {"Kc": Kc, "Kn": Kn[:, :, :seq_len].astype(np.float16), "Vc": None, "Vn": None}
     Vc = Vc.reshape(B, H, cap, d)[:, :, :seq_len]
     return {"Kc": Kc, "Kn": Kn[:, :, :seq_len].astype(np.float16),
             "Vc": Vc, "Vn": Vn[:, :, :seq_len].astype(np.float16)}
@@ -431,9 +516,29 @@ def decode_attention(q: np.ndarray, Khat: np.ndarray, Vhat: np.ndarray) -> np.nd
     return out
 
 
-def decode(q: np.ndarray, packed: np.ndarray, alloc: dict, bits_v: int, seq_len: int) -> np.ndarray:
-    """Fused-path reference: unpack the stored bits, dequantize, attend (fp64)."""
-    u = unpack_cache(packed, alloc, bits_v, seq_len)
-    Khat = dequantize_keys(u["Kc"], u["Kn"], alloc)
-    Vhat = dequantize_values(u["Vc"], u["Vn"], bits_v)
+def decode(q: np.ndarray, packed: np.ndarray, alloc: dict, bits_v: int, seq_len: int, V=None, K_recent=None,
+           V_recent=None) -> np.ndarray:
+    """Fused-path reference: unpack the stored bits, dequantize, attend (fp64).
+
+    Keys-only cache (bits_v = 0; the Block-GTQ page quotes its key error "K-only"): the
+    values of positions 0..seq_len-1 are the stored values V [B][Hkv][>= seq_len][d], taken
+    exactly. Recent-token buffer (reading: the Block-GTQ page reports its results without an
+    fp16 recent-key buffer, which names the variant; here the R most recent tokens keep
+    their keys and values unquantized): K_recent, V_recent [B][Hkv][R][d] hold positions
+    seq_len .. seq_len + R - 1, attended in the same softmax with their exact values.
+    seq_len may be 0 when R > 0.
+    """
+    parts_k, parts_v = [], []
+    if seq_len > 0:
+        u = unpack_cache(packed, alloc, bits_v, seq_len)
+        parts_k.append(dequantize_keys(u["Kc"], u["Kn"], alloc))
+        if bits_v == 0:
+            parts_v.append(np.asarray(V, dtype=np.float64)[:, :, :seq_len])
+        else:
+            parts_v.append(dequantize_values(u["Vc"], u["Vn"], bits_v))
+    if K_recent is not None and K_recent.shape[2] > 0:
+        parts_k.append(np.asarray(K_recent, dtype=np.float64))
+        parts_v.append(np.asarray(V_recent, dtype=np.float64))
+    Khat = np.concatenate(parts_k, axis=2)
+    Vhat = np.concatenate(parts_v, axis=2)
     return decode_attention(q, Khat, Vhat)

@@ -521,8 +521,12 @@ def test_packed_bytes_per_token():
     assert fp16_bytes / (bg.tile_record_bytes(128, 3, 3) / 32) == 5.12
     assert bg.tile_record_bytes(128, 2, 2) == 32 * 68
     assert bg.tile_record_bytes(128, 4, 4) == 32 * 132
-    assert bg.packed_bytes(1, 2, 131072, 128, 3, 3) == 26_214_400
-    assert bg.packed_bytes(1, 2, 100, 128, 3, 3) == 2 * 4 * 3200         # ragged tail rounds up to tiles
+    # the tile records, plus one 128-byte header (64 bytes of fields, 8 per KV head, rounded up)
+    assert bg.packed_bytes(1, 2, 131072, 128, 3, 3) == 26_214_400 + 128
+    assert bg.packed_bytes(1, 2, 100, 128, 3, 3) == 2 * 4 * 3200 + 128   # ragged tail rounds up to tiles
+    assert bg.header_bytes(8) == 128 and bg.header_bytes(9) == 256
+    # keys only (bits_v = 0): K part and K norms, 48 + 2 bytes per token at K3
+    assert bg.tile_record_bytes(128, 3, 0) == 32 * 50
     # NF4: 128 bytes of codes + one fp16 scale per 256 values
     assert (128 + 2) * 8 / 256 == 4.0625
     assert round(16 / 4.0625, 2) == 3.94
@@ -669,6 +673,96 @@ def test_decode_from_packed_equals_direct_dequant():
     # the dequantised keys approximate the originals (quantizer sanity, not exactness)
     rel = np.linalg.norm(Khat - K) / np.linalg.norm(K)
     assert rel < 0.25
+
+
+# ----------------------------------------------------------------- packed header
+
+def test_splitmix64_published_vectors():
+    """The digest's mixing function against the first outputs of SplitMix64 seeded with 0, as
+    published with the reference generator: mix(gamma), mix(2 gamma), mix(3 gamma)."""
+    g = 0x9E3779B97F4A7C15
+    assert bg.splitmix64(0) == 0xE220A8397B1DCDAF
+    assert bg.splitmix64(g) == 0x6E789E6AA1B965F4
+    assert bg.splitmix64((2 * g) % (1 << 64)) == 0x06C45D188009454F
+
+
+def test_header_fields_by_hand():
+    """Header of a 2-sequence, 3-KV-head, 77-token K3V2 cache: magic "KVQ1", layout 1,
+    d = 128, widths, the record size 4 * 128 * (3 + 2) + 128 = 2688, one digest per head,
+    64 + 3 * 8 = 88 bytes padded to 128."""
+    w = np.array([[3] * 64, [2] * 32 + [4] * 32, [3] * 64])
+    g = np.ones((3, 64), np.float32)
+    g[1, 5] = 1.5
+    alloc = {"w": w, "g": g, "w_max": 8, "mode": 0}
+    h = bg.packed_header(2, 3, 77, 128, 3, 2, alloc)
+    assert h.shape == (128,)
+    assert bytes(h[:4]) == b"KVQ1"
+    assert list(h[4:12]) == [1, 0, 128, 0, 3, 2, 8, 0]
+    assert list(h[12:16]) == [0, 0, 0, 0]
+    f = h[16:32].view("<u4")
+    assert list(f) == [2, 3, 77, 2688]
+    assert not h[32:64].any() and not h[88:].any()
+    dig = h[64:88].view("<u8")
+    assert dig[0] == dig[2] and dig[0] != dig[1]               # same allocation, same digest
+    # digest: sum mod 2^64 over blocks of splitmix64(b << 40 | w << 32 | bits(g)); g = 1.0 is 0x3F800000
+    want0 = sum(bg.splitmix64((b << 40) | (3 << 32) | 0x3F800000) for b in range(64)) % (1 << 64)
+    assert int(dig[0]) == want0
+    g2 = g.copy()
+    g2[1, 5] = np.float32(1.5) + np.float32(2 ** -23)         # one ulp of one gain changes it
+    assert bg.alloc_digest(w[1], g2[1]) != int(dig[1])
+
+
+# ----------------------------------------------------------------- keys-only cache and recent tokens
+
+def _small_cache(seed, T=45, bits_k=3, bits_v=2):
+    rng = np.random.default_rng(seed)
+    K = (rng.standard_normal((1, 2, T, 128)) * np.exp(rng.standard_normal(128))).astype(np.float32)
+    V = rng.standard_normal((1, 2, T, 128)).astype(np.float32)
+    q = rng.standard_normal((1, 4, 128)).astype(np.float32)
+    a = bg.calibrate(K, bits_k)
+    c = bg.quantize(K, V, a, bits_v)
+    return K, V, q, a, c
+
+
+def test_recent_buffer_alone_is_plain_attention():
+    """With no packed token (seq_len 0) and all T tokens in the recent buffer, the decode is
+    exact fp64 attention over the raw keys and values."""
+    K, V, q, a, _ = _small_cache(31)
+    out = bg.decode(q, None, a, 2, 0, K_recent=K, V_recent=V)
+    np.testing.assert_array_equal(out, bg.decode_attention(q, K.astype(np.float64), V.astype(np.float64)))
+
+
+def test_recent_buffer_duplicating_the_cache_changes_nothing():
+    """Appending every cached token again as a recent token (with its dequantized key and
+    value) doubles each softmax weight's numerator and denominator alike: the output equals
+    the packed-only decode (to rounding)."""
+    K, V, q, a, c = _small_cache(32)
+    packed = bg.pack_cache(c, a, 2, 64)
+    ref = bg.decode(q, packed, a, 2, 45)
+    Kh = bg.dequantize_keys(c["Kc"], c["Kn"], a)
+    Vh = bg.dequantize_values(c["Vc"], c["Vn"], 2)
+    out = bg.decode(q, packed, a, 2, 45, K_recent=Kh, V_recent=Vh)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+    # a recent token far more aligned with q than any cached one takes the whole softmax
+    Kr = np.zeros((1, 2, 1, 128))
+    Kr[0, :, 0] = 1e4 * q[0, ::2] / np.linalg.norm(q[0, ::2], axis=-1, keepdims=True)
+    Vr = np.full((1, 2, 1, 128), 7.0)
+    out2 = bg.decode(q[:, ::2], packed, a, 2, 45, K_recent=Kr, V_recent=Vr)
+    np.testing.assert_allclose(out2, 7.0, rtol=1e-12)
+
+
+def test_keys_only_cache_with_exact_values():
+    """A keys-only cache (bits_v = 0) holds the K part and K norms of every record; its decode
+    with the values given as the dequantized values of a K3V2 cache equals that cache's decode."""
+    K, V, q, a, c2 = _small_cache(33)
+    c0 = bg.quantize(K, V, a, 0)
+    assert c0["Vc"] is None
+    pk0 = bg.pack_cache(c0, a, 0, 64)
+    pk2 = bg.pack_cache(c2, a, 2, 64)
+    assert pk0.shape[-1] == bg.tile_record_bytes(128, 3, 0)
+    np.testing.assert_array_equal(pk0, pk2[..., :pk0.shape[-1]])      # same K half, byte for byte
+    Vh = bg.dequantize_values(c2["Vc"], c2["Vn"], 2)
+    np.testing.assert_array_equal(bg.decode(q, pk0, a, 0, 45, V=Vh), bg.decode(q, pk2, a, 2, 45))
 
 
 # ----------------------------------------------------------------- NF4
