@@ -30,7 +30,7 @@
 extern "C" {
 #endif
 
-#define KVQ_ABI_VERSION 3
+#define KVQ_ABI_VERSION 4
 #define KVQ_TILE_TOKENS 32     /* tokens per packed Block-GTQ tile */
 #define KVQ_HEAD_DIM 128       /* head dimension the kernels are built for */
 #define KVQ_MAX_WIDTH 8        /* widest Lloyd-Max codebook */
@@ -47,7 +47,8 @@ typedef enum {
   KVQ_ERR_WORKSPACE = 6,    /* workspace missing or smaller than the size query says */
   KVQ_ERR_CUDA = 7,         /* a CUDA runtime call or launch failed */
   KVQ_ERR_TIMEOUT = 8,      /* a device-side bounded wait gave up (read via kvq_workspace_status) */
-  KVQ_ERR_UNSUPPORTED = 9   /* a combination the library does not implement */
+  KVQ_ERR_UNSUPPORTED = 9,  /* a combination the library does not implement */
+  KVQ_ERR_MISMATCH = 10     /* packed cache header disagrees with the descriptor or the allocation */
 } kvq_status;
 
 typedef enum { KVQ_F32 = 0, KVQ_F16 = 1, KVQ_BF16 = 2 } kvq_dtype;
@@ -79,7 +80,9 @@ typedef struct {
 } kvq_calib_params;
 
 /* Shape of one packed Block-GTQ cache buffer (one layer). capacity = tokens per sequence
- * the buffer holds; storage is rounded up to whole 32-token tiles. */
+ * the buffer holds; storage is rounded up to whole 32-token tiles. bits_v = 0 makes a
+ * keys-only cache: the records hold no values, and the decode reads them from the caller's
+ * unquantized value tensor (kvq_decode_attn_ex). */
 typedef struct {
   int32_t batch;
   int32_t n_kv_heads;
@@ -114,19 +117,41 @@ typedef struct {
   int32_t k_words;          /* 32-bit words in a tile's K part (= bits_k * head_dim) */
   int32_t n_blocks;         /* blocks with w_b > 0 */
   int32_t reserved;
-  /* Decode plan, derived from the classes (written by kvq_calibrate, read by the decode).
-   * The K operand of the tensor-core product has one column per block pair, in stream order;
-   * each class is cut into groups of 4 pairs, its last group holding 2 pairs when at most 2
-   * remain (4 when 3 remain). Group x (counted over all classes) belongs to warp group
-   * g = x % 4 as its entry i = x / 4 and fills columns 24 g + 4 i .. 24 g + 4 i + 3; a run is a
-   * warp group's consecutive groups of one class. */
-  uint32_t plan_run[4][8];      /* width | first entry << 8 | groups << 16 | last group half << 24 */
-  uint32_t plan_group[4][16];   /* bit offset of the group in the K stream | first column << 16 */
-  int8_t plan_col_block[128];   /* block of column c, -1 for a padding column */
-  int32_t plan_n_runs[4];
-  int32_t plan_k_cols;          /* columns of the product (96) */
-  uint8_t reserved_c[108];
+  /* Decode plan (written by kvq_calibrate, read by the decode). The K operand of the
+   * tensor-core product has one column per block pair. Each width class, in stream order, is
+   * cut into slots of 4 consecutive block pairs; a class's last slot holds the 1..4 pairs left
+   * and the rest of it is padding. Slot s fills columns 4 s .. 4 s + 3. */
+  uint32_t plan_slot[24];       /* width | bit offset of the slot's first pair in the K stream << 8 */
+  int8_t plan_col_block[96];    /* block of column c, -1 for a padding column */
+  int32_t plan_n_slots;
+  int32_t plan_k_cols;          /* columns of the product: 4 * plan_n_slots rounded up to 8 */
+  uint64_t digest;              /* sum mod 2^64 over blocks b of splitmix64(b << 40 | w_b << 32 |
+                                   fp32 bits of g_b); also stored in the packed header */
+  uint8_t reserved_c[432];
 } kvq_head_alloc;
+
+/* Header at offset 0 of every packed Block-GTQ cache (kvq_packed_header_bytes(n_kv_heads)
+ * bytes; the tile records follow it). Written by kvq_quantize and by kvq_append with
+ * t_begin = 0; checked by kvq_append (t_begin > 0) and by the decode, which refuse a cache
+ * whose header disagrees with their descriptor or allocation (KVQ_ERR_MISMATCH) instead of
+ * returning attention over misread codes. */
+typedef struct {
+  uint32_t magic;           /* 0x3151564B, the bytes "KVQ1" */
+  uint16_t layout_version;  /* 1 */
+  uint16_t head_dim;
+  uint8_t bits_k;
+  uint8_t bits_v;           /* 0: keys only */
+  uint8_t w_max;
+  uint8_t mode;
+  uint32_t status;          /* 0, or the kvq_status of an append that found a mismatch */
+  int32_t batch;
+  int32_t n_kv_heads;
+  int32_t capacity;
+  uint32_t record_bytes;    /* bytes of one 32-token tile record */
+  uint8_t reserved[32];
+  /* followed (at byte 64) by uint64_t digest[n_kv_heads] (each head's kvq_head_alloc.digest), then zero
+   * padding to a multiple of 128 bytes */
+} kvq_packed_header;
 
 /* ---------------------------------------------------------------- queries (host only) */
 
@@ -150,8 +175,13 @@ size_t kvq_alloc_bytes(int n_kv_heads);
  * tokens per sequence. */
 size_t kvq_calibrate_workspace_bytes(int batch, int n_kv_heads, int n_calib_tokens);
 
-/* Bytes of one packed cache: batch * n_kv_heads * ceil(capacity/32) tile records, each
- * 4 * head_dim * (bits_k + bits_v) + 128 bytes. Returns 0 for an invalid descriptor. */
+/* Bytes of the header that starts every packed cache: 64 + 8 * n_kv_heads, rounded up to a
+ * multiple of 128 (0 for n_kv_heads < 1). */
+size_t kvq_packed_header_bytes(int n_kv_heads);
+
+/* Bytes of one packed cache: the header, then batch * n_kv_heads * ceil(capacity/32) tile
+ * records of 4 * head_dim * (bits_k + bits_v) + 128 bytes (keys only, bits_v = 0:
+ * 4 * head_dim * bits_k + 64 bytes). Returns 0 for an invalid descriptor. */
 size_t kvq_packed_bytes(const kvq_cache_desc* cache);
 
 /* Workspace bytes kvq_decode_attn needs for this cache and n_q_heads query heads. */
@@ -169,8 +199,25 @@ kvq_status kvq_init(void);
 kvq_status kvq_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronizes `stream`, copies the workspace status word to *device_code (host) and
- * returns KVQ_OK if it is 0, else the recorded kvq_status (e.g. KVQ_ERR_TIMEOUT). */
+ * returns KVQ_OK if it is 0, else the recorded kvq_status (e.g. KVQ_ERR_TIMEOUT,
+ * KVQ_ERR_MISMATCH). */
 kvq_status kvq_workspace_status(const void* ws, void* stream, int* device_code);
+
+/* Synchronizes `stream` and copies the status word of a packed cache's header to
+ * *device_code (host): 0, or KVQ_ERR_MISMATCH left by an append that refused to extend it.
+ * Returns KVQ_OK if it is 0, else that status. */
+kvq_status kvq_packed_status(const void* packed, void* stream, int* device_code);
+
+/* Text of the CUDA error behind the last KVQ_ERR_CUDA this process got from the library
+ * ("no error" if there was none). Host only. */
+const char* kvq_last_cuda_error(void);
+
+/* Test hook for the bounded waits of the Block-GTQ decode: later decode calls give up a wait
+ * after wait_limit tries (about 1 ms each; default 2000), and with no_loads != 0 they issue
+ * no copy at all, so their first wait on a stage runs out with no work in flight: the call
+ * then records KVQ_ERR_TIMEOUT in its workspace and writes nothing. Process-wide; meant
+ * for tests, never for production calls. Returns KVQ_ERR_ARG for wait_limit < 1. */
+kvq_status kvq_debug_decode(int wait_limit, int no_loads);
 
 /* ---------------------------------------------------------------- Block-GTQ hot path */
 
@@ -192,15 +239,18 @@ kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_p
 /* Quantize and pack the first kd->seq_len tokens of K and V into `packed` ([BGTQ]: Block-GTQ
  * on TQ-MSE, matched K/V budgets, packed cache). Per token row: fp16 norm, a = sqrt(d)/norm,
  * y = (x a) g_b in fp32, code = number of thresholds below y; K uses the allocation's
- * widths and gains, V uses width cache->bits_v and g = 1. Tiles past seq_len are not
- * written; tokens of the last tile beyond seq_len are stored as code 0, norm 0.
- * Layout: per (sequence, KV head) consecutive 32-token tile records of
+ * widths and gains, V uses width cache->bits_v and g = 1. Writes the packed header (see
+ * kvq_packed_header). Tiles past seq_len are not written; tokens of the last tile beyond
+ * seq_len are stored as code 0, norm 0.
+ * Layout after the header: per (sequence, KV head) consecutive 32-token tile records of
  * 4 * head_dim * (bits_k + bits_v) + 128 bytes, little-endian:
  *   K part: 32-bit word 32 i + t is word i (i < 4 bits_k) of token t's K stream (see
  *           kvq_head_alloc; codes least significant bit first, bits_k * head_dim bits).
  *   32 fp16 K norms, then 32 fp16 V norms, in token order.
  *   V part: word 128 i + j is word i (i < bits_v) of dim j's V stream: the codes of the
  *           tile's tokens 0..31 at dim j, bits_v bits each, least significant bit first.
+ * A keys-only cache (cache->bits_v = 0) stores the K part and the K norms only (records of
+ * 4 * head_dim * bits_k + 64 bytes); V and vd may then be NULL.
  * K, V: [batch][n_kv_heads][seq_len][128] (kd, vd may differ in strides, not in shape).
  * alloc: records from kvq_calibrate with bits_k == cache->bits_k.
  * packed: kvq_packed_bytes(cache) bytes, 16-byte aligned. */
@@ -217,6 +267,10 @@ kvq_status kvq_quantize(const void* K, const kvq_tensor4* kd, const void* V, con
  * tokens below t_begin in the first touched tile are kept (read back and merged); tokens from
  * t_begin + n to the end of the last touched tile are stored as code 0, norm 0. Tiles before
  * t_begin / 32 and after the last touched tile are not accessed.
+ * An append with t_begin = 0 writes the packed header. One with t_begin > 0 first checks it on
+ * the device: if it does not name this descriptor's shapes and widths and this allocation
+ * (or already holds a status), the call writes nothing and leaves KVQ_ERR_MISMATCH in the
+ * header's status word (kvq_packed_status; the decode reports it too).
  * Requires 0 <= t_begin and t_begin + n <= cache->capacity (else KVQ_ERR_RANGE); the stored
  * tokens below t_begin must have been written by an earlier call on the same stream (or one
  * that has completed). Attend over the grown cache with kvq_decode_attn(seq_len = t_begin + n). */
@@ -230,10 +284,42 @@ kvq_status kvq_append(const void* K, const kvq_tensor4* kd, const void* V, const
  * 0..seq_len-1: out = sum_t softmax_t(q . k_hat_t / sqrt(d)) v_hat_t with
  * k_hat = norm * c[code] * f_b and v_hat = norm * c[code] / sqrt(d).
  * packed, alloc: 16-byte aligned (as allocated by any CUDA allocator).
- * ws: kvq_decode_workspace_bytes bytes, zeroed once by kvq_workspace_init. */
+ * ws: kvq_decode_workspace_bytes bytes, zeroed once by kvq_workspace_init.
+ * The kernel checks the packed header against `cache` and `alloc` (per-head digest): on a
+ * mismatch, or a status an append left in the header, it records KVQ_ERR_MISMATCH in the
+ * workspace status word and writes nothing. Keys-only caches (bits_v = 0) need the values:
+ * use kvq_decode_attn_ex (KVQ_ERR_UNSUPPORTED here). */
 kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
                            const kvq_cache_desc* cache, int seq_len, float* out, void* ws,
                            size_t ws_bytes, void* stream);
+
+/* Extra inputs of kvq_decode_attn_ex. Every pointer may be NULL (then its view is ignored).
+ * V, vd: the values of a keys-only cache (cache->bits_v = 0; the Block-GTQ page quotes its key
+ *   error "K-only", with values left unquantized): [batch][n_kv_heads][>= seq_len][128] in
+ *   bf16 or fp16, row t = value of cached position t. Required for a keys-only cache, not
+ *   allowed with packed values.
+ * K_recent, V_recent, krd, vrd: the n_recent = krd.seq_len most recent tokens kept
+ *   unquantized (the Block-GTQ page reports its results "without an fp16 recent-key buffer",
+ *   which names this variant; here both their keys and values stay in the caller's dtype):
+ *   [batch][n_kv_heads][n_recent][128] each, any dtype; they are cached positions seq_len ..
+ *   seq_len + n_recent - 1 and join the packed positions in one softmax. */
+typedef struct {
+  const void* V;
+  kvq_tensor4 vd;
+  const void* K_recent;
+  kvq_tensor4 krd;
+  const void* V_recent;
+  kvq_tensor4 vrd;
+} kvq_decode_extra;
+
+/* kvq_decode_attn with the extra inputs above: out = sum over packed positions 0..seq_len-1
+ * and recent positions of softmax(q . k / sqrt(d)) v, where packed positions use k_hat (and
+ * v_hat, or the dense values of a keys-only cache) and recent positions their exact k and v.
+ * seq_len may be 0 when n_recent >= 1. Same workspace, header checks and status as
+ * kvq_decode_attn; extra = NULL is kvq_decode_attn. */
+kvq_status kvq_decode_attn_ex(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
+                              const kvq_cache_desc* cache, int seq_len, const kvq_decode_extra* extra, float* out,
+                              void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- NQKV-style NF4 variant */
 
@@ -278,19 +364,28 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
  * exactly what kvq_decode_attn computes (same arguments, without ws / ws_bytes) and uses as
  * its workspace a fixed scratch array of kvq_decode_noalloc_scratch_bytes() bytes (2 MiB)
  * that the library holds in device memory on every GPU that loads it, until the process
- * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
- * - The first call on a device looks up the array's address and zeroes it (synchronous);
- *   make that first call before any stream capture.
+ * exits. It calls no cudaMalloc, cudaFree or other allocating routine. It covers the
+ * Block-GTQ decode only (the NF4 decode has no allocation-free form).
+ * - The array's address is looked up on every call. The first call on a device (and the
+ *   first after its context was created again) zeroes the array with an asynchronous memset
+ *   on `stream`, ordered before the decode; make that first call before any stream capture.
  * - Shapes whose decode workspace (kvq_decode_workspace_bytes) exceeds the array return
  *   KVQ_ERR_WORKSPACE before anything is launched.
  * - Every call on a device shares the one array, which keeps the last call's contents; the
  *   split counters in it that must start at zero are returned to zero by every call. Calls
- *   that overlap on the GPU (other streams, other host threads) race on it: serialize them. */
+ *   that overlap on the GPU (other streams, other host threads) race on it: serialize them.
+ * - A device-side wait that gave up is recorded in the array's status word; read it with
+ *   kvq_decode_noalloc_status. */
 kvq_status kvq_decode_attn_noalloc(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
                                    const kvq_cache_desc* cache, int seq_len, float* out, void* stream);
 
 /* Size in bytes of the scratch array kvq_decode_attn_noalloc uses (2 MiB). */
 size_t kvq_decode_noalloc_scratch_bytes(void);
+
+/* Status of the allocation-free decode on the current device: synchronizes `stream`, copies
+ * the scratch array's status word to *device_code (host) and clears it. Returns KVQ_OK if it
+ * was 0, else the recorded kvq_status (e.g. KVQ_ERR_TIMEOUT). */
+kvq_status kvq_decode_noalloc_status(void* stream, int* device_code);
 
 #ifdef __cplusplus
 }

@@ -174,8 +174,8 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta, 32 / kCalibChunksPerC
 //     gains are non-increasing in w, so this is the step-by-step greedy with ties to the
 //     lowest block, the entries of a block that precede a given entry form a prefix (found
 //     by binary search), and the picked entries of a block are a prefix: w_b = their count.
-//  2. g_b, f_b, the K word offsets and the decode k-step table (blocks grouped by width,
-//     widest first, 4 per step, ascending block index within a width).
+//  2. g_b, f_b, the K stream order and bit offsets, the decode plan (width classes cut into
+//     slots of 4 block pairs) and the allocation digest.
 // The record is built in shared memory and copied out whole at the end.
 __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict__ energy, int bits_k, int w_max,
                                                         int mode, kvq_head_alloc* __restrict__ alloc) {
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
   __shared__ int sWidth[kH];
   __shared__ int sCount[9];
   __shared__ int sClsX0[9];
-  __shared__ int8_t sGrpCls[kH];   // class of each decode-plan group (at most 64 groups)
+  __shared__ uint64_t sDig[2];
   __shared__ double sSum;
   __shared__ __align__(16) kvq_head_alloc sRec;
   const int h = blockIdx.x, tid = threadIdx.x;
@@ -319,47 +319,39 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
     al->w_max = w_max;
     al->mode = mode;
     al->reserved = 0;
-    al->plan_k_cols = 96;
   }
   if (tid < kH && tid >= kH - sCount[0]) al->stream_block[tid] = 0xffu;   // positions past the last block
-  if (tid < 128) al->plan_col_block[tid] = -1;
+  if (tid < 96) al->plan_col_block[tid] = -1;
   __syncthreads();
-  // Decode plan: classes in stream order cut into groups of 4 block pairs (the last group
-  // 2 pairs when at most 2 remain); group x goes to warp group g = x % 4 as entry i = x / 4
-  // and fills columns 24 g + 4 i .. + 3 of the tensor-core operand. One thread per group.
-  const int n_groups = sClsX0[8];
-  if (tid < n_groups) {
+  // Decode plan: classes in stream order cut into slots of 4 consecutive block pairs (a
+  // class's last slot holds what is left); slot s covers columns 4s .. 4s + 3. One thread per
+  // slot; slots of a class start at that class's first slot index sClsX0[c].
+  const int n_slots = sClsX0[8];
+  if (tid < n_slots) {
     const int x = tid;
     int c = 0;
     while (sClsX0[c + 1] <= x) ++c;
     const int w = al->class_width[c], nb = al->class_blocks[c], first = al->class_first[c];
-    const int k = x - sClsX0[c], g = x & 3, col = 24 * g + 4 * (x >> 2);
-    sGrpCls[x] = static_cast<int8_t>(c);
-    al->plan_group[g][x >> 2] = static_cast<uint32_t>(al->class_bit[c] + 8 * w * k) | (static_cast<uint32_t>(col) << 16);
+    const int k = x - sClsX0[c];
+    al->plan_slot[x] = static_cast<uint32_t>(w) | (static_cast<uint32_t>(al->class_bit[c] + 8 * w * k) << 8);
     for (int i = 0; i < 4 && 4 * k + i < nb; ++i)
-      al->plan_col_block[col + i] = static_cast<int8_t>(al->stream_block[first + 4 * k + i]);
+      al->plan_col_block[4 * x + i] = static_cast<int8_t>(al->stream_block[first + 4 * k + i]);
+  }
+  if (tid == 0) {
+    al->plan_n_slots = n_slots;
+    al->plan_k_cols = (4 * n_slots + 7) / 8 * 8;
+  }
+  // Digest of the allocation: sum mod 2^64 over blocks of splitmix64(b << 40 | w_b << 32 | g_b bits).
+  if (tid < kH) {
+    uint64_t z = (static_cast<uint64_t>(tid) << 40) | (static_cast<uint64_t>(sWidth[tid]) << 32) |
+                 static_cast<uint64_t>(__float_as_uint(al->gain[tid]));
+    z = splitmix64(z);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if ((tid & 31) == 0) sDig[tid >> 5] = z;
   }
   __syncthreads();
-  // Runs: a warp group's consecutive entries of one class; flagged when the run holds its
-  // class's last group and that group has 1 or 2 pairs. One thread per warp group.
-  if (tid >= 128 && tid < 132) {
-    const int g = tid - 128;
-    int nr = 0, prev = -1;
-    uint32_t run = 0u;                          // the run being built
-    for (int x = g; x < n_groups; x += 4) {
-      const int c = sGrpCls[x];
-      if (c != prev) {
-        if (prev >= 0) al->plan_run[g][nr++] = run;
-        run = static_cast<uint32_t>(al->class_width[c]) | (static_cast<uint32_t>(x >> 2) << 8);
-        prev = c;
-      }
-      run += 1u << 16;
-      const int r = al->class_blocks[c] & 3;
-      if (x == sClsX0[c + 1] - 1 && r != 0 && r <= 2) run |= 1u << 24;
-    }
-    if (prev >= 0) al->plan_run[g][nr++] = run;
-    al->plan_n_runs[g] = nr;
-  }
+  if (tid == 0) al->digest = sDig[0] + sDig[1];
   __syncthreads();
   uint4* dst = reinterpret_cast<uint4*>(alloc + h);
   const uint4* src = reinterpret_cast<const uint4*>(&sRec);

@@ -62,32 +62,17 @@ __device__ __forceinline__ __nv_bfloat16 bits_to<__nv_bfloat16>(uint32_t b) {
 
 // ---------------------------------------------------------------- bit helpers
 
-__device__ __forceinline__ uint32_t rotr(uint32_t x, uint32_t n) { return __funnelshift_r(x, x, n); }
-
 __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
   return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }
 
-__device__ __forceinline__ uint32_t pack_u16x2(uint32_t lo, uint32_t hi) { return (lo & 0xffffu) | (hi << 16); }
-
-// ---------------------------------------------------------------- tensor-core fragments
-// mma.sync m16n8k8 / m16n8k16, fp16 operands, fp32 accumulate (row.col).
-
-__device__ __forceinline__ void mma_m16n8k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(b0));
-}
-
-__device__ __forceinline__ void mma_m16n8k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                             uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+// The SplitMix64 output function (Steele, Lea and Flood, OOPSLA 2014): one 64-bit mix. Used
+// for the allocation digest that ties a packed cache to the allocation it was written with.
+__host__ __device__ __forceinline__ uint64_t splitmix64(uint64_t z) {
+  z += 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -104,18 +89,7 @@ __device__ __forceinline__ void split_hilo(float x, __half& hi, __half& lo) {
 
 // ---------------------------------------------------------------- async copies (cp.async, 16 B)
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
-// Wait until at most n (0..2) of this thread's cp.async groups are pending.
-__device__ __forceinline__ void cp_async_wait_pending(int n) {
-  if (n <= 0) cp_async_wait<0>();
-  else if (n == 1) cp_async_wait<1>();
-  else cp_async_wait<2>();
-}
-
 }  // namespace kvq

@@ -2,31 +2,40 @@
 // allocation for KV cache quantization", abstract: attention served from the packed cache;
 // the NQKV review's editorial extensions propose folding the table lookup into attention).
 //
-// Grid: (splits, batch * n_kv_heads). Each CTA owns a contiguous range of 128-token chunks
-// (4 tile records) of one (sequence, KV head) and walks it in segments of up to 16 chunks,
-// each in two passes:
-//   pass 1 (keys)   16 warps dequantize K codes through shared-memory lookup tables into
-//                   tensor memory (K-hat rows, lane = token, one fp16 pair per column); one
-//                   thread issues S^T[128 tokens][16] = Khat x Q'^T (tcgen05.mma, M 128, N 16,
-//                   Q' hi rows 0-7 and lo rows 8-15 in shared memory); each thread keeps the
-//                   scaled logits of its token in shared memory and a running maximum;
-//   segment max     one exchange per warp group gives the segment's maximum per query row;
-//                   the running (m, l, O) are rescaled once;
-//   pass 2 (values) 16 warps dequantize V codes into V-hat^T rows (lane = dim); each thread
-//                   turns its logits into P' = 2^(s - m) vnorm / sqrt(d), split into fp16 hi
-//                   + lo (the B operand); O^T[128 dims][16] += Vhat^T x P'^T accumulates in
-//                   tensor memory over the whole segment and is read once at its end.
-// A load warp bulk-copies the key half (K words + norms) of every tile for pass 1 and the
-// value half (norms + V words) for pass 2 through a ring of shared-memory stages. Q' carries
-// f_b, log2(e)/sqrt(d) and a per-row power of two that keeps its fp16 split in range; the
-// key norm scales S after the MMA. The K operand's columns come from the allocation's decode
-// plan: width classes cut into groups of 4 block pairs (a class's last group 2 pairs when at
-// most 2 remain), warp group g owning columns 24 g .. 24 g + 23; each thread decodes its
-// groups into registers and writes them with one wide tensor-memory store per chunk. Warp
-// group g handles query rows 2g, 2g+1 of the softmax and of O. Every hand-off is an mbarrier
-// with a bounded wait.
-// Splits write (m, l, O) partials to the workspace; the last CTA of a (sequence, KV head),
-// found with an atomic ticket, merges them all and writes out = O / l.
+// Grid: (splits, batch * n_kv_heads), one CTA per SM. A CTA owns a contiguous range of
+// 128-token chunks (4 tile records, contiguous in memory) of one (sequence, KV head).
+// Four compute warpgroups each run their own chunk pipeline over chunks g, g + 4, g + 8, ..
+// of the range, so no warpgroup waits for another:
+//   load     the warpgroup's leader bulk-copies whole chunks (one copy of 4 records) into its
+//            own ring of stages, several chunks ahead;
+//   keys     lane = token: the K codes of each slot of the allocation's plan (4 block pairs of
+//            one width) are looked up in shared-memory pair tables and written to tensor
+//            memory, 16 columns per store (K-hat rows, one fp16 pair per column);
+//   S        the leader issues S^T[128 tokens][16] = Khat x Q'^T (tcgen05.mma, M 128, N 16;
+//            Q' rows 0-7 the fp16 high parts of the 8 query rows, rows 8-15 the low parts);
+//   values   lane = dim: the chunk's V codes go to tensor memory over the K-hat columns
+//            (V-hat^T rows, one fp16 pair of tokens per column);
+//   softmax  lane = token: logits s = S * key norm * 2^e (per row), the chunk's maximum per
+//            row over the warpgroup, and an online softmax whose running maximum is only raised
+//            when a chunk exceeds it by more than 2^8 (then O is rescaled in tensor memory);
+//            P' = 2^(s - m - 8) * value norm / sqrt(d), split into fp16 hi + lo, is the B
+//            operand of O;
+//   O        the leader issues O^T[128 dims][16] += Vhat^T x P'^T, accumulated over all of
+//            the warpgroup's chunks in tensor memory.
+// Q' carries f_b, log2(e)/sqrt(d) and a per-row power of two that keeps its fp16 split in
+// range. The four warpgroups' (m, l, O) are combined in shared memory; splits then meet in a
+// two-level tree: the last CTA of each group of about sqrt(splits) splits (atomic ticket)
+// merges the group, and the last group to finish merges the groups and writes out = O / l.
+// Keys-only caches (the Block-GTQ page quotes its key error "K-only"): the values of each
+// chunk arrive as dense bf16/fp16 rows next to the chunk's K records and are transposed into
+// tensor memory (lane = dim); O then runs on bf16 (or fp16) operands with P' split to match.
+// Recent tokens kept unquantized (reading of the page's "fp16 recent-key buffer"): the three
+// helper warps of every CTA, once Q' is built, attend over an even share of them on CUDA
+// cores (lane = 4 dims) and add a fifth partial to the CTA's combine.
+// Every wait is bounded. A wait that gives up records KVQ_ERR_TIMEOUT and stops the
+// warpgroup at its next barrier; the CTA waits (bounded) for its copies and products in
+// flight, frees tensor memory and writes nothing. A packed header or allocation that does
+// not match the call records KVQ_ERR_MISMATCH and writes nothing either.
 #pragma once
 
 #include "common.cuh"
@@ -34,33 +43,23 @@
 
 namespace kvq {
 
-constexpr int kDecComputeWarps = 16;
-constexpr int kDecMmaWarp = 16;      // builds Q', issues the MMAs of even chunks
-constexpr int kDecLoadWarp = 17;
-constexpr int kDecMma2Warp = 18;     // issues the MMAs of odd chunks
-constexpr int kDecThreads = 19 * 32;
+constexpr int kDecWG = 4;                 // compute warpgroups
+constexpr int kDecWgWarp0 = 4;            // first compute warp (warp % 4 = tensor-memory quarter)
+constexpr int kDecThreads = (kDecWgWarp0 + 4 * kDecWG) * 32;
 constexpr int kChunkTiles = 4;
 constexpr int kChunkTokens = kChunkTiles * kTile;   // = MMA M = tensor-memory lanes
-constexpr int kSegChunks = 16;                       // chunks per two-pass segment
-constexpr int kDecStagesMax = 8;
-constexpr int kMaxMergeSplits = 160;
-constexpr int kMergeGroup = 8;       // splits merged by the last CTA of each group (first level)
-constexpr int kTargetCtas = 148;     // one CTA per SM on a 148-SM B200
-constexpr int kGroupPairs = 4;       // block pairs (tensor-memory columns) per full K group
-constexpr int kMaxKGroups = 16;      // per warp group (at most 24 groups per head in all)
-constexpr int kMaxRuns = 8;          // runs of equal-width K groups per warp group
-constexpr int kSlots = 6;            // K groups per warp group
-constexpr int kSlotCols = 4 * kSlots;  // K columns per warp group
-constexpr uint32_t kWaitLimit = 2000;   // suspended tries (about 2 s) before a wait gives up
-
-// Tensor-memory columns (512 allocated).
+constexpr int kStagesMax = 4;             // chunk stages per warpgroup
+constexpr int kTau = 8;                   // lazy rescale threshold (log2 units)
 constexpr uint32_t kTmemCols = 512;
-// The key pass keeps 3 chunks in flight (its logits trail the dequantization by 2 chunks),
-// the value pass 2.
-__device__ __forceinline__ uint32_t col_ak(int b) { return 96u * b; }         // K-hat, 3 x 96
-__device__ __forceinline__ uint32_t col_s(int b) { return 288u + 16u * b; }   // S, 3 x 16
-__device__ __forceinline__ uint32_t col_av(int b) { return 336u + 64u * b; }  // V-hat^T, 2 x 64
-__device__ __forceinline__ uint32_t col_o(int p) { return 464u + 16u * p; }  // O, 2 x 16 (chunk parity)
+constexpr int kPlanSlots = 24;
+constexpr int kMergeMax = 64;             // entries one merge step reads
+constexpr uint32_t kHeaderMagic = 0x3151564Bu;   // "KVQ1"
+constexpr int kLayoutVersion = 1;
+
+// Tensor-memory columns of warpgroup g: A (K-hat, then V-hat^T) 96, S 16, O 16.
+__device__ __forceinline__ uint32_t col_a(int g) { return 128u * g; }
+__device__ __forceinline__ uint32_t col_s(int g) { return 128u * g + 96u; }
+__device__ __forceinline__ uint32_t col_o(int g) { return 128u * g + 112u; }
 
 // Lookup-table image, built once per device (decode_lut_image) and bulk-copied into every
 // CTA's shared memory at byte 0. Pair tables give the fp16 pair {c[i & m], c[i >> w]} for the
@@ -75,48 +74,44 @@ constexpr int kLutBytes = 33024;
 // Shared-memory map (byte offsets from the start of dynamic shared memory).
 constexpr int kAllocOff = kLutBytes;                 // copy of the KV head's kvq_head_alloc
 constexpr int kBQOff = ((kAllocOff + static_cast<int>(sizeof(kvq_head_alloc)) + 127) / 128) * 128;
-                                                     // Q' (B operand of S), K-major, <= 256 K elements
-constexpr int kBQBytes = 32 * 256;
-constexpr int kBPOff = kBQOff + kBQBytes;            // P' (B operand of O), 2 buffers, N-major
+constexpr int kBQBytes = 8192;                       // Q' (B operand of S), K-major, <= 256 K elements
+constexpr int kBPOff = kBQOff + kBQBytes;            // P' (B operand of O), one per warpgroup, N-major
 constexpr int kBPBytes = 4096;
-constexpr int kStashOff = kBPOff + 2 * kBPBytes;     // logits of a segment: [chunk][row][token] fp32
-constexpr int kStashBytes = kSegChunks * 8 * kChunkTokens * 4;
-constexpr int kHdrOff = kStashOff + kStashBytes;
+constexpr int kRecOff = kBPOff + kDecWG * kBPBytes;  // recent tokens' O share [8][128] fp32
+constexpr int kRecQOff = kRecOff + 8 * kD * 4;       // recent tokens' q * log2(e) / sqrt(d) [8][128]
+constexpr int kHdrOff = kRecQOff + 8 * kD * 4;
 static_assert(kLutBytes % 16 == 0 && kAllocOff % 16 == 0 && sizeof(kvq_head_alloc) % 16 == 0,
               "bulk-copied regions must be 16-byte multiples");
-static_assert(kBQOff >= kAllocOff + static_cast<int>(sizeof(kvq_head_alloc)) && kBQOff % 128 == 0,
-              "Q' must not overlap the allocation copy");
+static_assert(sizeof(kvq_head_alloc) == 2048 && sizeof(kvq_packed_header) == 64, "ABI record sizes");
 
 struct DecHeader {
-  uint64_t full[kDecStagesMax];
-  uint64_t empty[kDecStagesMax];
-  uint64_t kready[3], sfull[3], vpready[2], ofull[2];
+  uint64_t full[kDecWG][kStagesMax];
+  uint64_t sfull[kDecWG];
+  uint64_t ofull[kDecWG];
   uint64_t setup;                    // lookup tables + allocation record copied in
-  uint64_t qready;                   // Q' and qscale written (MMA warp)
+  uint64_t qready;                   // Q' and qscale written
   uint32_t tmem_base;
+  int bad;                           // header or allocation mismatch: the CTA writes nothing
+  int wg_abort[kDecWG];              // a wait of this warpgroup gave up
   float qscale[8];                   // 2^e that undoes the range scaling of Q' row h
-  float xmax[2][4][4][2];            // segment max: [segment parity][warp group][quarter][row]
-  float lpart[4][4][2];              // row sums: [warp group][quarter][row]
+  float xch[kDecWG][4][8];           // chunk maximum: [warpgroup][warp][row]
+  float lred[kDecWG][4][8];          // row sums: [warpgroup][warp][row]
+  float wg_m[kDecWG + 1][8];         // warpgroup (and recent-token) results: maximum
+  float wg_l[kDecWG + 1][8];         //                                        and row sum
+  float rx_m[3][8];                  // recent tokens: per helper warp maximum
+  float rx_l[3][8];                  //                              and row sum
   int last;
-  float mw[8][kMaxMergeSplits];      // cross-split merge: member m, then weight 2^(m_s - M)
-  float ml[8][kMaxMergeSplits];      // cross-split merge: member l
-  float Lsum[8];
-  float Mmax[8];
+  float mw[8][kMergeMax];            // merge: member maxima, then weights
+  float ml[8][kMergeMax];            //        member row sums
+  float Msum[8][2];                  //        merged maximum and row sum
 };
 
 __host__ __device__ constexpr int decode_stage_off() {
   return kHdrOff + ((static_cast<int>(sizeof(DecHeader)) + 127) / 128) * 128;
 }
 
-// Byte sizes of the key half (K words + K norms) and the value half (V norms + V words) of a
-// tile record. A stage holds 4 tiles; a tile's slot also covers K word rows 4 bits_k and
-// 4 bits_k + 1 (up to byte 512 bits_k + 256), which the last K groups of a token read past
-// the end of its stream, so every read stays inside the slot.
-__host__ __device__ constexpr int key_half_bytes(int bits_k) { return 4 * kD * bits_k + 2 * kTile; }
-__host__ __device__ constexpr int value_half_bytes(int bits_v) { return 2 * kTile + 4 * kD * bits_v; }
-__host__ __device__ constexpr int stage_tile_stride(int bits_k, int bits_v) {
-  return (4 * kD * bits_k + 256) > value_half_bytes(bits_v) ? (4 * kD * bits_k + 256) : value_half_bytes(bits_v);
-}
+// Bytes of a chunk stage: 4 tile records.
+__host__ __device__ constexpr int chunk_bytes(int rec_bytes) { return kChunkTiles * rec_bytes; }
 
 // Host: the lookup-table image from the fp16 centroid table (width w at c16 + 2^w - 2).
 inline void decode_lut_image(const uint16_t* c16, uint8_t* img) {
@@ -138,15 +133,6 @@ inline void decode_lut_image(const uint16_t* c16, uint8_t* img) {
 __device__ __align__(16) uint8_t g_dec_lut[kLutBytes];
 
 // ---------------------------------------------------------------- code extraction + lookup
-
-// Bits [p, p + n) of the 64-bit value hi:lo (p, n constant after unrolling, n <= 16).
-__device__ __forceinline__ uint32_t field(uint32_t lo, uint32_t hi, int p, int n) {
-  uint32_t v;
-  if (p >= 32) v = hi >> (p - 32);
-  else if (p + n <= 32) v = lo >> p;
-  else v = __funnelshift_r(lo, hi, p);
-  return v & ((1u << n) - 1u);
-}
 
 // Bits [p, p + n) of hi:lo moved to bit position `sh` (p, n, sh constant after unrolling):
 // one funnel shift (or plain shift) and one mask.
@@ -178,37 +164,34 @@ __device__ __forceinline__ uint32_t pair_value(uint32_t lo, uint32_t hi, int p, 
   }
 }
 
-// Values of NP consecutive block pairs of width W whose first code starts at bit `off` of
-// this lane's token stream; kw points at word 0 of the token (word i at kw[32 i]).
-template <int W, int NP>
+// Values of 4 consecutive block pairs of width W whose first code starts at bit `off` of this
+// lane's token stream; kw points at word 0 of the token (word i at kw[32 i]).
+template <int W>
 __device__ __forceinline__ void k_group_vals(const uint32_t* kw, uint32_t off, const uint8_t* sm, uint32_t lane4,
-                                             uint32_t (&v)[NP]) {
+                                             uint32_t (&v)[4]) {
   const uint32_t j0 = off >> 5, s = off & 31u;
   const uint32_t x0 = kw[j0 * 32], x1 = kw[(j0 + 1) * 32];
-  const uint32_t x2 = (2 * W * NP > 32) ? kw[(j0 + 2) * 32] : 0u;
+  const uint32_t x2 = (8 * W > 32) ? kw[(j0 + 2) * 32] : 0u;
   const uint32_t r0 = __funnelshift_r(x0, x1, s);
   const uint32_t r1 = __funnelshift_r(x1, x2, s);
 #pragma unroll
-  for (int k = 0; k < NP; ++k) v[k] = pair_value<W>(r0, r1, 2 * W * k, sm, lane4);
+  for (int k = 0; k < 4; ++k) v[k] = pair_value<W>(r0, r1, 2 * W * k, sm, lane4);
 }
 
-// Values of the K group in one register slot: e = width | bit offset << 8 (width 0: an empty
-// slot, left zero). A group with only 2 real pairs is decoded as 4; the other 2 columns have
-// a zero Q' row. Slots sit at compile-time register positions and reach tensor memory in one
-// wide store per chunk afterwards: small stores issued between the lookups were measured to
-// slow the whole dequantization several times over.
+// Values of one plan slot: e = width | bit offset << 8 (width 0: an empty slot, zeros). A
+// slot with fewer than 4 real pairs is decoded as 4; its other columns have zero Q' rows.
 __device__ __forceinline__ void k_slot(uint32_t e, const uint32_t* kw, const uint8_t* sm, uint32_t lane4,
-                                       uint32_t (&t)[kGroupPairs]) {
+                                       uint32_t (&t)[4]) {
   const uint32_t off = e >> 8;
   switch (e & 15u) {
-    case 1: k_group_vals<1, kGroupPairs>(kw, off, sm, lane4, t); break;
-    case 2: k_group_vals<2, kGroupPairs>(kw, off, sm, lane4, t); break;
-    case 3: k_group_vals<3, kGroupPairs>(kw, off, sm, lane4, t); break;
-    case 4: k_group_vals<4, kGroupPairs>(kw, off, sm, lane4, t); break;
-    case 5: k_group_vals<5, kGroupPairs>(kw, off, sm, lane4, t); break;
-    case 6: k_group_vals<6, kGroupPairs>(kw, off, sm, lane4, t); break;
-    case 7: k_group_vals<7, kGroupPairs>(kw, off, sm, lane4, t); break;
-    case 8: k_group_vals<8, kGroupPairs>(kw, off, sm, lane4, t); break;
+    case 1: k_group_vals<1>(kw, off, sm, lane4, t); break;
+    case 2: k_group_vals<2>(kw, off, sm, lane4, t); break;
+    case 3: k_group_vals<3>(kw, off, sm, lane4, t); break;
+    case 4: k_group_vals<4>(kw, off, sm, lane4, t); break;
+    case 5: k_group_vals<5>(kw, off, sm, lane4, t); break;
+    case 6: k_group_vals<6>(kw, off, sm, lane4, t); break;
+    case 7: k_group_vals<7>(kw, off, sm, lane4, t); break;
+    case 8: k_group_vals<8>(kw, off, sm, lane4, t); break;
     default: t[0] = 0u; t[1] = 0u; t[2] = 0u; t[3] = 0u; break;
   }
 }
@@ -238,496 +221,663 @@ __device__ __forceinline__ float from_ordered(int i) { return __int_as_float(i ^
 
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-__device__ __forceinline__ void record_timeout(unsigned* status) { atomicCAS(status, 0u, static_cast<unsigned>(KVQ_ERR_TIMEOUT)); }
+__device__ __forceinline__ void record_status(unsigned* status, unsigned code) { atomicCAS(status, 0u, code); }
 
-// ---------------------------------------------------------------- cross-split merge
+// Element i of a tensor of run-time dtype (kvq_dtype) as fp32.
+__device__ __forceinline__ float load_f32(const void* p, int dtype, int64_t i) {
+  if (dtype == KVQ_F32) return static_cast<const float*>(p)[i];
+  if (dtype == KVQ_F16) return __half2float(static_cast<const __half*>(p)[i]);
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+}
 
-// Merge the n (m, l, O) partials of (sequence, KV head) bh (entries 0..n-1 of its row of the
-// workspace) into out = O / l for its G real query heads. Called by every thread of the CTA:
-// all members' (m, l) are fetched in one round, then 512 threads sum O (256 float4 quads,
-// two halves of the member list each, 8 loads in flight).
-__device__ __forceinline__ void merge_partials(DecHeader& S, uint8_t* scratch, int bh, int pitch, int n,
-                                               const float* part_m, const float* part_l, const float* part_o,
-                                               float* out, int G) {
+// ---------------------------------------------------------------- kernel arguments
+
+struct DecArgs {
+  const void* q;
+  int64_t qsb, qsh;
+  int q_dtype;
+  int n_q_heads, n_kv_heads, batch;
+  // keys-only cache: dense values [batch][n_kv_heads][>= seq_len][128] (bf16 or fp16)
+  const void* v_dense;
+  int64_t vsb, vsh, vst;
+  int cbytes;                        // bytes of a chunk stage (records, then dense value rows)
+  // recent tokens kept unquantized: [batch][n_kv_heads][n_recent][128] keys and values
+  const void* k_rec;
+  const void* v_rec;
+  int64_t krsb, krsh, krst, vrsb, vrsh, vrst;
+  int kr_dtype, vr_dtype, n_recent;
+  const uint8_t* packed;             // header at byte 0, records at byte hdr_bytes
+  const kvq_head_alloc* alloc;
+  int hdr_bytes, tiles_cap, rec_bytes, bits_k, bits_v, capacity;
+  int seq_len, splits, n_groups, group_size, n_stages;
+  float* out;
+  float* part_m;                     // [bh][splits + n_groups][8]
+  float* part_l;
+  float* part_o;                     // [bh][splits + n_groups][8][128]
+  unsigned* tickets;                 // [bh][1 + n_groups]
+  unsigned* status;
+  uint32_t wait_limit;
+  int debug_no_loads;                // test hook: issue no copy, so every wait on a stage gives up
+};
+
+// ---------------------------------------------------------------- split merge
+
+// Merges entries e0 .. e0 + n - 1 (n <= kMergeMax) of row bh, each (m, l, O) with O
+// unnormalized and m in log2 units. Writes the merged entry to `dst_entry` (>= 0) or
+// out = O / l (dst_entry < 0). Called by every thread of the CTA.
+__device__ __forceinline__ void merge_entries(DecHeader& S, const DecArgs& a, int bh, int pitch, int e0, int n,
+                                              int dst_entry, float* out_bh, int G) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const size_t row = static_cast<size_t>(bh) * pitch * 8;
+  const size_t row = static_cast<size_t>(bh) * pitch;
   for (int i = tid; i < 8 * n; i += blockDim.x) {
-    const int s = i >> 3, hg = i & 7;
-    S.mw[hg][s] = __ldcg(part_m + row + i);
-    S.ml[hg][s] = __ldcg(part_l + row + i);
+    const int s = i >> 3, h = i & 7;
+    S.mw[h][s] = __ldcg(a.part_m + (row + e0 + s) * 8 + h);
+    S.ml[h][s] = __ldcg(a.part_l + (row + e0 + s) * 8 + h);
   }
   __syncthreads();
   if (warp < 8) {
-    const int hg = warp;
+    const int h = warp;
     float M = -INFINITY;
-    for (int s = lane; s < n; s += 32) M = fmaxf(M, S.mw[hg][s]);
+    for (int s = lane; s < n; s += 32) M = fmaxf(M, S.mw[h][s]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.0f;
     for (int s = lane; s < n; s += 32) {
-      const float ms = S.mw[hg][s];
+      const float ms = S.mw[h][s];
       const float wt = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-      S.mw[hg][s] = wt;
-      L += S.ml[hg][s] * wt;
+      S.mw[h][s] = wt;
+      L += S.ml[h][s] * wt;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) S.Lsum[hg] = L;
+    if (lane == 0) {
+      S.Msum[h][0] = M;
+      S.Msum[h][1] = L;
+    }
   }
   __syncthreads();
-  const int quad = tid & 255, half = tid >> 8;
-  const int hg = quad >> 5, j4 = quad & 31;
-  const int s_mid = n / 2;
-  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (half < 2) {
-    const int s0 = half ? s_mid : 0, s1 = half ? n : s_mid;
-    const float4* po = reinterpret_cast<const float4*>(part_o) + (row + hg) * (kD / 4) + j4;
-#pragma unroll 8
-    for (int s = s0; s < s1; ++s) {
-      const float wt = S.mw[hg][s];
+  if (tid < 256) {
+    const int h = tid >> 5, j4 = tid & 31;
+    const float4* po = reinterpret_cast<const float4*>(a.part_o) + ((row + e0) * 8 + h) * (kD / 4) + j4;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = 0; s < n; ++s) {
+      const float wt = S.mw[h][s];
       const float4 v = __ldcg(po + static_cast<size_t>(s) * 8 * (kD / 4));
       o.x += v.x * wt; o.y += v.y * wt; o.z += v.z * wt; o.w += v.w * wt;
     }
-  }
-  float4* red = reinterpret_cast<float4*>(scratch);
-  if (half == 1) red[quad] = o;
-  __syncthreads();
-  if (half == 0 && hg < G) {
-    const float4 v = red[quad];
-    const float inv = 1.0f / S.Lsum[hg];
-    reinterpret_cast<float4*>(out + static_cast<size_t>(hg) * kD)[j4] =
-        make_float4((o.x + v.x) * inv, (o.y + v.y) * inv, (o.z + v.z) * inv, (o.w + v.w) * inv);
+    if (dst_entry >= 0) {
+      reinterpret_cast<float4*>(a.part_o)[((row + dst_entry) * 8 + h) * (kD / 4) + j4] = o;
+      if (j4 == 0) {
+        a.part_m[(row + dst_entry) * 8 + h] = S.Msum[h][0];
+        a.part_l[(row + dst_entry) * 8 + h] = S.Msum[h][1];
+      }
+    } else if (h < G) {
+      const float inv = 1.0f / S.Msum[h][1];
+      reinterpret_cast<float4*>(out_bh + static_cast<size_t>(h) * kD)[j4] =
+          make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+    }
   }
 }
 
 // ---------------------------------------------------------------- the kernel
 
-// One instantiation per value width BVT (= bits_v).
-template <int DT, int BVT>
-__global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(
-    const typename Elem<DT>::T* __restrict__ q, int64_t qsb, int64_t qsh, int n_q_heads, int n_kv_heads,
-    const uint8_t* __restrict__ packed, const kvq_head_alloc* __restrict__ alloc, int tiles_cap, int rec_bytes,
-    int bits_k, int bits_v, int seq_len, int splits, int n_groups, int n_stages, float* __restrict__ out,
-    float* __restrict__ part_m, float* __restrict__ part_l, float* __restrict__ part_o,
-    unsigned* __restrict__ tickets, unsigned* __restrict__ status) {
+// Dense value modes of kvq_decode_gtq (keys-only caches): bf16 or fp16 value rows.
+constexpr int kDenseBf16 = 16;
+constexpr int kDenseF16 = 17;
+
+// Splits x into hi + lo of the 16-bit type of the O operands (bf16 when kBf, else fp16),
+// returned as their bit patterns.
+template <bool kBf>
+__device__ __forceinline__ void split16(float x, uint32_t& hi, uint32_t& lo) {
+  if constexpr (kBf) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi = __bfloat16_as_ushort(h);
+    lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
+  } else {
+    const __half h = __float2half_rn(x);
+    hi = __half_as_ushort(h);
+    lo = __half_as_ushort(__float2half_rn(x - __half2float(h)));
+  }
+}
+
+// One instantiation per value mode VM: 1..8 = packed values of that width; kDenseBf16 /
+// kDenseF16 = keys-only cache with dense value rows of that type.
+template <int VM>
+__global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a) {
+  constexpr bool kDense = VM >= kDenseBf16;
+  constexpr bool kBfO = VM == kDenseBf16;                  // O operands in bf16
   extern __shared__ __align__(1024) uint8_t sm[];
   DecHeader& S = *reinterpret_cast<DecHeader*>(sm + kHdrOff);
   uint8_t* stages = sm + decode_stage_off();
+  float* rec_o = reinterpret_cast<float*>(sm + kRecOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, bh = blockIdx.y;
-  const int b = bh / n_kv_heads, hkv = bh % n_kv_heads;
-  const int G = n_q_heads / n_kv_heads;
-  const kvq_head_alloc* al = alloc + hkv;
-  // An allocation made for another budget does not match the record size: write nothing.
-  if (al->k_words != bits_k * kD || al->bits_k != bits_k) return;
-  const int n_tiles = (seq_len + kTile - 1) / kTile;
+  const int b = bh / a.n_kv_heads, hkv = bh % a.n_kv_heads;
+  const int G = a.n_q_heads / a.n_kv_heads;
+  const kvq_head_alloc* al = a.alloc + hkv;
+  const int n_tiles = (a.seq_len + kTile - 1) / kTile;
   const int n_chunks_all = (n_tiles + kChunkTiles - 1) / kChunkTiles;
-  const int c_begin = static_cast<int>((static_cast<long long>(split) * n_chunks_all) / splits);
-  const int c_end = static_cast<int>((static_cast<long long>(split + 1) * n_chunks_all) / splits);
+  const int c_begin = static_cast<int>((static_cast<long long>(split) * n_chunks_all) / a.splits);
+  const int c_end = static_cast<int>((static_cast<long long>(split + 1) * n_chunks_all) / a.splits);
   const int n_chunks = c_end - c_begin;
-  const int n_segs = (n_chunks + kSegChunks - 1) / kSegChunks;
-  const int tile_end = min(n_tiles, c_end * kChunkTiles);
-  const uint8_t* src = packed + static_cast<size_t>(bh) * tiles_cap * rec_bytes;
-  const int khalf = key_half_bytes(bits_k), vhalf = value_half_bytes(bits_v);
-  const int tstride = stage_tile_stride(bits_k, bits_v);
-  const int stage_bytes = kChunkTiles * tstride;
+  const uint8_t* src = a.packed + a.hdr_bytes + static_cast<size_t>(bh) * a.tiles_cap * a.rec_bytes;
+  const int cbytes = a.cbytes;
+  const int kbytes = 4 * kD * a.bits_k;             // K words of a record
+  const int NS = a.n_stages;
   const float inv_sqrt_d = 0.08838834764831845f;
-  constexpr int kSetupThreads = (kDecComputeWarps + 2) * 32;   // compute warps and both MMA warps
+  const uint32_t WL = a.wait_limit;
 
-  // ------------------------------------------------------------------ barriers
+  // ------------------------------------------------------------------ barriers, TMEM
   if (tid == 0) {
-    for (int i = 0; i < kDecStagesMax; ++i) {
-      tc::mbar_init(&S.full[i], 1);
-      tc::mbar_init(&S.empty[i], kDecComputeWarps);
-    }
-    for (int i = 0; i < 3; ++i) {
-      tc::mbar_init(&S.kready[i], kDecComputeWarps);
-      tc::mbar_init(&S.sfull[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&S.vpready[i], kDecComputeWarps);
-      tc::mbar_init(&S.ofull[i], 1);
+    for (int g = 0; g < kDecWG; ++g) {
+      for (int i = 0; i < kStagesMax; ++i) tc::mbar_init(&S.full[g][i], 1);
+      tc::mbar_init(&S.sfull[g], 1);
+      tc::mbar_init(&S.ofull[g], 1);
+      S.wg_abort[g] = 0;
     }
     tc::mbar_init(&S.setup, 1);
     tc::mbar_init(&S.qready, 1);
+    S.bad = 0;
     tc::mbar_fence_init();
   }
+  if (tid < 8) S.wg_m[kDecWG][tid] = -INFINITY;             // no recent share unless the helpers add one
+  if (warp == 0) tc::tmem_alloc(&S.tmem_base, kTmemCols);
+  tc::fence_before_sync();
   __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = S.tmem_base;
 
-  if (warp == kDecLoadWarp) {
-    // ---------------------------------------------------------------- bulk loads
-    // Items in consumption order: per segment the key halves of its chunks, then the value
-    // halves; item k uses stage k % n_stages.
-    if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&S.setup, kLutBytes + static_cast<uint32_t>(sizeof(kvq_head_alloc)));
-      tc::bulk_g2s(sm, g_dec_lut, kLutBytes, &S.setup);
-      tc::bulk_g2s(sm + kAllocOff, al, sizeof(kvq_head_alloc), &S.setup);
-      int k = 0;
-      bool ok = true;
-      for (int sg = 0; sg < n_segs && ok; ++sg) {
-        const int u0 = sg * kSegChunks, nu = min(kSegChunks, n_chunks - u0);
-        for (int half = 0; half < 2 && ok; ++half) {
-          const int bytes = half ? vhalf : khalf, off = half ? khalf : 0;
-          for (int u = 0; u < nu; ++u, ++k) {
-            const int s = k % n_stages;
-            if (k >= n_stages && !tc::mbar_wait(&S.empty[s], ((k / n_stages) - 1) & 1, kWaitLimit)) {
-              ok = false;
-              break;
-            }
-            const int tile0 = (c_begin + u0 + u) * kChunkTiles;
-            const int nt = min(kChunkTiles, tile_end - tile0);
-            tc::mbar_arrive_expect_tx(&S.full[s], static_cast<uint32_t>(nt * bytes));
-            for (int t = 0; t < nt; ++t)
-              tc::bulk_g2s(stages + s * stage_bytes + t * tstride,
-                           src + static_cast<size_t>(tile0 + t) * rec_bytes + off, static_cast<uint32_t>(bytes),
-                           &S.full[s]);
-          }
-        }
-      }
-      if (!ok) record_timeout(status);
+  // Warpgroup coordinates (compute warps only).
+  const bool is_wg = warp >= kDecWgWarp0;
+  const int g = is_wg ? (warp - kDecWgWarp0) >> 2 : 0;
+  const int q = warp & 3;                                   // tensor-memory quarter
+  const int tid_wg = tid - 32 * kDecWgWarp0 - 128 * g;
+  const bool leader = is_wg && tid_wg == 0;
+  const int nj = (is_wg && n_chunks > g) ? (n_chunks - g + kDecWG - 1) / kDecWG : 0;   // this warpgroup's chunks
+  uint8_t* my_stages = stages + static_cast<size_t>(g) * NS * cbytes;
+  int issued = 0;                                           // chunks whose copy the leader has issued
+
+  auto issue_chunk = [&](int j) {                           // leader only
+    const int ci = c_begin + g + kDecWG * j;
+    const int tile0 = ci * kChunkTiles;
+    const int nt = min(kChunkTiles, n_tiles - tile0);
+    const int s = j % NS;
+    uint8_t* dst = my_stages + static_cast<size_t>(s) * cbytes;
+    uint32_t bytes = static_cast<uint32_t>(nt * a.rec_bytes);
+    int rows = 0;
+    if constexpr (kDense) {
+      rows = min(kChunkTokens, a.seq_len - ci * kChunkTokens);
+      bytes += static_cast<uint32_t>(rows) * (2 * kD);
     }
-  } else {
-    // ---------------------------------------------------------------- setup (warps 0..16)
-    // The compute warps start on the first chunk as soon as the tables and the allocation
-    // record (which carries the K group plan) are in; the MMA warp meanwhile builds Q'.
-    if (warp == kDecMmaWarp) tc::tmem_alloc(&S.tmem_base, kTmemCols);
-    tc::fence_before_sync();
-    named_sync(5, kSetupThreads);
-    tc::fence_after_sync();
-    const uint32_t tbase = S.tmem_base;
-    if (!tc::mbar_wait(&S.setup, 0, kWaitLimit)) record_timeout(status);
-    const kvq_head_alloc& A = *reinterpret_cast<const kvq_head_alloc*>(sm + kAllocOff);
+    tc::mbar_arrive_expect_tx(&S.full[g][s], bytes);
+    tc::bulk_g2s(dst, src + static_cast<size_t>(tile0) * a.rec_bytes, static_cast<uint32_t>(nt * a.rec_bytes),
+                 &S.full[g][s]);
+    if constexpr (kDense) {
+      const uint8_t* vsrc = static_cast<const uint8_t*>(a.v_dense) +
+                            2 * (b * a.vsb + hkv * a.vsh + static_cast<int64_t>(ci) * kChunkTokens * a.vst);
+      uint8_t* vdst = dst + kChunkTiles * a.rec_bytes;
+      if (a.vst == kD) {
+        tc::bulk_g2s(vdst, vsrc, static_cast<uint32_t>(rows) * (2 * kD), &S.full[g][s]);
+      } else {
+        for (int r = 0; r < rows; ++r)
+          tc::bulk_g2s(vdst + r * (2 * kD), vsrc + 2 * static_cast<int64_t>(r) * a.vst, 2 * kD, &S.full[g][s]);
+      }
+    }
+  };
 
-    if (warp == kDecMmaWarp || warp == kDecMma2Warp) {
-      const int par = (warp == kDecMmaWarp) ? 0 : 1;   // chunk parity this warp issues for
-      const int k_cols = 4 * kSlotCols;
-      if (par == 0) {
-      // -------------------------------------------------------------- Q' (whole warp)
-      // Row h: q_h * f_b * log2(e) / sqrt(d), scaled by 2^-e so that its largest |value| is in
-      // [0.5, 1); qscale[h] = 2^e multiplies the product back. B operand of S, K-major, no
-      // swizzle: element (n, k) at (k/8)*256 + (n/8)*128 + (n%8)*16 + (k%8)*2; K element
-      // k = 2c + r is dim b + 64 r of the block in column c; n < 8: hi part of row n, n >= 8:
-      // lo part of row n - 8.
-      float* qtmp = reinterpret_cast<float*>(sm + kBPOff);   // [8][128] fp32 until P' is first written
-      float qv[8][4];
+  // First copies go out before anything else, so HBM is busy from the start.
+  if (leader && !a.debug_no_loads) {
+    for (; issued < min(NS, nj); ++issued) issue_chunk(issued);
+  }
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(&S.setup, kLutBytes + static_cast<uint32_t>(sizeof(kvq_head_alloc)));
+    tc::bulk_g2s(sm, g_dec_lut, kLutBytes, &S.setup);
+    tc::bulk_g2s(sm + kAllocOff, al, sizeof(kvq_head_alloc), &S.setup);
+  }
+  if (tid == 32) {
+    // The packed header must name this layout, these widths and shapes, and this head's
+    // allocation; a status left by an append is reported as is.
+    const kvq_packed_header* H = reinterpret_cast<const kvq_packed_header*>(a.packed);
+    const uint64_t* dig = reinterpret_cast<const uint64_t*>(a.packed + sizeof(kvq_packed_header));
+    unsigned code = 0;
+    if (H->status != 0) code = H->status;
+    else if (H->magic != kHeaderMagic || H->layout_version != kLayoutVersion || H->head_dim != kD ||
+             H->bits_k != a.bits_k || H->bits_v != a.bits_v || H->batch != a.batch ||
+             H->n_kv_heads != a.n_kv_heads || H->capacity != a.capacity ||
+             static_cast<int>(H->record_bytes) != a.rec_bytes || dig[hkv] != al->digest ||
+             al->bits_k != a.bits_k || al->k_words != a.bits_k * kD || al->plan_k_cols > 96 ||
+             al->plan_k_cols < 8 || al->plan_n_slots > kPlanSlots)
+      code = KVQ_ERR_MISMATCH;
+    if (code) {
+      S.bad = 1;
+      record_status(a.status, code);
+    }
+  }
+  if (!tc::mbar_wait(&S.setup, 0, WL)) {
+    S.bad = 1;
+    record_status(a.status, KVQ_ERR_TIMEOUT);
+  }
+  __syncthreads();
+  const bool bad = S.bad != 0;
+  const kvq_head_alloc& A = *reinterpret_cast<const kvq_head_alloc*>(sm + kAllocOff);
+
+  float M[8], L[8];                                         // running max (log2) and row sums
 #pragma unroll
-      for (int hg = 0; hg < 8; ++hg)
+  for (int h = 0; h < 8; ++h) { M[h] = -INFINITY; L[h] = 0.0f; }
+  int done = 0;                                             // chunks this warpgroup completed
+  bool s_pending = false, o_pending = false;                // committed products not waited for yet
+
+  if (!bad && warp >= 1 && warp <= 3) {
+    // ------------------------------------------------------------------ Q' (warps 1..3)
+    // Row h: q_h * f_b * log2(e) / sqrt(d), scaled by 2^-e so its largest |value| is in
+    // [0.5, 1); qscale[h] = 2^e multiplies the product back. B operand of S, K-major, no
+    // swizzle: element (n, k) at (k/8)*256 + (n/8)*128 + (n%8)*16 + (k%8)*2; K element k = 2c + r
+    // is dim b + 64 r of the block in column c; n < 8: hi part of row n, n >= 8: lo part.
+    float* qtmp = reinterpret_cast<float*>(sm + kBPOff);    // [8][128] fp32 until P' is first written
+    for (int h = warp - 1; h < 8; h += 3) {
+      float qv[4], mx = 0.0f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          qv[hg][u] = (hg < G) ? Elem<DT>::to_f32(q[b * qsb + (hkv * G + hg) * qsh + lane + 32 * u]) : 0.0f;
+      for (int u = 0; u < 4; ++u) {
+        const int j = lane + 32 * u;
+        qv[u] = (h < G) ? load_f32(a.q, a.q_dtype, b * a.qsb + (hkv * G + h) * a.qsh + j) : 0.0f;
+        qv[u] *= A.dequant[j % kH] * (inv_sqrt_d * kLog2e);
+        mx = fmaxf(mx, fabsf(qv[u]));
+      }
 #pragma unroll
-      for (int hg = 0; hg < 8; ++hg) {
-        float mx = 0.0f;
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      int e = 0;
+      if (mx > 0.0f) frexpf(mx, &e);
+      if (lane == 0) S.qscale[h] = ldexpf(1.0f, e);
+      const float sc = ldexpf(1.0f, -e);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) qtmp[h * kD + lane + 32 * u] = qv[u] * sc;
+    }
+    named_sync(kDecWG + 1, 96);
+    const int k_elems = 2 * A.plan_k_cols;
+    for (int i = tid - 32; i < 8 * k_elems; i += 96) {
+      const int n = i / k_elems, k = i - n * k_elems;
+      const int blk = A.plan_col_block[k >> 1];
+      __half hi = __float2half_rn(0.0f), lo = hi;
+      if (blk >= 0) split_hilo(qtmp[n * kD + blk + kH * (k & 1)], hi, lo);
+      const int base = (k >> 3) * 256 + (k & 7) * 2;
+      *reinterpret_cast<__half*>(sm + kBQOff + base + n * 16) = hi;
+      *reinterpret_cast<__half*>(sm + kBQOff + base + 128 + n * 16) = lo;
+    }
+    tc::fence_proxy_async_smem();
+    named_sync(kDecWG + 1, 96);
+    if (tid == 32) tc::mbar_arrive(&S.qready);
+    // ---------------------------------------------------------------- recent tokens (CUDA cores)
+    // This CTA's even share of the row's recent tokens. Lane l owns dims l, l + 32, l + 64,
+    // l + 96; warp w walks every third token with its own online softmax over
+    // s = q . k * log2(e) / sqrt(d); the three warps then meet at a common maximum and add
+    // their O shares into rec_o in a fixed order.
+    const int r_begin = static_cast<int>((static_cast<long long>(split) * a.n_recent) / a.splits);
+    const int r_end = static_cast<int>((static_cast<long long>(split + 1) * a.n_recent) / a.splits);
+    if (r_end > r_begin) {
+      const int w = warp - 1;
+      float* rq = reinterpret_cast<float*>(sm + kRecQOff);
+      for (int i = tid - 32; i < 8 * kD; i += 96) {
+        const int h = i >> 7, j = i & (kD - 1);
+        rq[i] = (h < G) ? load_f32(a.q, a.q_dtype, b * a.qsb + (hkv * G + h) * a.qsh + j) * (inv_sqrt_d * kLog2e) : 0.0f;
+      }
+      named_sync(kDecWG + 1, 96);
+      float o[8][4];
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) o[h][u] = 0.0f;
+      for (int r = r_begin + w; r < r_end; r += 3) {
+        float kv[4], vv[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int j = lane + 32 * u;
-          qv[hg][u] *= A.dequant[j % kH] * (inv_sqrt_d * kLog2e);
-          mx = fmaxf(mx, fabsf(qv[hg][u]));
+          kv[u] = load_f32(a.k_rec, a.kr_dtype, b * a.krsb + hkv * a.krsh + r * a.krst + lane + 32 * u);
+          vv[u] = load_f32(a.v_rec, a.vr_dtype, b * a.vrsb + hkv * a.vrsh + r * a.vrst + lane + 32 * u);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        int e = 0;
-        if (mx > 0.0f) frexpf(mx, &e);
-        if (lane == 0) S.qscale[hg] = ldexpf(1.0f, e);
-        const float sc = ldexpf(1.0f, -e);
+        for (int h = 0; h < 8; ++h) {
+          const float* qh = rq + h * kD + lane;
+          float sdot = qh[0] * kv[0] + qh[32] * kv[1] + qh[64] * kv[2] + qh[96] * kv[3];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) qtmp[hg * kD + lane + 32 * u] = qv[hg][u] * sc;
+          for (int off = 16; off > 0; off >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, off);
+          const float mn = fmaxf(M[h], sdot);
+          const float alpha = (M[h] == -INFINITY) ? 0.0f : fast_exp2(M[h] - mn);
+          const float p = fast_exp2(sdot - mn);
+          M[h] = mn;
+          L[h] = L[h] * alpha + p;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) o[h][u] = o[h][u] * alpha + p * vv[u];
+        }
       }
-      __syncwarp();
-      const int k_elems = 2 * k_cols;
-      for (int i = lane; i < 8 * k_elems; i += 32) {
-        const int n = i / k_elems, k = i - n * k_elems;
-        const int blk = A.plan_col_block[k >> 1];
-        __half hi = __float2half_rn(0.0f), lo = hi;
-        if (blk >= 0) split_hilo(qtmp[n * kD + blk + kH * (k & 1)], hi, lo);
-        const int base = (k >> 3) * 256 + (k & 7) * 2;
-        *reinterpret_cast<__half*>(sm + kBQOff + base + n * 16) = hi;
-        *reinterpret_cast<__half*>(sm + kBQOff + base + 128 + n * 16) = lo;
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < 8; ++h) { S.rx_m[w][h] = M[h]; S.rx_l[w][h] = L[h]; }
+      }
+      named_sync(kDecWG + 1, 96);
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const float Mx = fmaxf(fmaxf(S.rx_m[0][h], S.rx_m[1][h]), S.rx_m[2][h]);
+        const float wt = (M[h] == -INFINITY) ? 0.0f : fast_exp2(M[h] - Mx);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) o[h][u] *= wt;
+        if (w == 0 && lane == 0) {
+          float lsum = 0.0f;
+#pragma unroll
+          for (int ww = 0; ww < 3; ++ww)
+            lsum += (S.rx_m[ww][h] == -INFINITY) ? 0.0f : S.rx_l[ww][h] * fast_exp2(S.rx_m[ww][h] - Mx);
+          S.wg_m[kDecWG][h] = Mx;
+          S.wg_l[kDecWG][h] = lsum;
+        }
+      }
+      for (int ww = 0; ww < 3; ++ww) {
+        if (w == ww) {
+#pragma unroll
+          for (int h = 0; h < 8; ++h)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              float* dst = rec_o + h * kD + lane + 32 * u;
+              *dst = (ww == 0) ? o[h][u] : *dst + o[h][u];
+            }
+        }
+        named_sync(kDecWG + 1, 96);
+      }
+#pragma unroll
+      for (int h = 0; h < 8; ++h) { M[h] = -INFINITY; L[h] = 0.0f; }
+    }
+  } else if (!bad && is_wg) {
+    // ------------------------------------------------------------------ chunk pipeline
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
+    const uint32_t tA = tbase + col_a(g), tS = tbase + col_s(g), tO = tbase + col_o(g);
+    const int n_batches = (min(A.plan_n_slots, kPlanSlots) + 3) >> 2;
+    const int k_steps = A.plan_k_cols >> 3;
+    uint8_t* pbuf = sm + kBPOff + g * kBPBytes;
+    const uint32_t id_s = tc::idesc_f16(128, 16, false), id_o = tc::idesc_f16(128, 16, true, kBfO);
+    const uint32_t bq = tc::smem_u32(sm + kBQOff), bp = tc::smem_u32(pbuf);
+    float qs[8];
+    bool have_q = false;
+    volatile int* abort_flag = &S.wg_abort[g];
+
+    for (int j = 0; j < nj; ++j) {
+      const int ci = c_begin + g + kDecWG * j;
+      const int s = j % NS;
+      const uint8_t* st = my_stages + static_cast<size_t>(s) * cbytes;
+      bool ok = tc::mbar_wait(&S.full[g][s], (j / NS) & 1, WL);
+      if (ok && j > 0) ok = tc::mbar_wait(&S.ofull[g], (j - 1) & 1, WL);
+      if (!ok) *abort_flag = 1;
+      tc::fence_after_sync();
+      // -------------------------------------------------------------- keys (lane = token)
+      const uint8_t* tq = st + q * a.rec_bytes;                       // tile q of the chunk
+      {
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(tq) + lane;
+        const uint32_t* slots = A.plan_slot;
+        for (int bt = 0; bt < n_batches; ++bt) {
+          uint32_t t[4][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) k_slot(slots[4 * bt + i], kw, sm, lane4, t[i]);
+          uint32_t v16[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v16[i] = t[i >> 2][i & 3];
+          tc::tmem_st<16>(tA + lane_base + 16 * bt, v16);
+        }
+      }
+      const float kn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(tq + kbytes)[lane]));
+      float vn = 1.0f;
+      if constexpr (!kDense) vn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(tq + kbytes + 2 * kTile)[lane]));
+      const int tok0 = ci * kChunkTokens;
+      const bool valid = tok0 + 32 * q + lane < a.seq_len;
+      tc::wait_st();
+      tc::fence_before_sync();
+      named_sync(1 + g, 128);
+      if (*abort_flag) break;
+      if (leader) {
+        tc::fence_after_sync();
+        bool qok = true;
+        if (j == 0) qok = tc::mbar_wait(&S.qready, 0, WL);
+        if (qok) {
+          for (int ks = 0; ks < k_steps; ++ks)
+            tc::mma_ts(tS, tA + 8 * ks, tc::sdesc(bq + 512 * ks, 256, 128), id_s, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&S.sfull[g]);                          // arrives even with nothing issued
+        if (!qok) *abort_flag = 1;
+      }
+      s_pending = true;
+      if (!have_q) {
+        if (!tc::mbar_wait(&S.qready, 0, WL)) *abort_flag = 1;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) qs[h] = S.qscale[h];
+        have_q = true;
+      }
+      if (!tc::mbar_wait(&S.sfull[g], j & 1, WL)) *abort_flag = 1;
+      else s_pending = false;
+      tc::fence_after_sync();
+      // -------------------------------------------------------------- logits
+      float sv[8];
+      {
+        uint32_t sr[16];
+        tc::tmem_ld<16>(tS + lane_base, sr);
+        tc::wait_ld();
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          const float x = (__uint_as_float(sr[h]) + __uint_as_float(sr[8 + h])) * (kn * qs[h]);
+          sv[h] = valid ? x : -INFINITY;
+        }
+      }
+      // -------------------------------------------------------------- values (lane = dim)
+      if constexpr (kDense) {
+        // dense rows [token][128] of 16-bit values after the chunk's records; rows past the
+        // sequence end are not copied and read as 0
+        const uint16_t* vr = reinterpret_cast<const uint16_t*>(st + kChunkTiles * a.rec_bytes) + 32 * q + lane;
+        const int nrows = a.seq_len - tok0;
+#pragma unroll
+        for (int u = 0; u < kChunkTiles; ++u) {
+          uint32_t v[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int t0 = 32 * u + 2 * c;
+            const uint32_t lo = (t0 < nrows) ? vr[t0 * kD] : 0u;
+            const uint32_t hi = (t0 + 1 < nrows) ? vr[(t0 + 1) * kD] : 0u;
+            v[c] = lo | (hi << 16);
+          }
+          tc::tmem_st<16>(tA + lane_base + 16 * u, v);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < kChunkTiles; ++u) {
+          const uint32_t* vw = reinterpret_cast<const uint32_t*>(st + u * a.rec_bytes + kbytes + 4 * kTile) + 32 * q + lane;
+          v_tile<VM>(vw, tA + lane_base + 16 * u, sm, lane4);
+        }
+      }
+      // -------------------------------------------------------------- chunk maximum
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const int m = __reduce_max_sync(0xffffffffu, ordered(sv[h]));
+        if (lane == 0) S.xch[g][q][h] = from_ordered(m);
+      }
+      named_sync(1 + g, 128);
+      if (*abort_flag) break;
+      bool resc = false;
+      float cm[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        cm[h] = fmaxf(fmaxf(S.xch[g][0][h], S.xch[g][1][h]), fmaxf(S.xch[g][2][h], S.xch[g][3][h]));
+        resc |= cm[h] > M[h] + static_cast<float>(kTau);
+      }
+      if (resc) {
+        float alpha[8];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          const float mn = fmaxf(M[h], cm[h]);
+          alpha[h] = (M[h] == -INFINITY) ? 0.0f : fast_exp2(M[h] - mn);
+          M[h] = mn;
+          L[h] *= alpha[h];
+        }
+        if (j > 0) {                                  // O holds earlier chunks: rescale it (lane = dim)
+          uint32_t o[16];
+          tc::tmem_ld<16>(tO + lane_base, o);
+          tc::wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha[c & 7]);
+          tc::tmem_st<16>(tO + lane_base, o);
+        }
+      }
+      // -------------------------------------------------------------- P' (lane = token)
+      {
+        // packed values: P' = p * value norm / sqrt(d) (v-hat = norm * c / sqrt(d)); dense: p
+        const float vs = valid ? (kDense ? 1.0f : vn * inv_sqrt_d) / static_cast<float>(1 << kTau) : 0.0f;
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int h = 0; h < 8; h += 2) {
+          const float p0 = valid ? fast_exp2(sv[h] - M[h]) : 0.0f;
+          const float p1 = valid ? fast_exp2(sv[h + 1] - M[h + 1]) : 0.0f;
+          L[h] += p0;
+          L[h + 1] += p1;
+          uint32_t h0, l0, h1, l1;
+          split16<kBfO>(p0 * vs, h0, l0);
+          split16<kBfO>(p1 * vs, h1, l1);
+          hi[h >> 1] = h0 | (h1 << 16);
+          lo[h >> 1] = l0 | (l1 << 16);
+        }
+        const int t = 32 * q + lane;
+        uint8_t* pb = pbuf + (t >> 3) * 256 + (t & 7) * 16;
+        *reinterpret_cast<uint4*>(pb) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(pb + 128) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&S.qready);
-      }
-      // -------------------------------------------------------------- MMA issue
-      // Two issuing threads, one per chunk parity: independent MMA chains overlap in the
-      // tensor pipe, whose cost per instruction is mostly latency at these small tiles.
-      if (lane == 0) {
-        if (par == 1 && !tc::mbar_wait(&S.qready, 0, kWaitLimit)) record_timeout(status);
-        const uint32_t id_s = tc::idesc_f16(128, 16, false), id_o = tc::idesc_f16(128, 16, true);
-        const uint32_t bq = tc::smem_u32(sm + kBQOff), bp = tc::smem_u32(sm + kBPOff);
-        // k-steps (8 columns each) that hold at least one real block pair
-        uint32_t kmask = 0u;
-        for (int c = 0; c < k_cols; ++c)
-          if (A.plan_col_block[c] >= 0) kmask |= 1u << (c >> 3);
-        const int first_ks = __ffs(kmask) - 1;
-        // Every k-step's B descriptor, built once (the 14-bit start field wraps, so offsets are
-        // not added to a built descriptor).
-        uint64_t dq[12], dpv[2][kChunkTokens / 16];
-#pragma unroll
-        for (int ks = 0; ks < 12; ++ks) dq[ks] = tc::sdesc(bq + 512 * ks, 256, 128);
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb)
-#pragma unroll
-          for (int ks = 0; ks < kChunkTokens / 16; ++ks)
-            dpv[bb][ks] = (bb == par) ? tc::sdesc(bp + kBPBytes * bb + 512 * ks, 256, 128) : 0ull;
-        int kc = 0, vc = 0;
-        bool ok = true;
-        for (int sg = 0; sg < n_segs && ok; ++sg) {
-          const int nu = min(kSegChunks, n_chunks - sg * kSegChunks);
-          for (int u = 0; u < nu; ++u, ++kc) {
-            if ((kc & 1) != par) continue;
-            const int bb = kc % 3;
-            if (!tc::mbar_wait(&S.kready[bb], (kc / 3) & 1, kWaitLimit)) { ok = false; break; }
-            tc::fence_after_sync();
-            const uint32_t d = tbase + col_s(bb), a = tbase + col_ak(bb);
-#pragma unroll
-            for (int ks = 0; ks < 12; ++ks)
-              if (kmask & (1u << ks)) tc::mma_ts(d, a + 8 * ks, dq[ks], id_s, ks != first_ks);
-            tc::mma_commit(&S.sfull[bb]);
-          }
-          for (int u = 0; u < nu && ok; ++u, ++vc) {
-            if ((vc & 1) != par) continue;
-            const int bb = vc & 1;
-            if (!tc::mbar_wait(&S.vpready[bb], (vc >> 1) & 1, kWaitLimit)) { ok = false; break; }
-            tc::fence_after_sync();
-            const uint32_t a = tbase + col_av(bb), d = tbase + col_o(bb);
-            tc::mma_ts(d, a, dpv[par][0], id_o, u >= 2);   // first chunk of this parity starts O
-#pragma unroll
-            for (int ks = 1; ks < kChunkTokens / 16; ++ks) tc::mma_ts(d, a + 8 * ks, dpv[par][ks], id_o, 1u);
-            tc::mma_commit(&S.ofull[bb]);
-          }
-        }
-        if (!ok) record_timeout(status);
-      }
-    } else {
-      // -------------------------------------------------------------- compute warps
-      const int wg = warp >> 2, qt = warp & 3;                // warp group, tensor-memory quarter
-      const uint32_t lane_base = static_cast<uint32_t>(32 * qt) << 16;
-      const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
-      const int t_lane = 32 * qt + lane;                      // token of a chunk (pass 1), dim (pass 2)
-      // This warp group's K slots: slot i = plan entry i, as width | bit offset << 8 (0 = empty).
-      uint32_t slot_e[kSlots];
-      {
-        uint32_t mine = 0u;
-        const int n_runs = min(max(A.plan_n_runs[wg], 0), kMaxRuns);
-        if (lane < kSlots)
-          for (int r = 0; r < n_runs; ++r) {
-            const uint32_t e = A.plan_run[wg][r];
-            const int first = (e >> 8) & 0xff, n = (e >> 16) & 0xff;
-            if (lane >= first && lane < first + n) mine = (e & 15u) | ((A.plan_group[wg][lane] & 0xffffu) << 8);
-          }
-#pragma unroll
-        for (int i = 0; i < kSlots; ++i) slot_e[i] = __shfl_sync(0xffffffffu, mine, i);
-      }
-      float qs0 = 1.0f, qs1 = 1.0f;
-      bool have_q = false;
-      float* stash = reinterpret_cast<float*>(sm + kStashOff);
-      // Zero both K buffers once: columns past the last group stay zero (their Q' is 0 too).
-      {
-        uint32_t z[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0u;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tc::tmem_st<16>(tbase + lane_base + 64 * wg + 16 * i, z);
-      }
-      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f, o0 = 0.0f, o1 = 0.0f;
-      int k = 0, kc0 = 0, vc0 = 0;
-      bool ok = true;
-
-      // Logits of chunk u of the segment (K count j): s = S * knorm * qscale, -inf past the end.
-      auto logits = [&](int u0, int u, int j, float kn, float& sm0, float& sm1) {
-        const int bj = j % 3;
-        if (!have_q) {   // Q' scaling of this warp group's rows (written by the MMA warp)
-          if (ok && !tc::mbar_wait(&S.qready, 0, kWaitLimit)) ok = false;
-          qs0 = S.qscale[2 * wg];
-          qs1 = S.qscale[2 * wg + 1];
-          have_q = true;
-        }
-        if (ok && !tc::mbar_wait(&S.sfull[bj], (j / 3) & 1, kWaitLimit)) ok = false;
+      tc::wait_st();
+      tc::fence_before_sync();
+      named_sync(1 + g, 128);
+      if (leader) {
         tc::fence_after_sync();
-        uint32_t sh[2], sl[2];
-        tc::tmem_ld2x2_wait(tbase + lane_base + col_s(bj) + 2 * wg, tbase + lane_base + col_s(bj) + 8 + 2 * wg, sh, sl);
-        const int tile = (c_begin + u0 + u) * kChunkTiles + qt;
-        const bool valid = tile < tile_end && tile * kTile + lane < seq_len;
-        float s0 = (__uint_as_float(sh[0]) + __uint_as_float(sl[0])) * (kn * qs0);
-        float s1 = (__uint_as_float(sh[1]) + __uint_as_float(sl[1])) * (kn * qs1);
-        if (!valid) { s0 = -INFINITY; s1 = -INFINITY; }
-        stash[(u * 8 + 2 * wg) * kChunkTokens + t_lane] = s0;
-        stash[(u * 8 + 2 * wg + 1) * kChunkTokens + t_lane] = s1;
-        sm0 = fmaxf(sm0, s0);
-        sm1 = fmaxf(sm1, s1);
-      };
+#pragma unroll
+        for (int ks = 0; ks < kChunkTokens / 16; ++ks)
+          tc::mma_ts(tO, tA + 8 * ks, tc::sdesc(bp + 512 * ks, 256, 128), id_o, (j > 0 || ks > 0) ? 1u : 0u);
+        tc::mma_commit(&S.ofull[g]);
+        // the stage is consumed (keys, values and norms): refill it with a later chunk
+        if (issued < nj && !a.debug_no_loads) issue_chunk(issued++);
+      }
+      o_pending = true;
+      done = j + 1;
+    }
+    // ------------------------------------------------------------------ warpgroup result
+    if (o_pending && !*abort_flag) {
+      if (tc::mbar_wait(&S.ofull[g], (done - 1) & 1, WL)) o_pending = false;
+      else *abort_flag = 1;
+    }
+    named_sync(1 + g, 128);
+    tc::fence_after_sync();
+    if (!*abort_flag) {
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        float l = L[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) S.lred[g][q][h] = l;
+      }
+    }
+  }
+  // In-flight work of a warpgroup that stopped early: its leader waits (bounded) for the
+  // products it committed and the copies it issued, so nothing lands after the CTA is gone.
+  if (leader && (bad || S.wg_abort[g])) {
+    if (s_pending) tc::mbar_wait(&S.sfull[g], done & 1, WL);
+    if (o_pending) tc::mbar_wait(&S.ofull[g], (done - 1) & 1, WL);
+    for (int j = done; j < issued; ++j) tc::mbar_wait(&S.full[g][j % NS], (j / NS) & 1, WL);
+  }
+  __syncthreads();
+  bool aborted = bad;
+#pragma unroll
+  for (int gg = 0; gg < kDecWG; ++gg) aborted |= S.wg_abort[gg] != 0;
+  if (aborted && !bad && tid == 0) record_status(a.status, KVQ_ERR_TIMEOUT);
 
-      for (int sg = 0; sg < n_segs; ++sg) {
-        const int u0 = sg * kSegChunks, nu = min(kSegChunks, n_chunks - u0);
-        // ------------------------------------------------------------ pass 1: keys
-        float sm0 = -INFINITY, sm1 = -INFINITY, kn1 = 0.0f, kn2 = 0.0f;   // norms of chunks u-1, u-2
-        for (int u = 0; u < nu; ++u, ++k) {
-          const int s = k % n_stages, j = kc0 + u;
-          if (ok && !tc::mbar_wait(&S.full[s], (k / n_stages) & 1, kWaitLimit)) ok = false;
-          const uint8_t* st = stages + s * stage_bytes + qt * tstride;   // tile qt: token `lane`
-          const uint32_t* kw = reinterpret_cast<const uint32_t*>(st) + lane;
-          const uint32_t ta = tbase + lane_base + col_ak(j % 3) + kSlotCols * wg;
-          {
-            uint32_t t[kSlots][kGroupPairs];
+  // ------------------------------------------------------------------ CTA result
+  // Warpgroup partials (m, l, O) combined in shared memory (the stage area is free now).
+  float* comb = reinterpret_cast<float*>(stages);           // [kDecWG][8][128] O, unscaled
+  if (!aborted && is_wg) {
+    const int d = 32 * q + lane;
+    if (nj > 0) {
+      uint32_t o[16];
+      tc::tmem_ld<16>(tbase + col_o(g) + (static_cast<uint32_t>(32 * q) << 16), o);
+      tc::wait_ld();
 #pragma unroll
-            for (int i = 0; i < kSlots; ++i) k_slot(slot_e[i], kw, sm, lane4, t[i]);
-            uint32_t v16[16], v8[8];
+      for (int h = 0; h < 8; ++h)
+        comb[(g * 8 + h) * kD + d] = (__uint_as_float(o[h]) + __uint_as_float(o[8 + h])) * static_cast<float>(1 << kTau);
+    }
+    if (tid_wg < 8) {
+      const int h = tid_wg;
+      float mh = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v16[i] = t[i / 4][i % 4];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v8[i] = t[4 + i / 4][i % 4];
-            tc::tmem_st<16>(ta, v16);
-            tc::tmem_st<8>(ta + 16, v8);
-          }
-          const float kn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + 4 * kD * bits_k)[lane]));
-          tc::wait_st();
-          tc::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) {
-            tc::mbar_arrive(&S.kready[j % 3]);
-            tc::mbar_arrive(&S.empty[s]);
-          }
-          if (u >= 2) logits(u0, u - 2, j - 2, kn2, sm0, sm1);
-          kn2 = kn1;
-          kn1 = kn;
-        }
-        if (nu >= 2) logits(u0, nu - 2, kc0 + nu - 2, kn2, sm0, sm1);
-        logits(u0, nu - 1, kc0 + nu - 1, kn1, sm0, sm1);
-        kc0 += nu;
-        // ------------------------------------------------------------ segment maximum
-        {
-          const int k0 = __reduce_max_sync(0xffffffffu, ordered(sm0));
-          const int k1 = __reduce_max_sync(0xffffffffu, ordered(sm1));
-          if (lane == 0) {
-            S.xmax[sg & 1][wg][qt][0] = from_ordered(k0);
-            S.xmax[sg & 1][wg][qt][1] = from_ordered(k1);
-          }
-          named_sync(1 + wg, 128);
-          float c0 = S.xmax[sg & 1][wg][0][0], c1 = S.xmax[sg & 1][wg][0][1];
-#pragma unroll
-          for (int v = 1; v < 4; ++v) {
-            c0 = fmaxf(c0, S.xmax[sg & 1][wg][v][0]);
-            c1 = fmaxf(c1, S.xmax[sg & 1][wg][v][1]);
-          }
-          const float n0 = fmaxf(m0, c0), n1 = fmaxf(m1, c1);
-          const float a0 = (m0 == -INFINITY) ? 0.0f : fast_exp2(m0 - n0);
-          const float a1 = (m1 == -INFINITY) ? 0.0f : fast_exp2(m1 - n1);
-          m0 = n0;
-          m1 = n1;
-          l0 *= a0; l1 *= a1;
-          o0 *= a0; o1 *= a1;
-        }
-        // ------------------------------------------------------------ pass 2: values
-        for (int u = 0; u < nu; ++u, ++k) {
-          const int s = k % n_stages, j = vc0 + u, bj = j & 1;
-          if (ok && !tc::mbar_wait(&S.full[s], (k / n_stages) & 1, kWaitLimit)) ok = false;
-          if (j >= 2 && ok && !tc::mbar_wait(&S.ofull[bj], ((j - 2) >> 1) & 1, kWaitLimit)) ok = false;
-          const uint8_t* st = stages + s * stage_bytes;
-          // V-hat^T row: dim t_lane, tokens of tile wg -> columns 16 wg .. 16 wg + 15.
-          const uint32_t* vw = reinterpret_cast<const uint32_t*>(st + wg * tstride + 2 * kTile) + t_lane;
-          v_tile<BVT>(vw, tbase + lane_base + col_av(bj) + 16 * wg, sm, lane4);
-          // P' of token t_lane (tile qt, token lane), rows 2 wg, 2 wg + 1.
-          const float vn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + qt * tstride)[lane]));
-          const float s0 = stash[(u * 8 + 2 * wg) * kChunkTokens + t_lane];
-          const float s1 = stash[(u * 8 + 2 * wg + 1) * kChunkTokens + t_lane];
-          const bool valid = s0 != -INFINITY;
-          const float p0 = valid ? fast_exp2(s0 - m0) : 0.0f;
-          const float p1 = valid ? fast_exp2(s1 - m1) : 0.0f;
-          l0 += p0;
-          l1 += p1;
-          const float vs = valid ? vn * inv_sqrt_d : 0.0f;
-          __half h0, lo0, h1, lo1;
-          split_hilo(p0 * vs, h0, lo0);
-          split_hilo(p1 * vs, h1, lo1);
-          uint8_t* pb = sm + kBPOff + kBPBytes * bj + (t_lane >> 3) * 256 + (t_lane & 7) * 16 + 4 * wg;
-          *reinterpret_cast<uint32_t*>(pb) = pack_half2(h0, h1);
-          *reinterpret_cast<uint32_t*>(pb + 128) = pack_half2(lo0, lo1);
-          tc::wait_st();
-          tc::fence_proxy_async_smem();
-          tc::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) {
-            tc::mbar_arrive(&S.vpready[bj]);
-            tc::mbar_arrive(&S.empty[s]);
-          }
-        }
-        vc0 += nu;
-        // ------------------------------------------------------------ segment O
-        // One accumulator per chunk parity: wait for the last chunk of each, add both.
-        {
-          const int jl = vc0 - 1;
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int jq = jl - q;
-            if (q == 1 && nu < 2) break;
-            if (ok && !tc::mbar_wait(&S.ofull[jq & 1], (jq >> 1) & 1, kWaitLimit)) ok = false;
-            tc::fence_after_sync();
-            uint32_t oh[2], ol[2];
-            tc::tmem_ld2x2_wait(tbase + lane_base + col_o(jq & 1) + 2 * wg, tbase + lane_base + col_o(jq & 1) + 8 + 2 * wg,
-                                oh, ol);
-            o0 += __uint_as_float(oh[0]) + __uint_as_float(ol[0]);
-            o1 += __uint_as_float(oh[1]) + __uint_as_float(ol[1]);
-          }
-          tc::fence_before_sync();
-        }
-      }
-      if (!ok) record_timeout(status);
-
-      // -------------------------------------------------------------- CTA result
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-      }
-      if (lane == 0) {
-        S.lpart[wg][qt][0] = l0;
-        S.lpart[wg][qt][1] = l1;
-      }
-      named_sync(1 + wg, 128);
-      const float L0 = S.lpart[wg][0][0] + S.lpart[wg][1][0] + S.lpart[wg][2][0] + S.lpart[wg][3][0];
-      const float L1 = S.lpart[wg][0][1] + S.lpart[wg][1][1] + S.lpart[wg][2][1] + S.lpart[wg][3][1];
-      const int d = t_lane;
-      const int h0 = 2 * wg, h1 = 2 * wg + 1;
-      if (splits == 1) {
-        float* ob = out + (static_cast<size_t>(b) * n_q_heads + hkv * G) * kD;
-        if (h0 < G) ob[h0 * kD + d] = o0 / L0;
-        if (h1 < G) ob[h1 * kD + d] = o1 / L1;
-      } else {
-        const size_t pb0 = (static_cast<size_t>(bh) * (splits + n_groups) + split) * 8;
-        part_o[(pb0 + h0) * kD + d] = o0;
-        part_o[(pb0 + h1) * kD + d] = o1;
-        if (d == 0) {
-          part_m[pb0 + h0] = m0;
-          part_l[pb0 + h0] = L0;
-          part_m[pb0 + h1] = m1;
-          part_l[pb0 + h1] = L1;
-        }
-      }
+      for (int r = 0; r < 8; ++r)
+        if (r == h) mh = M[r];                        // (a register array is never indexed at run time)
+      S.wg_m[g][h] = nj > 0 ? mh : -INFINITY;
+      S.wg_l[g][h] = nj > 0 ? (S.lred[g][0][h] + S.lred[g][1][h] + S.lred[g][2][h] + S.lred[g][3][h]) : 0.0f;
     }
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == kDecMmaWarp) tc::tmem_dealloc(S.tmem_base, kTmemCols);
-  if (splits == 1) return;
+  if (warp == 0) tc::tmem_dealloc(tbase, kTmemCols);
+  if (aborted) return;
 
-  // ------------------------------------------------------------------ cross-split merge
-  // The last CTA of this (sequence, KV head), found with an atomic ticket, merges all splits.
-  const int pitch = splits + n_groups;
-  float* out_bh = out + (static_cast<size_t>(b) * n_q_heads + hkv * G) * kD;
+  const int pitch = a.splits + a.n_groups;
+  float* out_bh = a.out + (static_cast<size_t>(b) * a.n_q_heads + hkv * G) * kD;
+  // combine the warpgroups and the recent share: m = max, l and O = sums weighted by 2^(m_g - m)
+  for (int i = tid; i < 8 * kD; i += blockDim.x) {
+    const int h = i >> 7, d = i & (kD - 1);
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int gg = 0; gg <= kDecWG; ++gg) Mx = fmaxf(Mx, S.wg_m[gg][h]);
+    float Ls = 0.0f, Os = 0.0f;
+#pragma unroll
+    for (int gg = 0; gg <= kDecWG; ++gg) {
+      if (S.wg_m[gg][h] == -INFINITY) continue;
+      const float w = fast_exp2(S.wg_m[gg][h] - Mx);
+      Ls += w * S.wg_l[gg][h];
+      Os += w * (gg < kDecWG ? comb[(gg * 8 + h) * kD + d] : rec_o[h * kD + d]);
+    }
+    if (a.splits == 1) {
+      if (h < G) out_bh[h * kD + d] = Os / Ls;
+    } else {
+      const size_t e = static_cast<size_t>(bh) * pitch + split;
+      a.part_o[(e * 8 + h) * kD + d] = Os;
+      if (d == 0) {
+        a.part_m[e * 8 + h] = Mx;
+        a.part_l[e * 8 + h] = Ls;
+      }
+    }
+  }
+  if (a.splits == 1) return;
+
+  // ------------------------------------------------------------------ two-level split merge
+  const int grp = split / a.group_size;
+  const int m0 = grp * a.group_size, m1 = min(a.splits, m0 + a.group_size);
+  unsigned* tk = a.tickets + static_cast<size_t>(bh) * (1 + a.n_groups);
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const unsigned t = atomicAdd(&tickets[bh], 1u);
-    S.last = (t == static_cast<unsigned>(splits - 1));
-    if (S.last) tickets[bh] = 0u;
+    const unsigned t = atomicAdd(&tk[1 + grp], 1u);
+    S.last = (t == static_cast<unsigned>(m1 - m0 - 1));
+    if (S.last) tk[1 + grp] = 0u;
   }
   __syncthreads();
   if (!S.last) return;
   __threadfence();
-  merge_partials(S, stages, bh, pitch, splits, part_m, part_l, part_o, out_bh, G);
+  if (a.n_groups == 1) {
+    merge_entries(S, a, bh, pitch, m0, m1 - m0, -1, out_bh, G);
+    return;
+  }
+  merge_entries(S, a, bh, pitch, m0, m1 - m0, a.splits + grp, out_bh, G);
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned t = atomicAdd(&tk[0], 1u);
+    S.last = (t == static_cast<unsigned>(a.n_groups - 1));
+    if (S.last) tk[0] = 0u;
+  }
+  __syncthreads();
+  if (!S.last) return;
+  __threadfence();
+  merge_entries(S, a, bh, pitch, a.splits, a.n_groups, -1, out_bh, G);
 }
 
 }  // namespace kvq

@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 
@@ -17,6 +19,15 @@ using namespace kvq;
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// Last CUDA error behind a KVQ_ERR_CUDA of this process (kvq_last_cuda_error).
+std::atomic<int> g_last_cuda_error{0};
+
+kvq_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error.store(static_cast<int>(e));
+  return KVQ_ERR_CUDA;
+}
+
 std::mutex g_upload_mu;
 bool g_uploaded[kMaxDevices] = {};
 
@@ -32,13 +43,13 @@ kvq_status ensure_tables() {
   std::memcpy(d.delta, t.delta, sizeof(d.delta));
   std::memcpy(d.nf4, t.nf4, sizeof(d.nf4));
   std::memcpy(d.nf4_mid, t.nf4_mid, sizeof(d.nf4_mid));
-  if (cudaMemcpyToSymbol(c_tab, &d, sizeof(d)) != cudaSuccess) return KVQ_ERR_CUDA;
+  { const cudaError_t e_ = cudaMemcpyToSymbol(c_tab, &d, sizeof(d)); if (e_ != cudaSuccess) return cuda_fail(e_); }
   static uint8_t lut[kLutBytes];
   decode_lut_image(t.centroid_f16, lut);
-  if (cudaMemcpyToSymbol(g_dec_lut, lut, sizeof(lut)) != cudaSuccess) return KVQ_ERR_CUDA;
+  { const cudaError_t e_ = cudaMemcpyToSymbol(g_dec_lut, lut, sizeof(lut)); if (e_ != cudaSuccess) return cuda_fail(e_); }
   static uint32_t qlut[2 * kLutEntries];
   if (!quant_lut_image(t.threshold, qlut)) return KVQ_ERR_UNSUPPORTED;
-  if (cudaMemcpyToSymbol(g_quant_lut, qlut, sizeof(qlut)) != cudaSuccess) return KVQ_ERR_CUDA;
+  { const cudaError_t e_ = cudaMemcpyToSymbol(g_quant_lut, qlut, sizeof(qlut)); if (e_ != cudaSuccess) return cuda_fail(e_); }
   g_uploaded[dev] = true;
   return KVQ_OK;
 }
@@ -70,32 +81,36 @@ kvq_status check_tensor(const void* ptr, const kvq_tensor4* t) {
 
 bool cache_ok(const kvq_cache_desc* c) {
   return c && c->batch >= 1 && c->n_kv_heads >= 1 && c->head_dim == kD && c->capacity >= 1 && c->bits_k >= 1 &&
-         c->bits_k <= 8 && c->bits_v >= 1 && c->bits_v <= 8;
+         c->bits_k <= 8 && c->bits_v >= 0 && c->bits_v <= 8;
 }
 
-size_t tile_record_bytes(int bits_k, int bits_v) { return 4ull * kD * (bits_k + bits_v) + 4ull * kTile; }
+// Record of 32 tokens: K words, K norms, then (unless keys only) V norms and V words.
+size_t tile_record_bytes(int bits_k, int bits_v) {
+  return bits_v == 0 ? 4ull * kD * bits_k + 2ull * kTile : 4ull * kD * (bits_k + bits_v) + 4ull * kTile;
+}
+
+// Packed header: 64 bytes of fields and one 64-bit digest per KV head, padded to 128 bytes.
+size_t header_bytes(int n_kv_heads) { return (64ull + 8ull * n_kv_heads + 127) / 128 * 128; }
 
 int n_tiles_of(int tokens) { return (tokens + kTile - 1) / kTile; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+int sm_count();
+
 // NF4 decode: about 8 waves of two 16-warp CTAs per SM, so the hardware's CTA scheduling
 // evens out the last wave, and at least one 32-token group per warp in every CTA.
 int nf4_splits(int bh, int n_groups) {
-  const int want = (16 * kTargetCtas + bh - 1) / bh;
-  return std::max(1, std::min(std::min(want, n_groups / kNf4DecWarps), kMaxMergeSplits));
-}
-
-int decode_splits(int bh, int n_tiles) {
-  const int want = (kTargetCtas + bh - 1) / bh;
-  return std::max(1, std::min(std::min(want, n_tiles), kMaxMergeSplits));
+  const int want = (16 * sm_count() + bh - 1) / bh;
+  return std::max(1, std::min(std::min(want, n_groups / kNf4DecWarps), kNf4MaxSplits));
 }
 
 // Block-GTQ decode: splits of whole 128-token chunks, about one CTA per SM in total.
+constexpr int kMaxGtqSplits = kMergeMax * kMergeMax;
 int gtq_splits(int bh, int n_tiles) {
   const int n_chunks = (n_tiles + kChunkTiles - 1) / kChunkTiles;
-  const int want = (kTargetCtas + bh - 1) / bh;
-  return std::max(1, std::min(std::min(want, n_chunks), kMaxMergeSplits));
+  const int want = (sm_count() + bh - 1) / bh;
+  return std::max(1, std::min(std::min(want, n_chunks), kMaxGtqSplits));
 }
 
 struct DecodeWs {
@@ -114,11 +129,19 @@ DecodeWs decode_ws_layout(int bh, int entries, int rows, int groups) {
   return w;
 }
 
-int merge_groups(int splits) { return (splits + kMergeGroup - 1) / kMergeGroup; }
+// Two-level merge of `splits` partials: groups of about sqrt(splits).
+struct MergePlan {
+  int group_size, n_groups;
+};
+MergePlan merge_plan(int splits) {
+  int gs = 1;
+  while (gs * gs < splits) ++gs;
+  return MergePlan{gs, (splits + gs - 1) / gs};
+}
 
 DecodeWs gtq_ws_layout(int bh, int splits) {
-  const int groups = merge_groups(splits);
-  return decode_ws_layout(bh, splits + groups, 8, groups);
+  const MergePlan mp = merge_plan(splits);
+  return decode_ws_layout(bh, splits + mp.n_groups, 8, mp.n_groups);
 }
 
 int sm_count() {
@@ -135,7 +158,7 @@ int sm_count() {
 
 kvq_status launch_status() {
   const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  return e == cudaSuccess ? KVQ_OK : cuda_fail(e);
 }
 
 Nf4Layout nf4_layout(int batch, int n_heads, int capacity) {
@@ -146,21 +169,35 @@ Nf4Layout nf4_layout(int batch, int n_heads, int capacity) {
   return L;
 }
 
-constexpr size_t kMaxSmem = 227 * 1024;
-
-// Deepest bulk-copy pipeline (1..4 stages of 4 tile halves) that fits in shared memory.
-int decode_stages(int bits_k, int bits_v) {
-  const size_t per = static_cast<size_t>(kChunkTiles) * stage_tile_stride(bits_k, bits_v);
-  const size_t room = kMaxSmem - decode_stage_off();
-  return static_cast<int>(std::max<size_t>(1, std::min<size_t>(kDecStagesMax, room / per)));
+// Opt-in shared memory per block of the current device (227 KB on a B200).
+size_t max_smem() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 227 * 1024;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cached[dev] = n > 0 ? n : 227 * 1024;
+  }
+  return static_cast<size_t>(cached[dev]);
 }
 
-size_t decode_smem_bytes(int bits_k, int bits_v) {
-  const size_t stage =
-      static_cast<size_t>(kChunkTiles) * stage_tile_stride(bits_k, bits_v) * decode_stages(bits_k, bits_v);
-  // the stage area also holds the merge scratch (4 KB)
-  return decode_stage_off() + std::max<size_t>(stage, 256 * sizeof(float4));
+// Chunk stages per warpgroup (1..4) that fit in shared memory; cbytes = bytes of one chunk stage.
+int decode_stages(int cbytes) {
+  const size_t per = static_cast<size_t>(kDecWG) * cbytes;
+  const size_t room = max_smem() - decode_stage_off();
+  return static_cast<int>(std::max<size_t>(1, std::min<size_t>(kStagesMax, room / per)));
 }
+
+size_t decode_smem_bytes(int cbytes) {
+  const size_t stage = static_cast<size_t>(kDecWG) * cbytes * decode_stages(cbytes);
+  // the stage area also holds the warpgroups' results at the end (kDecWG x 8 x 128 floats)
+  return decode_stage_off() + std::max<size_t>(stage, static_cast<size_t>(kDecWG) * 8 * kD * sizeof(float));
+}
+
+// Test hooks (kvq_debug_decode): bounded-wait limit and the no-copy switch of the next decodes.
+uint32_t g_wait_limit = 2000;
+int g_debug_no_loads = 0;
 
 }  // namespace
 
@@ -180,6 +217,7 @@ const char* kvq_status_string(int s) {
     case KVQ_ERR_CUDA: return "CUDA error";
     case KVQ_ERR_TIMEOUT: return "device wait timed out";
     case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_MISMATCH: return "packed cache does not match the descriptor or allocation";
     default: return "unknown status";
   }
 }
@@ -234,9 +272,12 @@ size_t kvq_calibrate_workspace_bytes(int batch, int n_kv_heads, int n_calib_toke
   return calib_ws_layout(batch, n_kv_heads, n_calib_tokens).total;
 }
 
+size_t kvq_packed_header_bytes(int n_kv_heads) { return n_kv_heads >= 1 ? header_bytes(n_kv_heads) : 0; }
+
 size_t kvq_packed_bytes(const kvq_cache_desc* c) {
   if (!cache_ok(c)) return 0;
-  return static_cast<size_t>(c->batch) * c->n_kv_heads * n_tiles_of(c->capacity) * tile_record_bytes(c->bits_k, c->bits_v);
+  return header_bytes(c->n_kv_heads) +
+         static_cast<size_t>(c->batch) * c->n_kv_heads * n_tiles_of(c->capacity) * tile_record_bytes(c->bits_k, c->bits_v);
 }
 
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* c, int n_q_heads) {
@@ -256,8 +297,8 @@ kvq_status kvq_workspace_status(const void* ws, void* stream, int* device_code) 
   if (!ws) return KVQ_ERR_WORKSPACE;
   unsigned int code = 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(&code, ws, sizeof(code), cudaMemcpyDeviceToHost, s) != cudaSuccess) return KVQ_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
+  { const cudaError_t e_ = cudaMemcpyAsync(&code, ws, sizeof(code), cudaMemcpyDeviceToHost, s); if (e_ != cudaSuccess) return cuda_fail(e_); }
+  { const cudaError_t e_ = cudaStreamSynchronize(s); if (e_ != cudaSuccess) return cuda_fail(e_); }
   if (device_code) *device_code = static_cast<int>(code);
   return code == 0 ? KVQ_OK : static_cast<kvq_status>(code);
 }
@@ -315,11 +356,14 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
                         const kvq_cache_desc* c, int t_begin, void* packed, void* stream) {
   kvq_status st;
   if ((st = check_tensor(K, kd)) != KVQ_OK) return st;
-  if ((st = check_tensor(V, vd)) != KVQ_OK) return st;
   if (!alloc || !packed || !aligned16(packed)) return KVQ_ERR_ARG;
   if (!cache_ok(c)) return KVQ_ERR_ARG;
-  if (vd->dtype != kd->dtype || vd->batch != kd->batch || vd->n_heads != kd->n_heads || vd->seq_len != kd->seq_len)
-    return KVQ_ERR_SHAPE;
+  const bool keys_only = c->bits_v == 0;
+  if (!keys_only) {
+    if ((st = check_tensor(V, vd)) != KVQ_OK) return st;
+    if (vd->dtype != kd->dtype || vd->batch != kd->batch || vd->n_heads != kd->n_heads || vd->seq_len != kd->seq_len)
+      return KVQ_ERR_SHAPE;
+  }
   if (kd->batch != c->batch || kd->n_heads != c->n_kv_heads) return KVQ_ERR_SHAPE;
   if (t_begin < 0 || static_cast<long long>(t_begin) + kd->seq_len > c->capacity) return KVQ_ERR_RANGE;
   if ((st = ensure_tables()) != KVQ_OK) return st;
@@ -332,13 +376,19 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
   const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
   const size_t smem = quant_smem_bytes(kd->dtype);
   const int qw = quant_warps(kd->dtype);
+  QHeader qh;
+  qh.mode = t_begin == 0 ? 1 : 2;
+  qh.batch = c->batch;
+  qh.capacity = c->capacity;
+  qh.hdr_bytes = static_cast<int>(header_bytes(c->n_kv_heads));
+  const int64_t vsb = keys_only ? 0 : vd->stride_b, vsh = keys_only ? 0 : vd->stride_h, vst = keys_only ? 0 : vd->stride_t;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Persistent grid: exactly the CTAs that are resident at once (registers and shared memory
   // both limit it), so every warp starts at launch and the tiles are spread evenly.
   // The shared-memory opt-in and the occupancy query are made once per device, dtype and value
   // width (they cost host time comparable to a small launch, e.g. a one-token append).
   static std::mutex occ_mu;
-  static int occ[kMaxDevices][24] = {};
+  static int occ[kMaxDevices][27] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
 #define KVQ_LAUNCH_QUANT(DT, TY, BV)                                                                              \
@@ -347,28 +397,29 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
     int per_sm = 0;                                                                                               \
     {                                                                                                             \
       std::lock_guard<std::mutex> lock(occ_mu);                                                                   \
-      if (occ[dev][DT * 8 + BV - 1] == 0) {                                                                       \
+      if (occ[dev][DT * 9 + BV] == 0) {                                                                           \
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=    \
             cudaSuccess)                                                                                          \
           return KVQ_ERR_CUDA;                                                                                    \
         int n = 0;                                                                                                \
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, qw * 32, smem) != cudaSuccess)                \
           return KVQ_ERR_CUDA;                                                                                    \
-        occ[dev][DT * 8 + BV - 1] = std::max(1, n);                                                               \
+        occ[dev][DT * 9 + BV] = std::max(1, n);                                                                   \
       }                                                                                                           \
-      per_sm = occ[dev][DT * 8 + BV - 1];                                                                         \
+      per_sm = occ[dev][DT * 9 + BV];                                                                             \
     }                                                                                                             \
     const long long want = (n_tasks + qw - 1) / qw;                                                             \
     const unsigned grid =                                                                                         \
         static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sm_count()) * std::max(1, per_sm))); \
     kern<<<grid, qw * 32, smem, s>>>(static_cast<const TY*>(K), kd->stride_b, kd->stride_h, kd->stride_t,         \
-                                     static_cast<const TY*>(V), vd->stride_b, vd->stride_h, vd->stride_t, t_begin, \
-                                     t_end, tile_lo, n_tiles, c->n_kv_heads, tiles_cap,                           \
-                                     static_cast<const kvq_head_alloc*>(alloc), c->bits_k, c->bits_v,             \
-                                     static_cast<uint8_t*>(packed), rec, static_cast<int>(n_tasks));              \
+                                     static_cast<const TY*>(V), vsb, vsh, vst, t_begin, t_end, tile_lo, n_tiles,  \
+                                     c->n_kv_heads, tiles_cap, static_cast<const kvq_head_alloc*>(alloc),         \
+                                     c->bits_k, c->bits_v, static_cast<uint8_t*>(packed), rec,                    \
+                                     static_cast<int>(n_tasks), qh);                                              \
   } while (0)
 #define KVQ_QUANT_BV(DT, TY)                                                                                      \
   switch (c->bits_v) {                                                                                            \
+    case 0: KVQ_LAUNCH_QUANT(DT, TY, 0); break;                                                                   \
     case 1: KVQ_LAUNCH_QUANT(DT, TY, 1); break;                                                                   \
     case 2: KVQ_LAUNCH_QUANT(DT, TY, 2); break;                                                                   \
     case 3: KVQ_LAUNCH_QUANT(DT, TY, 3); break;                                                                   \
@@ -400,61 +451,163 @@ kvq_status kvq_append(const void* K, const kvq_tensor4* kd, const void* V, const
   return launch_quant(K, kd, V, vd, alloc, c, t_begin, packed, stream);
 }
 
-kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
-                           const kvq_cache_desc* c, int seq_len, float* out, void* ws, size_t ws_bytes,
-                           void* stream) {
+}  // extern "C"
+namespace {
+
+// Checks a [batch][n_kv_heads][>= n][128] view against a cache descriptor.
+kvq_status check_kv_view(const void* p, const kvq_tensor4* t, const kvq_cache_desc* c, int n) {
+  kvq_status st = check_tensor(p, t);
+  if (st != KVQ_OK) return st;
+  if (t->batch != c->batch || t->n_heads != c->n_kv_heads || t->seq_len < n) return KVQ_ERR_SHAPE;
+  return KVQ_OK;
+}
+
+kvq_status launch_decode(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
+                         const kvq_cache_desc* c, int seq_len, const kvq_decode_extra* ex, float* out, void* ws,
+                         size_t ws_bytes, void* stream) {
   kvq_status st;
   if ((st = check_tensor(q, qd)) != KVQ_OK) return st;
   if (!packed || !alloc || !out || !aligned16(packed) || !aligned16(alloc)) return KVQ_ERR_ARG;
   if (!cache_ok(c)) return KVQ_ERR_ARG;
   if (qd->seq_len != 1 || qd->batch != c->batch) return KVQ_ERR_SHAPE;
   if (qd->n_heads % c->n_kv_heads != 0 || qd->n_heads / c->n_kv_heads > 8) return KVQ_ERR_UNSUPPORTED;
-  if (seq_len < 1 || seq_len > c->capacity) return KVQ_ERR_RANGE;
+  const bool keys_only = c->bits_v == 0;
+  const bool dense_v = ex && ex->V;
+  const int n_recent = (ex && ex->K_recent) ? ex->krd.seq_len : 0;
+  if (keys_only != dense_v) return keys_only ? KVQ_ERR_UNSUPPORTED : KVQ_ERR_ARG;
+  if (ex && (ex->K_recent != nullptr) != (ex->V_recent != nullptr)) return KVQ_ERR_ARG;
+  if (seq_len < (n_recent > 0 ? 0 : 1) || seq_len > c->capacity) return KVQ_ERR_RANGE;
+  if (dense_v) {
+    if ((st = check_kv_view(ex->V, &ex->vd, c, seq_len)) != KVQ_OK) return st;
+    if (ex->vd.dtype != KVQ_BF16 && ex->vd.dtype != KVQ_F16) return KVQ_ERR_DTYPE;
+  }
+  if (n_recent > 0) {
+    if ((st = check_kv_view(ex->K_recent, &ex->krd, c, n_recent)) != KVQ_OK) return st;
+    if ((st = check_kv_view(ex->V_recent, &ex->vrd, c, n_recent)) != KVQ_OK) return st;
+  }
   const int bh = c->batch * c->n_kv_heads;
   const int n_tiles = n_tiles_of(seq_len);
   const int splits = gtq_splits(bh, n_tiles);
+  const MergePlan mp = merge_plan(splits);
   const DecodeWs L = gtq_ws_layout(bh, splits);
   if (!ws || ws_bytes < L.total || !aligned16(ws) || ws_bytes < kvq_decode_workspace_bytes(c, qd->n_heads))
     return KVQ_ERR_WORKSPACE;
   if ((st = ensure_tables()) != KVQ_OK) return st;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
-  const size_t smem = decode_smem_bytes(c->bits_k, c->bits_v);
+  const int cb = chunk_bytes(rec) + (dense_v ? kChunkTokens * 2 * kD : 0);
+  const size_t smem = decode_smem_bytes(cb);
+  DecArgs a{};
+  a.q = q;
+  a.qsb = qd->stride_b;
+  a.qsh = qd->stride_h;
+  a.q_dtype = qd->dtype;
+  a.n_q_heads = qd->n_heads;
+  a.n_kv_heads = c->n_kv_heads;
+  a.batch = c->batch;
+  if (dense_v) {
+    a.v_dense = ex->V;
+    a.vsb = ex->vd.stride_b;
+    a.vsh = ex->vd.stride_h;
+    a.vst = ex->vd.stride_t;
+  }
+  a.cbytes = cb;
+  if (n_recent > 0) {
+    a.k_rec = ex->K_recent;
+    a.v_rec = ex->V_recent;
+    a.krsb = ex->krd.stride_b;
+    a.krsh = ex->krd.stride_h;
+    a.krst = ex->krd.stride_t;
+    a.vrsb = ex->vrd.stride_b;
+    a.vrsh = ex->vrd.stride_h;
+    a.vrst = ex->vrd.stride_t;
+    a.kr_dtype = ex->krd.dtype;
+    a.vr_dtype = ex->vrd.dtype;
+    a.n_recent = n_recent;
+  }
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.alloc = static_cast<const kvq_head_alloc*>(alloc);
+  a.hdr_bytes = static_cast<int>(header_bytes(c->n_kv_heads));
+  a.tiles_cap = n_tiles_of(c->capacity);
+  a.rec_bytes = rec;
+  a.bits_k = c->bits_k;
+  a.bits_v = c->bits_v;
+  a.capacity = c->capacity;
+  a.seq_len = seq_len;
+  a.splits = splits;
+  a.n_groups = splits > 1 ? mp.n_groups : 0;
+  a.group_size = mp.group_size;
+  a.n_stages = decode_stages(cb);
+  a.out = out;
+  a.part_m = reinterpret_cast<float*>(w8 + L.part_m);
+  a.part_l = reinterpret_cast<float*>(w8 + L.part_l);
+  a.part_o = reinterpret_cast<float*>(w8 + L.part_o);
+  a.tickets = reinterpret_cast<unsigned*>(w8 + L.tickets);
+  a.status = reinterpret_cast<unsigned*>(w8);
+  a.wait_limit = g_wait_limit;
+  a.debug_no_loads = g_debug_no_loads;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(splits, bh);
-#define KVQ_LAUNCH_DEC(DT, TY, BV)                                                                                    \
+  const int vm = dense_v ? (ex->vd.dtype == KVQ_BF16 ? kDenseBf16 : kDenseF16) : c->bits_v;
+#define KVQ_LAUNCH_DEC(VM)                                                                                            \
   do {                                                                                                                \
-    auto kern = kvq_decode_gtq<DT, BV>;                                                                               \
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=            \
-        cudaSuccess)                                                                                                  \
-      return KVQ_ERR_CUDA;                                                                                            \
-    kern<<<grid, kDecThreads, smem, s>>>(                                                                             \
-        static_cast<const TY*>(q), qd->stride_b, qd->stride_h, qd->n_heads, c->n_kv_heads,                             \
-        static_cast<const uint8_t*>(packed), static_cast<const kvq_head_alloc*>(alloc), n_tiles_of(c->capacity), rec, \
-        c->bits_k, c->bits_v, seq_len, splits, merge_groups(splits), decode_stages(c->bits_k, c->bits_v), out,       \
-        reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_l),                            \
-        reinterpret_cast<float*>(w8 + L.part_o), reinterpret_cast<unsigned*>(w8 + L.tickets),                        \
-        reinterpret_cast<unsigned*>(w8));                                                                             \
+    auto kern = kvq_decode_gtq<VM>;                                                                                   \
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,                     \
+                                               static_cast<int>(smem));                                               \
+    if (e != cudaSuccess) return cuda_fail(e);                                                                        \
+    kern<<<grid, kDecThreads, smem, s>>>(a);                                                                          \
   } while (0)
-#define KVQ_DEC_BV(DT, TY)                                                                                            \
-  switch (c->bits_v) {                                                                                                \
-    case 1: KVQ_LAUNCH_DEC(DT, TY, 1); break;                                                                         \
-    case 2: KVQ_LAUNCH_DEC(DT, TY, 2); break;                                                                         \
-    case 3: KVQ_LAUNCH_DEC(DT, TY, 3); break;                                                                         \
-    case 4: KVQ_LAUNCH_DEC(DT, TY, 4); break;                                                                         \
-    case 5: KVQ_LAUNCH_DEC(DT, TY, 5); break;                                                                         \
-    case 6: KVQ_LAUNCH_DEC(DT, TY, 6); break;                                                                         \
-    case 7: KVQ_LAUNCH_DEC(DT, TY, 7); break;                                                                         \
-    default: KVQ_LAUNCH_DEC(DT, TY, 8); break;                                                                        \
+  switch (vm) {
+    case 1: KVQ_LAUNCH_DEC(1); break;
+    case 2: KVQ_LAUNCH_DEC(2); break;
+    case 3: KVQ_LAUNCH_DEC(3); break;
+    case 4: KVQ_LAUNCH_DEC(4); break;
+    case 5: KVQ_LAUNCH_DEC(5); break;
+    case 6: KVQ_LAUNCH_DEC(6); break;
+    case 7: KVQ_LAUNCH_DEC(7); break;
+    case 8: KVQ_LAUNCH_DEC(8); break;
+    case kDenseBf16: KVQ_LAUNCH_DEC(kDenseBf16); break;
+    default: KVQ_LAUNCH_DEC(kDenseF16); break;
   }
-  switch (qd->dtype) {
-    case KVQ_F32: KVQ_DEC_BV(KVQ_F32, float); break;
-    case KVQ_F16: KVQ_DEC_BV(KVQ_F16, __half); break;
-    default: KVQ_DEC_BV(KVQ_BF16, __nv_bfloat16); break;
-  }
-#undef KVQ_DEC_BV
 #undef KVQ_LAUNCH_DEC
   return launch_status();
+}
+
+}  // namespace
+extern "C" {
+
+kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
+                           const kvq_cache_desc* c, int seq_len, float* out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  return launch_decode(q, qd, packed, alloc, c, seq_len, nullptr, out, ws, ws_bytes, stream);
+}
+
+kvq_status kvq_decode_attn_ex(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
+                              const kvq_cache_desc* c, int seq_len, const kvq_decode_extra* extra, float* out,
+                              void* ws, size_t ws_bytes, void* stream) {
+  return launch_decode(q, qd, packed, alloc, c, seq_len, extra, out, ws, ws_bytes, stream);
+}
+
+kvq_status kvq_packed_status(const void* packed, void* stream, int* device_code) {
+  if (!packed) return KVQ_ERR_ARG;
+  unsigned int code = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* p = static_cast<const uint8_t*>(packed) + offsetof(kvq_packed_header, status);
+  { const cudaError_t e_ = cudaMemcpyAsync(&code, p, sizeof(code), cudaMemcpyDeviceToHost, s); if (e_ != cudaSuccess) return cuda_fail(e_); }
+  { const cudaError_t e_ = cudaStreamSynchronize(s); if (e_ != cudaSuccess) return cuda_fail(e_); }
+  if (device_code) *device_code = static_cast<int>(code);
+  return code == 0 ? KVQ_OK : static_cast<kvq_status>(code);
+}
+
+const char* kvq_last_cuda_error(void) {
+  return cudaGetErrorString(static_cast<cudaError_t>(g_last_cuda_error.load()));
+}
+
+kvq_status kvq_debug_decode(int wait_limit, int no_loads) {
+  if (wait_limit < 1) return KVQ_ERR_ARG;
+  g_wait_limit = static_cast<uint32_t>(wait_limit);
+  g_debug_no_loads = no_loads ? 1 : 0;
+  return KVQ_OK;
 }
 
 size_t kvq_nf4_packed_bytes(int batch, int n_heads, int capacity, int head_dim) {
@@ -571,8 +724,9 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
 // inference-engine plugin whose interface forbids allocating on the hot path. They cannot
 // provide the split-merge workspace kvq_decode_attn needs. This entry point uses a fixed
 // scratch array instead: a file-scope __device__ array that every GPU loading the library
-// holds until the process exits. Its device address is looked up once per device (with that
-// device current) and handed to the ordinary decode kernel as its workspace.
+// holds until the process exits. Its device address is looked up on every call (with the
+// caller's device current) and handed to the ordinary Block-GTQ decode kernel as its
+// workspace.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 2u << 20;   // 2 MiB per device
@@ -581,20 +735,22 @@ __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device. The first call on a device
-// resolves it with cudaGetSymbolAddress and zeroes the array (the split tickets in it must
-// start at zero; the kernel returns them to zero after every call).
-kvq_status decode_scratch(void** out) {
+// Device address of the scratch array on the current device. When the address is new for
+// this device (its first call, or a context created again after a reset), the array is zeroed
+// by an asynchronous memset on the caller's stream, so the decode launched next on that
+// stream sees zero split tickets and a clear status word; the kernel returns the tickets to
+// zero after every call.
+kvq_status decode_scratch(cudaStream_t s, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return KVQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return KVQ_ERR_CUDA;
-    if (cudaMemset(p, 0, kNoAllocScratchBytes) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (g_scratch_ptr[dev] != p) {
+    { const cudaError_t e_ = cudaMemsetAsync(p, 0, kNoAllocScratchBytes, s); if (e_ != cudaSuccess) return cuda_fail(e_); }
     g_scratch_ptr[dev] = p;
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return KVQ_OK;
 }
 
@@ -613,9 +769,24 @@ kvq_status kvq_decode_attn_noalloc(const void* q, const kvq_tensor4* qd, const v
   kvq_status st = ensure_tables();
   if (st != KVQ_OK) return st;
   void* scratch = nullptr;
-  if ((st = decode_scratch(&scratch)) != KVQ_OK) return st;
+  if ((st = decode_scratch(static_cast<cudaStream_t>(stream), &scratch)) != KVQ_OK) return st;
   return kvq_decode_attn(q, qd, packed, alloc, cache, seq_len, out, scratch, kNoAllocScratchBytes, stream);
 }
 
-}  // extern "C"
+kvq_status kvq_decode_noalloc_status(void* stream, int* device_code) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  kvq_status st = decode_scratch(s, &scratch);
+  if (st != KVQ_OK) return st;
+  unsigned int code = 0;
+  { const cudaError_t e_ = cudaMemcpyAsync(&code, scratch, sizeof(code), cudaMemcpyDeviceToHost, s); if (e_ != cudaSuccess) return cuda_fail(e_); }
+  { const cudaError_t e_ = cudaStreamSynchronize(s); if (e_ != cudaSuccess) return cuda_fail(e_); }
+  if (code != 0) {
+    { const cudaError_t e_ = cudaMemsetAsync(scratch, 0, sizeof(code), s); if (e_ != cudaSuccess) return cuda_fail(e_); }
+    { const cudaError_t e_ = cudaStreamSynchronize(s); if (e_ != cudaSuccess) return cuda_fail(e_); }
+  }
+  if (device_code) *device_code = static_cast<int>(code);
+  return code == 0 ? KVQ_OK : static_cast<kvq_status>(code);
+}
 
+}  // extern "C"

@@ -25,6 +25,7 @@ struct Nf4Layout {
 
 constexpr int kNf4Rows = 4;   // token rows per warp task
 constexpr int kNf4DecWarps = 16;   // warps per CTA of the NF4 decode
+constexpr int kNf4MaxSplits = 160;  // splits per (sequence, head) the NF4 merge reads
 
 // One warp per (K-or-V, sequence, block, group of 4 token rows). Lane l holds values 8l..8l+7
 // of the block: head 2*blk + l/16, dims 8(l%16)..8(l%16)+7. All rows of the group are loaded

@@ -3,7 +3,8 @@
 // allocator sits on TurboQuant-MSE, K and V get matched bit budgets, the cache is packed).
 //
 // For a token row x (128 values):
-//   s2   = sum_j x_j^2 in fp32, j ascending: fl32(s2 + fl32(x_j x_j))
+//   s2   = sum_j x_j^2 in fp32: eight partial sums over j = r (mod 8), j ascending, each
+//          step fl32(s_r + fl32(x_j x_j)), combined ((s0+s1)+(s2+s3))+((s4+s5)+(s6+s7))
 //   norm = fp16(fp32 sqrt(s2)) (round to nearest even)
 //   a    = fp32(sqrt(128)) / fp32(norm), 0 if norm == 0
 //   y_j  = fp32(fp32(x_j a) g_b)            (V: g = 1, the multiply is skipped as exact)
@@ -150,32 +151,63 @@ __device__ __forceinline__ float2 unpack_pair(uint32_t w) {
   else return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
+// Two fp32 sums in one instruction, each rounded to nearest even.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t ua, ub, ud;
+  memcpy(&ua, &a, 8);
+  memcpy(&ub, &b, 8);
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(ud) : "l"(ua), "l"(ub));
+  float2 d;
+  memcpy(&d, &ud, 8);
+  return d;
+}
+
+// a * b + c for two pairs in one instruction, each rounded once.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t ua, ub, uc, ud;
+  memcpy(&ua, &a, 8);
+  memcpy(&ub, &b, 8);
+  memcpy(&uc, &c, 8);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(ud) : "l"(ua), "l"(ub), "l"(uc));
+  float2 d;
+  memcpy(&d, &ud, 8);
+  return d;
+}
+
 // fp16 norm of the lane's own staged row and the scale a = sqrt(128)/norm (0 for a zero norm).
+// The sum of squares is fixed to eight partial sums s_r over the coordinates j = r (mod 8),
+// j ascending, combined as ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)); acc[i] holds
+// (s_2i, s_2i+1). For 16-bit inputs x * x is exact in fp32, so one fused multiply-add per
+// step rounds exactly like the product followed by the sum.
 template <int DT>
 __device__ __forceinline__ void row_norm_scale(const uint32_t* row, __half& n16, float& a) {
-  float s2 = 0.0f;
-#pragma unroll 4
+  float2 acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
+#pragma unroll
   for (int c = 0; c < QTile<DT>::kPieces; ++c) {
     const uint4 v = *reinterpret_cast<const uint4*>(row + 4 * c);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     if constexpr (DT == KVQ_F32) {
+      // piece c holds coordinates 4c .. 4c + 3: pairs (s0, s1), (s2, s3) or (s4, s5), (s6, s7)
+      const int base = 2 * (c & 1);
 #pragma unroll
-      for (int i = 0; i < 4; i += 2) {
-        const float2 x = make_float2(__uint_as_float(w[i]), __uint_as_float(w[i + 1]));
-        const float2 q = mul2(x, x);
-        s2 = __fadd_rn(s2, q.x);
-        s2 = __fadd_rn(s2, q.y);
+      for (int i = 0; i < 2; ++i) {
+        const float2 x = make_float2(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
+        acc[base + i] = add2(acc[base + i], mul2(x, x));
       }
     } else {
+      // piece c holds coordinates 8c .. 8c + 7: word i is the pair (s_2i, s_2i+1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 x = unpack_pair<DT>(w[i]);
-        const float2 q = mul2(x, x);
-        s2 = __fadd_rn(s2, q.x);
-        s2 = __fadd_rn(s2, q.y);
+        acc[i] = fma2(x, x, acc[i]);
       }
     }
   }
+  const float lo = __fadd_rn(__fadd_rn(acc[0].x, acc[0].y), __fadd_rn(acc[1].x, acc[1].y));
+  const float hi = __fadd_rn(__fadd_rn(acc[2].x, acc[2].y), __fadd_rn(acc[3].x, acc[3].y));
+  const float s2 = __fadd_rn(lo, hi);
   n16 = __float2half_rn(__fsqrt_rn(s2));
   const float nf = __half2float(n16);
   const float sqd = 11.313708305358887f;       // fp32(sqrt(128))
@@ -317,32 +349,83 @@ template <int DT> struct QWarpSmem {
   static constexpr int kBytes = 2 * 4 * QTile<DT>::kWords + kTile * 8 + kKEntries * 8 + 8 * 4;
 };
 
-// One instantiation per value width BVT (= bits_v), so registers are allocated for one value
-// pass only.
+// Packed-header handling of a quantize or append call.
+struct QHeader {
+  int mode;              // 0: leave it, 1: write it (a call starting at token 0), 2: check it
+  int batch, capacity, hdr_bytes;
+};
+
+// Header fields and digests written by CTA 0 (one warp) of a call that starts at token 0.
+__device__ __forceinline__ void write_packed_header(uint8_t* packed, const QHeader& qh, int n_kv_heads, int bits_k,
+                                                    int bits_v, int rec_bytes, const kvq_head_alloc* alloc,
+                                                    int lane) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(packed);
+  for (int i = lane; i < qh.hdr_bytes / 4; i += 32) {
+    uint32_t v = 0u;
+    if (i == 0) v = 0x3151564Bu;                                             // "KVQ1"
+    else if (i == 1) v = 1u | (static_cast<uint32_t>(kD) << 16);           // layout 1, head_dim
+    else if (i == 2) v = static_cast<uint32_t>(bits_k) | (static_cast<uint32_t>(bits_v) << 8) |
+                         (static_cast<uint32_t>(alloc->w_max & 0xff) << 16) |
+                         (static_cast<uint32_t>(alloc->mode & 0xff) << 24);
+    else if (i == 4) v = static_cast<uint32_t>(qh.batch);
+    else if (i == 5) v = static_cast<uint32_t>(n_kv_heads);
+    else if (i == 6) v = static_cast<uint32_t>(qh.capacity);
+    else if (i == 7) v = static_cast<uint32_t>(rec_bytes);
+    else if (i >= 16 && i < 16 + 2 * n_kv_heads) {
+      const uint64_t d = alloc[(i - 16) >> 1].digest;
+      v = static_cast<uint32_t>((i & 1) ? (d >> 32) : d);
+    }
+    w[i] = v;
+  }
+}
+
+// An append (call not starting at token 0) may only extend a cache whose header names this
+// layout, these shapes and widths, and the same allocation, and carries no status; otherwise
+// it records KVQ_ERR_MISMATCH there (keeping an earlier status) and writes nothing.
+__device__ __forceinline__ bool packed_header_ok(uint8_t* packed, const QHeader& qh, int n_kv_heads, int bits_k,
+                                                 int bits_v, int rec_bytes, const kvq_head_alloc* alloc) {
+  const kvq_packed_header* H = reinterpret_cast<const kvq_packed_header*>(packed);
+  bool ok = H->status == 0 && H->magic == 0x3151564Bu && H->layout_version == 1 && H->head_dim == kD &&
+            H->bits_k == bits_k && H->bits_v == bits_v && H->batch == qh.batch && H->n_kv_heads == n_kv_heads &&
+            H->capacity == qh.capacity && static_cast<int>(H->record_bytes) == rec_bytes;
+  const uint64_t* dig = reinterpret_cast<const uint64_t*>(packed + sizeof(kvq_packed_header));
+  for (int h = 0; ok && h < n_kv_heads; ++h) ok = dig[h] == alloc[h].digest;
+  if (!ok) atomicCAS(const_cast<uint32_t*>(&H->status), 0u, static_cast<uint32_t>(KVQ_ERR_MISMATCH));
+  return ok;
+}
+
+// One instantiation per value width BVT (= bits_v; 0 = keys only), so registers are
+// allocated for one value pass only.
 template <int DT, int BVT>
 __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
     const typename Elem<DT>::T* __restrict__ K, int64_t ksb, int64_t ksh, int64_t kst,
     const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst,
     int t_begin, int t_end, int tile_lo, int n_tiles, int n_kv_heads, int tiles_cap,
     const kvq_head_alloc* __restrict__ alloc, int bits_k, int bits_v, uint8_t* __restrict__ packed, int rec_bytes,
-    int n_tasks) {
+    int n_tasks, QHeader qh) {
   using Q = QTile<DT>;
   constexpr int kWarps = Q::kWarps;
+  constexpr bool kKeysOnly = BVT == 0;
   extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ int sHeaderOk;
   uint2* sLut = reinterpret_cast<uint2*>(smem);
   for (int i = threadIdx.x; i < kLutEntries; i += blockDim.x)
     sLut[i] = make_uint2(g_quant_lut[2 * i], g_quant_lut[2 * i + 1]);
+  if (threadIdx.x == 0) sHeaderOk = (qh.mode == 2) ? packed_header_ok(packed, qh, n_kv_heads, bits_k, bits_v, rec_bytes, alloc) : 1;
+  if (qh.mode == 1 && blockIdx.x == 0 && threadIdx.x < 32)
+    write_packed_header(packed, qh, n_kv_heads, bits_k, bits_v, rec_bytes, alloc, threadIdx.x);
   __syncthreads();
+  if (!sHeaderOk) return;
+  uint8_t* records = packed + qh.hdr_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k_words = bits_k * kD;
   uint8_t* wbase = smem + kLutEntries * 8 + warp * QWarpSmem<DT>::kBytes;
   uint32_t* kbuf = reinterpret_cast<uint32_t*>(wbase);
-  uint32_t* vbuf = kbuf + Q::kWords;
+  uint32_t* vbuf = kbuf + Q::kWords;                // keys only: the second K tile buffer
   float2* sA2 = reinterpret_cast<float2*>(vbuf + Q::kWords);
   KEntry* sEnt = reinterpret_cast<KEntry*>(sA2 + kTile);
   uint32_t* sCls = reinterpret_cast<uint32_t*>(sEnt + kKEntries);     // width | first << 8 | blocks << 16
-  const uint32_t* myk = kbuf + lane * Q::kPitch;
   const uint32_t* myv = vbuf + lane * Q::kPitch;
   int cur_h = -1, n_cls = 0;
 
@@ -361,19 +444,22 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
     r_hi = min(kTile, t_end - t0);
     const int64_t i0 = static_cast<int64_t>(t0 + r_lo - t_begin);
     kp = K + b * ksb + h * ksh + i0 * kst;
-    vp = V + b * vsb + h * vsh + i0 * vst;
+    vp = kKeysOnly ? nullptr : V + b * vsb + h * vsh + i0 * vst;
   };
 
   // The current task's coordinates; each iteration computes the next task's.
   int bh = 0, tile = 0, r_lo = 0, r_hi = 0;
   bool write = false;
+  int kb = 0;                                       // keys only: the K buffer of the current task
   if (task < n_tasks) {
     const typename Elem<DT>::T *kp, *vp;
     task_src(task, bh, tile, r_lo, r_hi, kp, vp);
     tile_load_async<DT>(kbuf, kp, kst, r_lo, r_hi, lane);
     cp_async_commit();
-    tile_load_async<DT>(vbuf, vp, vst, r_lo, r_hi, lane);
-    cp_async_commit();
+    if constexpr (!kKeysOnly) {
+      tile_load_async<DT>(vbuf, vp, vst, r_lo, r_hi, lane);
+      cp_async_commit();
+    }
   }
 
   for (; task < n_tasks; task += stride) {
@@ -406,17 +492,27 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
       __syncwarp();
       cur_h = h;
     }
-    uint8_t* rec = packed + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
+    uint8_t* rec = records + (static_cast<size_t>(bh) * tiles_cap + tile) * rec_bytes;
     uint32_t* kout = reinterpret_cast<uint32_t*>(rec);
     uint16_t* norms = reinterpret_cast<uint16_t*>(kout + k_words);   // 32 K norms, then 32 V norms
     uint32_t* vout = kout + k_words + kTile;
+    uint32_t* kcur = (kKeysOnly && kb) ? vbuf : kbuf;
+    uint32_t* knext = (kKeysOnly && !kb) ? vbuf : kbuf;
 
     // ---------------------------------------------------------------- K (Block-GTQ widths)
-    cp_async_wait<1>();                          // this task's K rows (its V rows may be in flight)
+    if constexpr (kKeysOnly) {
+      // the next task's K rows load into the other buffer while this one is coded
+      if (nkp) tile_load_async<DT>(knext, nkp, kst, nlo, nhi, lane);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<1>();                        // this task's K rows (its V rows may be in flight)
+    }
     __syncwarp();
     if (write) {
       __half n16;
       float a;
+      const uint32_t* myk = kcur + lane * Q::kPitch;
       row_norm_scale<DT>(myk, n16, a);
       if (mine) norms[lane] = valid ? __half_as_ushort(n16) : 0;
       if (!valid) a = __int_as_float(0x7fc00000);   // NaN: every code is 0
@@ -441,26 +537,30 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
       }
     }
     __syncwarp();                               // every lane is done with the K tile
-    if (nkp) tile_load_async<DT>(kbuf, nkp, kst, nlo, nhi, lane);
-    cp_async_commit();
+    if constexpr (kKeysOnly) {
+      kb ^= 1;
+    } else {
+      if (nkp) tile_load_async<DT>(kbuf, nkp, kst, nlo, nhi, lane);
+      cp_async_commit();
 
-    // ---------------------------------------------------------------- V (uniform width)
-    cp_async_wait<1>();                          // this task's V rows (next K rows may be in flight)
-    __syncwarp();
-    if (write) {
-      __half n16;
-      float a;
-      row_norm_scale<DT>(myv, n16, a);
-      if (mine) norms[kTile + lane] = valid ? __half_as_ushort(n16) : 0;
-      if (!valid) a = __int_as_float(0x7fc00000);
-      sA2[lane] = make_float2(a, a);
-      const int keep = bits_v * r_lo;
+      // -------------------------------------------------------------- V (uniform width)
+      cp_async_wait<1>();                        // this task's V rows (next K rows may be in flight)
       __syncwarp();
-      quant_v_tile<DT, BVT>(vbuf, sA2, sLut, vout, keep, lane);
+      if (write) {
+        __half n16;
+        float a;
+        row_norm_scale<DT>(myv, n16, a);
+        if (mine) norms[kTile + lane] = valid ? __half_as_ushort(n16) : 0;
+        if (!valid) a = __int_as_float(0x7fc00000);
+        sA2[lane] = make_float2(a, a);
+        const int keep = bits_v * r_lo;
+        __syncwarp();
+        quant_v_tile<DT, BVT>(vbuf, sA2, sLut, vout, keep, lane);
+      }
+      __syncwarp();                               // every lane is done with the V tile and sA2
+      if (nvp) tile_load_async<DT>(vbuf, nvp, vst, nlo, nhi, lane);
+      cp_async_commit();
     }
-    __syncwarp();                               // every lane is done with the V tile and sA2
-    if (nvp) tile_load_async<DT>(vbuf, nvp, vst, nlo, nhi, lane);
-    cp_async_commit();
     bh = nbh; tile = ntile; r_lo = nlo; r_hi = nhi;
   }
   asm volatile("cp.async.wait_all;" ::: "memory");

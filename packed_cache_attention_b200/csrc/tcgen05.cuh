@@ -202,11 +202,12 @@ __device__ __forceinline__ void tmem_ld2x2_wait(uint32_t ta, uint32_t tb, uint32
 
 // ---------------------------------------------------------------- MMA
 
-// Instruction descriptor for kind::f16 with fp16 A and B, fp32 accumulate, A K-major.
-// n_major_b selects an N-major (transposed) B operand.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool n_major_b) {
+// Instruction descriptor for kind::f16 with fp16 (or, with bf16 set, bf16) A and B, fp32
+// accumulate, A K-major. n_major_b selects an N-major (transposed) B operand.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool n_major_b, bool bf16 = false) {
   return (1u << 4)                                   // D format: fp32
-         | (0u << 7) | (0u << 10)                     // A, B format: fp16
+         | ((bf16 ? 1u : 0u) << 7)                    // A format: fp16 / bf16
+         | ((bf16 ? 1u : 0u) << 10)                   // B format: fp16 / bf16
          | (0u << 15)                                 // A K-major
          | ((n_major_b ? 1u : 0u) << 16)              // B major
          | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8

@@ -16,7 +16,9 @@ LIB_PATH = os.path.join(_PKG, "libkvq.so")
 
 KVQ_OK = 0
 STATUS_NAMES = ["OK", "ERR_ARG", "ERR_SHAPE", "ERR_DTYPE", "ERR_BUDGET", "ERR_RANGE", "ERR_WORKSPACE",
-                "ERR_CUDA", "ERR_TIMEOUT", "ERR_UNSUPPORTED"]
+                "ERR_CUDA", "ERR_TIMEOUT", "ERR_UNSUPPORTED", "ERR_MISMATCH"]
+KVQ_ERR_TIMEOUT = 8
+KVQ_ERR_MISMATCH = 10
 KVQ_F32, KVQ_F16, KVQ_BF16 = 0, 1, 2
 MODE_BLOCKGTQ, MODE_UNIFORM = 0, 1
 TILE = 32
@@ -26,7 +28,10 @@ HEAD_DIM = 128
 class KvqError(RuntimeError):
     def __init__(self, fn: str, status: int):
         name = STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else str(status)
-        super().__init__(f"{fn} failed: KVQ_{name} ({status})")
+        detail = ""
+        if status == 7 and _lib is not None:
+            detail = f" [{_lib.kvq_last_cuda_error().decode()}]"
+        super().__init__(f"{fn} failed: KVQ_{name} ({status}){detail}")
         self.status = status
 
 
@@ -55,9 +60,22 @@ class HeadAlloc(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("bits_k", ctypes.c_int32), ("w_max", ctypes.c_int32),
                 ("mode", ctypes.c_int32), ("n_classes", ctypes.c_int32), ("k_words", ctypes.c_int32),
                 ("n_blocks", ctypes.c_int32), ("reserved", ctypes.c_int32),
-                ("plan_run", (ctypes.c_uint32 * 8) * 4), ("plan_group", (ctypes.c_uint32 * 16) * 4),
-                ("plan_col_block", ctypes.c_int8 * 128), ("plan_n_runs", ctypes.c_int32 * 4),
-                ("plan_k_cols", ctypes.c_int32), ("reserved_c", ctypes.c_uint8 * 108)]
+                ("plan_slot", ctypes.c_uint32 * 24), ("plan_col_block", ctypes.c_int8 * 96),
+                ("plan_n_slots", ctypes.c_int32), ("plan_k_cols", ctypes.c_int32), ("digest", ctypes.c_uint64),
+                ("reserved_c", ctypes.c_uint8 * 432)]
+
+
+class PackedHeader(ctypes.Structure):
+    _fields_ = [("magic", ctypes.c_uint32), ("layout_version", ctypes.c_uint16), ("head_dim", ctypes.c_uint16),
+                ("bits_k", ctypes.c_uint8), ("bits_v", ctypes.c_uint8), ("w_max", ctypes.c_uint8),
+                ("mode", ctypes.c_uint8), ("status", ctypes.c_uint32), ("batch", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("capacity", ctypes.c_int32), ("record_bytes", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint8 * 32)]
+
+
+class DecodeExtra(ctypes.Structure):
+    _fields_ = [("V", ctypes.c_void_p), ("vd", Tensor4), ("K_recent", ctypes.c_void_p), ("krd", Tensor4),
+                ("V_recent", ctypes.c_void_p), ("vrd", Tensor4)]
 
 
 _VP = ctypes.c_void_p
@@ -74,6 +92,10 @@ _SIGNATURES = {
     "kvq_alloc_bytes": ([_I], _SZ),
     "kvq_calibrate_workspace_bytes": ([_I, _I, _I], _SZ),
     "kvq_packed_bytes": ([_PC], _SZ),
+    "kvq_packed_header_bytes": ([_I], _SZ),
+    "kvq_packed_status": ([_VP, _VP, ctypes.POINTER(_I)], _I),
+    "kvq_debug_decode": ([_I, _I], _I),
+    "kvq_last_cuda_error": ([], ctypes.c_char_p),
     "kvq_decode_workspace_bytes": ([_PC, _I], _SZ),
     "kvq_init": ([], _I),
     "kvq_workspace_init": ([_VP, _SZ, _VP], _I),
@@ -82,6 +104,7 @@ _SIGNATURES = {
     "kvq_quantize": ([_VP, _P4, _VP, _P4, _VP, _PC, _VP, _VP], _I),
     "kvq_append": ([_VP, _P4, _VP, _P4, _VP, _PC, _I, _VP, _VP], _I),
     "kvq_decode_attn": ([_VP, _P4, _VP, _VP, _PC, _I, _VP, _VP, _SZ, _VP], _I),
+    "kvq_decode_attn_ex": ([_VP, _P4, _VP, _VP, _PC, _I, ctypes.POINTER(DecodeExtra), _VP, _VP, _SZ, _VP], _I),
     "kvq_nf4_packed_bytes": ([_I, _I, _I, _I], _SZ),
     "kvq_nf4_decode_workspace_bytes": ([_I, _I, _I, _I], _SZ),
     "kvq_nf4_quantize": ([_VP, _P4, _VP, _P4, _I, _VP, _VP], _I),
@@ -89,6 +112,7 @@ _SIGNATURES = {
     "kvq_nf4_decode_attn": ([_VP, _P4, _VP, _I, _I, _VP, _VP, _SZ, _VP], _I),
     "kvq_decode_attn_noalloc": ([_VP, _P4, _VP, _VP, _PC, _I, _VP, _VP], _I),
     "kvq_decode_noalloc_scratch_bytes": ([], _SZ),
+    "kvq_decode_noalloc_status": ([_VP, ctypes.POINTER(_I)], _I),
 }
 
 _lib = None
@@ -157,6 +181,22 @@ def kvq_packed_bytes(cache: CacheDesc) -> int:
     return lib().kvq_packed_bytes(ctypes.byref(cache))
 
 
+def kvq_packed_header_bytes(n_kv_heads: int) -> int:
+    return lib().kvq_packed_header_bytes(n_kv_heads)
+
+
+def kvq_packed_status(packed, stream=None) -> int:
+    """Status word of a packed cache's header (0, or the kvq_status an append recorded)."""
+    code = ctypes.c_int(0)
+    lib().kvq_packed_status(packed.data_ptr(), _stream(stream), ctypes.byref(code))
+    return code.value
+
+
+def kvq_debug_decode(wait_limit: int = 2000, no_loads: bool = False) -> None:
+    """Test hook: bounded-wait limit (tries of about 1 ms) and the no-copy switch of later decodes."""
+    _check("kvq_debug_decode", lib().kvq_debug_decode(int(wait_limit), 1 if no_loads else 0))
+
+
 def kvq_decode_workspace_bytes(cache: CacheDesc, n_q_heads: int) -> int:
     return lib().kvq_decode_workspace_bytes(ctypes.byref(cache), n_q_heads)
 
@@ -189,9 +229,8 @@ def parse_alloc(raw: np.ndarray) -> list[dict]:
             "class_blocks": np.array(rec.class_blocks[:], dtype=np.int64),
             "n_classes": rec.n_classes, "n_blocks": rec.n_blocks, "k_words": rec.k_words,
             "plan_col_block": np.array(rec.plan_col_block[:], dtype=np.int64), "plan_k_cols": rec.plan_k_cols,
-            "plan_n_runs": np.array(rec.plan_n_runs[:], dtype=np.int64),
-            "plan_run": np.array([list(r) for r in rec.plan_run], dtype=np.int64),
-            "plan_group": np.array([list(r) for r in rec.plan_group], dtype=np.int64),
+            "plan_slot": np.array(rec.plan_slot[:], dtype=np.int64), "plan_n_slots": rec.plan_n_slots,
+            "digest": int(rec.digest),
             "bits_k": rec.bits_k, "w_max": rec.w_max,
             "mode": rec.mode,
         })
@@ -259,23 +298,31 @@ def kvq_calibrate(K, bits_k: int, w_max: int = 8, n_calib: int = 0, mode: int = 
     return alloc
 
 
+def _opt_tensor(t):
+    """(pointer, tensor4 pointer) of an optional tensor; (None, None) for a keys-only call."""
+    if t is None:
+        return None, None
+    return t.data_ptr(), ctypes.byref(tensor4(t))
+
+
 def kvq_quantize(K, V, alloc, cache: CacheDesc, packed=None, stream=None):
-    """Quantize + pack K, V [B][Hkv][T][128] into a packed cache (uint8 device tensor)."""
+    """Quantize + pack K, V [B][Hkv][T][128] into a packed cache (uint8 device tensor).
+    V may be None for a keys-only cache (cache.bits_v = 0)."""
     if packed is None:
         packed = _empty_bytes(kvq_packed_bytes(cache), K.device)
-    kd, vd = tensor4(K), tensor4(V)
-    _check("kvq_quantize", lib().kvq_quantize(K.data_ptr(), ctypes.byref(kd), V.data_ptr(), ctypes.byref(vd),
-                                              alloc.data_ptr(), ctypes.byref(cache), packed.data_ptr(),
-                                              _stream(stream)))
+    kd = tensor4(K)
+    vp, vd = _opt_tensor(V)
+    _check("kvq_quantize", lib().kvq_quantize(K.data_ptr(), ctypes.byref(kd), vp, vd, alloc.data_ptr(),
+                                              ctypes.byref(cache), packed.data_ptr(), _stream(stream)))
     return packed
 
 
 def kvq_append(K, V, alloc, cache: CacheDesc, t_begin: int, packed, stream=None):
     """Quantize K, V [B][Hkv][n][128] as tokens t_begin .. t_begin + n - 1 of `packed`."""
-    kd, vd = tensor4(K), tensor4(V)
-    _check("kvq_append", lib().kvq_append(K.data_ptr(), ctypes.byref(kd), V.data_ptr(), ctypes.byref(vd),
-                                          alloc.data_ptr(), ctypes.byref(cache), int(t_begin), packed.data_ptr(),
-                                          _stream(stream)))
+    kd = tensor4(K)
+    vp, vd = _opt_tensor(V)
+    _check("kvq_append", lib().kvq_append(K.data_ptr(), ctypes.byref(kd), vp, vd, alloc.data_ptr(),
+                                          ctypes.byref(cache), int(t_begin), packed.data_ptr(), _stream(stream)))
     return packed
 
 
@@ -291,6 +338,30 @@ def kvq_decode_attn(q, packed, alloc, cache: CacheDesc, seq_len: int, out=None, 
     _check("kvq_decode_attn", lib().kvq_decode_attn(q.data_ptr(), ctypes.byref(qd), packed.data_ptr(),
                                                     alloc.data_ptr(), ctypes.byref(cache), seq_len, out.data_ptr(),
                                                     ws.data_ptr(), ws.numel(), _stream(stream)))
+    return out
+
+
+def kvq_decode_attn_ex(q, packed, alloc, cache: CacheDesc, seq_len: int, V=None, K_recent=None, V_recent=None,
+                       out=None, ws=None, stream=None):
+    """Decode attention with the values of a keys-only cache (V [B][Hkv][>= seq_len][128]) and/or
+    the most recent tokens kept unquantized (K_recent, V_recent [B][Hkv][R][128])."""
+    torch = _torch()
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = torch.zeros(kvq_decode_workspace_bytes(cache, Hq), dtype=torch.uint8, device=q.device)
+    ex = DecodeExtra()
+    if V is not None:
+        ex.V, ex.vd = V.data_ptr(), tensor4(V)
+    if K_recent is not None:
+        ex.K_recent, ex.krd = K_recent.data_ptr(), tensor4(K_recent)
+        ex.V_recent, ex.vrd = V_recent.data_ptr(), tensor4(V_recent)
+    qd = tensor4(q)
+    _check("kvq_decode_attn_ex", lib().kvq_decode_attn_ex(q.data_ptr(), ctypes.byref(qd), packed.data_ptr(),
+                                                          alloc.data_ptr(), ctypes.byref(cache), int(seq_len),
+                                                          ctypes.byref(ex), out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                          _stream(stream)))
     return out
 
 
@@ -310,6 +381,13 @@ def kvq_decode_attn_noalloc(q, packed, alloc, cache: CacheDesc, seq_len: int, ou
 
 def kvq_decode_noalloc_scratch_bytes() -> int:
     return lib().kvq_decode_noalloc_scratch_bytes()
+
+
+def kvq_decode_noalloc_status(stream=None) -> int:
+    """Status word of the allocation-free decode on the current device (read, then cleared)."""
+    code = ctypes.c_int(0)
+    lib().kvq_decode_noalloc_status(_stream(stream), ctypes.byref(code))
+    return code.value
 
 
 def kvq_nf4_quantize(K, V, capacity: int | None = None, packed=None, stream=None):

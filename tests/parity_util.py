@@ -36,6 +36,7 @@ def compare_alloc(gpu_heads, ref):
         assert g["k_words"] == int(2 * ref["w"][h].sum())
         check_classes(g, ref["w"][h])
         check_plan(g, ref["w"][h])
+        assert g["digest"] == bg.alloc_digest(ref["w"][h], ref["g"][h])
 
 
 def check_classes(g, w):
@@ -58,32 +59,33 @@ def check_classes(g, w):
 
 
 def check_plan(g, w):
-    """Decode plan: every block with w > 0 owns exactly one column; each group starts at the
-    bit offset of its first block and covers consecutive columns of one width."""
+    """Decode plan: width classes in stream order cut into slots of 4 consecutive block pairs;
+    slot s covers columns 4s..4s+3, starts at the bit offset of its first block, and every
+    block with w > 0 owns exactly one column."""
+    order = bg.k_stream_blocks(w)
+    off = bg.k_bit_offsets(w)
     cb = g["plan_col_block"]
-    kc = g["plan_k_cols"]
-    assert kc == 96
+    n_slots = int(g["plan_n_slots"])
+    assert g["plan_k_cols"] == -(-4 * n_slots // 8) * 8
+    widths = sorted({int(x) for x in w if x > 0}, reverse=True)
+    expect_slots = sum(-(-sum(1 for x in w if x == cw) // 4) for cw in widths)
+    assert n_slots == expect_slots
     blocks = [int(x) for x in cb if x >= 0]
     assert sorted(blocks) == [b for b in range(len(w)) if w[b] > 0]
-    assert all(x == -1 for x in cb[kc:])
-    off = bg.k_bit_offsets(w)
-    seen = 0
-    for wg in range(4):
-        for r in range(int(g["plan_n_runs"][wg])):
-            e = int(g["plan_run"][wg][r])
-            width, first, n, half = e & 15, (e >> 8) & 0xff, (e >> 16) & 0xff, e >> 24
-            for i in range(n):
-                ge = int(g["plan_group"][wg][first + i])
-                bit, col = ge & 0xffff, ge >> 16
-                npairs = 2 if (half and i == n - 1) else 4
-                b0 = int(cb[col])
-                assert b0 >= 0 and w[b0] == width and off[b0] == bit
-                for k in range(npairs):
-                    bk = int(cb[col + k])
-                    if bk >= 0:
-                        assert w[bk] == width and off[bk] == bit + 2 * width * k
-                seen += 1
-    assert seen == sum(-(-sum(1 for x in w if x == cw) // 4) for cw in set(int(x) for x in w if x > 0))
+    for s in range(24):
+        e = int(g["plan_slot"][s])
+        if s >= n_slots:
+            assert e == 0 and all(int(x) == -1 for x in cb[4 * s:4 * s + 4])
+            continue
+        width, bit = e & 0xff, e >> 8
+        b0 = int(cb[4 * s])
+        assert b0 >= 0 and w[b0] == width and off[b0] == bit
+        for k in range(4):
+            bk = int(cb[4 * s + k])
+            if bk >= 0:
+                assert w[bk] == width and off[bk] == bit + 2 * width * k
+    # columns follow the stream order, padding aside
+    assert blocks == order
 
 
 def oracle_pipeline(K, V, q, bits_k, bits_v, n_calib=0, w_max=8, mode=0, capacity=None):
@@ -102,3 +104,21 @@ def oracle_pipeline(K, V, q, bits_k, bits_v, n_calib=0, w_max=8, mode=0, capacit
 
 def tiles_written(T):
     return -(-T // bg.TILE)
+
+
+def split_packed(packed_np, B, H, cap, bits_k, bits_v):
+    """(header bytes, records [B][H][n_tiles][record]) of a host copy of a packed cache."""
+    hb = bg.header_bytes(H)
+    rec = bg.tile_record_bytes(128, bits_k, bits_v)
+    n = B * H * tiles_written(cap) * rec
+    return packed_np[:hb], packed_np[hb:hb + n].reshape(B, H, tiles_written(cap), rec)
+
+
+def check_packed(packed_np, ref_alloc, ref_records, B, H, cap, bits_k, bits_v, n_tiles=None):
+    """Header and (the first n_tiles of) the records byte for byte against the oracle."""
+    hdr, recs = split_packed(packed_np, B, H, cap, bits_k, bits_v)
+    np.testing.assert_array_equal(hdr, bg.packed_header(B, H, cap, 128, bits_k, bits_v, ref_alloc))
+    if n_tiles is None:
+        np.testing.assert_array_equal(recs, ref_records)
+    else:
+        np.testing.assert_array_equal(recs[:, :, :n_tiles], ref_records[:, :, :n_tiles])

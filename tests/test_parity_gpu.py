@@ -12,7 +12,8 @@ from oracle import blockgtq as bg
 from oracle import nqkv
 from packed_cache_attention_b200 import kvq
 from packed_cache_attention_b200 import workloads as wl
-from tests.parity_util import TOL, compare_alloc, host_f32, oracle_pipeline, rel_err, tiles_written
+from tests.parity_util import (TOL, check_packed, compare_alloc, host_f32, oracle_pipeline, rel_err, split_packed,
+                               tiles_written)
 
 pytestmark = pytest.mark.gpu
 
@@ -45,8 +46,8 @@ def run_gpu(K, V, q, bits_k, bits_v, n_calib=0, w_max=8, mode=0, capacity=None, 
 
 
 def packed_view(packed_np, B, H, cap, bits_k, bits_v):
-    rec = bg.tile_record_bytes(128, bits_k, bits_v)
-    return packed_np[:B * H * tiles_written(cap) * rec].reshape(B, H, tiles_written(cap), rec)
+    """The tile records of a host copy of a packed cache (the header skipped)."""
+    return split_packed(packed_np, B, H, cap, bits_k, bits_v)[1]
 
 
 CASES = [
@@ -70,9 +71,112 @@ def test_small_cases_match_oracle(dev, case):
     heads, packed, out, _ = run_gpu(x["K"], x["V"], x["q"], bk, bv, n_calib, w_max, mode)
     ref_alloc, ref_packed, ref_out = oracle_pipeline(x["K"], x["V"], x["q"], bk, bv, n_calib, w_max, mode)
     compare_alloc(heads, ref_alloc)
-    got = packed_view(packed, B, Hkv, T, bk, bv)
-    np.testing.assert_array_equal(got, ref_packed)
+    check_packed(packed, ref_alloc, ref_packed, B, Hkv, T, bk, bv)
     assert rel_err(out, ref_out) <= TOL
+
+
+def test_tiny_workload_seed0(dev):
+    """The tiny single-head workload exactly as stated: fp32, T 512, K3V3, seed 0."""
+    W = wl.WORKLOADS["tiny"]
+    x = wl.make_blockgtq_inputs(W.batch, W.n_q_heads, W.n_kv_heads, W.head_dim, W.seq_len, W.dtype, W.rope_base,
+                                W.key_profile, seed=0, device=dev)
+    heads, packed, out, _ = run_gpu(x["K"], x["V"], x["q"], W.bits_k, W.bits_v)
+    ref_alloc, ref_packed, ref_out = oracle_pipeline(x["K"], x["V"], x["q"], W.bits_k, W.bits_v)
+    compare_alloc(heads, ref_alloc)
+    np.testing.assert_array_equal(packed_view(packed, 1, 1, W.seq_len, W.bits_k, W.bits_v), ref_packed)
+    assert rel_err(out, ref_out) <= TOL
+
+
+def test_crafted_energy_order_and_norm_overflow(dev):
+    """Keys whose fp64 energies depend on the fixed summation order (64-token chunks, 64-chunk
+    segments, then segments): the kernel's energies equal the oracle's bit for bit. Their
+    rows of 2^26 and 2^27 have norms beyond the fp16 range, so they store norm +inf with every
+    code taken at y = 0; the packed cache equals the oracle's byte for byte."""
+    import torch
+    from tests.test_oracle_pins import crafted_energy_keys
+    Kh = crafted_energy_keys()
+    K = torch.from_numpy(Kh).to(dev).to(torch.bfloat16)
+    assert torch.equal(K.float().cpu(), torch.from_numpy(Kh))       # bf16-exact by construction
+    gen = torch.Generator(device=dev).manual_seed(3)
+    V = torch.randn(K.shape, generator=gen, device=dev).to(torch.bfloat16)
+    for mode in (0, 1):
+        heads, packed, _, _ = run_gpu(K, V, None, 3, 3, mode=mode)
+        ref_alloc, ref_packed, _ = oracle_pipeline(K, V, None, 3, 3, mode=mode)
+        compare_alloc(heads, ref_alloc)
+        np.testing.assert_array_equal(packed_view(packed, 1, 1, 8192, 3, 3), ref_packed)
+    u = bg.unpack_cache(ref_packed, ref_alloc, 3, 8192)
+    assert np.isinf(float(u["Kn"][0, 0, 0])) and np.isinf(float(u["Kn"][0, 0, 4096]))
+
+
+def _tie_rows(rng, T, widths, gains, n_ties=24):
+    """fp32 rows [T][128] in which n_ties coordinates of every row land exactly on a threshold:
+    fl32(fl32(x a) g) = t with a = fp32(sqrt 128) / fp16 norm of the row (the oracle's R5)."""
+    X = (rng.standard_normal((T, 128)) * 2.0).astype(np.float32)
+    sqd = np.float32(math.sqrt(128.0))
+    hit = np.zeros((T, 128), dtype=bool)
+    for t in range(T):
+        cols = rng.choice(128, size=n_ties, replace=False)
+        for _ in range(4):                       # the fp16 norm settles after a pass or two
+            n16 = bg.row_norms_f16(X[t][None])[0]
+            a = np.float32(sqd / np.float32(n16))
+            for j in cols:
+                w = int(widths[j])
+                if w == 0:
+                    continue
+                _, t32 = bg.codebooks.stored_codebook(w)
+                tau = t32[rng.integers(len(t32))]
+                g = np.float32(gains[j])
+                v0 = np.float32(tau / (a * g))
+                for k in range(-6, 7):
+                    v = np.float32(v0 + np.float32(k) * np.spacing(v0))
+                    if np.float32(np.float32(v * a) * g) == tau:
+                        X[t, j] = v
+                        break
+        n16 = bg.row_norms_f16(X[t][None])[0]
+        a = np.float32(sqd / np.float32(n16))
+        for j in cols:
+            w = int(widths[j])
+            if w:
+                y = np.float32(np.float32(X[t, j] * a) * np.float32(gains[j]))
+                hit[t, j] = bool(np.any(bg.codebooks.stored_codebook(w)[1] == y))
+    return X, hit
+
+
+@pytest.mark.parametrize("mode", [1, 0])
+def test_threshold_ties_at_full_head_dim(dev, mode):
+    """Coordinates exactly on a threshold at d = 128 take the lower code on the GPU as in the
+    oracle: fp32 keys and values built so that fl32(x a) (times g_b in Block-GTQ mode) equals
+    a stored threshold; the packed cache is compared byte for byte."""
+    import torch
+    rng = np.random.default_rng(77 + mode)
+    T = 64
+    x = wl.make_blockgtq_inputs(1, 2, 1, 128, T, "f32", 1e4, "loguniform", seed=8, device=dev)
+    Kh = host_f32(x["K"])
+    ref_alloc = bg.calibrate(Kh, 3, mode=mode)
+    wk = bg.widths_per_dim(ref_alloc["w"][0])
+    gk = np.concatenate([ref_alloc["g"][0], ref_alloc["g"][0]])
+    # keep the calibration input, change the rows that are quantized: calibrate on K, then
+    # quantize rows built against that allocation (the allocation only depends on K's energies)
+    Kt, hit_k = _tie_rows(rng, T, wk, gk)
+    Vt, hit_v = _tie_rows(rng, T, np.full(128, 4), np.ones(128, np.float32))
+    assert hit_k.sum() > T and hit_v.sum() > T
+    alloc = kvq.kvq_calibrate(x["K"], 3, mode=mode)
+    cache = kvq.cache_desc(1, 1, T, 3, 4)
+    Kd = torch.from_numpy(Kt).reshape(1, 1, T, 128).to(dev)
+    Vd = torch.from_numpy(Vt).reshape(1, 1, T, 128).to(dev)
+    packed = kvq.kvq_quantize(Kd, Vd, alloc, cache).cpu().numpy()
+    codes = bg.quantize(Kt.reshape(1, 1, T, 128), Vt.reshape(1, 1, T, 128), ref_alloc, 4)
+    ref_packed = bg.pack_cache(codes, ref_alloc, 4, T)
+    np.testing.assert_array_equal(packed_view(packed, 1, 1, T, 3, 4), ref_packed)
+    # the oracle took the lower code at every tie: the threshold itself is not below y
+    for X, hit, C, wd in ((Kt, hit_k, codes["Kc"][0, 0], wk), (Vt, hit_v, codes["Vc"][0, 0], np.full(128, 4))):
+        t_idx, j_idx = np.nonzero(hit)
+        for t, j in zip(t_idx[:50], j_idx[:50]):
+            _, t32 = bg.codebooks.stored_codebook(int(wd[j]))
+            n16 = bg.row_norms_f16(X[t][None])[0]
+            a = np.float32(np.float32(math.sqrt(128.0)) / np.float32(n16))
+            y = np.float32(X[t, j] * a) if X is Vt else np.float32(np.float32(X[t, j] * a) * np.float32(gk[j]))
+            assert C[t, j] == int(np.sum(t32 < y)) and np.any(t32 == y)
 
 
 def test_capacity_larger_than_tokens_and_prefix_decode(dev):
@@ -199,6 +303,115 @@ def test_append_full_size_matches_one_quantize(dev):
     assert torch.equal(grown, one)
 
 
+# ----------------------------------------------------------------------------- header, keys only, timeouts
+
+def _layer(dev, seed, T=300, Hq=8, Hkv=2, bk=3, bv=3, cap=None):
+    x = wl.make_blockgtq_inputs(1, Hq, Hkv, 128, T, "bf16", 1e6, "lognormal_outliers", seed=seed, device=dev)
+    alloc = kvq.kvq_calibrate(x["K"], bk)
+    cache = kvq.cache_desc(1, Hkv, T if cap is None else cap, bk, bv)
+    packed = kvq.kvq_quantize(x["K"], x["V"], alloc, cache)
+    return x, alloc, cache, packed
+
+
+def test_decode_refuses_another_layers_allocation(dev):
+    """The packed header names the allocation its codes were written with (per-head digest):
+    a decode given another layer's allocation, or a descriptor with other widths, records
+    KVQ_ERR_MISMATCH and leaves the output untouched."""
+    import torch
+    x, alloc, cache, packed = _layer(dev, 61)
+    _, alloc_b, _, _ = _layer(dev, 62)
+    ws = torch.zeros(kvq.kvq_decode_workspace_bytes(cache, 8), dtype=torch.uint8, device=dev)
+    out = torch.full((1, 8, 128), 12345.0, device=dev)
+    kvq.kvq_decode_attn(x["q"], packed, alloc_b, cache, 300, out=out, ws=ws)
+    assert kvq.kvq_workspace_status(ws) == kvq.KVQ_ERR_MISMATCH
+    assert torch.all(out == 12345.0)
+    kvq.kvq_workspace_init(ws)
+    other = kvq.cache_desc(1, 2, 300, 3, 2)                     # V width the cache was not written with
+    ws2 = torch.zeros(kvq.kvq_decode_workspace_bytes(other, 8), dtype=torch.uint8, device=dev)
+    kvq.kvq_decode_attn(x["q"], packed, alloc, other, 300, out=out, ws=ws2)
+    assert kvq.kvq_workspace_status(ws2) == kvq.KVQ_ERR_MISMATCH
+    assert torch.all(out == 12345.0)
+    # the right allocation still decodes, matching the oracle
+    got = kvq.kvq_decode_attn(x["q"], packed, alloc, cache, 300, ws=ws).cpu().numpy()
+    assert kvq.kvq_workspace_status(ws) == 0
+    _, _, ref = oracle_pipeline(x["K"], x["V"], x["q"], 3, 3)
+    assert rel_err(got, ref) <= TOL
+
+
+def test_append_refuses_another_allocation(dev):
+    """An append (t_begin > 0) extends only a cache whose header names its allocation: with
+    another layer's allocation it writes nothing and leaves KVQ_ERR_MISMATCH in the header,
+    which the decode then reports; quantizing from token 0 writes a fresh header."""
+    import torch
+    x, alloc, cache, packed = _layer(dev, 63, T=200, cap=256)
+    _, alloc_b, _, _ = _layer(dev, 64, T=200)
+    before = packed.clone()
+    kvq.kvq_append(x["K"][:, :, 100:150], x["V"][:, :, 100:150], alloc_b, cache, 100, packed)
+    assert kvq.kvq_packed_status(packed) == kvq.KVQ_ERR_MISMATCH
+    hb = kvq.kvq_packed_header_bytes(2)
+    assert torch.equal(packed[hb:], before[hb:])
+    ws = torch.zeros(kvq.kvq_decode_workspace_bytes(cache, 8), dtype=torch.uint8, device=dev)
+    out = torch.full((1, 8, 128), 7.0, device=dev)
+    kvq.kvq_decode_attn(x["q"], packed, alloc, cache, 200, out=out, ws=ws)
+    assert kvq.kvq_workspace_status(ws) == kvq.KVQ_ERR_MISMATCH and torch.all(out == 7.0)
+    kvq.kvq_quantize(x["K"], x["V"], alloc, cache, packed=packed)
+    assert kvq.kvq_packed_status(packed) == 0
+    assert torch.equal(packed, before)
+
+
+def test_decode_wait_timeout_is_reported(dev):
+    """Bounded waits (SURVEY failure detection, on the device): with the test hook that makes
+    the decode issue no copy at all, every warpgroup's first wait runs out with nothing in
+    flight; the call records KVQ_ERR_TIMEOUT, writes nothing, and the context stays usable."""
+    import torch
+    x, alloc, cache, packed = _layer(dev, 65, T=5000)
+    ws = torch.zeros(kvq.kvq_decode_workspace_bytes(cache, 8), dtype=torch.uint8, device=dev)
+    out = torch.full((1, 8, 128), -3.0, device=dev)
+    try:
+        kvq.kvq_debug_decode(wait_limit=3, no_loads=True)
+        kvq.kvq_decode_attn(x["q"], packed, alloc, cache, 5000, out=out, ws=ws)
+        torch.cuda.synchronize()
+    finally:
+        kvq.kvq_debug_decode(wait_limit=2000, no_loads=False)
+    assert kvq.kvq_workspace_status(ws) == kvq.KVQ_ERR_TIMEOUT
+    assert torch.all(out == -3.0)
+    kvq.kvq_workspace_init(ws)
+    got = kvq.kvq_decode_attn(x["q"], packed, alloc, cache, 5000, ws=ws).cpu().numpy()
+    assert kvq.kvq_workspace_status(ws) == 0
+    _, _, ref = oracle_pipeline(x["K"], x["V"], x["q"], 3, 3)
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_keys_only_quantize_matches_oracle(dev, dtype):
+    """A keys-only cache (bits_v = 0) holds each record's K words and K norms only, byte for
+    byte as the oracle packs them; appends in pieces store the same bytes."""
+    import torch
+    T = 150
+    x = wl.make_blockgtq_inputs(2, 8, 2, 128, T, dtype, 1e6, "lognormal_outliers", seed=66, device=dev)
+    alloc = kvq.kvq_calibrate(x["K"], 3)
+    cache = kvq.cache_desc(2, 2, 160, 3, 0)
+    packed = kvq.kvq_quantize(x["K"], None, alloc, cache)
+    Kh = host_f32(x["K"])
+    ra = bg.calibrate(Kh, 3)
+    ref = bg.pack_cache_bytes(bg.quantize(Kh, None, ra, 0), ra, 0, 160)
+    got = packed.cpu().numpy()
+    nt = tiles_written(T)
+    rec = bg.tile_record_bytes(128, 3, 0)
+    hb = bg.header_bytes(2)
+    n = 2 * 2 * tiles_written(160) * rec
+    np.testing.assert_array_equal(got[:hb], ref[:hb])
+    np.testing.assert_array_equal(got[hb:hb + n].reshape(2, 2, -1, rec)[:, :, :nt],
+                                  ref[hb:hb + n].reshape(2, 2, -1, rec)[:, :, :nt])
+    grown = torch.full_like(packed, 0x11)
+    for a, b in [(0, 1), (1, 40), (40, 64), (64, 150)]:
+        kvq.kvq_append(x["K"][:, :, a:b], None, alloc, cache, a, grown)
+    g2 = grown.cpu().numpy()
+    np.testing.assert_array_equal(g2[:hb], ref[:hb])
+    np.testing.assert_array_equal(g2[hb:hb + n].reshape(2, 2, -1, rec)[:, :, :nt],
+                                  ref[hb:hb + n].reshape(2, 2, -1, rec)[:, :, :nt])
+
+
 # ----------------------------------------------------------------------------- full-size workloads
 
 def _sample_tiles(n_tiles, k=6, seed=0):
@@ -208,7 +421,7 @@ def _sample_tiles(n_tiles, k=6, seed=0):
     return sorted(pick)
 
 
-@pytest.mark.parametrize("name", ["llama8b", "qwen3b", "batched"])
+@pytest.mark.parametrize("name", ["llama8b", "qwen3b", "qwen3b_256k", "batched"])
 def test_full_size_workloads(dev, name):
     """Full sizes, in the launch configuration the benchmark times: allocation bit-exact over
     the whole calibration set; packed records bit-exact on sampled tiles of every head;
@@ -229,9 +442,9 @@ def test_full_size_workloads(dev, name):
     ref_alloc = bg.calibrate(Kcal, W.bits_k, n_calib=0)
     compare_alloc(heads, ref_alloc)
 
-    rec = bg.tile_record_bytes(128, W.bits_k, W.bits_v)
-    nt = tiles_written(W.seq_len)
-    got = packed.cpu().numpy().reshape(W.batch, W.n_kv_heads, nt, rec)
+    hdr, got = split_packed(packed.cpu().numpy(), W.batch, W.n_kv_heads, W.seq_len, W.bits_k, W.bits_v)
+    np.testing.assert_array_equal(hdr, bg.packed_header(W.batch, W.n_kv_heads, W.seq_len, 128, W.bits_k, W.bits_v,
+                                                        ref_alloc))
     for b in sorted({0, W.batch - 1, W.batch // 2}):
         # the oracle quantizes and packs the whole sequence itself, then decodes its own cache
         codes = bg.quantize(host_f32(K[b:b + 1]), host_f32(V[b:b + 1]), ref_alloc, W.bits_v)
@@ -264,6 +477,36 @@ def test_nf4_small_cases_match_oracle(dev, case):
     np.testing.assert_array_equal(vs.view(np.uint16), rvs.view(np.uint16))
     ref = nqkv.decode(host_f32(x["q"]), rkc, rks, rvc, rvs, H, 128, T)
     assert rel_err(out, ref) <= TOL
+
+
+def test_nf4_edge_blocks(dev):
+    """NF4 special blocks, byte for byte against the oracle: an all-zero block (scale 0, every
+    index at the exact-zero level), values exactly on every midpoint of the table with the
+    block's absmax 1 (u = x, each takes the lower index), and a block whose absmax exceeds
+    the fp16 range (scale +inf, every u = 0)."""
+    import torch
+    B, H, T = 1, 4, 20
+    mids = bg.codebooks.nf4_midpoints()
+    X = np.random.default_rng(5).standard_normal((B, H, T, 128)).astype(np.float32)
+    X[0, 0:2, 3] = 0.0                                  # block 0 of token 3: all zero
+    X[0, 2:4, 4] = 0.0                                  # block 1 of token 4: midpoints, absmax 1
+    X[0, 2, 4, :15] = mids
+    X[0, 2, 4, 15] = 1.0
+    X[0, 3, 4, :15] = -mids[::-1]
+    X[0, 0, 5, 7] = 1.0e5                               # block 0 of token 5: absmax beyond fp16
+    K = torch.from_numpy(X).to(dev)
+    V = torch.from_numpy(X[:, ::-1].copy()).to(dev)
+    packed = kvq.kvq_nf4_quantize(K, V, capacity=T)
+    kc, vc, ks, vs = kvq.nf4_sections(packed.cpu().numpy(), B, H, T)
+    for got_c, got_s, Xs in ((kc, ks, X), (vc, vs, X[:, ::-1].copy())):
+        ri, rs = nqkv.quantize(Xs)
+        rc, rsc = nqkv.pack(ri, rs, T)
+        np.testing.assert_array_equal(got_c, rc)
+        np.testing.assert_array_equal(got_s.view(np.uint16), rsc.view(np.uint16))
+    ri, rs = nqkv.quantize(X)
+    assert float(rs[0, 0, 3]) == 0.0 and np.all(ri[0, 0, 3] == 7)
+    assert float(rs[0, 1, 4]) == 1.0 and list(ri[0, 1, 4, :15]) == list(range(15))
+    assert np.isinf(float(rs[0, 0, 5])) and np.all(ri[0, 0, 5] == 7)
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
