@@ -63,6 +63,7 @@ def parse():
     ap.add_argument("--seq-len", type=int, default=0, help="override the context length (profiling only)")
     ap.add_argument("--no-nf4", action="store_true", help="skip the NF4-variant measurement")
     ap.add_argument("--nf4-batch", type=int, default=0, help="override the NF4 batch (profiling only)")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload decode/quantize lines")
     return ap.parse_args()
 
 
@@ -249,6 +250,11 @@ def run_gpu(args, rank, world, local_rank):
     nf4 = (measure_nf4(kvq, wl, dev, stream, hbm_peak=peaks()[0], batch=args.nf4_batch)
            if (rank == 0 and not args.no_nf4) else None)
     append = measure_append(kvq, Ks[0], Vs[0], allocs[0], cache, packs[0], stream, T) if rank == 0 else None
+    configs = None
+    if rank == 0 and not args.no_configs:
+        del Ks, Vs
+        torch.cuda.empty_cache()
+        configs = measure_configs(kvq, wl, dev, stream, hbm_peak=peaks()[0])
 
     steps = args.steps
     ms_step = total_ms / steps
@@ -296,6 +302,7 @@ def run_gpu(args, rank, world, local_rank):
         },
         "nf4": nf4,
         "append": append,
+        "workloads": configs,
         "e2e": e2e,
         "gpu_launches": steps * L * 4,
         "clocks": clocks,
@@ -359,6 +366,94 @@ def measure_append(kvq, K, V, alloc, cache, packed, stream, T, iters=50, chunk=4
             "chunk_gb_s": B * H * chunk * per_tok / (chunk_ms * 1e-3) / 1e9, "timing": how}
 
 
+def timed_launches(fn, stream, iters, flush):
+    """Mean device time (ms) of fn() over `iters` launches, each preceded by a write of a
+    buffer larger than L2 (outside the timed interval) so every launch starts cold."""
+    import torch
+    for _ in range(3):
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for a, z in evs:
+        flush.add_(1)
+        a.record(stream)
+        fn()
+        z.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(z) for a, z in evs) / iters
+
+
+def measure_configs(kvq, wl, dev, stream, hbm_peak, iters=10):
+    """Decode and quantize/pack of the other Block-GTQ workloads, one layer each, every launch
+    after an L2 flush: Llama-3.1-8B-shaped 32K (K2V2), batched 16 x 16K (K4V4), the 128K
+    Qwen2.5-3B shape at 262144 tokens (K3V3), a keys-only K2 cache at the Llama shape (bf16
+    values), and the Qwen 128K layer with 128 recent tokens kept unquantized."""
+    import torch
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)     # 256 MB > L2
+    res = {}
+    for name in ("llama8b", "batched", "qwen3b_256k"):
+        W = wl.WORKLOADS[name]
+        x = wl.make_blockgtq_inputs(W.batch, W.n_q_heads, W.n_kv_heads, W.head_dim, W.seq_len, W.dtype,
+                                    W.rope_base, W.key_profile, seed=5, device=dev)
+        alloc = kvq.kvq_calibrate(x["K"], W.bits_k, n_calib=W.n_calib)
+        cache = kvq.cache_desc(W.batch, W.n_kv_heads, W.seq_len, W.bits_k, W.bits_v)
+        packed = kvq.kvq_quantize(x["K"], x["V"], alloc, cache)
+        out = torch.empty((W.batch, W.n_q_heads, W.head_dim), dtype=torch.float32, device=dev)
+        ws = torch.zeros(kvq.kvq_decode_workspace_bytes(cache, W.n_q_heads), dtype=torch.uint8, device=dev)
+        d_ms = timed_launches(lambda: kvq.kvq_decode_attn(x["q"], packed, alloc, cache, W.seq_len, out=out, ws=ws,
+                                                          stream=stream), stream, iters, flush)
+        q_ms = timed_launches(lambda: kvq.kvq_quantize(x["K"], x["V"], alloc, cache, packed=packed, stream=stream),
+                              stream, iters, flush)
+        assert kvq.kvq_workspace_status(ws) == 0
+        tok = W.batch * W.seq_len
+        rec = (kvq.kvq_packed_bytes(cache) - kvq.kvq_packed_header_bytes(W.n_kv_heads))
+        qb = W.batch * W.n_kv_heads * W.seq_len * W.head_dim * 2 * 2 + rec
+        res[name] = {"workload": f"{name}: B{W.batch} Hq{W.n_q_heads} Hkv{W.n_kv_heads} T{W.seq_len} K{W.bits_k}V{W.bits_v}",
+                     "decode": {"launch_ms": d_ms, "bytes_per_launch": rec, "gb_s": rec / (d_ms * 1e-3) / 1e9,
+                                "kv_tokens_per_s": tok / (d_ms * 1e-3)},
+                     "quantize": {"launch_ms": q_ms, "bytes_per_launch": qb, "gb_s": qb / (q_ms * 1e-3) / 1e9,
+                                  "tokens_per_s": tok / (q_ms * 1e-3)}}
+        for k in ("decode", "quantize"):
+            res[name][k]["hbm_frac"] = res[name][k]["gb_s"] / hbm_peak
+        if name == "llama8b":
+            # keys only: K2 codes packed, values read as bf16
+            ck = kvq.cache_desc(W.batch, W.n_kv_heads, W.seq_len, W.bits_k, 0)
+            pk = kvq.kvq_quantize(x["K"], None, alloc, ck)
+            wk = torch.zeros(kvq.kvq_decode_workspace_bytes(ck, W.n_q_heads), dtype=torch.uint8, device=dev)
+            k_ms = timed_launches(lambda: kvq.kvq_decode_attn_ex(x["q"], pk, alloc, ck, W.seq_len, V=x["V"], out=out,
+                                                                 ws=wk, stream=stream), stream, iters, flush)
+            assert kvq.kvq_workspace_status(wk) == 0
+            kb = (kvq.kvq_packed_bytes(ck) - kvq.kvq_packed_header_bytes(W.n_kv_heads)) + x["V"].numel() * 2
+            res["keys_only_llama8b"] = {"workload": f"llama8b keys only: K{W.bits_k}, bf16 values",
+                                        "decode": {"launch_ms": k_ms, "bytes_per_launch": kb,
+                                                   "gb_s": kb / (k_ms * 1e-3) / 1e9,
+                                                   "hbm_frac": kb / (k_ms * 1e-3) / 1e9 / hbm_peak}}
+        del x, packed, out, ws, alloc
+        torch.cuda.empty_cache()
+    # recent tokens kept unquantized: the 128K layer plus 128 bf16 tokens
+    W = wl.WORKLOADS["qwen3b"]
+    R = 128
+    x = wl.make_blockgtq_inputs(W.batch, W.n_q_heads, W.n_kv_heads, W.head_dim, W.seq_len, W.dtype, W.rope_base,
+                                W.key_profile, seed=6, device=dev)
+    alloc = kvq.kvq_calibrate(x["K"], W.bits_k)
+    cache = kvq.cache_desc(W.batch, W.n_kv_heads, W.seq_len, W.bits_k, W.bits_v)
+    packed = kvq.kvq_quantize(x["K"], x["V"], alloc, cache)
+    Kr = x["K"][:, :, -R:].contiguous()
+    Vr = x["V"][:, :, -R:].contiguous()
+    out = torch.empty((W.batch, W.n_q_heads, W.head_dim), dtype=torch.float32, device=dev)
+    ws = torch.zeros(kvq.kvq_decode_workspace_bytes(cache, W.n_q_heads), dtype=torch.uint8, device=dev)
+    r_ms = timed_launches(lambda: kvq.kvq_decode_attn_ex(x["q"], packed, alloc, cache, W.seq_len, K_recent=Kr,
+                                                         V_recent=Vr, out=out, ws=ws, stream=stream),
+                          stream, iters, flush)
+    assert kvq.kvq_workspace_status(ws) == 0
+    rb = (kvq.kvq_packed_bytes(cache) - kvq.kvq_packed_header_bytes(W.n_kv_heads)) + 2 * Kr.numel() * 2
+    res["recent_qwen3b"] = {"workload": f"qwen3b 128K + {R} recent bf16 tokens",
+                            "decode": {"launch_ms": r_ms, "bytes_per_launch": rb, "gb_s": rb / (r_ms * 1e-3) / 1e9,
+                                       "hbm_frac": rb / (r_ms * 1e-3) / 1e9 / hbm_peak}}
+    del x, packed, out, ws, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_nf4(kvq, wl, dev, stream, hbm_peak, iters=10, batch=0):
     """NQKV-style NF4 variant at the OPT-30B shape (one layer: B8 x 56 heads x 8192 tokens,
     fp16), timed outside the step: quantize/pack and MHA decode, CUDA events per launch."""
@@ -401,34 +496,62 @@ def measure_nf4(kvq, wl, dev, stream, hbm_peak, iters=10, batch=0):
 
 # ------------------------------------------------------------------------------------------ CPU oracle
 
-def oracle_sample(n_tokens: int, seed: int = 0):
+def oracle_sample(n_tokens: int, seed: int = 0, workload: str = WORKLOAD, batch: int = 0):
     """Time the oracle's calibrate + quantize/pack + decode on the first n_tokens of one layer
-    of the workload (both KV heads, all 16 q-heads). Returns (seconds, layer-tokens)."""
+    of a workload (all KV heads and q-heads; `batch` sequences, default the workload's).
+    Returns (seconds, layer-tokens)."""
     import numpy as np
     import torch
     from oracle import blockgtq as bg
     from packed_cache_attention_b200 import workloads as wl
-    W = wl.WORKLOADS[WORKLOAD]
-    x = wl.make_blockgtq_inputs(W.batch, W.n_q_heads, W.n_kv_heads, W.head_dim, n_tokens, W.dtype, W.rope_base,
+    W = wl.WORKLOADS[workload]
+    B = batch or W.batch
+    x = wl.make_blockgtq_inputs(B, W.n_q_heads, W.n_kv_heads, W.head_dim, n_tokens, W.dtype, W.rope_base,
                                 W.key_profile, seed=seed, device="cpu")
     K = x["K"].float().numpy()
     V = x["V"].float().numpy()
     q = x["q"].float().numpy()
     t0 = time.perf_counter()
-    alloc = bg.calibrate(K, W.bits_k)
+    alloc = bg.calibrate(K, W.bits_k, n_calib=min(W.n_calib, n_tokens) if W.n_calib else 0)
     codes = bg.quantize(K, V, alloc, W.bits_v)
     packed = bg.pack_cache(codes, alloc, W.bits_v, n_tokens)
     bg.decode(q, packed, alloc, W.bits_v, n_tokens)
-    return time.perf_counter() - t0, W.batch * n_tokens
+    return time.perf_counter() - t0, B * n_tokens
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def cpu_baseline(n_tokens: int = 131072):
+    """The oracle on the host cores: the 128K layer on one core, then bounded samples of every
+    Block-GTQ workload on one core and with numpy's default thread count (all cores)."""
     from threadpoolctl import threadpool_limits
     with threadpool_limits(limits=1):
         secs, toks = oracle_sample(n_tokens)
+    ncpu = os.cpu_count() or 1
+    per = {}
+    samples = {"tiny": (512, 0), "llama8b": (4096, 0), "qwen3b": (8192, 0), "batched": (2048, 2)}
+    for name, (n, bsz) in samples.items():
+        row = {}
+        for label, lim in (("one_core", 1), ("all_cores", None)):
+            with threadpool_limits(limits=lim):
+                sec, tk = oracle_sample(n, workload=name, batch=bsz)
+            row[label] = tk / sec
+        row["sample"] = f"first {n} tokens" + (f" of {bsz} sequences" if bsz else "")
+        per[name] = row
     return {"value": toks / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"one layer of {WORKLOAD}, first {n_tokens} tokens of both KV heads: calibrate + quantize/pack "
-                      f"+ decode for 16 q-heads ({secs:.1f} s)"}
+                      f"+ decode for 16 q-heads ({secs:.1f} s)",
+            "host": {"nproc": ncpu, "cpu_model": cpu_model()},
+            "per_workload_layer_tokens_per_s": per}
 
 
 def run_reference(args, rank, world):

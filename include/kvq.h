@@ -294,12 +294,12 @@ kvq_status kvq_decode_attn(const void* q, const kvq_tensor4* qd, const void* pac
                            size_t ws_bytes, void* stream);
 
 /* Extra inputs of kvq_decode_attn_ex. Every pointer may be NULL (then its view is ignored).
- * V, vd: the values of a keys-only cache (cache->bits_v = 0; the Block-GTQ page quotes its key
- *   error "K-only", with values left unquantized): [batch][n_kv_heads][>= seq_len][128] in
- *   bf16 or fp16, row t = value of cached position t. Required for a keys-only cache, not
+ * V, vd: the values of a keys-only cache (cache->bits_v = 0; the Block-GTQ page reports key
+ *   errors with only the keys quantized, values left as they are):
+ *   [batch][n_kv_heads][>= seq_len][128] in bf16 or fp16, row t = value of cached position t. Required for a keys-only cache, not
  *   allowed with packed values.
  * K_recent, V_recent, krd, vrd: the n_recent = krd.seq_len most recent tokens kept
- *   unquantized (the Block-GTQ page reports its results "without an fp16 recent-key buffer",
+ *   unquantized (the Block-GTQ page reports its results with no buffer of fp16 recent keys,
  *   which names this variant; here both their keys and values stay in the caller's dtype):
  *   [batch][n_kv_heads][n_recent][128] each, any dtype; they are cached positions seq_len ..
  *   seq_len + n_recent - 1 and join the packed positions in one softmax. */
@@ -316,7 +316,9 @@ typedef struct {
  * and recent positions of softmax(q . k / sqrt(d)) v, where packed positions use k_hat (and
  * v_hat, or the dense values of a keys-only cache) and recent positions their exact k and v.
  * seq_len may be 0 when n_recent >= 1. Same workspace, header checks and status as
- * kvq_decode_attn; extra = NULL is kvq_decode_attn. */
+ * kvq_decode_attn; extra = NULL is kvq_decode_attn. A keys-only cache above 4 bits per dim
+ * returns KVQ_ERR_UNSUPPORTED (its chunk stages, 128 value rows each, do not fit in the
+ * decode's shared memory). */
 kvq_status kvq_decode_attn_ex(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
                               const kvq_cache_desc* cache, int seq_len, const kvq_decode_extra* extra, float* out,
                               void* ws, size_t ws_bytes, void* stream);

@@ -520,11 +520,11 @@ def decode(q: np.ndarray, packed: np.ndarray, alloc: dict, bits_v: int, seq_len:
            V_recent=None) -> np.ndarray:
     """Fused-path reference: unpack the stored bits, dequantize, attend (fp64).
 
-    Keys-only cache (bits_v = 0; the Block-GTQ page quotes its key error "K-only"): the
-    values of positions 0..seq_len-1 are the stored values V [B][Hkv][>= seq_len][d], taken
-    exactly. Recent-token buffer (reading: the Block-GTQ page reports its results without an
-    fp16 recent-key buffer, which names the variant; here the R most recent tokens keep
-    their keys and values unquantized): K_recent, V_recent [B][Hkv][R][d] hold positions
+    Keys-only cache (bits_v = 0; the Block-GTQ page reports key errors with only the keys
+    quantized): the values of positions 0..seq_len-1 are the stored values V
+    [B][Hkv][>= seq_len][d], taken exactly. Recent-token buffer (reading: the Block-GTQ page
+    reports its results with no buffer of fp16 recent keys, which names the variant; here the
+    R most recent tokens keep their keys and values unquantized): K_recent, V_recent [B][Hkv][R][d] hold positions
     seq_len .. seq_len + R - 1, attended in the same softmax with their exact values.
     seq_len may be 0 when R > 0.
     """

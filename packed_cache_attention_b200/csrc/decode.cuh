@@ -4,38 +4,41 @@
 //
 // Grid: (splits, batch * n_kv_heads), one CTA per SM. A CTA owns a contiguous range of
 // 128-token chunks (4 tile records, contiguous in memory) of one (sequence, KV head).
-// Four compute warpgroups each run their own chunk pipeline over chunks g, g + 4, g + 8, ..
-// of the range, so no warpgroup waits for another:
-//   load     the warpgroup's leader bulk-copies whole chunks (one copy of 4 records) into its
-//            own ring of stages, several chunks ahead;
-//   keys     lane = token: the K codes of each slot of the allocation's plan (4 block pairs of
-//            one width) are looked up in shared-memory pair tables and written to tensor
-//            memory, 16 columns per store (K-hat rows, one fp16 pair per column);
-//   S        the leader issues S^T[128 tokens][16] = Khat x Q'^T (tcgen05.mma, M 128, N 16;
-//            Q' rows 0-7 the fp16 high parts of the 8 query rows, rows 8-15 the low parts);
-//   values   lane = dim: the chunk's V codes go to tensor memory over the K-hat columns
-//            (V-hat^T rows, one fp16 pair of tokens per column);
+// Four warpgroups each run their own chunk pipeline over chunks g, g + 4, g + 8, .. of the
+// range, each with four compute warps (warps 4g .. 4g + 3, warp % 4 = tensor-memory quarter)
+// and one issuer warp (warp 16 + g) whose first lane issues every copy and product:
+//   load     whole chunks (one bulk copy of 4 records) into the warpgroup's ring of stages,
+//            several chunks ahead;
+//   keys     lane = token: 16 K-hat columns at a time (4 slots of the allocation's plan, each
+//            4 block pairs of one width, looked up in shared-memory pair tables) go to a ring
+//            of two 16-column tensor-memory buffers; the issuer runs S^T[128 tokens][16] +=
+//            Khat x Q'^T (tcgen05.mma, M 128, N 16; Q' rows 0-7 fp16 high parts, 8-15 low
+//            parts) on each buffer as soon as it is full, while the next one is filled;
+//   values   lane = dim: V-hat^T rows (one fp16 pair of tokens per column) go to their own 64
+//            columns while the S products run;
 //   softmax  lane = token: logits s = S * key norm * 2^e (per row), the chunk's maximum per
-//            row over the warpgroup, and an online softmax whose running maximum is only raised
-//            when a chunk exceeds it by more than 2^8 (then O is rescaled in tensor memory);
-//            P' = 2^(s - m - 8) * value norm / sqrt(d), split into fp16 hi + lo, is the B
-//            operand of O;
-//   O        the leader issues O^T[128 dims][16] += Vhat^T x P'^T, accumulated over all of
-//            the warpgroup's chunks in tensor memory.
+//            row over the warpgroup, and an online softmax whose running maximum is only
+//            raised when a chunk exceeds it by more than 2^8 (then O is rescaled in tensor
+//            memory); P' = 2^(s - m - 8) * value norm / sqrt(d), split into fp16 hi + lo, is
+//            the B operand of O;
+//   O        the issuer runs O^T[128 dims][16] += Vhat^T x P'^T, accumulated over all of the
+//            warpgroup's chunks in tensor memory.
+// One issuing thread can have one product in flight at a time (about 130 cycles each at
+// these shapes), so four issuers keep four independent chains going.
 // Q' carries f_b, log2(e)/sqrt(d) and a per-row power of two that keeps its fp16 split in
 // range. The four warpgroups' (m, l, O) are combined in shared memory; splits then meet in a
 // two-level tree: the last CTA of each group of about sqrt(splits) splits (atomic ticket)
 // merges the group, and the last group to finish merges the groups and writes out = O / l.
-// Keys-only caches (the Block-GTQ page quotes its key error "K-only"): the values of each
+// Keys-only caches (the Block-GTQ page reports key errors with only the keys quantized): the values of each
 // chunk arrive as dense bf16/fp16 rows next to the chunk's K records and are transposed into
 // tensor memory (lane = dim); O then runs on bf16 (or fp16) operands with P' split to match.
-// Recent tokens kept unquantized (reading of the page's "fp16 recent-key buffer"): the three
-// helper warps of every CTA, once Q' is built, attend over an even share of them on CUDA
-// cores (lane = 4 dims) and add a fifth partial to the CTA's combine.
+// Recent tokens kept unquantized (our reading of the recent-token buffer the page names): the issuer
+// warps of every CTA, once their products are issued, attend over an even share of them on
+// CUDA cores (lane = 4 dims) and add a fifth partial to the CTA's combine.
 // Every wait is bounded. A wait that gives up records KVQ_ERR_TIMEOUT and stops the
-// warpgroup at its next barrier; the CTA waits (bounded) for its copies and products in
-// flight, frees tensor memory and writes nothing. A packed header or allocation that does
-// not match the call records KVQ_ERR_MISMATCH and writes nothing either.
+// warpgroup; the CTA waits (bounded) for its copies and products in flight, frees tensor
+// memory and writes nothing. A packed header or allocation that does not match the call
+// records KVQ_ERR_MISMATCH and writes nothing either.
 #pragma once
 
 #include "common.cuh"
@@ -43,9 +46,9 @@
 
 namespace kvq {
 
-constexpr int kDecWG = 4;                 // compute warpgroups
-constexpr int kDecWgWarp0 = 4;            // first compute warp (warp % 4 = tensor-memory quarter)
-constexpr int kDecThreads = (kDecWgWarp0 + 4 * kDecWG) * 32;
+constexpr int kDecWG = 4;                 // warpgroups
+constexpr int kDecIssuerWarp0 = 4 * kDecWG;   // issuer warp of warpgroup g: 16 + g
+constexpr int kDecThreads = 5 * kDecWG * 32;
 constexpr int kChunkTiles = 4;
 constexpr int kChunkTokens = kChunkTiles * kTile;   // = MMA M = tensor-memory lanes
 constexpr int kStagesMax = 4;             // chunk stages per warpgroup
@@ -56,21 +59,23 @@ constexpr int kMergeMax = 64;             // entries one merge step reads
 constexpr uint32_t kHeaderMagic = 0x3151564Bu;   // "KVQ1"
 constexpr int kLayoutVersion = 1;
 
-// Tensor-memory columns of warpgroup g: A (K-hat, then V-hat^T) 96, S 16, O 16.
-__device__ __forceinline__ uint32_t col_a(int g) { return 128u * g; }
+// Tensor-memory columns of warpgroup g: K-hat ring 2 x 16, V-hat^T 64, S 16, O 16.
+__device__ __forceinline__ uint32_t col_k(int g, int slot) { return 128u * g + 16u * slot; }
+__device__ __forceinline__ uint32_t col_v(int g) { return 128u * g + 32u; }
 __device__ __forceinline__ uint32_t col_s(int g) { return 128u * g + 96u; }
 __device__ __forceinline__ uint32_t col_o(int g) { return 128u * g + 112u; }
 
 // Lookup-table image, built once per device (decode_lut_image) and bulk-copied into every
-// CTA's shared memory at byte 0. Pair tables give the fp16 pair {c[i & m], c[i >> w]} for the
-// 2w-bit index i of two consecutive codes: widths 1..3 keep one copy per lane (entry e of
-// lane l at word 32 e + l) so that 32 lanes never share a bank; widths 4..6 keep one copy;
-// widths 7, 8 use single-code fp16 tables.
+// CTA's shared memory at byte 0. Widths 1..3 keep pair tables: the fp16 pair {c[i & m], c[i >> w]}
+// for the 2w-bit index i of two consecutive codes. Widths 4..6 keep single-code tables (c[e] in
+// the low half of a word). Both keep one copy per lane (entry e of lane l at word 32 e + l),
+// so the 32 lanes of a warp never share a bank whatever codes they look up. Widths 7 and 8
+// (rare: the highest-energy blocks) use single fp16 tables shared by all lanes.
 __host__ __device__ constexpr int lut_off(int w) {
-  return w == 1 ? 0 : w == 2 ? 512 : w == 3 ? 2560 : w == 4 ? 10752 : w == 5 ? 11776 : w == 6 ? 15872
-                                                                                       : w == 7 ? 32256 : 32512;
+  return w == 1 ? 0 : w == 2 ? 512 : w == 3 ? 2560 : w == 4 ? 10752 : w == 5 ? 12800 : w == 6 ? 16896
+                                                                                       : w == 7 ? 25088 : 25344;
 }
-constexpr int kLutBytes = 33024;
+constexpr int kLutBytes = 25856;
 // Shared-memory map (byte offsets from the start of dynamic shared memory).
 constexpr int kAllocOff = kLutBytes;                 // copy of the KV head's kvq_head_alloc
 constexpr int kBQOff = ((kAllocOff + static_cast<int>(sizeof(kvq_head_alloc)) + 127) / 128) * 128;
@@ -85,25 +90,29 @@ static_assert(kLutBytes % 16 == 0 && kAllocOff % 16 == 0 && sizeof(kvq_head_allo
 static_assert(sizeof(kvq_head_alloc) == 2048 && sizeof(kvq_packed_header) == 64, "ABI record sizes");
 
 struct DecHeader {
-  uint64_t full[kDecWG][kStagesMax];
-  uint64_t sfull[kDecWG];
-  uint64_t ofull[kDecWG];
-  uint64_t setup;                    // lookup tables + allocation record copied in
-  uint64_t qready;                   // Q' and qscale written
+  uint64_t full[kDecWG][kStagesMax];   // chunk stage loaded
+  uint64_t kready[kDecWG][2];          // K-hat ring buffer filled (4 compute warps)
+  uint64_t kfree[kDecWG][2];           // K-hat ring buffer read by its S products
+  uint64_t sfull[kDecWG];              // S of the chunk complete
+  uint64_t vready[kDecWG];             // V-hat^T and P' written (4 compute warps)
+  uint64_t ofull[kDecWG];              // O products of the chunk complete
+  uint64_t drain[kDecWG];              // every product the issuer committed is complete
+  uint64_t setup;                      // lookup tables + allocation record copied in
+  uint64_t qready;                     // Q' and qscale written
   uint32_t tmem_base;
-  int bad;                           // header or allocation mismatch: the CTA writes nothing
-  int wg_abort[kDecWG];              // a wait of this warpgroup gave up
-  float qscale[8];                   // 2^e that undoes the range scaling of Q' row h
-  float xch[kDecWG][4][8];           // chunk maximum: [warpgroup][warp][row]
-  float lred[kDecWG][4][8];          // row sums: [warpgroup][warp][row]
-  float wg_m[kDecWG + 1][8];         // warpgroup (and recent-token) results: maximum
-  float wg_l[kDecWG + 1][8];         //                                        and row sum
-  float rx_m[3][8];                  // recent tokens: per helper warp maximum
-  float rx_l[3][8];                  //                              and row sum
+  int bad;                             // header or allocation mismatch: the CTA writes nothing
+  int wg_abort[kDecWG];                // a wait of this warpgroup gave up
+  float qscale[8];                     // 2^e that undoes the range scaling of Q' row h
+  float xch[kDecWG][4][8];             // chunk maximum: [warpgroup][warp][row]
+  float lred[kDecWG][4][8];            // row sums: [warpgroup][warp][row]
+  float wg_m[kDecWG + 1][8];           // warpgroup (and recent-token) results: maximum
+  float wg_l[kDecWG + 1][8];           //                                        and row sum
+  float rx_m[4][8];                    // recent tokens: per issuer warp maximum
+  float rx_l[4][8];                    //                                and row sum
   int last;
-  float mw[8][kMergeMax];            // merge: member maxima, then weights
-  float ml[8][kMergeMax];            //        member row sums
-  float Msum[8][2];                  //        merged maximum and row sum
+  float mw[8][kMergeMax];              // merge: member maxima, then weights
+  float ml[8][kMergeMax];              //        member row sums
+  float Msum[8][2];                    //        merged maximum and row sum
 };
 
 __host__ __device__ constexpr int decode_stage_off() {
@@ -115,13 +124,18 @@ __host__ __device__ constexpr int chunk_bytes(int rec_bytes) { return kChunkTile
 
 // Host: the lookup-table image from the fp16 centroid table (width w at c16 + 2^w - 2).
 inline void decode_lut_image(const uint16_t* c16, uint8_t* img) {
-  for (int w = 1; w <= 6; ++w) {
+  for (int w = 1; w <= 3; ++w) {
     const uint16_t* c = c16 + (1 << w) - 2;
     uint32_t* t = reinterpret_cast<uint32_t*>(img + lut_off(w));
-    const int copies = (w <= 3) ? 32 : 1;
     for (int e = 0; e < (1 << (2 * w)); ++e)
-      for (int l = 0; l < copies; ++l)
-        t[e * copies + l] = static_cast<uint32_t>(c[e & ((1 << w) - 1)]) | (static_cast<uint32_t>(c[e >> w]) << 16);
+      for (int l = 0; l < 32; ++l)
+        t[e * 32 + l] = static_cast<uint32_t>(c[e & ((1 << w) - 1)]) | (static_cast<uint32_t>(c[e >> w]) << 16);
+  }
+  for (int w = 4; w <= 6; ++w) {
+    const uint16_t* c = c16 + (1 << w) - 2;
+    uint32_t* t = reinterpret_cast<uint32_t*>(img + lut_off(w));
+    for (int e = 0; e < (1 << w); ++e)
+      for (int l = 0; l < 32; ++l) t[e * 32 + l] = static_cast<uint32_t>(c[e]);
   }
   for (int w = 7; w <= 8; ++w) {
     uint16_t* t = reinterpret_cast<uint16_t*>(img + lut_off(w));
@@ -149,14 +163,17 @@ __device__ __forceinline__ uint32_t field_at(uint32_t lo, uint32_t hi, int p, in
 }
 
 // fp16 pair for two consecutive codes: code_a = bits [p, p + W), code_b = bits [p + W, p + 2W)
-// of hi:lo; code_a goes to the low half. The pair index lands directly at its table offset
-// (x 128 bytes plus the lane's word for the per-lane copies, x 4 bytes otherwise).
+// of hi:lo; code_a goes to the low half. Widths 1..3: the pair index lands directly at its
+// table offset (x 128 bytes plus the lane's word); widths 4..6: two per-lane single-code
+// lookups joined by a byte permute; widths 7, 8: two shared single-code lookups.
 template <int W>
 __device__ __forceinline__ uint32_t pair_value(uint32_t lo, uint32_t hi, int p, const uint8_t* sm, uint32_t lane4) {
   if constexpr (W <= 3) {
     return *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + (field_at(lo, hi, p, 2 * W, 7) | lane4));
   } else if constexpr (W <= 6) {
-    return *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + field_at(lo, hi, p, 2 * W, 2));
+    const uint32_t a = *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + (field_at(lo, hi, p, W, 7) | lane4));
+    const uint32_t b = *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + (field_at(lo, hi, p + W, W, 7) | lane4));
+    return __byte_perm(a, b, 0x5410);
   } else {
     const uint8_t* t = sm + lut_off(W);
     return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(t + field_at(lo, hi, p, W, 1))) |
@@ -194,6 +211,46 @@ __device__ __forceinline__ void k_slot(uint32_t e, const uint32_t* kw, const uin
     case 8: k_group_vals<8>(kw, off, sm, lane4, t); break;
     default: t[0] = 0u; t[1] = 0u; t[2] = 0u; t[3] = 0u; break;
   }
+}
+
+// Lookups of one slot whose 2 aligned stream words r0:r1 (the slot's first code at bit 0) are
+// already in registers: width W from the slot entry e (0: an empty slot, zeros).
+__device__ __forceinline__ void k_slot_vals(uint32_t e, uint32_t r0, uint32_t r1, const uint8_t* sm, uint32_t lane4,
+                                            uint32_t* v) {
+  switch (e & 15u) {
+#define KVQ_SLOT_CASE(W) \
+  case W:                \
+    _Pragma("unroll") for (int k = 0; k < 4; ++k) v[k] = pair_value<W>(r0, r1, 2 * W * k, sm, lane4); break;
+    KVQ_SLOT_CASE(1)
+    KVQ_SLOT_CASE(2)
+    KVQ_SLOT_CASE(3)
+    KVQ_SLOT_CASE(4)
+    KVQ_SLOT_CASE(5)
+    KVQ_SLOT_CASE(6)
+    KVQ_SLOT_CASE(7)
+    KVQ_SLOT_CASE(8)
+#undef KVQ_SLOT_CASE
+    default: v[0] = 0u; v[1] = 0u; v[2] = 0u; v[3] = 0u; break;
+  }
+}
+
+// 16 K-hat columns (4 plan slots) of this lane's token. The stream words of all four slots
+// are loaded and aligned before any width is dispatched, so the loads of one batch overlap
+// and only the table lookups follow the per-slot switch. kw points at word 0 of the token
+// (word i at kw[32 i]); every slot reads three words (the third lies inside the record).
+__device__ __forceinline__ void k_batch(const uint32_t* kw, uint4 e4, const uint8_t* sm, uint32_t lane4,
+                                        uint32_t (&v)[16]) {
+  const uint32_t e[4] = {e4.x, e4.y, e4.z, e4.w};
+  uint32_t r0[4], r1[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t off = e[i] >> 8, j0 = off >> 5, sh = off & 31u;
+    const uint32_t x0 = kw[j0 * 32], x1 = kw[(j0 + 1) * 32], x2 = kw[(j0 + 2) * 32];
+    r0[i] = __funnelshift_r(x0, x1, sh);
+    r1[i] = __funnelshift_r(x1, x2, sh);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) k_slot_vals(e[i], r0[i], r1[i], sm, lane4, v + 4 * i);
 }
 
 // V-hat^T row of one dim for one tile: 16 token pairs (2u, 2u+1) -> 16 columns.
@@ -369,37 +426,71 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   const float inv_sqrt_d = 0.08838834764831845f;
   const uint32_t WL = a.wait_limit;
 
-  // ------------------------------------------------------------------ barriers, TMEM
+  // roles: compute warps 0..15 (warpgroup g = warp / 4, quarter q = warp % 4), issuer warps 16..19
+  const bool is_issuer = warp >= kDecIssuerWarp0;
+  const int g = is_issuer ? warp - kDecIssuerWarp0 : warp >> 2;
+  const int q = warp & 3;
+  const bool issuer = is_issuer && lane == 0;
+  const int nj = (n_chunks > g) ? (n_chunks - g + kDecWG - 1) / kDecWG : 0;   // this warpgroup's chunks
+  uint8_t* my_stages = stages + static_cast<size_t>(g) * NS * cbytes;
+
+  // ------------------------------------------------------------------ barriers, TMEM, setup copy
   if (tid == 0) {
-    for (int g = 0; g < kDecWG; ++g) {
-      for (int i = 0; i < kStagesMax; ++i) tc::mbar_init(&S.full[g][i], 1);
-      tc::mbar_init(&S.sfull[g], 1);
-      tc::mbar_init(&S.ofull[g], 1);
-      S.wg_abort[g] = 0;
+    for (int gg = 0; gg < kDecWG; ++gg) {
+      for (int i = 0; i < kStagesMax; ++i) tc::mbar_init(&S.full[gg][i], 1);
+      for (int i = 0; i < 2; ++i) {
+        tc::mbar_init(&S.kready[gg][i], 4);
+        tc::mbar_init(&S.kfree[gg][i], 1);
+      }
+      tc::mbar_init(&S.sfull[gg], 1);
+      tc::mbar_init(&S.vready[gg], 4);
+      tc::mbar_init(&S.ofull[gg], 1);
+      tc::mbar_init(&S.drain[gg], 1);
+      S.wg_abort[gg] = 0;
     }
     tc::mbar_init(&S.setup, 1);
     tc::mbar_init(&S.qready, 1);
     S.bad = 0;
     tc::mbar_fence_init();
+    tc::mbar_arrive_expect_tx(&S.setup, kLutBytes + static_cast<uint32_t>(sizeof(kvq_head_alloc)));
+    tc::bulk_g2s(sm, g_dec_lut, kLutBytes, &S.setup);
+    tc::bulk_g2s(sm + kAllocOff, al, sizeof(kvq_head_alloc), &S.setup);
   }
-  if (tid < 8) S.wg_m[kDecWG][tid] = -INFINITY;             // no recent share unless the helpers add one
-  if (warp == 0) tc::tmem_alloc(&S.tmem_base, kTmemCols);
+  if (tid < 8) S.wg_m[kDecWG][tid] = -INFINITY;             // no recent share unless the issuers add one
+  if (warp == kDecIssuerWarp0) tc::tmem_alloc(&S.tmem_base, kTmemCols);
+  if (tid == 32) {
+    // The packed header must name this layout, these widths and shapes, and this head's
+    // allocation; a status left by an append is reported as is. All fields are loaded
+    // before any is compared, so the loads overlap.
+    const uint4 h0 = *reinterpret_cast<const uint4*>(a.packed);
+    const uint4 h1 = *reinterpret_cast<const uint4*>(a.packed + 16);
+    const uint64_t dg = reinterpret_cast<const uint64_t*>(a.packed + sizeof(kvq_packed_header))[hkv];
+    const uint64_t ad = al->digest;
+    const int abk = al->bits_k, akw = al->k_words, apk = al->plan_k_cols, aps = al->plan_n_slots;
+    const uint32_t want2 = static_cast<uint32_t>(a.bits_k) | (static_cast<uint32_t>(a.bits_v) << 8);
+    unsigned code = 0;
+    if (h0.w != 0) {
+      code = h0.w;                                          // status left by an append
+    } else {
+      const bool ok = (h0.x == kHeaderMagic) & (h0.y == (static_cast<uint32_t>(kLayoutVersion) | (kD << 16))) &
+                      ((h0.z & 0xffffu) == want2) & (static_cast<int>(h1.x) == a.batch) &
+                      (static_cast<int>(h1.y) == a.n_kv_heads) & (static_cast<int>(h1.z) == a.capacity) &
+                      (static_cast<int>(h1.w) == a.rec_bytes) & (dg == ad) & (abk == a.bits_k) &
+                      (akw == a.bits_k * kD) & (apk <= 96) & (apk >= 8) & (aps <= kPlanSlots);
+      if (!ok) code = KVQ_ERR_MISMATCH;
+    }
+    if (code) {
+      S.bad = 1;
+      record_status(a.status, code);
+    }
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = S.tmem_base;
 
-  // Warpgroup coordinates (compute warps only).
-  const bool is_wg = warp >= kDecWgWarp0;
-  const int g = is_wg ? (warp - kDecWgWarp0) >> 2 : 0;
-  const int q = warp & 3;                                   // tensor-memory quarter
-  const int tid_wg = tid - 32 * kDecWgWarp0 - 128 * g;
-  const bool leader = is_wg && tid_wg == 0;
-  const int nj = (is_wg && n_chunks > g) ? (n_chunks - g + kDecWG - 1) / kDecWG : 0;   // this warpgroup's chunks
-  uint8_t* my_stages = stages + static_cast<size_t>(g) * NS * cbytes;
-  int issued = 0;                                           // chunks whose copy the leader has issued
-
-  auto issue_chunk = [&](int j) {                           // leader only
+  int issued = 0;                                           // chunks whose copy this issuer started
+  auto issue_chunk = [&](int j) {                           // issuer only
     const int ci = c_begin + g + kDecWG * j;
     const int tile0 = ci * kChunkTiles;
     const int nt = min(kChunkTiles, n_tiles - tile0);
@@ -426,34 +517,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
       }
     }
   };
-
   // First copies go out before anything else, so HBM is busy from the start.
-  if (leader && !a.debug_no_loads) {
+  if (issuer && !S.bad && !a.debug_no_loads) {
     for (; issued < min(NS, nj); ++issued) issue_chunk(issued);
-  }
-  if (tid == 0) {
-    tc::mbar_arrive_expect_tx(&S.setup, kLutBytes + static_cast<uint32_t>(sizeof(kvq_head_alloc)));
-    tc::bulk_g2s(sm, g_dec_lut, kLutBytes, &S.setup);
-    tc::bulk_g2s(sm + kAllocOff, al, sizeof(kvq_head_alloc), &S.setup);
-  }
-  if (tid == 32) {
-    // The packed header must name this layout, these widths and shapes, and this head's
-    // allocation; a status left by an append is reported as is.
-    const kvq_packed_header* H = reinterpret_cast<const kvq_packed_header*>(a.packed);
-    const uint64_t* dig = reinterpret_cast<const uint64_t*>(a.packed + sizeof(kvq_packed_header));
-    unsigned code = 0;
-    if (H->status != 0) code = H->status;
-    else if (H->magic != kHeaderMagic || H->layout_version != kLayoutVersion || H->head_dim != kD ||
-             H->bits_k != a.bits_k || H->bits_v != a.bits_v || H->batch != a.batch ||
-             H->n_kv_heads != a.n_kv_heads || H->capacity != a.capacity ||
-             static_cast<int>(H->record_bytes) != a.rec_bytes || dig[hkv] != al->digest ||
-             al->bits_k != a.bits_k || al->k_words != a.bits_k * kD || al->plan_k_cols > 96 ||
-             al->plan_k_cols < 8 || al->plan_n_slots > kPlanSlots)
-      code = KVQ_ERR_MISMATCH;
-    if (code) {
-      S.bad = 1;
-      record_status(a.status, code);
-    }
   }
   if (!tc::mbar_wait(&S.setup, 0, WL)) {
     S.bad = 1;
@@ -462,21 +528,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   __syncthreads();
   const bool bad = S.bad != 0;
   const kvq_head_alloc& A = *reinterpret_cast<const kvq_head_alloc*>(sm + kAllocOff);
+  volatile int* abort_flag = &S.wg_abort[g];
 
   float M[8], L[8];                                         // running max (log2) and row sums
 #pragma unroll
   for (int h = 0; h < 8; ++h) { M[h] = -INFINITY; L[h] = 0.0f; }
   int done = 0;                                             // chunks this warpgroup completed
-  bool s_pending = false, o_pending = false;                // committed products not waited for yet
 
-  if (!bad && warp >= 1 && warp <= 3) {
-    // ------------------------------------------------------------------ Q' (warps 1..3)
+  if (!bad && is_issuer) {
+    // ------------------------------------------------------------------ Q' (issuer warps)
     // Row h: q_h * f_b * log2(e) / sqrt(d), scaled by 2^-e so its largest |value| is in
     // [0.5, 1); qscale[h] = 2^e multiplies the product back. B operand of S, K-major, no
     // swizzle: element (n, k) at (k/8)*256 + (n/8)*128 + (n%8)*16 + (k%8)*2; K element k = 2c + r
     // is dim b + 64 r of the block in column c; n < 8: hi part of row n, n >= 8: lo part.
-    float* qtmp = reinterpret_cast<float*>(sm + kBPOff);    // [8][128] fp32 until P' is first written
-    for (int h = warp - 1; h < 8; h += 3) {
+    const int it = tid - 32 * kDecIssuerWarp0;              // 0..127
+    float* qtmp = reinterpret_cast<float*>(sm + kRecQOff);  // [8][128] fp32
+    for (int h = g; h < 8; h += kDecWG) {
       float qv[4], mx = 0.0f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -494,9 +561,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
 #pragma unroll
       for (int u = 0; u < 4; ++u) qtmp[h * kD + lane + 32 * u] = qv[u] * sc;
     }
-    named_sync(kDecWG + 1, 96);
+    named_sync(kDecWG + 1, 128);
     const int k_elems = 2 * A.plan_k_cols;
-    for (int i = tid - 32; i < 8 * k_elems; i += 96) {
+    for (int i = it; i < 8 * k_elems; i += 128) {
       const int n = i / k_elems, k = i - n * k_elems;
       const int blk = A.plan_col_block[k >> 1];
       __half hi = __float2half_rn(0.0f), lo = hi;
@@ -506,29 +573,74 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
       *reinterpret_cast<__half*>(sm + kBQOff + base + 128 + n * 16) = lo;
     }
     tc::fence_proxy_async_smem();
-    named_sync(kDecWG + 1, 96);
-    if (tid == 32) tc::mbar_arrive(&S.qready);
+    named_sync(kDecWG + 1, 128);
+    if (tid == 32 * kDecIssuerWarp0) tc::mbar_arrive(&S.qready);   // Q' scales for the compute warps
+    // ---------------------------------------------------------------- issuing (one lane per warpgroup)
+    if (issuer) {
+      const uint32_t id_s = tc::idesc_f16(128, 16, false), id_o = tc::idesc_f16(128, 16, true, kBfO);
+      const uint32_t bq = tc::smem_u32(sm + kBQOff), bp = tc::smem_u32(sm + kBPOff + g * kBPBytes);
+      const int nb = (min(A.plan_n_slots, kPlanSlots) + 3) >> 2;
+      const int k_steps = A.plan_k_cols >> 3;
+      const uint32_t tS = tbase + col_s(g), tO = tbase + col_o(g), tV = tbase + col_v(g);
+      bool ok = true;
+      for (int j = 0; j < nj && ok; ++j) {
+        for (int bt = 0; bt < nb; ++bt) {
+          const int kb = j * nb + bt, slot = kb & 1;
+          if (!tc::mbar_wait(&S.kready[g][slot], (kb >> 1) & 1, WL)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t tK = tbase + col_k(g, slot);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int ks = 2 * bt + i;
+            if (ks < k_steps) tc::mma_ts(tS, tK + 8 * i, tc::sdesc(bq + 512 * ks, 256, 128), id_s, ks > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&S.kfree[g][slot]);
+        }
+        if (!ok) break;
+        tc::mma_commit(&S.sfull[g]);
+        if (!tc::mbar_wait(&S.vready[g], j & 1, WL)) { ok = false; break; }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int ks = 0; ks < kChunkTokens / 16; ++ks)
+          tc::mma_ts(tO, tV + 8 * ks, tc::sdesc(bp + 512 * ks, 256, 128), id_o, (j > 0 || ks > 0) ? 1u : 0u);
+        tc::mma_commit(&S.ofull[g]);
+        // the stage is consumed (keys, values and norms): refill it with a later chunk
+        if (issued < nj && !a.debug_no_loads) issue_chunk(issued++);
+      }
+      if (!ok) *abort_flag = 1;
+      // every product committed so far completes before the CTA can free tensor memory, and
+      // every copy started lands before the CTA can leave
+      tc::mma_commit(&S.drain[g]);
+      tc::mbar_wait(&S.drain[g], 0, WL);
+      for (int s = 0; s < NS; ++s) {
+        int last = -1;
+        for (int j = s; j < issued; j += NS) last = j;
+        if (last >= 0) tc::mbar_wait(&S.full[g][s], (last / NS) & 1, WL);
+      }
+    }
+    __syncwarp();
     // ---------------------------------------------------------------- recent tokens (CUDA cores)
     // This CTA's even share of the row's recent tokens. Lane l owns dims l, l + 32, l + 64,
-    // l + 96; warp w walks every third token with its own online softmax over
-    // s = q . k * log2(e) / sqrt(d); the three warps then meet at a common maximum and add
+    // l + 96; issuer warp w walks every fourth token with its own online softmax over
+    // s = q . k * log2(e) / sqrt(d); the four warps then meet at a common maximum and add
     // their O shares into rec_o in a fixed order.
     const int r_begin = static_cast<int>((static_cast<long long>(split) * a.n_recent) / a.splits);
     const int r_end = static_cast<int>((static_cast<long long>(split + 1) * a.n_recent) / a.splits);
     if (r_end > r_begin) {
-      const int w = warp - 1;
-      float* rq = reinterpret_cast<float*>(sm + kRecQOff);
-      for (int i = tid - 32; i < 8 * kD; i += 96) {
+      const int w = g;
+      float* rq = reinterpret_cast<float*>(sm + kRecQOff);  // reused: q * log2(e) / sqrt(d)
+      named_sync(kDecWG + 1, 128);
+      for (int i = it; i < 8 * kD; i += 128) {
         const int h = i >> 7, j = i & (kD - 1);
         rq[i] = (h < G) ? load_f32(a.q, a.q_dtype, b * a.qsb + (hkv * G + h) * a.qsh + j) * (inv_sqrt_d * kLog2e) : 0.0f;
       }
-      named_sync(kDecWG + 1, 96);
+      named_sync(kDecWG + 1, 128);
       float o[8][4];
 #pragma unroll
       for (int h = 0; h < 8; ++h)
 #pragma unroll
         for (int u = 0; u < 4; ++u) o[h][u] = 0.0f;
-      for (int r = r_begin + w; r < r_end; r += 3) {
+      for (int r = r_begin + w; r < r_end; r += kDecWG) {
         float kv[4], vv[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -554,23 +666,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
 #pragma unroll
         for (int h = 0; h < 8; ++h) { S.rx_m[w][h] = M[h]; S.rx_l[w][h] = L[h]; }
       }
-      named_sync(kDecWG + 1, 96);
+      named_sync(kDecWG + 1, 128);
 #pragma unroll
       for (int h = 0; h < 8; ++h) {
-        const float Mx = fmaxf(fmaxf(S.rx_m[0][h], S.rx_m[1][h]), S.rx_m[2][h]);
+        const float Mx = fmaxf(fmaxf(S.rx_m[0][h], S.rx_m[1][h]), fmaxf(S.rx_m[2][h], S.rx_m[3][h]));
         const float wt = (M[h] == -INFINITY) ? 0.0f : fast_exp2(M[h] - Mx);
 #pragma unroll
         for (int u = 0; u < 4; ++u) o[h][u] *= wt;
         if (w == 0 && lane == 0) {
           float lsum = 0.0f;
 #pragma unroll
-          for (int ww = 0; ww < 3; ++ww)
+          for (int ww = 0; ww < 4; ++ww)
             lsum += (S.rx_m[ww][h] == -INFINITY) ? 0.0f : S.rx_l[ww][h] * fast_exp2(S.rx_m[ww][h] - Mx);
           S.wg_m[kDecWG][h] = Mx;
           S.wg_l[kDecWG][h] = lsum;
         }
       }
-      for (int ww = 0; ww < 3; ++ww) {
+      for (int ww = 0; ww < kDecWG; ++ww) {
         if (w == ww) {
 #pragma unroll
           for (int h = 0; h < 8; ++h)
@@ -580,91 +692,59 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
               *dst = (ww == 0) ? o[h][u] : *dst + o[h][u];
             }
         }
-        named_sync(kDecWG + 1, 96);
+        named_sync(kDecWG + 1, 128);
       }
 #pragma unroll
       for (int h = 0; h < 8; ++h) { M[h] = -INFINITY; L[h] = 0.0f; }
     }
-  } else if (!bad && is_wg) {
-    // ------------------------------------------------------------------ chunk pipeline
+  } else if (!bad) {
+    // ------------------------------------------------------------------ compute warps
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     const uint32_t lane4 = static_cast<uint32_t>(lane) << 2;
-    const uint32_t tA = tbase + col_a(g), tS = tbase + col_s(g), tO = tbase + col_o(g);
-    const int n_batches = (min(A.plan_n_slots, kPlanSlots) + 3) >> 2;
-    const int k_steps = A.plan_k_cols >> 3;
+    const uint32_t tV = tbase + col_v(g), tS = tbase + col_s(g), tO = tbase + col_o(g);
+    const int nb = (min(A.plan_n_slots, kPlanSlots) + 3) >> 2;
     uint8_t* pbuf = sm + kBPOff + g * kBPBytes;
-    const uint32_t id_s = tc::idesc_f16(128, 16, false), id_o = tc::idesc_f16(128, 16, true, kBfO);
-    const uint32_t bq = tc::smem_u32(sm + kBQOff), bp = tc::smem_u32(pbuf);
+    const uint4* slots4 = reinterpret_cast<const uint4*>(A.plan_slot);
     float qs[8];
     bool have_q = false;
-    volatile int* abort_flag = &S.wg_abort[g];
 
     for (int j = 0; j < nj; ++j) {
       const int ci = c_begin + g + kDecWG * j;
       const int s = j % NS;
       const uint8_t* st = my_stages + static_cast<size_t>(s) * cbytes;
-      bool ok = tc::mbar_wait(&S.full[g][s], (j / NS) & 1, WL);
-      if (ok && j > 0) ok = tc::mbar_wait(&S.ofull[g], (j - 1) & 1, WL);
-      if (!ok) *abort_flag = 1;
-      tc::fence_after_sync();
+      if (!tc::mbar_wait(&S.full[g][s], (j / NS) & 1, WL)) *abort_flag = 1;
       // -------------------------------------------------------------- keys (lane = token)
       const uint8_t* tq = st + q * a.rec_bytes;                       // tile q of the chunk
-      {
-        const uint32_t* kw = reinterpret_cast<const uint32_t*>(tq) + lane;
-        const uint32_t* slots = A.plan_slot;
-        for (int bt = 0; bt < n_batches; ++bt) {
-          uint32_t t[4][4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) k_slot(slots[4 * bt + i], kw, sm, lane4, t[i]);
-          uint32_t v16[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v16[i] = t[i >> 2][i & 3];
-          tc::tmem_st<16>(tA + lane_base + 16 * bt, v16);
+      const uint32_t* kw = reinterpret_cast<const uint32_t*>(tq) + lane;
+      // Batch bt's lookups run before the wait for batch bt - 1's store, so the store's
+      // latency hides behind them; a ring buffer is refilled once its S products are done.
+      for (int bt = 0; bt < nb; ++bt) {
+        const int kb = j * nb + bt, slot = kb & 1;
+        uint32_t v16[16];
+        k_batch(kw, slots4[bt], sm, lane4, v16);
+        if (bt > 0) {
+          tc::wait_st();
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&S.kready[g][slot ^ 1]);
         }
+        if (kb >= 2 && !tc::mbar_wait(&S.kfree[g][slot], ((kb >> 1) - 1) & 1, WL)) *abort_flag = 1;
+        tc::fence_after_sync();
+        tc::tmem_st<16>(tbase + col_k(g, slot) + lane_base, v16);
       }
+      tc::wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&S.kready[g][(j * nb + nb - 1) & 1]);
       const float kn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(tq + kbytes)[lane]));
       float vn = 1.0f;
       if constexpr (!kDense) vn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(tq + kbytes + 2 * kTile)[lane]));
       const int tok0 = ci * kChunkTokens;
       const bool valid = tok0 + 32 * q + lane < a.seq_len;
-      tc::wait_st();
-      tc::fence_before_sync();
-      named_sync(1 + g, 128);
-      if (*abort_flag) break;
-      if (leader) {
-        tc::fence_after_sync();
-        bool qok = true;
-        if (j == 0) qok = tc::mbar_wait(&S.qready, 0, WL);
-        if (qok) {
-          for (int ks = 0; ks < k_steps; ++ks)
-            tc::mma_ts(tS, tA + 8 * ks, tc::sdesc(bq + 512 * ks, 256, 128), id_s, ks > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&S.sfull[g]);                          // arrives even with nothing issued
-        if (!qok) *abort_flag = 1;
-      }
-      s_pending = true;
-      if (!have_q) {
-        if (!tc::mbar_wait(&S.qready, 0, WL)) *abort_flag = 1;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) qs[h] = S.qscale[h];
-        have_q = true;
-      }
-      if (!tc::mbar_wait(&S.sfull[g], j & 1, WL)) *abort_flag = 1;
-      else s_pending = false;
-      tc::fence_after_sync();
-      // -------------------------------------------------------------- logits
-      float sv[8];
-      {
-        uint32_t sr[16];
-        tc::tmem_ld<16>(tS + lane_base, sr);
-        tc::wait_ld();
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          const float x = (__uint_as_float(sr[h]) + __uint_as_float(sr[8 + h])) * (kn * qs[h]);
-          sv[h] = valid ? x : -INFINITY;
-        }
-      }
       // -------------------------------------------------------------- values (lane = dim)
+      // V-hat^T and P' are free once the previous chunk's O products are complete
+      if (j > 0 && !tc::mbar_wait(&S.ofull[g], (j - 1) & 1, WL)) *abort_flag = 1;
+      tc::fence_after_sync();
       if constexpr (kDense) {
         // dense rows [token][128] of 16-bit values after the chunk's records; rows past the
         // sequence end are not copied and read as 0
@@ -680,13 +760,33 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
             const uint32_t hi = (t0 + 1 < nrows) ? vr[(t0 + 1) * kD] : 0u;
             v[c] = lo | (hi << 16);
           }
-          tc::tmem_st<16>(tA + lane_base + 16 * u, v);
+          tc::tmem_st<16>(tV + lane_base + 16 * u, v);
         }
       } else {
 #pragma unroll
         for (int u = 0; u < kChunkTiles; ++u) {
           const uint32_t* vw = reinterpret_cast<const uint32_t*>(st + u * a.rec_bytes + kbytes + 4 * kTile) + 32 * q + lane;
-          v_tile<VM>(vw, tA + lane_base + 16 * u, sm, lane4);
+          v_tile<VM>(vw, tV + lane_base + 16 * u, sm, lane4);
+        }
+      }
+      // -------------------------------------------------------------- logits
+      if (!have_q) {
+        if (!tc::mbar_wait(&S.qready, 0, WL)) *abort_flag = 1;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) qs[h] = S.qscale[h];
+        have_q = true;
+      }
+      if (!tc::mbar_wait(&S.sfull[g], j & 1, WL)) *abort_flag = 1;
+      tc::fence_after_sync();
+      float sv[8];
+      {
+        uint32_t sr[16];
+        tc::tmem_ld<16>(tS + lane_base, sr);
+        tc::wait_ld();
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          const float x = (__uint_as_float(sr[h]) + __uint_as_float(sr[8 + h])) * (kn * qs[h]);
+          sv[h] = valid ? x : -INFINITY;
         }
       }
       // -------------------------------------------------------------- chunk maximum
@@ -747,24 +847,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
       tc::fence_proxy_async_smem();
       tc::wait_st();
       tc::fence_before_sync();
-      named_sync(1 + g, 128);
-      if (leader) {
-        tc::fence_after_sync();
-#pragma unroll
-        for (int ks = 0; ks < kChunkTokens / 16; ++ks)
-          tc::mma_ts(tO, tA + 8 * ks, tc::sdesc(bp + 512 * ks, 256, 128), id_o, (j > 0 || ks > 0) ? 1u : 0u);
-        tc::mma_commit(&S.ofull[g]);
-        // the stage is consumed (keys, values and norms): refill it with a later chunk
-        if (issued < nj && !a.debug_no_loads) issue_chunk(issued++);
-      }
-      o_pending = true;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&S.vready[g]);
       done = j + 1;
     }
     // ------------------------------------------------------------------ warpgroup result
-    if (o_pending && !*abort_flag) {
-      if (tc::mbar_wait(&S.ofull[g], (done - 1) & 1, WL)) o_pending = false;
-      else *abort_flag = 1;
-    }
+    if (done > 0 && !*abort_flag && !tc::mbar_wait(&S.ofull[g], (done - 1) & 1, WL)) *abort_flag = 1;
     named_sync(1 + g, 128);
     tc::fence_after_sync();
     if (!*abort_flag) {
@@ -776,13 +864,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
         if (lane == 0) S.lred[g][q][h] = l;
       }
     }
-  }
-  // In-flight work of a warpgroup that stopped early: its leader waits (bounded) for the
-  // products it committed and the copies it issued, so nothing lands after the CTA is gone.
-  if (leader && (bad || S.wg_abort[g])) {
-    if (s_pending) tc::mbar_wait(&S.sfull[g], done & 1, WL);
-    if (o_pending) tc::mbar_wait(&S.ofull[g], (done - 1) & 1, WL);
-    for (int j = done; j < issued; ++j) tc::mbar_wait(&S.full[g][j % NS], (j / NS) & 1, WL);
+  } else if (issuer) {
+    // a mismatched CTA still waits for the copies its issuer started
+    for (int s = 0; s < NS; ++s) {
+      int last = -1;
+      for (int j = s; j < issued; j += NS) last = j;
+      if (last >= 0) tc::mbar_wait(&S.full[g][s], (last / NS) & 1, WL);
+    }
   }
   __syncthreads();
   bool aborted = bad;
@@ -793,7 +881,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   // ------------------------------------------------------------------ CTA result
   // Warpgroup partials (m, l, O) combined in shared memory (the stage area is free now).
   float* comb = reinterpret_cast<float*>(stages);           // [kDecWG][8][128] O, unscaled
-  if (!aborted && is_wg) {
+  if (!aborted && !is_issuer) {
     const int d = 32 * q + lane;
     if (nj > 0) {
       uint32_t o[16];
@@ -803,6 +891,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
       for (int h = 0; h < 8; ++h)
         comb[(g * 8 + h) * kD + d] = (__uint_as_float(o[h]) + __uint_as_float(o[8 + h])) * static_cast<float>(1 << kTau);
     }
+    const int tid_wg = 32 * q + lane;
     if (tid_wg < 8) {
       const int h = tid_wg;
       float mh = -INFINITY;
@@ -816,7 +905,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == 0) tc::tmem_dealloc(tbase, kTmemCols);
+  if (warp == kDecIssuerWarp0) tc::tmem_dealloc(tbase, kTmemCols);
   if (aborted) return;
 
   const int pitch = a.splits + a.n_groups;

@@ -497,6 +497,8 @@ kvq_status launch_decode(const void* q, const kvq_tensor4* qd, const void* packe
   const int rec = static_cast<int>(tile_record_bytes(c->bits_k, c->bits_v));
   const int cb = chunk_bytes(rec) + (dense_v ? kChunkTokens * 2 * kD : 0);
   const size_t smem = decode_smem_bytes(cb);
+  // one chunk stage per warpgroup must fit (keys-only caches above 4 bits per dim do not)
+  if (smem > max_smem()) return KVQ_ERR_UNSUPPORTED;
   DecArgs a{};
   a.q = q;
   a.qsb = qd->stride_b;

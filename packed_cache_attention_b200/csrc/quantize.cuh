@@ -84,9 +84,12 @@ inline bool quant_lut_image(const float* thresholds, uint32_t* out /* 2 * kLutEn
 
 __device__ __align__(16) uint32_t g_quant_lut[2 * kLutEntries];
 
-// Code of y for width W (1..8) from the table in shared memory.
+// Code of y for width W (1..8) from the table in shared memory (lut_s: its shared-memory
+// address). The entry of cell k sits at lut_s + 8 (offset + k), and k = bits(f) - 0x4B400000,
+// so the entry address is one multiply-add of bits(f) with a folded constant (32-bit shared
+// addresses wrap, so the constant's own wrap-around is harmless).
 template <int W>
-__device__ __forceinline__ uint32_t lut_code(float y, const uint2* __restrict__ lut) {
+__device__ __forceinline__ uint32_t lut_code(float y, uint32_t lut_s) {
   if constexpr (W == 1) {
     return y > 0.0f ? 1u : 0u;
   } else {
@@ -96,9 +99,11 @@ __device__ __forceinline__ uint32_t lut_code(float y, const uint2* __restrict__ 
     constexpr float hi = (static_cast<float>(K) - 0.5f) / s;   // inside the last cell
     const float yc = fminf(fmaxf(y, lo), hi);                  // NaN -> lo
     const float f = __fmaf_rd(yc, s, 12582912.0f + static_cast<float>(K));   // 1.5 * 2^23 + K + floor(yc s)
-    const int idx = __float_as_int(f) - 0x4B400000;
-    const uint2 e = lut[kLutOffset[W] + idx];
-    return e.x + (y > __uint_as_float(e.y) ? 1u : 0u);
+    const uint32_t addr = static_cast<uint32_t>(__float_as_int(f)) * 8u +
+                          (lut_s + 8u * (static_cast<uint32_t>(kLutOffset[W]) - 0x4B400000u));
+    uint32_t below, tau;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(below), "=r"(tau) : "r"(addr));
+    return below + (y > __uint_as_float(tau) ? 1u : 0u);
   }
 }
 
@@ -270,7 +275,7 @@ __device__ __forceinline__ float2 block_pair(const uint8_t* row, const KEntry& e
 // All blocks of one width class (entries first .. first + nb - 1).
 template <int DT, int W>
 __device__ __forceinline__ void quant_k_class(const uint8_t* row, float2 aa, const KEntry* __restrict__ ent, int nb,
-                                              const uint2* __restrict__ lut, KStream& ks, uint32_t* __restrict__ kout,
+                                              uint32_t lut, KStream& ks, uint32_t* __restrict__ kout,
                                               int lane) {
   constexpr int GB = (W <= 4) ? 4 : 2;                          // blocks per group: 2 W GB <= 32 bits
   for (int k = 0; k < nb; k += GB) {
@@ -299,7 +304,7 @@ __device__ __forceinline__ void quant_k_class(const uint8_t* row, float2 aa, con
 // of token t (NaN for tokens not written). Word i of dim j goes to vout[128 i + j]. The first
 // `keep_bits` bits of every dim stream (tokens that precede an append) keep their stored value.
 template <int DT, int BV>
-__device__ __forceinline__ void quant_v_tile(const uint32_t* rows, const float2* sA2, const uint2* __restrict__ lut,
+__device__ __forceinline__ void quant_v_tile(const uint32_t* rows, const float2* sA2, uint32_t lut,
                                              uint32_t* __restrict__ vout, int keep_bits, int lane) {
   using Q = QTile<DT>;
 #pragma unroll 1
@@ -411,6 +416,7 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
   uint2* sLut = reinterpret_cast<uint2*>(smem);
   for (int i = threadIdx.x; i < kLutEntries; i += blockDim.x)
     sLut[i] = make_uint2(g_quant_lut[2 * i], g_quant_lut[2 * i + 1]);
+  const uint32_t lut_s = static_cast<uint32_t>(__cvta_generic_to_shared(sLut));
   if (threadIdx.x == 0) sHeaderOk = (qh.mode == 2) ? packed_header_ok(packed, qh, n_kv_heads, bits_k, bits_v, rec_bytes, alloc) : 1;
   if (qh.mode == 1 && blockIdx.x == 0 && threadIdx.x < 32)
     write_packed_header(packed, qh, n_kv_heads, bits_k, bits_v, rec_bytes, alloc, threadIdx.x);
@@ -525,14 +531,14 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
         const int w = e & 0xffu, first = (e >> 8) & 0xffu, nb = e >> 16;
         const KEntry* ent = sEnt + first;
         switch (w) {
-          case 1: quant_k_class<DT, 1>(row, aa, ent, nb, sLut, ks, kout, lane); break;
-          case 2: quant_k_class<DT, 2>(row, aa, ent, nb, sLut, ks, kout, lane); break;
-          case 3: quant_k_class<DT, 3>(row, aa, ent, nb, sLut, ks, kout, lane); break;
-          case 4: quant_k_class<DT, 4>(row, aa, ent, nb, sLut, ks, kout, lane); break;
-          case 5: quant_k_class<DT, 5>(row, aa, ent, nb, sLut, ks, kout, lane); break;
-          case 6: quant_k_class<DT, 6>(row, aa, ent, nb, sLut, ks, kout, lane); break;
-          case 7: quant_k_class<DT, 7>(row, aa, ent, nb, sLut, ks, kout, lane); break;
-          default: quant_k_class<DT, 8>(row, aa, ent, nb, sLut, ks, kout, lane); break;
+          case 1: quant_k_class<DT, 1>(row, aa, ent, nb, lut_s, ks, kout, lane); break;
+          case 2: quant_k_class<DT, 2>(row, aa, ent, nb, lut_s, ks, kout, lane); break;
+          case 3: quant_k_class<DT, 3>(row, aa, ent, nb, lut_s, ks, kout, lane); break;
+          case 4: quant_k_class<DT, 4>(row, aa, ent, nb, lut_s, ks, kout, lane); break;
+          case 5: quant_k_class<DT, 5>(row, aa, ent, nb, lut_s, ks, kout, lane); break;
+          case 6: quant_k_class<DT, 6>(row, aa, ent, nb, lut_s, ks, kout, lane); break;
+          case 7: quant_k_class<DT, 7>(row, aa, ent, nb, lut_s, ks, kout, lane); break;
+          default: quant_k_class<DT, 8>(row, aa, ent, nb, lut_s, ks, kout, lane); break;
         }
       }
     }
@@ -555,7 +561,7 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
         sA2[lane] = make_float2(a, a);
         const int keep = bits_v * r_lo;
         __syncwarp();
-        quant_v_tile<DT, BVT>(vbuf, sA2, sLut, vout, keep, lane);
+        quant_v_tile<DT, BVT>(vbuf, sA2, lut_s, vout, keep, lane);
       }
       __syncwarp();                               // every lane is done with the V tile and sA2
       if (nvp) tile_load_async<DT>(vbuf, nvp, vst, nlo, nhi, lane);

@@ -412,6 +412,52 @@ def test_keys_only_quantize_matches_oracle(dev, dtype):
                                   ref[hb:hb + n].reshape(2, 2, -1, rec)[:, :, :nt])
 
 
+@pytest.mark.parametrize("case", [("bf16", 2, 4000), ("f16", 3, 777), ("bf16", 4, 33)], ids=lambda c: f"{c[0]}K{c[1]}T{c[2]}")
+def test_keys_only_decode_matches_oracle(dev, case):
+    """Keys-only cache: packed keys, values read from the caller's unquantized
+    tensor; attention within tolerance of the oracle's fp64 attention over k-hat and the exact
+    values, at every prefix length checked."""
+    dtype, bk, T = case
+    x = wl.make_blockgtq_inputs(1, 8, 2, 128, T, dtype, 1e6, "lognormal_outliers", seed=80 + bk, device=dev)
+    alloc = kvq.kvq_calibrate(x["K"], bk)
+    cache = kvq.cache_desc(1, 2, T + 7, bk, 0)
+    packed = kvq.kvq_quantize(x["K"], None, alloc, cache)
+    Kh, Vh, qh = host_f32(x["K"]), host_f32(x["V"]), host_f32(x["q"])
+    ra = bg.calibrate(Kh, bk)
+    rp = bg.pack_cache(bg.quantize(Kh, None, ra, 0), ra, 0, T + 7)
+    for sl in sorted({1, T // 2, T}):
+        out = kvq.kvq_decode_attn_ex(x["q"], packed, alloc, cache, sl, V=x["V"]).cpu().numpy()
+        ref = bg.decode(qh, rp, ra, 0, sl, V=Vh)
+        assert rel_err(out, ref) <= TOL, sl
+
+
+@pytest.mark.parametrize("case", [(3000, 64, "bf16"), (300, 1000, "f32"), (0, 37, "bf16"), (5000, 1, "f16")],
+                         ids=lambda c: f"T{c[0]}R{c[1]}{c[2]}")
+def test_recent_tokens_join_the_softmax(dev, case):
+    """Recent tokens kept unquantized (the buffer of fp16 recent keys the Block-GTQ page reports
+    its results without): R tokens after the packed ones, in the caller's dtype, attended in
+    the same softmax; within tolerance of the oracle's fp64 attention over the packed
+    tokens' k-hat, v-hat and the recent tokens' exact keys and values. T = 0 attends over the
+    recent tokens alone."""
+    T, R, rdtype = case
+    xs = wl.make_blockgtq_inputs(1, 16, 2, 128, T + R, "bf16", 1e6, "lognormal_outliers", seed=90 + R, device=dev)
+    K, V, q = xs["K"], xs["V"], xs["q"]
+    Tc = max(T, 1)
+    Kc = K[:, :, :Tc].contiguous()
+    alloc = kvq.kvq_calibrate(Kc, 3)
+    cache = kvq.cache_desc(1, 2, Tc, 3, 3)
+    packed = kvq.kvq_quantize(Kc, V[:, :, :Tc].contiguous(), alloc, cache)
+    tdt = wl.torch_dtype(rdtype)
+    Kr = K[:, :, T:T + R].to(tdt).contiguous()
+    Vr = V[:, :, T:T + R].to(tdt).contiguous()
+    out = kvq.kvq_decode_attn_ex(q, packed, alloc, cache, T, K_recent=Kr, V_recent=Vr).cpu().numpy()
+    Kh = host_f32(Kc)
+    ra = bg.calibrate(Kh, 3)
+    rp = bg.pack_cache(bg.quantize(Kh, host_f32(V[:, :, :Tc]), ra, 3), ra, 3, Tc)
+    ref = bg.decode(host_f32(q), rp, ra, 3, T, K_recent=host_f32(Kr), V_recent=host_f32(Vr))
+    assert rel_err(out, ref) <= TOL
+
+
 # ----------------------------------------------------------------------------- full-size workloads
 
 def _sample_tiles(n_tiles, k=6, seed=0):

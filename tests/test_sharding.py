@@ -1,0 +1,77 @@
+"""Sharding of the path over ranks, on CPU: two gloo ranks split the KV heads of one
+workload, each runs its share (here through the CPU oracle, since there is no GPU), and the
+outputs gathered in rank order equal the single-rank result byte for byte. The (sequence, KV
+head) units never exchange data: calibration, quantization and decode of a head read that
+head alone."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from oracle import blockgtq as bg
+from packed_cache_attention_b200 import shard
+from packed_cache_attention_b200 import workloads as wl
+
+B, HQ, HKV, T, BK, BV = 2, 6, 3, 200, 3, 3
+
+
+def _inputs():
+    x = wl.make_blockgtq_inputs(B, HQ, HKV, 128, T, "bf16", 5e5, "lognormal_outliers", seed=12, device="cpu")
+    return x["K"].float().numpy(), x["V"].float().numpy(), x["q"].float().numpy()
+
+
+def _oracle_heads(K, V, q, kv: range):
+    """The oracle's calibrate -> quantize -> pack -> decode on the KV heads of `kv` alone."""
+    G = HQ // HKV
+    Kl, Vl = K[:, kv.start:kv.stop], V[:, kv.start:kv.stop]
+    qh = shard.query_heads(kv, G)
+    a = bg.calibrate(Kl, BK)
+    p = bg.pack_cache(bg.quantize(Kl, Vl, a, BV), a, BV, T)
+    return bg.decode(q[:, qh.start:qh.stop], p, a, BV, T)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        K, V, q = _inputs()
+        kv = shard.kv_head_ranges(HKV, world)[rank]
+        local = torch.from_numpy(_oracle_heads(K, V, q, kv)) if len(kv) else torch.zeros((B, 0, 128),
+                                                                                          dtype=torch.float64)
+        full = shard.gather_outputs(local, kv, HKV, HQ // HKV, world)
+        np.save(os.path.join(out_dir, f"out{rank}.npy"), full.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_kv_head_ranges_cover_every_head_once():
+    for n, w in [(8, 2), (3, 2), (2, 3), (16, 8), (1, 4)]:
+        rs = shard.kv_head_ranges(n, w)
+        assert len(rs) == w and [h for r in rs for h in r] == list(range(n))
+        assert max(len(r) for r in rs) - min(len(r) for r in rs) <= 1
+    assert list(shard.query_heads(range(1, 3), 4)) == list(range(4, 12))
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world", [2, 4])
+def test_sharded_heads_equal_single_rank(tmp_path, world):
+    """3 KV heads over 2 ranks (1 + 2 heads) and over 4 ranks (one rank with none): the
+    gathered output equals the single-rank oracle result exactly."""
+    mp.start_processes(_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn")
+    K, V, q = _inputs()
+    ref = _oracle_heads(K, V, q, range(HKV))
+    for r in range(world):
+        got = np.load(tmp_path / f"out{r}.npy")
+        np.testing.assert_array_equal(got, ref)
