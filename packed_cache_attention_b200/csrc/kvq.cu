@@ -105,11 +105,12 @@ int nf4_splits(int bh, int n_groups) {
   return std::max(1, std::min(std::min(want, n_groups / kNf4DecWarps), kNf4MaxSplits));
 }
 
-// Block-GTQ decode: splits of whole 128-token chunks, about one CTA per SM in total.
+// Block-GTQ decode: splits of whole 128-token chunks, at most one CTA per SM in total (a
+// second partial wave would double the time of the CTAs in it).
 constexpr int kMaxGtqSplits = kMergeMax * kMergeMax;
 int gtq_splits(int bh, int n_tiles) {
   const int n_chunks = (n_tiles + kChunkTiles - 1) / kChunkTiles;
-  const int want = (sm_count() + bh - 1) / bh;
+  const int want = std::max(1, sm_count() / bh);
   return std::max(1, std::min(std::min(want, n_chunks), kMaxGtqSplits));
 }
 
