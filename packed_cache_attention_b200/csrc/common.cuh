@@ -75,6 +75,16 @@ __host__ __device__ __forceinline__ uint64_t splitmix64(uint64_t z) {
   return z ^ (z >> 31);
 }
 
+// Ticket of a split merge: one atomic add at GPU scope with acquire-release order. Taken by one
+// thread right after the CTA barrier that follows the CTA's writes of its partial result, it
+// publishes those writes (release); for the thread that draws the last ticket it also makes
+// the earlier arrivers' writes visible (acquire) to every thread past the next CTA barrier.
+__device__ __forceinline__ unsigned ticket_add(unsigned* p) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));

@@ -55,7 +55,7 @@ constexpr int kStagesMax = 4;             // chunk stages per warpgroup
 constexpr int kTau = 8;                   // lazy rescale threshold (log2 units)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPlanSlots = 24;
-constexpr int kMergeMax = 64;             // entries one merge step reads
+constexpr int kMergeMax = 64;             // group size bound of the split merge
 constexpr uint32_t kHeaderMagic = 0x3151564Bu;   // "KVQ1"
 constexpr int kLayoutVersion = 1;
 
@@ -66,16 +66,18 @@ __device__ __forceinline__ uint32_t col_s(int g) { return 128u * g + 96u; }
 __device__ __forceinline__ uint32_t col_o(int g) { return 128u * g + 112u; }
 
 // Lookup-table image, built once per device (decode_lut_image) and bulk-copied into every
-// CTA's shared memory at byte 0. Widths 1..3 keep pair tables: the fp16 pair {c[i & m], c[i >> w]}
-// for the 2w-bit index i of two consecutive codes. Widths 4..6 keep single-code tables (c[e] in
-// the low half of a word). Both keep one copy per lane (entry e of lane l at word 32 e + l),
-// so the 32 lanes of a warp never share a bank whatever codes they look up. Widths 7 and 8
-// (rare: the highest-energy blocks) use single fp16 tables shared by all lanes.
-__host__ __device__ constexpr int lut_off(int w) {
-  return w == 1 ? 0 : w == 2 ? 512 : w == 3 ? 2560 : w == 4 ? 10752 : w == 5 ? 12800 : w == 6 ? 16896
-                                                                                       : w == 7 ? 25088 : 25344;
+// CTA's shared memory at byte 0. Entries are fp16 centroid values c_w[e] of width w.
+//   Pair tables, one 32-bit word per pair index i = code_a | code_b << w (the 2w bits of two
+//   consecutive codes): {c[code_a], c[code_b]}. Widths 1..3 keep one copy per lane (entry i of
+//   lane l at word 32 i + l), so the 32 lanes of a warp never share a bank; they sit at byte 0
+//   (width 3, 8 KB), 8192 (width 2) and 10240 (width 1), so an entry's byte address is
+//   base | i << 7 | lane << 2. Widths 4 and 5 keep one shared copy (1 KB and 4 KB).
+//   Single tables of widths 6..8 (rare: the highest-energy blocks): one fp16 per code, shared.
+__host__ __device__ constexpr int pair_off(int w) {
+  return w == 3 ? 0 : w == 2 ? 8192 : w == 1 ? 10240 : w == 5 ? 10752 : 14848;
 }
-constexpr int kLutBytes = 25856;
+__host__ __device__ constexpr int single_off(int w) { return w == 6 ? 15872 : w == 7 ? 16000 : 16256; }
+constexpr int kLutBytes = 16768;
 // Shared-memory map (byte offsets from the start of dynamic shared memory).
 constexpr int kAllocOff = kLutBytes;                 // copy of the KV head's kvq_head_alloc
 constexpr int kBQOff = ((kAllocOff + static_cast<int>(sizeof(kvq_head_alloc)) + 127) / 128) * 128;
@@ -98,21 +100,21 @@ struct DecHeader {
   uint64_t ofull[kDecWG];              // O products of the chunk complete
   uint64_t drain[kDecWG];              // every product the issuer committed is complete
   uint64_t setup;                      // lookup tables + allocation record copied in
-  uint64_t qready;                     // Q' and qscale written
   uint32_t tmem_base;
   int bad;                             // header or allocation mismatch: the CTA writes nothing
   int wg_abort[kDecWG];                // a wait of this warpgroup gave up
   float qscale[8];                     // 2^e that undoes the range scaling of Q' row h
+  float qmax[16];                      // Q' row maxima: [row][half of the dims]
   float xch[kDecWG][4][8];             // chunk maximum: [warpgroup][warp][row]
   float lred[kDecWG][4][8];            // row sums: [warpgroup][warp][row]
   float wg_m[kDecWG + 1][8];           // warpgroup (and recent-token) results: maximum
   float wg_l[kDecWG + 1][8];           //                                        and row sum
   float rx_m[4][8];                    // recent tokens: per issuer warp maximum
   float rx_l[4][8];                    //                                and row sum
-  int last;
-  float mw[8][kMergeMax];              // merge: member maxima, then weights
-  float ml[8][kMergeMax];              //        member row sums
-  float Msum[8][2];                    //        merged maximum and row sum
+  int last;                            // this CTA drew the last ticket of its merge group
+  uint4 kdesc[kPlanSlots];             // per plan slot of width <= 5: word offset, shifts, mask, stride
+  uint32_t kbase[kPlanSlots];          //                                 pair-table byte offset
+  int bkind[kPlanSlots / 4];           // per batch of 4 slots: 0 all widths <= 5, 1 otherwise
 };
 
 __host__ __device__ constexpr int decode_stage_off() {
@@ -124,21 +126,16 @@ __host__ __device__ constexpr int chunk_bytes(int rec_bytes) { return kChunkTile
 
 // Host: the lookup-table image from the fp16 centroid table (width w at c16 + 2^w - 2).
 inline void decode_lut_image(const uint16_t* c16, uint8_t* img) {
-  for (int w = 1; w <= 3; ++w) {
+  for (int w = 1; w <= 5; ++w) {
     const uint16_t* c = c16 + (1 << w) - 2;
-    uint32_t* t = reinterpret_cast<uint32_t*>(img + lut_off(w));
+    uint32_t* t = reinterpret_cast<uint32_t*>(img + pair_off(w));
+    const int copies = w <= 3 ? 32 : 1;
     for (int e = 0; e < (1 << (2 * w)); ++e)
-      for (int l = 0; l < 32; ++l)
-        t[e * 32 + l] = static_cast<uint32_t>(c[e & ((1 << w) - 1)]) | (static_cast<uint32_t>(c[e >> w]) << 16);
+      for (int l = 0; l < copies; ++l)
+        t[e * copies + l] = static_cast<uint32_t>(c[e & ((1 << w) - 1)]) | (static_cast<uint32_t>(c[e >> w]) << 16);
   }
-  for (int w = 4; w <= 6; ++w) {
-    const uint16_t* c = c16 + (1 << w) - 2;
-    uint32_t* t = reinterpret_cast<uint32_t*>(img + lut_off(w));
-    for (int e = 0; e < (1 << w); ++e)
-      for (int l = 0; l < 32; ++l) t[e * 32 + l] = static_cast<uint32_t>(c[e]);
-  }
-  for (int w = 7; w <= 8; ++w) {
-    uint16_t* t = reinterpret_cast<uint16_t*>(img + lut_off(w));
+  for (int w = 6; w <= 8; ++w) {
+    uint16_t* t = reinterpret_cast<uint16_t*>(img + single_off(w));
     for (int e = 0; e < (1 << w); ++e) t[e] = c16[(1 << w) - 2 + e];
   }
 }
@@ -163,53 +160,18 @@ __device__ __forceinline__ uint32_t field_at(uint32_t lo, uint32_t hi, int p, in
 }
 
 // fp16 pair for two consecutive codes: code_a = bits [p, p + W), code_b = bits [p + W, p + 2W)
-// of hi:lo; code_a goes to the low half. Widths 1..3: the pair index lands directly at its
-// table offset (x 128 bytes plus the lane's word); widths 4..6: two per-lane single-code
-// lookups joined by a byte permute; widths 7, 8: two shared single-code lookups.
+// of hi:lo; code_a goes to the low half. Widths 1..5: one pair-table lookup (per-lane copy for
+// 1..3); widths 6..8: two single-code lookups.
 template <int W>
 __device__ __forceinline__ uint32_t pair_value(uint32_t lo, uint32_t hi, int p, const uint8_t* sm, uint32_t lane4) {
   if constexpr (W <= 3) {
-    return *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + (field_at(lo, hi, p, 2 * W, 7) | lane4));
-  } else if constexpr (W <= 6) {
-    const uint32_t a = *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + (field_at(lo, hi, p, W, 7) | lane4));
-    const uint32_t b = *reinterpret_cast<const uint32_t*>(sm + lut_off(W) + (field_at(lo, hi, p + W, W, 7) | lane4));
-    return __byte_perm(a, b, 0x5410);
+    return *reinterpret_cast<const uint32_t*>(sm + pair_off(W) + (field_at(lo, hi, p, 2 * W, 7) | lane4));
+  } else if constexpr (W <= 5) {
+    return *reinterpret_cast<const uint32_t*>(sm + pair_off(W) + field_at(lo, hi, p, 2 * W, 2));
   } else {
-    const uint8_t* t = sm + lut_off(W);
+    const uint8_t* t = sm + single_off(W);
     return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(t + field_at(lo, hi, p, W, 1))) |
            (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(t + field_at(lo, hi, p + W, W, 1))) << 16);
-  }
-}
-
-// Values of 4 consecutive block pairs of width W whose first code starts at bit `off` of this
-// lane's token stream; kw points at word 0 of the token (word i at kw[32 i]).
-template <int W>
-__device__ __forceinline__ void k_group_vals(const uint32_t* kw, uint32_t off, const uint8_t* sm, uint32_t lane4,
-                                             uint32_t (&v)[4]) {
-  const uint32_t j0 = off >> 5, s = off & 31u;
-  const uint32_t x0 = kw[j0 * 32], x1 = kw[(j0 + 1) * 32];
-  const uint32_t x2 = (8 * W > 32) ? kw[(j0 + 2) * 32] : 0u;
-  const uint32_t r0 = __funnelshift_r(x0, x1, s);
-  const uint32_t r1 = __funnelshift_r(x1, x2, s);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) v[k] = pair_value<W>(r0, r1, 2 * W * k, sm, lane4);
-}
-
-// Values of one plan slot: e = width | bit offset << 8 (width 0: an empty slot, zeros). A
-// slot with fewer than 4 real pairs is decoded as 4; its other columns have zero Q' rows.
-__device__ __forceinline__ void k_slot(uint32_t e, const uint32_t* kw, const uint8_t* sm, uint32_t lane4,
-                                       uint32_t (&t)[4]) {
-  const uint32_t off = e >> 8;
-  switch (e & 15u) {
-    case 1: k_group_vals<1>(kw, off, sm, lane4, t); break;
-    case 2: k_group_vals<2>(kw, off, sm, lane4, t); break;
-    case 3: k_group_vals<3>(kw, off, sm, lane4, t); break;
-    case 4: k_group_vals<4>(kw, off, sm, lane4, t); break;
-    case 5: k_group_vals<5>(kw, off, sm, lane4, t); break;
-    case 6: k_group_vals<6>(kw, off, sm, lane4, t); break;
-    case 7: k_group_vals<7>(kw, off, sm, lane4, t); break;
-    case 8: k_group_vals<8>(kw, off, sm, lane4, t); break;
-    default: t[0] = 0u; t[1] = 0u; t[2] = 0u; t[3] = 0u; break;
   }
 }
 
@@ -251,6 +213,36 @@ __device__ __forceinline__ void k_batch(const uint32_t* kw, uint4 e4, const uint
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) k_slot_vals(e[i], r0[i], r1[i], sm, lane4, v + 4 * i);
+}
+
+// 16 K-hat columns (4 plan slots) of this lane's token when every slot's width is at most 5
+// (or the slot is empty): the same instructions for every width, so the lookups of all four
+// slots are issued back to back. A slot's descriptor holds the byte offset of the stream word
+// with its first code (x), the bit shift of that code in the word and the shifts of its block
+// pairs 1..3 (y: one per byte, each read modulo 32 by the funnel shifts), the pair-index mask
+// (z) and the table stride (w: 128 for the per-lane tables of widths 1..3, 4 for the shared
+// ones); base is the table's byte offset.
+__device__ __forceinline__ void k_batch_gen(const uint32_t* kw, const uint4* desc, const uint32_t* base,
+                                            const uint8_t* sm, uint32_t lane4, uint32_t (&v)[16]) {
+  uint4 d[4];
+  uint32_t r0[4], r1[4], lb[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    d[i] = desc[i];
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(kw) + d[i].x);
+    const uint32_t x0 = p[0], x1 = p[32], x2 = p[64];
+    r0[i] = __funnelshift_r(x0, x1, d[i].y);
+    r1[i] = __funnelshift_r(x1, x2, d[i].y);
+    lb[i] = base[i] | (lane4 & (d[i].w - 4u));
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t t = (k == 0) ? r0[i] : __funnelshift_r(r0[i], r1[i], d[i].y >> (8 * k));
+      v[4 * i + k] = *reinterpret_cast<const uint32_t*>(sm + (t & d[i].z) * d[i].w + lb[i]);
+    }
+  }
 }
 
 // V-hat^T row of one dim for one tile: 16 token pairs (2u, 2u+1) -> 16 columns.
@@ -319,61 +311,62 @@ struct DecArgs {
 
 // ---------------------------------------------------------------- split merge
 
-// Merges entries e0 .. e0 + n - 1 (n <= kMergeMax) of row bh, each (m, l, O) with O
-// unnormalized and m in log2 units. Writes the merged entry to `dst_entry` (>= 0) or
-// out = O / l (dst_entry < 0). Called by every thread of the CTA.
-__device__ __forceinline__ void merge_entries(DecHeader& S, const DecArgs& a, int bh, int pitch, int e0, int n,
-                                              int dst_entry, float* out_bh, int G) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const size_t row = static_cast<size_t>(bh) * pitch;
-  for (int i = tid; i < 8 * n; i += blockDim.x) {
-    const int s = i >> 3, h = i & 7;
-    S.mw[h][s] = __ldcg(a.part_m + (row + e0 + s) * 8 + h);
-    S.ml[h][s] = __ldcg(a.part_l + (row + e0 + s) * 8 + h);
-  }
-  __syncthreads();
-  if (warp < 8) {
-    const int h = warp;
-    float M = -INFINITY;
-    for (int s = lane; s < n; s += 32) M = fmaxf(M, S.mw[h][s]);
+// Merges entries e0 .. e0 + n - 1 of row bh, each (m, l, O) with O unnormalized and m in log2
+// units, into entry `dst_entry` (>= 0) or into out = O / l (dst_entry < 0). Thread (h, j4) of
+// the first 256 keeps a running (M, L, O[4 j4 .. 4 j4 + 3]) of row h and folds the entries in
+// eight at a time: the loads of eight entries are issued together, so the merge costs
+// ceil(n / 8) round trips to L2 and no CTA barrier. The order of the sums is fixed.
+__device__ __forceinline__ void merge_entries(const DecArgs& a, int bh, int pitch, int e0, int n, int dst_entry,
+                                              float* out_bh, int G) {
+  const int tid = threadIdx.x;
+  if (tid >= 256) return;
+  const int h = tid >> 5, j4 = tid & 31;
+  const size_t row = static_cast<size_t>(bh) * pitch + e0;
+  const float4* po = reinterpret_cast<const float4*>(a.part_o);
+  float M = -INFINITY, L = 0.0f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < n; s0 += 8) {
+    float mv[8], lv[8];
+    float4 ov[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.0f;
-    for (int s = lane; s < n; s += 32) {
-      const float ms = S.mw[h][s];
-      const float wt = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-      S.mw[h][s] = wt;
-      L += S.ml[h][s] * wt;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) {
-      S.Msum[h][0] = M;
-      S.Msum[h][1] = L;
-    }
-  }
-  __syncthreads();
-  if (tid < 256) {
-    const int h = tid >> 5, j4 = tid & 31;
-    const float4* po = reinterpret_cast<const float4*>(a.part_o) + ((row + e0) * 8 + h) * (kD / 4) + j4;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int s = 0; s < n; ++s) {
-      const float wt = S.mw[h][s];
-      const float4 v = __ldcg(po + static_cast<size_t>(s) * 8 * (kD / 4));
-      o.x += v.x * wt; o.y += v.y * wt; o.z += v.z * wt; o.w += v.w * wt;
-    }
-    if (dst_entry >= 0) {
-      reinterpret_cast<float4*>(a.part_o)[((row + dst_entry) * 8 + h) * (kD / 4) + j4] = o;
-      if (j4 == 0) {
-        a.part_m[(row + dst_entry) * 8 + h] = S.Msum[h][0];
-        a.part_l[(row + dst_entry) * 8 + h] = S.Msum[h][1];
+    for (int u = 0; u < 8; ++u) {
+      if (s0 + u < n) {
+        const size_t e = row + s0 + u;
+        mv[u] = __ldcg(a.part_m + e * 8 + h);
+        lv[u] = __ldcg(a.part_l + e * 8 + h);
+        ov[u] = __ldcg(po + (e * 8 + h) * (kD / 4) + j4);
+      } else {
+        mv[u] = -INFINITY;
+        lv[u] = 0.0f;
+        ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
-    } else if (h < G) {
-      const float inv = 1.0f / S.Msum[h][1];
-      reinterpret_cast<float4*>(out_bh + static_cast<size_t>(h) * kD)[j4] =
-          make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
     }
+    float mx = M;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) mx = fmaxf(mx, mv[u]);
+    if (mx == -INFINITY) continue;
+    const float sc = (M == -INFINITY) ? 0.0f : fast_exp2(M - mx);
+    L *= sc;
+    o.x *= sc; o.y *= sc; o.z *= sc; o.w *= sc;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float wt = (mv[u] == -INFINITY) ? 0.0f : fast_exp2(mv[u] - mx);
+      L += lv[u] * wt;
+      o.x += ov[u].x * wt; o.y += ov[u].y * wt; o.z += ov[u].z * wt; o.w += ov[u].w * wt;
+    }
+    M = mx;
+  }
+  if (dst_entry >= 0) {
+    const size_t e = static_cast<size_t>(bh) * pitch + dst_entry;
+    reinterpret_cast<float4*>(a.part_o)[(e * 8 + h) * (kD / 4) + j4] = o;
+    if (j4 == 0) {
+      a.part_m[e * 8 + h] = M;
+      a.part_l[e * 8 + h] = L;
+    }
+  } else if (h < G) {
+    const float inv = 1.0f / L;
+    reinterpret_cast<float4*>(out_bh + static_cast<size_t>(h) * kD)[j4] =
+        make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
   }
 }
 
@@ -434,6 +427,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   const int nj = (n_chunks > g) ? (n_chunks - g + kDecWG - 1) / kDecWG : 0;   // this warpgroup's chunks
   uint8_t* my_stages = stages + static_cast<size_t>(g) * NS * cbytes;
 
+  // Q' inputs: threads 0..511 each own two consecutive dims of one query row (row tid / 64);
+  // their loads go out first, so their latency overlaps the setup below.
+  const int qh = tid >> 6, qd = 2 * (tid & 63);
+  float2 qin = make_float2(0.0f, 0.0f);
+  if (tid < 512 && qh < G) {
+    const int64_t qi = b * a.qsb + (hkv * G + qh) * a.qsh + qd;
+    qin = make_float2(load_f32(a.q, a.q_dtype, qi), load_f32(a.q, a.q_dtype, qi + 1));
+  }
+
   // ------------------------------------------------------------------ barriers, TMEM, setup copy
   if (tid == 0) {
     for (int gg = 0; gg < kDecWG; ++gg) {
@@ -449,7 +451,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
       S.wg_abort[gg] = 0;
     }
     tc::mbar_init(&S.setup, 1);
-    tc::mbar_init(&S.qready, 1);
     S.bad = 0;
     tc::mbar_fence_init();
     tc::mbar_arrive_expect_tx(&S.setup, kLutBytes + static_cast<uint32_t>(sizeof(kvq_head_alloc)));
@@ -526,8 +527,69 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
     record_status(a.status, KVQ_ERR_TIMEOUT);
   }
   __syncthreads();
-  const bool bad = S.bad != 0;
   const kvq_head_alloc& A = *reinterpret_cast<const kvq_head_alloc*>(sm + kAllocOff);
+  // ------------------------------------------------------------------ slot descriptors, Q'
+  // Q' row h: q_h * f_b * log2(e) / sqrt(d), scaled by 2^-e so its largest |value| is in
+  // [0.5, 1); qscale[h] = 2^e multiplies the product back. Built by all threads in three steps
+  // (row maxima, scaled rows, the B operand of S), one CTA barrier after each.
+  float* qtmp = reinterpret_cast<float*>(sm + kRecQOff);    // [8][128] fp32
+  if (tid < 512) {
+    const float sc = inv_sqrt_d * kLog2e;
+    qin.x *= A.dequant[qd % kH] * sc;
+    qin.y *= A.dequant[(qd + 1) % kH] * sc;
+    float mx = fmaxf(fabsf(qin.x), fabsf(qin.y));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) S.qmax[warp] = mx;
+  } else if (tid < 512 + kPlanSlots) {
+    // descriptor of plan slot i for the width-generic lookups (an empty slot reads the first
+    // codes of the stream through the width-1 table: finite values against zero Q' rows); a
+    // slot whose codes would start past the key stream marks the allocation unusable
+    const int i = tid - 512;
+    const uint32_t e = A.plan_slot[i];
+    uint32_t w = e & 15u, off = e >> 8;
+    if (w > 8 || (w > 0 && off >= static_cast<uint32_t>(kD * a.bits_k))) {
+      S.bad = 1;
+      record_status(a.status, KVQ_ERR_MISMATCH);
+    }
+    if (w == 0 || w > 5 || off >= static_cast<uint32_t>(kD * a.bits_k)) { w = 1; off = 0; }
+    S.kdesc[i] = make_uint4((off >> 5) * 128u, (off & 31u) | (2 * w) << 8 | (4 * w) << 16 | (6 * w) << 24,
+                            (1u << (2 * w)) - 1u, w <= 3 ? 128u : 4u);
+    S.kbase[i] = static_cast<uint32_t>(pair_off(static_cast<int>(w)));
+  } else if (tid >= 512 + 32 && tid < 512 + 32 + kPlanSlots / 4) {
+    const int bt = tid - 512 - 32;
+    uint32_t wmax = 0;
+    for (int i = 0; i < 4; ++i) wmax = max(wmax, A.plan_slot[4 * bt + i] & 15u);
+    S.bkind[bt] = wmax <= 5 ? 0 : 1;
+  }
+  __syncthreads();
+  if (tid < 512) {
+    const float mx = fmaxf(S.qmax[2 * qh], S.qmax[2 * qh + 1]);
+    int e = 0;
+    if (mx > 0.0f) frexpf(mx, &e);
+    const float sc = ldexpf(1.0f, -e);
+    *reinterpret_cast<float2*>(qtmp + qh * kD + qd) = make_float2(qin.x * sc, qin.y * sc);
+    if ((tid & 63) == 0) S.qscale[qh] = ldexpf(1.0f, e);
+  }
+  __syncthreads();
+  {
+    // B operand of S, K-major, no swizzle: element (n, k) at (k/8)*256 + (n/8)*128 + (n%8)*16 +
+    // (k%8)*2; K element k = 2c + r is dim b + 64 r of the block in column c; n < 8: hi part of
+    // row n, n >= 8: lo part.
+    const int k_elems = 2 * min(max(A.plan_k_cols, 0), 96);
+    for (int i = tid; i < 8 * k_elems; i += blockDim.x) {
+      const int n = i / k_elems, k = i - n * k_elems;
+      const int blk = A.plan_col_block[k >> 1];
+      __half hi = __float2half_rn(0.0f), lo = hi;
+      if (blk >= 0 && blk < kH) split_hilo(qtmp[n * kD + blk + kH * (k & 1)], hi, lo);
+      const int base = (k >> 3) * 256 + (k & 7) * 2;
+      *reinterpret_cast<__half*>(sm + kBQOff + base + n * 16) = hi;
+      *reinterpret_cast<__half*>(sm + kBQOff + base + 128 + n * 16) = lo;
+    }
+  }
+  tc::fence_proxy_async_smem();
+  __syncthreads();
+  const bool bad = S.bad != 0;
   volatile int* abort_flag = &S.wg_abort[g];
 
   float M[8], L[8];                                         // running max (log2) and row sums
@@ -536,45 +598,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   int done = 0;                                             // chunks this warpgroup completed
 
   if (!bad && is_issuer) {
-    // ------------------------------------------------------------------ Q' (issuer warps)
-    // Row h: q_h * f_b * log2(e) / sqrt(d), scaled by 2^-e so its largest |value| is in
-    // [0.5, 1); qscale[h] = 2^e multiplies the product back. B operand of S, K-major, no
-    // swizzle: element (n, k) at (k/8)*256 + (n/8)*128 + (n%8)*16 + (k%8)*2; K element k = 2c + r
-    // is dim b + 64 r of the block in column c; n < 8: hi part of row n, n >= 8: lo part.
     const int it = tid - 32 * kDecIssuerWarp0;              // 0..127
-    float* qtmp = reinterpret_cast<float*>(sm + kRecQOff);  // [8][128] fp32
-    for (int h = g; h < 8; h += kDecWG) {
-      float qv[4], mx = 0.0f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = lane + 32 * u;
-        qv[u] = (h < G) ? load_f32(a.q, a.q_dtype, b * a.qsb + (hkv * G + h) * a.qsh + j) : 0.0f;
-        qv[u] *= A.dequant[j % kH] * (inv_sqrt_d * kLog2e);
-        mx = fmaxf(mx, fabsf(qv[u]));
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      int e = 0;
-      if (mx > 0.0f) frexpf(mx, &e);
-      if (lane == 0) S.qscale[h] = ldexpf(1.0f, e);
-      const float sc = ldexpf(1.0f, -e);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) qtmp[h * kD + lane + 32 * u] = qv[u] * sc;
-    }
-    named_sync(kDecWG + 1, 128);
-    const int k_elems = 2 * A.plan_k_cols;
-    for (int i = it; i < 8 * k_elems; i += 128) {
-      const int n = i / k_elems, k = i - n * k_elems;
-      const int blk = A.plan_col_block[k >> 1];
-      __half hi = __float2half_rn(0.0f), lo = hi;
-      if (blk >= 0) split_hilo(qtmp[n * kD + blk + kH * (k & 1)], hi, lo);
-      const int base = (k >> 3) * 256 + (k & 7) * 2;
-      *reinterpret_cast<__half*>(sm + kBQOff + base + n * 16) = hi;
-      *reinterpret_cast<__half*>(sm + kBQOff + base + 128 + n * 16) = lo;
-    }
-    tc::fence_proxy_async_smem();
-    named_sync(kDecWG + 1, 128);
-    if (tid == 32 * kDecIssuerWarp0) tc::mbar_arrive(&S.qready);   // Q' scales for the compute warps
     // ---------------------------------------------------------------- issuing (one lane per warpgroup)
     if (issuer) {
       const uint32_t id_s = tc::idesc_f16(128, 16, false), id_o = tc::idesc_f16(128, 16, true, kBfO);
@@ -706,7 +730,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
     uint8_t* pbuf = sm + kBPOff + g * kBPBytes;
     const uint4* slots4 = reinterpret_cast<const uint4*>(A.plan_slot);
     float qs[8];
-    bool have_q = false;
+#pragma unroll
+    for (int h = 0; h < 8; ++h) qs[h] = S.qscale[h];
 
     for (int j = 0; j < nj; ++j) {
       const int ci = c_begin + g + kDecWG * j;
@@ -721,7 +746,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
       for (int bt = 0; bt < nb; ++bt) {
         const int kb = j * nb + bt, slot = kb & 1;
         uint32_t v16[16];
-        k_batch(kw, slots4[bt], sm, lane4, v16);
+        if (S.bkind[bt] == 0) k_batch_gen(kw, S.kdesc + 4 * bt, S.kbase + 4 * bt, sm, lane4, v16);
+        else k_batch(kw, slots4[bt], sm, lane4, v16);
         if (bt > 0) {
           tc::wait_st();
           tc::fence_before_sync();
@@ -770,12 +796,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
         }
       }
       // -------------------------------------------------------------- logits
-      if (!have_q) {
-        if (!tc::mbar_wait(&S.qready, 0, WL)) *abort_flag = 1;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) qs[h] = S.qscale[h];
-        have_q = true;
-      }
       if (!tc::mbar_wait(&S.sfull[g], j & 1, WL)) *abort_flag = 1;
       tc::fence_after_sync();
       float sv[8];
@@ -938,35 +958,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   if (a.splits == 1) return;
 
   // ------------------------------------------------------------------ two-level split merge
+  // The last CTA of each group of splits (ticket order) merges the group; the last group to
+  // finish merges the groups. A ticket is taken after the barrier that follows the writes it
+  // publishes, with acquire-release order at GPU scope (no separate fences).
   const int grp = split / a.group_size;
   const int m0 = grp * a.group_size, m1 = min(a.splits, m0 + a.group_size);
   unsigned* tk = a.tickets + static_cast<size_t>(bh) * (1 + a.n_groups);
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const unsigned t = atomicAdd(&tk[1 + grp], 1u);
+    const unsigned t = ticket_add(&tk[1 + grp]);
     S.last = (t == static_cast<unsigned>(m1 - m0 - 1));
     if (S.last) tk[1 + grp] = 0u;
   }
   __syncthreads();
   if (!S.last) return;
-  __threadfence();
   if (a.n_groups == 1) {
-    merge_entries(S, a, bh, pitch, m0, m1 - m0, -1, out_bh, G);
+    merge_entries(a, bh, pitch, m0, m1 - m0, -1, out_bh, G);
     return;
   }
-  merge_entries(S, a, bh, pitch, m0, m1 - m0, a.splits + grp, out_bh, G);
-  __threadfence();
+  merge_entries(a, bh, pitch, m0, m1 - m0, a.splits + grp, out_bh, G);
   __syncthreads();
   if (tid == 0) {
-    const unsigned t = atomicAdd(&tk[0], 1u);
+    const unsigned t = ticket_add(&tk[0]);
     S.last = (t == static_cast<unsigned>(a.n_groups - 1));
     if (S.last) tk[0] = 0u;
   }
   __syncthreads();
   if (!S.last) return;
-  __threadfence();
-  merge_entries(S, a, bh, pitch, a.splits, a.n_groups, -1, out_bh, G);
+  merge_entries(a, bh, pitch, a.splits, a.n_groups, -1, out_bh, G);
 }
 
 }  // namespace kvq

@@ -28,14 +28,50 @@ kvq_status cuda_fail(cudaError_t e) {
   return KVQ_ERR_CUDA;
 }
 
+// Identity of the calling thread's current CUDA context. Per-device state the library sets up
+// once (uploaded tables, shared-memory opt-ins, occupancy) is keyed on it, so a device whose
+// context was reset and created again gets that state again instead of trusting a stale flag.
+// The two driver functions are reached through the runtime, so the library has no link-time
+// dependency on the driver library. Returns 1 when the identity cannot be read (then every
+// context of the device counts as one).
+uint64_t context_id() {
+  using GetCurrent = int (*)(void**);
+  using GetId = int (*)(void*, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  });
+  if (!get_current || !get_id) return 1;
+  void* ctx = nullptr;
+  if (get_current(&ctx) != 0) return 1;
+  if (!ctx) {                               // no runtime call has made the primary context current yet
+    cudaFree(nullptr);
+    if (get_current(&ctx) != 0 || !ctx) return 1;
+  }
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != 0) return 1;
+  return static_cast<uint64_t>(id) + 2;
+}
+
 std::mutex g_upload_mu;
-bool g_uploaded[kMaxDevices] = {};
+uint64_t g_uploaded[kMaxDevices] = {};      // context the tables were uploaded to (0: none)
 
 kvq_status ensure_tables() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  const uint64_t ctx = context_id();
   std::lock_guard<std::mutex> lock(g_upload_mu);
-  if (g_uploaded[dev]) return KVQ_OK;
+  if (g_uploaded[dev] == ctx) return KVQ_OK;
   const Tables& t = tables();
   DevTables d;
   std::memcpy(d.centroid_f16, t.centroid_f16, sizeof(d.centroid_f16));
@@ -50,7 +86,7 @@ kvq_status ensure_tables() {
   static uint32_t qlut[2 * kLutEntries];
   if (!quant_lut_image(t.threshold, qlut)) return KVQ_ERR_UNSUPPORTED;
   { const cudaError_t e_ = cudaMemcpyToSymbol(g_quant_lut, qlut, sizeof(qlut)); if (e_ != cudaSuccess) return cuda_fail(e_); }
-  g_uploaded[dev] = true;
+  g_uploaded[dev] = ctx;
   return KVQ_OK;
 }
 
@@ -390,15 +426,17 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
   // width (they cost host time comparable to a small launch, e.g. a one-token append).
   static std::mutex occ_mu;
   static int occ[kMaxDevices][27] = {};
+  static uint64_t occ_ctx[kMaxDevices][27] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  const uint64_t ctx = context_id();
 #define KVQ_LAUNCH_QUANT(DT, TY, BV)                                                                              \
   do {                                                                                                            \
     auto kern = kvq_quant_pack<DT, BV>;                                                                           \
     int per_sm = 0;                                                                                               \
     {                                                                                                             \
       std::lock_guard<std::mutex> lock(occ_mu);                                                                   \
-      if (occ[dev][DT * 9 + BV] == 0) {                                                                           \
+      if (occ_ctx[dev][DT * 9 + BV] != ctx) {                                                                     \
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=    \
             cudaSuccess)                                                                                          \
           return KVQ_ERR_CUDA;                                                                                    \
@@ -406,6 +444,7 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, qw * 32, smem) != cudaSuccess)                \
           return KVQ_ERR_CUDA;                                                                                    \
         occ[dev][DT * 9 + BV] = std::max(1, n);                                                                   \
+        occ_ctx[dev][DT * 9 + BV] = ctx;                                                                          \
       }                                                                                                           \
       per_sm = occ[dev][DT * 9 + BV];                                                                             \
     }                                                                                                             \
@@ -552,12 +591,27 @@ kvq_status launch_decode(const void* q, const kvq_tensor4* qd, const void* packe
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(splits, bh);
   const int vm = dense_v ? (ex->vd.dtype == KVQ_BF16 ? kDenseBf16 : kDenseF16) : c->bits_v;
+  // The shared-memory opt-in is raised once per device and value mode to the largest size
+  // launched so far (the call costs host time comparable to the launch itself).
+  static std::mutex smem_mu;
+  static int smem_set[kMaxDevices][kDenseF16 + 1] = {};
+  static uint64_t smem_ctx[kMaxDevices][kDenseF16 + 1] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  const uint64_t ctx = context_id();
 #define KVQ_LAUNCH_DEC(VM)                                                                                            \
   do {                                                                                                                \
     auto kern = kvq_decode_gtq<VM>;                                                                                   \
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,                     \
-                                               static_cast<int>(smem));                                               \
-    if (e != cudaSuccess) return cuda_fail(e);                                                                        \
+    {                                                                                                                 \
+      std::lock_guard<std::mutex> lock(smem_mu);                                                                      \
+      if (smem_ctx[dev][VM] != ctx || smem_set[dev][VM] < static_cast<int>(smem)) {                                  \
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,                 \
+                                                   static_cast<int>(smem));                                           \
+        if (e != cudaSuccess) return cuda_fail(e);                                                                    \
+        smem_set[dev][VM] = static_cast<int>(smem);                                                                   \
+        smem_ctx[dev][VM] = ctx;                                                                                      \
+      }                                                                                                               \
+    }                                                                                                                 \
     kern<<<grid, kDecThreads, smem, s>>>(a);                                                                          \
   } while (0)
   switch (vm) {

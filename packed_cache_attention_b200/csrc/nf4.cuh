@@ -222,22 +222,38 @@ __global__ void __launch_bounds__(kNf4DecWarps * 32) kvq_nf4_decode(
     }
   }
   if (splits == 1) return;
-  __threadfence();
+  // ticket after the barrier that follows this CTA's writes (acquire-release at GPU scope);
+  // the last CTA folds the splits in eight at a time (one round trip to L2 per eight)
   __syncthreads();
-  if (tid == 0) sLast = (atomicAdd(&tickets[bh], 1u) == static_cast<unsigned>(splits - 1));
+  if (tid == 0) sLast = (ticket_add(&tickets[bh]) == static_cast<unsigned>(splits - 1));
   __syncthreads();
   if (!sLast) return;
-  __threadfence();
   if (tid < kD) {
     const size_t p0 = static_cast<size_t>(bh) * splits;
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(part_m + p0 + s));
-    float Ls = 0.0f, O = 0.0f;
-    for (int s = 0; s < splits; ++s) {
-      const float ms = __ldcg(part_m + p0 + s);
-      const float wt = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-      Ls += __ldcg(part_l + p0 + s) * wt;
-      O += __ldcg(part_o + (p0 + s) * kD + tid) * wt;
+    float M = -INFINITY, Ls = 0.0f, O = 0.0f;
+    for (int s0 = 0; s0 < splits; s0 += 8) {
+      float mv[8], lv[8], ov[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool in = s0 + u < splits;
+        mv[u] = in ? __ldcg(part_m + p0 + s0 + u) : -INFINITY;
+        lv[u] = in ? __ldcg(part_l + p0 + s0 + u) : 0.0f;
+        ov[u] = in ? __ldcg(part_o + (p0 + s0 + u) * kD + tid) : 0.0f;
+      }
+      float mx = M;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx = fmaxf(mx, mv[u]);
+      if (mx == -INFINITY) continue;
+      const float sc = (M == -INFINITY) ? 0.0f : fast_exp2(M - mx);
+      Ls *= sc;
+      O *= sc;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float wt = (mv[u] == -INFINITY) ? 0.0f : fast_exp2(mv[u] - mx);
+        Ls += lv[u] * wt;
+        O += ov[u] * wt;
+      }
+      M = mx;
     }
     out[static_cast<size_t>(bh) * kD + tid] = O / Ls;
   }
