@@ -10,7 +10,8 @@
 //   load     whole chunks (one bulk copy of 4 records) into the warpgroup's ring of stages,
 //            several chunks ahead;
 //   keys     lane = token: 16 K-hat columns at a time (4 slots of the allocation's plan, each
-//            4 block pairs of one width, looked up in shared-memory pair tables) go to a ring
+//            4 block pairs of one width, looked up in shared-memory pair tables; batches of
+//            widths <= 5 take one width-generic instruction sequence) go to a ring
 //            of two 16-column tensor-memory buffers; the issuer runs S^T[128 tokens][16] +=
 //            Khat x Q'^T (tcgen05.mma, M 128, N 16; Q' rows 0-7 fp16 high parts, 8-15 low
 //            parts) on each buffer as soon as it is full, while the next one is filled;
@@ -26,8 +27,9 @@
 // One issuing thread can have one product in flight at a time (about 130 cycles each at
 // these shapes), so four issuers keep four independent chains going.
 // Q' carries f_b, log2(e)/sqrt(d) and a per-row power of two that keeps its fp16 split in
-// range. The four warpgroups' (m, l, O) are combined in shared memory; splits then meet in a
-// two-level tree: the last CTA of each group of about sqrt(splits) splits (atomic ticket)
+// range; all threads build it once the tables land (q itself is loaded at kernel entry). The
+// four warpgroups' (m, l, O) are combined in shared memory; splits then meet in a two-level
+// tree: the last CTA of each group of about sqrt(splits) splits (acquire-release ticket)
 // merges the group, and the last group to finish merges the groups and writes out = O / l.
 // Keys-only caches (the Block-GTQ page reports key errors with only the keys quantized): the values of each
 // chunk arrive as dense bf16/fp16 rows next to the chunk's K records and are transposed into
