@@ -36,32 +36,68 @@
 //   token t's code at bit bits_v * t of the dim's stream (positions known at compile time).
 #pragma once
 
+#include <cmath>
 #include <cstring>
 
 #include "common.cuh"
 
 namespace kvq {
 
+// a * b + c for two pairs in one instruction, each rounded toward -infinity.
+__device__ __forceinline__ float2 fma2_rm(float2 a, float2 b, float2 c) {
+  uint64_t ua, ub, uc, ud;
+  memcpy(&ua, &a, 8);
+  memcpy(&ub, &b, 8);
+  memcpy(&uc, &c, 8);
+  asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(ud) : "l"(ua), "l"(ub), "l"(uc));
+  float2 d;
+  memcpy(&d, &ud, 8);
+  return d;
+}
+
 // ---------------------------------------------------------------- code lookup table
 
-// Grid of width w (2..8): cells of 1/s_w, s_w = 2^max(w-2, 1), half-range kLutHalf[w] cells.
-constexpr int kLutHalf[9] = {0, 0, 2, 4, 10, 24, 56, 128, 288};
-constexpr int kLutOffset[9] = {0, 0, 0, 4, 12, 32, 80, 192, 448};
-constexpr int kLutEntries = 1024;
+// Code of y for width w: the number of thresholds below y. A table maps y to a grid cell that
+// holds at most one threshold; entry {below, tau} of a cell is the number of thresholds below
+// its left edge and the threshold inside it (+inf if none), so code = below + (y > tau).
+// Widths 2..7: y in [-R, R), R = 2^(p-1), is mapped to u = y 2^-p + 0.5 in [0, 1) by one
+// multiply-add rounded down and saturated to [0, 1] (NaN to 0), and u to cell floor(u 2^q) by
+// a second one (the magic constant 1.5 * 2^23 puts the cell index in the low bits). Both round
+// down and 2^-q is a multiple of the spacing of fp32 values near u, so the cell is exactly
+// that of the real y; y >= R lands in the extra cell 2^q (all thresholds below). Cells are
+// 2^(p-q) = 1/s_w wide with s_w = 2^max(w-2, 1). Width 8 (1024 cells would not fit) clamps y
+// to [-K/s, K/s) first and takes the cell from one multiply-add.
+constexpr int kLutP[9] = {0, 0, 1, 2, 3, 3, 3, 3, 0};               // R = 2^(p-1)
+constexpr int kLutQ[9] = {0, 0, 2, 3, 5, 6, 7, 8, 0};               // 2^q cells (+1)
+constexpr int kLutHalf8 = 288;                                      // width 8: half-range in cells
+constexpr int kLutOffset[9] = {0, 0, 0, 5, 14, 47, 112, 241, 498};
+constexpr int kLutEntries = 498 + 2 * kLutHalf8;                    // 1074
 
 __host__ __device__ constexpr int lut_scale(int w) { return 1 << (w > 3 ? w - 2 : 1); }
 
 // Host: builds the table from the fp32 thresholds (all widths concatenated, width w at
-// 2^w - w - 1). Entry k of width w is {number of thresholds below the cell's left edge,
-// bits of the threshold inside the cell or +inf}. Returns false if a cell would hold two
-// thresholds or a threshold falls outside the grid.
+// 2^w - w - 1). Returns false if a cell would hold two thresholds or a threshold falls outside
+// the grid.
 inline bool quant_lut_image(const float* thresholds, uint32_t* out /* 2 * kLutEntries */) {
   for (int w = 2; w <= 8; ++w) {
     const float* t = thresholds + ((1 << w) - w - 1);
-    const int n = (1 << w) - 1, K = kLutHalf[w];
-    const double s = lut_scale(w);
-    for (int k = 0; k < 2 * K; ++k) {
-      const double lo = (k - K) / s, hi = (k - K + 1) / s;
+    const int n = (1 << w) - 1;
+    int cells;
+    double lo0, cw;
+    if (w <= 7) {
+      cells = (1 << kLutQ[w]) + 1;
+      cw = std::ldexp(1.0, kLutP[w] - kLutQ[w]);
+      lo0 = -std::ldexp(1.0, kLutP[w] - 1);
+      if (static_cast<double>(t[0]) < lo0 || static_cast<double>(t[n - 1]) >= -lo0) return false;
+    } else {
+      cells = 2 * kLutHalf8;
+      cw = 1.0 / lut_scale(8);
+      lo0 = -kLutHalf8 * cw;
+      if (static_cast<double>(t[0]) < lo0 || static_cast<double>(t[n - 1]) >= -lo0) return false;
+    }
+    for (int k = 0; k < cells; ++k) {
+      const double lo = lo0 + k * cw;
+      const double hi = (w <= 7 && k == cells - 1) ? INFINITY : lo + cw;
       uint32_t below = 0, inside = 0, tau = 0x7f800000u;
       for (int i = 0; i < n; ++i) {
         const double ti = t[i];
@@ -77,33 +113,47 @@ inline bool quant_lut_image(const float* thresholds, uint32_t* out /* 2 * kLutEn
       out[2 * (kLutOffset[w] + k)] = below;
       out[2 * (kLutOffset[w] + k) + 1] = tau;
     }
-    if (static_cast<double>(t[0]) < -K / s || static_cast<double>(t[n - 1]) >= K / s) return false;
   }
   return true;
 }
 
 __device__ __align__(16) uint32_t g_quant_lut[2 * kLutEntries];
 
-// Code of y for width W (1..8) from the table in shared memory (lut_s: its shared-memory
-// address). The entry of cell k sits at lut_s + 8 (offset + k), and k = bits(f) - 0x4B400000,
-// so the entry address is one multiply-add of bits(f) with a folded constant (32-bit shared
-// addresses wrap, so the constant's own wrap-around is harmless).
+// Entry of table address `addr` (a shared-memory byte address) compared with y.
+__device__ __forceinline__ uint32_t lut_entry_code(float y, uint32_t addr) {
+  uint32_t below, tau;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(below), "=r"(tau) : "r"(addr));
+  return below + (y > __uint_as_float(tau) ? 1u : 0u);
+}
+
+// Codes of y.x and y.y for width W (1..8) from the table in shared memory (lut_s: its
+// shared-memory address). The entry of cell k sits at lut_s + 8 (offset + k), and
+// k = bits(f) - 0x4B400000, so the entry address is one multiply-add of bits(f) with a folded
+// constant (32-bit shared addresses wrap, so the constant's own wrap-around is harmless).
 template <int W>
-__device__ __forceinline__ uint32_t lut_code(float y, uint32_t lut_s) {
+__device__ __forceinline__ uint2 lut_code2(float2 y, uint32_t lut_s) {
   if constexpr (W == 1) {
-    return y > 0.0f ? 1u : 0u;
+    return make_uint2(y.x > 0.0f ? 1u : 0u, y.y > 0.0f ? 1u : 0u);
   } else {
-    constexpr int K = kLutHalf[W];
-    constexpr float s = static_cast<float>(lut_scale(W));
-    constexpr float lo = -static_cast<float>(K) / s;
-    constexpr float hi = (static_cast<float>(K) - 0.5f) / s;   // inside the last cell
-    const float yc = fminf(fmaxf(y, lo), hi);                  // NaN -> lo
-    const float f = __fmaf_rd(yc, s, 12582912.0f + static_cast<float>(K));   // 1.5 * 2^23 + K + floor(yc s)
-    const uint32_t addr = static_cast<uint32_t>(__float_as_int(f)) * 8u +
-                          (lut_s + 8u * (static_cast<uint32_t>(kLutOffset[W]) - 0x4B400000u));
-    uint32_t below, tau;
-    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(below), "=r"(tau) : "r"(addr));
-    return below + (y > __uint_as_float(tau) ? 1u : 0u);
+    constexpr uint32_t base = 8u * (static_cast<uint32_t>(kLutOffset[W]) - 0x4B400000u);
+    float2 f;
+    if constexpr (W <= 7) {
+      constexpr float sp = 1.0f / static_cast<float>(1 << kLutP[W]);
+      constexpr float sq = static_cast<float>(1 << kLutQ[W]);
+      float2 u;
+      asm("fma.rm.sat.f32 %0, %1, %2, 0f3F000000;" : "=f"(u.x) : "f"(y.x), "f"(sp));
+      asm("fma.rm.sat.f32 %0, %1, %2, 0f3F000000;" : "=f"(u.y) : "f"(y.y), "f"(sp));
+      f = fma2_rm(u, make_float2(sq, sq), make_float2(12582912.0f, 12582912.0f));
+    } else {
+      constexpr float s = static_cast<float>(lut_scale(8));
+      constexpr float lo = -static_cast<float>(kLutHalf8) / s;
+      constexpr float hi = (static_cast<float>(kLutHalf8) - 0.5f) / s;   // inside the last cell
+      const float c = 12582912.0f + static_cast<float>(kLutHalf8);       // 1.5 * 2^23 + K + floor(yc s)
+      f.x = __fmaf_rd(fminf(fmaxf(y.x, lo), hi), s, c);                  // NaN -> lo
+      f.y = __fmaf_rd(fminf(fmaxf(y.y, lo), hi), s, c);
+    }
+    return make_uint2(lut_entry_code(y.x, static_cast<uint32_t>(__float_as_int(f.x)) * 8u + (lut_s + base)),
+                      lut_entry_code(y.y, static_cast<uint32_t>(__float_as_int(f.y)) * 8u + (lut_s + base)));
   }
 }
 
@@ -285,8 +335,9 @@ __device__ __forceinline__ void quant_k_class(const uint8_t* row, float2 aa, con
       const KEntry e = ent[k + j];
       const float2 x = block_pair<DT>(row, e);
       const float2 y = mul2(mul2(x, aa), make_float2(e.g, e.g));
-      buf += lut_code<W>(y.x, lut) << (2 * W * j);          // disjoint bit fields: + is |
-      buf += lut_code<W>(y.y, lut) << (2 * W * j + W);
+      const uint2 c = lut_code2<W>(y, lut);
+      buf += c.x << (2 * W * j);                            // disjoint bit fields: + is |
+      buf += c.y << (2 * W * j + W);
     }
     const int left = nb - k;
     int nbits = 2 * W * GB;
@@ -319,8 +370,8 @@ __device__ __forceinline__ void quant_v_tile(const uint32_t* rows, const float2*
       if constexpr (DT == KVQ_F32) x = *reinterpret_cast<const float2*>(rows + tok * Q::kPitch + j0);
       else x = unpack_pair<DT>(rows[tok * Q::kPitch + (j0 >> 1)]);
       const float2 y = mul2(x, sA2[tok]);
-      const uint32_t c0 = lut_code<BV>(y.x, lut);
-      const uint32_t c1 = lut_code<BV>(y.y, lut);
+      const uint2 cc = lut_code2<BV>(y, lut);
+      const uint32_t c0 = cc.x, c1 = cc.y;
       const int bit = BV * tok, wi = bit >> 5, sh = bit & 31;
       w0[wi] += c0 << sh;                                   // disjoint bit fields: + is |
       w1[wi] += c1 << sh;
