@@ -519,6 +519,23 @@ def oracle_sample(n_tokens: int, seed: int = 0, workload: str = WORKLOAD, batch:
     return time.perf_counter() - t0, B * n_tokens
 
 
+def oracle_nf4_sample(n_tokens: int, batch: int = 1, seed: int = 0):
+    """Time the oracle's NF4 quantize/pack of K and V and its MHA decode on the first n_tokens
+    of `batch` sequences of the OPT-30B-shaped workload (56 heads). Returns (seconds, layer-tokens)."""
+    from oracle import nqkv
+    from packed_cache_attention_b200 import workloads as wl
+    W = wl.WORKLOADS["nqkv_opt30b"]
+    y = wl.make_nf4_inputs(batch, W.n_q_heads, W.head_dim, n_tokens, W.dtype, seed=seed, device="cpu")
+    K, V, q = (t.float().numpy() for t in (y["K"], y["V"], y["q"]))
+    t0 = time.perf_counter()
+    ki, ks = nqkv.quantize(K)
+    vi, vs = nqkv.quantize(V)
+    kc, kss = nqkv.pack(ki, ks, n_tokens)
+    vc, vss = nqkv.pack(vi, vs, n_tokens)
+    nqkv.decode(q, kc, kss, vc, vss, W.n_q_heads, W.head_dim, n_tokens)
+    return time.perf_counter() - t0, batch * n_tokens
+
+
 def cpu_model() -> str:
     try:
         with open("/proc/cpuinfo") as fh:
@@ -532,7 +549,7 @@ def cpu_model() -> str:
 
 def cpu_baseline(n_tokens: int = 131072):
     """The oracle on the host cores: the 128K layer on one core, then bounded samples of every
-    Block-GTQ workload on one core and with numpy's default thread count (all cores)."""
+    workload on one core and with numpy's default thread count (all cores)."""
     from threadpoolctl import threadpool_limits
     with threadpool_limits(limits=1):
         secs, toks = oracle_sample(n_tokens)
@@ -547,6 +564,13 @@ def cpu_baseline(n_tokens: int = 131072):
             row[label] = tk / sec
         row["sample"] = f"first {n} tokens" + (f" of {bsz} sequences" if bsz else "")
         per[name] = row
+    row = {}
+    for label, lim in (("one_core", 1), ("all_cores", None)):
+        with threadpool_limits(limits=lim):
+            sec, tk = oracle_nf4_sample(1024)
+        row[label] = tk / sec
+    row["sample"] = "first 1024 tokens of 1 sequence, 56 heads"
+    per["nqkv_opt30b"] = row
     return {"value": toks / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"one layer of {WORKLOAD}, first {n_tokens} tokens of both KV heads: calibrate + quantize/pack "
                       f"+ decode for 16 q-heads ({secs:.1f} s)",

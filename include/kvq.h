@@ -184,7 +184,8 @@ size_t kvq_packed_header_bytes(int n_kv_heads);
  * 4 * head_dim * bits_k + 64 bytes). Returns 0 for an invalid descriptor. */
 size_t kvq_packed_bytes(const kvq_cache_desc* cache);
 
-/* Workspace bytes kvq_decode_attn needs for this cache and n_q_heads query heads. */
+/* Workspace bytes kvq_decode_attn needs for this cache and n_q_heads query heads (any
+ * seq_len up to the capacity). */
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* cache, int n_q_heads);
 
 /* ---------------------------------------------------------------- setup and status */
@@ -195,7 +196,10 @@ kvq_status kvq_init(void);
 
 /* Zero a decode or calibrate workspace (async memset on `stream`). Both hold counters that
  * must start at zero: zero a workspace once before its first use; the kernels return the
- * counters to zero, so it stays reusable. Calls sharing one workspace must not overlap. */
+ * counters to zero, so it stays reusable for every call on the same cache descriptor (the
+ * decode's counters sit where the descriptor's capacity puts them, whatever seq_len). Zero
+ * it again before using it with a descriptor of another batch, head count or capacity.
+ * Calls sharing one workspace must not overlap. */
 kvq_status kvq_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronizes `stream`, copies the workspace status word to *device_code (host) and
@@ -371,11 +375,15 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
  * - The array's address is looked up on every call. The first call on a device (and the
  *   first after its context was created again) zeroes the array with an asynchronous memset
  *   on `stream`, ordered before the decode; make that first call before any stream capture.
- * - Shapes whose decode workspace (kvq_decode_workspace_bytes) exceeds the array return
- *   KVQ_ERR_WORKSPACE before anything is launched.
+ * - The array's first 64 KiB hold the status word and the split counters of every call, the
+ *   partials follow. Shapes whose counters (batch * n_kv_heads rows) do not fit there, or
+ *   whose partials do not fit in the rest, return KVQ_ERR_WORKSPACE before anything is
+ *   launched.
  * - Every call on a device shares the one array, which keeps the last call's contents; the
- *   split counters in it that must start at zero are returned to zero by every call. Calls
- *   that overlap on the GPU (other streams, other host threads) race on it: serialize them.
+ *   split counters, which must start at zero, are returned to zero by every call and never
+ *   share bytes with partials, so calls on caches of different shapes can follow each
+ *   other. Calls that overlap on the GPU (other streams, other host threads) race on it:
+ *   serialize them.
  * - A device-side wait that gave up is recorded in the array's status word; read it with
  *   kvq_decode_noalloc_status. */
 kvq_status kvq_decode_attn_noalloc(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,

@@ -85,6 +85,15 @@ __device__ __forceinline__ unsigned ticket_add(unsigned* p) {
   return old;
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization may
+// start while the previous kernel in its stream is still finishing; it must not touch memory
+// that kernel may write (or read) before grid_dependency_wait(), which returns once the previous
+// grid has completed and its writes are visible (at once for a normal launch).
+// allow_dependents() lets the next such kernel start as soon as every CTA of this grid has
+// called it or exited.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));

@@ -58,6 +58,7 @@ constexpr int kTau = 8;                   // lazy rescale threshold (log2 units)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPlanSlots = 24;
 constexpr int kMergeMax = 64;             // group size bound of the split merge
+constexpr int kMergeBatch = 10;           // merge entries loaded in one round trip
 constexpr uint32_t kHeaderMagic = 0x3151564Bu;   // "KVQ1"
 constexpr int kLayoutVersion = 1;
 
@@ -305,7 +306,8 @@ struct DecArgs {
   float* part_m;                     // [bh][splits + n_groups][8]
   float* part_l;
   float* part_o;                     // [bh][splits + n_groups][8][128]
-  unsigned* tickets;                 // [bh][1 + n_groups]
+  unsigned* tickets;                 // [bh][ticket_stride]: final counter, then one per merge group
+  int ticket_stride;
   unsigned* status;
   uint32_t wait_limit;
   int debug_no_loads;                // test hook: issue no copy, so every wait on a stage gives up
@@ -316,8 +318,9 @@ struct DecArgs {
 // Merges entries e0 .. e0 + n - 1 of row bh, each (m, l, O) with O unnormalized and m in log2
 // units, into entry `dst_entry` (>= 0) or into out = O / l (dst_entry < 0). Thread (h, j4) of
 // the first 256 keeps a running (M, L, O[4 j4 .. 4 j4 + 3]) of row h and folds the entries in
-// eight at a time: the loads of eight entries are issued together, so the merge costs
-// ceil(n / 8) round trips to L2 and no CTA barrier. The order of the sums is fixed.
+// kMergeBatch at a time: the loads of a batch are issued together, so a merge of up to
+// kMergeBatch entries (every merge step when splits <= kMergeBatch^2) costs one round trip to
+// L2 and no CTA barrier. The order of the sums is fixed.
 __device__ __forceinline__ void merge_entries(const DecArgs& a, int bh, int pitch, int e0, int n, int dst_entry,
                                               float* out_bh, int G) {
   const int tid = threadIdx.x;
@@ -327,11 +330,11 @@ __device__ __forceinline__ void merge_entries(const DecArgs& a, int bh, int pitc
   const float4* po = reinterpret_cast<const float4*>(a.part_o);
   float M = -INFINITY, L = 0.0f;
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < n; s0 += 8) {
-    float mv[8], lv[8];
-    float4 ov[8];
+  for (int s0 = 0; s0 < n; s0 += kMergeBatch) {
+    float mv[kMergeBatch], lv[kMergeBatch];
+    float4 ov[kMergeBatch];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < kMergeBatch; ++u) {
       if (s0 + u < n) {
         const size_t e = row + s0 + u;
         mv[u] = __ldcg(a.part_m + e * 8 + h);
@@ -345,13 +348,13 @@ __device__ __forceinline__ void merge_entries(const DecArgs& a, int bh, int pitc
     }
     float mx = M;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) mx = fmaxf(mx, mv[u]);
+    for (int u = 0; u < kMergeBatch; ++u) mx = fmaxf(mx, mv[u]);
     if (mx == -INFINITY) continue;
     const float sc = (M == -INFINITY) ? 0.0f : fast_exp2(M - mx);
     L *= sc;
     o.x *= sc; o.y *= sc; o.z *= sc; o.w *= sc;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < kMergeBatch; ++u) {
       const float wt = (mv[u] == -INFINITY) ? 0.0f : fast_exp2(mv[u] - mx);
       L += lv[u] * wt;
       o.x += ov[u].x * wt; o.y += ov[u].y * wt; o.z += ov[u].z * wt; o.w += ov[u].w * wt;
@@ -429,16 +432,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   const int nj = (n_chunks > g) ? (n_chunks - g + kDecWG - 1) / kDecWG : 0;   // this warpgroup's chunks
   uint8_t* my_stages = stages + static_cast<size_t>(g) * NS * cbytes;
 
-  // Q' inputs: threads 0..511 each own two consecutive dims of one query row (row tid / 64);
-  // their loads go out first, so their latency overlaps the setup below.
-  const int qh = tid >> 6, qd = 2 * (tid & 63);
-  float2 qin = make_float2(0.0f, 0.0f);
-  if (tid < 512 && qh < G) {
-    const int64_t qi = b * a.qsb + (hkv * G + qh) * a.qsh + qd;
-    qin = make_float2(load_f32(a.q, a.q_dtype, qi), load_f32(a.q, a.q_dtype, qi + 1));
-  }
-
   // ------------------------------------------------------------------ barriers, TMEM, setup copy
+  // Barrier initialisation, the tensor-memory allocation and the copy of the library's own
+  // lookup tables read none of the caller's memory: they run before the wait for the previous
+  // kernel in the stream (programmatic dependent launch), everything else after it.
   if (tid == 0) {
     for (int gg = 0; gg < kDecWG; ++gg) {
       for (int i = 0; i < kStagesMax; ++i) tc::mbar_init(&S.full[gg][i], 1);
@@ -457,10 +454,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
     tc::mbar_fence_init();
     tc::mbar_arrive_expect_tx(&S.setup, kLutBytes + static_cast<uint32_t>(sizeof(kvq_head_alloc)));
     tc::bulk_g2s(sm, g_dec_lut, kLutBytes, &S.setup);
-    tc::bulk_g2s(sm + kAllocOff, al, sizeof(kvq_head_alloc), &S.setup);
   }
   if (tid < 8) S.wg_m[kDecWG][tid] = -INFINITY;             // no recent share unless the issuers add one
   if (warp == kDecIssuerWarp0) tc::tmem_alloc(&S.tmem_base, kTmemCols);
+  grid_dependency_wait();
+  if (tid == 0) tc::bulk_g2s(sm + kAllocOff, al, sizeof(kvq_head_alloc), &S.setup);
+  // Q' inputs: threads 0..511 each own two consecutive dims of one query row (row tid / 64);
+  // their loads go out first, so their latency overlaps the setup below.
+  const int qh = tid >> 6, qd = 2 * (tid & 63);
+  float2 qin = make_float2(0.0f, 0.0f);
+  if (tid < 512 && qh < G) {
+    const int64_t qi = b * a.qsb + (hkv * G + qh) * a.qsh + qd;
+    qin = make_float2(load_f32(a.q, a.q_dtype, qi), load_f32(a.q, a.q_dtype, qi + 1));
+  }
   if (tid == 32) {
     // The packed header must name this layout, these widths and shapes, and this head's
     // allocation; a status left by an append is reported as is. All fields are loaded
@@ -895,6 +901,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
     }
   }
   __syncthreads();
+  allow_dependents();                                       // the next kernel may start on freed SMs
   bool aborted = bad;
 #pragma unroll
   for (int gg = 0; gg < kDecWG; ++gg) aborted |= S.wg_abort[gg] != 0;
@@ -965,7 +972,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   // publishes, with acquire-release order at GPU scope (no separate fences).
   const int grp = split / a.group_size;
   const int m0 = grp * a.group_size, m1 = min(a.splits, m0 + a.group_size);
-  unsigned* tk = a.tickets + static_cast<size_t>(bh) * (1 + a.n_groups);
+  unsigned* tk = a.tickets + static_cast<size_t>(bh) * a.ticket_stride;
   __syncthreads();
   if (tid == 0) {
     const unsigned t = ticket_add(&tk[1 + grp]);

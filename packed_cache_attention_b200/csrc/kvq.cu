@@ -7,6 +7,7 @@
 #include <cstddef>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "calibrate.cuh"
 #include "common.cuh"
@@ -142,24 +143,37 @@ int nf4_splits(int bh, int n_groups) {
 }
 
 // Block-GTQ decode: splits of whole 128-token chunks, at most one CTA per SM in total (a
-// second partial wave would double the time of the CTAs in it).
+// second partial wave would double the time of the CTAs in it). A CTA's four warpgroups take
+// its chunks in turn, so its time is set by ceil(chunks / 4); the fewest splits that keep that
+// number are used, which leaves the time as it is and makes the split merge smaller.
 constexpr int kMaxGtqSplits = kMergeMax * kMergeMax;
+// Upper bound of the split count for any length up to n_tiles tiles (it grows with n_tiles):
+// the decode workspace is sized with it, so one workspace serves every length of a cache.
+int gtq_splits_max(int bh, int n_tiles) {
+  const int n_chunks = (n_tiles + kChunkTiles - 1) / kChunkTiles;
+  return std::max(1, std::min(std::min(sm_count() / bh, n_chunks), kMaxGtqSplits));
+}
 int gtq_splits(int bh, int n_tiles) {
   const int n_chunks = (n_tiles + kChunkTiles - 1) / kChunkTiles;
-  const int want = std::max(1, sm_count() / bh);
-  return std::max(1, std::min(std::min(want, n_chunks), kMaxGtqSplits));
+  if (n_chunks == 0) return 1;                              // recent tokens only
+  const int most = gtq_splits_max(bh, n_tiles);
+  const int per_wg = (n_chunks + kDecWG * most - 1) / (kDecWG * most);
+  return std::max(1, (n_chunks + kDecWG * per_wg - 1) / (kDecWG * per_wg));
 }
 
 struct DecodeWs {
   size_t tickets, part_m, part_l, part_o, total;
 };
 
-// Workspace of the decode kernels: tickets (per row: one final counter, then one counter per
-// merge group), then (m, l, O) partials for `entries` entries per row.
-DecodeWs decode_ws_layout(int bh, int entries, int rows, int groups) {
+// Workspace of the decode kernels: tickets (`ticket_stride` counters per row: one final
+// counter, then one per merge group), then (m, l, O) partials for `entries` entries per row,
+// starting no earlier than `part_base`. The ticket region of a workspace must not move between
+// calls: the last CTA returns every counter it used to zero, and a counter that once held a
+// partial would start a later call at a wrong count.
+DecodeWs decode_ws_layout(int bh, int entries, int rows, int ticket_stride, size_t part_base = 0) {
   DecodeWs w;
   w.tickets = sizeof(WsHeader);
-  w.part_m = align_up(w.tickets + 4ull * bh * (1 + groups), 128);
+  w.part_m = std::max<size_t>(align_up(w.tickets + 4ull * bh * ticket_stride, 128), part_base);
   w.part_l = align_up(w.part_m + 4ull * bh * entries * rows, 128);
   w.part_o = align_up(w.part_l + 4ull * bh * entries * rows, 128);
   w.total = align_up(w.part_o + 4ull * bh * entries * rows * kD, 128);
@@ -170,15 +184,23 @@ DecodeWs decode_ws_layout(int bh, int entries, int rows, int groups) {
 struct MergePlan {
   int group_size, n_groups;
 };
+// Split merge plan: one level (the last CTA merges every split) while that takes at most two
+// batched round trips to L2; above that, groups of about sqrt(splits), so each level is one.
 MergePlan merge_plan(int splits) {
+  if (splits <= 2 * kMergeBatch) return MergePlan{splits, 1};
   int gs = 1;
   while (gs * gs < splits) ++gs;
   return MergePlan{gs, (splits + gs - 1) / gs};
 }
 
-DecodeWs gtq_ws_layout(int bh, int splits) {
+// Tickets per row for a cache: one final counter plus the merge groups of the largest split
+// count any of its lengths uses, so the ticket region stays put for every call on the cache.
+int gtq_ticket_stride(int bh, int capacity_tiles) {
+  return 1 + merge_plan(gtq_splits_max(bh, capacity_tiles)).n_groups;
+}
+DecodeWs gtq_ws_layout(int bh, int splits, int ticket_stride, size_t part_base = 0) {
   const MergePlan mp = merge_plan(splits);
-  return decode_ws_layout(bh, splits + mp.n_groups, 8, mp.n_groups);
+  return decode_ws_layout(bh, splits + mp.n_groups, 8, ticket_stride, part_base);
 }
 
 int sm_count() {
@@ -191,6 +213,24 @@ int sm_count() {
     cached[dev] = n > 0 ? n : 148;
   }
   return cached[dev];
+}
+
+// Launches `kern` with programmatic stream serialization: it may begin (barrier setup, its
+// own tables) while the previous kernel in the stream finishes; the kernels wait for that
+// grid before they touch the caller's memory.
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
 }
 
 kvq_status launch_status() {
@@ -320,7 +360,8 @@ size_t kvq_packed_bytes(const kvq_cache_desc* c) {
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* c, int n_q_heads) {
   if (!cache_ok(c) || n_q_heads < 1) return 0;
   const int bh = c->batch * c->n_kv_heads;
-  return gtq_ws_layout(bh, gtq_splits(bh, n_tiles_of(c->capacity))).total;
+  const int cap_tiles = n_tiles_of(c->capacity);
+  return gtq_ws_layout(bh, gtq_splits_max(bh, cap_tiles), gtq_ticket_stride(bh, cap_tiles)).total;
 }
 
 kvq_status kvq_init(void) { return ensure_tables(); }
@@ -451,11 +492,12 @@ kvq_status launch_quant(const void* K, const kvq_tensor4* kd, const void* V, con
     const long long want = (n_tasks + qw - 1) / qw;                                                             \
     const unsigned grid =                                                                                         \
         static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sm_count()) * std::max(1, per_sm))); \
-    kern<<<grid, qw * 32, smem, s>>>(static_cast<const TY*>(K), kd->stride_b, kd->stride_h, kd->stride_t,         \
-                                     static_cast<const TY*>(V), vsb, vsh, vst, t_begin, t_end, tile_lo, n_tiles,  \
-                                     c->n_kv_heads, tiles_cap, static_cast<const kvq_head_alloc*>(alloc),         \
-                                     c->bits_k, c->bits_v, static_cast<uint8_t*>(packed), rec,                    \
-                                     static_cast<int>(n_tasks), qh);                                              \
+    const cudaError_t le = launch_pdl(kern, dim3(grid), dim3(qw * 32), smem, s, static_cast<const TY*>(K),         \
+                                      kd->stride_b, kd->stride_h, kd->stride_t, static_cast<const TY*>(V), vsb,  \
+                                      vsh, vst, t_begin, t_end, tile_lo, n_tiles, c->n_kv_heads, tiles_cap,      \
+                                      static_cast<const kvq_head_alloc*>(alloc), c->bits_k, c->bits_v,           \
+                                      static_cast<uint8_t*>(packed), rec, static_cast<int>(n_tasks), qh);        \
+    if (le != cudaSuccess) return cuda_fail(le);                                                                  \
   } while (0)
 #define KVQ_QUANT_BV(DT, TY)                                                                                      \
   switch (c->bits_v) {                                                                                            \
@@ -504,7 +546,7 @@ kvq_status check_kv_view(const void* p, const kvq_tensor4* t, const kvq_cache_de
 
 kvq_status launch_decode(const void* q, const kvq_tensor4* qd, const void* packed, const void* alloc,
                          const kvq_cache_desc* c, int seq_len, const kvq_decode_extra* ex, float* out, void* ws,
-                         size_t ws_bytes, void* stream) {
+                         size_t ws_bytes, void* stream, size_t part_base = 0) {
   kvq_status st;
   if ((st = check_tensor(q, qd)) != KVQ_OK) return st;
   if (!packed || !alloc || !out || !aligned16(packed) || !aligned16(alloc)) return KVQ_ERR_ARG;
@@ -529,7 +571,8 @@ kvq_status launch_decode(const void* q, const kvq_tensor4* qd, const void* packe
   const int n_tiles = n_tiles_of(seq_len);
   const int splits = gtq_splits(bh, n_tiles);
   const MergePlan mp = merge_plan(splits);
-  const DecodeWs L = gtq_ws_layout(bh, splits);
+  const int ticket_stride = gtq_ticket_stride(bh, n_tiles_of(c->capacity));
+  const DecodeWs L = gtq_ws_layout(bh, splits, ticket_stride, part_base);
   if (!ws || ws_bytes < L.total || !aligned16(ws) || ws_bytes < kvq_decode_workspace_bytes(c, qd->n_heads))
     return KVQ_ERR_WORKSPACE;
   if ((st = ensure_tables()) != KVQ_OK) return st;
@@ -585,6 +628,7 @@ kvq_status launch_decode(const void* q, const kvq_tensor4* qd, const void* packe
   a.part_l = reinterpret_cast<float*>(w8 + L.part_l);
   a.part_o = reinterpret_cast<float*>(w8 + L.part_o);
   a.tickets = reinterpret_cast<unsigned*>(w8 + L.tickets);
+  a.ticket_stride = ticket_stride;
   a.status = reinterpret_cast<unsigned*>(w8);
   a.wait_limit = g_wait_limit;
   a.debug_no_loads = g_debug_no_loads;
@@ -612,7 +656,8 @@ kvq_status launch_decode(const void* q, const kvq_tensor4* qd, const void* packe
         smem_ctx[dev][VM] = ctx;                                                                                      \
       }                                                                                                               \
     }                                                                                                                 \
-    kern<<<grid, kDecThreads, smem, s>>>(a);                                                                          \
+    const cudaError_t le = launch_pdl(kern, grid, dim3(kDecThreads), smem, s, a);                                     \
+    if (le != cudaSuccess) return cuda_fail(le);                                                                      \
   } while (0)
   switch (vm) {
     case 1: KVQ_LAUNCH_DEC(1); break;
@@ -676,7 +721,7 @@ size_t kvq_nf4_packed_bytes(int batch, int n_heads, int capacity, int head_dim) 
 size_t kvq_nf4_decode_workspace_bytes(int batch, int n_heads, int capacity, int head_dim) {
   if (batch < 1 || n_heads < 1 || capacity < 1 || head_dim != kD) return 0;
   const int bh = batch * n_heads;
-  return decode_ws_layout(bh, nf4_splits(bh, (capacity + 31) / 32), 1, 0).total;
+  return decode_ws_layout(bh, nf4_splits(bh, (capacity + 31) / 32), 1, 1).total;
 }
 
 namespace {
@@ -748,7 +793,7 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
   if (seq_len < 1 || seq_len > capacity) return KVQ_ERR_RANGE;
   const int bh = qd->batch * qd->n_heads;
   const int splits = nf4_splits(bh, (seq_len + 31) / 32);
-  const DecodeWs Lw = decode_ws_layout(bh, splits, 1, 0);
+  const DecodeWs Lw = decode_ws_layout(bh, splits, 1, 1);
   if (!ws || ws_bytes < Lw.total || !aligned16(ws) ||
       ws_bytes < kvq_nf4_decode_workspace_bytes(qd->batch, qd->n_heads, capacity, kD))
     return KVQ_ERR_WORKSPACE;
@@ -787,6 +832,7 @@ kvq_status kvq_nf4_decode_attn(const void* q, const kvq_tensor4* qd, const void*
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 2u << 20;   // 2 MiB per device
+constexpr size_t kNoAllocTicketBytes = 64 * 1024;   // status word and split tickets of every call
 __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
 std::mutex g_scratch_mu;
@@ -822,12 +868,20 @@ kvq_status kvq_decode_attn_noalloc(const void* q, const kvq_tensor4* qd, const v
   if (!qd || !cache_ok(cache)) return KVQ_ERR_ARG;
   const size_t need = kvq_decode_workspace_bytes(cache, qd->n_heads);
   if (need == 0) return KVQ_ERR_ARG;
-  if (need > kNoAllocScratchBytes) return KVQ_ERR_WORKSPACE;
+  // Split tickets live in a fixed area at the start of the array, so calls on caches of any
+  // shape use counters that the previous calls returned to zero; the partials follow it.
+  const int bh = cache->batch * cache->n_kv_heads;
+  const int cap_tiles = n_tiles_of(cache->capacity);
+  const int stride = gtq_ticket_stride(bh, cap_tiles);
+  if (sizeof(WsHeader) + 4ull * bh * stride > kNoAllocTicketBytes) return KVQ_ERR_WORKSPACE;
+  if (gtq_ws_layout(bh, gtq_splits_max(bh, cap_tiles), stride, kNoAllocTicketBytes).total > kNoAllocScratchBytes)
+    return KVQ_ERR_WORKSPACE;
   kvq_status st = ensure_tables();
   if (st != KVQ_OK) return st;
   void* scratch = nullptr;
   if ((st = decode_scratch(static_cast<cudaStream_t>(stream), &scratch)) != KVQ_OK) return st;
-  return kvq_decode_attn(q, qd, packed, alloc, cache, seq_len, out, scratch, kNoAllocScratchBytes, stream);
+  return launch_decode(q, qd, packed, alloc, cache, seq_len, nullptr, out, scratch, kNoAllocScratchBytes, stream,
+                       kNoAllocTicketBytes);
 }
 
 kvq_status kvq_decode_noalloc_status(void* stream, int* device_code) {

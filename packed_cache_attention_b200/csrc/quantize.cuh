@@ -468,6 +468,9 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
   for (int i = threadIdx.x; i < kLutEntries; i += blockDim.x)
     sLut[i] = make_uint2(g_quant_lut[2 * i], g_quant_lut[2 * i + 1]);
   const uint32_t lut_s = static_cast<uint32_t>(__cvta_generic_to_shared(sLut));
+  // The table is the library's own; the caller's memory is touched only after the previous
+  // kernel in the stream is done with it (programmatic dependent launch).
+  grid_dependency_wait();
   if (threadIdx.x == 0) sHeaderOk = (qh.mode == 2) ? packed_header_ok(packed, qh, n_kv_heads, bits_k, bits_v, rec_bytes, alloc) : 1;
   if (qh.mode == 1 && blockIdx.x == 0 && threadIdx.x < 32)
     write_packed_header(packed, qh, n_kv_heads, bits_k, bits_v, rec_bytes, alloc, threadIdx.x);
@@ -620,6 +623,7 @@ __global__ void __launch_bounds__(QTile<DT>::kWarps * 32, 1) kvq_quant_pack(
     }
     bh = nbh; tile = ntile; r_lo = nlo; r_hi = nhi;
   }
+  allow_dependents();                                       // this warp has no task left
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 

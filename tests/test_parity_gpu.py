@@ -221,6 +221,26 @@ def test_repeated_decode_reuses_workspace(dev):
     assert kvq.kvq_workspace_status(ws) == 0
 
 
+def test_workspace_serves_every_length_of_a_cache(dev):
+    """One workspace sized for a cache serves decodes of any length in any order, including a
+    long length (two-level split merge) right after short ones (one split, one-level merge):
+    each output equals the decode with a freshly zeroed workspace, bit for bit."""
+    import torch
+    T = 131072
+    x = wl.make_blockgtq_inputs(1, 16, 2, 128, T, "bf16", 1e6, "lognormal_outliers", seed=17, device=dev)
+    alloc = kvq.kvq_calibrate(x["K"], 3)
+    cache = kvq.cache_desc(1, 2, T, 3, 3)
+    packed = kvq.kvq_quantize(x["K"], x["V"], alloc, cache)
+    nbytes = kvq.kvq_decode_workspace_bytes(cache, 16)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    for n in (300, 5000, T, 700, 40000, T, 1):
+        got = kvq.kvq_decode_attn(x["q"], packed, alloc, cache, n, ws=ws).clone()
+        fresh = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        want = kvq.kvq_decode_attn(x["q"], packed, alloc, cache, n, ws=fresh)
+        assert torch.equal(got, want), n
+        assert kvq.kvq_workspace_status(ws) == 0
+
+
 APPEND_CASES = [("bf16", 3, 3), ("f16", 5, 7), ("f32", 2, 4)]
 
 
@@ -336,6 +356,25 @@ def test_decode_refuses_another_layers_allocation(dev):
     assert kvq.kvq_workspace_status(ws) == 0
     _, _, ref = oracle_pipeline(x["K"], x["V"], x["q"], 3, 3)
     assert rel_err(got, ref) <= TOL
+
+
+def test_decode_refuses_a_slot_plan_past_the_key_stream(dev):
+    """An allocation whose decode plan points a slot of KV head 0 past the key stream (its
+    digest still matching the cache) is refused before any lookup: KVQ_ERR_MISMATCH, the
+    query rows of head 0 untouched, head 1 decoded as with the intact allocation."""
+    import torch
+    x, alloc, cache, packed = _layer(dev, 65)
+    bad = alloc.clone()
+    off = kvq.HeadAlloc.plan_slot.offset                         # head 0, slot 0
+    word = 3 | ((128 * 3 + 5) << 8)                              # width 3, first code past 384 bits
+    bad[off:off + 4] = torch.tensor(list(int(word).to_bytes(4, "little")), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(kvq.kvq_decode_workspace_bytes(cache, 8), dtype=torch.uint8, device=dev)
+    out = torch.full((1, 8, 128), 3.0, device=dev)
+    kvq.kvq_decode_attn(x["q"], packed, bad, cache, 300, out=out, ws=ws)
+    assert kvq.kvq_workspace_status(ws) == kvq.KVQ_ERR_MISMATCH
+    assert torch.all(out[:, :4] == 3.0)
+    good = kvq.kvq_decode_attn(x["q"], packed, alloc, cache, 300)
+    assert torch.equal(out[:, 4:], good[:, 4:])
 
 
 def test_append_refuses_another_allocation(dev):
