@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta, 32 / kCalibChunksPerC
   const int chunk = blockIdx.x * kCalibChunksPerCta + (threadIdx.x >> 4);
   const int k = threadIdx.x & 15;
   const int n_seg = (n_chunks + kCalibSegment - 1) / kCalibSegment;
+  grid_dependency_wait();                                   // K and the counters may be the previous kernel's
   if (chunk < n_chunks) {
     const int u0 = chunk * kCalibChunk;
     const int n = min(N - u0, kCalibChunk);
@@ -129,17 +130,18 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta, 32 / kCalibChunksPerC
   const int seg = (blockIdx.x * kCalibChunksPerCta) / kCalibSegment;
   const int c0 = seg * kCalibSegment, c1 = min(n_chunks, c0 + kCalibSegment);
   const int mine = min(n_chunks, (blockIdx.x + 1) * kCalibChunksPerCta) - blockIdx.x * kCalibChunksPerCta;
-  __threadfence();
+  allow_dependents();
+  // tickets are taken after the barrier that follows the writes they publish, with
+  // acquire-release order at GPU scope (no separate fences)
   __syncthreads();
   if (threadIdx.x == 0) {
     unsigned* cnt = ws.seg_count + static_cast<size_t>(h) * n_seg + seg;
-    const unsigned done = atomicAdd(cnt, static_cast<unsigned>(mine)) + mine;
+    const unsigned done = ticket_add(cnt, static_cast<unsigned>(mine)) + mine;
     sTicket = (done == static_cast<unsigned>(c1 - c0));
     if (sTicket) *cnt = 0u;
   }
   __syncthreads();
   if (!sTicket) return;
-  __threadfence();
   if (threadIdx.x < kH) {
     const double* src = ws.chunk_sum + (static_cast<size_t>(h) * n_chunks) * kH + threadIdx.x;
     double acc = 0.0;
@@ -148,16 +150,14 @@ __global__ void __launch_bounds__(16 * kCalibChunksPerCta, 32 / kCalibChunksPerC
     ws.seg_sum[(static_cast<size_t>(h) * n_seg + seg) * kH + threadIdx.x] = acc;
   }
   // ---- head completion
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    const unsigned done = atomicAdd(ws.head_count + h, 1u) + 1u;
+    const unsigned done = ticket_add(ws.head_count + h) + 1u;
     sTicket = (done == static_cast<unsigned>(n_seg));
     if (sTicket) ws.head_count[h] = 0u;
   }
   __syncthreads();
   if (!sTicket) return;
-  __threadfence();
   if (threadIdx.x < kH) {
     const double* src = ws.seg_sum + static_cast<size_t>(h) * n_seg * kH + threadIdx.x;
     double S = 0.0;
@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(512) kvq_greedy_alloc(const double* __restrict
   uint32_t* rec_words = reinterpret_cast<uint32_t*>(&sRec);
   constexpr int kRecWords = static_cast<int>(sizeof(kvq_head_alloc) / 4);
   for (int i = tid; i < kRecWords; i += blockDim.x) rec_words[i] = 0u;
+  grid_dependency_wait();                                   // the energies come from the reduction
   if (tid < kH) sE[tid] = __ldcg(energy + static_cast<size_t>(h) * kH + tid);
   __syncthreads();
   if (tid == 0) {

@@ -79,9 +79,9 @@ __host__ __device__ __forceinline__ uint64_t splitmix64(uint64_t z) {
 // thread right after the CTA barrier that follows the CTA's writes of its partial result, it
 // publishes those writes (release); for the thread that draws the last ticket it also makes
 // the earlier arrivers' writes visible (acquire) to every thread past the next CTA barrier.
-__device__ __forceinline__ unsigned ticket_add(unsigned* p) {
+__device__ __forceinline__ unsigned ticket_add(unsigned* p, unsigned n = 1u) {
   unsigned old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(n) : "memory");
   return old;
 }
 

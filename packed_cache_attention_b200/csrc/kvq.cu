@@ -407,22 +407,24 @@ kvq_status kvq_calibrate(const void* K, const kvq_tensor4* kd, const kvq_calib_p
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid((n_chunks + kCalibChunksPerCta - 1) / kCalibChunksPerCta, kd->n_heads);
   const int threads = 16 * kCalibChunksPerCta;
+  cudaError_t le;
   switch (kd->dtype) {
     case KVQ_F32:
-      kvq_calib_reduce<KVQ_F32><<<grid, threads, 0, s>>>(static_cast<const float*>(K), n_calib, kd->stride_b,
-                                                         kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
+      le = launch_pdl(kvq_calib_reduce<KVQ_F32>, grid, dim3(threads), 0, s, static_cast<const float*>(K), n_calib,
+                      kd->stride_b, kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
       break;
     case KVQ_F16:
-      kvq_calib_reduce<KVQ_F16><<<grid, threads, 0, s>>>(static_cast<const __half*>(K), n_calib, kd->stride_b,
-                                                         kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
+      le = launch_pdl(kvq_calib_reduce<KVQ_F16>, grid, dim3(threads), 0, s, static_cast<const __half*>(K), n_calib,
+                      kd->stride_b, kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
       break;
     default:
-      kvq_calib_reduce<KVQ_BF16><<<grid, threads, 0, s>>>(static_cast<const __nv_bfloat16*>(K), n_calib, kd->stride_b,
-                                                          kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
+      le = launch_pdl(kvq_calib_reduce<KVQ_BF16>, grid, dim3(threads), 0, s, static_cast<const __nv_bfloat16*>(K),
+                      n_calib, kd->stride_b, kd->stride_h, kd->stride_t, static_cast<int>(N), n_chunks, cws);
   }
-  if ((st = launch_status()) != KVQ_OK) return st;
-  kvq_greedy_alloc<<<kd->n_heads, 512, 0, s>>>(cws.energy, p->bits_k, p->w_max, p->mode,
-                                               static_cast<kvq_head_alloc*>(alloc_out));
+  if (le != cudaSuccess) return cuda_fail(le);
+  le = launch_pdl(kvq_greedy_alloc, dim3(kd->n_heads), dim3(512), 0, s, static_cast<const double*>(cws.energy),
+                  p->bits_k, p->w_max, p->mode, static_cast<kvq_head_alloc*>(alloc_out));
+  if (le != cudaSuccess) return cuda_fail(le);
   return launch_status();
 }
 
