@@ -27,10 +27,13 @@
 // One issuing thread can have one product in flight at a time (about 130 cycles each at
 // these shapes), so four issuers keep four independent chains going.
 // Q' carries f_b, log2(e)/sqrt(d) and a per-row power of two that keeps its fp16 split in
-// range; all threads build it once the tables land (q itself is loaded at kernel entry). The
-// four warpgroups' (m, l, O) are combined in shared memory; splits then meet in a two-level
-// tree: the last CTA of each group of about sqrt(splits) splits (acquire-release ticket)
+// range; all threads build it once the tables land. The four warpgroups' (m, l, O) are
+// combined in shared memory; up to 20 splits then meet at the last CTA to finish (acquire-
+// release ticket), more in two levels: the last CTA of each group of about sqrt(splits) splits
 // merges the group, and the last group to finish merges the groups and writes out = O / l.
+// Launched with programmatic dependent launch: barrier setup, the tensor-memory allocation
+// and the copy of the library's own tables run before the wait for the previous kernel in the
+// stream; nothing of the caller's memory is read or written before it.
 // Keys-only caches (the Block-GTQ page reports key errors with only the keys quantized): the values of each
 // chunk arrive as dense bf16/fp16 rows next to the chunk's K records and are transposed into
 // tensor memory (lane = dim); O then runs on bf16 (or fp16) operands with P' split to match.
@@ -966,7 +969,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
   }
   if (a.splits == 1) return;
 
-  // ------------------------------------------------------------------ two-level split merge
+  // ------------------------------------------------------------------ split merge (one or two levels)
   // The last CTA of each group of splits (ticket order) merges the group; the last group to
   // finish merges the groups. A ticket is taken after the barrier that follows the writes it
   // publishes, with acquire-release order at GPU scope (no separate fences).

@@ -180,7 +180,7 @@ DecodeWs decode_ws_layout(int bh, int entries, int rows, int ticket_stride, size
   return w;
 }
 
-// Two-level merge of `splits` partials: groups of about sqrt(splits).
+// Merge of `splits` partials: groups of group_size splits, n_groups of them (1: one level).
 struct MergePlan {
   int group_size, n_groups;
 };
