@@ -13,6 +13,11 @@
  * levels) to that device with a synchronous copy, so it must not be made while a stream is
  * being captured; kvq_init() does the upload explicitly.
  *
+ * Calibrate, quantize/append and the Block-GTQ decode are launched with programmatic
+ * dependent launch: such a kernel may start (barriers, tensor memory, the library's own tables)
+ * while the previous kernel in the stream is finishing, but reads and writes none of the
+ * caller's memory until that kernel has completed, so stream order holds as for any launch.
+ *
  * Sources (restated in each declaration):
  *   [BGTQ] "RoPE-aware bit allocation for KV cache quantization" (Liang, Zhang, Jia;
  *          arXiv 2606.24033), abstract.
