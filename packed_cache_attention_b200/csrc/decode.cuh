@@ -276,6 +276,20 @@ __device__ __forceinline__ float from_ordered(int i) { return __int_as_float(i ^
 
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
+// Named barrier over n threads that also returns the OR of `v` over them.
+__device__ __forceinline__ bool named_sync_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void record_status(unsigned* status, unsigned code) { atomicCAS(status, 0u, code); }
 
 // Element i of a tensor of run-time dtype (kvq_dtype) as fp32.
@@ -821,25 +835,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
         }
       }
       // -------------------------------------------------------------- chunk maximum
+      // The running maximum moves only when a logit of the chunk exceeds it by more than
+      // 2^tau. One barrier with an OR vote over the warpgroup finds out; only then are the
+      // row maxima of the chunk exchanged and O rescaled.
+      bool over = false;
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        const int m = __reduce_max_sync(0xffffffffu, ordered(sv[h]));
-        if (lane == 0) S.xch[g][q][h] = from_ordered(m);
-      }
-      named_sync(1 + g, 128);
+      for (int h = 0; h < 8; ++h) over |= sv[h] > M[h] + static_cast<float>(kTau);
+      const bool any_over = named_sync_or(1 + g, 128, over);
       if (*abort_flag) break;
-      bool resc = false;
-      float cm[8];
+      if (any_over) {
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        cm[h] = fmaxf(fmaxf(S.xch[g][0][h], S.xch[g][1][h]), fmaxf(S.xch[g][2][h], S.xch[g][3][h]));
-        resc |= cm[h] > M[h] + static_cast<float>(kTau);
-      }
-      if (resc) {
+        for (int h = 0; h < 8; ++h) {
+          const int m = __reduce_max_sync(0xffffffffu, ordered(sv[h]));
+          if (lane == 0) S.xch[g][q][h] = from_ordered(m);
+        }
+        named_sync(1 + g, 128);
         float alpha[8];
 #pragma unroll
         for (int h = 0; h < 8; ++h) {
-          const float mn = fmaxf(M[h], cm[h]);
+          const float cm = fmaxf(fmaxf(S.xch[g][0][h], S.xch[g][1][h]), fmaxf(S.xch[g][2][h], S.xch[g][3][h]));
+          const float mn = fmaxf(M[h], cm);
           alpha[h] = (M[h] == -INFINITY) ? 0.0f : fast_exp2(M[h] - mn);
           M[h] = mn;
           L[h] *= alpha[h];
