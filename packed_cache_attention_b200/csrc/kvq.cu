@@ -87,6 +87,9 @@ kvq_status ensure_tables() {
   static uint32_t qlut[2 * kLutEntries];
   if (!quant_lut_image(t.threshold, qlut)) return KVQ_ERR_UNSUPPORTED;
   { const cudaError_t e_ = cudaMemcpyToSymbol(g_quant_lut, qlut, sizeof(qlut)); if (e_ != cudaSuccess) return cuda_fail(e_); }
+  static uint32_t nlut[2 * kNf4LutCells];
+  if (!nf4_lut_image(t.nf4_mid, nlut)) return KVQ_ERR_UNSUPPORTED;
+  { const cudaError_t e_ = cudaMemcpyToSymbol(g_nf4_lut, nlut, sizeof(nlut)); if (e_ != cudaSuccess) return cuda_fail(e_); }
   g_uploaded[dev] = ctx;
   return KVQ_OK;
 }

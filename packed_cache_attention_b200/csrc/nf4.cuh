@@ -9,6 +9,9 @@
 //   block blk of a token covers heads 2*blk (values 0..127) and 2*blk+1 (values 128..255).
 #pragma once
 
+#include <cmath>
+#include <cstring>
+
 #include "common.cuh"
 
 namespace kvq {
@@ -22,6 +25,51 @@ struct Nf4Layout {
     return (static_cast<size_t>(b) * nblk + blk) * t_pad + t;
   }
 };
+
+// Index search: u = x / scale lies in [-1, 1] (up to the fp16 rounding of the scale). A
+// table cuts [-1, 1) into 32 cells of 1/16, narrower than the smallest gap between the stored
+// midpoints, so a cell holds at most one; entry {below, tau} of a cell is the number of
+// midpoints below its left edge and the midpoint inside it (+inf if none), and the index
+// #{midpoints < u} is below + (u > tau). The cell comes from v = u/2 + 1/2 rounded down and
+// saturated to [0, 1] (NaN to 0), then floor(32 v) from a second round-down multiply-add
+// against 1.5 * 2^23: both steps round down at power-of-two scales, so the cell is exactly
+// the real u's cell; u >= 1 lands in the extra cell 32 (all midpoints below).
+constexpr int kNf4LutCells = 33;
+
+// Host: the index table from the 15 fp32 midpoints; false if a cell would hold two or a
+// midpoint lies outside [-1, 1).
+inline bool nf4_lut_image(const float* mid, uint32_t* out /* 2 * kNf4LutCells */) {
+  if (static_cast<double>(mid[0]) < -1.0 || static_cast<double>(mid[14]) >= 1.0) return false;
+  for (int k = 0; k < kNf4LutCells; ++k) {
+    const double lo = -1.0 + k / 16.0, hi = (k == kNf4LutCells - 1) ? INFINITY : lo + 1.0 / 16.0;
+    uint32_t below = 0, inside = 0, tau = 0x7f800000u;
+    for (int i = 0; i < 15; ++i) {
+      const double m = mid[i];
+      if (m < lo) ++below;
+      else if (m < hi) {
+        ++inside;
+        std::memcpy(&tau, &mid[i], 4);
+      }
+    }
+    if (inside > 1) return false;
+    out[2 * k] = below;
+    out[2 * k + 1] = tau;
+  }
+  return true;
+}
+
+__device__ __align__(16) uint32_t g_nf4_lut[2 * kNf4LutCells];
+
+// NF4 index of u from the table in shared memory (lut_s: its shared-memory address).
+__device__ __forceinline__ uint32_t nf4_index(float u, uint32_t lut_s) {
+  float v;
+  asm("fma.rm.sat.f32 %0, %1, 0f3F000000, 0f3F000000;" : "=f"(v) : "f"(u));
+  const float f = __fmaf_rd(v, 32.0f, 12582912.0f);
+  const uint32_t addr = static_cast<uint32_t>(__float_as_int(f)) * 8u + (lut_s - 8u * 0x4B400000u);
+  uint32_t below, tau;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(below), "=r"(tau) : "r"(addr));
+  return below + (u > __uint_as_float(tau) ? 1u : 0u);
+}
 
 constexpr int kNf4Rows = 4;   // token rows per warp task
 constexpr int kNf4DecWarps = 16;   // warps per CTA of the NF4 decode
@@ -39,9 +87,10 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
     const typename Elem<DT>::T* __restrict__ V, int64_t vsb, int64_t vsh, int64_t vst, int batch,
     int t_begin, int t_end, int t_stop, Nf4Layout L, uint8_t* __restrict__ packed) {
   using T = typename Elem<DT>::T;
-  __shared__ float sMid[16];
-  if (threadIdx.x < 15) sMid[threadIdx.x] = c_tab.nf4_mid[threadIdx.x];
+  __shared__ uint2 sLut[kNf4LutCells];
+  if (threadIdx.x < kNf4LutCells) sLut[threadIdx.x] = make_uint2(g_nf4_lut[2 * threadIdx.x], g_nf4_lut[2 * threadIdx.x + 1]);
   __syncthreads();
+  const uint32_t lut_s = static_cast<uint32_t>(__cvta_generic_to_shared(sLut));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g_lo = t_begin / kNf4Rows;
   const int groups = (t_stop + kNf4Rows - 1) / kNf4Rows - g_lo;
@@ -100,10 +149,7 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float u = (s == 0.0f) ? 0.0f : __fdiv_rn(x[rr][i], s);
-      int idx = 0;
-#pragma unroll
-      for (int k = 3; k >= 0; --k) idx += (u > sMid[idx + (1 << k) - 1]) ? (1 << k) : 0;
-      word |= static_cast<uint32_t>(idx) << (4 * i);
+      word |= nf4_index(u, lut_s) << (4 * i);
     }
     if (t >= t_end) word = 0u;
     codes[lane] = word;
