@@ -138,8 +138,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int sm_count();
 
-// NF4 decode: about 8 waves of two 16-warp CTAs per SM, so the hardware's CTA scheduling
-// evens out the last wave, and at least one 32-token group per warp in every CTA.
+// NF4 decode: about 16 CTAs per SM in all (four waves of four 8-warp CTAs), so the hardware's
+// CTA scheduling evens out the last wave, and at least one 32-token group per warp in every
+// CTA.
 int nf4_splits(int bh, int n_groups) {
   const int want = (16 * sm_count() + bh - 1) / bh;
   return std::max(1, std::min(std::min(want, n_groups / kNf4DecWarps), kNf4MaxSplits));

@@ -72,7 +72,7 @@ __device__ __forceinline__ uint32_t nf4_index(float u, uint32_t lut_s) {
 }
 
 constexpr int kNf4Rows = 4;   // token rows per warp task
-constexpr int kNf4DecWarps = 16;   // warps per CTA of the NF4 decode
+constexpr int kNf4DecWarps = 8;    // warps per CTA of the NF4 decode (four CTAs per SM)
 constexpr int kNf4MaxSplits = 160;  // splits per (sequence, head) the NF4 merge reads
 
 // One warp per (K-or-V, sequence, block, group of 4 token rows). Lane l holds values 8l..8l+7
@@ -157,8 +157,8 @@ __global__ void __launch_bounds__(kNf4Warps * 32, 4) kvq_nf4_quant_pack(
   }
 }
 
-// MHA decode (G = 1), CUDA cores. Grid (splits, batch * n_heads), 4 warps per CTA, each
-// warp every 4th 32-token group of the CTA's range. Q.K: lane t scores token t of the
+// MHA decode (G = 1), CUDA cores. Grid (splits, batch * n_heads), kNf4DecWarps warps per CTA,
+// each warp every kNf4DecWarps-th 32-token group of the CTA's range. Q.K: lane t scores token t of the
 // group from its 64 code bytes; P.V: lane l accumulates dims 4l..4l+3 over the group.
 template <int DT>
 __global__ void __launch_bounds__(kNf4DecWarps * 32) kvq_nf4_decode(
