@@ -17,11 +17,12 @@
 //            parts) on each buffer as soon as it is full, while the next one is filled;
 //   values   lane = dim: V-hat^T rows (one fp16 pair of tokens per column) go to their own 64
 //            columns while the S products run;
-//   softmax  lane = token: logits s = S * key norm * 2^e (per row), the chunk's maximum per
-//            row over the warpgroup, and an online softmax whose running maximum is only
-//            raised when a chunk exceeds it by more than 2^8 (then O is rescaled in tensor
-//            memory); P' = 2^(s - m - 8) * value norm / sqrt(d), split into fp16 hi + lo, is
-//            the B operand of O;
+//   softmax  lane = token: logits s = S * key norm * 2^e (per row, log2 units); an online
+//            softmax whose running maximum m is only raised when some logit of the chunk
+//            exceeds it by more than 8: one OR vote over the warpgroup decides, and only then
+//            are the chunk's row maxima exchanged and O rescaled in tensor memory;
+//            P' = 2^(s - m - 8) * value norm / sqrt(d), split into fp16 hi + lo, is the B
+//            operand of O;
 //   O        the issuer runs O^T[128 dims][16] += Vhat^T x P'^T, accumulated over all of the
 //            warpgroup's chunks in tensor memory.
 // One issuing thread can have one product in flight at a time (about 130 cycles each at
@@ -835,9 +836,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) kvq_decode_gtq(const DecArgs a
         }
       }
       // -------------------------------------------------------------- chunk maximum
-      // The running maximum moves only when a logit of the chunk exceeds it by more than
-      // 2^tau. One barrier with an OR vote over the warpgroup finds out; only then are the
-      // row maxima of the chunk exchanged and O rescaled.
+      // The running maximum moves only when a logit of the chunk exceeds it by more than tau
+      // (log2 units: a factor 2^tau once exponentiated). One barrier with an OR vote over the
+      // warpgroup finds out; only then are the row maxima of the chunk exchanged and O
+      // rescaled.
       bool over = false;
 #pragma unroll
       for (int h = 0; h < 8; ++h) over |= sv[h] > M[h] + static_cast<float>(kTau);

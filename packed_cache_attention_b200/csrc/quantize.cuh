@@ -21,11 +21,11 @@
 // Code search. Width 1 is the sign. Wider codebooks use a lookup table on a uniform grid
 // of cells of 2^-max(w-2, 1) over [-R_w, R_w): no cell holds two thresholds, so for y in cell k
 //   code = (thresholds below the cell) + (y > the threshold inside the cell, if any),
-// with y clamped into the grid (NaN clamps to the lowest cell and compares false, so a NaN
-// scale yields code 0: tokens past the sequence end are written as code 0). The cell is
-// floor(y / cell) read off an fp32 fma rounded toward minus infinity into [2^23, 2^24).
-// This is the same count as a search over the sorted thresholds, ties going to the lower
-// code, for every fp32 y.
+// with y brought into the grid by a saturating multiply-add (widths 2..7) or a clamp (width
+// 8); NaN lands in the lowest cell and compares false, so a NaN scale yields code 0 (tokens
+// past the sequence end are written as code 0). The cell index is read off an fp32
+// multiply-add rounded toward minus infinity into [2^23, 2^24). This is the same count as a
+// search over the sorted thresholds, ties going to the lower code, for every fp32 y.
 //
 // K: lane t quantizes token t and appends its codes, in the allocation's stream order, to a
 //   32-bit accumulator; the accumulator fills at the same code for every lane, so each full
