@@ -271,6 +271,14 @@ def test_greedy_tie_breaks_to_lowest_block():
     gains = [E[b] * (delta[w[b]] - delta[w[b] + 1]) for b in range(2)]
     assert gains[0] == gains[1]
     np.testing.assert_array_equal(bg.greedy_widths(E, 1, 8), [1, 1])
+    # a tie that decides the result: E = (1, 1, 4), budget 3. With delta = (1, 0.3634,
+    # 0.1175, 0.0345, ..) the gains are: step 1 (0.637, 0.637, 2.55) -> block 2; step 2
+    # (0.637, 0.637, 0.984) -> block 2; step 3 (0.637, 0.637, 0.332): blocks 0 and 1 tie
+    # exactly (the same product), the lower one wins -> (1, 0, 2), not (0, 1, 2)
+    E = np.array([1.0, 1.0, 4.0])
+    assert E[2] * (delta[1] - delta[2]) > delta[0] - delta[1] > E[2] * (delta[2] - delta[3])
+    np.testing.assert_array_equal(bg.greedy_widths(E, 1, 8), [1, 0, 2])
+    assert _objective(E, [1, 0, 2]) == _objective(E, [0, 1, 2])      # both optimal: only the rule decides
 
 
 def test_equal_energies_give_uniform_tqmse():
@@ -406,6 +414,17 @@ def test_quantizer_tie_goes_to_lower_code():
     x[0] = np.nextafter(t32[5], np.float32(10))
     codes, _ = bg.quantize_rows(x[None], np.full(4, 3), np.ones(4, np.float32))
     assert codes[0, 0] == 6
+    # with the block gain g_0 = 2 the coordinate t/2 lands on the threshold (y_0 = (t/2 * 1) * 2
+    # = t exactly: code 5), and the next fp32 value above t/2 lands above it (code 6)
+    g = np.ones(4, np.float32)
+    g[0] = 2.0
+    x[0] = t32[5] / np.float32(2)
+    x[1] = np.float32(math.sqrt(4.0 - float(x[0]) ** 2))              # the norm stays exactly 2
+    codes, n16 = bg.quantize_rows(x[None], np.full(4, 3), g)
+    assert float(n16[0]) == 2.0 and codes[0, 0] == 5
+    x[0] = np.nextafter(t32[5] / np.float32(2), np.float32(10))
+    codes, n16 = bg.quantize_rows(x[None], np.full(4, 3), g)
+    assert float(n16[0]) == 2.0 and codes[0, 0] == 6
 
 
 def _norm_row(ones_at):
@@ -780,6 +799,24 @@ def test_nf4_quantize_special_cases():
     assert s[0, 0, 2] == 0.25 and np.all(idx[0, 0, 2] == 0)           # every value equals -absmax -> -1
 
 
+def test_nf4_midpoint_goes_to_lower_index():
+    """idx = #{midpoints < u}: a value exactly on midpoint i takes index i (the lower level),
+    the next fp32 value above it index i + 1. One 256-value block with absmax 1 (scale 1, so
+    u = x exactly): x_0 = 1, x_{1+i} = m_i, x_{16+i} = nextafter(m_i, +inf), the rest 0."""
+    m = np.asarray(cb.nf4_midpoints(), dtype=np.float32)
+    X = np.zeros((1, 2, 1, 128), np.float32)
+    row = X[0, 0, 0]
+    row[0] = 1.0
+    row[1:16] = m
+    row[16:31] = np.nextafter(m, np.float32(2))
+    idx, s = nqkv.quantize(X)
+    assert s[0, 0, 0] == 1.0
+    assert idx[0, 0, 0, 0] == 15
+    np.testing.assert_array_equal(idx[0, 0, 0, 1:16], np.arange(15))
+    np.testing.assert_array_equal(idx[0, 0, 0, 16:31], np.arange(1, 16))
+    assert np.all(idx[0, 0, 0, 31:] == 7)                                # zeros: the exact-zero level
+
+
 def test_nf4_pack_roundtrip_and_padding():
     rng = np.random.default_rng(19)
     idx = rng.integers(0, 16, size=(2, 3, 21, 256)).astype(np.uint8)
@@ -820,9 +857,11 @@ def test_nf4_decode_masks_padding():
     idx, s = nqkv.quantize(X)
     kc, ks = nqkv.pack(idx, s, 19)
     out = nqkv.decode(q, kc, ks, kc, ks, 2, 128, 19)
-    kc2 = kc.copy()
-    kc2[:, :, 19:] = 0x77                                             # garbage in the padded rows
-    out2 = nqkv.decode(q, kc2, ks, kc2, ks, 2, 128, 19)
+    kc2, ks2 = kc.copy(), ks.copy()
+    kc2[:, :, 19:] = 0x77                                             # garbage codes in the padded rows
+    ks2[:, :, 19:] = 1.0                                              # and non-zero scales
+    out2 = nqkv.decode(q, kc2, ks2, kc2, ks2, 2, 128, 19)
     np.testing.assert_array_equal(out, out2)
-    xh = nqkv.dequantize(*nqkv.unpack(kc, ks, 19), 2, 128)
+    # attention over exactly the 19 quantized tokens, straight from the quantizer's output
+    xh = nqkv.dequantize(idx, s, 2, 128)
     np.testing.assert_allclose(out, bg.decode_attention(q.astype(np.float64), xh, xh), rtol=1e-14)
