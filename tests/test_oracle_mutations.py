@@ -9,12 +9,25 @@ import math
 
 import numpy as np
 import pytest
+from scipy.special import ndtri
 
 from oracle import blockgtq as bg
 from oracle import codebooks as cb
 from oracle import nqkv
 from oracle import rope
 from tests import test_oracle_pins as pins
+
+@pytest.fixture(autouse=True, scope="module")
+def _true_tables_cached():
+    """Fill the oracle's cached tables before any mutation, so that no cached table is ever
+    built from a mutated function and carried into later tests."""
+    for w in range(1, 9):
+        cb.lloyd_max_f64(w)
+        cb.stored_codebook(w)
+    cb.delta_table()
+    cb.nf4_values()
+    cb.nf4_midpoints()
+
 
 _orig = {
     "calibration_energies": bg.calibration_energies,
@@ -240,6 +253,46 @@ def nf4_unpack_padding_too(codes, scales, seq_len):
     return _orig["nqkv_unpack"](codes, scales, codes.shape[2])
 
 
+# ---------------------------------------------------------------- codebooks
+
+def lloyd_five_iterations(w):
+    """Lloyd-Max stopped after five Lloyd iterations from the compander start."""
+    n = 1 << w
+    c = math.sqrt(3.0) * ndtri((np.arange(n) + 0.5) / n)
+    for _ in range(5):
+        c = cb._conditional_means(c)[0]
+    return c, 0.5 * (c[:-1] + c[1:])
+
+
+def thresholds_from_exact_centroids(w):
+    """Stored thresholds as midpoints of the exact centroids instead of the stored fp16 ones."""
+    c, _ = cb.lloyd_max_f64(w)
+    return c.astype(np.float16), (0.5 * (c[:-1] + c[1:])).astype(np.float32)
+
+
+def centroids_rounded_toward_zero(w):
+    c, _ = cb.lloyd_max_f64(w)
+    c16 = c.astype(np.float16)
+    away = np.abs(c16.astype(np.float64)) > np.abs(c)
+    c16 = np.where(away, np.nextafter(c16, np.float16(0)), c16).astype(np.float16)
+    c16d = c16.astype(np.float64)
+    return c16, (0.5 * (c16d[:-1] + c16d[1:])).astype(np.float32)
+
+
+def delta_of_exact_quantizer():
+    """Distortions of the exact Lloyd-Max quantizers instead of the stored ones."""
+    return np.array([1.0] + [cb.quantizer_mse(*cb.lloyd_max_f64(w)) for w in range(1, 9)]).astype(np.float32)
+
+
+def nf4_sides_swapped():
+    """Eight negative and seven positive quantiles instead of seven and eight."""
+    off = 0.5 * ((1.0 - 1.0 / 30) + (1.0 - 1.0 / 32))
+    pos = ndtri(np.linspace(off, 0.5, 8)[:-1])
+    neg = -ndtri(np.linspace(off, 0.5, 9)[:-1])
+    v = np.sort(np.concatenate([neg, [0.0], pos]))
+    return (v / np.max(np.abs(v))).astype(np.float32)
+
+
 _pack_bits = bg.pack_bits
 _rotate = rope.rotate
 _nf4_quantize = nqkv.quantize
@@ -299,6 +352,16 @@ CASES = [
      [pins.test_nf4_pack_roundtrip_and_padding]),
     ("NF4: padded rows attended", nqkv, "unpack", nf4_unpack_padding_too,
      [pins.test_nf4_decode_masks_padding]),
+    ("Lloyd-Max: not run to convergence", cb, "lloyd_max_f64", lloyd_five_iterations,
+     [lambda: pins.test_lloyd_max_centroids_are_conditional_means(3), pins.test_lloyd_max_textbook_distortions]),
+    ("codebook: thresholds from the exact centroids", cb, "stored_codebook", thresholds_from_exact_centroids,
+     [pins.test_threshold_count_is_nearest_centroid]),
+    ("codebook: centroids rounded toward zero", cb, "stored_codebook", centroids_rounded_toward_zero,
+     [pins.test_stored_codebooks_symmetric_and_sorted]),
+    ("greedy table: exact instead of stored distortions", cb, "delta_table", delta_of_exact_quantizer,
+     [pins.test_delta_table_is_the_stored_quantizers_mse]),
+    ("NF4 levels: the two sides swapped", cb, "nf4_values", nf4_sides_swapped,
+     [pins.test_nf4_matches_published_table, pins.test_nf4_structure_and_quantile_spacing]),
 ]
 
 

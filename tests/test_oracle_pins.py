@@ -136,6 +136,25 @@ def test_delta_table_convex_and_close_to_exact():
         assert exact * (1 - 1e-7) <= delta[w] <= exact * (1 + 1e-7) + shift ** 2
 
 
+def test_delta_table_is_the_stored_quantizers_mse():
+    """delta[w] is the MSE on N(0,1) of the quantizer as stored (fp16 centroids, fp32
+    thresholds), by adaptive quadrature of (x - c)^2 phi(x) over its cells, within one fp32
+    ulp; for w >= 3 that is several ulps away from the exact Lloyd-Max MSE, so the table
+    cannot be the exact quantizer's."""
+    delta = cb.delta_table()
+    for w in range(1, 9):
+        c16, t32 = cb.stored_codebook(w)
+        c = c16.astype(np.float64)
+        edges = np.concatenate([[-np.inf], t32.astype(np.float64), [np.inf]])
+        mse = math.fsum(integrate.quad(lambda x: (x - ci) ** 2 * norm.pdf(x), lo, hi, epsabs=1e-16, epsrel=1e-13)[0]
+                        for lo, hi, ci in zip(edges[:-1], edges[1:], c))
+        ulp = float(np.spacing(delta[w]))
+        assert abs(float(delta[w]) - mse) <= ulp, (w, float(delta[w]), mse)
+        if w >= 3:
+            ce, te = cb.lloyd_max_f64(w)
+            assert abs(float(delta[w]) - cb.quantizer_mse(ce, te)) > 2 * ulp
+
+
 @pytest.mark.parametrize("w", [1, 2, 3, 4])
 def test_stored_quantizer_monte_carlo(w):
     """10^7 N(0,1) draws through the fp32 threshold quantizer: MSE within 3 sigma of delta(w)."""
