@@ -293,6 +293,44 @@ def nf4_sides_swapped():
     return (v / np.max(np.abs(v))).astype(np.float32)
 
 
+# ---------------------------------------------------------------- tile records and header
+
+def k_words_token_major(codes, alloc, bits_v, capacity):
+    """A token's K words stored contiguously (token-major) instead of word-planar."""
+    out = _pack_cache(codes, alloc, bits_v, capacity).copy()
+    nk = bg.tile_k_words(int(alloc["bits_k"]), int(alloc["d"]))
+    kw = out[..., :4 * nk].copy().view("<u4")
+    kw = kw.reshape(kw.shape[:-1] + (nk // bg.TILE, bg.TILE)).swapaxes(-1, -2).reshape(kw.shape)
+    out[..., :4 * nk] = np.ascontiguousarray(kw).view(np.uint8)
+    return out
+
+
+def norms_k_and_v_swapped(codes, alloc, bits_v, capacity):
+    out = _pack_cache(codes, alloc, bits_v, capacity).copy()
+    a = 4 * bg.tile_k_words(int(alloc["bits_k"]), int(alloc["d"]))
+    kn, vn = out[..., a:a + 64].copy(), out[..., a + 64:a + 128].copy()
+    out[..., a:a + 64], out[..., a + 64:a + 128] = vn, kn
+    return out
+
+
+def block_pair_reversed(codes, alloc, bits_v, capacity):
+    """Each block's pair streamed as (dim b + h, dim b) instead of (dim b, dim b + h)."""
+    c = dict(codes)
+    h = codes["Kc"].shape[-1] // 2
+    c["Kc"] = np.concatenate([codes["Kc"][..., h:], codes["Kc"][..., :h]], axis=-1)
+    return _pack_cache(c, alloc, bits_v, capacity)
+
+
+def header_record_without_norms(batch, n_kv_heads, capacity, d, bits_k, bits_v, alloc):
+    """Record size written without the 32 K and 32 V norms."""
+    hdr = _packed_header(batch, n_kv_heads, capacity, d, bits_k, bits_v, alloc).copy()
+    fields = hdr[16:32].view("<u4")
+    fields[3] = 4 * d * (bits_k + bits_v)
+    return hdr
+
+
+_pack_cache = bg.pack_cache
+_packed_header = bg.packed_header
 _pack_bits = bg.pack_bits
 _rotate = rope.rotate
 _nf4_quantize = nqkv.quantize
@@ -352,6 +390,14 @@ CASES = [
      [pins.test_nf4_pack_roundtrip_and_padding]),
     ("NF4: padded rows attended", nqkv, "unpack", nf4_unpack_padding_too,
      [pins.test_nf4_decode_masks_padding]),
+    ("layout: K words token-major", bg, "pack_cache", k_words_token_major,
+     [pins.test_pack_single_code_position_by_hand, pins.test_pack_unpack_roundtrip_mixed_widths]),
+    ("layout: K and V norms swapped", bg, "pack_cache", norms_k_and_v_swapped,
+     [pins.test_pack_single_code_position_by_hand]),
+    ("layout: a block's two codes in reverse order", bg, "pack_cache", block_pair_reversed,
+     [pins.test_pack_single_code_position_by_hand]),
+    ("header: record size without the norms", bg, "packed_header", header_record_without_norms,
+     [pins.test_header_fields_by_hand]),
     ("Lloyd-Max: not run to convergence", cb, "lloyd_max_f64", lloyd_five_iterations,
      [lambda: pins.test_lloyd_max_centroids_are_conditional_means(3), pins.test_lloyd_max_textbook_distortions]),
     ("codebook: thresholds from the exact centroids", cb, "stored_codebook", thresholds_from_exact_centroids,
