@@ -34,6 +34,42 @@ def _oracle_heads(K, V, q, kv: range):
     return bg.decode(q[:, qh.start:qh.stop], p, a, BV, T)
 
 
+class OracleLib:
+    """Stands in for the ctypes binding on the CPU: the calls decode_step_sharded makes, with
+    the same arguments and result types (fp32 output), computed by the oracle."""
+
+    @staticmethod
+    def kvq_calibrate(K, bits_k, n_calib=0):
+        return bg.calibrate(K.numpy(), bits_k, n_calib)
+
+    @staticmethod
+    def cache_desc(batch, n_kv_heads, capacity, bits_k, bits_v):
+        return {"batch": batch, "n_kv_heads": n_kv_heads, "capacity": capacity, "bits_k": bits_k, "bits_v": bits_v}
+
+    @staticmethod
+    def kvq_quantize(K, V, alloc, cache):
+        assert K.shape[1] == cache["n_kv_heads"] == len(alloc["w"])
+        codes = bg.quantize(K.numpy(), V.numpy(), alloc, cache["bits_v"])
+        return bg.pack_cache(codes, alloc, cache["bits_v"], cache["capacity"])
+
+    @staticmethod
+    def kvq_decode_attn(q, packed, alloc, cache, seq_len):
+        return torch.from_numpy(bg.decode(q.numpy(), packed, alloc, cache["bits_v"], seq_len)).float()
+
+
+def _step_rank(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        K, V, q = (torch.from_numpy(a) for a in _inputs())
+        full = shard.decode_step_sharded(K, V, q, BK, BV, world, rank, kvq=OracleLib)
+        np.save(os.path.join(out_dir, f"step{rank}.npy"), full.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -74,4 +110,19 @@ def test_sharded_heads_equal_single_rank(tmp_path, world):
     ref = _oracle_heads(K, V, q, range(HKV))
     for r in range(world):
         got = np.load(tmp_path / f"out{r}.npy")
+        np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world", [2, 4])
+def test_decode_step_sharded_equals_single_rank(tmp_path, world):
+    """The library's own sharded step (head ranges, query-head slices, padded all-gather), run
+    over gloo ranks with the oracle standing in for the kernels: every rank ends with the
+    single-rank output, fp32 bits equal."""
+    mp.start_processes(_step_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn")
+    K, V, q = _inputs()
+    ref = _oracle_heads(K, V, q, range(HKV)).astype(np.float32)
+    for r in range(world):
+        got = np.load(tmp_path / f"step{r}.npy")
+        assert got.dtype == np.float32
         np.testing.assert_array_equal(got, ref)
