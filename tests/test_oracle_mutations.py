@@ -181,6 +181,20 @@ def attention(q, Khat, Vhat, scale=True, kv_of=lambda hq, G, Hkv: hq // G):
     return out
 
 
+def decode_recent_in_own_softmax(q, packed, alloc, bits_v, seq_len, V=None, K_recent=None, V_recent=None):
+    """Recent tokens attended in a softmax of their own, averaged with the packed tokens'."""
+    if K_recent is None or seq_len == 0:
+        return _decode(q, packed, alloc, bits_v, seq_len, V=V, K_recent=K_recent, V_recent=V_recent)
+    return 0.5 * (_decode(q, packed, alloc, bits_v, seq_len, V=V) + bg.decode_attention(q, K_recent, V_recent))
+
+
+def decode_keys_only_values_rounded(q, packed, alloc, bits_v, seq_len, V=None, K_recent=None, V_recent=None):
+    """A keys-only cache's values rounded to fp16 instead of taken exactly."""
+    if bits_v == 0 and V is not None:
+        V = np.asarray(V).astype(np.float16).astype(np.float64)
+    return _decode(q, packed, alloc, bits_v, seq_len, V=V, K_recent=K_recent, V_recent=V_recent)
+
+
 # ---------------------------------------------------------------- layout, header, RoPE, NF4
 
 def pack_msb_first(values, widths):
@@ -329,6 +343,7 @@ def header_record_without_norms(batch, n_kv_heads, capacity, d, bits_k, bits_v, 
     return hdr
 
 
+_decode = bg.decode
 _pack_cache = bg.pack_cache
 _packed_header = bg.packed_header
 _pack_bits = bg.pack_bits
@@ -372,6 +387,10 @@ CASES = [
     ("attention: q head j reads KV head j mod Hkv", bg, "decode_attention",
      lambda q, K, V: attention(q, K, V, kv_of=lambda hq, G, Hkv: hq % Hkv),
      [pins.test_attention_single_token_returns_its_value]),
+    ("decode: recent tokens in a softmax of their own", bg, "decode", decode_recent_in_own_softmax,
+     [pins.test_recent_buffer_duplicating_the_cache_changes_nothing]),
+    ("decode: keys-only values rounded to fp16", bg, "decode", decode_keys_only_values_rounded,
+     [pins.test_keys_only_cache_with_exact_values]),
     ("layout: codes packed most significant bit first", bg, "pack_bits", pack_msb_first,
      [pins.test_pack_bits_by_hand]),
     ("layout: stream by ascending width", bg, "k_stream_blocks", stream_widths_ascending,
