@@ -3,6 +3,7 @@ include/kvq.h, compiled by gcc with warnings as errors and linked against libkvq
 host-only queries (sizes, tables, status strings; nothing that launches, so it passes no
 pointer the library could hand to a kernel). What it prints is checked against the layout's
 closed forms and the oracle's tables."""
+import ctypes
 import os
 import re
 import shutil
@@ -59,23 +60,103 @@ int main(void) {
 """
 
 
-@pytest.fixture(scope="module")
-def c_output(tmp_path_factory):
+# header struct -> the binding's ctypes mirror of it
+STRUCTS = [("kvq_tensor4", kvq.Tensor4), ("kvq_calib_params", kvq.CalibParams), ("kvq_cache_desc", kvq.CacheDesc),
+           ("kvq_head_alloc", kvq.HeadAlloc), ("kvq_packed_header", kvq.PackedHeader),
+           ("kvq_decode_extra", kvq.DecodeExtra)]
+
+
+def _layout_source():
+    """A C program printing sizeof of every header struct and offsetof of every field the
+    binding declares (a field the header lacks fails the compile)."""
+    lines = ["#include <stddef.h>", "#include <stdio.h>", '#include "kvq.h"', "int main(void) {"]
+    for cname, cls in STRUCTS:
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["  return 0;", "}"]
+    return "\n".join(lines) + "\n"
+
+
+def _build_and_run(tmp, name, source, link):
     gcc = shutil.which("gcc")
     if gcc is None:
         pytest.skip("no C compiler")
+    src, exe = tmp / f"{name}.c", tmp / name
+    src.write_text(source)
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+           str(src), "-o", str(exe)]
+    if link:
+        libdir = os.path.dirname(kvq.LIB_PATH)
+        cmd += ["-L", libdir, "-lkvq", f"-Wl,-rpath,{libdir}"]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    return subprocess.run([str(exe)], check=True, capture_output=True, text=True, timeout=60).stdout
+
+
+@pytest.fixture(scope="module")
+def c_output(tmp_path_factory):
     if not os.path.exists(kvq.LIB_PATH):
         from packed_cache_attention_b200 import build
         build.build()
-    d = tmp_path_factory.mktemp("c_client")
-    src, exe = d / "client.c", d / "client"
-    src.write_text(C_SOURCE)
-    libdir = os.path.dirname(kvq.LIB_PATH)
-    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
-                    str(src), "-o", str(exe), "-L", libdir, "-lkvq", f"-Wl,-rpath,{libdir}"],
-                   check=True, capture_output=True, text=True)
-    run = subprocess.run([str(exe)], check=True, capture_output=True, text=True, timeout=60)
-    return {line.split()[0]: line.split()[1:] for line in run.stdout.splitlines() if line.strip()}
+    out = _build_and_run(tmp_path_factory.mktemp("c_client"), "client", C_SOURCE, link=True)
+    return {line.split()[0]: line.split()[1:] for line in out.splitlines() if line.strip()}
+
+
+def test_binding_structs_have_the_headers_layout(tmp_path):
+    """Every ctypes mirror has the C compiler's size and field offsets for its struct."""
+    out = _build_and_run(tmp_path, "layout", _layout_source(), link=False)
+    got = {}
+    for line in out.splitlines():
+        cname, key, val = line.split()
+        got[(cname, key)] = int(val)
+    for cname, cls in STRUCTS:
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for field, _ in cls._fields_:
+            assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)
+
+
+def _c_params(text, name):
+    """Parameter types of `name` in the header, comments removed; [] for (void)."""
+    m = re.search(r"\b" + name + r"\s*\(([^)]*)\)\s*;", text)
+    params = " ".join(m.group(1).split())
+    if params in ("", "void"):
+        return []
+    return [re.sub(r"\s*\b\w+$", "", p.strip()) if not p.strip().endswith("*") else p.strip()
+            for p in params.split(",")]
+
+
+def _ctypes_kind(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "pointer"
+    if t is ctypes.c_size_t:
+        return "size_t"
+    if t is ctypes.c_int:
+        return "int"
+    raise AssertionError(t)
+
+
+def _c_kind(t):
+    if "*" in t:
+        return "pointer"
+    if t.endswith("size_t"):
+        return "size_t"
+    if t in ("int", "kvq_status") or t.endswith("int32_t"):
+        return "int"
+    raise AssertionError(t)
+
+
+def test_binding_signatures_follow_the_header():
+    """Every entry point the binding declares takes as many arguments as the header's
+    prototype, each of the same kind (pointer, int or size_t), and returns the same kind."""
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "kvq.h")).read(), flags=re.S)
+    for name, (args, res) in kvq._SIGNATURES.items():
+        params = _c_params(text, name)
+        assert len(params) == len(args), (name, params)
+        for c, t in zip(params, args):
+            assert _c_kind(c) == _ctypes_kind(t), (name, c, t)
+        ret = re.search(r"([\w\s\*]+?)\b" + name + r"\s*\(", text).group(1).split()
+        ret_t = " ".join(ret).replace("const ", "")
+        assert _c_kind(ret_t) == _ctypes_kind(res), (name, ret_t, res)
 
 
 def test_c_program_sees_the_layout(c_output):
