@@ -157,6 +157,26 @@ def test_quantize_and_decode_reject_bad_arguments(L):
     assert L.kvq_workspace_init(None, 0, None) == 6
 
 
+def test_empty_inputs_are_refused(L):
+    """Zero tokens, zero sequences or zero heads are refused on the host, before any launch."""
+    mem = buf()
+    p = kvq.CalibParams(3, 8, 0, 0)
+    c = kvq.cache_desc(1, 2, 64, 3, 3)
+    assert _calib(L, mem, _t4(T=0), p) == 2
+    assert _calib(L, mem, _t4(B=0), p) == 2
+    assert _calib(L, mem, _t4(H=0), p) == 2
+    assert L.kvq_quantize(mem, ctypes.byref(_t4(T=0)), mem, ctypes.byref(_t4(T=0)), mem, ctypes.byref(c), mem,
+                          None) == 2
+    assert L.kvq_append(mem, ctypes.byref(_t4(T=0)), mem, ctypes.byref(_t4(T=0)), mem, ctypes.byref(c), 0, mem,
+                        None) == 2
+    assert L.kvq_nf4_quantize(mem, ctypes.byref(_t4(T=0)), mem, ctypes.byref(_t4(T=0)), 64, mem, None) == 2
+    qd = kvq.Tensor4(1, 2, 1, 128, 2 * 128, 128, 128, kvq.KVQ_BF16, 0)
+    assert L.kvq_nf4_decode_attn(mem, ctypes.byref(qd), mem, 64, 0, mem, buf(WS_BYTES), WS_BYTES, None) == 5
+    assert kvq.kvq_packed_bytes(kvq.cache_desc(1, 2, 0, 3, 3)) == 0
+    assert kvq.kvq_packed_bytes(kvq.cache_desc(0, 2, 64, 3, 3)) == 0
+    assert kvq.kvq_nf4_packed_bytes(1, 2, 0) == 0
+
+
 def test_nf4_append_rejects_ranges_outside_the_cache(L):
     mem = buf()
     app = lambda kd_, cap, t0: L.kvq_nf4_append(mem, ctypes.byref(kd_), mem, ctypes.byref(kd_), cap, t0, mem, None)
