@@ -181,6 +181,16 @@ def attention(q, Khat, Vhat, scale=True, kv_of=lambda hq, G, Hkv: hq // G):
     return out
 
 
+def widths_interleaved(w_blocks):
+    """Per-dim widths (w_0, w_0, w_1, w_1, ..) instead of block b on dims b and b + h."""
+    return np.repeat(np.asarray(w_blocks), 2)
+
+
+def nf4_scales_shifted(idx, scale, n_heads, d):
+    """Each token dequantized with the next token's block scales."""
+    return _nf4_dequantize(idx, np.roll(scale, -1, axis=2), n_heads, d)
+
+
 def decode_recent_in_own_softmax(q, packed, alloc, bits_v, seq_len, V=None, K_recent=None, V_recent=None):
     """Recent tokens attended in a softmax of their own, averaged with the packed tokens'."""
     if K_recent is None or seq_len == 0:
@@ -344,6 +354,7 @@ def header_record_without_norms(batch, n_kv_heads, capacity, d, bits_k, bits_v, 
 
 
 _decode = bg.decode
+_nf4_dequantize = nqkv.dequantize
 _pack_cache = bg.pack_cache
 _packed_header = bg.packed_header
 _pack_bits = bg.pack_bits
@@ -387,6 +398,10 @@ CASES = [
     ("attention: q head j reads KV head j mod Hkv", bg, "decode_attention",
      lambda q, K, V: attention(q, K, V, kv_of=lambda hq, G, Hkv: hq % Hkv),
      [pins.test_attention_single_token_returns_its_value]),
+    ("widths: per-dim widths interleaved", bg, "widths_per_dim", widths_interleaved,
+     [pins.test_dequantizer_by_hand]),
+    ("NF4: each token dequantized with the next token's scales", nqkv, "dequantize", nf4_scales_shifted,
+     [pins.test_nf4_fig5_worked_shape]),
     ("decode: recent tokens in a softmax of their own", bg, "decode", decode_recent_in_own_softmax,
      [pins.test_recent_buffer_duplicating_the_cache_changes_nothing]),
     ("decode: keys-only values rounded to fp16", bg, "decode", decode_keys_only_values_rounded,
@@ -437,7 +452,10 @@ def test_planted_mistake_is_caught(monkeypatch, name, module, attr, bad, checks)
     for check in checks:
         try:
             check()
-        except AssertionError:
+        except (AssertionError, IndexError, ValueError):
+            # a failed assertion, or a pin that can no longer run on the mutated oracle (a code
+            # out of its codebook's range, a shape that no longer fits); a NameError or
+            # TypeError would be a broken stand-in and is not taken as a catch
             caught.append(check)
     assert caught, f"no pin catches the planted mistake: {name}"
 
