@@ -5,6 +5,8 @@ head) units never exchange data: calibration, quantization and decode of a head 
 head alone."""
 import os
 import socket
+import time
+from datetime import timedelta
 
 import numpy as np
 import pytest
@@ -126,3 +128,32 @@ def test_decode_step_sharded_equals_single_rank(tmp_path, world):
         got = np.load(tmp_path / f"step{r}.npy")
         assert got.dtype == np.float32
         np.testing.assert_array_equal(got, ref)
+
+
+def _rank_that_leaves(rank, world, port, out_dir):
+    """Rank 1 leaves the job before the gather (it exits between steps, with nothing in
+    flight); rank 0 goes on to the gather and records what happened."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
+    if rank == 1:
+        dist.destroy_process_group()
+        return
+    t0 = time.monotonic()
+    try:
+        shard.gather_outputs(torch.zeros((1, 2, 128)), range(0, 1), 2, 2, world)
+        outcome = "returned"
+    except Exception as e:                                   # the collective reports the missing rank
+        outcome = "error " + type(e).__name__
+    with open(os.path.join(out_dir, "rank0.txt"), "w") as fh:
+        fh.write(f"{outcome} {time.monotonic() - t0:.1f}")
+
+
+@pytest.mark.timeout(120)
+def test_gather_reports_a_rank_that_left(tmp_path):
+    """A rank that left is seen by the others at their next collective: the gather raises
+    within the process group's timeout instead of waiting for good."""
+    mp.start_processes(_rank_that_leaves, args=(2, _free_port(), str(tmp_path)), nprocs=2, start_method="spawn")
+    outcome, seconds = (tmp_path / "rank0.txt").read_text().rsplit(" ", 1)
+    assert outcome.startswith("error"), outcome
+    assert float(seconds) < 60
