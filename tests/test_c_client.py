@@ -191,3 +191,22 @@ def test_c_program_gets_status_strings_and_workspace_sizes(c_output):
     assert " ".join(c_output["status_out_of_range"]) == "unknown status"
     # counters + energies + segment sums + chunk sums (fp64) at least
     assert int(c_output["calib_ws"][0]) >= 8 * (16 * 2048 // 64) * 64 * 8 + 8 * 64 * 8
+
+
+def test_readme_c_example_compiles(tmp_path):
+    """The C example in README.md compiles against the header as C99 with warnings as errors,
+    and links against libkvq.so with no undefined symbol."""
+    text = open(os.path.join(ROOT, "README.md")).read()
+    block = re.search(r"```c\n(.*?)```", text, flags=re.S).group(1)
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "example.c"
+    src.write_text(block)
+    if not os.path.exists(kvq.LIB_PATH):
+        from packed_cache_attention_b200 import build
+        build.build()
+    libdir = os.path.dirname(kvq.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fPIC", "-shared",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(tmp_path / "example.so"),
+                    "-Wl,--no-undefined", "-L", libdir, "-lkvq"], check=True, capture_output=True, text=True)
