@@ -13,6 +13,10 @@
  * levels) to that device with a synchronous copy, so it must not be made while a stream is
  * being captured; kvq_init() does the upload explicitly.
  *
+ * Host threads may call the library at once: its one-time setup per device and CUDA context
+ * (tables, kernel attributes, occupancy) is serialized inside it. Calls that share a workspace
+ * or write the same packed cache must still not overlap on the GPU.
+ *
  * Calibrate, quantize/append and the Block-GTQ decode are launched with programmatic
  * dependent launch: such a kernel may start (barriers, tensor memory, the library's own tables)
  * while the previous kernel in the stream is finishing, but reads and writes none of the

@@ -207,16 +207,19 @@ DecodeWs gtq_ws_layout(int bh, int splits, int ticket_stride, size_t part_base =
   return decode_ws_layout(bh, splits + mp.n_groups, 8, ticket_stride, part_base);
 }
 
+// Per-device attribute memos: atomics, so host threads calling in at once read either 0 (and
+// query the attribute themselves) or the stored value.
 int sm_count() {
-  static int cached[kMaxDevices] = {};
+  static std::atomic<int> cached[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
+    if (n <= 0) n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 // Launches `kern` with programmatic stream serialization: it may begin (barrier setup, its
@@ -252,15 +255,16 @@ Nf4Layout nf4_layout(int batch, int n_heads, int capacity) {
 
 // Opt-in shared memory per block of the current device (227 KB on a B200).
 size_t max_smem() {
-  static int cached[kMaxDevices] = {};
+  static std::atomic<int> cached[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 227 * 1024;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    cached[dev] = n > 0 ? n : 227 * 1024;
+    if (n <= 0) n = 227 * 1024;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return static_cast<size_t>(cached[dev]);
+  return static_cast<size_t>(n);
 }
 
 // Chunk stages per warpgroup (1..4) that fit in shared memory; cbytes = bytes of one chunk stage.
