@@ -281,8 +281,8 @@ size_t decode_smem_bytes(int cbytes) {
 }
 
 // Test hooks (kvq_debug_decode): bounded-wait limit and the no-copy switch of the next decodes.
-uint32_t g_wait_limit = 2000;
-int g_debug_no_loads = 0;
+std::atomic<uint32_t> g_wait_limit{2000};   // test hook settings (kvq_debug_decode)
+std::atomic<int> g_debug_no_loads{0};
 
 }  // namespace
 
@@ -640,8 +640,8 @@ kvq_status launch_decode(const void* q, const kvq_tensor4* qd, const void* packe
   a.tickets = reinterpret_cast<unsigned*>(w8 + L.tickets);
   a.ticket_stride = ticket_stride;
   a.status = reinterpret_cast<unsigned*>(w8);
-  a.wait_limit = g_wait_limit;
-  a.debug_no_loads = g_debug_no_loads;
+  a.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+  a.debug_no_loads = g_debug_no_loads.load(std::memory_order_relaxed);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(splits, bh);
   const int vm = dense_v ? (ex->vd.dtype == KVQ_BF16 ? kDenseBf16 : kDenseF16) : c->bits_v;
@@ -717,8 +717,8 @@ const char* kvq_last_cuda_error(void) {
 
 kvq_status kvq_debug_decode(int wait_limit, int no_loads) {
   if (wait_limit < 1) return KVQ_ERR_ARG;
-  g_wait_limit = static_cast<uint32_t>(wait_limit);
-  g_debug_no_loads = no_loads ? 1 : 0;
+  g_wait_limit.store(static_cast<uint32_t>(wait_limit), std::memory_order_relaxed);
+  g_debug_no_loads.store(no_loads ? 1 : 0, std::memory_order_relaxed);
   return KVQ_OK;
 }
 
